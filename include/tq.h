@@ -1,0 +1,220 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) rotated-codebook KV-cache codec.
+ *
+ * The method (TurboQuant as described on the pages this library follows):
+ *   - store the norm nu = ||x|| and quantize the unit vector x / nu
+ *     ("FibQuant: Quantizzazione Vettoriale Universale ...", section 2.3);
+ *   - rotate it with one shared random orthogonal map, a randomized
+ *     Walsh-Hadamard transform Pi = H_d diag(D) / sqrt(d)
+ *     ("Ablazione, Inferenza Statistica e Validazione ...", "Configurazione
+ *     Sperimentale");
+ *   - quantize every rotated coordinate with a Lloyd-Max codebook solved
+ *     offline for the Beta coordinate law ("Google presenta TurboQuant ...",
+ *     "La mecanica geometrica de TurboQuant", MSE cost C(f_X, b));
+ *   - keys use TURBOQUANT_prod: b-1 MSE bits plus a 1-bit QJL sketch
+ *     sigma = sign(S r) of the rotated residual r, with rho = ||r||, giving an
+ *     unbiased inner-product estimator (same page, "Eliminacion del sesgo
+ *     interno del producto");
+ *   - attention logits are estimated straight from the packed codes and the
+ *     values are accumulated in the rotated domain, with one inverse rotation
+ *     per output ("TurboESM ...", section 2.E "Kernel Fuso Triton").
+ *
+ * Conventions for every call
+ *   - Return value: tq_status.  On failure tq_last_error() gives a message
+ *     (thread-local, valid until the next call on the same thread).
+ *   - Pointers documented "device" must be CUDA device memory of the device
+ *     that is current when the call is made; "host" pointers are ordinary
+ *     host memory.  The caller owns every buffer it passes in.
+ *   - Calls taking a stream are stream-ordered and asynchronous: arguments are
+ *     validated synchronously, kernels are enqueued on `stream`
+ *     (a cudaStream_t; NULL = legacy default stream), and no call blocks the
+ *     host.  Launch failures return TQ_ERR_CUDA; faults inside a kernel
+ *     surface at the caller's next synchronisation.
+ *   - Supported: d in {64, 128}; key MSE bits 1..4 (with QJL: 2 <= bits_k <= 5
+ *     total); value bits 1..4.
+ */
+#ifndef TQ_B200_H
+#define TQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* NULL where a buffer is required, bad size or shape */
+  TQ_ERR_UNSUPPORTED = 2,   /* head dim or bit width this build has no kernel for */
+  TQ_ERR_ALIGNMENT = 3,     /* a device buffer misses its required alignment */
+  TQ_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  TQ_ERR_WORKSPACE = 5      /* workspace too small (query tq_attention_workspace) */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* ------------------------------------------------------------------------
+ * Offline codebook ("Google presenta TurboQuant ...", "La mecanica
+ * geometrica de TurboQuant": minimise C(f_X, b) once per bit width and store).
+ *
+ * Solves the Lloyd-Max conditions for the density of one coordinate of a
+ * uniform point on the unit sphere S^{d-1},
+ *     f_d(x) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - x^2)^((d-3)/2),
+ * on [-1, 1] (outer cells reach the support ends).  fp64 solve on the host,
+ * fp32 results.
+ *   centroids  host, 2^bits floats, ascending, odd-symmetric.
+ *   thresholds host, 2^bits - 1 floats, midpoints of adjacent centroids; a
+ *              coordinate u gets code #{k : u >= thresholds[k]}.
+ *   mse_per_coord host, nullable: E[(X - Q(X))^2] at the solution.
+ * Errors: TQ_ERR_INVALID_ARG for d < 4, bits outside 1..8 or NULL outputs.
+ * ------------------------------------------------------------------------ */
+int tq_build_codebook(int d, int bits, float *centroids, float *thresholds,
+                      double *mse_per_coord);
+
+/* ------------------------------------------------------------------------
+ * Codec: immutable description shared by every call (thread-safe to share).
+ *
+ * rotation_signs  host, d entries, each +1 or -1: the diagonal D of
+ *                 Pi = H_d diag(D) / sqrt(d), H_d Sylvester-ordered.
+ * qjl_bf16        host, d*d bf16 bit patterns, row-major S[i][j]: the QJL
+ *                 sketch (i.i.d. N(0,1) values stored as bf16).  Required iff
+ *                 qjl_k != 0.
+ * bits_k          total key bits; with qjl_k the MSE stage uses bits_k - 1.
+ * bits_v          value bits (TURBOQUANT_mse).
+ * tq_codec_create solves both codebooks with tq_build_codebook and copies D,
+ * S and the codebooks to the current device (the only allocation the library
+ * makes); tq_codec_destroy frees them.
+ * ------------------------------------------------------------------------ */
+typedef struct tq_codec tq_codec;
+
+typedef struct {
+  int d;
+  int bits_k;
+  int qjl_k;
+  int bits_v;
+  const int8_t *rotation_signs;
+  const uint16_t *qjl_bf16;
+} tq_codec_desc;
+
+int tq_codec_create(const tq_codec_desc *desc, tq_codec **out);
+void tq_codec_destroy(tq_codec *codec);
+/* Host copies of the codec's codebooks (fp32) for inspection; any pointer may
+ * be NULL.  Sizes: 2^mse_bits_k, 2^mse_bits_k - 1, 2^bits_v, 2^bits_v - 1. */
+int tq_codec_codebooks(const tq_codec *codec, float *ck, float *tk, float *cv, float *tv);
+
+/* ------------------------------------------------------------------------
+ * Compressed cache: fixed rate, every token at fixed addresses
+ * ("FibQuant ...", section 1: decode any token on its own by address
+ * arithmetic).  All four planes are device memory owned by the caller.
+ *
+ *   kcode  uint8  [B][Hkv][rows_cap][planes_k][d/8]  planes_k = mse bits (+1
+ *          with QJL).  Plane p < mse bits holds bit p of each coordinate's
+ *          code; the last plane holds sigma.  Coordinate i: byte i/8, bit i%8.
+ *   kscale fp16   [B][Hkv][rows_cap][2]  (nu, rho) per key; rho = 0 without QJL.
+ *   vcode  uint32 [B][Hkv][rows_cap/32][bits_v][d]  32-token column groups:
+ *          bit (t % 32) of word [t/32][p][i] is bit p of coordinate i's code
+ *          of token t.
+ *   vnorm  fp16   [B][Hkv][rows_cap]  nu per value.
+ * rows_cap must be a multiple of 32; kcode, vcode, kscale need 16-byte
+ * alignment, vnorm 4-byte.  Bytes per (token, head): d/8*planes_k + 4 for
+ * keys, d/8*bits_v + 2 for values.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  uint8_t *kcode;
+  uint16_t *kscale;
+  uint32_t *vcode;
+  uint16_t *vnorm;
+  int B;
+  int Hkv;
+  int64_t rows_cap;
+} tq_cache;
+
+/* Bytes of each plane (kcode, kscale, vcode, vnorm) for a cache shape. */
+int tq_cache_bytes(const tq_codec *codec, int B, int Hkv, int64_t rows_cap, size_t bytes[4]);
+
+/* ------------------------------------------------------------------------
+ * Quantize-append (prefill or decode append).  One fused kernel per call.
+ *
+ * k, v     device, [B][Hkv][T][d] with element strides (stride_b, stride_h,
+ *          stride_t) and d contiguous; dtype TQ_F32 or TQ_BF16.
+ * rope_cos, rope_sin  device fp32 [*][d/2], nullable together: rotate-half
+ *          RoPE is applied to keys at positions pos0 + t before encoding
+ *          ("TurboESM ...", section 2.A: RoPE first, then Pi).
+ * cache    rows [row0, row0 + T) of every (b, h) are written; other tokens of
+ *          a partially covered 32-token value group are preserved (calls that
+ *          touch the same group must be stream-ordered).
+ * status   device uint32, nullable: incremented once per row (key or value)
+ *          whose input had a non-finite element or whose fp16 norm overflowed;
+ *          such rows are encoded as zero vectors.
+ * ------------------------------------------------------------------------ */
+int tq_quantize_kv(const tq_codec *codec, const void *k, const void *v, int dtype,
+                   int B, int Hkv, int T, int64_t stride_b, int64_t stride_h,
+                   int64_t stride_t, const float *rope_cos, const float *rope_sin,
+                   int64_t pos0, const tq_cache *cache, int64_t row0, uint32_t *status,
+                   void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode attention straight from the compressed cache (split-K).
+ *
+ * For query head h (KV head h / (Hq/Hkv)) of batch b with length T_b:
+ *   q'  = Pi RoPE(q, T_b - 1),  q'' = S q'
+ *   l_j = scale * nu_j * (<q', c_k[idx_j]> + sqrt(pi/2)/d * rho_j * <q'', 2 sigma_j - 1>)
+ *   out = Pi^T ( sum_j softmax(l)_j * nu^v_j * c_v[idx^v_j] )
+ * q        device [B][Hq][d], dtype TQ_F32 or TQ_BF16.
+ * seq_lens device int32 [B], nullable (then every batch has max_seq_len);
+ *          entries are clamped to 1..max_seq_len; max_seq_len <= rows_cap.
+ * rope_cos/rope_sin  as for tq_quantize_kv (nullable together).
+ * num_splits  chunks per (b, KV head); 0 picks a default.
+ * workspace   device, >= tq_attention_workspace(...) bytes, 16-byte aligned;
+ *             scratch owned by the caller, contents need no initialisation.
+ * out      device fp32 [B][Hq][d].
+ * ------------------------------------------------------------------------ */
+int tq_attention_workspace(const tq_codec *codec, int B, int Hq, int num_splits, size_t *bytes);
+int tq_attention_decode(const tq_codec *codec, const void *q, int dtype, int B, int Hq,
+                        int Hkv, const tq_cache *cache, const int32_t *seq_lens,
+                        int max_seq_len, float scale, const float *rope_cos,
+                        const float *rope_sin, int num_splits, void *workspace,
+                        size_t ws_bytes, float *out, void *stream);
+
+/* Same as tq_attention_decode, and also writes the estimated logits
+ * l_j (the formula above, scale included) of every query head:
+ * logits  device fp32 [B][Hq][max_seq_len]; entries j >= T_b are left
+ *         untouched.  Meant for inspection and scoring; costs one extra
+ *         store per (head, key). */
+int tq_attention_logits(const tq_codec *codec, const void *q, int dtype, int B, int Hq,
+                        int Hkv, const tq_cache *cache, const int32_t *seq_lens,
+                        int max_seq_len, float scale, const float *rope_cos,
+                        const float *rope_sin, int num_splits, void *workspace,
+                        size_t ws_bytes, float *out, float *logits, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Dequantize rows [row0, row0 + rows) of every (b, h) ("FibQuant ...",
+ * section 2.3 decoder): keys  nu Pi^T (c_k[idx] + sqrt(pi/2)/d rho S^T(2 sigma - 1)),
+ * values nu Pi^T c_v[idx].
+ * which  0 = keys, 1 = values.   out  device fp32 [B][Hkv][rows][d].
+ * ------------------------------------------------------------------------ */
+int tq_dequantize(const tq_codec *codec, const tq_cache *cache, int which, int64_t row0,
+                  int64_t rows, float *out, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Profiling hooks (no counterpart on the pages; used by the benchmark).
+ * tq_set_timing_events: when both are non-NULL, every later
+ *   tq_attention_decode / tq_attention_logits on this thread records `start`
+ *   (a cudaEvent_t) on its stream right before the split-K chunk kernel and
+ *   `stop` right after it (event records are captured into CUDA graphs like
+ *   any stream work).  Pass NULL, NULL to stop.
+ * tq_launch_count: number of kernels this process has launched through the
+ *   library so far (all threads).
+ * ------------------------------------------------------------------------ */
+int tq_set_timing_events(void *start, void *stop);
+uint64_t tq_launch_count(void);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char *tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_B200_H */

@@ -1,0 +1,249 @@
+// C ABI entry points: argument validation, codec lifetime, kernel dispatch.
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "tq_internal.h"
+
+#include <atomic>
+
+namespace {
+thread_local std::string g_last_error;
+thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+std::atomic<uint64_t> g_launches{0};
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+int check_cache(const tq_codec *c, const tq_cache *cache) {
+  if (!cache || !cache->kcode || !cache->kscale || !cache->vcode || !cache->vnorm)
+    return tq_fail(TQ_ERR_INVALID_ARG, "cache: every plane pointer is required");
+  if (cache->B <= 0 || cache->Hkv <= 0 || cache->rows_cap <= 0 || cache->rows_cap % 32)
+    return tq_fail(TQ_ERR_INVALID_ARG, "cache: B, Hkv > 0 and rows_cap a positive multiple of 32");
+  if (!aligned(cache->kcode, 16) || !aligned(cache->vcode, 16) || !aligned(cache->kscale, 16) ||
+      !aligned(cache->vnorm, 4))
+    return tq_fail(TQ_ERR_ALIGNMENT, "cache: kcode/vcode/kscale need 16-byte, vnorm 4-byte alignment");
+  (void)c;
+  return TQ_OK;
+}
+}  // namespace
+
+int tq_fail(int code, const std::string &msg) {
+  g_last_error = msg;
+  return code;
+}
+
+void tq_count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+void tq_timing_events(cudaEvent_t *start, cudaEvent_t *stop) {
+  *start = g_ev_start;
+  *stop = g_ev_stop;
+}
+
+int tq_check_launch(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return tq_fail(TQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+extern "C" {
+
+const char *tq_last_error(void) { return g_last_error.c_str(); }
+
+int tq_set_timing_events(void *start, void *stop) {
+  if ((start == nullptr) != (stop == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "timing events: pass both or neither");
+  g_ev_start = static_cast<cudaEvent_t>(start);
+  g_ev_stop = static_cast<cudaEvent_t>(stop);
+  return TQ_OK;
+}
+
+uint64_t tq_launch_count(void) { return g_launches.load(); }
+
+int tq_build_codebook(int d, int bits, float *centroids, float *thresholds,
+                      double *mse_per_coord) {
+  if (!centroids || !thresholds) return tq_fail(TQ_ERR_INVALID_ARG, "codebook: NULL output");
+  std::vector<double> c, t;
+  double mse = 0.0;
+  if (!tqhost::lloyd_max(d, bits, c, t, mse))
+    return tq_fail(TQ_ERR_INVALID_ARG, "codebook: need d >= 4 and 1 <= bits <= 8");
+  for (size_t i = 0; i < c.size(); ++i) centroids[i] = static_cast<float>(c[i]);
+  for (size_t i = 0; i < t.size(); ++i) thresholds[i] = static_cast<float>(t[i]);
+  if (mse_per_coord) *mse_per_coord = mse;
+  return TQ_OK;
+}
+
+int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
+  if (!desc || !out) return tq_fail(TQ_ERR_INVALID_ARG, "codec: NULL argument");
+  *out = nullptr;
+  if (!supported_d(desc->d)) return tq_fail(TQ_ERR_UNSUPPORTED, "codec: d must be 64 or 128");
+  const int mse_k = desc->qjl_k ? desc->bits_k - 1 : desc->bits_k;
+  if (mse_k < 1 || mse_k > 4 || desc->bits_v < 1 || desc->bits_v > 4)
+    return tq_fail(TQ_ERR_UNSUPPORTED,
+                   "codec: key MSE bits and value bits must be 1..4 (bits_k >= 2 with QJL)");
+  if (!desc->rotation_signs) return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs required");
+  if (desc->qjl_k && !desc->qjl_bf16)
+    return tq_fail(TQ_ERR_INVALID_ARG, "codec: qjl_bf16 required when qjl_k != 0");
+  for (int i = 0; i < desc->d; ++i)
+    if (desc->rotation_signs[i] != 1 && desc->rotation_signs[i] != -1)
+      return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs entries must be +1 or -1");
+
+  tq_codec *c = new tq_codec();
+  std::memset(&c->books, 0, sizeof(c->books));
+  c->d = desc->d;
+  c->bits_k = desc->bits_k;
+  c->qjl_k = desc->qjl_k ? 1 : 0;
+  c->bits_v = desc->bits_v;
+  c->mse_bits_k = mse_k;
+  c->S_dev = nullptr;
+  cudaGetDevice(&c->device);
+
+  std::vector<double> cc, tt;
+  double mse;
+  tqhost::lloyd_max(c->d, mse_k, cc, tt, mse);
+  for (size_t i = 0; i < cc.size(); ++i) c->books.ck[i] = static_cast<float>(cc[i]);
+  for (size_t i = 0; i < tt.size(); ++i) c->books.tk[i] = static_cast<float>(tt[i]);
+  tqhost::lloyd_max(c->d, c->bits_v, cc, tt, mse);
+  for (size_t i = 0; i < cc.size(); ++i) c->books.cv[i] = static_cast<float>(cc[i]);
+  for (size_t i = 0; i < tt.size(); ++i) c->books.tv[i] = static_cast<float>(tt[i]);
+  for (int i = 0; i < c->d; ++i)
+    if (desc->rotation_signs[i] < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
+  c->books.mse_bits_k = mse_k;
+  c->books.qjl = c->qjl_k;
+  c->books.bits_v = c->bits_v;
+
+  if (c->qjl_k) {
+    const size_t bytes = sizeof(uint16_t) * c->d * c->d;
+    if (cudaMalloc(&c->S_dev, bytes) != cudaSuccess) {
+      delete c;
+      return tq_check_launch("codec: cudaMalloc");
+    }
+    if (cudaMemcpy(c->S_dev, desc->qjl_bf16, bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(c->S_dev);
+      delete c;
+      return tq_check_launch("codec: cudaMemcpy");
+    }
+  }
+  *out = c;
+  return TQ_OK;
+}
+
+void tq_codec_destroy(tq_codec *codec) {
+  if (!codec) return;
+  if (codec->S_dev) cudaFree(codec->S_dev);
+  delete codec;
+}
+
+int tq_codec_codebooks(const tq_codec *c, float *ck, float *tk, float *cv, float *tv) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "codebooks: NULL codec");
+  const int nk = 1 << c->mse_bits_k, nv = 1 << c->bits_v;
+  if (ck) std::memcpy(ck, c->books.ck, sizeof(float) * nk);
+  if (tk) std::memcpy(tk, c->books.tk, sizeof(float) * (nk - 1));
+  if (cv) std::memcpy(cv, c->books.cv, sizeof(float) * nv);
+  if (tv) std::memcpy(tv, c->books.tv, sizeof(float) * (nv - 1));
+  return TQ_OK;
+}
+
+int tq_cache_bytes(const tq_codec *c, int B, int Hkv, int64_t rows_cap, size_t bytes[4]) {
+  if (!c || !bytes || B <= 0 || Hkv <= 0 || rows_cap <= 0 || rows_cap % 32)
+    return tq_fail(TQ_ERR_INVALID_ARG, "cache_bytes: bad shape (rows_cap multiple of 32)");
+  const size_t rows = static_cast<size_t>(B) * Hkv * rows_cap;
+  bytes[0] = rows * (c->mse_bits_k + c->qjl_k) * (c->d / 8);
+  bytes[1] = rows * 2 * sizeof(uint16_t);
+  bytes[2] = rows / 32 * c->bits_v * c->d * sizeof(uint32_t);
+  bytes[3] = rows * sizeof(uint16_t);
+  return TQ_OK;
+}
+
+int tq_quantize_kv(const tq_codec *c, const void *k, const void *v, int dtype, int B, int Hkv,
+                   int T, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                   const float *rope_cos, const float *rope_sin, int64_t pos0,
+                   const tq_cache *cache, int64_t row0, uint32_t *status, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "quantize: NULL codec");
+  if (int e = check_cache(c, cache)) return e;
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "quantize: dtype");
+  if (B != cache->B || Hkv != cache->Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize: B/Hkv differ from the cache's");
+  if (T < 0 || row0 < 0 || row0 + T > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize: rows [row0, row0+T) outside the cache");
+  if (T == 0) return TQ_OK;
+  if (!k || !v) return tq_fail(TQ_ERR_INVALID_ARG, "quantize: NULL k or v");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize: rope_cos and rope_sin go together");
+  if (rope_cos && pos0 < 0) return tq_fail(TQ_ERR_INVALID_ARG, "quantize: pos0 < 0");
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(k, es) || !aligned(v, es))
+    return tq_fail(TQ_ERR_ALIGNMENT, "quantize: k/v not aligned to their element size");
+  return launch_quantize(c, k, v, dtype, B, Hkv, T, stride_b, stride_h, stride_t, rope_cos,
+                         rope_sin, pos0, cache, row0, status, static_cast<cudaStream_t>(stream));
+}
+
+int tq_attention_workspace(const tq_codec *c, int B, int Hq, int num_splits, size_t *bytes) {
+  if (!c || !bytes || B <= 0 || Hq <= 0 || num_splits < 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "workspace: bad arguments");
+  *bytes = decode_workspace_bytes(c, B, Hq, num_splits > 0 ? num_splits : 64);
+  return TQ_OK;
+}
+
+namespace {
+int decode_common(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                  const tq_cache *cache, const int32_t *seq_lens, int max_seq_len, float scale,
+                  const float *rope_cos, const float *rope_sin, int num_splits, void *workspace,
+                  size_t ws_bytes, float *out, float *logits, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "decode: NULL codec");
+  if (int e = check_cache(c, cache)) return e;
+  if (!q || !out || !workspace) return tq_fail(TQ_ERR_INVALID_ARG, "decode: NULL q/out/workspace");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "decode: dtype");
+  if (B != cache->B || Hkv != cache->Hkv || Hq <= 0 || Hq % Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode: B/Hkv differ from the cache's or Hq % Hkv != 0");
+  if (max_seq_len < 1 || max_seq_len > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode: max_seq_len outside 1..rows_cap");
+  if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "decode: scale not finite");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode: rope_cos and rope_sin go together");
+  const int splits = num_splits > 0 ? num_splits : 64;
+  if (decode_workspace_bytes(c, B, Hq, splits) > ws_bytes)
+    return tq_fail(TQ_ERR_WORKSPACE, "decode: workspace smaller than tq_attention_workspace()");
+  if (!aligned(workspace, 16)) return tq_fail(TQ_ERR_ALIGNMENT, "decode: workspace alignment");
+  if (!aligned(out, 4) || !aligned(q, dtype == TQ_BF16 ? 2 : 4) || !aligned(logits, 4))
+    return tq_fail(TQ_ERR_ALIGNMENT, "decode: q/out/logits alignment");
+  return launch_decode(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale, rope_cos,
+                       rope_sin, splits, workspace, out, logits,
+                       static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int tq_attention_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                        const tq_cache *cache, const int32_t *seq_lens, int max_seq_len,
+                        float scale, const float *rope_cos, const float *rope_sin,
+                        int num_splits, void *workspace, size_t ws_bytes, float *out,
+                        void *stream) {
+  return decode_common(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale, rope_cos,
+                       rope_sin, num_splits, workspace, ws_bytes, out, nullptr, stream);
+}
+
+int tq_attention_logits(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                        const tq_cache *cache, const int32_t *seq_lens, int max_seq_len,
+                        float scale, const float *rope_cos, const float *rope_sin,
+                        int num_splits, void *workspace, size_t ws_bytes, float *out,
+                        float *logits, void *stream) {
+  if (!logits) return tq_fail(TQ_ERR_INVALID_ARG, "logits: NULL logits");
+  return decode_common(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale, rope_cos,
+                       rope_sin, num_splits, workspace, ws_bytes, out, logits, stream);
+}
+
+int tq_dequantize(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
+                  int64_t rows, float *out, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: NULL codec");
+  if (int e = check_cache(c, cache)) return e;
+  if (which != 0 && which != 1) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: which is 0 or 1");
+  if (row0 < 0 || rows < 0 || row0 + rows > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: rows outside the cache");
+  if (rows > 0 && !out) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: NULL out");
+  return launch_dequant(c, cache, which, row0, rows, out, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

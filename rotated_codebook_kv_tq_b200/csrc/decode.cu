@@ -1,0 +1,378 @@
+// Split-K decode attention straight from the compressed cache.
+//
+// Sources: "TurboESM ..." section 2.E (one pass over the compressed cache:
+// unpack, residual correction, inverse rotation, attention with online
+// softmax; no intermediate dequantized buffer) and section 2.A (RoPE before
+// the rotation); "Google presenta TurboQuant ..." ("Eliminacion del sesgo":
+// the prod estimator of <q, k> is unbiased).
+//
+// Three kernels per call:
+//   qprep   one warp per query head: q' = Pi RoPE(q), q'' = S q' (fp32).
+//   chunk   one CTA per (chunk, KV head, batch): logits of the G query heads
+//           of the group from the packed key planes, softmax statistics and the
+//           value sum in the rotated domain (unnormalised, relative to the
+//           chunk max), written to the workspace.
+//   combine one warp per query head: log-sum-exp merge of the chunks, then
+//           out = Pi^T o / l = D (H o) / (sqrt(d) l).
+#include <math_constants.h>
+
+#include "tq_device.cuh"
+
+namespace {
+
+constexpr int CT = 256;       // threads of the chunk kernel
+constexpr int QW = 8;         // warps per block in qprep / combine
+
+struct DecodeArgs {
+  const void *q;
+  int dtype;
+  int B, Hq, Hkv, G;
+  const uint8_t *kcode;
+  const uint16_t *kscale;
+  const uint32_t *vcode;
+  const uint16_t *vnorm;
+  int64_t rows_cap;
+  const int32_t *seq_lens;
+  int max_len;
+  float scale;
+  float qjl_coef;
+  const float *rc;
+  const float *rs;
+  int splits;
+  int chunk;          // rows per chunk (multiple of 32)
+  const uint16_t *S;
+  float *q1;          // [B][Hq][D]
+  float *q2;          // [B][Hq][D]
+  float *po;          // [B][Hq][splits][D]
+  float *pml;         // [B][Hq][splits][2]
+  float *out;         // [B][Hq][D]
+  float *logits;      // optional [B][Hq][max_len] (phase-1 logits)
+  TqBooks books;
+};
+
+__device__ __forceinline__ int seq_len_of(const DecodeArgs &a, int b) {
+  return a.seq_lens ? min(max(a.seq_lens[b], 1), a.max_len) : a.max_len;
+}
+
+template <int D>
+__global__ void __launch_bounds__(QW * 32) qprep_kernel(DecodeArgs a) {
+  constexpr int NPL = D / 32;
+  __shared__ float qs[QW][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int head = blockIdx.x * QW + warp;
+  if (head >= a.B * a.Hq) return;
+  const int b = head / a.Hq;
+  const int64_t pos = seq_len_of(a, b) - 1;
+  float x[NPL];
+#pragma unroll
+  for (int k = 0; k < NPL; ++k)
+    x[k] = tq_load_elem(a.q, static_cast<int64_t>(head) * D + lane + 32 * k, a.dtype);
+  if (a.rc != nullptr) {
+    constexpr int HALF = NPL / 2;
+#pragma unroll
+    for (int k = 0; k < HALF; ++k) {
+      const float c = a.rc[pos * (D / 2) + lane + 32 * k];
+      const float s = a.rs[pos * (D / 2) + lane + 32 * k];
+      const float u = x[k], v = x[k + HALF];
+      x[k] = u * c - v * s;
+      x[k + HALF] = v * c + u * s;
+    }
+  }
+  tq_apply_signs<NPL>(x, a.books.dneg, lane);
+  tq_warp_wht<NPL>(x, lane);
+  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) {
+    x[k] *= inv_sqrt_d;
+    a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
+    qs[warp][lane + 32 * k] = x[k];
+  }
+  __syncwarp();
+  if (!a.books.qjl) return;
+  // q'' = S q': row i of S read coalesced by the warp, reduced by shuffles
+  for (int i = 0; i < D; ++i) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k)
+      acc = fmaf(tq_bf16_to_f32(a.S[i * D + lane + 32 * k]), qs[warp][lane + 32 * k], acc);
+    acc = tq_warp_sum(acc);
+    if (lane == 0) a.q2[static_cast<int64_t>(head) * D + i] = acc;
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(CT) chunk_kernel(DecodeArgs a) {
+  constexpr int NPL = D / 32;
+  constexpr int SLICES = CT / D;         // thread groups sharing one coordinate
+  constexpr int SUB = G >= 8 ? 512 : 1024;  // rows per pass inside a chunk
+  __shared__ float q1s[D][G], q2s[D][G];
+  __shared__ float cks[TQ_MAX_LEVELS], cvs[TQ_MAX_LEVELS];
+  __shared__ float w[SUB][G];            // logits, then weights p * nu_v
+  __shared__ float red[CT / 32][G];
+  __shared__ float stat[2][G];           // running max, running sum
+  __shared__ float oacc[SLICES][G][D];
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int len = seq_len_of(a, b);
+  const int c0 = split * a.chunk;
+  const int c1 = min(len, c0 + a.chunk);
+  const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
+  const int hq0 = kvh * G;
+
+  for (int e = tid; e < D * G; e += CT) {
+    const int i = e / G, h = e % G;
+    const int64_t qi = (static_cast<int64_t>(b) * a.Hq + hq0 + h) * D + i;
+    q1s[i][h] = a.q1[qi];
+    q2s[i][h] = a.books.qjl ? a.q2[qi] : 0.f;
+  }
+  if (tid < TQ_MAX_LEVELS) {
+    cks[tid] = a.books.ck[tid];
+    cvs[tid] = a.books.cv[tid];
+  }
+  if (tid < G) {
+    stat[0][tid] = -CUDART_INF_F;
+    stat[1][tid] = 0.f;
+  }
+  __syncthreads();
+
+  const int planes_k = a.books.mse_bits_k + a.books.qjl;
+  const int mbk = a.books.mse_bits_k;
+  const int coord = tid % D, slice = tid / D;
+  float o[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) o[h] = 0.f;
+
+  for (int s0 = c0; s0 < c1; s0 += SUB) {
+    const int s1 = min(c1, s0 + SUB);
+    // ---------------- phase 1: logits from the key planes (thread per row)
+    for (int r = s0 + tid; r < s1; r += CT) {
+      const uint32_t *krow = reinterpret_cast<const uint32_t *>(
+          a.kcode + (bh * a.rows_cap + r) * planes_k * (D / 8));
+      uint32_t kw[4][NPL], sw[NPL];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) kw[p][k] = p < mbk ? krow[p * NPL + k] : 0u;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) sw[k] = planes_k > mbk ? krow[mbk * NPL + k] : 0u;
+      const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale)[bh * a.rows_cap + r];
+      const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+      const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+      float acc[G], accs[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = accs[h] = 0.f;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+#pragma unroll 8
+        for (int bit = 0; bit < 32; ++bit) {
+          const int i = 32 * k + bit;
+          int idx = 0;
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+            if (p < mbk) idx |= ((kw[p][k] >> bit) & 1) << p;
+          const float cval = cks[idx];
+          const bool sg = (sw[k] >> bit) & 1;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            acc[h] = fmaf(q1s[i][h], cval, acc[h]);
+            accs[h] += sg ? q2s[i][h] : -q2s[i][h];
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float est = a.books.qjl ? acc[h] + a.qjl_coef * rho * accs[h] : acc[h];
+        const float l = a.scale * nu * est;
+        w[r - s0][h] = l;
+        if (a.logits)
+          a.logits[(static_cast<int64_t>(b) * a.Hq + hq0 + h) * a.max_len + r] = l;
+      }
+    }
+    __syncthreads();
+    // ---------------- phase 2: softmax statistics, weights p * nu_v
+    float lmax[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) lmax[h] = -CUDART_INF_F;
+    for (int r = tid; r < s1 - s0; r += CT)
+#pragma unroll
+      for (int h = 0; h < G; ++h) lmax[h] = fmaxf(lmax[h], w[r][h]);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float m = tq_warp_max(lmax[h]);
+      if (lane == 0) red[warp][h] = m;
+    }
+    __syncthreads();
+    float mnew[G], corr[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float m = red[0][h];
+      for (int i = 1; i < CT / 32; ++i) m = fmaxf(m, red[i][h]);
+      mnew[h] = fmaxf(stat[0][h], m);
+      corr[h] = __expf(stat[0][h] - mnew[h]);
+    }
+    __syncthreads();
+    float lsum[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) lsum[h] = 0.f;
+    for (int r = tid; r < s1 - s0; r += CT) {
+      const float nv = tq_half_to_f32(a.vnorm[bh * a.rows_cap + s0 + r]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float p = __expf(w[r][h] - mnew[h]);
+        lsum[h] += p;
+        w[r][h] = p * nv;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float sm = tq_warp_sum(lsum[h]);
+      if (lane == 0) red[warp][h] = sm;
+    }
+    __syncthreads();
+    if (tid < G) {
+      float sm = 0.f;
+      for (int i = 0; i < CT / 32; ++i) sm += red[i][tid];
+      stat[1][tid] = stat[1][tid] * corr[tid] + sm;
+      stat[0][tid] = mnew[tid];
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) o[h] *= corr[h];
+    // ---------------- phase 3: rotated-domain value sum (thread per coordinate)
+    const int nbv = a.books.bits_v;
+    for (int g = s0 / 32 + slice; g * 32 < s1; g += SLICES) {
+      const uint32_t *vg = a.vcode + (bh * (a.rows_cap / 32) + g) * nbv * D + coord;
+      uint32_t vw[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) vw[p] = p < nbv ? vg[p * D] : 0u;
+      const int rlo = max(s0, g * 32), rhi = min(s1, g * 32 + 32);
+      for (int r = rlo; r < rhi; ++r) {
+        const int bit = r & 31;
+        int idx = 0;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) idx |= ((vw[p] >> bit) & 1) << p;
+        const float cval = cvs[idx];
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = fmaf(w[r - s0][h], cval, o[h]);
+      }
+    }
+    __syncthreads();
+  }
+  // reduce the coordinate slices and write the chunk partials
+#pragma unroll
+  for (int h = 0; h < G; ++h) oacc[slice][h][coord] = o[h];
+  __syncthreads();
+  for (int e = tid; e < G * D; e += CT) {
+    const int h = e / D, i = e % D;
+    float s = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SLICES; ++sl) s += oacc[sl][h][i];
+    const int64_t hq = static_cast<int64_t>(b) * a.Hq + hq0 + h;
+    a.po[(hq * a.splits + split) * D + i] = s;
+  }
+  if (tid < G) {
+    const int64_t hq = static_cast<int64_t>(b) * a.Hq + hq0 + tid;
+    a.pml[(hq * a.splits + split) * 2 + 0] = stat[0][tid];
+    a.pml[(hq * a.splits + split) * 2 + 1] = stat[1][tid];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(QW * 32) combine_kernel(DecodeArgs a) {
+  constexpr int NPL = D / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int head = blockIdx.x * QW + warp;
+  if (head >= a.B * a.Hq) return;
+  float m = -CUDART_INF_F;
+  for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.pml[(static_cast<int64_t>(head) * a.splits + s) * 2]);
+  m = tq_warp_max(m);
+  float x[NPL], l = 0.f;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) x[k] = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const int64_t base = static_cast<int64_t>(head) * a.splits + s;
+    const float ms = a.pml[base * 2], ls = a.pml[base * 2 + 1];
+    if (ls == 0.f) continue;
+    const float f = __expf(ms - m);
+    l += ls * f;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) x[k] = fmaf(a.po[base * D + lane + 32 * k], f, x[k]);
+  }
+  tq_warp_wht<NPL>(x, lane);
+  tq_apply_signs<NPL>(x, a.books.dneg, lane);
+  const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * l);
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) a.out[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k] * norm;
+}
+
+template <int D>
+int run_decode(DecodeArgs &a, cudaStream_t stream) {
+  const int heads = a.B * a.Hq;
+  qprep_kernel<D><<<(heads + QW - 1) / QW, QW * 32, 0, stream>>>(a);
+  if (int e = tq_check_launch("qprep_kernel")) return e;
+  dim3 grid(a.splits, a.Hkv, a.B);
+  cudaEvent_t ev0, ev1;
+  tq_timing_events(&ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, stream);
+  switch (a.G) {
+    case 1: chunk_kernel<D, 1><<<grid, CT, 0, stream>>>(a); break;
+    case 2: chunk_kernel<D, 2><<<grid, CT, 0, stream>>>(a); break;
+    case 4: chunk_kernel<D, 4><<<grid, CT, 0, stream>>>(a); break;
+    case 8: chunk_kernel<D, 8><<<grid, CT, 0, stream>>>(a); break;
+    default: return tq_fail(TQ_ERR_UNSUPPORTED, "decode: GQA group size must be 1, 2, 4 or 8");
+  }
+  if (int e = tq_check_launch("chunk_kernel")) return e;
+  if (ev1) cudaEventRecord(ev1, stream);
+  combine_kernel<D><<<(heads + QW - 1) / QW, QW * 32, 0, stream>>>(a);
+  tq_count_launch(3);
+  return tq_check_launch("combine_kernel");
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits) {
+  const size_t heads = static_cast<size_t>(B) * Hq;
+  return sizeof(float) * heads * (2 * c->d + static_cast<size_t>(splits) * (c->d + 2));
+}
+
+int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                  const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
+                  const float *rc, const float *rs, int splits, void *ws, float *out,
+                  float *logits, cudaStream_t stream) {
+  DecodeArgs a;
+  a.q = q;
+  a.dtype = dtype;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.kcode = cache->kcode;
+  a.kscale = cache->kscale;
+  a.vcode = cache->vcode;
+  a.vnorm = cache->vnorm;
+  a.rows_cap = cache->rows_cap;
+  a.seq_lens = seq_lens;
+  a.max_len = max_len;
+  a.scale = scale;
+  a.qjl_coef = c->qjl_k ? sqrtf(static_cast<float>(M_PI) / 2.0f) / c->d : 0.f;
+  a.rc = rc;
+  a.rs = rs;
+  a.splits = splits;
+  const int per = (max_len + splits - 1) / splits;
+  a.chunk = (per + 31) / 32 * 32;
+  a.S = c->S_dev;
+  const size_t heads = static_cast<size_t>(B) * Hq;
+  float *f = static_cast<float *>(ws);
+  a.q1 = f;
+  a.q2 = f + heads * c->d;
+  a.po = f + 2 * heads * c->d;
+  a.pml = a.po + heads * static_cast<size_t>(splits) * c->d;
+  a.out = out;
+  a.logits = logits;
+  a.books = c->books;
+  switch (c->d) {
+    case 64: return run_decode<64>(a, stream);
+    case 128: return run_decode<128>(a, stream);
+    default: return tq_fail(TQ_ERR_UNSUPPORTED, "decode: head dim not built");
+  }
+}

@@ -1,0 +1,91 @@
+// Device helpers: number formats, warp reductions and the warp-resident
+// Walsh-Hadamard transform.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "tq_internal.h"
+
+#define TQ_FULL 0xffffffffu
+
+__device__ __forceinline__ float tq_load_elem(const void *p, int64_t i, int dtype) {
+  if (dtype == TQ_BF16) {
+    const uint16_t b = reinterpret_cast<const uint16_t *>(p)[i];
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+  }
+  return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ float tq_bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float tq_half_to_f32(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ uint16_t tq_f32_to_half(float f) {
+  return __half_as_ushort(__float2half_rn(f));
+}
+
+__device__ __forceinline__ float tq_warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(TQ_FULL, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float tq_warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(TQ_FULL, v, o));
+  return v;
+}
+
+// Unnormalised Walsh-Hadamard transform (Sylvester / natural order) of a
+// d-vector held by one warp with coordinate i = lane + 32 k in x[k],
+// k < NPL = d / 32.  Output y = H_d x.
+template <int NPL>
+__device__ __forceinline__ void tq_warp_wht(float (&x)[NPL], int lane) {
+  // strides 1..16: lane bits, exchanged with shuffles
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+    const bool upper = lane & s;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      const float o = __shfl_xor_sync(TQ_FULL, x[k], s);
+      x[k] = upper ? (o - x[k]) : (x[k] + o);
+    }
+  }
+  // strides 32, 64, ...: register index bits
+#pragma unroll
+  for (int s = 1; s < NPL; s <<= 1) {
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      if (!(k & s)) {
+        const float a = x[k], b = x[k + s];
+        x[k] = a + b;
+        x[k + s] = a - b;
+      }
+    }
+  }
+}
+
+// x_i *= D_i for coordinate i = lane + 32 k (dneg bit set <=> D_i = -1).
+template <int NPL>
+__device__ __forceinline__ void tq_apply_signs(float (&x)[NPL], const uint32_t *dneg, int lane) {
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) {
+    const uint32_t neg = (dneg[k] >> lane) & 1u;
+    x[k] = __uint_as_float(__float_as_uint(x[k]) ^ (neg << 31));
+  }
+}
+
+// Scalar code: #{k : u >= t[k]} over `nt` thresholds (ties go up).
+__device__ __forceinline__ int tq_code(float u, const float *t, int nt) {
+  int idx = 0;
+#pragma unroll
+  for (int k = 0; k < TQ_MAX_LEVELS - 1; ++k)
+    if (k < nt) idx += (u >= t[k]) ? 1 : 0;
+  return idx;
+}

@@ -1,0 +1,60 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/tq.h"
+
+namespace tqhost {
+bool lloyd_max(int d, int bits, std::vector<double> &c, std::vector<double> &t, double &mse);
+}
+
+// Largest head dim the kernels are instantiated for.
+constexpr int TQ_MAX_D = 128;
+constexpr int TQ_MAX_LEVELS = 16;
+
+// Codebooks and rotation signs passed by value to every kernel (kernel
+// parameter space is broadcast-friendly and needs no device allocation).
+struct TqBooks {
+  float ck[TQ_MAX_LEVELS];   // key centroids (MSE stage)
+  float tk[TQ_MAX_LEVELS];   // key thresholds (count = levels - 1)
+  float cv[TQ_MAX_LEVELS];   // value centroids
+  float tv[TQ_MAX_LEVELS];   // value thresholds
+  uint32_t dneg[TQ_MAX_D / 32];  // bit i set <=> D_i = -1
+  int mse_bits_k;
+  int qjl;
+  int bits_v;
+};
+
+struct tq_codec {
+  int d;
+  int bits_k, qjl_k, bits_v, mse_bits_k;
+  TqBooks books;
+  uint16_t *S_dev;     // bf16 [d][d] row-major S[i][j]
+  int device;
+};
+
+// Profiling hooks (api.cu).
+void tq_count_launch(int n);
+void tq_timing_events(cudaEvent_t *start, cudaEvent_t *stop);
+
+// Error reporting (thread-local message).
+int tq_fail(int code, const std::string &msg);
+int tq_check_launch(const char *what);
+
+// Kernel launchers (defined in the .cu files).
+int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
+                    int T, int64_t sb, int64_t sh, int64_t st, const float *rc, const float *rs,
+                    int64_t pos0, const tq_cache *cache, int64_t row0, uint32_t *status,
+                    cudaStream_t stream);
+size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits);
+int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                  const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
+                  const float *rc, const float *rs, int splits, void *ws, float *out,
+                  float *logits, cudaStream_t stream);
+int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
+                   int64_t rows, float *out, cudaStream_t stream);

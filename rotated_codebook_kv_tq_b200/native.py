@@ -1,0 +1,258 @@
+"""ctypes binding of ``libtq_b200.so`` (the C ABI declared in ``include/tq.h``).
+
+Argument marshalling only: every step of the codec runs in the library's CUDA
+kernels.  Tensors are PyTorch tensors used for device memory and streams.  If
+the shared library is missing the import of this module's functions raises:
+there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtq_b200.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(6)
+TQ_F32, TQ_BF16 = 0, 1
+
+EXPORTS = [
+    "tq_build_codebook", "tq_codec_create", "tq_codec_destroy", "tq_codec_codebooks",
+    "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
+    "tq_attention_logits", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
+    "tq_last_error",
+]
+
+
+class TqError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"tq status {code}: {msg}")
+        self.code = code
+
+
+class CodecDesc(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("bits_k", ctypes.c_int), ("qjl_k", ctypes.c_int),
+                ("bits_v", ctypes.c_int), ("rotation_signs", ctypes.c_void_p),
+                ("qjl_bf16", ctypes.c_void_p)]
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("kcode", ctypes.c_void_p), ("kscale", ctypes.c_void_p),
+                ("vcode", ctypes.c_void_p), ("vnorm", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("rows_cap", ctypes.c_int64)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m rotated_codebook_kv_tq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        sz = ctypes.c_size_t
+        L.tq_build_codebook.argtypes = [i32, i32, vp, vp, vp]
+        L.tq_codec_create.argtypes = [ctypes.POINTER(CodecDesc), ctypes.POINTER(vp)]
+        L.tq_codec_destroy.argtypes = [vp]
+        L.tq_codec_destroy.restype = None
+        L.tq_codec_codebooks.argtypes = [vp, vp, vp, vp, vp]
+        L.tq_cache_bytes.argtypes = [vp, i32, i32, i64, ctypes.POINTER(sz)]
+        L.tq_quantize_kv.argtypes = [vp, vp, vp, i32, i32, i32, i32, i64, i64, i64, vp, vp, i64,
+                                     ctypes.POINTER(CacheDesc), i64, vp, vp]
+        L.tq_attention_workspace.argtypes = [vp, i32, i32, i32, ctypes.POINTER(sz)]
+        L.tq_attention_decode.argtypes = [vp, vp, i32, i32, i32, i32, ctypes.POINTER(CacheDesc),
+                                          vp, i32, f32, vp, vp, i32, vp, sz, vp, vp]
+        L.tq_attention_logits.argtypes = L.tq_attention_decode.argtypes[:-1] + [vp, vp]
+        L.tq_dequantize.argtypes = [vp, ctypes.POINTER(CacheDesc), i32, i64, i64, vp, vp]
+        L.tq_set_timing_events.argtypes = [vp, vp]
+        L.tq_launch_count.argtypes = []
+        L.tq_launch_count.restype = ctypes.c_uint64
+        L.tq_last_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def check(code: int) -> None:
+    if code != TQ_OK:
+        raise TqError(code, lib().tq_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+# ---------------------------------------------------------------- codebook
+
+def build_codebook(d: int, bits: int):
+    """tq_build_codebook -> (centroids fp32, thresholds fp32, mse_per_coord)."""
+    c = np.zeros(1 << bits, np.float32)
+    t = np.zeros((1 << bits) - 1 if bits > 0 else 0, np.float32)
+    mse = ctypes.c_double(0.0)
+    check(lib().tq_build_codebook(d, bits, c.ctypes.data, t.ctypes.data, ctypes.addressof(mse)))
+    return c, t, mse.value
+
+
+# ---------------------------------------------------------------- codec
+
+class Codec:
+    """Owns a ``tq_codec`` (device copies of D, S and the codebooks)."""
+
+    def __init__(self, d: int, bits_k: int, qjl_k: bool, bits_v: int,
+                 rotation_signs: np.ndarray, qjl_bf16: Optional[np.ndarray]):
+        self.d, self.bits_k, self.qjl_k, self.bits_v = d, bits_k, bool(qjl_k), bits_v
+        self.mse_bits_k = bits_k - 1 if qjl_k else bits_k
+        self.planes_k = self.mse_bits_k + (1 if qjl_k else 0)
+        signs = np.ascontiguousarray(rotation_signs, dtype=np.int8)
+        s = None if qjl_bf16 is None else np.ascontiguousarray(qjl_bf16, dtype=np.uint16)
+        desc = CodecDesc(d, bits_k, 1 if qjl_k else 0, bits_v, signs.ctypes.data,
+                         None if s is None else s.ctypes.data)
+        h = ctypes.c_void_p()
+        check(lib().tq_codec_create(ctypes.byref(desc), ctypes.byref(h)))
+        self.handle = h
+
+    def codebooks(self):
+        nk, nv = 1 << self.mse_bits_k, 1 << self.bits_v
+        ck, tk = np.zeros(nk, np.float32), np.zeros(nk - 1, np.float32)
+        cv, tv = np.zeros(nv, np.float32), np.zeros(nv - 1, np.float32)
+        check(lib().tq_codec_codebooks(self.handle, ck.ctypes.data, tk.ctypes.data,
+                                       cv.ctypes.data, tv.ctypes.data))
+        return ck, tk, cv, tv
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            lib().tq_codec_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+@dataclass
+class Cache:
+    """Compressed cache planes (device tensors owned by the caller)."""
+    kcode: "object"
+    kscale: "object"
+    vcode: "object"
+    vnorm: "object"
+    B: int
+    Hkv: int
+    rows_cap: int
+
+    def desc(self) -> CacheDesc:
+        return CacheDesc(self.kcode.data_ptr(), self.kscale.data_ptr(), self.vcode.data_ptr(),
+                         self.vnorm.data_ptr(), self.B, self.Hkv, self.rows_cap)
+
+
+def cache_bytes(codec: Codec, B: int, Hkv: int, rows_cap: int):
+    out = (ctypes.c_size_t * 4)()
+    check(lib().tq_cache_bytes(codec.handle, B, Hkv, rows_cap, out))
+    return list(out)
+
+
+def alloc_cache(codec: Codec, B: int, Hkv: int, rows_cap: int, device="cuda") -> Cache:
+    import torch
+    d = codec.d
+    return Cache(
+        kcode=torch.zeros((B, Hkv, rows_cap, codec.planes_k, d // 8), dtype=torch.uint8, device=device),
+        kscale=torch.zeros((B, Hkv, rows_cap, 2), dtype=torch.float16, device=device),
+        vcode=torch.zeros((B, Hkv, rows_cap // 32, codec.bits_v, d), dtype=torch.int32, device=device),
+        vnorm=torch.zeros((B, Hkv, rows_cap), dtype=torch.float16, device=device),
+        B=B, Hkv=Hkv, rows_cap=rows_cap)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return TQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ---------------------------------------------------------------- calls
+
+def quantize_kv(codec: Codec, k, v, cache: Cache, row0: int = 0, rope=None, pos0: int = 0,
+                status=None, stream=None) -> None:
+    """tq_quantize_kv on k, v [B, Hkv, T, d] (last dim contiguous, same strides)."""
+    B, H, T, d = k.shape
+    if tuple(v.shape) != tuple(k.shape) or v.stride() != k.stride() or k.stride(3) != 1:
+        raise ValueError("k and v need the same shape and strides, last dim contiguous")
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    check(lib().tq_quantize_kv(codec.handle, k.data_ptr(), v.data_ptr(), _dtype_code(k), B, H, T,
+                               k.stride(0), k.stride(1), k.stride(2), _ptr(rc), _ptr(rs), pos0,
+                               ctypes.byref(desc), row0, _ptr(status), _stream(stream)))
+
+
+def attention_workspace(codec: Codec, B: int, Hq: int, num_splits: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().tq_attention_workspace(codec.handle, B, Hq, num_splits, ctypes.byref(n)))
+    return n.value
+
+
+def attention_decode(codec: Codec, q, cache: Cache, max_seq_len: int, scale: float, out,
+                     workspace, seq_lens=None, rope=None, num_splits: int = 0,
+                     stream=None) -> None:
+    """tq_attention_decode: q [B, Hq, d] -> out [B, Hq, d] fp32."""
+    B, Hq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib().tq_attention_decode(codec.handle, q.data_ptr(), _dtype_code(q), B, Hq, cache.Hkv,
+                                    ctypes.byref(desc), _ptr(seq_lens), max_seq_len,
+                                    float(scale), _ptr(rc), _ptr(rs), num_splits,
+                                    workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                                    _stream(stream)))
+
+
+def attention_logits(codec: Codec, q, cache: Cache, max_seq_len: int, scale: float, out,
+                     logits, workspace, seq_lens=None, rope=None, num_splits: int = 0,
+                     stream=None) -> None:
+    """tq_attention_logits: decode plus the estimated logits [B, Hq, max_seq_len]."""
+    B, Hq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib().tq_attention_logits(codec.handle, q.data_ptr(), _dtype_code(q), B, Hq, cache.Hkv,
+                                    ctypes.byref(desc), _ptr(seq_lens), max_seq_len,
+                                    float(scale), _ptr(rc), _ptr(rs), num_splits,
+                                    workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                                    logits.data_ptr(), _stream(stream)))
+
+
+def dequantize(codec: Codec, cache: Cache, which: int, row0: int, rows: int, out,
+               stream=None) -> None:
+    """tq_dequantize: rows [row0, row0+rows) of every (b, h) -> out [B, Hkv, rows, d]."""
+    desc = cache.desc()
+    check(lib().tq_dequantize(codec.handle, ctypes.byref(desc), which, row0, rows,
+                              _ptr(out), _stream(stream)))
+
+
+def set_timing_events(start=None, stop=None) -> None:
+    """tq_set_timing_events with torch.cuda.Event objects (or None, None)."""
+    check(lib().tq_set_timing_events(None if start is None else start.cuda_event,
+                                     None if stop is None else stop.cuda_event))
+
+
+def launch_count() -> int:
+    return int(lib().tq_launch_count())

@@ -1,0 +1,203 @@
+"""GPU-vs-oracle parity through the C ABI (quantize, dequantize, decode).
+
+Sizes are small enough for the oracle to finish in seconds but span several
+tiles, ragged tails, partially covered 32-token value groups and empty split-K
+chunks.  Full-size checks (the launch configuration bench.py times) live in
+test_gpu_fullsize.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oatt
+from oracle import codec as oc
+from rotated_codebook_kv_tq_b200 import native, synth
+import tq_testlib as tl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    tl.require_cuda()
+
+
+def _inputs(w):
+    K, V = synth.kv_inputs(w)
+    return K, V, synth.as_float64(K, w.dtype), synth.as_float64(V, w.dtype)
+
+
+QUANT_CASES = {
+    "tiny": (synth.WORKLOADS["tiny"], [(0, 1024)]),
+    "llama_ragged": (synth.WORKLOADS["llama_decode"].scaled(T=200), [(0, 200)]),
+    "llama_appends": (synth.WORKLOADS["llama_decode"].scaled(T=138), [(0, 100), (100, 1), (101, 37)]),
+    "esm_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=3, Hkv=3, T=100), [(0, 100)]),
+    "long_2bit": (synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=300), [(0, 300)]),
+}
+
+
+def _quantize_both(w, segments, rows_cap=None):
+    ocodec, ncodec = tl.codecs(w)
+    K, V, K64, V64 = _inputs(w)
+    rows_cap = rows_cap or (w.T + 31) // 32 * 32
+    rope = synth.rope_for(w, rows_cap)
+    ocache = oc.empty_cache(ocodec, w.B, w.Hkv, rows_cap)
+    ncache = native.alloc_cache(ncodec, w.B, w.Hkv, rows_cap)
+    kd, vd = tl.to_device(K, w.dtype), tl.to_device(V, w.dtype)
+    rd = tl.rope_device(rope)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    encs = {}
+    for row0, T in segments:
+        sl = slice(row0, row0 + T)
+        diag = oc.quantize_into(ocache, K64[:, :, sl], V64[:, :, sl], ocodec, rope=rope,
+                                pos0=row0, row0=row0)
+        native.quantize_kv(ncodec, kd[:, :, sl], vd[:, :, sl], ncache, row0=row0, rope=rd,
+                           pos0=row0, status=status)
+        i = 0
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                encs.setdefault((b, h), []).append((np.arange(row0, row0 + T), diag["k"][i], diag["v"][i]))
+                i += 1
+    torch.cuda.synchronize()
+    return ocodec, ncodec, ocache, ncache, encs, int(status.item())
+
+
+@pytest.mark.parametrize("case", list(QUANT_CASES))
+def test_quantize_parity(case):
+    w, segments = QUANT_CASES[case]
+    ocodec, ncodec, ocache, ncache, encs, bad = _quantize_both(w, segments)
+    gpu = tl.download_cache(ncache)
+    stats = tl.new_stats()
+    for (b, h), parts in encs.items():
+        for rows, ek, ev in parts:
+            tl.compare_rows(gpu, ocache, ocodec, b, h, rows, ek, ev, stats)
+    tl.assert_mismatch_budget(stats)
+    assert bad == 0
+    # rows outside the written ranges stay zero
+    written = max(r0 + T for r0, T in segments)
+    assert not gpu["kcode"][:, :, written:].any()
+    assert not gpu["vnorm"][:, :, written:].any()
+
+
+def test_quantize_zero_and_nonfinite_rows():
+    w = synth.WORKLOADS["llama_decode"].scaled(B=1, Hkv=2, Hq=8, T=64)
+    ocodec, ncodec = tl.codecs(w)
+    K, V, K64, V64 = _inputs(w)
+    Kf = synth.bf16_bits_to_f32(K).copy()
+    Vf = synth.bf16_bits_to_f32(V).copy()
+    Kf[0, 0, 3] = 0.0
+    Kf[0, 1, 5, 17] = np.nan
+    Vf[0, 0, 9, 2] = np.inf
+    Vf[0, 1, 10] = 0.0
+    Kf[0, 1, 40, 0] = 1e6          # key norm overflows fp16
+    w32 = w.scaled(dtype="fp32")
+    rope = synth.rope_for(w32, 64)
+    ocache = oc.empty_cache(ocodec, 1, 2, 64)
+    diag = oc.quantize_into(ocache, Kf.astype(np.float64), Vf.astype(np.float64), ocodec, rope=rope)
+    ncache = native.alloc_cache(ncodec, 1, 2, 64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    native.quantize_kv(ncodec, tl.to_device(Kf, "fp32"), tl.to_device(Vf, "fp32"), ncache,
+                       rope=tl.rope_device(rope), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == diag["bad_rows"] == 3
+    gpu = tl.download_cache(ncache)
+    stats = tl.new_stats()
+    for i, (b, h) in enumerate([(0, 0), (0, 1)]):
+        tl.compare_rows(gpu, ocache, ocodec, b, h, np.arange(64), diag["k"][i], diag["v"][i], stats)
+    tl.assert_mismatch_budget(stats)
+    assert gpu["kscale"][0, 1, 5, 0] == 0 and gpu["vnorm"][0, 0, 9] == 0
+
+
+@pytest.mark.parametrize("case", ["tiny", "llama_ragged", "esm_d64", "long_2bit"])
+def test_dequantize_parity(case):
+    w, segments = QUANT_CASES[case]
+    ocodec, ncodec = tl.codecs(w)
+    K, V, K64, V64 = _inputs(w)
+    rows_cap = (w.T + 31) // 32 * 32
+    rope = synth.rope_for(w, rows_cap)
+    ocache = oc.empty_cache(ocodec, w.B, w.Hkv, rows_cap)
+    oc.quantize_into(ocache, K64, V64, ocodec, rope=rope)
+    ncache = tl.upload_cache(ocache, ncodec, w.B, w.Hkv)
+    row0, rows = 3, w.T - 3
+    for which in (0, 1):
+        out = torch.empty((w.B, w.Hkv, rows, w.d), dtype=torch.float32, device="cuda")
+        native.dequantize(ncodec, ncache, which, row0, rows, out)
+        got = out.cpu().numpy().astype(np.float64)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                ik, sg, nk, rk, iv, nv = oc.cache_rows(ocache, ocodec, b, h, w.T)
+                ref = (oc.dequant_keys(ik, sg, nk, rk, ocodec) if which == 0
+                       else oc.dequant_values(iv, nv, ocodec))[row0:]
+                err = np.linalg.norm(got[b, h] - ref, axis=1)
+                nrm = np.linalg.norm(ref, axis=1)
+                assert np.all(err <= 1e-3 * nrm + 1e-30), (which, b, h, np.max(err / np.maximum(nrm, 1e-30)))
+
+
+DECODE_CASES = {
+    "tiny": (synth.WORKLOADS["tiny"], None, 8),
+    "llama_splits7": (synth.WORKLOADS["llama_decode"].scaled(T=1000), None, 7),
+    "llama_one_split": (synth.WORKLOADS["llama_decode"].scaled(B=1, Hq=8, Hkv=2, T=3000), None, 1),
+    "long_empty_splits": (synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=3000), None, 128),
+    "esm_mha_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=3, Hkv=3, T=300, Lq=1), None, 4),
+    "ragged_lens": (synth.WORKLOADS["llama_decode"].scaled(B=3, Hq=8, Hkv=2, T=300), [1, 77, 300], 5),
+    "gqa8": (synth.WORKLOADS["long_decode"].scaled(B=1, Hq=16, Hkv=2, T=500), None, 3),
+}
+
+
+def _decode_case(w, lens, splits):
+    ocodec, ncodec = tl.codecs(w)
+    K, V, K64, V64 = _inputs(w)
+    rows_cap = (w.T + 31) // 32 * 32
+    rope = synth.rope_for(w, rows_cap)
+    ocache = oc.empty_cache(ocodec, w.B, w.Hkv, rows_cap)
+    oc.quantize_into(ocache, K64, V64, ocodec, rope=rope)
+    ncache = tl.upload_cache(ocache, ncodec, w.B, w.Hkv)
+    q = synth.query_inputs(w, Lq=1)[:, :, 0]
+    q64 = synth.as_float64(q, w.dtype)
+    scale = 1.0 / math.sqrt(w.d)
+    lens = [w.T] * w.B if lens is None else lens
+    ref, ref_logits = oatt.decode(q64, ocache, ocodec, lens, scale, rope=rope, want_logits=True)
+    ws = torch.empty(native.attention_workspace(ncodec, w.B, w.Hq, splits) // 4 + 4,
+                     dtype=torch.float32, device="cuda")
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    logits = torch.full((w.B, w.Hq, w.T), float("nan"), dtype=torch.float32, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    native.attention_logits(ncodec, tl.to_device(q, w.dtype), ncache, w.T, scale, out, logits, ws,
+                            seq_lens=sl, rope=tl.rope_device(rope), num_splits=splits)
+    torch.cuda.synchronize()
+    return ref, ref_logits, out.cpu().numpy().astype(np.float64), logits.cpu().numpy(), lens
+
+
+@pytest.mark.parametrize("case", list(DECODE_CASES))
+def test_decode_parity(case):
+    w, lens, splits = DECODE_CASES[case]
+    ref, ref_logits, got, got_logits, lens = _decode_case(w, lens, splits)
+    vscale = tl.channel_scale_of_values(w)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            lr = ref_logits[(b, h)]
+            lg = got_logits[b, h, :lens[b]].astype(np.float64)
+            rms = math.sqrt(np.mean(lr * lr))
+            assert np.max(np.abs(lg - lr)) <= 1e-3 * rms, (b, h, np.max(np.abs(lg - lr)) / rms)
+            err = np.abs(got[b, h] - ref[b, h]) / vscale[h // w.G]
+            assert np.max(err) <= 2e-3, (b, h, np.max(err))
+
+
+def test_decode_rejects_bad_arguments():
+    w = synth.WORKLOADS["tiny"]
+    _, ncodec = tl.codecs(w)
+    cache = native.alloc_cache(ncodec, 1, 1, 64)
+    q = torch.zeros((1, 1, 128), device="cuda")
+    out = torch.empty((1, 1, 128), device="cuda")
+    small = torch.empty(4, device="cuda")
+    with pytest.raises(native.TqError) as e:
+        native.attention_decode(ncodec, q, cache, 64, 0.1, out, small, num_splits=4)
+    assert e.value.code == native.TQ_ERR_WORKSPACE
+    ws = torch.empty(native.attention_workspace(ncodec, 1, 1, 4), dtype=torch.uint8, device="cuda")
+    with pytest.raises(native.TqError) as e:
+        native.attention_decode(ncodec, q, cache, 65, 0.1, out, ws, num_splits=4)
+    assert e.value.code == native.TQ_ERR_INVALID_ARG
+    with pytest.raises(native.TqError):
+        native.quantize_kv(ncodec, torch.zeros((1, 1, 70, 128), device="cuda"),
+                           torch.zeros((1, 1, 70, 128), device="cuda"), cache)
