@@ -1,0 +1,602 @@
+#!/usr/bin/env python
+"""Benchmark of the compressed-KV hot path on B200.
+
+One step = quantize-append of the new token's K/V (all KV heads) into the
+compressed cache + split-K decode attention of every query head over the T
+cached tokens, on the Llama-3.1-8B-shaped decode layer (B=1, 32 query / 8 KV
+heads, d=128, T=32768, keys 3+QJL bits, values 4 bits, bf16 inputs, RoPE).
+Prints ONE JSON line (rank 0).  Extra workloads (ESM-2-shaped prefill quantize
+GB/s, long-context decode) are reported under "extras".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torch.distributed.run (one rank per GPU); every rank runs
+its own independent replica of the workload (weak scaling, no collective on the
+data path); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=200)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="llama_decode")
+    p.add_argument("--no-extras", action="store_true")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sust=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"], samples=0)
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=float(rows[0][2]), reasons=reasons,
+                    samples=len(rows), power_w_max=max(float(r[3]) for r in rows
+                                                        if r[3].replace(".", "").isdigit()))
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# Decode workload (quantize-append + split-K decode per step)
+# ---------------------------------------------------------------------------
+
+def row_bytes(w) -> int:
+    """Compressed bytes per (token, KV head): key planes + (nu, rho), value planes + nu."""
+    mse_k = w.bits_k - 1 if w.qjl_k else w.bits_k
+    planes_k = mse_k + (1 if w.qjl_k else 0)
+    return planes_k * w.d // 8 + 4 + w.bits_v * w.d // 8 + 2
+
+
+def describe(w) -> str:
+    mse_k = w.bits_k - 1 if w.qjl_k else w.bits_k
+    kdesc = f"{mse_k}+QJL" if w.qjl_k else f"{mse_k}"
+    rope = f" RoPE theta={w.rope_theta:g}" if w.rope_theta else ""
+    return (f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} T={w.T} keys {kdesc} bits, "
+            f"values {w.bits_v} bits, {w.dtype} inputs{rope}, {w.num_splits} splits")
+
+
+class DecodeBench:
+    def __init__(self, w, n_sets: int):
+        import torch
+        from rotated_codebook_kv_tq_b200 import native, synth
+        self.w, self.n_sets = w, n_sets
+        self.native = native
+        D = synth.rotation_signs(w.d, w.seed)
+        S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
+        self.D, self.S = D, S
+        self.codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
+        T = w.T
+        self.rows_cap = (T + 31) // 32 * 32
+        K, V = synth.kv_inputs_torch(w, T=T)
+        self.K, self.V = K, V
+        r = synth.rope_for(w, self.rows_cap)
+        self.rope_np = r
+        self.rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+        self.caches = []
+        for _ in range(n_sets):
+            c = native.alloc_cache(self.codec, w.B, w.Hkv, self.rows_cap)
+            native.quantize_kv(self.codec, K[:, :, :T - 1], V[:, :, :T - 1], c, row0=0,
+                               rope=self.rope, pos0=0)
+            self.caches.append(c)
+        self.knew = K[:, :, T - 1:T].contiguous()
+        self.vnew = V[:, :, T - 1:T].contiguous()
+        self.q = synth.query_inputs_torch(w)[:, :, 0].contiguous()
+        self.scale = 1.0 / math.sqrt(w.d)
+        self.splits = w.num_splits
+        nbytes = native.attention_workspace(self.codec, w.B, w.Hq, self.splits)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+
+    def step(self, s: int, knew=None, vnew=None, q=None) -> None:
+        w, n = self.w, self.native
+        c = self.caches[s % self.n_sets]
+        n.quantize_kv(self.codec, self.knew if knew is None else knew,
+                      self.vnew if vnew is None else vnew, c, row0=w.T - 1, rope=self.rope,
+                      pos0=w.T - 1)
+        n.attention_decode(self.codec, self.q if q is None else q, c, w.T, self.scale, self.out,
+                           self.ws, rope=self.rope, num_splits=self.splits)
+
+    def cache_bytes_per_step(self) -> int:
+        return self.w.B * self.w.Hkv * self.w.T * row_bytes(self.w)
+
+
+def time_decode(bench: DecodeBench, K: int, W: int, world: int, sampler):
+    """Warm up W steps, then time exactly K steps replayed from CUDA graphs.
+    Returns (total seconds, mean chunk-kernel seconds, launches per step)."""
+    import torch
+    native = bench.native
+    c0 = native.launch_count()
+    bench.step(0)
+    torch.cuda.synchronize()
+    per_step = native.launch_count() - c0
+    M = min(K, 250)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(M)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(M)]
+    for ev in starts + stops:      # torch creates the CUDA event on first record
+        ev.record()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(M):
+            native.set_timing_events(starts[i], stops[i])
+            bench.step(i)
+        native.set_timing_events(None, None)
+    rem = K % M
+    tail = None
+    if rem:
+        tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail):
+            for i in range(rem):
+                bench.step(i)
+    for i in range(W):
+        bench.step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    e0.record()
+    for _ in range(K // M):
+        graph.replay()
+    if tail is not None:
+        tail.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    total = e0.elapsed_time(e1) / 1e3
+    try:
+        kern = statistics.mean(starts[i].elapsed_time(stops[i]) for i in range(M)) / 1e3
+    except Exception:
+        # events in graphs unusable: bracket the kernel in direct launches instead
+        kern = None
+    del graph, tail
+    if kern is None:
+        sa, so = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for i in range(50):
+            native.set_timing_events(sa, so)
+            bench.step(i)
+            native.set_timing_events(None, None)
+            torch.cuda.synchronize()
+            ts.append(sa.elapsed_time(so) / 1e3)
+        kern = statistics.median(ts)
+    return total, kern, per_step, clocks
+
+
+def time_e2e(bench: DecodeBench, K: int, W: int):
+    """Same step through the public API with host buffers: pinned H2D of the new
+    token's K/V and the query, the calls, D2H of the output, host sync each step."""
+    import torch
+    kh = bench.knew.cpu().pin_memory()
+    vh = bench.vnew.cpu().pin_memory()
+    qh = bench.q.cpu().pin_memory()
+    oh = torch.empty(bench.out.shape, dtype=torch.float32).pin_memory()
+    kd, vd, qd = torch.empty_like(bench.knew), torch.empty_like(bench.vnew), torch.empty_like(bench.q)
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qd.copy_(qh, non_blocking=True)
+        bench.step(i, kd, vd, qd)
+        oh.copy_(bench.out, non_blocking=True)
+        stream.synchronize()
+
+    for i in range(W):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(K):
+        one(i)
+    dt = time.perf_counter() - t0
+    h2d = (kh.numel() + vh.numel() + qh.numel()) * kh.element_size()
+    d2h = oh.numel() * oh.element_size()
+    return dt, h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# Oracle (CPU) baseline
+# ---------------------------------------------------------------------------
+
+class OracleDecode:
+    """The CPU oracle run on the same workload: quantize-append of the new token,
+    then estimator-form attention of every query head (fp64 numpy)."""
+
+    def __init__(self, bench: DecodeBench):
+        import numpy as np
+        from oracle import codec as oc
+        w = bench.w
+        self.w, self.oc = w, oc
+        self.codec = oc.make_codec(w.d, w.bits_k, w.qjl_k, w.bits_v, bench.D, bench.S)
+        self.K = bench.K.float().cpu().numpy().astype(np.float64)
+        self.V = bench.V.float().cpu().numpy().astype(np.float64)
+        self.q = bench.q.float().cpu().numpy().astype(np.float64)
+        self.rope = bench.rope_np
+        self.rows_cap = bench.rows_cap
+        self.cache = None
+
+    def prefill(self, rows: int):
+        """Untimed setup: cache rows 0 .. rows-2 (the new token is row rows-1)."""
+        oc, w = self.oc, self.w
+        self.n = rows
+        self.cache = oc.empty_cache(self.codec, w.B, w.Hkv, (rows + 31) // 32 * 32)
+        oc.quantize_into(self.cache, self.K[:, :, :rows - 1], self.V[:, :, :rows - 1], self.codec,
+                         rope=self.rope)
+
+    def step(self):
+        from oracle import attention as oatt
+        oc, w, n = self.oc, self.w, self.n
+        oc.quantize_into(self.cache, self.K[:, :, n - 1:n], self.V[:, :, n - 1:n], self.codec,
+                         rope=self.rope, pos0=n - 1, row0=n - 1)
+        return oatt.decode(self.q, self.cache, self.codec, [n] * w.B, 1.0 / math.sqrt(w.d),
+                           rope=self.rope)
+
+
+def oracle_rate(bench: DecodeBench, seconds: float, rows: int = None):
+    """Tokens/s of the oracle on a bounded sample: full decode steps over the
+    first ``rows`` tokens of the context, scaled linearly to the full context
+    (cost is linear in the number of cached tokens)."""
+    w = bench.w
+    rows = w.T if rows is None else rows
+    o = OracleDecode(bench)
+    o.prefill(rows)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        o.step()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds or n >= 1000:
+            break
+    per_step_full = dt / n * (w.T / rows)
+    return w.B / per_step_full, n, dt, rows
+
+
+# ---------------------------------------------------------------------------
+# Extra workloads
+# ---------------------------------------------------------------------------
+
+def quantize_extra(wname: str, pk: dict, steps: int = 40):
+    """Prefill quantize of a whole [B, H, T, d] K/V batch: input GB/s and the
+    kernel's HBM roofline fraction.  Rotates over input sets larger than L2."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.WORKLOADS[wname]
+    D = synth.rotation_signs(w.d, w.seed)
+    S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
+    codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
+    rows_cap = (w.T + 31) // 32 * 32
+    in_bytes = 2 * w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    n_sets = max(2, math.ceil(3 * l2 / in_bytes))
+    sets = []
+    for s in range(n_sets):
+        K, V = synth.kv_inputs_torch(w, seed_salt=s)
+        sets.append((K, V, native.alloc_cache(codec, w.B, w.Hkv, rows_cap)))
+    r = synth.rope_for(w, rows_cap)
+    rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+    for K, V, c in sets:
+        native.quantize_kv(codec, K, V, c, rope=rope)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        K, V, c = sets[i % n_sets]
+        evs[i][0].record()
+        native.quantize_kv(codec, K, V, c, rope=rope)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    t = statistics.median(a.elapsed_time(b) for a, b in evs) / 1e3
+    out_bytes = w.B * w.Hkv * w.T * row_bytes(w)
+    alg = in_bytes + out_bytes
+    return dict(workload=describe(w), input_GBps=in_bytes / t / 1e9, us_per_call=t * 1e6,
+                roofline=dict(bound="hbm", achieved=alg / t / 1e9, peak=pk["hbm"], unit="GB/s",
+                              frac=alg / t / 1e9 / pk["hbm"], algorithmic_bytes=alg),
+                l2="rotating %d input sets (%.0f MB)" % (n_sets, n_sets * in_bytes / 1e6))
+
+
+def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
+    import torch
+    from rotated_codebook_kv_tq_b200 import synth
+    w = synth.WORKLOADS[wname]
+    bench = DecodeBench(w, n_sets=1)
+
+    class _Null:
+        def start(self):
+            pass
+
+        def stop(self):
+            return {}
+
+    total, kern, _, _ = time_decode(bench, steps, warmup, 1, _Null())
+    alg = bench.cache_bytes_per_step()
+    res = dict(workload=describe(w), us_per_step=total / steps * 1e6,
+               tokens_per_s=w.B * steps / total,
+               roofline=dict(bound="hbm", achieved=alg / kern / 1e9, peak=pk["hbm"], unit="GB/s",
+                             frac=alg / kern / 1e9 / pk["hbm"], algorithmic_bytes=alg,
+                             kernel_us=kern * 1e6),
+               l2="cache %.0f MB per step > L2" % (alg / 1e6))
+    del bench
+    torch.cuda.empty_cache()
+    return res
+
+
+def ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of ``kernel`` from the committed ncu summary, or
+    None when the kernel's source changed after the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "rotated_codebook_kv_tq_b200", "csrc", d["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
+    return d["bytes_per_launch"] if h == d.get("source_sha") else None
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the CPU oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import numpy as np
+    from rotated_codebook_kv_tq_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    budget = 150.0
+    steps = args.steps + args.warmup
+
+    def oracle_for(rows):
+        ww = w.scaled(T=rows)
+        K, V = synth.kv_inputs(ww)
+        q = synth.query_inputs(ww, Lq=1)[:, :, 0]
+        o = OracleDecode.__new__(OracleDecode)
+        from oracle import codec as oc
+        o.w, o.oc = w, oc
+        S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
+        o.codec = oc.make_codec(w.d, w.bits_k, w.qjl_k, w.bits_v, synth.rotation_signs(w.d, w.seed), S)
+        o.K, o.V = synth.as_float64(K, w.dtype), synth.as_float64(V, w.dtype)
+        o.q = synth.as_float64(q, w.dtype)
+        o.rope = synth.rope_for(w, (rows + 31) // 32 * 32)
+        o.prefill(rows)
+        return o
+
+    probe = oracle_for(256)
+    t0 = time.perf_counter()
+    for _ in range(3):
+        probe.step()
+    t256 = (time.perf_counter() - t0) / 3
+    # cost ~ a + b * rows; take the probe as the per-step floor and size rows
+    per_step_budget = budget / steps
+    rows = int(max(32, min(w.T, 256 * per_step_budget / max(t256, 1e-9))))
+    rows = rows // 32 * 32 or 32
+    o = probe if rows == 256 else oracle_for(rows)
+    for _ in range(args.warmup):
+        o.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.step()
+    dt = time.perf_counter() - t0
+    per_step_full = dt / args.steps * (w.T / rows)
+    value = w.B / per_step_full
+    cores = blas_threads()
+    sample = (f"each step: oracle quantize-append + decode of all {w.Hq} query heads over the "
+              f"first {rows} of {w.T} cached tokens, time scaled by {w.T}/{rows}")
+    line = dict(impl="reference", metric="compressed-KV decode tokens/s", value=value,
+                unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=per_step_full * 1e3, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=describe(w)),
+                cpu_baseline=dict(value=value, unit="tokens/s", cores=cores, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Main
+# ---------------------------------------------------------------------------
+
+def smi_index(local: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    import torch
+    from rotated_codebook_kv_tq_b200 import synth
+    from rotated_codebook_kv_tq_b200.build import build
+    if rank == 0:
+        build()
+    barrier(world)
+    torch.cuda.set_device(local)
+    w = synth.WORKLOADS[args.workload]
+    pk = peaks()
+    K, W = args.steps, max(3, args.warmup)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    per_set = w.B * w.Hkv * ((w.T + 31) // 32 * 32) * row_bytes(w)
+    n_sets = max(1, math.ceil(3 * l2 / per_set))
+    bench = DecodeBench(w, n_sets)
+    sampler = ClockSampler(smi_index(local))
+    total, kern, per_step, clocks = time_decode(bench, K, W, world, sampler)
+    total = max_over_ranks(total, world)
+    kern = max_over_ranks(kern, world)
+    value = world * w.B * K / total
+    alg = bench.cache_bytes_per_step()
+    achieved = alg / kern / 1e9
+
+    K_e2e = max(10, min(K, 300))
+    dt, h2d, d2h = time_e2e(bench, K_e2e, 20)
+    dt = max_over_ranks(dt, world)
+    e2e_value = world * w.B * K_e2e / dt
+
+    line = dict(metric="compressed-KV decode tokens/s", value=value, unit="tokens/s",
+                n_gpus=world, steps=K, warmup=W, ms_per_step=total / K * 1e3,
+                us_per_step=total / K * 1e6, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f32", data="synthetic",
+                config=dict(workload=describe(w),
+                            l2=f"rotating {n_sets} compressed caches "
+                               f"({n_sets * per_set / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)",
+                            parallelism=f"{world} independent replicas" if world > 1 else "1 GPU"),
+                roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                              frac=achieved / pk["hbm"], traffic=ncu_traffic("chunk_kernel"),
+                              kernel="chunk_kernel (split-K decode main loop)",
+                              kernel_us=kern * 1e6, algorithmic_bytes=alg,
+                              bytes_per_token_head=row_bytes(w),
+                              peak_source=f"{pk['source']} hbm_gbs"),
+                e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
+                         d2h_bytes_per_step=d2h, us_per_step=dt / K_e2e * 1e6,
+                         note="public API, pinned host buffers, host sync every step"),
+                clocks=dict(sm_mhz=clocks.get("sm_mhz"), sm_max_mhz=clocks.get("sm_max_mhz"),
+                            reasons=clocks.get("reasons"), samples=clocks.get("samples")),
+                gpu_launches=per_step * K)
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rows = min(w.T, 8192)
+        rate, n, secs, rows = oracle_rate(bench, args.cpu_seconds, rows)
+        line["cpu_baseline"] = dict(
+            value=rate, unit="tokens/s", cores=blas_threads(), kind="oracle",
+            sample=f"{n} oracle decode steps (quantize-append + all {w.Hq} heads) over the first "
+                   f"{rows} of {w.T} tokens in {secs:.1f} s, scaled by {w.T}/{rows}")
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras = {}
+        try:
+            extras["quantize_esm_prefill"] = quantize_extra("esm_prefill", pk)
+        except Exception as e:  # report, do not hide
+            extras["quantize_esm_prefill"] = dict(error=repr(e))
+        try:
+            extras["decode_long_context"] = decode_extra("long_decode", pk)
+        except Exception as e:
+            extras["decode_long_context"] = dict(error=repr(e))
+        line["extras"] = extras
+    if rank == 0:
+        print(json.dumps(line))
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

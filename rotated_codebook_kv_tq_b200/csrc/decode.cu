@@ -313,7 +313,15 @@ int run_decode(DecodeArgs &a, cudaStream_t stream) {
   dim3 grid(a.splits, a.Hkv, a.B);
   cudaEvent_t ev0, ev1;
   tq_timing_events(&ev0, &ev1);
-  if (ev0) cudaEventRecord(ev0, stream);
+  // inside stream capture an event record is only a dependency marker unless
+  // it is recorded as an external event node
+  unsigned ev_flags = cudaEventRecordDefault;
+  if (ev0) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(stream, &cs);
+    if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
+    cudaEventRecordWithFlags(ev0, stream, ev_flags);
+  }
   switch (a.G) {
     case 1: chunk_kernel<D, 1><<<grid, CT, 0, stream>>>(a); break;
     case 2: chunk_kernel<D, 2><<<grid, CT, 0, stream>>>(a); break;
@@ -322,7 +330,7 @@ int run_decode(DecodeArgs &a, cudaStream_t stream) {
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "decode: GQA group size must be 1, 2, 4 or 8");
   }
   if (int e = tq_check_launch("chunk_kernel")) return e;
-  if (ev1) cudaEventRecord(ev1, stream);
+  if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
   combine_kernel<D><<<(heads + QW - 1) / QW, QW * 32, 0, stream>>>(a);
   tq_count_launch(3);
   return tq_check_launch("combine_kernel");

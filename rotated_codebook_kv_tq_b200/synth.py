@@ -50,9 +50,13 @@ def generator(seed: int, stream: int) -> np.random.Generator:
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round to nearest even); returns uint16 bits."""
-    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    rounded = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).reshape(-1)
+    out = np.empty(b.shape, dtype=np.uint16)
+    step = 1 << 24
+    for a in range(0, b.size, step):      # finite inputs: no uint32 overflow
+        c = b[a:a + step]
+        out[a:a + step] = ((c + np.uint32(0x7FFF) + ((c >> 16) & 1)) >> 16).astype(np.uint16)
+    return out.reshape(np.shape(x))
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -175,8 +179,8 @@ def kv_inputs(w: Workload, T: Optional[int] = None):
     sk, sv = channel_scales(w)
     k = _normal_rows(generator(w.seed, STREAM_K), (w.B, w.Hkv, T, w.d))
     v = _normal_rows(generator(w.seed, STREAM_V), (w.B, w.Hkv, T, w.d))
-    k = (k * sk[None, :, None, :].astype(np.float32)).astype(np.float32)
-    v = (v * sv[None, :, None, :].astype(np.float32)).astype(np.float32)
+    k *= sk[None, :, None, :].astype(np.float32)
+    v *= sv[None, :, None, :].astype(np.float32)
     if w.dtype == "bf16":
         return f32_to_bf16_bits(k), f32_to_bf16_bits(v)
     return k, v
@@ -214,3 +218,28 @@ def rope_for(w: Workload, t_max: Optional[int] = None):
     if w.rope_theta is None:
         return None
     return rope_table(w.T if t_max is None else t_max, w.d, w.rope_theta)
+
+
+def kv_inputs_torch(w: Workload, T: Optional[int] = None, device: str = "cuda", seed_salt: int = 0):
+    """Same recipe as ``kv_inputs`` drawn on the device with torch's generator
+    (used where only timing matters, e.g. the benchmark; values differ from the
+    numpy stream).  Returns bf16 (or fp32) tensors [B, Hkv, T, d]."""
+    import torch
+    T = w.T if T is None else T
+    sk, sv = channel_scales(w)
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1000 + seed_salt)
+    out = []
+    for s in (sk, sv):
+        x = torch.randn((w.B, w.Hkv, T, w.d), generator=g, device=device, dtype=torch.float32)
+        x *= torch.as_tensor(s, dtype=torch.float32, device=device)[None, :, None, :]
+        out.append(x.to(torch.bfloat16) if w.dtype == "bf16" else x)
+    return out[0], out[1]
+
+
+def query_inputs_torch(w: Workload, Lq: int = 1, device: str = "cuda", seed_salt: int = 0):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1000 + 500 + seed_salt)
+    q = torch.randn((w.B, w.Hq, Lq, w.d), generator=g, device=device, dtype=torch.float32)
+    return q.to(torch.bfloat16) if w.dtype == "bf16" else q
