@@ -189,6 +189,33 @@ int tq_attention_logits(const tq_codec *codec, const void *q, int dtype, int B, 
                         size_t ws_bytes, float *out, float *logits, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Decode without a workspace, for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages.  Callers that cannot call cudaMalloc (a plugin
+ * inside a host application that owns all device allocations, or a serving
+ * process whose memory is reserved up front) cannot hand tq_attention_decode
+ * a workspace.  This variant runs the same kernels with its scratch taken from
+ * a static device array of TQ_NOALLOC_SCRATCH_BYTES (16 MiB) inside the
+ * library, held by every GPU that loads the library until the process exits.
+ * It calls no cudaMalloc/cudaFree.  Arguments as tq_attention_decode, minus the
+ * workspace.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, that device current) and caches it.
+ *   - Shapes needing more scratch than the limit, i.e.
+ *     B*Hq*(2d + num_splits*(d+2))*4 bytes > 16 MiB, return TQ_ERR_WORKSPACE.
+ *   - All calls share the array (each leaves its contents there; every word is
+ *     written before it is read, so nothing needs clearing).  Calls whose
+ *     kernels overlap on the GPU (other streams, other host threads) race on
+ *     it: the caller must serialise them.
+ * ------------------------------------------------------------------------ */
+#define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+int tq_attention_decode_noalloc(const tq_codec *codec, const void *q, int dtype, int B, int Hq,
+                                int Hkv, const tq_cache *cache, const int32_t *seq_lens,
+                                int max_seq_len, float scale, const float *rope_cos,
+                                const float *rope_sin, int num_splits, float *out,
+                                void *stream);
+
+/* ------------------------------------------------------------------------
  * Dequantize rows [row0, row0 + rows) of every (b, h) ("FibQuant ...",
  * section 2.3 decoder): keys  nu Pi^T (c_k[idx] + sqrt(pi/2)/d rho S^T(2 sigma - 1)),
  * values nu Pi^T c_v[idx].

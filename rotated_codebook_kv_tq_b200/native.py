@@ -23,7 +23,7 @@ TQ_F32, TQ_BF16 = 0, 1
 EXPORTS = [
     "tq_build_codebook", "tq_codec_create", "tq_codec_destroy", "tq_codec_codebooks",
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
-    "tq_attention_logits", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
+    "tq_attention_logits", "tq_attention_decode_noalloc", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
     "tq_last_error",
 ]
 
@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.tq_attention_decode.argtypes = [vp, vp, i32, i32, i32, i32, ctypes.POINTER(CacheDesc),
                                           vp, i32, f32, vp, vp, i32, vp, sz, vp, vp]
         L.tq_attention_logits.argtypes = L.tq_attention_decode.argtypes[:-1] + [vp, vp]
+        L.tq_attention_decode_noalloc.argtypes = [vp, vp, i32, i32, i32, i32,
+                                                  ctypes.POINTER(CacheDesc), vp, i32, f32, vp,
+                                                  vp, i32, vp, vp]
         L.tq_dequantize.argtypes = [vp, ctypes.POINTER(CacheDesc), i32, i64, i64, vp, vp]
         L.tq_set_timing_events.argtypes = [vp, vp]
         L.tq_launch_count.argtypes = []
@@ -238,6 +241,22 @@ def attention_logits(codec: Codec, q, cache: Cache, max_seq_len: int, scale: flo
                                     float(scale), _ptr(rc), _ptr(rs), num_splits,
                                     workspace.data_ptr(), ws_bytes, out.data_ptr(),
                                     logits.data_ptr(), _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def attention_decode_noalloc(codec: Codec, q, cache: Cache, max_seq_len: int, scale: float, out,
+                             seq_lens=None, rope=None, num_splits: int = 0, stream=None) -> None:
+    """tq_attention_decode_noalloc: decode with the library's static scratch
+    (for callers that cannot allocate a workspace)."""
+    B, Hq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    check(lib().tq_attention_decode_noalloc(codec.handle, q.data_ptr(), _dtype_code(q), B, Hq,
+                                            cache.Hkv, ctypes.byref(desc), _ptr(seq_lens),
+                                            max_seq_len, float(scale), _ptr(rc), _ptr(rs),
+                                            num_splits, out.data_ptr(), _stream(stream)))
 
 
 def dequantize(codec: Codec, cache: Cache, which: int, row0: int, rows: int, out,
