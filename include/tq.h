@@ -165,7 +165,7 @@ int tq_quantize_kv(const tq_codec *codec, const void *k, const void *v, int dtyp
  * seq_lens device int32 [B], nullable (then every batch has max_seq_len);
  *          entries are clamped to 1..max_seq_len; max_seq_len <= rows_cap.
  * rope_cos/rope_sin  as for tq_quantize_kv (nullable together).
- * num_splits  chunks per (b, KV head); 0 picks a default.
+ * num_splits  chunks per (b, KV head), at most 512; 0 picks the default 64.
  * workspace   device, >= tq_attention_workspace(...) bytes, 16-byte aligned;
  *             scratch owned by the caller, contents need no initialisation.
  * out      device fp32 [B][Hq][d].

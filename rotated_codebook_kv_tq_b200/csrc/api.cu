@@ -115,13 +115,22 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   c->books.qjl = c->qjl_k;
   c->books.bits_v = c->bits_v;
 
+  c->ST_dev = nullptr;
   if (c->qjl_k) {
-    const size_t bytes = sizeof(uint16_t) * c->d * c->d;
-    if (cudaMalloc(&c->S_dev, bytes) != cudaSuccess) {
+    const size_t n = static_cast<size_t>(c->d) * c->d;
+    std::vector<uint16_t> both(2 * n);
+    for (int i = 0; i < c->d; ++i)
+      for (int j = 0; j < c->d; ++j) {
+        both[static_cast<size_t>(i) * c->d + j] = desc->qjl_bf16[static_cast<size_t>(i) * c->d + j];
+        both[n + static_cast<size_t>(j) * c->d + i] = desc->qjl_bf16[static_cast<size_t>(i) * c->d + j];
+      }
+    if (cudaMalloc(&c->S_dev, 2 * n * sizeof(uint16_t)) != cudaSuccess) {
       delete c;
       return tq_check_launch("codec: cudaMalloc");
     }
-    if (cudaMemcpy(c->S_dev, desc->qjl_bf16, bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+    c->ST_dev = c->S_dev + n;
+    if (cudaMemcpy(c->S_dev, both.data(), 2 * n * sizeof(uint16_t), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
       cudaFree(c->S_dev);
       delete c;
       return tq_check_launch("codec: cudaMemcpy");
@@ -205,6 +214,7 @@ int decode_common(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   if ((rope_cos == nullptr) != (rope_sin == nullptr))
     return tq_fail(TQ_ERR_INVALID_ARG, "decode: rope_cos and rope_sin go together");
   const int splits = num_splits > 0 ? num_splits : 64;
+  if (splits > 512) return tq_fail(TQ_ERR_INVALID_ARG, "decode: num_splits must be <= 512");
   if (decode_workspace_bytes(c, B, Hq, splits) > ws_bytes)
     return tq_fail(TQ_ERR_WORKSPACE, "decode: workspace smaller than tq_attention_workspace()");
   if (!aligned(workspace, 16)) return tq_fail(TQ_ERR_ALIGNMENT, "decode: workspace alignment");

@@ -21,7 +21,6 @@
 namespace {
 
 constexpr int CT = 256;       // threads of the chunk kernel
-constexpr int QW = 8;         // warps per block in qprep / combine
 
 struct DecodeArgs {
   const void *q;
@@ -41,6 +40,7 @@ struct DecodeArgs {
   int splits;
   int chunk;          // rows per chunk (multiple of 32)
   const uint16_t *S;
+  const uint16_t *ST;  // S transposed
   float *q1;          // [B][Hq][D]
   float *q2;          // [B][Hq][D]
   float *po;          // [B][Hq][splits][D]
@@ -54,50 +54,52 @@ __device__ __forceinline__ int seq_len_of(const DecodeArgs &a, int b) {
   return a.seq_lens ? min(max(a.seq_lens[b], 1), a.max_len) : a.max_len;
 }
 
+// One block of D threads per query head.  Warp 0 applies RoPE and the
+// rotation (4 or 2 coordinates per lane); then thread i forms
+// q''_i = sum_j S[i][j] q'_j from the transposed copy of S (coalesced loads).
 template <int D>
-__global__ void __launch_bounds__(QW * 32) qprep_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(D) qprep_kernel(DecodeArgs a) {
   constexpr int NPL = D / 32;
-  __shared__ float qs[QW][D];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int head = blockIdx.x * QW + warp;
-  if (head >= a.B * a.Hq) return;
+  __shared__ float qs[D];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int head = blockIdx.x;
   const int b = head / a.Hq;
   const int64_t pos = seq_len_of(a, b) - 1;
-  float x[NPL];
-#pragma unroll
-  for (int k = 0; k < NPL; ++k)
-    x[k] = tq_load_elem(a.q, static_cast<int64_t>(head) * D + lane + 32 * k, a.dtype);
-  if (a.rc != nullptr) {
-    constexpr int HALF = NPL / 2;
-#pragma unroll
-    for (int k = 0; k < HALF; ++k) {
-      const float c = a.rc[pos * (D / 2) + lane + 32 * k];
-      const float s = a.rs[pos * (D / 2) + lane + 32 * k];
-      const float u = x[k], v = x[k + HALF];
-      x[k] = u * c - v * s;
-      x[k + HALF] = v * c + u * s;
-    }
-  }
-  tq_apply_signs<NPL>(x, a.books.dneg, lane);
-  tq_warp_wht<NPL>(x, lane);
-  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
-#pragma unroll
-  for (int k = 0; k < NPL; ++k) {
-    x[k] *= inv_sqrt_d;
-    a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
-    qs[warp][lane + 32 * k] = x[k];
-  }
-  __syncwarp();
-  if (!a.books.qjl) return;
-  // q'' = S q': row i of S read coalesced by the warp, reduced by shuffles
-  for (int i = 0; i < D; ++i) {
-    float acc = 0.f;
+  if (tid < 32) {
+    float x[NPL];
 #pragma unroll
     for (int k = 0; k < NPL; ++k)
-      acc = fmaf(tq_bf16_to_f32(a.S[i * D + lane + 32 * k]), qs[warp][lane + 32 * k], acc);
-    acc = tq_warp_sum(acc);
-    if (lane == 0) a.q2[static_cast<int64_t>(head) * D + i] = acc;
+      x[k] = tq_load_elem(a.q, static_cast<int64_t>(head) * D + lane + 32 * k, a.dtype);
+    if (a.rc != nullptr) {
+      constexpr int HALF = NPL / 2;
+#pragma unroll
+      for (int k = 0; k < HALF; ++k) {
+        const float c = a.rc[pos * (D / 2) + lane + 32 * k];
+        const float s = a.rs[pos * (D / 2) + lane + 32 * k];
+        const float u = x[k], v = x[k + HALF];
+        x[k] = u * c - v * s;
+        x[k + HALF] = v * c + u * s;
+      }
+    }
+    tq_apply_signs<NPL>(x, a.books.dneg, lane);
+    tq_warp_wht<NPL>(x, lane);
+    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      x[k] *= inv_sqrt_d;
+      a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
+      qs[lane + 32 * k] = x[k];
+    }
   }
+  __syncthreads();
+  if (!a.books.qjl) return;
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < D; j += 2) {
+    acc0 = fmaf(tq_bf16_to_f32(a.ST[j * D + tid]), qs[j], acc0);
+    acc1 = fmaf(tq_bf16_to_f32(a.ST[(j + 1) * D + tid]), qs[j + 1], acc1);
+  }
+  a.q2[static_cast<int64_t>(head) * D + tid] = acc0 + acc1;
 }
 
 template <int D, int G>
@@ -277,38 +279,67 @@ __global__ void __launch_bounds__(CT) chunk_kernel(DecodeArgs a) {
   }
 }
 
+// One block of D threads per query head: log-sum-exp weights of the chunks,
+// thread i sums coordinate i over the chunks, then warp 0 applies
+// Pi^T = D H / sqrt(d) and the 1/l normalisation.
 template <int D>
-__global__ void __launch_bounds__(QW * 32) combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
   constexpr int NPL = D / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int head = blockIdx.x * QW + warp;
-  if (head >= a.B * a.Hq) return;
+  constexpr int MAXS = 512;
+  __shared__ float fs[MAXS];
+  __shared__ float red[D / 32][2];
+  __shared__ float os[D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t head = blockIdx.x;
+  const int S = a.splits;
   float m = -CUDART_INF_F;
-  for (int s = lane; s < a.splits; s += 32) m = fmaxf(m, a.pml[(static_cast<int64_t>(head) * a.splits + s) * 2]);
+  for (int s = tid; s < S; s += D) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
-  float x[NPL], l = 0.f;
+  if (lane == 0) red[warp][0] = m;
+  __syncthreads();
+  float M = red[0][0];
 #pragma unroll
-  for (int k = 0; k < NPL; ++k) x[k] = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const int64_t base = static_cast<int64_t>(head) * a.splits + s;
-    const float ms = a.pml[base * 2], ls = a.pml[base * 2 + 1];
-    if (ls == 0.f) continue;
-    const float f = __expf(ms - m);
-    l += ls * f;
-#pragma unroll
-    for (int k = 0; k < NPL; ++k) x[k] = fmaf(a.po[base * D + lane + 32 * k], f, x[k]);
+  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w][0]);
+  float l = 0.f;
+  for (int s = tid; s < S; s += D) {
+    const float ls = a.pml[(head * S + s) * 2 + 1];
+    const float f = ls > 0.f ? __expf(a.pml[(head * S + s) * 2] - M) : 0.f;
+    fs[s] = f;
+    l += f * ls;
   }
-  tq_warp_wht<NPL>(x, lane);
-  tq_apply_signs<NPL>(x, a.books.dneg, lane);
-  const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * l);
+  l = tq_warp_sum(l);
+  __syncthreads();
+  if (lane == 0) red[warp][1] = l;
+  __syncthreads();
+  float L = 0.f;
 #pragma unroll
-  for (int k = 0; k < NPL; ++k) a.out[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k] * norm;
+  for (int w = 0; w < D / 32; ++w) L += red[w][1];
+  float o0 = 0.f, o1 = 0.f;
+  const float *po = a.po + head * S * D + tid;
+  int s = 0;
+  for (; s + 1 < S; s += 2) {
+    o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
+    o1 = fmaf(po[static_cast<int64_t>(s + 1) * D], fs[s + 1], o1);
+  }
+  if (s < S) o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
+  os[tid] = o0 + o1;
+  __syncthreads();
+  if (warp == 0) {
+    float x[NPL];
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) x[k] = os[lane + 32 * k];
+    tq_warp_wht<NPL>(x, lane);
+    tq_apply_signs<NPL>(x, a.books.dneg, lane);
+    const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * L);
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) a.out[head * D + lane + 32 * k] = x[k] * norm;
+  }
 }
 
 template <int D>
 int run_decode(DecodeArgs &a, cudaStream_t stream) {
   const int heads = a.B * a.Hq;
-  qprep_kernel<D><<<(heads + QW - 1) / QW, QW * 32, 0, stream>>>(a);
+  qprep_kernel<D><<<heads, D, 0, stream>>>(a);
   if (int e = tq_check_launch("qprep_kernel")) return e;
   dim3 grid(a.splits, a.Hkv, a.B);
   cudaEvent_t ev0, ev1;
@@ -331,7 +362,7 @@ int run_decode(DecodeArgs &a, cudaStream_t stream) {
   }
   if (int e = tq_check_launch("chunk_kernel")) return e;
   if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
-  combine_kernel<D><<<(heads + QW - 1) / QW, QW * 32, 0, stream>>>(a);
+  combine_kernel<D><<<heads, D, 0, stream>>>(a);
   tq_count_launch(3);
   return tq_check_launch("combine_kernel");
 }
@@ -369,6 +400,7 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   const int per = (max_len + splits - 1) / splits;
   a.chunk = (per + 31) / 32 * 32;
   a.S = c->S_dev;
+  a.ST = c->ST_dev;
   const size_t heads = static_cast<size_t>(B) * Hq;
   float *f = static_cast<float *>(ws);
   a.q1 = f;

@@ -35,6 +35,7 @@ struct tq_codec {
   int bits_k, qjl_k, bits_v, mse_bits_k;
   TqBooks books;
   uint16_t *S_dev;     // bf16 [d][d] row-major S[i][j]
+  uint16_t *ST_dev;    // bf16 [d][d] transpose, ST[j][i] = S[i][j] (same allocation)
   int device;
 };
 
