@@ -116,8 +116,7 @@ int tq_codec_codebooks(const tq_codec *codec, float *ck, float *tk, float *cv, f
  *          bit (t % 32) of word [t/32][p][i] is bit p of coordinate i's code
  *          of token t.
  *   vnorm  fp16   [B][Hkv][rows_cap]  nu per value.
- * rows_cap must be a multiple of 32; kcode, vcode, kscale need 16-byte
- * alignment, vnorm 4-byte.  Bytes per (token, head): d/8*planes_k + 4 for
+ * rows_cap must be a multiple of 32; every plane needs 16-byte alignment.  Bytes per (token, head): d/8*planes_k + 4 for
  * keys, d/8*bits_v + 2 for values.
  * ------------------------------------------------------------------------ */
 typedef struct {

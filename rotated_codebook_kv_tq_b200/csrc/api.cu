@@ -17,14 +17,38 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
+// a_t = 2^-b sum_idx c[idx] prod_{p in S_t} (2 bit_p(idx) - 1) for the odd
+// subsets S_t of the b code bits, in increasing bit-mask order.
+void walsh_coefficients(const float *c, int bits, float *out, float *absmax, float *sum) {
+  int t = 0;
+  double amax = 0.0, total = 0.0;
+  for (int m = 1; m < (1 << bits) && t < 8; ++m) {
+    if (!(__builtin_popcount(m) & 1)) continue;
+    double acc = 0.0;
+    for (int idx = 0; idx < (1 << bits); ++idx) {
+      double sgn = 1.0;
+      for (int p = 0; p < bits; ++p)
+        if ((m >> p) & 1) sgn *= ((idx >> p) & 1) ? 1.0 : -1.0;
+      acc += static_cast<double>(c[idx]) * sgn;
+    }
+    acc /= static_cast<double>(1 << bits);
+    out[t++] = static_cast<float>(acc);
+    amax = std::fmax(amax, std::fabs(acc));
+    total += acc;
+  }
+  for (; t < 8; ++t) out[t] = 0.f;
+  if (absmax) *absmax = static_cast<float>(amax);
+  if (sum) *sum = static_cast<float>(total);
+}
+
 int check_cache(const tq_codec *c, const tq_cache *cache) {
   if (!cache || !cache->kcode || !cache->kscale || !cache->vcode || !cache->vnorm)
     return tq_fail(TQ_ERR_INVALID_ARG, "cache: every plane pointer is required");
   if (cache->B <= 0 || cache->Hkv <= 0 || cache->rows_cap <= 0 || cache->rows_cap % 32)
     return tq_fail(TQ_ERR_INVALID_ARG, "cache: B, Hkv > 0 and rows_cap a positive multiple of 32");
   if (!aligned(cache->kcode, 16) || !aligned(cache->vcode, 16) || !aligned(cache->kscale, 16) ||
-      !aligned(cache->vnorm, 4))
-    return tq_fail(TQ_ERR_ALIGNMENT, "cache: kcode/vcode/kscale need 16-byte, vnorm 4-byte alignment");
+      !aligned(cache->vnorm, 16))
+    return tq_fail(TQ_ERR_ALIGNMENT, "cache: every plane needs 16-byte alignment");
   (void)c;
   return TQ_OK;
 }
@@ -113,6 +137,8 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
     if (desc->rotation_signs[i] < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
   c->books.mse_bits_k = mse_k;
   c->books.qjl = c->qjl_k;
+  walsh_coefficients(c->books.ck, mse_k, c->walsh_k, &c->walsh_k_absmax, nullptr);
+  walsh_coefficients(c->books.cv, c->bits_v, c->walsh_v, nullptr, &c->walsh_v_sum);
   c->books.bits_v = c->bits_v;
 
   c->ST_dev = nullptr;

@@ -16,7 +16,10 @@
 //           out = Pi^T o / l = D (H o) / (sqrt(d) l).
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "tq_device.cuh"
+#include "tq_tc.h"
 
 namespace {
 
@@ -369,9 +372,23 @@ int run_decode(DecodeArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits) {
+namespace {
+size_t ws_core_bytes(const tq_codec *c, int B, int Hq, int splits) {
   const size_t heads = static_cast<size_t>(B) * Hq;
-  return sizeof(float) * heads * (2 * c->d + static_cast<size_t>(splits) * (c->d + 2));
+  const size_t f = sizeof(float) * heads * (2 * c->d + static_cast<size_t>(splits) * (c->d + 2));
+  return (f + 127) / 128 * 128;
+}
+// Upper bound of the tensor-core path's per-group B-operand region, per
+// query head (covers every group size it supports).
+size_t ws_bk_bytes(const tq_codec *c, int B, int Hq) {
+  if (c->d != 128) return 0;
+  const size_t ktot = static_cast<size_t>((1 << (c->mse_bits_k - 1)) + c->qjl_k) * 128;
+  return static_cast<size_t>(B) * Hq * (8 * ktot + 144);
+}
+}  // namespace
+
+size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits) {
+  return ws_core_bytes(c, B, Hq, splits) + ws_bk_bytes(c, B, Hq);
 }
 
 int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
@@ -410,6 +427,19 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   a.out = out;
   a.logits = logits;
   a.books = c->books;
+  // TQ_DECODE_IMPL=simt selects the CUDA-core kernels (a complete second
+  // implementation, used to cross-check the tensor-core path)
+  const char *impl = getenv("TQ_DECODE_IMPL");
+  const bool want_tc = !(impl && impl[0] == 's');
+  if (want_tc && tc_supported(c, a.G)) {
+    uint8_t *bk = static_cast<uint8_t *>(ws) + ws_core_bytes(c, B, Hq, splits);
+    if (int e = launch_decode_tc(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_len, scale, rc,
+                                 rs, splits, a.po, a.pml, bk, logits, stream))
+      return e;
+    combine_kernel<128><<<B * Hq, 128, 0, stream>>>(a);
+    tq_count_launch(1);
+    return tq_check_launch("combine_kernel");
+  }
   switch (c->d) {
     case 64: return run_decode<64>(a, stream);
     case 128: return run_decode<128>(a, stream);

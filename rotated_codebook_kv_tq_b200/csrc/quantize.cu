@@ -14,7 +14,10 @@
 // __ballot_sync over the warp produces each 32-coordinate key-plane word
 // directly.  Value codes are accumulated per coordinate across the group's
 // 32 tokens and stored as column-group words.
+#include <cstdlib>
+
 #include "tq_device.cuh"
+#include "tq_sm100.cuh"
 
 namespace {
 
@@ -37,6 +40,8 @@ struct QuantArgs {
   int64_t row0;
   uint32_t *status;
   const uint16_t *S;
+  const uint16_t *ST;  // S transposed (bf16)
+  int stage_s;         // 1: stage S^T in shared memory (large calls)
   int64_t g_first;   // first 32-token group touched
   int64_t n_groups;  // groups touched per (b, h)
   TqBooks books;
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
     tks[threadIdx.x] = a.books.tk[threadIdx.x];
     tvs[threadIdx.x] = a.books.tv[threadIdx.x];
   }
-  if (a.books.qjl) {
+  if (a.books.qjl && a.stage_s) {
     for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
       const int i = e / D, j = e % D;
       ST[j * D + i] = tq_bf16_to_f32(a.S[e]);
@@ -162,10 +167,19 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
         float z[NPL];
 #pragma unroll
         for (int k = 0; k < NPL; ++k) z[k] = 0.f;
-        for (int j = 0; j < D; ++j) {
-          const float rj = rbuf[warp][j];
+        if (a.stage_s) {
+          for (int j = 0; j < D; ++j) {
+            const float rj = rbuf[warp][j];
 #pragma unroll
-          for (int k = 0; k < NPL; ++k) z[k] = fmaf(ST[j * D + lane + 32 * k], rj, z[k]);
+            for (int k = 0; k < NPL; ++k) z[k] = fmaf(ST[j * D + lane + 32 * k], rj, z[k]);
+          }
+        } else {
+          for (int j = 0; j < D; ++j) {
+            const float rj = rbuf[warp][j];
+#pragma unroll
+            for (int k = 0; k < NPL; ++k)
+              z[k] = fmaf(tq_bf16_to_f32(a.ST[j * D + lane + 32 * k]), rj, z[k]);
+          }
         }
         __syncwarp();
         const int p = a.books.mse_bits_k;
@@ -219,9 +233,238 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// tcgen05 variant for large calls: the QJL sketch z = S r of a 128-row tile
+// is one tensor-core contraction.  Each warp runs the fused per-row pipeline
+// above for one 32-token group and writes its residuals, split into bf16
+// hi + lo (r = hi + lo + O(2^-18 |r|)), into the shared A tile; one thread
+// issues 2d/16 kind::f16 MMAs against S (exactly representable: S is stored
+// as bf16) with fp32 accumulation in tensor memory; thread t then reads row
+// t of z and writes that key's sign plane.
+// Shared layouts (K-major, no swizzle): A byte (m, kb) at
+// (kb/16)*2048 + (m/8)*128 + (m%8)*16 + kb%16 for K = 2d elements (hi | lo);
+// B = S, byte (i, kb) at (kb/16)*(16d) + (i/8)*128 + (i%8)*16 + kb%16.
+template <int D>
+__global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
+  constexpr int NPL = D / 32;
+  constexpr int KE = 2 * D;                       // K elements (hi | lo)
+  constexpr uint32_t A_BYTES = 128u * KE * 2u;
+  constexpr uint32_t IDESC = sm100::idesc_bf16(128, D);
+  extern __shared__ __align__(128) float smem_tc[];
+  uint8_t *As = reinterpret_cast<uint8_t *>(smem_tc);
+  uint8_t *Bs = As + A_BYTES;
+  __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
+  __shared__ __align__(8) uint64_t mb;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nlk = 1 << a.books.mse_bits_k, nlv = 1 << a.books.bits_v;
+  if (tid < TQ_MAX_LEVELS) {
+    cks[tid] = a.books.ck[tid];
+    tks[tid] = a.books.tk[tid];
+    tvs[tid] = a.books.tv[tid];
+  }
+  for (int e = tid; e < D * D; e += 128) {
+    const int i = e / D, kb = 2 * (e % D);
+    *reinterpret_cast<uint16_t *>(Bs + (kb >> 4) * (D * 16) + (i >> 3) * 128 + (i & 7) * 16 +
+                                  (kb & 15)) = a.S[e];
+  }
+  if (warp == 0) sm100::tmem_alloc(&tmem_s, D);
+  if (tid == 0) {
+    sm100::mbar_init(&mb, 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  sm100::fence_async_smem();
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  const uint32_t tm = tmem_s;
+  const uint32_t a_addr = sm100::smem_addr(As), b_addr = sm100::smem_addr(Bs);
+  const int planes_k = a.books.mse_bits_k + 1;
+  const int64_t items = static_cast<int64_t>(a.B) * a.H * a.n_groups;
+  const int64_t tiles = (items + 3) / 4;
+  uint32_t phase = 0;
+
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int64_t it = tile * 4 + warp;
+    const bool have = it < items;
+    int64_t g = 0, cache_bh = 0, r_begin = 0, r_end = 0;
+    int b = 0, h = 0;
+    if (have) {
+      g = a.g_first + it % a.n_groups;
+      const int64_t bh = it / a.n_groups;
+      b = static_cast<int>(bh / a.H);
+      h = static_cast<int>(bh % a.H);
+      r_begin = max(a.row0, g * 32);
+      r_end = min(a.row0 + a.T, g * 32 + 32);
+      cache_bh = static_cast<int64_t>(b) * a.H + h;
+    }
+    uint32_t vw[4][NPL];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) vw[p][k] = 0u;
+    for (int64_t r = r_begin; r < r_end; ++r) {
+      const int64_t t = r - a.row0;
+      const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
+      float x[NPL];
+      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+      bool bad;
+      const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      int idx[NPL];
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks, nlk - 1);
+      uint32_t myword = 0u;
+      for (int p = 0; p < a.books.mse_bits_k; ++p) {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          const uint32_t w = __ballot_sync(TQ_FULL, (idx[k] >> p) & 1);
+          if (lane == p * NPL + k) myword = w;
+        }
+      }
+      const int m = warp * 32 + static_cast<int>(r & 31);
+      float r2 = 0.f;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const float rr = x[k] - cks[idx[k]];
+        r2 += rr * rr;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(rr);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(rr - __bfloat162float(hi));
+        const int j = lane + 32 * k;
+        const int kb_hi = 2 * j, kb_lo = 2 * (D + j);
+        const int row_off = (m >> 3) * 128 + (m & 7) * 16;
+        *reinterpret_cast<__nv_bfloat16 *>(As + (kb_hi >> 4) * 2048 + row_off + (kb_hi & 15)) = hi;
+        *reinterpret_cast<__nv_bfloat16 *>(As + (kb_lo >> 4) * 2048 + row_off + (kb_lo & 15)) = lo;
+      }
+      const float rho = sqrtf(tq_warp_sum(r2));
+      uint32_t *krow = reinterpret_cast<uint32_t *>(
+          a.kcode + (cache_bh * a.rows_cap + r) * planes_k * (D / 8));
+      if (lane < a.books.mse_bits_k * NPL) krow[lane] = myword;
+      if (lane == 0) {
+        const uint32_t pair = static_cast<uint32_t>(tq_f32_to_half(nu)) |
+                              (static_cast<uint32_t>(tq_f32_to_half(rho)) << 16);
+        reinterpret_cast<uint32_t *>(a.kscale)[cache_bh * a.rows_cap + r] = pair;
+        if (bad && a.status) atomicAdd(a.status, 1u);
+      }
+      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+      const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      const uint32_t bit = 1u << (r & 31);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const int iv = tq_code(x[k], tvs, nlv - 1);
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if ((iv >> p) & 1) vw[p][k] |= bit;
+      }
+      if (lane == 0) {
+        a.vnorm[cache_bh * a.rows_cap + r] = tq_f32_to_half(nv);
+        if (bad && a.status) atomicAdd(a.status, 1u);
+      }
+    }
+    if (have) {
+      const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
+      const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
+      uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (p >= a.books.bits_v) break;
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          uint32_t *w = vg + p * D + lane + 32 * k;
+          if (mask == TQ_FULL) {
+            *w = vw[p][k];
+          } else {
+            atomicAnd(w, ~mask);
+            atomicOr(w, vw[p][k] & mask);
+          }
+        }
+      }
+    }
+    // ---- the sketch of the whole tile on the tensor cores
+    sm100::fence_async_smem();
+    sm100::fence_before_sync();
+    __syncthreads();
+    sm100::fence_after_sync();
+    if (tid == 0) {
+#pragma unroll
+      for (int s = 0; s < KE / 16; ++s) {
+        const int kk = (16 * s) % D;
+        sm100::mma_bf16_ss(tm, sm100::smem_desc(a_addr + s * 2 * 2048, 2048, 128),
+                           sm100::smem_desc(b_addr + (kk / 8) * (D * 16), D * 16, 128), IDESC,
+                           s > 0);
+      }
+      sm100::mma_commit(&mb);
+    }
+    if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
+    phase ^= 1;
+    __syncthreads();
+    if (abort_s) break;
+    sm100::fence_after_sync();
+    const int64_t myr = g * 32 + lane;
+    const bool row_ok = have && myr >= r_begin && myr < r_end;
+    uint32_t sw[NPL];
+#pragma unroll
+    for (int wd = 0; wd < NPL; ++wd) {
+      uint32_t z0[16], z1[16];
+      sm100::tmem_ld16(sm100::tmem_lane(tm + 32 * wd, warp), z0);
+      sm100::tmem_ld16(sm100::tmem_lane(tm + 32 * wd + 16, warp), z1);
+      sm100::wait_ld();
+      uint32_t word = 0u;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        word |= (__uint_as_float(z0[c]) >= 0.f ? 1u : 0u) << c;
+        word |= (__uint_as_float(z1[c]) >= 0.f ? 1u : 0u) << (16 + c);
+      }
+      sw[wd] = word;
+    }
+    if (row_ok) {
+      uint32_t *srow = reinterpret_cast<uint32_t *>(
+          a.kcode + (cache_bh * a.rows_cap + myr) * planes_k * (D / 8) + a.books.mse_bits_k * (D / 8));
+#pragma unroll
+      for (int wd = 0; wd < NPL; ++wd) srow[wd] = sw[wd];
+    }
+    sm100::fence_before_sync();
+    __syncthreads();
+    sm100::fence_after_sync();
+  }
+  if (abort_s) {
+    sm100::mbar_wait(&mb, phase, 1u << 20);
+    if (tid == 0 && a.status) atomicAdd(a.status, 1u << 31);
+  }
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  if (warp == 0) sm100::tmem_dealloc(tm, D);
+}
+
+template <int D>
+int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
+  constexpr size_t shm = 128u * 2 * D * 2 + static_cast<size_t>(D) * D * 2;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool done[64] = {};
+  if (dev < 64 && !done[dev]) {
+    if (cudaFuncSetAttribute(quantize_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(shm)) != cudaSuccess)
+      return tq_check_launch("cudaFuncSetAttribute(quantize_tc)");
+    done[dev] = true;
+  }
+  const int64_t items = static_cast<int64_t>(a.B) * a.H * a.n_groups;
+  const int64_t tiles = (items + 3) / 4;
+  const int64_t cap = static_cast<int64_t>(sms) * (D == 128 ? 2 : 4);
+  const int grid = static_cast<int>(tiles < cap ? tiles : cap);
+  quantize_tc_kernel<D><<<grid, 128, shm, stream>>>(a);
+  tq_count_launch(1);
+  return tq_check_launch("quantize_tc_kernel");
+}
+
 template <int D>
 int run_quantize(const QuantArgs &a, cudaStream_t stream) {
-  const size_t shm = a.books.qjl ? sizeof(float) * D * D : 0;
+  const size_t shm = a.books.qjl && a.stage_s ? sizeof(float) * D * D : 0;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(quantize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -267,13 +510,20 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   a.row0 = row0;
   a.status = status;
   a.S = c->S_dev;
+  a.ST = c->ST_dev;
   a.g_first = row0 / 32;
   a.n_groups = (row0 + T - 1) / 32 - row0 / 32 + 1;
   a.books = c->books;
   if (T == 0) return TQ_OK;
+  const int64_t items = static_cast<int64_t>(B) * H * a.n_groups;
+  a.stage_s = items > 64 ? 1 : 0;
+  // TQ_QUANT_IMPL=simt keeps the CUDA-core sketch (a complete second
+  // implementation, used to cross-check the tensor-core one)
+  const char *impl = getenv("TQ_QUANT_IMPL");
+  const bool tc = c->qjl_k && items >= 256 && !(impl && impl[0] == 's');
   switch (c->d) {
-    case 64: return run_quantize<64>(a, stream);
-    case 128: return run_quantize<128>(a, stream);
+    case 64: return tc ? run_quantize_tc<64>(a, stream) : run_quantize<64>(a, stream);
+    case 128: return tc ? run_quantize_tc<128>(a, stream) : run_quantize<128>(a, stream);
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "quantize: head dim not built");
   }
 }

@@ -1,0 +1,50 @@
+// Arguments and sizes of the tensor-core decode path (decode_tc.cu).
+#pragma once
+
+#include <stdint.h>
+
+#include "tq_internal.h"
+
+// MMA N: 4 limbs per query head, at least 8.
+__host__ __device__ constexpr int tc_n(int G) { return 4 * G < 8 ? 8 : 4 * G; }
+
+struct TcArgs {
+  const void *q;
+  int dtype;
+  int B, Hq, Hkv;
+  const uint8_t *kcode;
+  const uint16_t *kscale;
+  const uint32_t *vcode;
+  const uint16_t *vnorm;
+  int64_t rows_cap;
+  const int32_t *seq_lens;
+  int max_len;
+  float scale;
+  float qjl_coef;
+  const float *rc;
+  const float *rs;
+  const uint16_t *ST;   // S transposed (bf16)
+  int splits;
+  int chunk;            // rows per split (multiple of 128)
+  int sub;              // rows per shared-memory unit (multiple of 128, <= chunk)
+  uint8_t *bk;          // per (b, KV head): B operand bytes then 4 floats per head
+  int bk_stride;        // bytes between groups (multiple of 128)
+  float *po;            // [B][Hq][splits][128]
+  float *pml;           // [B][Hq][splits][2]
+  float *logits;        // optional [B][Hq][max_len]
+  float wk[8];          // key Walsh coefficients a_S
+  float wk_absmax;
+  float wv[8];          // value Walsh coefficients
+  float wv_sum;
+  uint32_t *err;        // optional device flag set when a bounded wait times out
+  TqBooks books;
+};
+
+// Whether the tensor-core path has a kernel for this codec / group size.
+bool tc_supported(const tq_codec *c, int G);
+// Bytes of the per-group B-operand region (one group).
+int tc_bk_stride(const tq_codec *c, int G);
+int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                     const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
+                     const float *rc, const float *rs, int splits, float *po, float *pml,
+                     uint8_t *bk, float *logits, cudaStream_t stream);

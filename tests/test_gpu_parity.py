@@ -34,6 +34,9 @@ QUANT_CASES = {
     "llama_appends": (synth.WORKLOADS["llama_decode"].scaled(T=138), [(0, 100), (100, 1), (101, 37)]),
     "esm_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=3, Hkv=3, T=100), [(0, 100)]),
     "long_2bit": (synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=300), [(0, 300)]),
+    # >= 256 groups of 32 tokens: large calls take the tcgen05 sketch kernel
+    "llama_tc_sketch": (synth.WORKLOADS["llama_decode"].scaled(T=1100), [(0, 1037), (1037, 63)]),
+    "esm_tc_sketch_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=100), [(0, 100)]),
 }
 
 
@@ -63,8 +66,15 @@ def _quantize_both(w, segments, rows_cap=None):
     return ocodec, ncodec, ocache, ncache, encs, int(status.item())
 
 
+@pytest.mark.parametrize("impl", ["default", "simt"])
 @pytest.mark.parametrize("case", list(QUANT_CASES))
-def test_quantize_parity(case):
+def test_quantize_parity(case, impl, monkeypatch):
+    # "default": tensor-core sketch for calls of >= 256 token groups with QJL;
+    # "simt": the CUDA-core sketch everywhere
+    if impl == "simt":
+        monkeypatch.setenv("TQ_QUANT_IMPL", "simt")
+    else:
+        monkeypatch.delenv("TQ_QUANT_IMPL", raising=False)
     w, segments = QUANT_CASES[case]
     ocodec, ncodec, ocache, ncache, encs, bad = _quantize_both(w, segments)
     gpu = tl.download_cache(ncache)
@@ -142,6 +152,8 @@ DECODE_CASES = {
     "esm_mha_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=3, Hkv=3, T=300, Lq=1), None, 4),
     "ragged_lens": (synth.WORKLOADS["llama_decode"].scaled(B=3, Hq=8, Hkv=2, T=300), [1, 77, 300], 5),
     "gqa8": (synth.WORKLOADS["long_decode"].scaled(B=1, Hq=16, Hkv=2, T=500), None, 3),
+    "gqa2_multi_sub": (synth.WORKLOADS["llama_decode"].scaled(B=1, Hq=4, Hkv=2, T=2500), None, 1),
+    "tiny_two_chunks": (synth.WORKLOADS["tiny"].scaled(T=1000), None, 2),
 }
 
 
@@ -169,8 +181,16 @@ def _decode_case(w, lens, splits):
     return ref, ref_logits, out.cpu().numpy().astype(np.float64), logits.cpu().numpy(), lens
 
 
+@pytest.mark.parametrize("impl", ["default", "simt"])
 @pytest.mark.parametrize("case", list(DECODE_CASES))
-def test_decode_parity(case):
+def test_decode_parity(case, impl, monkeypatch):
+    # "default" takes the tensor-core kernels where they are built (d=128,
+    # group size 1/2/4, the bit widths of the workloads) and the CUDA-core
+    # kernels elsewhere; "simt" forces the CUDA-core kernels everywhere.
+    if impl == "simt":
+        monkeypatch.setenv("TQ_DECODE_IMPL", "simt")
+    else:
+        monkeypatch.delenv("TQ_DECODE_IMPL", raising=False)
     w, lens, splits = DECODE_CASES[case]
     ref, ref_logits, got, got_logits, lens = _decode_case(w, lens, splits)
     vscale = tl.channel_scale_of_values(w)
