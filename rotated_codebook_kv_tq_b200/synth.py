@@ -137,6 +137,31 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class SearchWorkload:
+    """Vector-search recipe: ``n`` database rows and ``nq`` queries, unit-norm
+    N(0,1) fp32 of dimension d (streams 0 and 2 of ``seed``), TurboQuant_prod
+    at ``bits`` total bits, top-``k`` per query."""
+    name: str
+    seed: int
+    n: int
+    nq: int
+    d: int
+    bits: int
+    k: int
+
+    def scaled(self, **kw) -> "SearchWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+VECTOR_SEARCH = SearchWorkload("vector_search", 4, 1_000_000, 1024, 1536, 4, 10)
+
+
+def search_inputs(w: SearchWorkload):
+    """(database [n, d], queries [nq, d]) fp32 unit rows."""
+    return unit_rows(w.n, w.d, w.seed, STREAM_K), unit_rows(w.nq, w.d, w.seed, STREAM_Q)
+
+
 def channel_scales(w: Workload) -> tuple[np.ndarray, np.ndarray]:
     """Per (KV head, channel) scales for K and V: lognormal(0, sigma) with
     ``n_outliers`` random channels per head multiplied by ``outlier_gain``."""
@@ -208,10 +233,16 @@ def as_float64(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def unit_rows(n: int, d: int, seed: int, stream: int) -> np.ndarray:
-    """n rows of N(0,1) fp32 normalised to unit length (vector-search inputs)."""
-    x = _normal_rows(generator(seed, stream), (n, d)).astype(np.float64)
-    x /= np.linalg.norm(x, axis=1, keepdims=True)
-    return x.astype(np.float32)
+    """n rows of N(0,1) fp32 normalised to unit length (vector-search inputs).
+    The norm is taken in fp64 row by row; rows are processed in chunks so a
+    10^6 x 1536 database needs no fp64 copy of itself."""
+    x = _normal_rows(generator(seed, stream), (n, d))
+    step = 1 << 16
+    for a in range(0, n, step):
+        c = x[a:a + step].astype(np.float64)
+        c /= np.linalg.norm(c, axis=1, keepdims=True)
+        x[a:a + step] = c.astype(np.float32)
+    return x
 
 
 def rope_for(w: Workload, t_max: Optional[int] = None):

@@ -281,3 +281,27 @@ def test_attention_degenerate_cases():
     # single key -> its value
     out1 = att.decode(q, cache, c, [1], 0.1)
     assert np.max(np.abs(out1[0] - vals[0])) < 1e-12
+
+
+# ---------------------------------------------------------------- vector search (d = 1536)
+
+def test_scan_scores_equal_dequantized_inner_products_d1536():
+    """Scores of the oracle scan equal <q, x~_j> with x~ the dequantized rows
+    (identity of the estimator form), and top-k matches a brute-force sort."""
+    from oracle import scan
+    d = 1536
+    c = oc.make_codec(d, 4, True, 4, synth.rotation_signs(d, 4), synth.qjl_matrix_bf16(d, 4))
+    x = synth.unit_rows(40, d, 4, 0).astype(np.float64)
+    q = synth.unit_rows(3, d, 4, 2).astype(np.float64)
+    enc = oc.quantize_keys(x, c)
+    kcode, kscale = oc.pack_keys(enc, c)
+    s = scan.scores(q, kcode, kscale, c)
+    ik, sg, nk, rk = oc.unpack_keys(kcode, kscale, c)
+    xt = oc.dequant_keys(ik, sg, nk, rk, c)
+    assert np.max(np.abs(s - q @ xt.T)) < 1e-12
+    idx, val = scan.topk(s, 5)
+    for i in range(3):
+        brute = sorted(range(40), key=lambda j: (-s[i, j], j))[:5]
+        assert list(idx[i]) == brute
+    # the estimator tracks the true inner products (unit rows, 3+1 bits)
+    assert np.corrcoef(s.ravel(), (q @ x.T).ravel())[0, 1] > 0.9
