@@ -403,6 +403,53 @@ def quantize_extra(wname: str, pk: dict, steps: int = 40):
                 l2="rotating %d input sets (%.0f MB)" % (n_sets, n_sets * in_bytes / 1e6))
 
 
+def bidir_extra(pk: dict, steps: int = 10):
+    """ESM-2-shaped bidirectional pass over the compressed cache (every query
+    attends to every key): algorithmic flops 2 T^2 (2d) + 2 T^2 d per head
+    (logits from the rotated MSE + QJL columns, then P V)."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.WORKLOADS["esm_prefill"]
+    D = synth.rotation_signs(w.d, w.seed)
+    S = synth.qjl_matrix_bf16(w.d, w.seed)
+    codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
+    rows_cap = (w.T + 31) // 32 * 32
+    r = synth.rope_for(w, max(rows_cap, w.Lq))
+    rope = (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+    K, V = synth.kv_inputs_torch(w)
+    cache = native.alloc_cache(codec, w.B, w.Hkv, rows_cap)
+    native.quantize_kv(codec, K, V, cache, rope=rope)
+    q = synth.query_inputs_torch(w, Lq=w.Lq)
+    out = torch.empty((w.B, w.Hq, w.Lq, w.d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(native.attention_bidir_workspace(codec, w.B, w.Hq, w.Lq), dtype=torch.uint8,
+                     device="cuda")
+    scale = 1.0 / math.sqrt(w.d)
+    sa, so = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for ev in (sa, so, e0, e1):      # torch creates the CUDA event on first record
+        ev.record()
+    for _ in range(2):
+        native.attention_bidir(codec, q, cache, w.T, scale, out, ws, rope=rope)
+    torch.cuda.synchronize()
+    kt, tt = [], []
+    for _ in range(steps):
+        native.set_timing_events(sa, so)
+        e0.record()
+        native.attention_bidir(codec, q, cache, w.T, scale, out, ws, rope=rope)
+        e1.record()
+        native.set_timing_events(None, None)
+        torch.cuda.synchronize()
+        kt.append(sa.elapsed_time(so) / 1e3)
+        tt.append(e0.elapsed_time(e1) / 1e3)
+    flops = w.B * w.Hq * (2 * w.T * w.Lq * 2 * w.d + 2 * w.T * w.Lq * w.d)
+    k = statistics.median(kt)
+    return dict(workload=describe(w) + f", Lq={w.Lq} bidirectional", us_per_call=statistics.median(tt) * 1e6,
+                roofline=dict(bound="tensor", achieved=flops / k / 1e12, peak=pk["bf16"], unit="TFLOP/s",
+                              frac=flops / k / 1e12 / pk["bf16"], algorithmic_flops=flops,
+                              kernel="bidir_tile_kernel", kernel_us=k * 1e6,
+                              note="bf16 hi/lo split: 3 MMAs per product, not counted in flops"))
+
+
 def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
     import torch
     from rotated_codebook_kv_tq_b200 import synth
@@ -584,6 +631,10 @@ def main():
             extras["quantize_esm_prefill"] = quantize_extra("esm_prefill", pk)
         except Exception as e:  # report, do not hide
             extras["quantize_esm_prefill"] = dict(error=repr(e))
+        try:
+            extras["bidir_esm_prefill"] = bidir_extra(pk)
+        except Exception as e:
+            extras["bidir_esm_prefill"] = dict(error=repr(e))
         try:
             extras["decode_long_context"] = decode_extra("long_decode", pk)
         except Exception as e:

@@ -30,7 +30,8 @@
  *     (a cudaStream_t; NULL = legacy default stream), and no call blocks the
  *     host.  Launch failures return TQ_ERR_CUDA; faults inside a kernel
  *     surface at the caller's next synchronisation.
- *   - Supported: d in {64, 128}; key MSE bits 1..4 (with QJL: 2 <= bits_k <= 5
+ *   - Supported: d in {64, 128} for the KV-cache calls and d = 1536 for the
+ *     vector-search calls; key MSE bits 1..4 (with QJL: 2 <= bits_k <= 5
  *     total); value bits 1..4.
  */
 #ifndef TQ_B200_H
@@ -186,6 +187,65 @@ int tq_attention_logits(const tq_codec *codec, const void *q, int dtype, int B, 
                         int max_seq_len, float scale, const float *rope_cos,
                         const float *rope_sin, int num_splits, void *workspace,
                         size_t ws_bytes, float *out, float *logits, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Bidirectional attention over the compressed cache (prefill-style pass):
+ * every query i of a sequence attends to all T cached keys, no mask
+ * ("TurboESM ...", sections 2.A and 2.E: RoPE then rotation, attention straight
+ * from the compressed cache).  Query i is RoPE-rotated at position i.
+ * Same estimator as tq_attention_decode, evaluated as dense tiles in the
+ * rotated domain on the tensor cores.
+ * q      device [B][H][Lq][d] (TQ_F32 or TQ_BF16); query head h reads KV head
+ *        h / (H / Hkv).   out  device fp32 [B][H][Lq][d].
+ * T      cached tokens per (b, KV head), 1..rows_cap.
+ * Supported: d = 64 with the codec's key MSE bits 1..3 (+QJL) and value bits 1..4.
+ * workspace: >= tq_attention_bidir_workspace(...) bytes, 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+int tq_attention_bidir_workspace(const tq_codec *codec, int B, int H, int Lq, size_t *bytes);
+int tq_attention_bidir(const tq_codec *codec, const void *q, int dtype, int B, int H, int Hkv,
+                       int Lq, const tq_cache *cache, int T, float scale, const float *rope_cos,
+                       const float *rope_sin, void *workspace, size_t ws_bytes, float *out,
+                       void *stream);
+
+/* ------------------------------------------------------------------------
+ * Vector search over TURBOQUANT_prod codes, d = 1536 ("Google presenta
+ * TurboQuant ...", "Velocidad y eficiencia de indexacion": the codes are
+ * data-oblivious, so indexing is a single encode pass with no training;
+ * "Eliminacion del sesgo interno del producto": the prod estimator of <q, x>).
+ * The codec must have d = 1536 and QJL keys with key MSE bits 1..4.  For
+ * d = 1536 the rotation is Pi = (H_12 kron H_128) diag(D) / sqrt(1536), H_12
+ * the Paley type-I matrix of GF(11) (H = I + [[0, 1^T], [-1, Q]],
+ * Q[i][j] = chi(j - i)), H_128 Sylvester-ordered.
+ *
+ * tq_index_build encodes n database rows exactly like keys (no RoPE):
+ *   x        device fp32 [n][1536], 16-byte aligned.
+ *   kcode    device u8 [n][planes][192] (planes = MSE bits + 1; plane p bit i of
+ *            row j = bit p of code i, the last plane = the QJL sign bits),
+ *            16-byte aligned.
+ *   kscale   device fp16 [n][2] = (nu, rho), 4-byte aligned.
+ *   status   device u32, nullable: incremented once per row that had a
+ *            non-finite entry (or a norm above the fp16 range); such rows are
+ *            stored as zero rows.
+ *   workspace >= tq_index_workspace(...) bytes (residual scratch of at most
+ *            65536 rows), 16-byte aligned.
+ * tq_scan_topk scores nq queries against the n rows with
+ *   s_qj = nu_j (<Pi q, c[idx_j]> + sqrt(pi/2)/1536 rho_j <S Pi q, 2 sigma_j - 1>)
+ * and returns, per query, the k best rows by (score descending, index
+ * ascending):
+ *   q        device fp32 [nq][1536], 16-byte aligned (unit norm is not required).
+ *   idx      device int32 [nq][k];  score  device fp32 [nq][k].
+ *   1 <= k <= min(16, n);  workspace >= tq_scan_workspace(...) bytes, 16-byte aligned.
+ * Scores are evaluated in fp32 on the tensor cores (bf16 hi + lo operands);
+ * rows whose scores differ by less than ~1e-5 relative may swap places.
+ * ------------------------------------------------------------------------ */
+int tq_index_workspace(const tq_codec *codec, int64_t n, size_t *bytes);
+int tq_index_build(const tq_codec *codec, const float *x, int64_t n, uint8_t *kcode,
+                   uint16_t *kscale, uint32_t *status, void *workspace, size_t ws_bytes,
+                   void *stream);
+int tq_scan_workspace(const tq_codec *codec, int64_t n, int nq, int k, size_t *bytes);
+int tq_scan_topk(const tq_codec *codec, const uint8_t *kcode, const uint16_t *kscale, int64_t n,
+                 const float *q, int nq, int k, int32_t *idx, float *score, void *workspace,
+                 size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Decode without a workspace, for callers that cannot allocate device memory.

@@ -15,7 +15,7 @@ std::atomic<uint64_t> g_launches{0};
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool supported_d(int d) { return d == 64 || d == 128; }
+bool supported_d(int d) { return d == 64 || d == 128 || d == 1536; }
 
 // a_t = 2^-b sum_idx c[idx] prod_{p in S_t} (2 bit_p(idx) - 1) for the odd
 // subsets S_t of the b code bits, in increasing bit-mask order.
@@ -42,6 +42,8 @@ void walsh_coefficients(const float *c, int bits, float *out, float *absmax, flo
 }
 
 int check_cache(const tq_codec *c, const tq_cache *cache) {
+  if (c && c->d > 128)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "KV-cache calls support d = 64 and 128 (d = 1536 is index-only)");
   if (!cache || !cache->kcode || !cache->kscale || !cache->vcode || !cache->vnorm)
     return tq_fail(TQ_ERR_INVALID_ARG, "cache: every plane pointer is required");
   if (cache->B <= 0 || cache->Hkv <= 0 || cache->rows_cap <= 0 || cache->rows_cap % 32)
@@ -103,7 +105,8 @@ int tq_build_codebook(int d, int bits, float *centroids, float *thresholds,
 int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   if (!desc || !out) return tq_fail(TQ_ERR_INVALID_ARG, "codec: NULL argument");
   *out = nullptr;
-  if (!supported_d(desc->d)) return tq_fail(TQ_ERR_UNSUPPORTED, "codec: d must be 64 or 128");
+  if (!supported_d(desc->d))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "codec: d must be 64 or 128 (KV cache) or 1536 (index)");
   const int mse_k = desc->qjl_k ? desc->bits_k - 1 : desc->bits_k;
   if (mse_k < 1 || mse_k > 4 || desc->bits_v < 1 || desc->bits_v > 4)
     return tq_fail(TQ_ERR_UNSUPPORTED,
@@ -269,6 +272,35 @@ int tq_attention_logits(const tq_codec *c, const void *q, int dtype, int B, int 
   if (!logits) return tq_fail(TQ_ERR_INVALID_ARG, "logits: NULL logits");
   return decode_common(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale, rope_cos,
                        rope_sin, num_splits, workspace, ws_bytes, out, logits, stream);
+}
+
+int tq_attention_bidir_workspace(const tq_codec *c, int B, int H, int Lq, size_t *bytes) {
+  if (!c || !bytes || B <= 0 || H <= 0 || Lq <= 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "bidir workspace: bad arguments");
+  *bytes = bidir_workspace_bytes(c, B, H, Lq);
+  return TQ_OK;
+}
+
+int tq_attention_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int Hkv,
+                       int Lq, const tq_cache *cache, int T, float scale, const float *rope_cos,
+                       const float *rope_sin, void *workspace, size_t ws_bytes, float *out,
+                       void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: NULL codec");
+  if (int e = check_cache(c, cache)) return e;
+  if (!q || !out || !workspace) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: NULL q/out/workspace");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: dtype");
+  if (B != cache->B || Hkv != cache->Hkv || H <= 0 || H % Hkv || Lq <= 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "bidir: B/Hkv differ from the cache's, H % Hkv, or Lq");
+  if (T < 1 || T > cache->rows_cap) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: T outside 1..rows_cap");
+  if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: scale not finite");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "bidir: rope_cos and rope_sin go together");
+  if (bidir_workspace_bytes(c, B, H, Lq) > ws_bytes)
+    return tq_fail(TQ_ERR_WORKSPACE, "bidir: workspace smaller than tq_attention_bidir_workspace()");
+  if (!aligned(workspace, 16) || !aligned(out, 4))
+    return tq_fail(TQ_ERR_ALIGNMENT, "bidir: workspace/out alignment");
+  return launch_bidir(c, q, dtype, B, H, Hkv, Lq, cache, T, scale, rope_cos, rope_sin, workspace,
+                      out, static_cast<cudaStream_t>(stream));
 }
 
 int tq_dequantize(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,

@@ -27,6 +27,8 @@
 // main loop); the chunk partials are merged by decode.cu's combine kernel.
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "tq_device.cuh"
 #include "tq_sm100.cuh"
 #include "tq_tc.h"
@@ -49,6 +51,18 @@ __host__ __device__ constexpr int odd_mask(int nb, int t) {
     }
   }
   return 0;
+}
+
+__host__ __device__ constexpr int tc_tmem_cols(int G, int MBK, int BV, bool QJL) {
+  return (32 + 32 * ((1 << (MBK - 1)) + (QJL ? 1 : 0))) > (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G))
+             ? (32 + 32 * ((1 << (MBK - 1)) + (QJL ? 1 : 0)))
+             : (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G));
+}
+__host__ __device__ constexpr int tc_tmem_alloc(int G, int MBK, int BV, bool QJL) {
+  return tc_tmem_cols(G, MBK, BV, QJL) <= 64    ? 64
+         : tc_tmem_cols(G, MBK, BV, QJL) <= 128 ? 128
+         : tc_tmem_cols(G, MBK, BV, QJL) <= 256 ? 256
+                                                 : 512;
 }
 
 // Signed base-256 digits of v (|v| < 2^31): v = L0 + 2^8 L1 + 2^16 L2 + 2^24 L3.
@@ -90,6 +104,7 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
   __shared__ double dred[TCT / 32][2 * G];
   __shared__ float Fs[2 * G];
   __shared__ __align__(16) int8_t bks[N * KTOT];
+  extern __shared__ __align__(16) uint16_t sts[];   // S^T, bf16 [TD][TD] (dynamic)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x;
@@ -119,13 +134,18 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
 #pragma unroll
     for (int k = 0; k < TNW; ++k) q1s[warp][lane + 32 * k] = x[k] * inv_sqrt_d;
   }
+  if (QJL) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.ST);
+    for (int e = tid; e < TD * TD / 8; e += TCT) reinterpret_cast<uint4 *>(sts)[e] = src[e];
+  }
   __syncthreads();
   if (QJL) {
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 8
     for (int j = 0; j < TD; ++j) {
-      const float s = tq_bf16_to_f32(a.ST[j * TD + tid]);
+      const float s = tq_bf16_to_f32(sts[j * TD + tid]);
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[h] = fmaf(s, q1s[h][j], acc[h]);
     }
@@ -265,7 +285,7 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
 }
 
 template <int G, int MBK, int BV, bool QJL>
-__global__ void __launch_bounds__(TCT, 1) tc_chunk_kernel(TcArgs a) {
+__global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
   constexpr int TK = 1 << (MBK - 1);
   constexpr int TV = 1 << (BV - 1);
   constexpr int N = tc_n(G);
@@ -274,12 +294,16 @@ __global__ void __launch_bounds__(TCT, 1) tc_chunk_kernel(TcArgs a) {
   constexpr int KTOT = KM + (QJL ? TD : 0);
   constexpr int BKB = N * KTOT;
   constexpr int BKC = BKB + G * 16;
+  // Tensor memory: the key phase and the value phase of a unit never overlap
+  // in time, so their regions share columns.
+  //   key phase:   DK [0, 2N)   AK [32, 32 + 32 (TK + QJL))
+  //   value phase: AV [0, 16 TV) (two buffers)   DV [16 TV, 16 TV + N TV)
   constexpr int C_DK = 0;
   constexpr int C_AK = 32;
-  constexpr int C_AV = C_AK + (TK + (QJL ? 1 : 0)) * 32;
-  constexpr int C_DV = C_AV + 2 * TV * 8;
-  constexpr int USED = C_DV + TV * N;
-  constexpr int NCOLS = USED <= 64 ? 64 : USED <= 128 ? 128 : USED <= 256 ? 256 : 512;
+  constexpr int C_AV = 0;
+  constexpr int C_DV = 2 * TV * 8;
+  constexpr int USED = tc_tmem_cols(G, MBK, BV, QJL);
+  constexpr int NCOLS = tc_tmem_alloc(G, MBK, BV, QJL);
   static_assert(USED <= 512, "tensor memory budget");
   static_assert(2 * N <= 32, "key accumulators must fit in 32 columns");
   constexpr uint32_t IDESC = sm100::idesc_i8(128, N);
@@ -711,8 +735,18 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // CTAs per SM: one by default (largest sub-chunks); TQ_TC_CTAS_PER_SM asks
+  // for more, capped by tensor-memory slots, after which the sub-chunk shrinks
+  // until that many fit in shared memory (each unit is double-buffered)
+  constexpr int NCOLS = tc_tmem_alloc(G, MBK, BV, QJL);
+  int per_sm = 1;
+  if (const char *e = getenv("TQ_TC_CTAS_PER_SM")) per_sm = atoi(e);
+  if (per_sm > 512 / NCOLS) per_sm = 512 / NCOLS;
+  if (per_sm > 4) per_sm = 4;
+  if (per_sm < 1) per_sm = 1;
+  const int budget = per_sm == 1 ? 200 * 1024 : (227 * 1024) / per_sm - 2048;
   int sub = a.chunk;
-  while (sub > 128 && tc_layout(sub, PK, BV, G, N, BKC).total > 200 * 1024) sub -= 128;
+  while (sub > 128 && tc_layout(sub, PK, BV, G, N, BKC).total > budget) sub -= 128;
   a.sub = sub;
   const int smem = tc_layout(sub, PK, BV, G, N, BKC).total;
   static bool attr_done[64] = {};
@@ -722,10 +756,14 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
       return tq_check_launch("cudaFuncSetAttribute(tc_chunk)");
     attr_done[dev] = true;
   }
-  tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, 0, stream>>>(a);
+  int occ = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tc_chunk_kernel<G, MBK, BV, QJL>, TCT, smem);
+  if (occ < 1) occ = 1;
+  if (occ < per_sm) per_sm = occ;
+  tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, QJL ? TD * TD * 2 : 0, stream>>>(a);
   if (int e = tq_check_launch("tc_prep_kernel")) return e;
   const int items = a.B * a.Hkv * a.splits;
-  const int grid = items < sms ? items : sms;
+  const int grid = items < sms * per_sm ? items : sms * per_sm;
   cudaEvent_t ev0, ev1;
   tq_timing_events(&ev0, &ev1);
   unsigned ev_flags = cudaEventRecordDefault;

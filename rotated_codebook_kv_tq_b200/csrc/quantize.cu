@@ -41,7 +41,6 @@ struct QuantArgs {
   uint32_t *status;
   const uint16_t *S;
   const uint16_t *ST;  // S transposed (bf16)
-  int stage_s;         // 1: stage S^T in shared memory (large calls)
   int64_t g_first;   // first 32-token group touched
   int64_t n_groups;  // groups touched per (b, h)
   TqBooks books;
@@ -109,10 +108,17 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
     tks[threadIdx.x] = a.books.tk[threadIdx.x];
     tvs[threadIdx.x] = a.books.tv[threadIdx.x];
   }
-  if (a.books.qjl && a.stage_s) {
-    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-      const int i = e / D, j = e % D;
-      ST[j * D + i] = tq_bf16_to_f32(a.S[e]);
+  if (a.books.qjl) {
+    // stage S^T as fp32: coalesced 16-byte loads of the transposed bf16 copy
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.ST);
+    for (int e = threadIdx.x; e < D * D / 8; e += blockDim.x) {
+      const uint4 v = src[e];
+      const float4 lo = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                    __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+      const float4 hi = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                                    __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+      reinterpret_cast<float4 *>(ST)[2 * e] = lo;
+      reinterpret_cast<float4 *>(ST)[2 * e + 1] = hi;
     }
   }
   __syncthreads();
@@ -167,19 +173,11 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
         float z[NPL];
 #pragma unroll
         for (int k = 0; k < NPL; ++k) z[k] = 0.f;
-        if (a.stage_s) {
-          for (int j = 0; j < D; ++j) {
-            const float rj = rbuf[warp][j];
+#pragma unroll 4
+        for (int j = 0; j < D; ++j) {
+          const float rj = rbuf[warp][j];
 #pragma unroll
-            for (int k = 0; k < NPL; ++k) z[k] = fmaf(ST[j * D + lane + 32 * k], rj, z[k]);
-          }
-        } else {
-          for (int j = 0; j < D; ++j) {
-            const float rj = rbuf[warp][j];
-#pragma unroll
-            for (int k = 0; k < NPL; ++k)
-              z[k] = fmaf(tq_bf16_to_f32(a.ST[j * D + lane + 32 * k]), rj, z[k]);
-          }
+          for (int k = 0; k < NPL; ++k) z[k] = fmaf(ST[j * D + lane + 32 * k], rj, z[k]);
         }
         __syncwarp();
         const int p = a.books.mse_bits_k;
@@ -464,7 +462,7 @@ int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
 
 template <int D>
 int run_quantize(const QuantArgs &a, cudaStream_t stream) {
-  const size_t shm = a.books.qjl && a.stage_s ? sizeof(float) * D * D : 0;
+  const size_t shm = a.books.qjl ? sizeof(float) * D * D : 0;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(quantize_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -516,7 +514,6 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   a.books = c->books;
   if (T == 0) return TQ_OK;
   const int64_t items = static_cast<int64_t>(B) * H * a.n_groups;
-  a.stage_s = items > 64 ? 1 : 0;
   // TQ_QUANT_IMPL=simt keeps the CUDA-core sketch (a complete second
   // implementation, used to cross-check the tensor-core one)
   const char *impl = getenv("TQ_QUANT_IMPL");

@@ -14,7 +14,7 @@ bool lloyd_max(int d, int bits, std::vector<double> &c, std::vector<double> &t, 
 }
 
 // Largest head dim the kernels are instantiated for.
-constexpr int TQ_MAX_D = 128;
+constexpr int TQ_MAX_D = 1536;
 constexpr int TQ_MAX_LEVELS = 16;
 
 // Codebooks and rotation signs passed by value to every kernel (kernel
@@ -61,5 +61,9 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
                   const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
                   const float *rc, const float *rs, int splits, void *ws, float *out,
                   float *logits, cudaStream_t stream);
+size_t bidir_workspace_bytes(const tq_codec *c, int B, int H, int Lq);
+int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int Hkv, int Lq,
+                 const tq_cache *cache, int T, float scale, const float *rc, const float *rs,
+                 void *ws, float *out, cudaStream_t stream);
 int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
                    int64_t rows, float *out, cudaStream_t stream);

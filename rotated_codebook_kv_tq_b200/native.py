@@ -23,7 +23,9 @@ TQ_F32, TQ_BF16 = 0, 1
 EXPORTS = [
     "tq_build_codebook", "tq_codec_create", "tq_codec_destroy", "tq_codec_codebooks",
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
-    "tq_attention_logits", "tq_attention_decode_noalloc", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
+    "tq_attention_logits", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
+    "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
+    "tq_scan_topk", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
     "tq_last_error",
 ]
 
@@ -74,6 +76,13 @@ def lib() -> ctypes.CDLL:
         L.tq_attention_decode_noalloc.argtypes = [vp, vp, i32, i32, i32, i32,
                                                   ctypes.POINTER(CacheDesc), vp, i32, f32, vp,
                                                   vp, i32, vp, vp]
+        L.tq_attention_bidir_workspace.argtypes = [vp, i32, i32, i32, ctypes.POINTER(sz)]
+        L.tq_attention_bidir.argtypes = [vp, vp, i32, i32, i32, i32, i32, ctypes.POINTER(CacheDesc),
+                                         i32, f32, vp, vp, vp, sz, vp, vp]
+        L.tq_index_workspace.argtypes = [vp, i64, ctypes.POINTER(sz)]
+        L.tq_index_build.argtypes = [vp, vp, i64, vp, vp, vp, vp, sz, vp]
+        L.tq_scan_workspace.argtypes = [vp, i64, i32, i32, ctypes.POINTER(sz)]
+        L.tq_scan_topk.argtypes = [vp, vp, vp, i64, vp, i32, i32, vp, vp, vp, sz, vp]
         L.tq_dequantize.argtypes = [vp, ctypes.POINTER(CacheDesc), i32, i64, i64, vp, vp]
         L.tq_set_timing_events.argtypes = [vp, vp]
         L.tq_launch_count.argtypes = []
@@ -241,6 +250,56 @@ def attention_logits(codec: Codec, q, cache: Cache, max_seq_len: int, scale: flo
                                     float(scale), _ptr(rc), _ptr(rs), num_splits,
                                     workspace.data_ptr(), ws_bytes, out.data_ptr(),
                                     logits.data_ptr(), _stream(stream)))
+
+
+def attention_bidir_workspace(codec: Codec, B: int, H: int, Lq: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().tq_attention_bidir_workspace(codec.handle, B, H, Lq, ctypes.byref(n)))
+    return n.value
+
+
+def attention_bidir(codec: Codec, q, cache: Cache, T: int, scale: float, out, workspace,
+                    rope=None, stream=None) -> None:
+    """tq_attention_bidir: q [B, H, Lq, d] (query i at position i) -> out fp32."""
+    B, H, Lq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib().tq_attention_bidir(codec.handle, q.data_ptr(), _dtype_code(q), B, H, cache.Hkv,
+                                   Lq, ctypes.byref(desc), T, float(scale), _ptr(rc), _ptr(rs),
+                                   workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                                   _stream(stream)))
+
+
+def index_workspace(codec: Codec, n: int) -> int:
+    b = ctypes.c_size_t(0)
+    check(lib().tq_index_workspace(codec.handle, ctypes.c_int64(n), ctypes.byref(b)))
+    return b.value
+
+
+def index_build(codec: Codec, x, kcode, kscale, workspace, status=None, stream=None) -> None:
+    """tq_index_build: x fp32 [n, 1536] -> kcode u8 [n, planes, 192], kscale fp16 [n, 2]."""
+    n = x.shape[0]
+    check(lib().tq_index_build(codec.handle, x.data_ptr(), ctypes.c_int64(n), kcode.data_ptr(),
+                               kscale.data_ptr(), _ptr(status), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def scan_workspace(codec: Codec, n: int, nq: int, k: int) -> int:
+    b = ctypes.c_size_t(0)
+    check(lib().tq_scan_workspace(codec.handle, ctypes.c_int64(n), nq, k, ctypes.byref(b)))
+    return b.value
+
+
+def scan_topk(codec: Codec, kcode, kscale, q, k: int, idx, score, workspace,
+              stream=None) -> None:
+    """tq_scan_topk: q fp32 [nq, 1536] against n encoded rows -> idx int32 / score fp32 [nq, k]."""
+    n = kcode.shape[0]
+    nq = q.shape[0]
+    check(lib().tq_scan_topk(codec.handle, kcode.data_ptr(), kscale.data_ptr(), ctypes.c_int64(n),
+                             q.data_ptr(), nq, k, idx.data_ptr(), score.data_ptr(),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
