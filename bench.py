@@ -105,7 +105,10 @@ class ClockSampler:
                                                         if r[3].replace(".", "").isdigit()))
 
 
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """Rank setup from the torchrun environment.  The process group carries
+    only the barrier and the max-over-ranks timing (replicas share no data);
+    ``backend="gloo"`` runs the same host logic on CPU."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -113,9 +116,12 @@ def dist_init():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return world, rank, local
 
 
@@ -130,9 +136,16 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_value(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput of N independent replicas: the units all ranks
+    processed over the slowest rank's time."""
+    return world * units_per_rank / max_seconds
 
 
 def blas_threads() -> int:
@@ -447,7 +460,73 @@ def bidir_extra(pk: dict, steps: int = 10):
                 roofline=dict(bound="tensor", achieved=flops / k / 1e12, peak=pk["bf16"], unit="TFLOP/s",
                               frac=flops / k / 1e12 / pk["bf16"], algorithmic_flops=flops,
                               kernel="bidir_tile_kernel", kernel_us=k * 1e6,
-                              note="bf16 hi/lo split: 3 MMAs per product, not counted in flops"))
+                              note="three-term bf16 split: 6 MMA sets per product, not counted in flops"))
+
+
+def search_extra(pk: dict, steps: int = 5):
+    """Vector search, d = 1536, TurboQuant_prod at 4 bits: index build of 10^6
+    unit rows (input fp32 GB/s; the QJL sketch is 2 d^2 flops per row on the
+    tensor cores) and the inner-product scan + top-10 of 1024 queries
+    (2 * 3072 flops per (row, query), the estimator as one GEMM)."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.VECTOR_SEARCH
+    codec = native.Codec(w.d, w.bits, True, 4, synth.rotation_signs(w.d, w.seed),
+                         synth.qjl_matrix_bf16(w.d, w.seed))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed * 1000)
+    x = torch.randn((w.n, w.d), generator=g, device="cuda")
+    x /= x.norm(dim=1, keepdim=True)
+    q = torch.randn((w.nq, w.d), generator=g, device="cuda")
+    q /= q.norm(dim=1, keepdim=True)
+    kcode = torch.empty((w.n, codec.planes_k, w.d // 8), dtype=torch.uint8, device="cuda")
+    kscale = torch.empty((w.n, 2), dtype=torch.float16, device="cuda")
+    iws = torch.empty(native.index_workspace(codec, w.n), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((w.nq, w.k), dtype=torch.int32, device="cuda")
+    score = torch.empty((w.nq, w.k), dtype=torch.float32, device="cuda")
+    sws = torch.empty(native.scan_workspace(codec, w.n, w.nq, w.k), dtype=torch.uint8, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:
+        e.record()
+    native.index_build(codec, x, kcode, kscale, iws)
+    native.scan_topk(codec, kcode, kscale, q, w.k, idx, score, sws)
+    torch.cuda.synchronize()
+    bt, st, kt = [], [], []
+    for _ in range(steps):
+        ev[0].record()
+        native.index_build(codec, x, kcode, kscale, iws)
+        ev[1].record()
+        native.set_timing_events(ev[2], ev[3])
+        e_s0, e_s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_s0.record()
+        native.scan_topk(codec, kcode, kscale, q, w.k, idx, score, sws)
+        e_s1.record()
+        native.set_timing_events(None, None)
+        torch.cuda.synchronize()
+        bt.append(ev[0].elapsed_time(ev[1]) / 1e3)
+        st.append(e_s0.elapsed_time(e_s1) / 1e3)
+        kt.append(ev[2].elapsed_time(ev[3]) / 1e3)
+    b, s_, k = statistics.median(bt), statistics.median(st), statistics.median(kt)
+    in_bytes = w.n * w.d * 4
+    sketch_flops = 2 * w.n * w.d * w.d
+    scan_flops = 2 * 2 * w.d * w.n * w.nq
+    return dict(
+        workload=f"vector_search: n={w.n} d={w.d} fp32 unit rows, nq={w.nq}, TurboQuant_prod "
+                 f"{w.bits} bits, top-{w.k}",
+        index_build=dict(ms_per_call=b * 1e3, input_GBps=in_bytes / b / 1e9,
+                         rows_per_s=w.n / b,
+                         roofline=dict(bound="tensor", achieved=sketch_flops / b / 1e12,
+                                       peak=pk["bf16"], unit="TFLOP/s",
+                                       frac=sketch_flops / b / 1e12 / pk["bf16"],
+                                       algorithmic_flops=sketch_flops,
+                                       note="whole call (encode + sketch GEMM); bf16 hi/lo split: "
+                                            "2 MMA passes, not counted")),
+        scan_topk=dict(ms_per_call=s_ * 1e3, queries_per_s=w.nq / s_,
+                       roofline=dict(bound="tensor", achieved=scan_flops / k / 1e12, peak=pk["bf16"],
+                                     unit="TFLOP/s", frac=scan_flops / k / 1e12 / pk["bf16"],
+                                     algorithmic_flops=scan_flops, kernel="ix_scan_kernel",
+                                     kernel_ms=k * 1e3)),
+        l2="database codes 772 MB and input 6.1 GB > L2")
 
 
 def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
@@ -588,14 +667,14 @@ def main():
     total, kern, per_step, clocks = time_decode(bench, K, W, world, sampler)
     total = max_over_ranks(total, world)
     kern = max_over_ranks(kern, world)
-    value = world * w.B * K / total
+    value = weak_value(w.B * K, world, total)
     alg = bench.cache_bytes_per_step()
     achieved = alg / kern / 1e9
 
     K_e2e = max(10, min(K, 300))
     dt, h2d, d2h = time_e2e(bench, K_e2e, 20)
     dt = max_over_ranks(dt, world)
-    e2e_value = world * w.B * K_e2e / dt
+    e2e_value = weak_value(w.B * K_e2e, world, dt)
 
     line = dict(metric="compressed-KV decode tokens/s", value=value, unit="tokens/s",
                 n_gpus=world, steps=K, warmup=W, ms_per_step=total / K * 1e3,
@@ -639,6 +718,10 @@ def main():
             extras["decode_long_context"] = decode_extra("long_decode", pk)
         except Exception as e:
             extras["decode_long_context"] = dict(error=repr(e))
+        try:
+            extras["vector_search"] = search_extra(pk)
+        except Exception as e:
+            extras["vector_search"] = dict(error=repr(e))
         line["extras"] = extras
     if rank == 0:
         print(json.dumps(line))

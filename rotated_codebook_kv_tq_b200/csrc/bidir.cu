@@ -14,10 +14,16 @@
 // A CTA owns 128 queries of one (batch, head) (TMEM lane = query) and walks the
 // keys in tiles of 64: S = Q_rot K_rot^T and O_tile = P V_rot each run as six
 // bf16 kind::f16 MMA sets (the order <= 2 products of a three-term bf16 split,
-// about 2^-26 relative: the logits reach ~100 on data with outlier channels,
-// and a two-term split's 2^-17 would shift them by ~1e-3) with fp32
+// about 2^-26 relative: the logits reach a few hundred on data with outlier
+// channels, and a two-term split's 2^-17 would shift them by ~1e-3) with fp32
 // accumulators in tensor memory; softmax statistics and the output sum stay
 // in fp32 registers of the query's thread.
+// The tensor core's fp32 accumulation does not round to nearest: every MMA
+// that adds into an accumulator can lose up to an ulp of it, and a chain of
+// 48 MMAs into one accumulator moves logits of ~200 by ~5e-4.  So S is split
+// over five accumulators: the five small split products share one (its
+// magnitude is ~2^-8 of the logit), and the leading hi*hi product spreads its
+// K steps over four, each a chain of two; they are added in fp32 registers.
 #include <math_constants.h>
 
 #include "tq_device.cuh"
@@ -122,19 +128,27 @@ __device__ __forceinline__ void split3_store(uint8_t *base, uint32_t stride, int
   *reinterpret_cast<__nv_bfloat16 *>(base + 2 * stride + off) = c;
 }
 
-// D (+)= sum over the six split products of order <= 2:
-// a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0 (about 2^-26 relative).
-__device__ __forceinline__ void mma6(uint32_t d, uint32_t a, uint32_t astr, uint32_t b,
-                                     uint32_t bstr, int ksteps, uint32_t lbo_a, uint32_t lbo_b,
-                                     uint32_t idesc) {
-  const int pa[6] = {0, 0, 1, 0, 1, 2}, pb[6] = {0, 1, 0, 2, 1, 0};
+// The six split products of order <= 2: a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0
+// (about 2^-26 relative).  The five small ones go first into d_small; the
+// K steps of a0 b0 go round-robin into `nbig` accumulators d_big + i * dstride
+// (nbig = 1 folds everything into d_small, for the P V product).
+__device__ __forceinline__ void mma6(uint32_t d_small, uint32_t d_big, uint32_t dstride, int nbig,
+                                     uint32_t a, uint32_t astr, uint32_t b, uint32_t bstr,
+                                     int ksteps, uint32_t lbo_a, uint32_t lbo_b, uint32_t idesc) {
+  const int pa[6] = {2, 1, 0, 1, 0, 0}, pb[6] = {0, 1, 2, 0, 1, 0};
   int n = 0;
 #pragma unroll
-  for (int t = 0; t < 6; ++t)
+  for (int t = 0; t < 5; ++t)
     for (int s = 0; s < ksteps; ++s, ++n)
-      sm100::mma_bf16_ss(d, sm100::smem_desc(a + pa[t] * astr + s * 2 * lbo_a, lbo_a, 128),
+      sm100::mma_bf16_ss(d_small, sm100::smem_desc(a + pa[t] * astr + s * 2 * lbo_a, lbo_a, 128),
                          sm100::smem_desc(b + pb[t] * bstr + s * 2 * lbo_b, lbo_b, 128), idesc,
                          n > 0);
+  for (int s = 0; s < ksteps; ++s) {
+    const uint32_t d = nbig > 1 ? d_big + (s % nbig) * dstride : d_small;
+    sm100::mma_bf16_ss(d, sm100::smem_desc(a + s * 2 * lbo_a, lbo_a, 128),
+                       sm100::smem_desc(b + s * 2 * lbo_b, lbo_b, 128), idesc,
+                       nbig > 1 ? (s >= nbig ? 1u : 0u) : 1u);
+  }
 }
 
 template <int D>
@@ -169,7 +183,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     cks[tid] = a.books.ck[tid];
     cvs[tid] = a.books.cv[tid];
   }
-  if (warp == 0) sm100::tmem_alloc(&tmem_s, 128);
+  if (warp == 0) sm100::tmem_alloc(&tmem_s, 512);
   if (tid == 0) {
     sm100::mbar_init(&mb, 1);
     abort_s = 0;
@@ -185,7 +199,9 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  const uint32_t tm = tmem_s, tS = tm, tO = tm + BK;
+  // columns: S small-product accumulator, four hi*hi accumulators, O
+  constexpr int NBIG = 4;
+  const uint32_t tm = tmem_s, tS = tm, tSb = tm + BK, tO = tm + (1 + NBIG) * BK;
   const uint32_t a_q = sm100::smem_addr(qs3), a_k = sm100::smem_addr(ks3);
   const uint32_t a_p = sm100::smem_addr(ps3), a_v = sm100::smem_addr(vs3);
 
@@ -194,43 +210,51 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   for (int i = 0; i < D; ++i) o[i] = 0.f;
   uint32_t phase = 0;
   for (int j0 = 0; j0 < a.T; j0 += BK) {
-    // ---- key tile (rows tid < BK) and value tile (coordinates tid < D)
-    if (tid < BK) {
-      const int j = j0 + tid;
+    // ---- key tile: thread (row tid % BK, half tid / BK) writes the MSE half
+    // (c[idx]) or the sign half (+-coef rho) of one key row; value tile:
+    // thread (coordinate tid % D, key group tid / D) writes 32 keys of V_rot^T.
+    static_assert(BQ == 2 * BK && BQ == 2 * D && BK == 64, "thread mapping");
+    {
+      const int row = tid % BK, half = tid / BK;
+      const int j = j0 + row;
       const bool ok = j < a.T;
       const uint8_t *krow = a.kcode + (bh * a.rows_cap + (ok ? j : 0)) * planes_k * (D / 8);
       const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale)[bh * a.rows_cap + (ok ? j : 0)];
       const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
       const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-      nuk[tid] = ok ? nu : 0.f;
+      if (half == 0) nuk[row] = ok ? nu : 0.f;
       const float qv = a.qjl_coef * rho;
       for (int w = 0; w < D / 32; ++w) {
         uint32_t pw[4] = {0u, 0u, 0u, 0u};
         for (int p = 0; p < planes_k; ++p) pw[p] = reinterpret_cast<const uint32_t *>(krow)[p * (D / 32) + w];
         for (int bit = 0; bit < 32; ++bit) {
           const int i = 32 * w + bit;
-          int idx = 0;
-          for (int p = 0; p < mbk; ++p) idx |= ((pw[p] >> bit) & 1) << p;
-          split3_store(ks3, K_BYTES, kmaj16(tid, i, BK), ok ? cks[idx] : 0.f);
-          const float sg = a.books.qjl ? (((pw[mbk] >> bit) & 1) ? qv : -qv) : 0.f;
-          split3_store(ks3, K_BYTES, kmaj16(tid, D + i, BK), ok ? sg : 0.f);
+          float val;
+          if (half == 0) {
+            int idx = 0;
+            for (int p = 0; p < mbk; ++p) idx |= ((pw[p] >> bit) & 1) << p;
+            val = ok ? cks[idx] : 0.f;
+          } else {
+            val = (ok && a.books.qjl) ? (((pw[mbk] >> bit) & 1) ? qv : -qv) : 0.f;
+          }
+          split3_store(ks3, K_BYTES, kmaj16(row, half * D + i, BK), val);
         }
       }
     }
-    if (tid < D) {
-      // V_rot^T row `tid` (coordinate), K = BK keys
-      for (int g = 0; g < BK / 32; ++g) {
+    {
+      const int coord = tid % D, g = tid / D;
+      {
         const int jg = j0 + 32 * g;
         uint32_t vw[4] = {0u, 0u, 0u, 0u};
         if (jg < a.T)
           for (int p = 0; p < nbv; ++p)
-            vw[p] = a.vcode[(bh * (a.rows_cap / 32) + jg / 32) * nbv * D + p * D + tid];
+            vw[p] = a.vcode[(bh * (a.rows_cap / 32) + jg / 32) * nbv * D + p * D + coord];
         for (int t = 0; t < 32; ++t) {
           const int j = jg + t;
           int idx = 0;
           for (int p = 0; p < nbv; ++p) idx |= ((vw[p] >> t) & 1) << p;
           const float val = j < a.T ? tq_half_to_f32(a.vnorm[bh * a.rows_cap + j]) * cvs[idx] : 0.f;
-          split3_store(vs3, V_BYTES, kmaj16(tid, 32 * g + t, D), val);
+          split3_store(vs3, V_BYTES, kmaj16(coord, 32 * g + t, D), val);
         }
       }
     }
@@ -240,7 +264,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     sm100::fence_after_sync();
     // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d)
     if (tid == 0) {
-      mma6(tS, a_q, Q_BYTES, a_k, K_BYTES, DP / 16, BQ * 16, BK * 16, IDESC_S);
+      mma6(tS, tSb, BK, NBIG, a_q, Q_BYTES, a_k, K_BYTES, DP / 16, BQ * 16, BK * 16, IDESC_S);
       sm100::mma_commit(&mb);
     }
     if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
@@ -256,6 +280,13 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
       sm100::wait_ld();
 #pragma unroll
       for (int e = 0; e < 16; ++e) sv[c + e] = __uint_as_float(r[e]);
+#pragma unroll
+      for (int i = 0; i < NBIG; ++i) {
+        sm100::tmem_ld16(sm100::tmem_lane(tSb + i * BK + c, warp), r);
+        sm100::wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sv[c + e] += __uint_as_float(r[e]);
+      }
     }
     float tmax = -CUDART_INF_F;
 #pragma unroll
@@ -282,7 +313,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     sm100::fence_after_sync();
     // ---- O_tile = P V_rot (M = 128 queries, N = d, K = 64 keys)
     if (tid == 0) {
-      mma6(tO, a_p, P_BYTES, a_v, V_BYTES, BK / 16, BQ * 16, D * 16, IDESC_O);
+      mma6(tO, tO, 0, 1, a_p, P_BYTES, a_v, V_BYTES, BK / 16, BQ * 16, D * 16, IDESC_O);
       sm100::mma_commit(&mb);
     }
     if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
@@ -328,7 +359,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  if (warp == 0) sm100::tmem_dealloc(tm, 128);
+  if (warp == 0) sm100::tmem_dealloc(tm, 512);
   (void)NPL;
 }
 
