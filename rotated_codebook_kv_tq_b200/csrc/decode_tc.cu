@@ -20,7 +20,10 @@
 //   column groups give each lane its own words), N = 4 limbs x G heads,
 //   K = 32 tokens; one accumulator per Walsh term, combined at the end.
 // * Persistent CTAs, one per SM, stream (chunk, sub-chunk) units through a
-//   double-buffered shared-memory ring filled by cp.async.bulk.
+//   double-buffered shared-memory ring filled by cp.async.bulk.  Each CTA has
+//   two 4-warp slices over the same 128 TMEM lanes that split the Walsh terms
+//   of every expansion, and key tiles are double-buffered in tensor memory so
+//   the expansion of tile j+1 overlaps the MMAs of tile j.
 //
 // Kernels: tc_prep (per (batch, KV head): RoPE, rotation and sketch of the G
 // query heads, fixed-point B operand for the keys) and tc_chunk (the split-K
@@ -37,7 +40,9 @@ namespace {
 
 constexpr int TD = 128;   // head dim of this path
 constexpr int TNW = TD / 32;
-constexpr int TCT = 128;  // threads per CTA: one TMEM lane each
+constexpr int TCT = 128;  // threads of tc_prep: one TMEM lane each
+constexpr int CW = 256;   // worker threads of tc_chunk: two slices of 128 TMEM lanes
+constexpr int CT = CW + 32;   // + the MMA-issuing warp
 
 // Odd subsets of {0..nb-1} in increasing bit-mask order (the Walsh terms).
 __host__ __device__ constexpr int odd_mask(int nb, int t) {
@@ -53,9 +58,12 @@ __host__ __device__ constexpr int odd_mask(int nb, int t) {
   return 0;
 }
 
+// Columns used by tc_chunk: key phase (two accumulator pairs in [0, 64), two
+// A buffers of 32 columns per key term from 64) or value phase (two A buffers
+// of 8 columns per Walsh term, then one accumulator of N columns per term).
 __host__ __device__ constexpr int tc_tmem_cols(int G, int MBK, int BV, bool QJL) {
-  return (32 + 32 * ((1 << (MBK - 1)) + (QJL ? 1 : 0))) > (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G))
-             ? (32 + 32 * ((1 << (MBK - 1)) + (QJL ? 1 : 0)))
+  return (64 + 64 * ((1 << (MBK - 1)) + (QJL ? 1 : 0))) > (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G))
+             ? (64 + 64 * ((1 << (MBK - 1)) + (QJL ? 1 : 0)))
              : (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G));
 }
 __host__ __device__ constexpr int tc_tmem_alloc(int G, int MBK, int BV, bool QJL) {
@@ -284,8 +292,18 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
   return false;
 }
 
+// tc_chunk: 288 threads = 8 worker warps (two slices of 4) + 1 MMA warp.
+// Worker warp w serves TMEM lane quarter w % 4 (rows or coordinates
+// 32 (w % 4) .. +31) for slice w / 4; the slices split the Walsh terms of
+// every expansion and the rows of the value B-operand build.  A tcgen05.mma
+// issue blocks for about as long as the MMA runs, so one lane of the last
+// warp does nothing but issue: workers publish each filled tensor-memory
+// buffer on an mbarrier (ak_full / av_full) and the MMA warp waits on those;
+// workers wait on the MMA commits (mb_k / mb_v) before reusing a buffer.
+// Key tiles are double-buffered: tile j+1 is expanded while tile j runs.
 template <int G, int MBK, int BV, bool QJL>
-__global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
+__global__ void __launch_bounds__(CT, 1) tc_chunk_kernel(TcArgs a) {
+  constexpr int NWW = CW / 32;               // worker warps
   constexpr int TK = 1 << (MBK - 1);
   constexpr int TV = 1 << (BV - 1);
   constexpr int N = tc_n(G);
@@ -294,12 +312,13 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
   constexpr int KTOT = KM + (QJL ? TD : 0);
   constexpr int BKB = N * KTOT;
   constexpr int BKC = BKB + G * 16;
+  constexpr int NKT = TK + (QJL ? 1 : 0);   // key terms: TK Walsh terms + the sign plane
   // Tensor memory: the key phase and the value phase of a unit never overlap
   // in time, so their regions share columns.
-  //   key phase:   DK [0, 2N)   AK [32, 32 + 32 (TK + QJL))
+  //   key phase:   DK[b] [32 b, 32 b + 2N)   AK[b] [64 + 32 NKT b, 64 + 32 NKT (b + 1))
   //   value phase: AV [0, 16 TV) (two buffers)   DV [16 TV, 16 TV + N TV)
   constexpr int C_DK = 0;
-  constexpr int C_AK = 32;
+  constexpr int C_AK = 64;
   constexpr int C_AV = 0;
   constexpr int C_DV = 2 * TV * 8;
   constexpr int USED = tc_tmem_cols(G, MBK, BV, QJL);
@@ -309,13 +328,17 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
   constexpr uint32_t IDESC = sm100::idesc_i8(128, N);
 
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t mb_load[2], mb_k, mb_v[2];
+  __shared__ __align__(8) uint64_t mb_load[2], mb_k[2], mb_v[2], ak_full[2], av_full[2];
   __shared__ uint32_t tmem_s;
-  __shared__ float redf[TCT / 32][2 * G + 1];
-  __shared__ long long redi[TCT / 32][G];
+  __shared__ float redf[NWW][2 * G + 1];
+  __shared__ long long redi[NWW][G];
+  __shared__ float part[G][TD];
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wq = warp & 3;            // TMEM lane quarter
+  const int slice = warp >> 2;        // 0 or 1
+  const int lt = tid & 127;           // TMEM lane = row (keys) or coordinate (values)
   const int sub = a.sub;
   const TcLayout L = tc_layout(sub, PK, BV, G, N, BKC);
   int8_t *bvs = reinterpret_cast<int8_t *>(smem + L.o_bv);
@@ -325,9 +348,14 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
   if (tid == 0) {
     sm100::mbar_init(&mb_load[0], 1);
     sm100::mbar_init(&mb_load[1], 1);
-    sm100::mbar_init(&mb_k, 1);
+    sm100::mbar_init(&mb_k[0], 1);
+    sm100::mbar_init(&mb_k[1], 1);
     sm100::mbar_init(&mb_v[0], 1);
     sm100::mbar_init(&mb_v[1], 1);
+    sm100::mbar_init(&ak_full[0], NWW);
+    sm100::mbar_init(&ak_full[1], NWW);
+    sm100::mbar_init(&av_full[0], NWW);
+    sm100::mbar_init(&av_full[1], NWW);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -336,19 +364,80 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
   sm100::fence_after_sync();
   const uint32_t tm = tmem_s;
 
+  if (warp == NWW) {
+    // ---------------- MMA warp: walks the same units as the workers
+    if (lane == 0) {
+      int cit = blockIdx.x, cr0 = -1, u = 0;
+      uint32_t akph = 0, avph = 0;
+      bool have = tc_next(a, cit, cr0);
+      bool ok = true;
+      while (have && ok) {
+        int nit = cit, nr0 = cr0 + sub;
+        const bool nhave = tc_next(a, nit, nr0);
+        uint8_t *ub = smem + (u & 1) * L.ubytes;
+        const int b = cit / (a.Hkv * a.splits), sp = cit % a.splits;
+        const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
+        const int nvalid = min(sub, c1 - cr0);
+        const uint32_t bk_addr = sm100::smem_addr(ub + L.o_bk);
+        const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
+        for (int j = 0; j < ntile && ok; ++j) {
+          const int kb = j & 1;
+          ok = sm100::mbar_wait(&ak_full[kb], (akph >> kb) & 1);
+          akph ^= 1u << kb;
+          if (!ok) break;
+          sm100::fence_after_sync();
+          const uint32_t ak = tm + C_AK + kb * 32 * NKT, dk = tm + C_DK + kb * 32;
+#pragma unroll
+          for (int s = 0; s < TK * 4; ++s)
+            sm100::mma_i8_ts(dk, ak + s * 8, sm100::smem_desc(bk_addr + s * 2 * N * 16, N * 16, 128),
+                             IDESC, s > 0);
+          if (QJL) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+              sm100::mma_i8_ts(dk + N, ak + TK * 32 + s * 8,
+                               sm100::smem_desc(bk_addr + N * KM + s * 2 * N * 16, N * 16, 128),
+                               IDESC, s > 0);
+          }
+          sm100::mma_commit(&mb_k[kb]);
+        }
+        const uint32_t bv_addr = sm100::smem_addr(bvs);
+        for (int g = 0; g < ngroups && ok; ++g) {
+          const int ab = g & 1;
+          ok = sm100::mbar_wait(&av_full[ab], (avph >> ab) & 1);
+          avph ^= 1u << ab;
+          if (!ok) break;
+          sm100::fence_after_sync();
+          const uint64_t bd = sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128);
+#pragma unroll
+          for (int ti = 0; ti < TV; ++ti)
+            sm100::mma_i8_ts(tm + C_DV + ti * N, tm + C_AV + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
+          sm100::mma_commit(&mb_v[ab]);
+        }
+        cit = nit;
+        cr0 = nr0;
+        have = nhave;
+        ++u;
+      }
+      // a wait that gave up leaves the workers to time out on the commits
+      // they expect and take their own abort path
+    }
+    __syncwarp();
+  } else {
+  // ---------------- workers
   // empty chunks (beyond a batch's length) merge with weight zero
   const int items = a.B * a.Hkv * a.splits;
   for (int it = blockIdx.x; it < items; it += gridDim.x) {
     const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv, sp = it % a.splits;
     if (sp * a.chunk < tc_len(a, b)) continue;
-    for (int h = 0; h < G; ++h) {
-      const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-      a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
-      if (tid == 0) {
-        a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
-        a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
+    if (tid < TD)
+      for (int h = 0; h < G; ++h) {
+        const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
+        a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
+        if (tid == 0) {
+          a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
+          a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
+        }
       }
-    }
   }
 
   auto issue = [&](int buf, int it, int r0) {
@@ -366,17 +455,30 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     sm100::bulk_g2s(u + L.o_vn, a.vnorm + bh * a.rows_cap + r0, b_vn, &mb_load[buf]);
     sm100::bulk_g2s(u + L.o_bk, a.bk + bh * a.bk_stride, b_bk, &mb_load[buf]);
   };
+  // worker-only barrier (named barrier 1 over the 256 worker threads)
+  auto wsync = [&]() { sm100::named_sync(1, CW); };
   auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
-    if (!sm100::mbar_wait(bar, parity)) abort_s = 1;
-    __syncthreads();
+    if (lane == 0 && !sm100::mbar_wait(bar, parity)) abort_s = 1;
+    wsync();
     return abort_s == 0;
+  };
+  auto sync_tc = [&]() {
+    sm100::fence_before_sync();
+    wsync();
+    sm100::fence_after_sync();
+  };
+  // this warp's tcgen05.st are complete: publish them to the MMA warp
+  auto publish = [&](uint64_t *bar) {
+    sm100::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(bar);
   };
 
   int cit = blockIdx.x, cr0 = -1;
   bool have = tc_next(a, cit, cr0);
   if (have && tid == 0) issue(0, cit, cr0);
   int inflight = have ? 0 : -1;   // buffer whose bulk copies were issued, not yet waited
-  // barrier parities: bit ab of vph / lph is the parity to wait for next
+  // barrier parities: bit b of kph / vph / lph is the parity to wait for next on buffer b
   uint32_t kph = 0, vph = 0, lph = 0;
   float o[G], m_run[G], l_run[G];
   int u = 0;
@@ -409,14 +511,9 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     const uint32_t bk_addr = sm100::smem_addr(ub + L.o_bk);
 
     // ---------------- keys: logits of the G heads, 128 rows per tile
-    float mloc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
-    const int ntile = (nvalid + 127) / 128;
-    bool ok = true;
-    for (int j = 0; j < ntile && ok; ++j) {
-      const int rl = j * 128 + tid;
-      const bool valid = rl < nvalid;
+    // expand tile j's bit planes (this slice's terms) into AK[kb]
+    auto expand_keys = [&](int j, int kb) {
+      const int rl = j * 128 + lt;
       uint32_t pw[PK][TNW];
       const uint4 *kr = reinterpret_cast<const uint4 *>(ub + rl * PK * 16);
 #pragma unroll
@@ -427,90 +524,90 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
         pw[p][2] = v.z;
         pw[p][3] = v.w;
       }
-      const uint32_t sc = reinterpret_cast<const uint32_t *>(ub + L.o_ks)[rl];
+      const uint32_t ak = tm + C_AK + kb * 32 * NKT;
 #pragma unroll
-      for (int ti = 0; ti < TK; ++ti) {
-        const int mask = odd_mask(MBK, ti);
+      for (int t = 0; t < NKT; ++t) {
+        if ((t & 1) != slice) continue;
 #pragma unroll
         for (int w = 0; w < TNW; ++w) {
           uint32_t x = 0;
+          if (t < TK) {
+            const int mask = odd_mask(MBK, t);
 #pragma unroll
-          for (int p = 0; p < MBK; ++p)
-            if ((mask >> p) & 1) x ^= pw[p][w];
+            for (int p = 0; p < MBK; ++p)
+              if ((mask >> p) & 1) x ^= pw[p][w];
+          } else {
+            x = pw[PK - 1][w];
+          }
           uint32_t r8[8];
 #pragma unroll
           for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-          sm100::tmem_st8(sm100::tmem_lane(tm + C_AK + ti * 32 + w * 8, warp), r8);
-        }
-      }
-      if (QJL) {
-#pragma unroll
-        for (int w = 0; w < TNW; ++w) {
-          uint32_t r8[8];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) r8[r] = pw[PK - 1][w] & (0x01010101u << r);
-          sm100::tmem_st8(sm100::tmem_lane(tm + C_AK + TK * 32 + w * 8, warp), r8);
+          sm100::tmem_st8(sm100::tmem_lane(ak + t * 32 + w * 8, wq), r8);
         }
       }
       sm100::wait_st();
-      sm100::fence_before_sync();
-      __syncthreads();
-      sm100::fence_after_sync();
-      if (tid == 0) {
+    };
+    float mloc[G];
 #pragma unroll
-        for (int s = 0; s < TK * 4; ++s)
-          sm100::mma_i8_ts(tm + C_DK, tm + C_AK + s * 8,
-                           sm100::smem_desc(bk_addr + s * 2 * N * 16, N * 16, 128), IDESC, s > 0);
-        if (QJL) {
-#pragma unroll
-          for (int s = 0; s < 4; ++s)
-            sm100::mma_i8_ts(tm + C_DK + N, tm + C_AK + TK * 32 + s * 8,
-                             sm100::smem_desc(bk_addr + N * KM + s * 2 * N * 16, N * 16, 128),
-                             IDESC, s > 0);
-        }
-        sm100::mma_commit(&mb_k);
+    for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
+    const int ntile = (nvalid + 127) / 128;
+    bool ok = true;
+    expand_keys(0, 0);
+    publish(&ak_full[0]);
+    for (int j = 0; j < ntile; ++j) {
+      const int kb = j & 1;
+      if (j + 1 < ntile) {
+        // AK[kb ^ 1] and DK[kb ^ 1] were released by tile j - 1 (waited, read)
+        expand_keys(j + 1, kb ^ 1);
+        publish(&ak_full[kb ^ 1]);
       }
-      ok = wait_all(&mb_k, kph);
-      kph ^= 1;
+      ok = wait_all(&mb_k[kb], (kph >> kb) & 1);
+      kph ^= 1u << kb;
       if (!ok) break;
       sm100::fence_after_sync();
-      uint32_t dk[2 * N];
-      if (N == 16) {
-        uint32_t t0[16], t1[16];
-        sm100::tmem_ld16(sm100::tmem_lane(tm + C_DK, warp), t0);
-        sm100::tmem_ld16(sm100::tmem_lane(tm + C_DK + 16, warp), t1);
-        sm100::wait_ld();
+      if (slice == 0) {
+        const int rl = j * 128 + lt;
+        const bool valid = rl < nvalid;
+        uint32_t dk[2 * N];
+        const uint32_t dka = tm + C_DK + kb * 32;
+        if (N == 16) {
+          uint32_t t0[16], t1[16];
+          sm100::tmem_ld16(sm100::tmem_lane(dka, wq), t0);
+          sm100::tmem_ld16(sm100::tmem_lane(dka + 16, wq), t1);
+          sm100::wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          dk[c] = t0[c];
-          dk[N + c] = t1[c];
-        }
-      } else {
-        uint32_t t0[8], t1[8];
-        sm100::tmem_ld8(sm100::tmem_lane(tm + C_DK, warp), t0);
-        sm100::tmem_ld8(sm100::tmem_lane(tm + C_DK + N, warp), t1);
-        sm100::wait_ld();
+          for (int c = 0; c < 16; ++c) {
+            dk[c] = t0[c];
+            dk[N + c] = t1[c];
+          }
+        } else {
+          uint32_t t0[8], t1[8];
+          sm100::tmem_ld8(sm100::tmem_lane(dka, wq), t0);
+          sm100::tmem_ld8(sm100::tmem_lane(dka + N, wq), t1);
+          sm100::wait_ld();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          dk[c] = t0[c];
-          dk[N + c] = t1[c];
+          for (int c = 0; c < 8; ++c) {
+            dk[c] = t0[c];
+            dk[N + c] = t1[c];
+          }
         }
-      }
-      const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
-      const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+        const uint32_t sc = reinterpret_cast<const uint32_t *>(ub + L.o_ks)[rl];
+        const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+        const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float dm = comb_limbs(dk + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
-        float est = dm;
-        if (QJL) {
-          const float dj = comb_limbs(dk + N + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
-          est = fmaf(a.qjl_coef * rho, dj, dm);
+        for (int h = 0; h < G; ++h) {
+          const float dm = comb_limbs(dk + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
+          float est = dm;
+          if (QJL) {
+            const float dj = comb_limbs(dk + N + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
+            est = fmaf(a.qjl_coef * rho, dj, dm);
+          }
+          const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
+          lg[rl * G + h] = l;
+          mloc[h] = fmaxf(mloc[h], l);
+          if (a.logits && valid)
+            a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
         }
-        const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
-        lg[rl * G + h] = l;
-        mloc[h] = fmaxf(mloc[h], l);
-        if (a.logits && valid)
-          a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
       }
     }
     if (!ok) break;
@@ -521,13 +618,13 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
       const float m = tq_warp_max(mloc[h]);
       if (lane == 0) redf[warp][h] = m;
     }
-    __syncthreads();
+    sync_tc();   // the key epilogue's TMEM reads are complete before any value-phase store
     float mnew[G], corr[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float m = redf[0][h];
 #pragma unroll
-      for (int w = 1; w < TCT / 32; ++w) m = fmaxf(m, redf[w][h]);
+      for (int w = 1; w < NWW; ++w) m = fmaxf(m, redf[w][h]);
       mnew[h] = fmaxf(m_run[h], m);
       corr[h] = __expf(m_run[h] - mnew[h]);
     }
@@ -535,7 +632,7 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     float lsum[G], numax = 0.f;
 #pragma unroll
     for (int h = 0; h < G; ++h) lsum[h] = 0.f;
-    for (int rl = tid; rl < nvalid; rl += TCT) {
+    for (int rl = tid; rl < nvalid; rl += CW) {
       numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -544,7 +641,7 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
         lsum[h] += p;
       }
     }
-    __syncthreads();
+    wsync();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float s = tq_warp_sum(lsum[h]);
@@ -554,17 +651,17 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
       const float m = tq_warp_max(numax);
       if (lane == 0) redf[warp][2 * G] = m;
     }
-    __syncthreads();
+    wsync();
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float s = 0.f;
 #pragma unroll
-      for (int w = 0; w < TCT / 32; ++w) s += redf[w][h];
+      for (int w = 0; w < NWW; ++w) s += redf[w][h];
       lsum[h] = s;
     }
     float nmax = redf[0][2 * G];
 #pragma unroll
-    for (int w = 1; w < TCT / 32; ++w) nmax = fmaxf(nmax, redf[w][2 * G]);
+    for (int w = 1; w < NWW; ++w) nmax = fmaxf(nmax, redf[w][2 * G]);
     const float FV = pow2_scale(nmax);
     const float invFV = 1.0f / (128.0f * FV);
 
@@ -573,7 +670,7 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     long long wsum[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) wsum[h] = 0;
-    for (int rl = tid; rl < ngroups * 32; rl += TCT) {
+    for (int rl = tid; rl < ngroups * 32; rl += CW) {
       const int g = rl >> 5, jj = rl & 31, r = jj & 7, nb = jj >> 3;
       const int k = 4 * r + nb;
       int8_t *dst = bvs + g * N * 32;
@@ -596,13 +693,13 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
       if (lane == 0) redi[warp][h] = s;
     }
     sm100::fence_async_smem();
-    __syncthreads();
+    wsync();
     float wtot[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       long long s = 0;
 #pragma unroll
-      for (int w = 0; w < TCT / 32; ++w) s += redi[w][h];
+      for (int w = 0; w < NWW; ++w) s += redi[w][h];
       wtot[h] = static_cast<float>(s) / FV;
       o[h] *= corr[h];
       l_run[h] = l_run[h] * corr[h] + lsum[h];
@@ -611,7 +708,6 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
 
     // ---------------- values: rotated-domain sums, 32 tokens per MMA step
     const uint32_t *vc = reinterpret_cast<const uint32_t *>(ub + L.o_vc);
-    const uint32_t bv_addr = sm100::smem_addr(bvs);
     for (int g = 0; g < ngroups && ok; ++g) {
       const int ab = g & 1;
       if (g >= 2) {  // buffer ab was last fed to the MMAs of group g - 2
@@ -621,9 +717,10 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
       }
       uint32_t pw[BV];
 #pragma unroll
-      for (int p = 0; p < BV; ++p) pw[p] = vc[(g * BV + p) * TD + tid];
+      for (int p = 0; p < BV; ++p) pw[p] = vc[(g * BV + p) * TD + lt];
 #pragma unroll
       for (int ti = 0; ti < TV; ++ti) {
+        if ((ti & 1) != slice) continue;
         const int mask = odd_mask(BV, ti);
         uint32_t x = 0;
 #pragma unroll
@@ -632,19 +729,10 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
         uint32_t r8[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-        sm100::tmem_st8(sm100::tmem_lane(tm + C_AV + ab * TV * 8 + ti * 8, warp), r8);
+        sm100::tmem_st8(sm100::tmem_lane(tm + C_AV + ab * TV * 8 + ti * 8, wq), r8);
       }
       sm100::wait_st();
-      sm100::fence_before_sync();
-      __syncthreads();
-      sm100::fence_after_sync();
-      if (tid == 0) {
-        const uint64_t bd = sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128);
-#pragma unroll
-        for (int ti = 0; ti < TV; ++ti)
-          sm100::mma_i8_ts(tm + C_DV + ti * N, tm + C_AV + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
-        sm100::mma_commit(&mb_v[ab]);
-      }
+      publish(&av_full[ab]);
     }
     // the last one or two groups' MMAs are still outstanding
     for (int g = ngroups > 2 ? ngroups - 2 : 0; g < ngroups && ok; ++g) {
@@ -654,23 +742,25 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     }
     if (!ok) break;
     sm100::fence_after_sync();
-    // read the per-term accumulators of coordinate `tid` and fold the terms
+    // each slice folds its Walsh terms for coordinate lt; slice 1 hands its
+    // partial sums to slice 0, which keeps the running output
     {
       float acc[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll
       for (int ti = 0; ti < TV; ++ti) {
+        if ((ti & 1) != slice) continue;
         uint32_t dv[N];
         if (N == 16) {
           uint32_t t0[16];
-          sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, warp), t0);
+          sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
           sm100::wait_ld();
 #pragma unroll
           for (int c = 0; c < 16; ++c) dv[c] = t0[c];
         } else {
           uint32_t t0[8];
-          sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, warp), t0);
+          sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
           sm100::wait_ld();
 #pragma unroll
           for (int c = 0; c < 8; ++c) dv[c] = t0[c];
@@ -678,23 +768,28 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
 #pragma unroll
         for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
       }
+      if (slice == 1) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) o[h] += acc[h] * invFV - a.wv_sum * wtot[h];
+        for (int h = 0; h < G; ++h) part[h][lt] = acc[h];
+      }
+      wsync();
+      if (slice == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] += (acc[h] + part[h][lt]) * invFV - a.wv_sum * wtot[h];
+      }
     }
-    if (cr0 + sub >= c1) {
+    if (cr0 + sub >= c1 && slice == 0) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-        a.po[(hq * a.splits + sp) * TD + tid] = o[h];
+        a.po[(hq * a.splits + sp) * TD + lt] = o[h];
         if (tid == 0) {
           a.pml[(hq * a.splits + sp) * 2] = m_run[h];
           a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
         }
       }
     }
-    sm100::fence_before_sync();
-    __syncthreads();
-    sm100::fence_after_sync();
+    sync_tc();
     cit = nit;
     cr0 = nr0;
     have = nhave;
@@ -704,11 +799,13 @@ __global__ void __launch_bounds__(TCT) tc_chunk_kernel(TcArgs a) {
     // a bounded wait gave up: let this CTA's own outstanding copies and MMAs
     // land (again bounded) before its shared and tensor memory are released
     if (inflight >= 0) sm100::mbar_wait(&mb_load[inflight], (lph >> inflight) & 1, 1u << 20);
-    sm100::mbar_wait(&mb_k, kph, 1u << 20);
+    sm100::mbar_wait(&mb_k[0], kph & 1, 1u << 20);
+    sm100::mbar_wait(&mb_k[1], (kph >> 1) & 1, 1u << 20);
     sm100::mbar_wait(&mb_v[0], vph & 1, 1u << 20);
     sm100::mbar_wait(&mb_v[1], (vph >> 1) & 1, 1u << 20);
     if (tid == 0 && a.err) atomicExch(a.err, 1u);
   }
+  }  // workers
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
@@ -757,7 +854,7 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
     attr_done[dev] = true;
   }
   int occ = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tc_chunk_kernel<G, MBK, BV, QJL>, TCT, smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tc_chunk_kernel<G, MBK, BV, QJL>, CT, smem);
   if (occ < 1) occ = 1;
   if (occ < per_sm) per_sm = occ;
   tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, QJL ? TD * TD * 2 : 0, stream>>>(a);
@@ -773,7 +870,7 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
     if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
     cudaEventRecordWithFlags(ev0, stream, ev_flags);
   }
-  tc_chunk_kernel<G, MBK, BV, QJL><<<grid, TCT, smem, stream>>>(a);
+  tc_chunk_kernel<G, MBK, BV, QJL><<<grid, CT, smem, stream>>>(a);
   if (int e = tq_check_launch("tc_chunk_kernel")) return e;
   if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
   tq_count_launch(2);
