@@ -212,7 +212,7 @@ int tq_attention_bidir(const tq_codec *codec, const void *q, int dtype, int B, i
  * TurboQuant ...", "Velocidad y eficiencia de indexacion": the codes are
  * data-oblivious, so indexing is a single encode pass with no training;
  * "Eliminacion del sesgo interno del producto": the prod estimator of <q, x>).
- * The codec must have d = 1536 and QJL keys with key MSE bits 1..4.  For
+ * The codec must have d = 1536 and QJL keys with key MSE bits 1..3.  For
  * d = 1536 the rotation is Pi = (H_12 kron H_128) diag(D) / sqrt(1536), H_12
  * the Paley type-I matrix of GF(11) (H = I + [[0, 1^T], [-1, Q]],
  * Q[i][j] = chi(j - i)), H_128 Sylvester-ordered.
@@ -235,8 +235,10 @@ int tq_attention_bidir(const tq_codec *codec, const void *q, int dtype, int B, i
  *   q        device fp32 [nq][1536], 16-byte aligned (unit norm is not required).
  *   idx      device int32 [nq][k];  score  device fp32 [nq][k].
  *   1 <= k <= min(16, n);  workspace >= tq_scan_workspace(...) bytes, 16-byte aligned.
- * Scores are evaluated in fp32 on the tensor cores (bf16 hi + lo operands);
- * rows whose scores differ by less than ~1e-5 relative may swap places.
+ * Scores come from one fp16 product per element on the tensor cores (rows
+ * [c[idx] | rho (2 sigma - 1)] against the query scaled by a power of two),
+ * accumulated in fp32: about 1e-5 |q| absolute error for unit rows, so rows
+ * whose scores differ by less than that may swap places.
  * ------------------------------------------------------------------------ */
 int tq_index_workspace(const tq_codec *codec, int64_t n, size_t *bytes);
 int tq_index_build(const tq_codec *codec, const float *x, int64_t n, uint8_t *kcode,

@@ -22,6 +22,7 @@
 //                      fp32 in tensor memory, sign bits -> the QJL plane.
 #include <math_constants.h>
 
+#include <cstring>
 #include <vector>
 
 #include "tq_device.cuh"
@@ -162,8 +163,6 @@ struct GemmArgs {
   uint8_t *plane;        // MODE 0: bit plane base, row stride plane_stride bytes
   int64_t plane_stride;
   float *out;            // MODE 1: [M][N]
-  uint16_t *out_hl;      // MODE 2: [M][2N] bf16 hi | lo of scale * value
-  float scale;
   uint32_t *status;
 };
 
@@ -280,18 +279,6 @@ __global__ void __launch_bounds__(128, 1) ix_gemm_kernel(GemmArgs g) {
             word |= (__uint_as_float(z1[c]) >= 0.f ? 1u : 0u) << (16 + c);
           }
           reinterpret_cast<uint32_t *>(g.plane + row * g.plane_stride)[(n0 + c0) >> 5] = word;
-        } else if (MODE == 2) {
-          uint16_t *o = g.out_hl + row * 2 * g.N + n0 + c0;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v = g.scale * __uint_as_float(c < 16 ? z0[c] : z1[c - 16]);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-            if (n0 + c0 + c < g.N) {
-              o[c] = __bfloat16_as_ushort(hi);
-              o[g.N + c] = __bfloat16_as_ushort(lo);
-            }
-          }
         } else {
           float *o = g.out + row * g.N + n0 + c0;
 #pragma unroll
@@ -354,201 +341,310 @@ __global__ void __launch_bounds__(256) ix_qrot_kernel(QrotArgs a) {
 
 // ---------------------------------------------------------------------------
 // Scan: scores s_ij = nu_j (<q'_i, c[idx_j]> + sqrt(pi/2)/d rho_j <q''_i, 2 sigma_j - 1>)
-// for 128 queries (TMEM lane = query) against 128-row database tiles, K = 1536
-// in chunks of 64.  Database codes are dequantized per chunk into bf16 tiles
-// c_hi, c_lo (c = c_hi + c_lo to ~2^-17) and s = +-1 (exact); the queries'
-// q', q'' come as bf16 hi | lo.  Two fp32 accumulators:
-//   D_m = q'_hi c_hi + q'_hi c_lo + q'_lo c_hi,   D_s = q''_hi s + q''_lo s.
-// Each query lane keeps its top-k in registers over the CTA's tile range.
+// as ONE fp16 product per element over K = 2d:
+//   A (database row j, in tensor memory)  = [ c[idx_j] | rho_j (2 sigma_j - 1) ]
+//   B (query i, in shared memory)         = 2^e_i [ q'_i | sqrt(pi/2)/d q''_i ]
+// with K ordered in 48 chunks of 64 = [32 MSE coordinates | the same 32 sign
+// coordinates].  A row's codes are dequantized into TMEM by the worker lane
+// that owns the row (tcgen05.st), the query chunks stream into shared memory
+// by cp.async.bulk, and one warp issues tcgen05.mma kind::f16 (M = 128 rows,
+// N = 256 queries) into fp32 accumulators.  Per-element rounding: centroids
+// and rho are fp16 (2^-11 relative), queries fp16 after the power-of-two
+// scale; the score error is ~1e-5 of |q| for unit data.
+// Epilogue: the 128 x 256 scores go through shared memory (two passes of 128
+// queries) so each worker thread walks 64 rows of one query and keeps a
+// running top-k in registers; a merge kernel combines the per-CTA lists.
 // ---------------------------------------------------------------------------
-constexpr int SQ = 128, SR = 128, SK = 64;
-constexpr int SKMAX = 16;                       // largest k of the top-k
+constexpr int QN = 256;                       // queries per CTA (MMA N)
+constexpr int RM = 128;                       // database rows per tile (MMA M)
+constexpr int XCH = XD / 32;                  // K chunks
+constexpr int NAS = 4;                        // pipeline stages (A in TMEM, B in smem)
+constexpr uint32_t QCH_BYTES = QN * 64 * 2;   // one query chunk, fp16
+constexpr int SCW = 8;                        // worker warps
+constexpr int SCT = (SCW + 1) * 32;           // + the MMA warp
+constexpr int SBP = RM + 1;                   // padded stride of the score transpose
+constexpr int SKMAX = 16;                     // largest k of the top-k
+constexpr uint32_t SC_B_OFF = 0;
+constexpr uint32_t SC_SB_OFF = NAS * QCH_BYTES;
+constexpr uint32_t SC_LUT_OFF = SC_SB_OFF + 128 * SBP * 4;
+constexpr uint32_t SC_SMEM = SC_LUT_OFF + 64 * 32 * 4;
 
-struct ScanArgs {
-  const uint16_t *q1hl;   // [nq][2 XD]
-  const uint16_t *q2hl;   // [nq][2 XD]
-  const uint8_t *kcode;
-  const uint16_t *kscale;
+// Element offset (16-bit units) of (n, k) in a K-major, no-swizzle operand of QN rows.
+__host__ __device__ constexpr uint32_t qop_off(int n, int k) {
+  return ((k >> 3) * (QN * 16) + (n >> 3) * 128 + (n & 7) * 16) / 2 + (k & 7);
+}
+
+struct QpackArgs {
+  const float *q1;      // [nq][XD] q' = Pi q
+  const float *q2;      // [nq][XD] q'' = S q'
+  int nq;
+  float coef;           // sqrt(pi/2) / d
+  uint16_t *qop;        // [ceil(nq / QN)][XCH][QN * 64] fp16
+  float *qinv;          // [nq] 2^-e
+};
+
+// One warp per (padded) query: power-of-two scale putting max |B| in
+// [2^14, 2^15), then the fp16 operand in chunk order.
+__global__ void __launch_bounds__(256) ix_qpack_kernel(QpackArgs a) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = blockIdx.x * 8 + warp;
+  const int nqp = (a.nq + QN - 1) / QN * QN;
+  if (q >= nqp) return;
+  const bool valid = q < a.nq;
+  const float *s1 = a.q1 + static_cast<int64_t>(valid ? q : 0) * XD;
+  const float *s2 = a.q2 + static_cast<int64_t>(valid ? q : 0) * XD;
+  float mx = 0.f;
+  if (valid)
+    for (int i = lane; i < XD; i += 32) mx = fmaxf(mx, fmaxf(fabsf(s1[i]), a.coef * fabsf(s2[i])));
+  mx = tq_warp_max(mx);
+  int e2 = 0;
+  if (mx > 0.f) frexpf(mx, &e2);            // mx in [2^(e2-1), 2^e2)
+  const float sc = mx > 0.f ? ldexpf(1.f, 15 - e2) : 1.f;
+  if (lane == 0 && valid) a.qinv[q] = mx > 0.f ? ldexpf(1.f, e2 - 15) : 1.f;
+  uint16_t *dst = a.qop + static_cast<int64_t>(q / QN) * XCH * (QN * 64);
+  const int n = q % QN;
+  for (int c = 0; c < XCH; ++c) {
+    const int coord = 32 * c + lane;
+    const float v1 = valid ? s1[coord] * sc : 0.f;
+    const float v2 = valid ? a.coef * s2[coord] * sc : 0.f;
+    dst[c * (QN * 64) + qop_off(n, lane)] = __half_as_ushort(__float2half_rn(v1));
+    dst[c * (QN * 64) + qop_off(n, 32 + lane)] = __half_as_ushort(__float2half_rn(v2));
+  }
+}
+
+struct Scan2Args {
+  const uint8_t *kcode;   // [n][planes][XD / 8]
+  const uint16_t *kscale; // [n][2]
   int64_t n;
-  int nq, k;
+  const uint16_t *qop;
+  const float *qinv;
+  int nq;
   int tiles_per_cta;
-  float coef;
-  float ck[TQ_MAX_LEVELS];
-  int mbk;
-  float *cand_s;          // [nq][grid.y][k]
+  int mbk;                // MSE planes (1..3)
+  uint32_t lut[64];       // half2 (c[m_even], c[m_odd]); index bits (b0e b0o b1e b1o b2e b2o)
+  float *cand_s;          // [nq][lists][k]
   int32_t *cand_i;
+  int k;
   uint32_t *err;
 };
 
-__device__ __forceinline__ int kmaj_off(int row, int k, int R) {   // bf16 element offset in bytes
-  const int kb = 2 * k;
-  return (kb >> 4) * (R * 16) + (row >> 3) * 128 + (row & 7) * 16 + (kb & 15);
-}
-
-__global__ void __launch_bounds__(128, 1) ix_scan_kernel(ScanArgs a) {
-  constexpr uint32_t QB = SQ * SK * 2;         // one query operand chunk
-  constexpr uint32_t RB = SR * SK * 2;         // one database operand chunk
-  extern __shared__ __align__(128) float ssm[];
-  uint8_t *base = reinterpret_cast<uint8_t *>(ssm);
-  uint8_t *q1h = base, *q1l = q1h + QB, *q2h = q1l + QB, *q2l = q2h + QB;
-  uint8_t *chi = q2l + QB, *clo = chi + RB, *sgn = clo + RB;
-  __shared__ float cks[TQ_MAX_LEVELS];
-  __shared__ float nus[SR], rhos[SR];
-  __shared__ __align__(8) uint64_t mb;
+__global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
+  extern __shared__ __align__(1024) uint8_t ssm[];
+  uint8_t *bst = ssm + SC_B_OFF;
+  float *sb = reinterpret_cast<float *>(ssm + SC_SB_OFF);
+  uint32_t *lut = reinterpret_cast<uint32_t *>(ssm + SC_LUT_OFF);
+  __shared__ __align__(8) uint64_t a_full[NAS], b_full[NAS], done[NAS], acc_full, acc_free;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int qb = blockIdx.x;
-  if (tid < TQ_MAX_LEVELS) cks[tid] = a.ck[tid];
-  if (warp == 0) sm100::tmem_alloc(&tmem_s, 256);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < 64 * 32; e += SCT) lut[e] = a.lut[e >> 5];
+  if (warp == 0) sm100::tmem_alloc(&tmem_s, 512);
   if (tid == 0) {
-    sm100::mbar_init(&mb, 1);
+    for (int s = 0; s < NAS; ++s) {
+      sm100::mbar_init(&a_full[s], 4);
+      sm100::mbar_init(&b_full[s], 1);
+      sm100::mbar_init(&done[s], 1);
+    }
+    sm100::mbar_init(&acc_full, 1);
+    sm100::mbar_init(&acc_free, SCW);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  const uint32_t tm = tmem_s, tDm = tm, tDs = tm + SR;
-  const int planes = a.mbk + 1;
-  const int q = qb * SQ + tid;
-  float ts[SKMAX];
-  int ti[SKMAX];
-#pragma unroll
-  for (int e = 0; e < SKMAX; ++e) {
-    ts[e] = -CUDART_INF_F;
-    ti[e] = 0x7fffffff;
-  }
-  uint32_t ph = 0;
-  const int64_t ntiles = (a.n + SR - 1) / SR;
+  const uint32_t tm = tmem_s;            // D: columns [0, 256); A stages: [256, 256 + 32 NAS)
+  const int64_t ntiles = (a.n + RM - 1) / RM;
   const int64_t t_begin = static_cast<int64_t>(blockIdx.y) * a.tiles_per_cta;
   const int64_t t_end = t_begin + a.tiles_per_cta < ntiles ? t_begin + a.tiles_per_cta : ntiles;
-  const uint32_t idesc = sm100::idesc_bf16(SQ, SR);
-  for (int64_t t = t_begin; t < t_end && !abort_s; ++t) {
-    const int64_t r0 = t * SR;
-    {
-      const int64_t r = r0 + tid < a.n ? r0 + tid : a.n - 1;
-      const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale)[r];
-      nus[tid] = r0 + tid < a.n ? tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu)) : 0.f;
-      rhos[tid] = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-    }
-    for (int kc = 0; kc < XD / SK; ++kc) {
-      const int k0 = kc * SK;
-      // query operand chunks (rows past nq repeat the last query)
-      const int qq = q < a.nq ? q : a.nq - 1;
-      for (int seg = 0; seg < 8; ++seg) {
-        const int off = seg * (SQ * 16) + (tid >> 3) * 128 + (tid & 7) * 16;
-        cp_async16(q1h + off, a.q1hl + static_cast<int64_t>(qq) * 2 * XD + k0 + seg * 8);
-        cp_async16(q1l + off, a.q1hl + static_cast<int64_t>(qq) * 2 * XD + XD + k0 + seg * 8);
-        cp_async16(q2h + off, a.q2hl + static_cast<int64_t>(qq) * 2 * XD + k0 + seg * 8);
-        cp_async16(q2l + off, a.q2hl + static_cast<int64_t>(qq) * 2 * XD + XD + k0 + seg * 8);
-      }
-      cp_commit();
-      // database operand: thread tid dequantizes row r0 + tid, coordinates k0 .. k0+63
-      {
-        const int64_t r = r0 + tid < a.n ? r0 + tid : a.n - 1;
-        const uint32_t *kr = reinterpret_cast<const uint32_t *>(a.kcode + r * planes * (XD / 8));
-        uint32_t pw[5][2];
-#pragma unroll
-        for (int p = 0; p < 5; ++p)
-#pragma unroll
-          for (int w = 0; w < 2; ++w) pw[p][w] = p < planes ? kr[p * XW + (k0 >> 5) + w] : 0u;
-#pragma unroll
-        for (int w = 0; w < 2; ++w)
-#pragma unroll 8
-          for (int bit = 0; bit < 32; ++bit) {
-            int idx = 0;
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-              if (p < a.mbk) idx |= ((pw[p][w] >> bit) & 1) << p;
-            const float c = cks[idx];
-            const __nv_bfloat16 h = __float2bfloat16_rn(c);
-            const __nv_bfloat16 l = __float2bfloat16_rn(c - __bfloat162float(h));
-            const int off = kmaj_off(tid, 32 * w + bit, SR);
-            *reinterpret_cast<__nv_bfloat16 *>(chi + off) = h;
-            *reinterpret_cast<__nv_bfloat16 *>(clo + off) = l;
-            const bool sb = (pw[planes - 1][w] >> bit) & 1;
-            *reinterpret_cast<uint16_t *>(sgn + off) = sb ? 0x3F80u : 0xBF80u;   // +-1 in bf16
-          }
-      }
-      cp_wait<0>();
-      sm100::fence_async_smem();
-      sm100::fence_before_sync();
-      __syncthreads();
-      sm100::fence_after_sync();
-      if (tid == 0) {
-        const uint32_t aq1h = sm100::smem_addr(q1h), aq1l = sm100::smem_addr(q1l);
-        const uint32_t aq2h = sm100::smem_addr(q2h), aq2l = sm100::smem_addr(q2l);
-        const uint32_t ach = sm100::smem_addr(chi), acl = sm100::smem_addr(clo), asg = sm100::smem_addr(sgn);
-#pragma unroll
-        for (int ks = 0; ks < SK / 16; ++ks) {
-          const uint32_t oq = ks * 2 * (SQ * 16), orr = ks * 2 * (SR * 16);
-          const uint32_t first = (kc > 0 || ks > 0) ? 1u : 0u;
-          sm100::mma_bf16_ss(tDm, sm100::smem_desc(aq1h + oq, SQ * 16, 128), sm100::smem_desc(ach + orr, SR * 16, 128), idesc, first);
-          sm100::mma_bf16_ss(tDm, sm100::smem_desc(aq1h + oq, SQ * 16, 128), sm100::smem_desc(acl + orr, SR * 16, 128), idesc, 1);
-          sm100::mma_bf16_ss(tDm, sm100::smem_desc(aq1l + oq, SQ * 16, 128), sm100::smem_desc(ach + orr, SR * 16, 128), idesc, 1);
-          sm100::mma_bf16_ss(tDs, sm100::smem_desc(aq2h + oq, SQ * 16, 128), sm100::smem_desc(asg + orr, SR * 16, 128), idesc, first);
-          sm100::mma_bf16_ss(tDs, sm100::smem_desc(aq2l + oq, SQ * 16, 128), sm100::smem_desc(asg + orr, SR * 16, 128), idesc, 1);
+  const int nt = t_end > t_begin ? static_cast<int>(t_end - t_begin) : 0;
+  const int total = nt * XCH;
+
+  if (warp == SCW) {
+    // ---------------- MMA warp: query-chunk copies and the MMAs
+    if (lane == 0 && total > 0) {
+      const uint16_t *qsrc = a.qop + static_cast<int64_t>(blockIdx.x) * XCH * (QN * 64);
+      auto copy = [&](int g) {
+        const int s = g % NAS, c = g % XCH;
+        sm100::mbar_expect_tx(&b_full[s], QCH_BYTES);
+        sm100::bulk_g2s(bst + s * QCH_BYTES, qsrc + c * (QN * 64), QCH_BYTES, &b_full[s]);
+      };
+      for (int g = 0; g < NAS - 1 && g < total; ++g) copy(g);
+      constexpr uint32_t IDESC = sm100::idesc_f16(RM, QN);
+      bool ok = true;
+      for (int tl = 0; tl < nt && ok; ++tl) {
+        if (tl >= 1) {
+          ok = sm100::mbar_wait(&acc_free, (tl - 1) & 1);
+          if (!ok) break;
+          sm100::fence_after_sync();
         }
-        sm100::mma_commit(&mb);
-      }
-      if (!sm100::mbar_wait(&mb, ph)) abort_s = 1;
-      ph ^= 1;
-      __syncthreads();
-      if (abort_s) break;
-    }
-    if (abort_s) break;
-    sm100::fence_after_sync();
-    // scores of query `q` against the tile's rows; running top-k
-    for (int c0 = 0; c0 < SR; c0 += 16) {
-      uint32_t dm[16], ds[16];
-      sm100::tmem_ld16(sm100::tmem_lane(tDm + c0, warp), dm);
-      sm100::tmem_ld16(sm100::tmem_lane(tDs + c0, warp), ds);
-      sm100::wait_ld();
+        for (int c = 0; c < XCH && ok; ++c) {
+          const int g = tl * XCH + c, s = g % NAS, u = g / NAS;
+          ok = sm100::mbar_wait(&a_full[s], u & 1) && sm100::mbar_wait(&b_full[s], u & 1);
+          if (!ok) break;
+          sm100::fence_after_sync();
+          const uint32_t bb = sm100::smem_addr(bst + s * QCH_BYTES);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int64_t r = r0 + c0 + c;
-        if (r >= a.n) continue;
-        const float s = nus[c0 + c] * fmaf(a.coef * rhos[c0 + c], __uint_as_float(ds[c]), __uint_as_float(dm[c]));
-        if (s > ts[SKMAX - 1]) {
-          ts[SKMAX - 1] = s;
-          ti[SKMAX - 1] = static_cast<int>(r);
-#pragma unroll
-          for (int e = SKMAX - 1; e > 0; --e) {
-            if (ts[e] > ts[e - 1]) {
-              const float fs = ts[e];
-              ts[e] = ts[e - 1];
-              ts[e - 1] = fs;
-              const int fi = ti[e];
-              ti[e] = ti[e - 1];
-              ti[e - 1] = fi;
+          for (int kk = 0; kk < 4; ++kk)
+            sm100::mma_f16_ts(tm, tm + 256 + s * 32 + kk * 8,
+                              sm100::smem_desc(bb + kk * 2 * (QN * 16), QN * 16, 128), IDESC,
+                              (c > 0 || kk > 0) ? 1u : 0u);
+          sm100::mma_commit(&done[s]);
+          if (c == XCH - 1) sm100::mma_commit(&acc_full);
+          // refill: chunk g + NAS - 1 reuses the stage of chunk g - 1
+          const int gn = g + NAS - 1;
+          if (gn < total) {
+            if (gn >= NAS) {
+              ok = sm100::mbar_wait(&done[gn % NAS], ((gn / NAS) - 1) & 1);
+              if (!ok) break;
             }
+            copy(gn);
           }
         }
       }
+      if (!ok) abort_s = 1;
     }
-    sm100::fence_before_sync();
-    __syncthreads();
-    sm100::fence_after_sync();
-  }
-  if (!abort_s && q < a.nq) {
-    float *cs = a.cand_s + (static_cast<int64_t>(q) * gridDim.y + blockIdx.y) * a.k;
-    int32_t *ci = a.cand_i + (static_cast<int64_t>(q) * gridDim.y + blockIdx.y) * a.k;
+    __syncwarp();
+  } else {
+    // ---------------- workers: warp (quarter wq, half h); thread = row 32 wq + lane
+    const int wq = warp & 3, h = warp >> 2;
+    const int r = 32 * wq + lane;
+    const int planes = a.mbk + 1;
+    float ts0[SKMAX], ts1[SKMAX];
+    int ti0[SKMAX], ti1[SKMAX];
 #pragma unroll
-    for (int e = 0; e < SKMAX; ++e)
-      if (e < a.k) {
-        cs[e] = ts[e];
-        ci[e] = ti[e];
+    for (int e = 0; e < SKMAX; ++e) {
+      ts0[e] = ts1[e] = -CUDART_INF_F;
+      ti0[e] = ti1[e] = 0x7fffffff;
+    }
+    const int qq = tid & 127, rh = tid >> 7;   // top-k role: query qq of a pass, rows 64 rh ..
+    const int qbase = blockIdx.x * QN;
+    const float qs0 = qbase + qq < a.nq ? a.qinv[qbase + qq] : 0.f;
+    const float qs1 = qbase + 128 + qq < a.nq ? a.qinv[qbase + 128 + qq] : 0.f;
+    // Waits are bounded; after one gives up (abort_s) every later wait is
+    // skipped but the loops keep their fixed trip counts, so all worker warps
+    // still meet at every named barrier.
+    auto wwait = [&](uint64_t *bar, uint32_t par) {
+      if (lane == 0 && !abort_s && !sm100::mbar_wait(bar, par)) abort_s = 1;
+      __syncwarp();
+    };
+    auto insert = [&](float (&ts)[SKMAX], int (&ti)[SKMAX], float v, int idx) {
+      if (v > ts[SKMAX - 1]) {
+        ts[SKMAX - 1] = v;
+        ti[SKMAX - 1] = idx;
+#pragma unroll
+        for (int e = SKMAX - 1; e > 0; --e) {
+          if (ts[e] > ts[e - 1]) {
+            const float fs = ts[e];
+            ts[e] = ts[e - 1];
+            ts[e - 1] = fs;
+            const int fi = ti[e];
+            ti[e] = ti[e - 1];
+            ti[e - 1] = fi;
+          }
+        }
       }
+    };
+    for (int tl = 0; tl < nt; ++tl) {
+      const int64_t row = (t_begin + tl) * RM + r;
+      const bool valid = row < a.n;
+      uint32_t sc = 0;
+      if (valid) sc = reinterpret_cast<const uint32_t *>(a.kscale)[row];
+      const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+      const uint32_t rho2 = (sc >> 16) | (sc & 0xffff0000u);     // half2 (rho, rho)
+      const uint32_t *kr = reinterpret_cast<const uint32_t *>(a.kcode + (valid ? row : 0) * planes * (XD / 8));
+      // chunks of this half: pairs (c, c + 1) with (c / 2) % 2 == h
+      for (int c2 = 2 * h; c2 < XCH; c2 += 4) {
+        uint2 w[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          w[p] = (valid && p < planes) ? *reinterpret_cast<const uint2 *>(kr + p * XW + c2) : make_uint2(0u, 0u);
+        // plane order: MSE planes 0 .. mbk-1, then the sign plane (index mbk)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = c2 + cc;
+          const int g = tl * XCH + c, s = g % NAS, u = g / NAS;
+          if (u >= 1) {
+            wwait(&done[s], (u - 1) & 1);
+            sm100::fence_after_sync();
+          }
+          const uint32_t p0 = cc ? w[0].y : w[0].x;
+          const uint32_t p1 = a.mbk > 1 ? (cc ? w[1].y : w[1].x) : 0u;
+          const uint32_t p2 = a.mbk > 2 ? (cc ? w[2].y : w[2].x) : 0u;
+          const uint32_t sg = a.mbk == 1 ? (cc ? w[1].y : w[1].x)
+                              : a.mbk == 2 ? (cc ? w[2].y : w[2].x)
+                                           : (cc ? w[3].y : w[3].x);
+          const uint32_t nsg = ~sg;
+          uint32_t out[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t idx = ((p0 >> (2 * j)) & 3u) | (((p1 >> (2 * j)) & 3u) << 2) |
+                                 (((p2 >> (2 * j)) & 3u) << 4);
+            out[j] = lut[idx * 32 + lane];
+            out[16 + j] = rho2 ^ (((nsg >> (2 * j)) & 1u) << 15) ^ (((nsg >> (2 * j + 1)) & 1u) << 31);
+          }
+          sm100::tmem_st32(sm100::tmem_lane(tm + 256 + s * 32, wq), out);
+          sm100::wait_st();
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&a_full[s]);
+        }
+      }
+      // ---- epilogue of the tile
+      wwait(&acc_full, tl & 1);
+      sm100::fence_after_sync();
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 32) {
+          uint32_t v[32];
+          sm100::tmem_ld32(sm100::tmem_lane(tm + 128 * qh + 64 * h + cc, wq), v);
+          sm100::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sb[(64 * h + cc + e) * SBP + r] = nu * __uint_as_float(v[e]);
+        }
+        if (qh == 1) {   // this warp has read its part of D
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&acc_free);
+        }
+        sm100::named_sync(1, SCW * 32);
+        const float qs = qh ? qs1 : qs0;
+        const float *srow = sb + qq * SBP + 64 * rh;
+        const int64_t r0 = (t_begin + tl) * RM + 64 * rh;
+        const int nr = a.n - r0 < 64 ? static_cast<int>(a.n - r0) : 64;
+        if (qh == 0) {
+          for (int rr = 0; rr < nr; ++rr) insert(ts0, ti0, srow[rr] * qs, static_cast<int>(r0 + rr));
+        } else {
+          for (int rr = 0; rr < nr; ++rr) insert(ts1, ti1, srow[rr] * qs, static_cast<int>(r0 + rr));
+        }
+        sm100::named_sync(1, SCW * 32);
+      }
+    }
+    // candidate lists: one per (query, CTA row range, row half)
+    const int lists = gridDim.y * 2, list = blockIdx.y * 2 + rh;
+    if (!abort_s) {
+#pragma unroll
+      for (int qh = 0; qh < 2; ++qh) {
+        const int q = qbase + 128 * qh + qq;
+        if (q < a.nq) {
+          float *cs = a.cand_s + (static_cast<int64_t>(q) * lists + list) * a.k;
+          int32_t *ci = a.cand_i + (static_cast<int64_t>(q) * lists + list) * a.k;
+#pragma unroll
+          for (int e = 0; e < SKMAX; ++e)
+            if (e < a.k) {
+              cs[e] = qh ? ts1[e] : ts0[e];
+              ci[e] = qh ? ti1[e] : ti0[e];
+            }
+        }
+      }
+    }
   }
-  if (abort_s) {
-    sm100::mbar_wait(&mb, ph, 1u << 20);
-    if (tid == 0 && a.err) atomicExch(a.err, 1u);
-  }
+  if (abort_s && tid == 0 && a.err) atomicExch(a.err, 1u);
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  if (warp == 0) sm100::tmem_dealloc(tm, 256);
+  if (warp == 0) sm100::tmem_dealloc(tm, 512);
 }
 
 // Merge the per-CTA candidate lists of each query: order (-score, index).
@@ -645,11 +741,18 @@ int run_gemm(const GemmArgs &g, cudaStream_t stream) {
   return tq_check_launch("ix_gemm_kernel");
 }
 
-bool index_codec_ok(const tq_codec *c) { return c->d == XD && c->qjl_k && c->mse_bits_k <= 4; }
+bool index_codec_ok(const tq_codec *c) { return c->d == XD && c->qjl_k && c->mse_bits_k <= 3; }
+
+uint32_t half_bits(float x) {   // fp32 -> fp16 bit pattern, round to nearest even
+  const __half h = __float2half_rn(x);
+  uint16_t b;
+  memcpy(&b, &h, 2);
+  return b;
+}
 
 int scan_grid_y(int64_t n, int nq) {
-  const int64_t tiles = (n + SR - 1) / SR;
-  const int qblocks = (nq + SQ - 1) / SQ;
+  const int64_t tiles = (n + RM - 1) / RM;
+  const int qblocks = (nq + QN - 1) / QN;
   int64_t gy = sm_count() / qblocks;   // one wave: grid.x * grid.y <= SMs (one CTA per SM)
   if (gy > tiles) gy = tiles;
   return static_cast<int>(gy < 1 ? 1 : gy);
@@ -670,7 +773,7 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
                    uint32_t *status, void *workspace, size_t ws_bytes, void *stream) {
   if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "index: NULL codec");
   if (!index_codec_ok(c))
-    return tq_fail(TQ_ERR_UNSUPPORTED, "index: needs a d = 1536 codec with QJL keys");
+    return tq_fail(TQ_ERR_UNSUPPORTED, "index: needs a d = 1536 codec with QJL keys and 1..3 MSE bits");
   if (!x || !kcode || !kscale || !workspace || n < 1)
     return tq_fail(TQ_ERR_INVALID_ARG, "index: NULL buffer or n < 1");
   size_t need = 0;
@@ -711,24 +814,46 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
     g.plane = a.kcode + c->mse_bits_k * (XD / 8);
     g.plane_stride = planes * (XD / 8);
     g.out = nullptr;
-    g.out_hl = nullptr;
-    g.scale = 1.f;
     g.status = status;
     if (int e = run_gemm<0>(g, st)) return e;
   }
   return TQ_OK;
 }
 
+// Scan workspace, 256-byte aligned pieces: q' fp32, q' bf16 hi | lo (GEMM A),
+// q'' fp32, the packed fp16 query operand, 2^-e per query, candidate lists.
+struct ScanWs {
+  size_t q1, q1hl, q2, qop, qinv, cand_s, cand_i, total;
+};
+
+ScanWs scan_ws(int nq, int k, int gy) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t nqb = (nq + QN - 1) / QN;
+  ScanWs w;
+  size_t o = 0;
+  w.q1 = o;
+  o += up(static_cast<size_t>(nq) * XD * 4);
+  w.q1hl = o;
+  o += up(static_cast<size_t>(nq) * 2 * XD * 2);
+  w.q2 = o;
+  o += up(static_cast<size_t>(nq) * XD * 4);
+  w.qop = o;
+  o += up(nqb * XCH * QCH_BYTES);
+  w.qinv = o;
+  o += up(static_cast<size_t>(nq) * 4);
+  const size_t nc = static_cast<size_t>(nq) * (2 * gy) * k;
+  w.cand_s = o;
+  o += up(nc * 4);
+  w.cand_i = o;
+  o += up(nc * 4);
+  w.total = o;
+  return w;
+}
+
 int tq_scan_workspace(const tq_codec *c, int64_t n, int nq, int k, size_t *bytes) {
   if (!c || !bytes || n < 1 || nq < 1 || k < 1 || k > SKMAX)
     return tq_fail(TQ_ERR_INVALID_ARG, "scan workspace: bad arguments (1 <= k <= 16)");
-  const int gy = scan_grid_y(n, nq);
-  size_t b = 0;
-  b += static_cast<size_t>(nq) * XD * 4;          // q'
-  b += static_cast<size_t>(nq) * 2 * XD * 2;      // q' hi | lo
-  b += static_cast<size_t>(nq) * 2 * XD * 2;      // q'' hi | lo
-  b += static_cast<size_t>(nq) * gy * k * 8;      // candidates
-  *bytes = b + 256;
+  *bytes = scan_ws(nq, k, scan_grid_y(n, nq)).total;
   return TQ_OK;
 }
 
@@ -737,24 +862,27 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
                  size_t ws_bytes, void *stream) {
   if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "scan: NULL codec");
   if (!index_codec_ok(c))
-    return tq_fail(TQ_ERR_UNSUPPORTED, "scan: needs a d = 1536 codec with QJL keys");
+    return tq_fail(TQ_ERR_UNSUPPORTED, "scan: needs a d = 1536 codec with QJL keys and 1..3 MSE bits");
   if (!kcode || !kscale || !q || !idx || !score || !workspace || n < 1 || nq < 1 || k < 1 ||
       k > SKMAX || k > n)
     return tq_fail(TQ_ERR_INVALID_ARG, "scan: NULL buffer or bad n / nq / k (1 <= k <= min(16, n))");
-  size_t need = 0;
-  tq_scan_workspace(c, n, nq, k, &need);
-  if (ws_bytes < need) return tq_fail(TQ_ERR_WORKSPACE, "scan: workspace too small");
+  if (n > 0x7fffffffLL) return tq_fail(TQ_ERR_INVALID_ARG, "scan: n must fit in int32 indices");
+  const int gy = scan_grid_y(n, nq);
+  const ScanWs W = scan_ws(nq, k, gy);
+  if (ws_bytes < W.total) return tq_fail(TQ_ERR_WORKSPACE, "scan: workspace too small");
   if ((reinterpret_cast<uintptr_t>(kcode) | reinterpret_cast<uintptr_t>(q) |
        reinterpret_cast<uintptr_t>(workspace)) % 16 || reinterpret_cast<uintptr_t>(kscale) % 4)
     return tq_fail(TQ_ERR_ALIGNMENT, "scan: kcode/q/workspace need 16-byte, kscale 4-byte alignment");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(workspace);
-  float *q1 = reinterpret_cast<float *>(w);
-  uint16_t *q1hl = reinterpret_cast<uint16_t *>(q1 + static_cast<size_t>(nq) * XD);
-  uint16_t *q2hl = q1hl + static_cast<size_t>(nq) * 2 * XD;
-  float *cand_s = reinterpret_cast<float *>(q2hl + static_cast<size_t>(nq) * 2 * XD);
-  const int gy = scan_grid_y(n, nq);
-  int32_t *cand_i = reinterpret_cast<int32_t *>(cand_s + static_cast<size_t>(nq) * gy * k);
+  float *q1 = reinterpret_cast<float *>(w + W.q1);
+  uint16_t *q1hl = reinterpret_cast<uint16_t *>(w + W.q1hl);
+  float *q2 = reinterpret_cast<float *>(w + W.q2);
+  uint16_t *qop = reinterpret_cast<uint16_t *>(w + W.qop);
+  float *qinv = reinterpret_cast<float *>(w + W.qinv);
+  float *cand_s = reinterpret_cast<float *>(w + W.cand_s);
+  int32_t *cand_i = reinterpret_cast<int32_t *>(w + W.cand_i);
+  // q' = Pi q (fp32 and bf16 hi | lo)
   QrotArgs qa;
   qa.q = q;
   qa.nq = nq;
@@ -765,6 +893,7 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   ix_qrot_kernel<<<(nq + 7) / 8, 256, 0, st>>>(qa);
   tq_count_launch(1);
   if (int e = tq_check_launch("ix_qrot_kernel")) return e;
+  // q'' = S q' (fp32) on the tensor cores
   GemmArgs g;
   g.A = q1hl;
   g.B = c->S_dev;
@@ -774,44 +903,62 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   g.KB = XD;
   g.plane = nullptr;
   g.plane_stride = 0;
-  g.out = nullptr;
-  g.out_hl = q2hl;
-  g.scale = 1.f;
+  g.out = q2;
   g.status = nullptr;
-  if (int e = run_gemm<2>(g, st)) return e;
-  ScanArgs sa;
-  sa.q1hl = q1hl;
-  sa.q2hl = q2hl;
+  if (int e = run_gemm<1>(g, st)) return e;
+  // fp16 B operand with a power-of-two scale per query
+  const float coef = sqrtf(static_cast<float>(M_PI) / 2.0f) / XD;
+  QpackArgs pa;
+  pa.q1 = q1;
+  pa.q2 = q2;
+  pa.nq = nq;
+  pa.coef = coef;
+  pa.qop = qop;
+  pa.qinv = qinv;
+  const int nqp = (nq + QN - 1) / QN * QN;
+  ix_qpack_kernel<<<(nqp + 7) / 8, 256, 0, st>>>(pa);
+  tq_count_launch(1);
+  if (int e = tq_check_launch("ix_qpack_kernel")) return e;
+  // scan
+  Scan2Args sa;
   sa.kcode = kcode;
   sa.kscale = kscale;
   sa.n = n;
+  sa.qop = qop;
+  sa.qinv = qinv;
   sa.nq = nq;
-  sa.k = k;
-  const int64_t tiles = (n + SR - 1) / SR;
+  const int64_t tiles = (n + RM - 1) / RM;
   sa.tiles_per_cta = static_cast<int>((tiles + gy - 1) / gy);
-  sa.coef = sqrtf(static_cast<float>(M_PI) / 2.0f) / XD;
-  for (int i = 0; i < TQ_MAX_LEVELS; ++i) sa.ck[i] = c->books.ck[i];
   sa.mbk = c->mse_bits_k;
+  for (int e = 0; e < 64; ++e) {
+    // index bits (b0 even, b0 odd, b1 even, b1 odd, b2 even, b2 odd)
+    const int me = (e & 1) | ((e >> 2) & 1) << 1 | ((e >> 4) & 1) << 2;
+    const int mo = ((e >> 1) & 1) | ((e >> 3) & 1) << 1 | ((e >> 5) & 1) << 2;
+    const uint32_t lo = half_bits(me < (1 << sa.mbk) ? c->books.ck[me] : 0.f);
+    const uint32_t hi = half_bits(mo < (1 << sa.mbk) ? c->books.ck[mo] : 0.f);
+    sa.lut[e] = lo | (hi << 16);
+  }
   sa.cand_s = cand_s;
   sa.cand_i = cand_i;
+  sa.k = k;
   sa.err = nullptr;
-  constexpr int shm = 4 * (SQ * SK * 2) + 3 * (SR * SK * 2);
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !done[dev]) {
-    if (cudaFuncSetAttribute(ix_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shm) != cudaSuccess)
-      return tq_check_launch("cudaFuncSetAttribute(ix_scan)");
+    if (cudaFuncSetAttribute(ix_scan2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(SC_SMEM)) != cudaSuccess)
+      return tq_check_launch("cudaFuncSetAttribute(ix_scan2)");
     done[dev] = true;
   }
-  dim3 grid((nq + SQ - 1) / SQ, gy);
+  dim3 grid((nq + QN - 1) / QN, gy);
   cudaEvent_t ev0, ev1;
   tq_timing_events(&ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, st);
-  ix_scan_kernel<<<grid, 128, shm, st>>>(sa);
-  if (int e = tq_check_launch("ix_scan_kernel")) return e;
+  ix_scan2_kernel<<<grid, SCT, SC_SMEM, st>>>(sa);
+  if (int e = tq_check_launch("ix_scan2_kernel")) return e;
   if (ev1) cudaEventRecord(ev1, st);
-  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(cand_s, cand_i, nq, gy, k, idx, score);
+  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(cand_s, cand_i, nq, 2 * gy, k, idx, score);
   tq_count_launch(2);
   return tq_check_launch("ix_merge_kernel");
 }
