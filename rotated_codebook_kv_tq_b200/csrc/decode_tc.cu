@@ -111,8 +111,6 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
   __shared__ float red[TCT / 32][2 * G];
   __shared__ double dred[TCT / 32][2 * G];
   __shared__ float Fs[2 * G];
-  __shared__ __align__(16) int8_t bks[N * KTOT];
-  extern __shared__ __align__(16) uint16_t sts[];   // S^T, bf16 [TD][TD] (dynamic)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x;
@@ -142,20 +140,23 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
 #pragma unroll
     for (int k = 0; k < TNW; ++k) q1s[warp][lane + 32 * k] = x[k] * inv_sqrt_d;
   }
-  if (QJL) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.ST);
-    for (int e = tid; e < TD * TD / 8; e += TCT) reinterpret_cast<uint4 *>(sts)[e] = src[e];
-  }
   __syncthreads();
   if (QJL) {
+    // q''_i = sum_j S[i][j] q'_j: thread i reads row i of S (bf16) as 16-byte loads
+    const uint4 *srow = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * TD);
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < TD; ++j) {
-      const float s = tq_bf16_to_f32(sts[j * TD + tid]);
+#pragma unroll 4
+    for (int q = 0; q < TD / 8; ++q) {
+      const uint4 v = srow[q];
+      const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(s, q1s[h][j], acc[h]);
+      for (int e = 0; e < 8; ++e) {
+        const float sv = __uint_as_float((e & 1) ? (wds[e >> 1] & 0xffff0000u) : (wds[e >> 1] << 16));
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, q1s[h][8 * q + e], acc[h]);
+      }
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) q2s[h][tid] = acc[h];
@@ -183,23 +184,44 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
     }
     __syncthreads();
   }
-  // B operand bytes (K-major, no swizzle): MSE part then QJL part
-  for (int e = tid; e < N * KTOT; e += TCT) {
-    const int n = e / KTOT, k = e % KTOT;
-    const int h = n >> 2, l = n & 3;
-    int8_t byte = 0;
-    if (h < G) {
-      const bool mse = k < KM;
-      const int kk = mse ? k : k - KM;
+  // B operand (K-major, no swizzle): MSE part then QJL part.  One item =
+  // (head h, K chunk kc): its 16 fixed-point values are computed once and
+  // split into the four limb rows n = 4h + l, each stored as one 16-byte
+  // write straight to the group's global B region.
+  uint8_t *dst = a.bk + static_cast<int64_t>(bh) * a.bk_stride;
+  constexpr int NKC = KTOT / 16, NKM = KM / 16;
+  for (int it = tid; it < G * NKC; it += TCT) {
+    const int h = it % G, kc = it / G;
+    const bool mse = kc < NKM;
+    const int kb = mse ? kc * 16 : (kc - NKM) * 16;
+    uint32_t wv[4][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int kk = kb + e;
       const int col = kk >> 2, nb = kk & 3;
       const int ti = col >> 5, w = (col & 31) >> 3, r = col & 7;
       const int i = 32 * w + 8 * nb + r;
       const float val = mse ? 2.f * a.wk[ti] * q1s[h][i] * Fs[h] : 2.f * q2s[h][i] * Fs[G + h];
-      const int qv = __float2int_rn(val);
-      byte = limb_of(qv * (1 << (7 - r)), l);
+      int v = __float2int_rn(val) * (1 << (7 - r));
+      // signed base-256 digits: v = L0 + 2^8 L1 + 2^16 L2 + 2^24 L3
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        const int8_t d = static_cast<int8_t>(v & 0xff);
+        wv[l][e >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(d)) << (8 * (e & 3));
+        v = (v - d) >> 8;
+      }
     }
-    const int part = k < KM ? 0 : N * KM;
-    bks[part + kmajor_off(n, k < KM ? k : k - KM, N)] = byte;
+#pragma unroll
+    for (int l = 0; l < 4; ++l)
+      *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(4 * h + l, kb, N)) =
+          make_uint4(wv[l][0], wv[l][1], wv[l][2], wv[l][3]);
+  }
+  // rows beyond the G heads' limbs (N > 4 G) are zero
+  for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
+    const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
+    const bool mse = kc < NKM;
+    const int kb = mse ? kc * 16 : (kc - NKM) * 16;
+    *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
   }
   // constants: C = sum of the quantized B values / (2F), per head and part
   {
@@ -228,9 +250,6 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
       }
   }
   __syncthreads();
-  uint8_t *dst = a.bk + static_cast<int64_t>(bh) * a.bk_stride;
-  for (int e = tid; e < N * KTOT / 16; e += TCT)
-    reinterpret_cast<int4 *>(dst)[e] = reinterpret_cast<const int4 *>(bks)[e];
   if (tid < G) {
     double s1 = 0.0, s2 = 0.0;
     for (int w = 0; w < TCT / 32; ++w) {
@@ -857,7 +876,7 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tc_chunk_kernel<G, MBK, BV, QJL>, CT, smem);
   if (occ < 1) occ = 1;
   if (occ < per_sm) per_sm = occ;
-  tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, QJL ? TD * TD * 2 : 0, stream>>>(a);
+  tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, 0, stream>>>(a);
   if (int e = tq_check_launch("tc_prep_kernel")) return e;
   const int items = a.B * a.Hkv * a.splits;
   const int grid = items < sms * per_sm ? items : sms * per_sm;
@@ -913,6 +932,7 @@ int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq,
   a.qjl_coef = c->qjl_k ? sqrtf(static_cast<float>(M_PI) / 2.0f) / c->d : 0.f;
   a.rc = rc;
   a.rs = rs;
+  a.S = c->S_dev;
   a.ST = c->ST_dev;
   a.splits = splits;
   const int per = (max_len + splits - 1) / splits;

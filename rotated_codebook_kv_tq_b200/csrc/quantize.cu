@@ -233,6 +233,146 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
 
 
 // ---------------------------------------------------------------------------
+// Small calls (decode appends): one 128-thread block per (b, h, 32-token
+// group).  Warp 0 runs the key pipeline of a row and warp 1 the value
+// pipeline (same steps as quantize_kernel); the sketch z = S r of the key row
+// is spread over the block: thread i computes z_i from row i of S (bf16,
+// row-major, read from L2 as 16-byte loads), so no block stages S^T.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
+  constexpr int NPL = D / 32;
+  __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
+  __shared__ __align__(16) float rsm[D];
+  __shared__ uint32_t sgw[NPL];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nlk = 1 << a.books.mse_bits_k, nlv = 1 << a.books.bits_v;
+  if (tid < TQ_MAX_LEVELS) {
+    cks[tid] = a.books.ck[tid];
+    tks[tid] = a.books.tk[tid];
+    tvs[tid] = a.books.tv[tid];
+  }
+  __syncthreads();
+  const int planes_k = a.books.mse_bits_k + a.books.qjl;
+  const int64_t it = blockIdx.x;
+  const int64_t g = a.g_first + it % a.n_groups;
+  const int64_t bh = it / a.n_groups;
+  const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
+  const int64_t r_begin = max(a.row0, g * 32), r_end = min(a.row0 + a.T, g * 32 + 32);
+  const int64_t cache_bh = static_cast<int64_t>(b) * a.H + h;
+  uint32_t vw[4][NPL];
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) vw[p][k] = 0u;
+
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    const int64_t t = r - a.row0;
+    const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
+    uint32_t myword = 0u;
+    float nu = 0.f, rho = 0.f;
+    bool bad = false;
+    if (warp == 0) {
+      float x[NPL];
+      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+      nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      int idx[NPL];
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks, nlk - 1);
+      for (int p = 0; p < a.books.mse_bits_k; ++p) {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          const uint32_t w = __ballot_sync(TQ_FULL, (idx[k] >> p) & 1);
+          if (lane == p * NPL + k) myword = w;
+        }
+      }
+      if (a.books.qjl) {
+        float r2 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          const float rr = x[k] - cks[idx[k]];
+          rsm[lane + 32 * k] = rr;
+          r2 += rr * rr;
+        }
+        rho = sqrtf(tq_warp_sum(r2));
+      }
+    } else if (warp == 1) {
+      float x[NPL];
+      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+      bool vbad;
+      const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, vbad);
+      const uint32_t bit = 1u << (r & 31);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        const int iv = tq_code(x[k], tvs, nlv - 1);
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if ((iv >> p) & 1) vw[p][k] |= bit;
+      }
+      if (lane == 0) {
+        a.vnorm[cache_bh * a.rows_cap + r] = tq_f32_to_half(nv);
+        if (vbad && a.status) atomicAdd(a.status, 1u);
+      }
+    }
+    __syncthreads();
+    if (a.books.qjl && tid < D) {
+      // z_tid = sum_j S[tid][j] r_j; whole warps take part (D is a multiple of 32)
+      const uint4 *srow = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * D);
+      float z = 0.f;
+#pragma unroll 4
+      for (int q = 0; q < D / 8; ++q) {
+        const uint4 v = srow[q];
+        const float4 r0 = reinterpret_cast<const float4 *>(rsm)[2 * q];
+        const float4 r1 = reinterpret_cast<const float4 *>(rsm)[2 * q + 1];
+        z = fmaf(__uint_as_float(v.x << 16), r0.x, z);
+        z = fmaf(__uint_as_float(v.x & 0xffff0000u), r0.y, z);
+        z = fmaf(__uint_as_float(v.y << 16), r0.z, z);
+        z = fmaf(__uint_as_float(v.y & 0xffff0000u), r0.w, z);
+        z = fmaf(__uint_as_float(v.z << 16), r1.x, z);
+        z = fmaf(__uint_as_float(v.z & 0xffff0000u), r1.y, z);
+        z = fmaf(__uint_as_float(v.w << 16), r1.z, z);
+        z = fmaf(__uint_as_float(v.w & 0xffff0000u), r1.w, z);
+      }
+      const uint32_t w = __ballot_sync(TQ_FULL, z >= 0.f);
+      if (lane == 0) sgw[warp] = w;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int p = a.books.mse_bits_k;
+      if (a.books.qjl && lane >= p * NPL && lane < (p + 1) * NPL) myword = sgw[lane - p * NPL];
+      uint32_t *krow = reinterpret_cast<uint32_t *>(
+          a.kcode + (cache_bh * a.rows_cap + r) * planes_k * (D / 8));
+      if (lane < planes_k * NPL) krow[lane] = myword;
+      if (lane == 0) {
+        const uint32_t pair = static_cast<uint32_t>(tq_f32_to_half(nu)) |
+                              (static_cast<uint32_t>(tq_f32_to_half(rho)) << 16);
+        reinterpret_cast<uint32_t *>(a.kscale)[cache_bh * a.rows_cap + r] = pair;
+        if (bad && a.status) atomicAdd(a.status, 1u);
+      }
+    }
+    __syncthreads();   // rsm and sgw are reused by the next row
+  }
+  if (warp == 1) {
+    // the group's value words (read-modify-write for partial groups)
+    const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
+    const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
+    uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
+    for (int p = 0; p < a.books.bits_v; ++p) {
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        uint32_t *w = vg + p * D + lane + 32 * k;
+        if (mask == TQ_FULL) {
+          *w = vw[p][k];
+        } else {
+          atomicAnd(w, ~mask);
+          atomicOr(w, vw[p][k] & mask);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // tcgen05 variant for large calls: the QJL sketch z = S r of a 128-row tile
 // is one tensor-core contraction.  Each warp runs the fused per-row pipeline
 // above for one 32-token group and writes its residuals, split into bf16
@@ -461,6 +601,13 @@ int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
 }
 
 template <int D>
+int run_quantize_append(const QuantArgs &a, int64_t items, cudaStream_t stream) {
+  quantize_append_kernel<D><<<static_cast<unsigned>(items), 128, 0, stream>>>(a);
+  tq_count_launch(1);
+  return tq_check_launch("quantize_append_kernel");
+}
+
+template <int D>
 int run_quantize(const QuantArgs &a, cudaStream_t stream) {
   const size_t shm = a.books.qjl ? sizeof(float) * D * D : 0;
   static bool attr_set = false;
@@ -517,10 +664,16 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   // TQ_QUANT_IMPL=simt keeps the CUDA-core sketch (a complete second
   // implementation, used to cross-check the tensor-core one)
   const char *impl = getenv("TQ_QUANT_IMPL");
-  const bool tc = c->qjl_k && items >= 256 && !(impl && impl[0] == 's');
+  const bool simt = impl && impl[0] == 's';
+  const bool tc = c->qjl_k && items >= 256 && !simt;
+  const bool append = items < 256 && !simt;
   switch (c->d) {
-    case 64: return tc ? run_quantize_tc<64>(a, stream) : run_quantize<64>(a, stream);
-    case 128: return tc ? run_quantize_tc<128>(a, stream) : run_quantize<128>(a, stream);
+    case 64:
+      return tc ? run_quantize_tc<64>(a, stream)
+                : append ? run_quantize_append<64>(a, items, stream) : run_quantize<64>(a, stream);
+    case 128:
+      return tc ? run_quantize_tc<128>(a, stream)
+                : append ? run_quantize_append<128>(a, items, stream) : run_quantize<128>(a, stream);
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "quantize: head dim not built");
   }
 }

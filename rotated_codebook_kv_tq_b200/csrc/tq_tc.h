@@ -23,6 +23,7 @@ struct TcArgs {
   float qjl_coef;
   const float *rc;
   const float *rs;
+  const uint16_t *S;    // S (bf16, row-major)
   const uint16_t *ST;   // S transposed (bf16)
   int splits;
   int chunk;            // rows per split (multiple of 128)
