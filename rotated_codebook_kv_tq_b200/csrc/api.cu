@@ -136,6 +136,10 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   tqhost::lloyd_max(c->d, c->bits_v, cc, tt, mse);
   for (size_t i = 0; i < cc.size(); ++i) c->books.cv[i] = static_cast<float>(cc[i]);
   for (size_t i = 0; i < tt.size(); ++i) c->books.tv[i] = static_cast<float>(tt[i]);
+  // unused threshold slots stay above every input (the kernels' code search
+  // runs over all TQ_MAX_LEVELS - 1 slots)
+  for (int i = (1 << mse_k) - 1; i < TQ_MAX_LEVELS; ++i) c->books.tk[i] = INFINITY;
+  for (int i = (1 << c->bits_v) - 1; i < TQ_MAX_LEVELS; ++i) c->books.tv[i] = INFINITY;
   for (int i = 0; i < c->d; ++i)
     if (desc->rotation_signs[i] < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
   c->books.mse_bits_k = mse_k;

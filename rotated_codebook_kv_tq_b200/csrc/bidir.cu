@@ -16,8 +16,9 @@
 // bf16 kind::f16 MMA sets (the order <= 2 products of a three-term bf16 split,
 // about 2^-26 relative: the logits reach a few hundred on data with outlier
 // channels, and a two-term split's 2^-17 would shift them by ~1e-3) with fp32
-// accumulators in tensor memory; softmax statistics and the output sum stay
-// in fp32 registers of the query's thread.
+// accumulators in tensor memory; softmax statistics stay in fp32 registers
+// of the query's thread and the output sum accumulates in tensor memory
+// (rescaled in place when a row's running maximum moves).
 // The tensor core's fp32 accumulation does not round to nearest: every MMA
 // that adds into an accumulator can lose up to an ulp of it, and a chain of
 // 48 MMAs into one accumulator moves logits of ~200 by ~5e-4.  So S is split
@@ -134,7 +135,8 @@ __device__ __forceinline__ void split3_store(uint8_t *base, uint32_t stride, int
 // (nbig = 1 folds everything into d_small, for the P V product).
 __device__ __forceinline__ void mma6(uint32_t d_small, uint32_t d_big, uint32_t dstride, int nbig,
                                      uint32_t a, uint32_t astr, uint32_t b, uint32_t bstr,
-                                     int ksteps, uint32_t lbo_a, uint32_t lbo_b, uint32_t idesc) {
+                                     int ksteps, uint32_t lbo_a, uint32_t lbo_b, uint32_t idesc,
+                                     bool acc_first) {
   const int pa[6] = {2, 1, 0, 1, 0, 0}, pb[6] = {0, 1, 2, 0, 1, 0};
   int n = 0;
 #pragma unroll
@@ -142,7 +144,7 @@ __device__ __forceinline__ void mma6(uint32_t d_small, uint32_t d_big, uint32_t 
     for (int s = 0; s < ksteps; ++s, ++n)
       sm100::mma_bf16_ss(d_small, sm100::smem_desc(a + pa[t] * astr + s * 2 * lbo_a, lbo_a, 128),
                          sm100::smem_desc(b + pb[t] * bstr + s * 2 * lbo_b, lbo_b, 128), idesc,
-                         n > 0);
+                         (n > 0 || acc_first) ? 1u : 0u);
   for (int s = 0; s < ksteps; ++s) {
     const uint32_t d = nbig > 1 ? d_big + (s % nbig) * dstride : d_small;
     sm100::mma_bf16_ss(d, sm100::smem_desc(a + s * 2 * lbo_a, lbo_a, 128),
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   uint8_t *vs3 = ps3 + 3 * P_BYTES;
   float *nuk = reinterpret_cast<float *>(vs3 + 3 * V_BYTES);  // [BK]
   __shared__ float cks[TQ_MAX_LEVELS], cvs[TQ_MAX_LEVELS];
+  __shared__ float vns[BK];   // value norms of the current key tile
   __shared__ __align__(8) uint64_t mb;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
@@ -205,15 +208,16 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   const uint32_t a_q = sm100::smem_addr(qs3), a_k = sm100::smem_addr(ks3);
   const uint32_t a_p = sm100::smem_addr(ps3), a_v = sm100::smem_addr(vs3);
 
-  float o[D], m = -CUDART_INF_F, l = 0.f;
-#pragma unroll
-  for (int i = 0; i < D; ++i) o[i] = 0.f;
+  float m = -CUDART_INF_F, l = 0.f;
   uint32_t phase = 0;
   for (int j0 = 0; j0 < a.T; j0 += BK) {
     // ---- key tile: thread (row tid % BK, half tid / BK) writes the MSE half
     // (c[idx]) or the sign half (+-coef rho) of one key row; value tile:
     // thread (coordinate tid % D, key group tid / D) writes 32 keys of V_rot^T.
     static_assert(BQ == 2 * BK && BQ == 2 * D && BK == 64, "thread mapping");
+    if (tid < BK)
+      vns[tid] = j0 + tid < a.T ? tq_half_to_f32(a.vnorm[bh * a.rows_cap + j0 + tid]) : 0.f;
+    __syncthreads();
     {
       const int row = tid % BK, half = tid / BK;
       const int j = j0 + row;
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
           const int j = jg + t;
           int idx = 0;
           for (int p = 0; p < nbv; ++p) idx |= ((vw[p] >> t) & 1) << p;
-          const float val = j < a.T ? tq_half_to_f32(a.vnorm[bh * a.rows_cap + j]) * cvs[idx] : 0.f;
+          const float val = j < a.T ? vns[32 * g + t] * cvs[idx] : 0.f;
           split3_store(vs3, V_BYTES, kmaj16(coord, 32 * g + t, D), val);
         }
       }
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     sm100::fence_after_sync();
     // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d)
     if (tid == 0) {
-      mma6(tS, tSb, BK, NBIG, a_q, Q_BYTES, a_k, K_BYTES, DP / 16, BQ * 16, BK * 16, IDESC_S);
+      mma6(tS, tSb, BK, NBIG, a_q, Q_BYTES, a_k, K_BYTES, DP / 16, BQ * 16, BK * 16, IDESC_S, false);
       sm100::mma_commit(&mb);
     }
     if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
@@ -305,15 +309,27 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     }
     l = l * corr + ps;
     m = mn;
+    // the running output lives in TMEM (columns tO): rescale a warp's rows
+    // when some row's maximum moved, before the P V MMAs add this tile
+    if (j0 > 0 && __any_sync(TQ_FULL, corr != 1.f)) {
 #pragma unroll
-    for (int i = 0; i < D; ++i) o[i] *= corr;
+      for (int c = 0; c < D; c += 8) {
+        uint32_t r[8];
+        sm100::tmem_ld8(sm100::tmem_lane(tO + c, warp), r);
+        sm100::wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+        sm100::tmem_st8(sm100::tmem_lane(tO + c, warp), r);
+      }
+      sm100::wait_st();
+    }
     sm100::fence_async_smem();
     sm100::fence_before_sync();
     __syncthreads();
     sm100::fence_after_sync();
     // ---- O_tile = P V_rot (M = 128 queries, N = d, K = 64 keys)
     if (tid == 0) {
-      mma6(tO, tO, 0, 1, a_p, P_BYTES, a_v, V_BYTES, BK / 16, BQ * 16, D * 16, IDESC_O);
+      mma6(tO, tO, 0, 1, a_p, P_BYTES, a_v, V_BYTES, BK / 16, BQ * 16, D * 16, IDESC_O, j0 > 0);
       sm100::mma_commit(&mb);
     }
     if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
@@ -321,17 +337,15 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
+  }
+  float o[D];
 #pragma unroll
-    for (int c = 0; c < D; c += 16) {
-      uint32_t r[16];
-      sm100::tmem_ld16(sm100::tmem_lane(tO + c, warp), r);
-      sm100::wait_ld();
+  for (int c = 0; c < D; c += 16) {
+    uint32_t r[16];
+    sm100::tmem_ld16(sm100::tmem_lane(tO + c, warp), r);
+    sm100::wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) o[c + e] += __uint_as_float(r[e]);
-    }
-    sm100::fence_before_sync();
-    __syncthreads();
-    sm100::fence_after_sync();
+    for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r[e]);
   }
   // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l)
   if (!abort_s && q0 + tid < a.Lq) {

@@ -22,6 +22,7 @@
 namespace {
 
 constexpr int QWARPS = 8;
+constexpr int QTC_T = 512;   // threads of quantize_tc_kernel: 4 groups x 4 row slices
 
 struct QuantArgs {
   const void *k;
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
 // (kb/16)*2048 + (m/8)*128 + (m%8)*16 + kb%16 for K = 2d elements (hi | lo);
 // B = S, byte (i, kb) at (kb/16)*(16d) + (i/8)*128 + (i%8)*16 + kb%16.
 template <int D>
-__global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   constexpr int NPL = D / 32;
   constexpr int KE = 2 * D;                       // K elements (hi | lo)
   constexpr uint32_t A_BYTES = 128u * KE * 2u;
@@ -393,6 +394,7 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
   uint8_t *As = reinterpret_cast<uint8_t *>(smem_tc);
   uint8_t *Bs = As + A_BYTES;
   __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
+  __shared__ uint32_t vbuf[4][4][D];   // value column words of the tile's 4 groups
   __shared__ __align__(8) uint64_t mb;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
     tks[tid] = a.books.tk[tid];
     tvs[tid] = a.books.tv[tid];
   }
-  for (int e = tid; e < D * D; e += 128) {
+  for (int e = tid; e < D * D; e += QTC_T) {
     const int i = e / D, kb = 2 * (e % D);
     *reinterpret_cast<uint16_t *>(Bs + (kb >> 4) * (D * 16) + (i >> 3) * 128 + (i & 7) * 16 +
                                   (kb & 15)) = a.S[e];
@@ -426,8 +428,11 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
   const int64_t tiles = (items + 3) / 4;
   uint32_t phase = 0;
 
+  // warp w: group grp = w / 4 of the tile, rows 8 (w % 4) .. +7 of that group
+  const int grp = warp >> 2, sub8 = warp & 3;
   for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    const int64_t it = tile * 4 + warp;
+    for (int e = tid; e < 4 * 4 * D; e += QTC_T) (&vbuf[0][0][0])[e] = 0u;
+    const int64_t it = tile * 4 + grp;
     const bool have = it < items;
     int64_t g = 0, cache_bh = 0, r_begin = 0, r_end = 0;
     int b = 0, h = 0;
@@ -445,11 +450,29 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
     for (int p = 0; p < 4; ++p)
 #pragma unroll
       for (int k = 0; k < NPL; ++k) vw[p][k] = 0u;
-    for (int64_t r = r_begin; r < r_end; ++r) {
-      const int64_t t = r - a.row0;
-      const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
+    const int64_t rb = max(r_begin, g * 32 + 8 * sub8), re = min(r_end, g * 32 + 8 * sub8 + 8);
+    __syncthreads();   // vbuf cleared
+    // rows are loaded PF at a time (all loads issued before any row is
+    // processed) so each warp keeps PF rows of K and V in flight
+    constexpr int PF = D == 64 ? 8 : 4;
+    for (int64_t r0 = rb; r0 < re; r0 += PF) {
+    float xk[PF][NPL], xv[PF][NPL];
+#pragma unroll
+    for (int i = 0; i < PF; ++i) {
+      if (r0 + i < re) {
+        const int64_t t = r0 + i - a.row0;
+        const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
+        load_row<NPL>(xk[i], a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+        load_row<NPL>(xv[i], a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < PF; ++i) {
+      const int64_t r = r0 + i;
+      if (r >= re) break;
       float x[NPL];
-      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) x[k] = xk[i][k];
       bool bad;
       const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
@@ -463,7 +486,7 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
           if (lane == p * NPL + k) myword = w;
         }
       }
-      const int m = warp * 32 + static_cast<int>(r & 31);
+      const int m = grp * 32 + static_cast<int>(r & 31);
       float r2 = 0.f;
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
@@ -487,7 +510,8 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
         reinterpret_cast<uint32_t *>(a.kscale)[cache_bh * a.rows_cap + r] = pair;
         if (bad && a.status) atomicAdd(a.status, 1u);
       }
-      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) x[k] = xv[i][k];
       const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
@@ -502,23 +526,13 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
         if (bad && a.status) atomicAdd(a.status, 1u);
       }
     }
-    if (have) {
-      const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
-      const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
-      uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
+    }
+    if (have && rb < re) {
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         if (p >= a.books.bits_v) break;
 #pragma unroll
-        for (int k = 0; k < NPL; ++k) {
-          uint32_t *w = vg + p * D + lane + 32 * k;
-          if (mask == TQ_FULL) {
-            *w = vw[p][k];
-          } else {
-            atomicAnd(w, ~mask);
-            atomicOr(w, vw[p][k] & mask);
-          }
-        }
+        for (int k = 0; k < NPL; ++k) atomicOr(&vbuf[grp][p][lane + 32 * k], vw[p][k]);
       }
     }
     // ---- the sketch of the whole tile on the tensor cores
@@ -526,6 +540,25 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
     sm100::fence_before_sync();
     __syncthreads();
     sm100::fence_after_sync();
+    // the group's value words (read-modify-write for partial groups)
+    if (have && sub8 == 0) {
+      const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
+      const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
+      uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
+      for (int p = 0; p < a.books.bits_v; ++p) {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) {
+          uint32_t *w = vg + p * D + lane + 32 * k;
+          const uint32_t v = vbuf[grp][p][lane + 32 * k];
+          if (mask == TQ_FULL) {
+            *w = v;
+          } else {
+            atomicAnd(w, ~mask);
+            atomicOr(w, v & mask);
+          }
+        }
+      }
+    }
     if (tid == 0) {
 #pragma unroll
       for (int s = 0; s < KE / 16; ++s) {
@@ -541,8 +574,19 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
-    const int64_t myr = g * 32 + lane;
-    const bool row_ok = have && myr >= r_begin && myr < r_end;
+    // warps 0..3 read TMEM lane quarter q = warp: rows of group q of the tile
+    if (warp < 4) {
+    const int64_t itq = tile * 4 + warp;
+    bool row_ok = false;
+    int64_t myr = 0, cbq = 0;
+    if (itq < items) {
+      const int64_t gq = a.g_first + itq % a.n_groups;
+      const int64_t bhq = itq / a.n_groups;
+      cbq = (bhq / a.H) * a.H + bhq % a.H;
+      const int64_t rbq = max(a.row0, gq * 32), req = min(a.row0 + a.T, gq * 32 + 32);
+      myr = gq * 32 + lane;
+      row_ok = myr >= rbq && myr < req;
+    }
     uint32_t sw[NPL];
 #pragma unroll
     for (int wd = 0; wd < NPL; ++wd) {
@@ -560,9 +604,10 @@ __global__ void __launch_bounds__(128, 1) quantize_tc_kernel(QuantArgs a) {
     }
     if (row_ok) {
       uint32_t *srow = reinterpret_cast<uint32_t *>(
-          a.kcode + (cache_bh * a.rows_cap + myr) * planes_k * (D / 8) + a.books.mse_bits_k * (D / 8));
+          a.kcode + (cbq * a.rows_cap + myr) * planes_k * (D / 8) + a.books.mse_bits_k * (D / 8));
 #pragma unroll
       for (int wd = 0; wd < NPL; ++wd) srow[wd] = sw[wd];
+    }
     }
     sm100::fence_before_sync();
     __syncthreads();
@@ -593,9 +638,9 @@ int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
   }
   const int64_t items = static_cast<int64_t>(a.B) * a.H * a.n_groups;
   const int64_t tiles = (items + 3) / 4;
-  const int64_t cap = static_cast<int64_t>(sms) * (D == 128 ? 2 : 4);
+  const int64_t cap = static_cast<int64_t>(sms) * (D == 128 ? 1 : 2);
   const int grid = static_cast<int>(tiles < cap ? tiles : cap);
-  quantize_tc_kernel<D><<<grid, 128, shm, stream>>>(a);
+  quantize_tc_kernel<D><<<grid, QTC_T, shm, stream>>>(a);
   tq_count_launch(1);
   return tq_check_launch("quantize_tc_kernel");
 }

@@ -81,11 +81,14 @@ __device__ __forceinline__ void tq_apply_signs(float (&x)[NPL], const uint32_t *
   }
 }
 
-// Scalar code: #{k : u >= t[k]} over `nt` thresholds (ties go up).
-__device__ __forceinline__ int tq_code(float u, const float *t, int nt) {
-  int idx = 0;
-#pragma unroll
-  for (int k = 0; k < TQ_MAX_LEVELS - 1; ++k)
-    if (k < nt) idx += (u >= t[k]) ? 1 : 0;
+// Code of u: #{k : u >= t_k} for ascending thresholds t[0 .. TQ_MAX_LEVELS-2]
+// whose unused slots hold +inf (the codec pads them): a branch-free binary
+// search over the 15 slots (the count is the same as a linear scan's).
+__device__ __forceinline__ int tq_code(float u, const float *t, int /*nt*/) {
+  static_assert(TQ_MAX_LEVELS == 16, "binary search covers 15 thresholds");
+  int idx = (u >= t[7]) ? 8 : 0;
+  idx += (u >= t[idx + 3]) ? 4 : 0;
+  idx += (u >= t[idx + 1]) ? 2 : 0;
+  idx += (u >= t[idx]) ? 1 : 0;
   return idx;
 }

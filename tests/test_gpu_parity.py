@@ -37,6 +37,9 @@ QUANT_CASES = {
     # >= 256 groups of 32 tokens: large calls take the tcgen05 sketch kernel
     "llama_tc_sketch": (synth.WORKLOADS["llama_decode"].scaled(T=1100), [(0, 1037), (1037, 63)]),
     "esm_tc_sketch_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=100), [(0, 100)]),
+    # large call, fp32 input, MSE-only keys (no sketch)
+    "llama_lanes_fp32_mse": (synth.WORKLOADS["llama_decode"].scaled(T=1100, dtype="fp32", qjl_k=False,
+                                                                     bits_k=3), [(0, 1100)]),
 }
 
 
@@ -90,8 +93,9 @@ def test_quantize_parity(case, impl, monkeypatch):
     assert not gpu["vnorm"][:, :, written:].any()
 
 
-def test_quantize_zero_and_nonfinite_rows():
-    w = synth.WORKLOADS["llama_decode"].scaled(B=1, Hkv=2, Hq=8, T=64)
+@pytest.mark.parametrize("T", [64, 4096])   # 4096: 256 token groups, the tensor-core sketch kernel
+def test_quantize_zero_and_nonfinite_rows(T):
+    w = synth.WORKLOADS["llama_decode"].scaled(B=1, Hkv=2, Hq=8, T=T)
     ocodec, ncodec = tl.codecs(w)
     K, V, K64, V64 = _inputs(w)
     Kf = synth.bf16_bits_to_f32(K).copy()
@@ -102,10 +106,10 @@ def test_quantize_zero_and_nonfinite_rows():
     Vf[0, 1, 10] = 0.0
     Kf[0, 1, 40, 0] = 1e6          # key norm overflows fp16
     w32 = w.scaled(dtype="fp32")
-    rope = synth.rope_for(w32, 64)
-    ocache = oc.empty_cache(ocodec, 1, 2, 64)
+    rope = synth.rope_for(w32, T)
+    ocache = oc.empty_cache(ocodec, 1, 2, T)
     diag = oc.quantize_into(ocache, Kf.astype(np.float64), Vf.astype(np.float64), ocodec, rope=rope)
-    ncache = native.alloc_cache(ncodec, 1, 2, 64)
+    ncache = native.alloc_cache(ncodec, 1, 2, T)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     native.quantize_kv(ncodec, tl.to_device(Kf, "fp32"), tl.to_device(Vf, "fp32"), ncache,
                        rope=tl.rope_device(rope), status=status)
@@ -114,7 +118,7 @@ def test_quantize_zero_and_nonfinite_rows():
     gpu = tl.download_cache(ncache)
     stats = tl.new_stats()
     for i, (b, h) in enumerate([(0, 0), (0, 1)]):
-        tl.compare_rows(gpu, ocache, ocodec, b, h, np.arange(64), diag["k"][i], diag["v"][i], stats)
+        tl.compare_rows(gpu, ocache, ocodec, b, h, np.arange(T), diag["k"][i], diag["v"][i], stats)
     tl.assert_mismatch_budget(stats)
     assert gpu["kscale"][0, 1, 5, 0] == 0 and gpu["vnorm"][0, 0, 9] == 0
 
