@@ -129,6 +129,33 @@ __device__ __forceinline__ void split3_store(uint8_t *base, uint32_t stride, int
   *reinterpret_cast<__nv_bfloat16 *>(base + 2 * stride + off) = c;
 }
 
+// Eight consecutive K elements (k0 a multiple of 8) of one row: the three
+// split planes are each one 16-byte core-matrix row, stored with one write.
+__device__ __forceinline__ void split3_store8(uint8_t *base, uint32_t stride, int off, const float (&v)[8]) {
+  uint32_t w0[4], w1[4], w2[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint32_t p0[2], p1[2], p2[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x = v[2 * e + h];
+      const __nv_bfloat16 a = __float2bfloat16_rn(x);
+      const float r1 = x - __bfloat162float(a);
+      const __nv_bfloat16 b = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 c = __float2bfloat16_rn(r1 - __bfloat162float(b));
+      p0[h] = __bfloat16_as_ushort(a);
+      p1[h] = __bfloat16_as_ushort(b);
+      p2[h] = __bfloat16_as_ushort(c);
+    }
+    w0[e] = p0[0] | (p0[1] << 16);
+    w1[e] = p1[0] | (p1[1] << 16);
+    w2[e] = p2[0] | (p2[1] << 16);
+  }
+  *reinterpret_cast<uint4 *>(base + off) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+  *reinterpret_cast<uint4 *>(base + stride + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+  *reinterpret_cast<uint4 *>(base + 2 * stride + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+}
+
 // The six split products of order <= 2: a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0
 // (about 2^-26 relative).  The five small ones go first into d_small; the
 // K steps of a0 b0 go round-robin into `nbig` accumulators d_big + i * dstride
@@ -228,20 +255,33 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
       const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
       if (half == 0) nuk[row] = ok ? nu : 0.f;
       const float qv = a.qjl_coef * rho;
+#pragma unroll 1
       for (int w = 0; w < D / 32; ++w) {
         uint32_t pw[4] = {0u, 0u, 0u, 0u};
-        for (int p = 0; p < planes_k; ++p) pw[p] = reinterpret_cast<const uint32_t *>(krow)[p * (D / 32) + w];
-        for (int bit = 0; bit < 32; ++bit) {
-          const int i = 32 * w + bit;
-          float val;
-          if (half == 0) {
-            int idx = 0;
-            for (int p = 0; p < mbk; ++p) idx |= ((pw[p] >> bit) & 1) << p;
-            val = ok ? cks[idx] : 0.f;
-          } else {
-            val = (ok && a.books.qjl) ? (((pw[mbk] >> bit) & 1) ? qv : -qv) : 0.f;
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (p < planes_k) pw[p] = reinterpret_cast<const uint32_t *>(krow)[p * (D / 32) + w];
+        uint32_t sgn = 0u;
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (p == mbk) sgn = pw[p];
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int bit = 8 * c8 + e;
+            if (half == 0) {
+              int idx = 0;
+#pragma unroll
+              for (int p = 0; p < 3; ++p)
+                if (p < mbk) idx |= ((pw[p] >> bit) & 1) << p;
+              v[e] = ok ? cks[idx] : 0.f;
+            } else {
+              v[e] = (ok && a.books.qjl) ? (((sgn >> bit) & 1) ? qv : -qv) : 0.f;
+            }
           }
-          split3_store(ks3, K_BYTES, kmaj16(row, half * D + i, BK), val);
+          split3_store8(ks3, K_BYTES, kmaj16(row, half * D + 32 * w + 8 * c8, BK), v);
         }
       }
     }
@@ -253,12 +293,19 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
         if (jg < a.T)
           for (int p = 0; p < nbv; ++p)
             vw[p] = a.vcode[(bh * (a.rows_cap / 32) + jg / 32) * nbv * D + p * D + coord];
-        for (int t = 0; t < 32; ++t) {
-          const int j = jg + t;
-          int idx = 0;
-          for (int p = 0; p < nbv; ++p) idx |= ((vw[p] >> t) & 1) << p;
-          const float val = j < a.T ? vns[32 * g + t] * cvs[idx] : 0.f;
-          split3_store(vs3, V_BYTES, kmaj16(coord, 32 * g + t, D), val);
+#pragma unroll
+        for (int t8 = 0; t8 < 4; ++t8) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int t = 8 * t8 + e;
+            int idx = 0;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+              if (p < nbv) idx |= ((vw[p] >> t) & 1) << p;
+            v[e] = jg + t < a.T ? vns[32 * g + t] * cvs[idx] : 0.f;
+          }
+          split3_store8(vs3, V_BYTES, kmaj16(coord, 32 * g + 8 * t8, D), v);
         }
       }
     }
@@ -276,36 +323,49 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
-    float sv[BK];
-#pragma unroll
-    for (int c = 0; c < BK; c += 16) {
+    // scores of 16 keys (c .. c+15) of this query row from the five accumulators
+    auto scores16 = [&](int c, float (&v)[16]) {
       uint32_t r[16];
       sm100::tmem_ld16(sm100::tmem_lane(tS + c, warp), r);
       sm100::wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) sv[c + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
 #pragma unroll
       for (int i = 0; i < NBIG; ++i) {
         sm100::tmem_ld16(sm100::tmem_lane(tSb + i * BK + c, warp), r);
         sm100::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c + e] += __uint_as_float(r[e]);
+        for (int e = 0; e < 16; ++e) v[e] += __uint_as_float(r[e]);
       }
-    }
-    float tmax = -CUDART_INF_F;
 #pragma unroll
-    for (int c = 0; c < BK; ++c) {
-      sv[c] = j0 + c < a.T ? a.scale * nuk[c] * sv[c] : -CUDART_INF_F;
-      tmax = fmaxf(tmax, sv[c]);
+      for (int e = 0; e < 16; ++e) v[e] = j0 + c + e < a.T ? a.scale * nuk[c + e] * v[e] : -CUDART_INF_F;
+    };
+    // pass 1: the tile's maximum; pass 2: probabilities into the P planes
+    float tmax = -CUDART_INF_F;
+#pragma unroll 1
+    for (int c = 0; c < BK; c += 16) {
+      float v[16];
+      scores16(c, v);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) tmax = fmaxf(tmax, v[e]);
     }
     const float mn = fmaxf(m, tmax);
     const float corr = __expf(m - mn);
     float ps = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BK; c += 16) {
+      float v[16];
+      scores16(c, v);
 #pragma unroll
-    for (int c = 0; c < BK; ++c) {
-      const float p = __expf(sv[c] - mn);
-      ps += p;
-      split3_store(ps3, P_BYTES, kmaj16(tid, c, BQ), p);
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          w[e] = __expf(v[8 * h8 + e] - mn);
+          ps += w[e];
+        }
+        split3_store8(ps3, P_BYTES, kmaj16(tid, c + 8 * h8, BQ), w);
+      }
     }
     l = l * corr + ps;
     m = mn;
