@@ -44,6 +44,11 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
+                                      "vector_search"],
+                   help="run one extra workload alone and print its JSON (1 GPU)")
+    p.add_argument("--search-rows", type=int, default=0,
+                   help="vector-search database rows for --only vector_search (default 10^6)")
     return p.parse_args()
 
 
@@ -524,7 +529,7 @@ def search_extra(pk: dict, steps: int = 5):
         scan_topk=dict(ms_per_call=s_ * 1e3, queries_per_s=w.nq / s_,
                        roofline=dict(bound="tensor", achieved=scan_flops / k / 1e12, peak=pk["bf16"],
                                      unit="TFLOP/s", frac=scan_flops / k / 1e12 / pk["bf16"],
-                                     algorithmic_flops=scan_flops, kernel="ix_scan_kernel",
+                                     algorithmic_flops=scan_flops, kernel="ix_scan2_kernel",
                                      kernel_ms=k * 1e3)),
         l2="database codes 772 MB and input 6.1 GB > L2")
 
@@ -644,8 +649,30 @@ def smi_index(local: int) -> str:
     return str(local)
 
 
+def run_only(args) -> int:
+    """One extra workload on its own (profiling entry point)."""
+    from rotated_codebook_kv_tq_b200.build import build
+    build()
+    pk = peaks()
+    if args.only == "quantize_esm_prefill":
+        r = quantize_extra("esm_prefill", pk, steps=3)
+    elif args.only == "bidir_esm_prefill":
+        r = bidir_extra(pk, steps=1)
+    elif args.only == "decode_long_context":
+        r = decode_extra("long_decode", pk, steps=5, warmup=3)
+    else:
+        from rotated_codebook_kv_tq_b200 import synth
+        if args.search_rows:
+            synth.VECTOR_SEARCH = synth.VECTOR_SEARCH.scaled(n=args.search_rows)
+        r = search_extra(pk, steps=1)
+    print(json.dumps({args.only: r}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.only:
+        return run_only(args)
     world, rank, local = dist_init()
     if args.impl == "reference":
         return run_reference(args, world, rank)
@@ -685,8 +712,8 @@ def main():
                                f"({n_sets * per_set / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)",
                             parallelism=f"{world} independent replicas" if world > 1 else "1 GPU"),
                 roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
-                              frac=achieved / pk["hbm"], traffic=ncu_traffic("chunk_kernel"),
-                              kernel="chunk_kernel (split-K decode main loop)",
+                              frac=achieved / pk["hbm"], traffic=ncu_traffic("tc_chunk_kernel"),
+                              kernel="tc_chunk_kernel (split-K decode main loop, tcgen05)",
                               kernel_us=kern * 1e6, algorithmic_bytes=alg,
                               bytes_per_token_head=row_bytes(w),
                               peak_source=f"{pk['source']} hbm_gbs"),
