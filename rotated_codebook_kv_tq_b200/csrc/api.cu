@@ -149,20 +149,32 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   c->books.bits_v = c->bits_v;
 
   c->ST_dev = nullptr;
+  c->S_tile = nullptr;
   if (c->qjl_k) {
     const size_t n = static_cast<size_t>(c->d) * c->d;
-    std::vector<uint16_t> both(2 * n);
+    // S, S^T, and for d = 1536 (vector search) S again as the sketch GEMM's B
+    // operand: K-major core-matrix tiles of 256 output rows x 64 inputs,
+    // tile (i / 256, j / 64) at ((i / 256) * (d / 64) + j / 64) * 32 KB
+    const bool tiled = c->d == 1536;
+    std::vector<uint16_t> both((tiled ? 3 : 2) * n);
     for (int i = 0; i < c->d; ++i)
       for (int j = 0; j < c->d; ++j) {
-        both[static_cast<size_t>(i) * c->d + j] = desc->qjl_bf16[static_cast<size_t>(i) * c->d + j];
-        both[n + static_cast<size_t>(j) * c->d + i] = desc->qjl_bf16[static_cast<size_t>(i) * c->d + j];
+        const uint16_t v = desc->qjl_bf16[static_cast<size_t>(i) * c->d + j];
+        both[static_cast<size_t>(i) * c->d + j] = v;
+        both[n + static_cast<size_t>(j) * c->d + i] = v;
+        if (tiled) {
+          const size_t tile = static_cast<size_t>(i / 256) * (c->d / 64) + j / 64;
+          const size_t off = tile * 16384 + ((j % 64) / 8) * 2048 + ((i % 256) / 8) * 64 + (i % 8) * 8 + j % 8;
+          both[2 * n + off] = v;
+        }
       }
-    if (cudaMalloc(&c->S_dev, 2 * n * sizeof(uint16_t)) != cudaSuccess) {
+    if (cudaMalloc(&c->S_dev, both.size() * sizeof(uint16_t)) != cudaSuccess) {
       delete c;
       return tq_check_launch("codec: cudaMalloc");
     }
     c->ST_dev = c->S_dev + n;
-    if (cudaMemcpy(c->S_dev, both.data(), 2 * n * sizeof(uint16_t), cudaMemcpyHostToDevice) !=
+    if (tiled) c->S_tile = c->S_dev + 2 * n;
+    if (cudaMemcpy(c->S_dev, both.data(), both.size() * sizeof(uint16_t), cudaMemcpyHostToDevice) !=
         cudaSuccess) {
       cudaFree(c->S_dev);
       delete c;

@@ -39,7 +39,7 @@ struct IxArgs {
   int64_t n;
   uint8_t *kcode;        // [n][planes][XD/8]
   uint16_t *kscale;      // [n][2]
-  uint16_t *rbuf;        // [n][2*XD] bf16 residual hi | lo
+  uint16_t *rbuf;        // residual hi | lo, tiled for ix_sketch_kernel (rows rounded up to 128)
   uint32_t h12[XNB];     // row masks of H_12: bit j set <=> entry -1
   uint32_t dneg[XW];
   float ck[TQ_MAX_LEVELS], tk[TQ_MAX_LEVELS];
@@ -109,7 +109,9 @@ __global__ void __launch_bounds__(256) ix_encode_kernel(IxArgs a) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) mw[p][0] = mw[p][1] = 0u;
     float r2 = 0.f;
-    uint16_t *rrow = a.rbuf + row * 2 * XD;
+    // residual hi | lo in the sketch GEMM's A layout: K-major core-matrix
+    // tiles of 128 rows x 64 K elements (16 KB), tile (row / 128, k / 64)
+    uint16_t *rtile = a.rbuf + (row >> 7) * (2 * XD / 64) * 8192 + ((row & 127) >> 3) * 64 + (row & 7) * 8;
 #pragma unroll
     for (int j1 = 0; j1 < XNB; ++j1)
 #pragma unroll
@@ -129,8 +131,9 @@ __global__ void __launch_bounds__(256) ix_encode_kernel(IxArgs a) {
         const __nv_bfloat16 hi = __float2bfloat16_rn(r);
         const __nv_bfloat16 lo = __float2bfloat16_rn(r - __bfloat162float(hi));
         const int i = 128 * j1 + 32 * k + lane;
-        rrow[i] = __bfloat16_as_ushort(hi);
-        rrow[XD + i] = __bfloat16_as_ushort(lo);
+        const int kl = XD + i;
+        rtile[(i >> 6) * 8192 + ((i & 63) >> 3) * 1024 + (i & 7)] = __bfloat16_as_ushort(hi);
+        rtile[(kl >> 6) * 8192 + ((kl & 63) >> 3) * 1024 + (kl & 7)] = __bfloat16_as_ushort(lo);
       }
     const float rho = sqrtf(tq_warp_sum(r2));
     uint32_t *krow = reinterpret_cast<uint32_t *>(a.kcode + row * planes * (XD / 8));
@@ -148,21 +151,157 @@ __global__ void __launch_bounds__(256) ix_encode_kernel(IxArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Index-build sketch: sign(S r) for every residual row as one GEMM on the
+// tensor cores, z = [r_hi | r_lo] [S | S]^T (S is exactly bf16).  Both
+// operands sit in global memory as K-major core-matrix tiles (A: 128 rows x
+// 64 K = 16 KB, written by ix_encode_kernel; B: 256 rows of S x 64 K = 32 KB,
+// built with the codec), so one warp streams them into a 4-stage shared ring
+// with cp.async.bulk and issues M128 x N256 kind::f16 MMAs into one of two
+// fp32 accumulators in TMEM; four epilogue warps turn the other accumulator
+// into sign words.  Persistent CTAs walk (m tile, n tile) pairs, m-major, so
+// the six n tiles of an m tile run at the same time and share its A tiles in L2.
+// ---------------------------------------------------------------------------
+constexpr int SKN_T = XD / 256;                 // 6 n tiles
+constexpr int SKA_CH = 2 * XD / 64;             // 48 A chunks (hi | lo)
+constexpr int SKB_CH = XD / 64;                 // 24 B chunks
+constexpr uint32_t SKA_BYTES = 128 * 64 * 2;
+constexpr uint32_t SKB_BYTES = 256 * 64 * 2;
+constexpr int SKS = 4;                          // ring stages
+constexpr int SK_T = 5 * 32;                    // 4 epilogue warps + the MMA warp
+constexpr uint32_t SK_SMEM = SKS * (SKA_BYTES + SKB_BYTES);
+
+struct SketchArgs {
+  const uint16_t *A;      // residual tiles of this batch
+  const uint16_t *B;      // S tiles
+  int64_t M;              // rows in the batch
+  uint8_t *plane;         // sign plane of row 0 of the batch; row stride plane_stride bytes
+  int64_t plane_stride;
+  uint32_t *status;
+};
+
+__global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
+  extern __shared__ __align__(1024) uint8_t skm[];
+  __shared__ __align__(8) uint64_t full[SKS], empty[SKS], acc_full[2], acc_free[2];
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (warp == 0) sm100::tmem_alloc(&tmem_s, 512);
+  if (tid == 0) {
+    for (int s = 0; s < SKS; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(&acc_full[b], 1);
+      sm100::mbar_init(&acc_free[b], 4);
+    }
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  const uint32_t tm = tmem_s;
+  const int64_t tiles = (g.M + 127) / 128 * SKN_T;
+  const int ntl = tiles > blockIdx.x ? static_cast<int>((tiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  const int total = ntl * SKA_CH;
+  if (warp == 4) {
+    if (lane == 0 && total > 0) {
+      auto copy = [&](int gc) {
+        const int tl = gc / SKA_CH, c = gc % SKA_CH, s = gc % SKS;
+        const int64_t t = blockIdx.x + static_cast<int64_t>(tl) * gridDim.x;
+        const int64_t mt = t / SKN_T;
+        const int nt = static_cast<int>(t % SKN_T);
+        uint8_t *dst = skm + s * (SKA_BYTES + SKB_BYTES);
+        sm100::mbar_expect_tx(&full[s], SKA_BYTES + SKB_BYTES);
+        sm100::bulk_g2s(dst, g.A + (mt * SKA_CH + c) * (SKA_BYTES / 2), SKA_BYTES, &full[s]);
+        sm100::bulk_g2s(dst + SKA_BYTES, g.B + (static_cast<int64_t>(nt) * SKB_CH + c % SKB_CH) * (SKB_BYTES / 2),
+                        SKB_BYTES, &full[s]);
+      };
+      for (int gc = 0; gc < SKS - 1 && gc < total; ++gc) copy(gc);
+      constexpr uint32_t IDESC = sm100::idesc_bf16(128, 256);
+      bool ok = true;
+      for (int tl = 0; tl < ntl && ok; ++tl) {
+        const int ab = tl & 1;
+        if (tl >= 2) {
+          ok = sm100::mbar_wait(&acc_free[ab], ((tl >> 1) - 1) & 1);
+          if (!ok) break;
+          sm100::fence_after_sync();
+        }
+        for (int c = 0; c < SKA_CH && ok; ++c) {
+          const int gc = tl * SKA_CH + c, s = gc % SKS;
+          ok = sm100::mbar_wait(&full[s], (gc / SKS) & 1);
+          if (!ok) break;
+          sm100::fence_after_sync();
+          const uint32_t a_addr = sm100::smem_addr(skm + s * (SKA_BYTES + SKB_BYTES));
+          const uint32_t b_addr = a_addr + SKA_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            sm100::mma_bf16_ss(tm + ab * 256, sm100::smem_desc(a_addr + kk * 2 * 2048, 2048, 128),
+                               sm100::smem_desc(b_addr + kk * 2 * 4096, 4096, 128), IDESC,
+                               (c > 0 || kk > 0) ? 1u : 0u);
+          sm100::mma_commit(&empty[s]);
+          if (c == SKA_CH - 1) sm100::mma_commit(&acc_full[ab]);
+          // refill: chunk gc + SKS - 1 reuses the stage of chunk gc - 1
+          const int gn = gc + SKS - 1;
+          if (gn < total) {
+            if (gn >= SKS) {
+              ok = sm100::mbar_wait(&empty[gn % SKS], ((gn / SKS) - 1) & 1);
+              if (!ok) break;
+            }
+            copy(gn);
+          }
+        }
+      }
+      if (!ok) abort_s = 1;
+    }
+    __syncwarp();
+  } else {
+    // epilogue warp = TMEM lane quarter: row 32 warp + lane of the m tile
+    for (int tl = 0; tl < ntl; ++tl) {
+      const int ab = tl & 1;
+      if (lane == 0 && !abort_s && !sm100::mbar_wait(&acc_full[ab], (tl >> 1) & 1)) abort_s = 1;
+      __syncwarp();
+      sm100::fence_after_sync();
+      const int64_t t = blockIdx.x + static_cast<int64_t>(tl) * gridDim.x;
+      const int64_t row = (t / SKN_T) * 128 + 32 * warp + lane;
+      const int nt = static_cast<int>(t % SKN_T);
+      uint32_t *dst = reinterpret_cast<uint32_t *>(g.plane + row * g.plane_stride) + nt * 8;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t z[32];
+        sm100::tmem_ld32(sm100::tmem_lane(tm + ab * 256 + 32 * cc, warp), z);
+        sm100::wait_ld();
+        uint32_t word = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) word |= (__uint_as_float(z[e]) >= 0.f ? 1u : 0u) << e;
+        if (row < g.M) dst[cc] = word;
+      }
+      sm100::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&acc_free[ab]);
+    }
+  }
+  if (abort_s && tid == 0 && g.status) atomicAdd(g.status, 1u << 31);
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  if (warp == 0) sm100::tmem_dealloc(tm, 512);
+}
+
+// ---------------------------------------------------------------------------
 // C = A B^T on the tensor cores for A [M][KA] and B [N][KB] bf16 row-major
 // (K contiguous), KA a multiple of KB: A's K range wraps over B (A = [r_hi |
 // r_lo] against B = S gives S r_hi + S r_lo).  Tile 128 x 256, K chunks of 64
-// through a 3-stage cp.async ring; fp32 accumulators in 256 TMEM columns.
-// MODE 0 writes sign bits (z >= 0) of each row into a bit plane; MODE 1 writes
-// the fp32 values.
+// through a 3-stage cp.async ring; fp32 accumulators in 256 TMEM columns,
+// written out as fp32 (the scan's q'' = S q' for a block of queries).
 // ---------------------------------------------------------------------------
 struct GemmArgs {
   const uint16_t *A;
   const uint16_t *B;
   int64_t M;
   int N, KA, KB;
-  uint8_t *plane;        // MODE 0: bit plane base, row stride plane_stride bytes
-  int64_t plane_stride;
-  float *out;            // MODE 1: [M][N]
+  float *out;            // [M][N]
   uint32_t *status;
 };
 
@@ -179,7 +318,6 @@ __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <int MODE>
 __global__ void __launch_bounds__(128, 1) ix_gemm_kernel(GemmArgs g) {
   extern __shared__ __align__(128) float gsm[];
   uint8_t *base = reinterpret_cast<uint8_t *>(gsm);
@@ -271,21 +409,11 @@ __global__ void __launch_bounds__(128, 1) ix_gemm_kernel(GemmArgs g) {
       sm100::tmem_ld16(sm100::tmem_lane(tm + c0 + 16, warp), z1);
       sm100::wait_ld();
       if (row < g.M && n0 + c0 < g.N) {
-        if (MODE == 0) {
-          uint32_t word = 0u;
+        float *o = g.out + row * g.N + n0 + c0;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            word |= (__uint_as_float(z0[c]) >= 0.f ? 1u : 0u) << c;
-            word |= (__uint_as_float(z1[c]) >= 0.f ? 1u : 0u) << (16 + c);
-          }
-          reinterpret_cast<uint32_t *>(g.plane + row * g.plane_stride)[(n0 + c0) >> 5] = word;
-        } else {
-          float *o = g.out + row * g.N + n0 + c0;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (n0 + c0 + c < g.N) o[c] = __uint_as_float(z0[c]);
-            if (n0 + c0 + 16 + c < g.N) o[16 + c] = __uint_as_float(z1[c]);
-          }
+        for (int c = 0; c < 16; ++c) {
+          if (n0 + c0 + c < g.N) o[c] = __uint_as_float(z0[c]);
+          if (n0 + c0 + 16 + c < g.N) o[16 + c] = __uint_as_float(z1[c]);
         }
       }
     }
@@ -723,20 +851,19 @@ int sm_count() {
   return sms;
 }
 
-template <int MODE>
 int run_gemm(const GemmArgs &g, cudaStream_t stream) {
   constexpr int shm = GST * (GA_BYTES + GB_BYTES);
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !done[dev]) {
-    if (cudaFuncSetAttribute(ix_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, shm) !=
+    if (cudaFuncSetAttribute(ix_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shm) !=
         cudaSuccess)
       return tq_check_launch("cudaFuncSetAttribute(ix_gemm)");
     done[dev] = true;
   }
   dim3 grid(static_cast<unsigned>((g.M + GM - 1) / GM), (g.N + GN - 1) / GN);
-  ix_gemm_kernel<MODE><<<grid, 128, shm, stream>>>(g);
+  ix_gemm_kernel<<<grid, 128, shm, stream>>>(g);
   tq_count_launch(1);
   return tq_check_launch("ix_gemm_kernel");
 }
@@ -765,7 +892,7 @@ extern "C" {
 int tq_index_workspace(const tq_codec *c, int64_t n, size_t *bytes) {
   if (!c || !bytes || n < 1) return tq_fail(TQ_ERR_INVALID_ARG, "index workspace: bad arguments");
   const int64_t rows = n < kIxBatch ? n : kIxBatch;
-  *bytes = static_cast<size_t>(rows) * 2 * XD * sizeof(uint16_t);
+  *bytes = static_cast<size_t>((rows + 127) / 128 * 128) * 2 * XD * sizeof(uint16_t);   // whole 128-row tiles
   return TQ_OK;
 }
 
@@ -804,18 +931,27 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
     ix_encode_kernel<<<static_cast<int>(blocks < 16LL * sm_count() ? blocks : 16LL * sm_count()), 256, 0, st>>>(a);
     tq_count_launch(1);
     if (int e = tq_check_launch("ix_encode_kernel")) return e;
-    GemmArgs g;
+    SketchArgs g;
     g.A = a.rbuf;
-    g.B = c->S_dev;
+    g.B = c->S_tile;
     g.M = rows;
-    g.N = XD;
-    g.KA = 2 * XD;
-    g.KB = XD;
     g.plane = a.kcode + c->mse_bits_k * (XD / 8);
     g.plane_stride = planes * (XD / 8);
-    g.out = nullptr;
     g.status = status;
-    if (int e = run_gemm<0>(g, st)) return e;
+    static bool sk_attr[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !sk_attr[dev]) {
+      if (cudaFuncSetAttribute(ix_sketch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(SK_SMEM)) != cudaSuccess)
+        return tq_check_launch("cudaFuncSetAttribute(ix_sketch)");
+      sk_attr[dev] = true;
+    }
+    const int64_t sk_tiles = (rows + 127) / 128 * SKN_T;
+    const int sk_grid = static_cast<int>(sk_tiles < sm_count() ? sk_tiles : sm_count());
+    ix_sketch_kernel<<<sk_grid, SK_T, SK_SMEM, st>>>(g);
+    tq_count_launch(1);
+    if (int e = tq_check_launch("ix_sketch_kernel")) return e;
   }
   return TQ_OK;
 }
@@ -901,11 +1037,9 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   g.N = XD;
   g.KA = 2 * XD;
   g.KB = XD;
-  g.plane = nullptr;
-  g.plane_stride = 0;
   g.out = q2;
   g.status = nullptr;
-  if (int e = run_gemm<1>(g, st)) return e;
+  if (int e = run_gemm(g, st)) return e;
   // fp16 B operand with a power-of-two scale per query
   const float coef = sqrtf(static_cast<float>(M_PI) / 2.0f) / XD;
   QpackArgs pa;

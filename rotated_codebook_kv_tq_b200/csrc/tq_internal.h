@@ -36,6 +36,7 @@ struct tq_codec {
   TqBooks books;
   uint16_t *S_dev;     // bf16 [d][d] row-major S[i][j]
   uint16_t *ST_dev;    // bf16 [d][d] transpose, ST[j][i] = S[i][j] (same allocation)
+  uint16_t *S_tile;    // d = 1536 only: S as 256 x 64 K-major core-matrix tiles (same allocation)
   // Walsh expansion of the odd-symmetric codebooks: c[idx] = sum_t a_t (2 x_t - 1)
   // over the odd subsets of the code bits (tensor-core decode path)
   float walsh_k[8], walsh_v[8];
