@@ -23,6 +23,8 @@
 
 namespace {
 
+constexpr int CMB = 4;   // thread groups of combine_kernel (each sums every 4th split)
+
 constexpr int CT = 256;       // threads of the chunk kernel
 
 struct DecodeArgs {
@@ -286,25 +288,29 @@ __global__ void __launch_bounds__(CT) chunk_kernel(DecodeArgs a) {
 // thread i sums coordinate i over the chunks, then warp 0 applies
 // Pi^T = D H / sqrt(d) and the 1/l normalisation.
 template <int D>
-__global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
+  // CMB groups of D threads: group gq sums splits gq, gq + CMB, ... of every
+  // coordinate (short independent load chains), then the groups are added
   constexpr int NPL = D / 32;
   constexpr int MAXS = 512;
+  constexpr int NT = CMB * D;
   __shared__ float fs[MAXS];
-  __shared__ float red[D / 32][2];
-  __shared__ float os[D];
+  __shared__ float red[NT / 32][2];
+  __shared__ float os[CMB][D];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid % D, gq = tid / D;
   const int64_t head = blockIdx.x;
   const int S = a.splits;
   float m = -CUDART_INF_F;
-  for (int s = tid; s < S; s += D) m = fmaxf(m, a.pml[(head * S + s) * 2]);
+  for (int s = tid; s < S; s += NT) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
   if (lane == 0) red[warp][0] = m;
   __syncthreads();
   float M = red[0][0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w][0]);
+  for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w][0]);
   float l = 0.f;
-  for (int s = tid; s < S; s += D) {
+  for (int s = tid; s < S; s += NT) {
     const float ls = a.pml[(head * S + s) * 2 + 1];
     const float f = ls > 0.f ? __expf(a.pml[(head * S + s) * 2] - M) : 0.f;
     fs[s] = f;
@@ -316,21 +322,26 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
   __syncthreads();
   float L = 0.f;
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) L += red[w][1];
+  for (int w = 0; w < NT / 32; ++w) L += red[w][1];
   float o0 = 0.f, o1 = 0.f;
-  const float *po = a.po + head * S * D + tid;
-  int s = 0;
-  for (; s + 1 < S; s += 2) {
+  const float *po = a.po + head * S * D + c;
+  int s = gq;
+  for (; s + CMB < S; s += 2 * CMB) {
     o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
-    o1 = fmaf(po[static_cast<int64_t>(s + 1) * D], fs[s + 1], o1);
+    o1 = fmaf(po[static_cast<int64_t>(s + CMB) * D], fs[s + CMB], o1);
   }
   if (s < S) o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
-  os[tid] = o0 + o1;
+  os[gq][c] = o0 + o1;
   __syncthreads();
   if (warp == 0) {
     float x[NPL];
 #pragma unroll
-    for (int k = 0; k < NPL; ++k) x[k] = os[lane + 32 * k];
+    for (int k = 0; k < NPL; ++k) {
+      float v = 0.f;
+#pragma unroll
+      for (int g = 0; g < CMB; ++g) v += os[g][lane + 32 * k];
+      x[k] = v;
+    }
     tq_warp_wht<NPL>(x, lane);
     tq_apply_signs<NPL>(x, a.books.dneg, lane);
     const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * L);
@@ -365,7 +376,7 @@ int run_decode(DecodeArgs &a, cudaStream_t stream) {
   }
   if (int e = tq_check_launch("chunk_kernel")) return e;
   if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
-  combine_kernel<D><<<heads, D, 0, stream>>>(a);
+  combine_kernel<D><<<heads, CMB * D, 0, stream>>>(a);
   tq_count_launch(3);
   return tq_check_launch("combine_kernel");
 }
@@ -436,7 +447,7 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
     if (int e = launch_decode_tc(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_len, scale, rc,
                                  rs, splits, a.po, a.pml, bk, logits, stream))
       return e;
-    combine_kernel<128><<<B * Hq, 128, 0, stream>>>(a);
+    combine_kernel<128><<<B * Hq, CMB * 128, 0, stream>>>(a);
     tq_count_launch(1);
     return tq_check_launch("combine_kernel");
   }
