@@ -2,8 +2,8 @@
 codecs from a workload, move seeded inputs to the device, upload an oracle
 cache, and compare codes under the boundary-window rule.
 
-Tolerances (from the benchmark spec's north star, with the readings listed in
-DESIGN.md):
+Tolerances (the acceptance bars of the hot path, with the boundary window
+measured on the unit-variance scale):
 * codes and signs bit-exact, except coordinates whose rotated value lies
   within 1e-5 (unit-variance scale: sqrt(d) * |u - t|) of a decision
   threshold, or signs with |S r|_i / rho < 1e-5; mismatches must all be in the
