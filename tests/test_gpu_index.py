@@ -201,3 +201,43 @@ def test_vector_search_fullsize_sampled(codecs):
         kth = gv[qi, -1]
         better = pool[sp > kth + 2 * tol]
         assert set(better.tolist()) <= set(gi[qi].tolist()), qi
+
+
+@pytest.mark.parametrize("bits", [2, 3])   # key MSE bits 1 and 2 (+ QJL)
+def test_index_and_scan_other_bit_widths(bits):
+    """Index build and scan parity for the narrower key codecs the
+    vector-search calls accept (the 4-bit default covers 3 MSE bits)."""
+    w = synth.VECTOR_SEARCH
+    Dv = synth.rotation_signs(D, w.seed)
+    S = synth.qjl_matrix_bf16(D, w.seed)
+    ocodec = oc.make_codec(D, bits, True, 4, Dv, S)
+    ncodec = native.Codec(D, bits, True, 4, Dv, S)
+    n, nq, k = 700, 70, 10
+    x = synth.unit_rows(n, D, 80 + bits, 0)
+    kcode, kscale, status = _encode_gpu(ncodec, torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    enc = oc.quantize_keys(x.astype(np.float64), ocodec)
+    stats = tl.new_stats()
+    _check_codes(ocodec, kcode.cpu().numpy(), kscale.cpu().numpy(), enc, stats)
+    tl.assert_mismatch_budget(stats)
+    # scan over the oracle's own codes
+    kc, ks = oc.pack_keys(enc, ocodec)
+    q = synth.unit_rows(nq, D, 80 + bits, 2)
+    s = oscan.scores(q.astype(np.float64), kc, ks, ocodec)
+    idx = torch.empty((nq, k), dtype=torch.int32, device="cuda")
+    score = torch.empty((nq, k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(native.scan_workspace(ncodec, n, nq, k), dtype=torch.uint8, device="cuda")
+    native.scan_topk(ncodec, torch.from_numpy(kc).cuda(), torch.from_numpy(ks).cuda(),
+                     torch.from_numpy(q).cuda(), k, idx, score, ws)
+    torch.cuda.synchronize()
+    exact = _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k)
+    assert exact >= nq - max(1, nq // 10)
+
+
+def test_index_rejects_four_mse_bits():
+    Dv = synth.rotation_signs(D, 4)
+    ncodec = native.Codec(D, 5, True, 4, Dv, synth.qjl_matrix_bf16(D, 4))
+    x = torch.zeros((8, D), device="cuda")
+    with pytest.raises(native.TqError) as e:
+        _encode_gpu(ncodec, x)
+    assert e.value.code == native.TQ_ERR_UNSUPPORTED
