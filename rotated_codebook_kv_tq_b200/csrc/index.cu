@@ -67,7 +67,7 @@ __device__ __forceinline__ void rotate1536(float (&x)[XNB][4], const uint32_t (&
   }
 }
 
-__global__ void __launch_bounds__(256) ix_encode_kernel(IxArgs a) {
+__global__ void __launch_bounds__(256, 2) ix_encode_kernel(IxArgs a) {
   __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x < TQ_MAX_LEVELS) {
