@@ -40,16 +40,25 @@ struct IxArgs {
   uint8_t *kcode;        // [n][planes][XD/8]
   uint16_t *kscale;      // [n][2]
   uint16_t *rbuf;        // residual hi | lo, tiled for ix_sketch_kernel (rows rounded up to 128)
-  uint32_t h12[XNB];     // row masks of H_12: bit j set <=> entry -1
   uint32_t dneg[XW];
   float ck[TQ_MAX_LEVELS], tk[TQ_MAX_LEVELS];
   int mbk;
   uint32_t *status;
 };
 
+// Sign of entry (i, j) of the Paley (type I) Hadamard matrix of order 12
+// built from the quadratic residues {1, 3, 4, 5, 9} of GF(11): row 0 is all
+// +1, column 0 is -1 below row 0, the diagonal is +1 and entry (i, j) of the
+// remaining 11 x 11 core is the Legendre symbol of (j - i) mod 11.  Called
+// with constant indices only, so every sign folds at compile time.
+__host__ __device__ __forceinline__ constexpr bool h12_neg(int i, int j) {
+  return i == 0 || i == j ? false
+         : j == 0         ? true
+                          : ((0x23Au >> (((j - i) % 11 + 11) % 11)) & 1u) == 0u;
+}
+
 // x[j1][k] holds coordinate 128 j1 + 32 k + lane; y = (H_12 kron H_128) x.
-__device__ __forceinline__ void rotate1536(float (&x)[XNB][4], const uint32_t (&h12)[XNB],
-                                           int lane) {
+__device__ __forceinline__ void rotate1536(float (&x)[XNB][4], int lane) {
 #pragma unroll
   for (int j1 = 0; j1 < XNB; ++j1) tq_warp_wht<4>(x[j1], lane);
 #pragma unroll
@@ -59,7 +68,7 @@ __device__ __forceinline__ void rotate1536(float (&x)[XNB][4], const uint32_t (&
     for (int i1 = 0; i1 < XNB; ++i1) {
       float s = 0.f;
 #pragma unroll
-      for (int j1 = 0; j1 < XNB; ++j1) s += ((h12[i1] >> j1) & 1) ? -x[j1][k] : x[j1][k];
+      for (int j1 = 0; j1 < XNB; ++j1) s += h12_neg(i1, j1) ? -x[j1][k] : x[j1][k];
       t[i1] = s;
     }
 #pragma unroll
@@ -103,7 +112,7 @@ __global__ void __launch_bounds__(256, 2) ix_encode_kernel(IxArgs a) {
         const uint32_t neg = (a.dneg[4 * j1 + k] >> lane) & 1u;
         x[j1][k] = zero ? 0.f : __uint_as_float(__float_as_uint(x[j1][k]) ^ (neg << 31));
       }
-    rotate1536(x, a.h12, lane);
+    rotate1536(x, lane);
     const float inv = zero ? 0.f : 1.0f / (sqrtf(static_cast<float>(XD)) * nu);
     uint32_t mw[4][2];
 #pragma unroll
@@ -434,7 +443,6 @@ struct QrotArgs {
   int nq;
   float *q1;            // [nq][XD]
   uint16_t *q1hl;       // [nq][2 XD] bf16 hi | lo
-  uint32_t h12[XNB];
   uint32_t dneg[XW];
 };
 
@@ -451,7 +459,7 @@ __global__ void __launch_bounds__(256) ix_qrot_kernel(QrotArgs a) {
       const float v = a.q[static_cast<int64_t>(qi) * XD + 128 * j1 + 32 * k + lane];
       x[j1][k] = __uint_as_float(__float_as_uint(v) ^ (neg << 31));
     }
-  rotate1536(x, a.h12, lane);
+  rotate1536(x, lane);
   const float inv = 1.0f / sqrtf(static_cast<float>(XD));
 #pragma unroll
   for (int j1 = 0; j1 < XNB; ++j1)
@@ -822,28 +830,6 @@ constexpr int64_t kIxBatch = 65536;   // rows encoded per residual-scratch batch
 
 // Paley construction I for q = 11: H = I + [[0, 1^T], [-1, Q]] with the
 // Jacobsthal matrix Q[i][j] = chi(j - i) of the quadratic character mod 11.
-void paley12(uint32_t masks[12]) {
-  int chi[11] = {0};
-  for (int x = 1; x < 11; ++x) chi[(x * x) % 11] = 1;
-  for (int a = 1; a < 11; ++a)
-    if (chi[a] != 1) chi[a] = -1;
-  int h[12][12];
-  for (int i = 0; i < 12; ++i)
-    for (int j = 0; j < 12; ++j) h[i][j] = 0;
-  for (int j = 1; j < 12; ++j) {
-    h[0][j] = 1;
-    h[j][0] = -1;
-  }
-  for (int i = 0; i < 11; ++i)
-    for (int j = 0; j < 11; ++j) h[i + 1][j + 1] = chi[((j - i) % 11 + 11) % 11];
-  for (int i = 0; i < 12; ++i) h[i][i] += 1;
-  for (int i = 0; i < 12; ++i) {
-    masks[i] = 0;
-    for (int j = 0; j < 12; ++j)
-      if (h[i][j] < 0) masks[i] |= 1u << j;
-  }
-}
-
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -912,7 +898,6 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   IxArgs a;
   a.mbk = c->mse_bits_k;
-  paley12(a.h12);
   for (int i = 0; i < XW; ++i) a.dneg[i] = c->books.dneg[i];
   for (int i = 0; i < TQ_MAX_LEVELS; ++i) {
     a.ck[i] = c->books.ck[i];
@@ -1024,7 +1009,6 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   qa.nq = nq;
   qa.q1 = q1;
   qa.q1hl = q1hl;
-  paley12(qa.h12);
   for (int i = 0; i < XW; ++i) qa.dneg[i] = c->books.dneg[i];
   ix_qrot_kernel<<<(nq + 7) / 8, 256, 0, st>>>(qa);
   tq_count_launch(1);
