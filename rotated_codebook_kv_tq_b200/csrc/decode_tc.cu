@@ -217,11 +217,13 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
           make_uint4(wv[l][0], wv[l][1], wv[l][2], wv[l][3]);
   }
   // rows beyond the G heads' limbs (N > 4 G) are zero
-  for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
-    const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
-    const bool mse = kc < NKM;
-    const int kb = mse ? kc * 16 : (kc - NKM) * 16;
-    *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (N > 4 * G) {
+    for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
+      const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
+      const bool mse = kc < NKM;
+      const int kb = mse ? kc * 16 : (kc - NKM) * 16;
+      *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
   // constants: C = sum of the quantized B values / (2F), per head and part
   {

@@ -60,15 +60,15 @@ __host__ __device__ __forceinline__ constexpr bool h12_neg(int i, int j) {
 // x[j1][k] holds coordinate 128 j1 + 32 k + lane; y = (H_12 kron H_128) x.
 __device__ __forceinline__ void rotate1536(float (&x)[XNB][4], int lane) {
 #pragma unroll
-  for (int j1 = 0; j1 < XNB; ++j1) tq_warp_wht<4>(x[j1], lane);
+  for (int j1 = 0; j1 < XNB; ++j1) tq_warp_wht<4, true>(x[j1], lane);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     float t[XNB];
 #pragma unroll
     for (int i1 = 0; i1 < XNB; ++i1) {
-      float s = 0.f;
+      float s = h12_neg(i1, 0) ? -x[0][k] : x[0][k];
 #pragma unroll
-      for (int j1 = 0; j1 < XNB; ++j1) s += h12_neg(i1, j1) ? -x[j1][k] : x[j1][k];
+      for (int j1 = 1; j1 < XNB; ++j1) s += h12_neg(i1, j1) ? -x[j1][k] : x[j1][k];
       t[i1] = s;
     }
 #pragma unroll
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(256, 2) ix_encode_kernel(IxArgs a) {
     tks[threadIdx.x] = a.tk[threadIdx.x];
   }
   __syncthreads();
-  const int nl = 1 << a.mbk, planes = a.mbk + 1;
+  const int planes = a.mbk + 1;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp; row < a.n;
        row += static_cast<int64_t>(gridDim.x) * 8) {
     const float *src = a.x + row * XD;
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(256, 2) ix_encode_kernel(IxArgs a) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float u = x[j1][k] * inv;
-        const int idx = tq_code(u, tks, nl - 1);
+        const int idx = tq_code<3>(u, tks);   // index codecs have at most 3 MSE bits
         const int w = 4 * j1 + k;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {

@@ -103,7 +103,6 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
   __shared__ float rbuf[QWARPS][D];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nlk = 1 << a.books.mse_bits_k, nlv = 1 << a.books.bits_v;
   if (threadIdx.x < TQ_MAX_LEVELS) {
     cks[threadIdx.x] = a.books.ck[threadIdx.x];
     tks[threadIdx.x] = a.books.tk[threadIdx.x];
@@ -150,7 +149,7 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
       const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks, nlk - 1);
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
       // plane words: lane p*NPL + k stores word k of plane p
       uint32_t myword = 0u;
       for (int p = 0; p < a.books.mse_bits_k; ++p) {
@@ -203,7 +202,7 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
-        const int iv = tq_code(x[k], tvs, nlv - 1);
+        const int iv = tq_code(x[k], tvs);
 #pragma unroll
         for (int p = 0; p < 4; ++p)
           if ((iv >> p) & 1) vw[p][k] |= bit;
@@ -247,7 +246,6 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
   __shared__ __align__(16) float rsm[D];
   __shared__ uint32_t sgw[NPL];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nlk = 1 << a.books.mse_bits_k, nlv = 1 << a.books.bits_v;
   if (tid < TQ_MAX_LEVELS) {
     cks[tid] = a.books.ck[tid];
     tks[tid] = a.books.tk[tid];
@@ -279,7 +277,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks, nlk - 1);
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
       for (int p = 0; p < a.books.mse_bits_k; ++p) {
 #pragma unroll
         for (int k = 0; k < NPL; ++k) {
@@ -305,7 +303,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
-        const int iv = tq_code(x[k], tvs, nlv - 1);
+        const int iv = tq_code(x[k], tvs);
 #pragma unroll
         for (int p = 0; p < 4; ++p)
           if ((iv >> p) & 1) vw[p][k] |= bit;
@@ -400,7 +398,6 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nlk = 1 << a.books.mse_bits_k, nlv = 1 << a.books.bits_v;
   if (tid < TQ_MAX_LEVELS) {
     cks[tid] = a.books.ck[tid];
     tks[tid] = a.books.tk[tid];
@@ -477,7 +474,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks, nlk - 1);
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
       uint32_t myword = 0u;
       for (int p = 0; p < a.books.mse_bits_k; ++p) {
 #pragma unroll
@@ -516,7 +513,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
-        const int iv = tq_code(x[k], tvs, nlv - 1);
+        const int iv = tq_code(x[k], tvs);
 #pragma unroll
         for (int p = 0; p < 4; ++p)
           if ((iv >> p) & 1) vw[p][k] |= bit;

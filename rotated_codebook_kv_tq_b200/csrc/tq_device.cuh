@@ -45,16 +45,20 @@ __device__ __forceinline__ float tq_warp_max(float v) {
 // Unnormalised Walsh-Hadamard transform (Sylvester / natural order) of a
 // d-vector held by one warp with coordinate i = lane + 32 k in x[k],
 // k < NPL = d / 32.  Output y = H_d x.
-template <int NPL>
+// FMA = true does each shuffle stage as one fma with a +-1 factor (fewer
+// instructions, identical results; the factors take registers).
+template <int NPL, bool FMA = false>
 __device__ __forceinline__ void tq_warp_wht(float (&x)[NPL], int lane) {
   // strides 1..16: lane bits, exchanged with shuffles
 #pragma unroll
   for (int s = 1; s < 32; s <<= 1) {
     const bool upper = lane & s;
+    const float sg = upper ? -1.f : 1.f;
 #pragma unroll
     for (int k = 0; k < NPL; ++k) {
       const float o = __shfl_xor_sync(TQ_FULL, x[k], s);
-      x[k] = upper ? (o - x[k]) : (x[k] + o);
+      // o - x or x + o: one rounding either way
+      x[k] = FMA ? fmaf(sg, x[k], o) : (upper ? (o - x[k]) : (x[k] + o));
     }
   }
   // strides 32, 64, ...: register index bits
@@ -81,14 +85,15 @@ __device__ __forceinline__ void tq_apply_signs(float (&x)[NPL], const uint32_t *
   }
 }
 
-// Code of u: #{k : u >= t_k} for ascending thresholds t[0 .. TQ_MAX_LEVELS-2]
-// whose unused slots hold +inf (the codec pads them): a branch-free binary
-// search over the 15 slots (the count is the same as a linear scan's).
-__device__ __forceinline__ int tq_code(float u, const float *t, int /*nt*/) {
-  static_assert(TQ_MAX_LEVELS == 16, "binary search covers 15 thresholds");
-  int idx = (u >= t[7]) ? 8 : 0;
-  idx += (u >= t[idx + 3]) ? 4 : 0;
-  idx += (u >= t[idx + 1]) ? 2 : 0;
-  idx += (u >= t[idx]) ? 1 : 0;
+// Code of u: #{k : u >= t_k} for ascending thresholds t[0 .. 2^STEPS - 2]
+// (STEPS <= 4) whose later slots hold +inf (the codec pads them): a
+// branch-free binary search of STEPS steps (the count is the same as a
+// linear scan's), valid for every codebook of at most STEPS bits.
+template <int STEPS = 4>
+__device__ __forceinline__ int tq_code(float u, const float *t) {
+  static_assert(STEPS >= 1 && STEPS <= 4 && TQ_MAX_LEVELS == 16, "at most 15 thresholds");
+  int idx = 0;
+#pragma unroll
+  for (int s = STEPS - 1; s >= 0; --s) idx += (u >= t[idx + (1 << s) - 1]) ? (1 << s) : 0;
   return idx;
 }
