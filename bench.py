@@ -45,7 +45,7 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
-                                      "vector_search"],
+                                      "vector_search", "quality"],
                    help="run one extra workload alone and print its JSON (1 GPU)")
     p.add_argument("--search-rows", type=int, default=0,
                    help="vector-search database rows for --only vector_search (default 10^6)")
@@ -421,6 +421,92 @@ def quantize_extra(wname: str, pk: dict, steps: int = 40):
                 l2="rotating %d input sets (%.0f MB)" % (n_sets, n_sets * in_bytes / 1e6))
 
 
+def _rope_rows(x, c, s):
+    """Rotate-half RoPE of fp32 rows x [..., d] with cos/sin tables [..., d/2]."""
+    import torch
+    h = x.shape[-1] // 2
+    u, v = x[..., :h], x[..., h:]
+    return torch.cat((u * c - v * s, v * c + u * s), dim=-1)
+
+
+def quality_extra(wname: str, T: int = 0, variants=("prod", "mse"), overrides=None):
+    """Quality of the compressed cache on one workload, for the key codec with
+    the 1-bit QJL residual sketch ("prod": TQ-QKV) and with the same key bits
+    spent on the MSE stage alone ("mse": TQ-KV): relMSE_K and relMSE_V =
+    sum ||x_hat - x||^2 / sum ||x||^2 over every cached row (x the post-RoPE
+    key, the value as given, x_hat from tq_dequantize), and the cosine between
+    each query head's compressed attention output (tq_attention_decode, or
+    tq_attention_bidir for the bidirectional workload) and fp32 attention over
+    the exact K/V, mean and minimum over heads (and queries)."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.WORKLOADS[wname]
+    if T:
+        w = w.scaled(T=T, Lq=min(w.Lq, T))
+    if overrides:
+        w = w.scaled(**overrides)
+    rows_cap = (w.T + 31) // 32 * 32
+    K, V = synth.kv_inputs_torch(w)
+    bidir = w.Lq > 1
+    q = synth.query_inputs_torch(w, Lq=w.Lq if bidir else 1)
+    r = synth.rope_for(w, max(rows_cap, w.Lq))
+    rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+    Kf, Vf, qf = K.float(), V.float(), q.float()
+    if rope is not None:
+        Kf = _rope_rows(Kf, rope[0][:w.T], rope[1][:w.T])
+        if bidir:
+            qf = _rope_rows(qf, rope[0][:w.Lq], rope[1][:w.Lq])
+        else:
+            qf = _rope_rows(qf, rope[0][w.T - 1], rope[1][w.T - 1])
+    scale = 1.0 / math.sqrt(w.d)
+    # exact attention, fp32, GQA: query head h reads KV head h // G
+    Ke = Kf.repeat_interleave(w.G, dim=1)
+    Ve = Vf.repeat_interleave(w.G, dim=1)
+    p = torch.softmax(torch.matmul(qf, Ke.transpose(-1, -2)) * scale, dim=-1)
+    o_ref = torch.matmul(p, Ve)                       # [B, Hq, Lq, d]
+    del Ke, Ve, p
+    D = synth.rotation_signs(w.d, w.seed)
+    S = synth.qjl_matrix_bf16(w.d, w.seed)
+    out = {}
+    for var in variants:
+        qjl = var == "prod"
+        codec = native.Codec(w.d, w.bits_k, qjl, w.bits_v, D, S if qjl else None)
+        cache = native.alloc_cache(codec, w.B, w.Hkv, rows_cap)
+        native.quantize_kv(codec, K, V, cache, rope=rope)
+        rel = {}
+        for which, x in ((0, Kf), (1, Vf)):
+            xh = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.float32, device="cuda")
+            native.dequantize(codec, cache, which, 0, w.T, xh)
+            rel["K" if which == 0 else "V"] = float(((xh - x) ** 2).sum() / (x ** 2).sum())
+            del xh
+        res = dict(key_bits=w.bits_k, key_mse_bits=w.bits_k - 1 if qjl else w.bits_k,
+                   value_bits=w.bits_v, relMSE_K=rel["K"], relMSE_V=rel["V"])
+        try:
+            if bidir:
+                o = torch.empty((w.B, w.Hq, w.Lq, w.d), dtype=torch.float32, device="cuda")
+                ws = torch.empty(native.attention_bidir_workspace(codec, w.B, w.Hq, w.Lq),
+                                 dtype=torch.uint8, device="cuda")
+                native.attention_bidir(codec, q, cache, w.T, scale, o, ws, rope=rope)
+            else:
+                o = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+                ws = torch.empty(native.attention_workspace(codec, w.B, w.Hq, w.num_splits),
+                                 dtype=torch.uint8, device="cuda")
+                native.attention_decode(codec, q[:, :, 0], cache, w.T, scale, o, ws, rope=rope,
+                                        num_splits=w.num_splits)
+                o = o[:, :, None]
+            cos = torch.nn.functional.cosine_similarity(o, o_ref, dim=-1)
+            res.update(output_cosine_mean=float(cos.mean()), output_cosine_min=float(cos.min()))
+        except native.TqError as e:
+            res.update(output_cosine_mean=None, output_cosine_min=None, attention=str(e))
+        out[var] = res
+        del cache
+        codec.close()
+    torch.cuda.synchronize()
+    return dict(workload=describe(w), variants=out,
+                definition="relMSE = sum||x_hat-x||^2/sum||x||^2 over all rows (K post-RoPE); "
+                           "cosine of each head's output vs fp32 attention over exact K/V")
+
+
 def bidir_extra(pk: dict, steps: int = 10):
     """ESM-2-shaped bidirectional pass over the compressed cache (every query
     attends to every key): algorithmic flops 2 T^2 (2d) + 2 T^2 d per head
@@ -660,6 +746,10 @@ def run_only(args) -> int:
         r = bidir_extra(pk, steps=1)
     elif args.only == "decode_long_context":
         r = decode_extra("long_decode", pk, steps=5, warmup=3)
+    elif args.only == "quality":
+        r = {name: quality_extra(name) for name in ("tiny", "llama_decode", "esm_prefill", "long_decode")}
+        r["llama_decode_without_outliers"] = quality_extra(
+            "llama_decode", overrides=dict(n_outliers=0, sigma_scale=None))
     else:
         from rotated_codebook_kv_tq_b200 import synth
         if args.search_rows:
