@@ -382,7 +382,11 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
 // Shared layouts (K-major, no swizzle): A byte (m, kb) at
 // (kb/16)*2048 + (m/8)*128 + (m%8)*16 + kb%16 for K = 2d elements (hi | lo);
 // B = S, byte (i, kb) at (kb/16)*(16d) + (i/8)*128 + (i%8)*16 + kb%16.
-template <int D>
+// MBK / BV: key MSE bits and value bits the kernel is specialised for (the
+// code searches and plane loops then have fixed trip counts); MBK = BV = 4
+// takes any codec of at most 4 + 4 bits, with the plane loops bounded by the
+// codec's own widths.
+template <int D, int MBK, int BV>
 __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   constexpr int NPL = D / 32;
   constexpr int KE = 2 * D;                       // K elements (hi | lo)
@@ -474,9 +478,11 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
+      for (int k = 0; k < NPL; ++k) idx[k] = tq_code<MBK>(x[k], tks);
       uint32_t myword = 0u;
-      for (int p = 0; p < a.books.mse_bits_k; ++p) {
+#pragma unroll
+      for (int p = 0; p < MBK; ++p) {
+        if (MBK == 4 && p >= a.books.mse_bits_k) break;
 #pragma unroll
         for (int k = 0; k < NPL; ++k) {
           const uint32_t w = __ballot_sync(TQ_FULL, (idx[k] >> p) & 1);
@@ -513,9 +519,9 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
-        const int iv = tq_code(x[k], tvs);
+        const int iv = tq_code<BV>(x[k], tvs);
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
+        for (int p = 0; p < BV; ++p)
           if ((iv >> p) & 1) vw[p][k] |= bit;
       }
       if (lane == 0) {
@@ -526,7 +532,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
     }
     if (have && rb < re) {
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < BV; ++p) {
         if (p >= a.books.bits_v) break;
 #pragma unroll
         for (int k = 0; k < NPL; ++k) atomicOr(&vbuf[grp][p][lane + 32 * k], vw[p][k]);
@@ -620,15 +626,16 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   if (warp == 0) sm100::tmem_dealloc(tm, D);
 }
 
-template <int D>
-int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
+template <int D, int MBK, int BV>
+int run_quantize_tc_bits(const QuantArgs &a, cudaStream_t stream) {
   constexpr size_t shm = 128u * 2 * D * 2 + static_cast<size_t>(D) * D * 2;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static bool done[64] = {};
   if (dev < 64 && !done[dev]) {
-    if (cudaFuncSetAttribute(quantize_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(quantize_tc_kernel<D, MBK, BV>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(shm)) != cudaSuccess)
       return tq_check_launch("cudaFuncSetAttribute(quantize_tc)");
     done[dev] = true;
@@ -637,9 +644,19 @@ int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
   const int64_t tiles = (items + 3) / 4;
   const int64_t cap = static_cast<int64_t>(sms) * (D == 128 ? 1 : 2);
   const int grid = static_cast<int>(tiles < cap ? tiles : cap);
-  quantize_tc_kernel<D><<<grid, QTC_T, shm, stream>>>(a);
+  quantize_tc_kernel<D, MBK, BV><<<grid, QTC_T, shm, stream>>>(a);
   tq_count_launch(1);
   return tq_check_launch("quantize_tc_kernel");
+}
+
+// The Llama- and ESM-2-shaped codecs get their own instantiations; any other
+// codec takes the generic one (a (1, 2) instantiation spills at d = 128).
+template <int D>
+int run_quantize_tc(const QuantArgs &a, cudaStream_t stream) {
+  const int mbk = a.books.mse_bits_k, bv = a.books.bits_v;
+  if (mbk == 3 && bv == 4) return run_quantize_tc_bits<D, 3, 4>(a, stream);
+  if (mbk == 2 && bv == 3) return run_quantize_tc_bits<D, 2, 3>(a, stream);
+  return run_quantize_tc_bits<D, 4, 4>(a, stream);
 }
 
 template <int D>
