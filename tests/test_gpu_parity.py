@@ -123,9 +123,21 @@ def test_quantize_zero_and_nonfinite_rows(T):
     assert gpu["kscale"][0, 1, 5, 0] == 0 and gpu["vnorm"][0, 0, 9] == 0
 
 
-@pytest.mark.parametrize("case", ["tiny", "llama_ragged", "esm_d64", "long_2bit"])
+DEQUANT_CASES = {
+    "tiny": synth.WORKLOADS["tiny"],
+    "llama_ragged": synth.WORKLOADS["llama_decode"].scaled(T=200),
+    "esm_d64": synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=3, Hkv=3, T=100),
+    "long_2bit": synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=300),
+    "tiny_mse_keys": synth.WORKLOADS["tiny"].scaled(qjl_k=False, bits_k=3),
+    "llama_mse_keys": synth.WORKLOADS["llama_decode"].scaled(T=200, qjl_k=False, bits_k=4),
+    "long_mse_keys": synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=300, qjl_k=False,
+                                                          bits_k=2),
+}
+
+
+@pytest.mark.parametrize("case", list(DEQUANT_CASES))
 def test_dequantize_parity(case):
-    w, segments = QUANT_CASES[case]
+    w = DEQUANT_CASES[case]
     ocodec, ncodec = tl.codecs(w)
     K, V, K64, V64 = _inputs(w)
     rows_cap = (w.T + 31) // 32 * 32
@@ -158,6 +170,13 @@ DECODE_CASES = {
     "gqa8": (synth.WORKLOADS["long_decode"].scaled(B=1, Hq=16, Hkv=2, T=500), None, 3),
     "gqa2_multi_sub": (synth.WORKLOADS["llama_decode"].scaled(B=1, Hq=4, Hkv=2, T=2500), None, 1),
     "tiny_two_chunks": (synth.WORKLOADS["tiny"].scaled(T=1000), None, 2),
+    # MSE-only keys (TQ-KV, no QJL plane): all key bits on the Lloyd-Max stage
+    "tiny_mse_keys": (synth.WORKLOADS["tiny"].scaled(qjl_k=False, bits_k=3), None, 8),
+    "llama_mse_keys": (synth.WORKLOADS["llama_decode"].scaled(T=1000, qjl_k=False, bits_k=4), None, 7),
+    "long_mse_keys": (synth.WORKLOADS["long_decode"].scaled(B=2, Hq=8, Hkv=2, T=3000, qjl_k=False,
+                                                           bits_k=2), None, 128),
+    "esm_mse_keys_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=4, Hkv=2, T=300, Lq=1,
+                                                               qjl_k=False, bits_k=3), None, 4),
 }
 
 

@@ -117,8 +117,17 @@ def new_stats():
     return dict(code_mism=0, sign_mism=0, code_window=0, sign_window=0, coords=0)
 
 
-def assert_mismatch_budget(stats: dict) -> None:
+# Boundary-window accounting of every parity check in this session: the
+# mismatch count, the window population and the fraction of coordinates are
+# printed in pytest's terminal summary (conftest.py) so they appear in the log.
+MISMATCH_REPORT: list = []
+
+
+def assert_mismatch_budget(stats: dict, label: str = "") -> None:
+    import os
     frac = (stats["code_mism"] + stats["sign_mism"]) / max(1, stats["coords"])
+    label = label or os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    MISMATCH_REPORT.append(dict(stats, test=label, fraction=frac))
     assert frac <= MISMATCH_CAP, stats
 
 
