@@ -766,11 +766,32 @@ def run_only(args) -> int:
     return 0
 
 
+def relaunch_cmd(script: str, args_list, gpus: int, port: int):
+    """torchrun command that runs ``script`` on ``gpus`` ranks of one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            script, *args_list]
+
+
+def check_world(gpus: int, world: int) -> None:
+    """--gpus must agree with the launcher's world size."""
+    if gpus != world:
+        raise SystemExit(f"bench.py: --gpus {gpus} but WORLD_SIZE={world}; launch one rank per GPU")
+
+
 def main():
     args = parse_args()
     if args.only:
         return run_only(args)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started without a launcher: start one rank per GPU ourselves
+        import socket
+        with socket.socket() as s:
+            s.bind(("127.0.0.1", 0))
+            port = s.getsockname()[1]
+        return subprocess.call(relaunch_cmd(os.path.abspath(__file__), sys.argv[1:], args.gpus, port))
     world, rank, local = dist_init()
+    check_world(args.gpus, world)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     import torch

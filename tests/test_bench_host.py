@@ -55,3 +55,44 @@ def test_single_rank_needs_no_process_group(monkeypatch):
     assert bench.dist_init(backend="gloo") == (1, 0, 0)
     assert bench.max_over_ranks(3.0, 1) == 3.0
     assert bench.weak_value(10.0, 1, 2.0) == 5.0
+
+
+RANK_SCRIPT = """
+import os, sys
+sys.path.insert(0, {root!r})
+import bench
+w, r, local = bench.dist_init(backend="gloo")
+bench.check_world(int(sys.argv[1]), w)
+t = bench.max_over_ranks(1.0 + r, w)
+if r == 0:
+    print("RESULT", w, t, bench.weak_value(10.0, w, t), flush=True)
+bench.barrier(w)
+import torch.distributed as dist
+dist.destroy_process_group()
+"""
+
+
+def test_relaunch_command_starts_one_rank_per_gpu(tmp_path):
+    """bench.py --gpus N started without a launcher re-executes itself through
+    torch.distributed.run; the command it builds starts N ranks that find each
+    other on 127.0.0.1 and agree on the slowest rank's time."""
+    import subprocess
+    import sys
+    import bench
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    script = tmp_path / "ranks.py"
+    script.write_text(RANK_SCRIPT.format(root=root))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    cmd = bench.relaunch_cmd(str(script), ["2"], 2, _free_port())
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=2" in cmd
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=180, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = [l for l in res.stdout.splitlines() if l.startswith("RESULT")][0].split()
+    assert int(line[1]) == 2 and float(line[2]) == 2.0 and float(line[3]) == 10.0
+
+
+def test_gpus_must_match_world_size():
+    import bench
+    bench.check_world(1, 1)
+    with pytest.raises(SystemExit):
+        bench.check_world(8, 1)
