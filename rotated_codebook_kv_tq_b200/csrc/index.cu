@@ -17,9 +17,18 @@
 // Encoding a database row (tq_index_build):
 //   ix_encode_kernel   norm, rotation, 3-bit codes -> MSE bit planes, residual
 //                      r written as bf16 hi | lo into a scratch matrix [n][2d]
-//   ix_gemm_kernel     z = S r for 128 x 256 tiles: tcgen05 kind::f16 MMAs of
-//                      [r_hi | r_lo] against [S | S] (S is exactly bf16),
-//                      fp32 in tensor memory, sign bits -> the QJL plane.
+//   ix_sketch_kernel   z = S r for 128 x 256 tiles: one warp streams the
+//                      [r_hi | r_lo] and S tiles by cp.async.bulk into a
+//                      4-stage ring and issues tcgen05 kind::f16 MMAs (S is
+//                      exactly bf16), fp32 in tensor memory; four epilogue
+//                      warps turn the signs into the QJL plane.
+// Scanning (tq_scan_topk):
+//   ix_qrot_kernel     q' = Pi q per query
+//   ix_gemm_kernel     q'' = S q' (fp32 GEMM on CUDA cores)
+//   ix_qpack_kernel    fp16 B operand [2^e q' | 2^e coef q''] in chunk order
+//   ix_scan2_kernel    rows dequantized into tensor memory, M128 x N256 MMAs,
+//                      per-thread top-k lists
+//   ix_merge_kernel    merge of the per-CTA lists into the final top-k
 #include <math_constants.h>
 
 #include <cstring>
