@@ -385,6 +385,104 @@ def oracle_rate(bench: DecodeBench, seconds: float, rows: int = None):
     return w.B / per_step_full, n, dt, rows
 
 
+def _time_loop(fn, seconds: float) -> float:
+    """Seconds per call of ``fn``: at least one call, then repeat until
+    ``seconds`` have passed."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            return dt / n
+
+
+def _one_and_all(fn, seconds: float):
+    """(seconds per call on one thread, on every BLAS thread, thread count)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        t1 = _time_loop(fn, seconds)
+    return t1, _time_loop(fn, seconds), blas_threads()
+
+
+def cpu_baselines(seconds: float = 1.0) -> dict:
+    """The oracle, as it stands, timed on this host on bounded samples of every
+    workload, single-threaded and with all BLAS threads (numpy fp64; the Python
+    loops over heads and rows stay on one core either way).  Each figure is in
+    the unit of the matching GPU figure, scaled from the sample as stated."""
+    import numpy as np
+    from oracle import attention as oatt
+    from oracle import codec as oc
+    from oracle import scan as oscan
+    from rotated_codebook_kv_tq_b200 import synth
+    out = dict(nproc=os.cpu_count())
+
+    def codec_of(w):
+        S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
+        return oc.make_codec(w.d, w.bits_k, w.qjl_k, w.bits_v, synth.rotation_signs(w.d, w.seed), S)
+
+    def entry(unit, t1, tn, threads, to_value, sample):
+        return dict(unit=unit, one_thread=to_value(t1), all_threads=to_value(tn), threads=threads,
+                    sample=sample)
+
+    # decode steps: quantize-append of the new token + attention of every head
+    # over the first `rows` cached tokens; cost is linear in rows, scaled to T
+    for name, rows in (("tiny", 1024), ("llama_decode", 1024), ("long_decode", 512)):
+        w = synth.WORKLOADS[name]
+        ww = w.scaled(T=rows)
+        K, V = synth.kv_inputs(ww)
+        q = synth.as_float64(synth.query_inputs(ww, Lq=1)[:, :, 0], w.dtype)
+        K64, V64 = synth.as_float64(K, w.dtype), synth.as_float64(V, w.dtype)
+        codec = codec_of(w)
+        rope = synth.rope_for(w, (rows + 31) // 32 * 32)
+        cache = oc.empty_cache(codec, w.B, w.Hkv, (rows + 31) // 32 * 32)
+        oc.quantize_into(cache, K64[:, :, :rows - 1], V64[:, :, :rows - 1], codec, rope=rope)
+
+        def step():
+            oc.quantize_into(cache, K64[:, :, rows - 1:], V64[:, :, rows - 1:], codec, rope=rope,
+                             pos0=rows - 1, row0=rows - 1)
+            oatt.decode(q, cache, codec, [rows] * w.B, 1.0 / math.sqrt(w.d), rope=rope)
+        t1, tn, th = _one_and_all(step, seconds)
+        scale = w.T / rows
+        out[name] = entry("tokens/s", t1, tn, th, lambda t: w.B / (t * scale),
+                          f"one decode step over the first {rows} of {w.T} tokens, all "
+                          f"{w.B * w.Hq} query heads, time x {w.T}/{rows}")
+    # ESM-2-shaped prefill quantize: two (batch, head) pairs of the 320
+    w = synth.WORKLOADS["esm_prefill"]
+    ww = w.scaled(B=1, Hq=2, Hkv=2)
+    K, V = synth.kv_inputs(ww)
+    K64, V64 = synth.as_float64(K, w.dtype), synth.as_float64(V, w.dtype)
+    codec = codec_of(w)
+    rope = synth.rope_for(w, w.T)
+    cache = oc.empty_cache(codec, 1, 2, w.T)
+    t1, tn, th = _one_and_all(lambda: oc.quantize_into(cache, K64, V64, codec, rope=rope), seconds)
+    in_bytes = 2 * 2 * w.T * w.d * 2
+    out["quantize_esm_prefill"] = entry("GB/s of bf16 input", t1, tn, th, lambda t: in_bytes / t / 1e9,
+                                        f"K+V of 2 of the {w.B * w.Hkv} (batch, head) pairs, T={w.T}")
+    # ESM-2-shaped bidirectional pass: one head, all 1024 queries
+    q = synth.as_float64(synth.query_inputs(ww, Lq=w.T), w.dtype)
+    ropeq = synth.rope_for(w, w.T)
+    flops = 2 * w.T * w.T * 2 * w.d + 2 * w.T * w.T * w.d
+    t1, tn, th = _one_and_all(
+        lambda: oatt.bidirectional(q, cache, codec, w.T, 1.0 / math.sqrt(w.d), rope=ropeq,
+                                   heads=[(0, 0)]), seconds)
+    out["bidir_esm_prefill"] = entry("TFLOP/s (algorithmic)", t1, tn, th, lambda t: flops / t / 1e12,
+                                     f"one of the {w.B * w.Hq} heads, {w.T} queries x {w.T} keys")
+    # vector search: index build of 2048 rows; scan of 8 queries over 8192 rows
+    sw = synth.VECTOR_SEARCH
+    scodec = oc.make_codec(sw.d, sw.bits, True, 4, synth.rotation_signs(sw.d, sw.seed),
+                           synth.qjl_matrix_bf16(sw.d, sw.seed))
+    x = synth.unit_rows(8192, sw.d, sw.seed, synth.STREAM_K).astype(np.float64)
+    qs = synth.unit_rows(8, sw.d, sw.seed, synth.STREAM_Q).astype(np.float64)
+    t1, tn, th = _one_and_all(lambda: oc.pack_keys(oc.quantize_keys(x[:2048], scodec), scodec), seconds)
+    out["index_build"] = entry("rows/s", t1, tn, th, lambda t: 2048 / t, "2048 of the 10^6 rows")
+    kc, ks = oc.pack_keys(oc.quantize_keys(x, scodec), scodec)
+    t1, tn, th = _one_and_all(lambda: oscan.topk(oscan.scores(qs, kc, ks, scodec), sw.k), seconds)
+    out["scan_topk"] = entry("queries/s over 10^6 rows", t1, tn, th,
+                             lambda t: 8 * 8192 / t / sw.n, "8 queries x 8192 rows, scaled to 10^6 rows")
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Extra workloads
 # ---------------------------------------------------------------------------
@@ -849,6 +947,13 @@ def main():
             value=rate, unit="tokens/s", cores=blas_threads(), kind="oracle",
             sample=f"{n} oracle decode steps (quantize-append + all {w.Hq} heads) over the first "
                    f"{rows} of {w.T} tokens in {secs:.1f} s, scaled by {w.T}/{rows}")
+        try:
+            per = cpu_baselines()
+            line["cpu_baseline"]["nproc"] = per["nproc"]
+            line["cpu_baseline"]["one_thread"] = per["llama_decode"]["one_thread"]
+            line["cpu_baseline"]["per_workload"] = per
+        except Exception as e:  # report, do not hide
+            line["cpu_baseline"]["per_workload"] = dict(error=repr(e))
     if rank == 0 and world == 1 and not args.no_extras:
         extras = {}
         try:
