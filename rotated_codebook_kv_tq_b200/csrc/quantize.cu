@@ -724,6 +724,12 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   // implementation, used to cross-check the tensor-core one)
   const char *impl = getenv("TQ_QUANT_IMPL");
   const bool simt = impl && impl[0] == 's';
+  if (items >= 256 && !simt) {
+    // large bf16 calls: one thread per row, TMA tiles (quantize_tile.cu)
+    const int e = launch_quantize_tile(c, k, v, dtype, B, H, T, sb, sh, st, rc, rs, pos0, cache,
+                                       row0, status, stream);
+    if (e != TQ_ERR_UNSUPPORTED) return e;
+  }
   const bool tc = c->qjl_k && items >= 256 && !simt;
   const bool append = items < 256 && !simt;
   switch (c->d) {

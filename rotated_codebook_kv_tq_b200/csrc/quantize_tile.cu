@@ -1,0 +1,604 @@
+// Prefill quantize, one thread per token row (sm_100a).
+//
+// Same per-row computation as quantize.cu ("TurboESM ..." section 2.A: RoPE,
+// then the rotation; "FibQuant ..." section 2.3: store nu, rotate x / nu,
+// quantize; "Ablazione ..." "Configurazione Sperimentale": randomized
+// Walsh-Hadamard rotation and Beta Lloyd-Max codebooks; "Google presenta
+// TurboQuant ..." "Eliminacion del sesgo": b-1 MSE bits plus the 1-bit QJL
+// sketch of the residual), laid out for throughput on large calls:
+//
+// * A tile is 128 consecutive cache rows of one (batch, head), aligned to 128
+//   rows, so each warp owns exactly one 32-token value column group.  The
+//   K, V and RoPE-table tiles arrive by TMA tensor copies with the 128-byte
+//   swizzle, so thread r reads its own row from shared memory without bank
+//   conflicts.  Rows outside the call are zero-filled by the copy and skipped
+//   on store.
+// * Every thread runs its row alone: RoPE, norm, the d-point Walsh-Hadamard
+//   transform in registers (no shuffles), codes by compares against the upper
+//   half of the symmetric codebook (the middle threshold is 0), and bit planes
+//   accumulated one funnel shift per coordinate.  Value planes are moved into
+//   the 32-token column layout with warp-wide 32 x 32 bit transposes.
+// * Keys: the residual of the tile, split into bf16 hi + lo, is stored into
+//   tensor memory and sketched against S (exactly bf16) by tcgen05 kind::f16
+//   MMAs with fp32 accumulation; each thread reads its row of S r back.
+// * Warps 0-3 take key rows, warps 4-7 value rows, warp 8 issues the copies of
+//   the next tile (as soon as every row of the current one is in registers)
+//   and the sketch MMAs.  CTAs are persistent over tile ranges ordered by
+//   position first, so the RoPE table tile is reloaded only when the position
+//   range changes.
+//
+// Codes are decided on the scaled transform y = H D x against t_k * sqrt(d) nu
+// (the same decision as u = y / (sqrt(d) nu) against t_k, up to fp32
+// rounding); the sketch signs are invariant to that positive scale.
+#include <cuda.h>
+
+#include <cstdlib>
+#include <cstring>
+
+#include "tq_device.cuh"
+#include "tq_sm100.cuh"
+
+namespace {
+
+constexpr int QR = 128;         // rows per tile
+constexpr int QT = 288;         // 4 key warps, 4 value warps, 1 copy / MMA warp
+constexpr uint32_t BOX = QR * 128;   // bytes of one swizzled 128-row box
+
+struct TileArgs {
+  int B, H, T;
+  int64_t row0, pos0, rows_cap;
+  int64_t R_first;   // cache row of the first row tile (multiple of 128)
+  int64_t nrt;       // row tiles per (batch, head)
+  int64_t ntiles;    // nrt * B * H, ordered (row tile, batch, head)
+  uint8_t *kcode;
+  uint16_t *kscale;
+  uint32_t *vcode;
+  uint16_t *vnorm;
+  uint32_t *status;
+  const uint16_t *S;
+  int rope;
+  float ck[8];       // key centroid magnitudes c[half + m], m = 0 .. half-1
+  float tk[8];       // key thresholds above 0: t[half - 1 + j], j = 1 .. half-1 (tk[j - 1])
+  float tv[8];       // value thresholds above 0
+  uint32_t dneg[4];  // bit i set <=> D_i = -1
+};
+
+// ---------------------------------------------------------------- TMA
+
+__device__ __forceinline__ void tma_4d(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                       int c3, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(sm100::smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(sm100::smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                       uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(sm100::smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(sm100::smem_addr(bar))
+      : "memory");
+}
+
+// 16-byte chunk c of row r in a 128-byte-swizzled box (1024-byte aligned).
+__device__ __forceinline__ uint4 swz_ld(const uint8_t *box, int r, int c) {
+  return *reinterpret_cast<const uint4 *>(box + r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Bounded wait that also gives up as soon as another thread has.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  for (int it = 0; it < 4096; ++it) {
+    if (sm100::mbar_wait(bar, parity, 1u << 14)) return true;
+    if (*abort_flag) return false;
+  }
+  return false;
+}
+
+// In-register Walsh-Hadamard transform, Sylvester natural order: y = H_D x.
+template <int D>
+__device__ __forceinline__ void wht_regs(float (&x)[D]) {
+#pragma unroll
+  for (int s = 1; s < D; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      if (!(i & s)) {
+        const float a = x[i], b = x[i + s];
+        x[i] = a + b;
+        x[i + s] = a - b;
+      }
+    }
+  }
+}
+
+// Sign bits of the code planes of one coordinate: plane p's bit, inverted,
+// sits in the top bit of the returned word p (see the thermometer identities
+// in the kernel comment).  y: transformed coordinate; th: thresholds above 0
+// times the row scale, ascending; NB: code bits.
+template <int NB>
+__device__ __forceinline__ void plane_msbs(float y, const float *th, uint32_t (&w)[4]) {
+  constexpr int NT = (1 << (NB - 1)) - 1;   // thresholds above 0
+  const float a = fabsf(y);
+  uint32_t s[NT > 0 ? NT : 1];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) s[j] = __float_as_uint(a - th[j]);
+  const uint32_t sy = __float_as_uint(y);
+  w[NB - 1] = sy;                       // top bit = [y >= 0]
+  if (NB == 2) {
+    w[0] = s[0] ^ sy;
+  } else if (NB == 3) {
+    w[1] = s[1] ^ sy;
+    w[0] = s[0] ^ s[1] ^ s[2] ^ sy;
+  } else if (NB == 4) {
+    w[2] = s[3] ^ sy;
+    w[1] = s[1] ^ s[3] ^ s[5] ^ sy;
+    w[0] = s[0] ^ s[1] ^ s[2] ^ s[3] ^ s[4] ^ s[5] ^ s[6] ^ sy;
+  }
+}
+
+// 32 x 32 bit transpose across a warp: on return bit L of lane i's word is
+// bit i of lane L's input word.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  const uint32_t masks[5] = {0xffff0000u, 0xff00ff00u, 0xf0f0f0f0u, 0xccccccccu, 0xaaaaaaaau};
+#pragma unroll
+  for (int st = 0; st < 5; ++st) {
+    const int j = 16 >> st;
+    const uint32_t y = __shfl_xor_sync(TQ_FULL, x, j);
+    const bool hi = lane & j;
+    // lanes without bit j take the partner's low bits into their high
+    // positions; lanes with bit j take the partner's high bits into their low
+    x = hi ? ((x & masks[st]) | ((y >> j) & ~masks[st])) : ((x & ~masks[st]) | ((y << j) & masks[st]));
+  }
+  return x;
+}
+
+template <int D, int MBK, int BV, bool QJL>
+__global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
+    qtile_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 const __grid_constant__ CUtensorMap tmc, const __grid_constant__ CUtensorMap tms,
+                 TileArgs a) {
+  constexpr int NBX = D / 64;             // boxes per row (64 bf16 or 32 fp32 table entries)
+  constexpr int PK = MBK + (QJL ? 1 : 0);
+  constexpr int NW = D / 32;              // words per plane row
+  constexpr int HK = 1 << (MBK - 1), HV = 1 << (BV - 1);
+  constexpr uint32_t IDESC = sm100::idesc_bf16(128, D);
+  constexpr int TCOLS = 2 * D;            // A (hi | lo, D/2 columns each) + z (D columns)
+  extern __shared__ uint8_t qsm_raw[];
+  uint8_t *qsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *Kt = qsm;
+  uint8_t *Vt = Kt + NBX * BOX;
+  uint8_t *Ct = Vt + NBX * BOX;
+  uint8_t *Snt = Ct + NBX * BOX;
+  uint8_t *Bs = Snt + NBX * BOX;
+  __shared__ __align__(8) uint64_t full, empty, a_ready, z_ready;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t BH = static_cast<int64_t>(a.B) * a.H;
+  const int64_t t_begin = a.ntiles * blockIdx.x / gridDim.x;
+  const int64_t t_end = a.ntiles * (blockIdx.x + 1) / gridDim.x;
+
+  if (QJL) {
+    for (int e = tid; e < D * D; e += QT) {
+      const int i = e / D, kb = 2 * (e % D);
+      *reinterpret_cast<uint16_t *>(Bs + (kb >> 4) * (D * 16) + (i >> 3) * 128 + (i & 7) * 16 +
+                                    (kb & 15)) = a.S[e];
+    }
+    if (warp == 0) sm100::tmem_alloc(&tmem_s, TCOLS);
+  }
+  if (tid == 0) {
+    sm100::mbar_init(&full, 1);
+    sm100::mbar_init(&empty, 8);
+    sm100::mbar_init(&a_ready, 4);
+    sm100::mbar_init(&z_ready, 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  sm100::fence_async_smem();
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  const uint32_t tm = QJL ? tmem_s : 0u;
+
+  if (warp == 8) {
+    // ------------------------------------------------ copies and sketch MMAs
+    if (lane == 0) {
+      int64_t cur_pt = -1;
+      int issued = -1, committed = -1;
+      auto issue = [&](int64_t tau) {
+        const int64_t pt = tau / BH, bh = tau % BH;
+        const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
+        const int t0 = static_cast<int>(a.R_first + pt * QR - a.row0);
+        const bool table = a.rope && pt != cur_pt;
+        sm100::mbar_expect_tx(&full, (2 + (table ? 2 : 0)) * NBX * BOX);
+#pragma unroll
+        for (int x = 0; x < NBX; ++x) {
+          tma_4d(Kt + x * BOX, &tmk, 64 * x, t0, h, b, &full);
+          tma_4d(Vt + x * BOX, &tmv, 64 * x, t0, h, b, &full);
+        }
+        if (table) {
+          const int p0 = static_cast<int>(a.pos0) + t0;
+#pragma unroll
+          for (int x = 0; x < NBX; ++x) {
+            tma_2d(Ct + x * BOX, &tmc, 32 * x, p0, &full);
+            tma_2d(Snt + x * BOX, &tms, 32 * x, p0, &full);
+          }
+          cur_pt = pt;
+        }
+        ++issued;
+      };
+      if (t_begin < t_end) issue(t_begin);
+      int i = 0;
+      for (int64_t tau = t_begin; tau < t_end && !abort_s; ++tau, ++i) {
+        if (tau + 1 < t_end) {
+          // every row of tile i is in registers: the buffers are free
+          if (!wait_or_abort(&empty, i & 1, &abort_s)) { abort_s = 1; break; }
+          issue(tau + 1);
+        }
+        if (QJL) {
+          if (!wait_or_abort(&a_ready, i & 1, &abort_s)) { abort_s = 1; break; }
+          sm100::fence_after_sync();
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s)
+            sm100::mma_f16_ts(tm + D, tm + 8 * s,
+                              sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
+                              IDESC, s > 0);
+#pragma unroll
+          for (int s = 0; s < D / 16; ++s)
+            sm100::mma_f16_ts(tm + D, tm + D / 2 + 8 * s,
+                              sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
+                              IDESC, 1);
+          sm100::mma_commit(&z_ready);
+          committed = i;
+        }
+      }
+      if (abort_s) {
+        // let this CTA's own copies and MMAs land before its memory is released
+        if (issued >= 0) sm100::mbar_wait(&full, issued & 1, 1u << 20);
+        if (committed >= 0) sm100::mbar_wait(&z_ready, committed & 1, 1u << 20);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ row threads
+    const bool is_key = warp < 4;
+    const int rl = tid & 127;                 // row of the tile = TMEM lane
+    const int wq = warp & 3;
+    const uint8_t *Xt = is_key ? Kt : Vt;
+    float thr[8];
+    int i = 0;
+    for (int64_t tau = t_begin; tau < t_end; ++tau, ++i) {
+      if (abort_s) break;
+      const int64_t pt = tau / BH, bh = tau % BH;
+      const int64_t R = a.R_first + pt * QR + rl;     // cache row
+      const int64_t t = R - a.row0;                    // token of the call
+      const bool active = t >= 0 && t < a.T;
+      if (!wait_or_abort(&full, i & 1, &abort_s)) { abort_s = 1; break; }
+      // ---- row into registers (+ RoPE for keys)
+      float x[D];
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = swz_ld(Xt + (c >> 3) * BOX, rl, c & 7);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * c + 2 * e] = __uint_as_float(w4[e] << 16);
+          x[8 * c + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+        }
+      }
+      if (is_key && a.rope) {
+        constexpr int HALF = D / 2;
+#pragma unroll
+        for (int c = 0; c < HALF / 4; ++c) {
+          const uint4 cv = swz_ld(Ct + (c >> 3) * BOX, rl, c & 7);
+          const uint4 sv = swz_ld(Snt + (c >> 3) * BOX, rl, c & 7);
+          const float cs[4] = {__uint_as_float(cv.x), __uint_as_float(cv.y), __uint_as_float(cv.z),
+                               __uint_as_float(cv.w)};
+          const float sn[4] = {__uint_as_float(sv.x), __uint_as_float(sv.y), __uint_as_float(sv.z),
+                               __uint_as_float(sv.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * c + e;
+            const float u = x[j], w = x[j + HALF];
+            x[j] = u * cs[e] - w * sn[e];
+            x[j + HALF] = w * cs[e] + u * sn[e];
+          }
+        }
+      }
+      // the tile's buffers may be refilled now
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&empty);
+      // ---- norm, sign flip, transform
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < D; ++j) ss = fmaf(x[j], x[j], ss);
+      float nu = sqrtf(ss);
+      bool bad = !(ss <= 3.402823466e38f) || isinf(__half2float(__float2half_rn(nu)));
+      if (bad) nu = 0.f;
+#pragma unroll
+      for (int j = 0; j < D; ++j)
+        x[j] = __uint_as_float(__float_as_uint(x[j]) ^ (((a.dneg[j >> 5] >> (j & 31)) & 1u) << 31));
+      wht_regs<D>(x);
+      if (bad || !(nu > 0.f)) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) x[j] = 0.f;   // zero row: u = 0 (+0 decides the upper half)
+      }
+      const float sc = nu > 0.f ? sqrtf(static_cast<float>(D)) * nu : 1.f;
+      if (bad && active && a.status) atomicAdd(a.status, 1u);
+      if (is_key) {
+        // ---------------------------------------------- key row
+#pragma unroll
+        for (int j = 0; j < HK - 1; ++j) thr[j] = a.tk[j] * sc;
+        uint32_t pw[PK][NW];
+#pragma unroll
+        for (int p = 0; p < PK; ++p)
+#pragma unroll
+          for (int w = 0; w < NW; ++w) pw[p][w] = 0u;
+        float r2 = 0.f;
+        float cks[HK];
+#pragma unroll
+        for (int m = 0; m < HK; ++m) cks[m] = a.ck[m] * sc;
+#pragma unroll
+        for (int j = D - 1; j >= 0; --j) {
+          uint32_t ms[4];
+          plane_msbs<MBK>(x[j], thr, ms);
+#pragma unroll
+          for (int p = 0; p < MBK; ++p) pw[p][j >> 5] = __funnelshift_l(ms[p], pw[p][j >> 5], 1);
+          if (QJL) {
+            const float aa = fabsf(x[j]);
+            float cm = cks[0];
+#pragma unroll
+            for (int m = 1; m < HK; ++m) cm = aa >= thr[m - 1] ? cks[m] : cm;
+            const float cval = x[j] >= 0.f ? cm : -cm;
+            x[j] = x[j] - cval;            // residual (scaled by sc)
+            r2 = fmaf(x[j], x[j], r2);
+          }
+        }
+        // funnel shifts accumulated coordinate 32 w + 31 first: bit i = coord 32 w + i
+#pragma unroll
+        for (int p = 0; p < MBK; ++p)
+#pragma unroll
+          for (int w = 0; w < NW; ++w) pw[p][w] = ~pw[p][w];
+        float rho = 0.f;
+        if (QJL) {
+          rho = sqrtf(r2) / sc;
+          // tensor memory A: columns [0, D/2) hi, [D/2, D) lo (two bf16 per
+          // column, lower K index in the low half); lane = row
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t h32[32], l32[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int j = 32 * c + e;
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+              const float2 hf = __bfloat1622float2(hi);
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
+              h32[e] = *reinterpret_cast<const uint32_t *>(&hi);
+              l32[e] = *reinterpret_cast<const uint32_t *>(&lo);
+            }
+            sm100::tmem_st32(sm100::tmem_lane(tm + 32 * c, wq), h32);
+            sm100::tmem_st32(sm100::tmem_lane(tm + D / 2 + 32 * c, wq), l32);
+          }
+          sm100::wait_st();
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&a_ready);
+        }
+        const int64_t crow = bh * a.rows_cap + R;
+        if (active) {
+          uint8_t *kr = a.kcode + crow * (PK * (D / 8));
+#pragma unroll
+          for (int p = 0; p < MBK; ++p) {
+            if (NW == 2)
+              *reinterpret_cast<uint2 *>(kr + p * (D / 8)) = make_uint2(pw[p][0], pw[p][1]);
+            else
+              *reinterpret_cast<uint4 *>(kr + p * (D / 8)) =
+                  make_uint4(pw[p][0], pw[p][1 % NW], pw[p][2 % NW], pw[p][3 % NW]);
+          }
+          reinterpret_cast<uint32_t *>(a.kscale)[crow] =
+              static_cast<uint32_t>(tq_f32_to_half(nu)) | (static_cast<uint32_t>(tq_f32_to_half(rho)) << 16);
+        }
+        if (QJL) {
+          if (!wait_or_abort(&z_ready, i & 1, &abort_s)) { abort_s = 1; break; }
+          sm100::fence_after_sync();
+          uint32_t sg[NW];
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            uint32_t z[32];
+            sm100::tmem_ld32(sm100::tmem_lane(tm + D + 32 * w, wq), z);
+            sm100::wait_ld();
+            uint32_t acc = 0u;
+#pragma unroll
+            for (int e = 31; e >= 0; --e) acc = __funnelshift_l(z[e], acc, 1);
+            sg[w] = ~acc;                  // bit e = [z >= 0]
+          }
+          if (active) {
+            uint8_t *kr = a.kcode + crow * (PK * (D / 8)) + MBK * (D / 8);
+            if (NW == 2)
+              *reinterpret_cast<uint2 *>(kr) = make_uint2(sg[0], sg[1]);
+            else
+              *reinterpret_cast<uint4 *>(kr) = make_uint4(sg[0], sg[1 % NW], sg[2 % NW], sg[3 % NW]);
+          }
+        }
+      } else {
+        // ---------------------------------------------- value row
+#pragma unroll
+        for (int j = 0; j < HV - 1; ++j) thr[j] = a.tv[j] * sc;
+        uint32_t pw[BV][NW];
+#pragma unroll
+        for (int p = 0; p < BV; ++p)
+#pragma unroll
+          for (int w = 0; w < NW; ++w) pw[p][w] = 0u;
+#pragma unroll
+        for (int j = D - 1; j >= 0; --j) {
+          uint32_t ms[4];
+          plane_msbs<BV>(x[j], thr, ms);
+#pragma unroll
+          for (int p = 0; p < BV; ++p) pw[p][j >> 5] = __funnelshift_l(ms[p], pw[p][j >> 5], 1);
+        }
+        const int64_t crow = bh * a.rows_cap + R;
+        if (active) a.vnorm[crow] = tq_f32_to_half(nu);
+        // column words: lane i gets coordinate 32 w + i of the warp's 32 rows
+        const uint32_t act = __ballot_sync(TQ_FULL, active);
+        uint32_t *vg = a.vcode + (bh * (a.rows_cap / 32) + (R >> 5)) * (BV * D);
+#pragma unroll
+        for (int p = 0; p < BV; ++p) {
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+            const uint32_t col = warp_transpose32(~pw[p][w], lane);
+            uint32_t *dst = vg + p * D + 32 * w + lane;
+            if (act == TQ_FULL) {
+              *dst = col;
+            } else if (act) {
+              atomicAnd(dst, ~act);
+              atomicOr(dst, col & act);
+            }
+          }
+        }
+      }
+    }
+  }
+  sm100::fence_before_sync();
+  __syncthreads();
+  sm100::fence_after_sync();
+  if (abort_s && tid == 0 && a.status) atomicOr(a.status, 1u << 31);
+  if (QJL && warp == 0) sm100::tmem_dealloc(tm, TCOLS);
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+template <int D, int MBK, int BV, bool QJL>
+int run_tile(const TileArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mc,
+             const CUtensorMap &ms, cudaStream_t stream) {
+  constexpr size_t shm = 1024 + 4 * (D / 64) * BOX + (QJL ? static_cast<size_t>(D) * D * 2 : 0);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool done[64] = {};
+  if (dev < 64 && !done[dev]) {
+    if (cudaFuncSetAttribute(qtile_kernel<D, MBK, BV, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(shm)) != cudaSuccess)
+      return tq_check_launch("cudaFuncSetAttribute(qtile)");
+    done[dev] = true;
+  }
+  int occ = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, qtile_kernel<D, MBK, BV, QJL>, QT, shm);
+  if (occ < 1) occ = 1;
+  const int64_t cap = static_cast<int64_t>(sms) * occ;
+  const int grid = static_cast<int>(a.ntiles < cap ? a.ntiles : cap);
+  qtile_kernel<D, MBK, BV, QJL><<<grid, QT, shm, stream>>>(mk, mv, mc, ms, a);
+  tq_count_launch(1);
+  return tq_check_launch("qtile_kernel");
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, void *base, const cuuint64_t *dims,
+              const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, dt, rank, base, dims, strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Returns TQ_ERR_UNSUPPORTED (without launching) when the call does not fit
+// this kernel's layout rules; the caller then takes another kernel.
+int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
+                         int T, int64_t sb, int64_t sh, int64_t st, const float *rc,
+                         const float *rs, int64_t pos0, const tq_cache *cache, int64_t row0,
+                         uint32_t *status, cudaStream_t stream) {
+  if (getenv("TQ_QUANT_IMPL")) return TQ_ERR_UNSUPPORTED;   // explicit kernel choice
+  if (dtype != TQ_BF16 || (c->d != 64 && c->d != 128) || T <= 0) return TQ_ERR_UNSUPPORTED;
+  const int d = c->d;
+  const int mbk = c->mse_bits_k, bv = c->bits_v;
+  if (mbk < 1 || mbk > 4 || bv < 1 || bv > 4) return TQ_ERR_UNSUPPORTED;
+  auto al16 = [](int64_t x) { return (x * 2) % 16 == 0; };
+  if (!al16(sb) || !al16(sh) || !al16(st) || (reinterpret_cast<uintptr_t>(k) % 16) ||
+      (reinterpret_cast<uintptr_t>(v) % 16))
+    return TQ_ERR_UNSUPPORTED;
+  if ((rc != nullptr) && ((reinterpret_cast<uintptr_t>(rc) % 16) || (reinterpret_cast<uintptr_t>(rs) % 16)))
+    return TQ_ERR_UNSUPPORTED;
+  if (pos0 + T > (int64_t(1) << 30) || row0 + T > (int64_t(1) << 30)) return TQ_ERR_UNSUPPORTED;
+  TileArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = T;
+  a.row0 = row0;
+  a.pos0 = pos0;
+  a.rows_cap = cache->rows_cap;
+  a.R_first = row0 / QR * QR;
+  a.nrt = (row0 + T - 1) / QR - row0 / QR + 1;
+  a.ntiles = a.nrt * B * H;
+  a.kcode = cache->kcode;
+  a.kscale = cache->kscale;
+  a.vcode = cache->vcode;
+  a.vnorm = cache->vnorm;
+  a.status = status;
+  a.S = c->S_dev;
+  a.rope = rc != nullptr;
+  const int hk = 1 << (mbk - 1), hv = 1 << (bv - 1);
+  for (int m = 0; m < 8; ++m) {
+    a.ck[m] = m < hk ? c->books.ck[hk + m] : 0.f;
+    a.tk[m] = m < hk - 1 ? c->books.tk[hk + m] : 0.f;
+    a.tv[m] = m < hv - 1 ? c->books.tv[hv + m] : 0.f;
+  }
+  for (int w = 0; w < 4; ++w) a.dneg[w] = w < d / 32 ? c->books.dneg[w] : 0u;
+  // tensor maps: K and V [B][H][T][d] bf16 (4-D, innermost d); RoPE tables [pos0 + T][d/2] fp32
+  CUtensorMap mk, mv, mc, ms;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t str[3] = {static_cast<cuuint64_t>(st * 2), static_cast<cuuint64_t>(sh * 2),
+                             static_cast<cuuint64_t>(sb * 2)};
+  const cuuint32_t box[4] = {64, QR, 1, 1};
+  if (!make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(k), dims, str, box) ||
+      !make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(v), dims, str, box))
+    return TQ_ERR_UNSUPPORTED;
+  if (a.rope) {
+    const cuuint64_t tdims[2] = {static_cast<cuuint64_t>(d / 2), static_cast<cuuint64_t>(pos0 + T)};
+    const cuuint64_t tstr[1] = {static_cast<cuuint64_t>(d / 2 * 4)};
+    const cuuint32_t tbox[2] = {32, QR};
+    if (!make_map(&mc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(rc), tdims, tstr, tbox) ||
+        !make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(rs), tdims, tstr, tbox))
+      return TQ_ERR_UNSUPPORTED;
+  } else {
+    mc = mk;   // unused
+    ms = mk;
+  }
+  const int key = d * 1000 + mbk * 100 + bv * 10 + c->qjl_k;
+  switch (key) {
+    case 64231: return run_tile<64, 2, 3, true>(a, mk, mv, mc, ms, stream);
+    case 128341: return run_tile<128, 3, 4, true>(a, mk, mv, mc, ms, stream);
+    case 128121: return run_tile<128, 1, 2, true>(a, mk, mv, mc, ms, stream);
+    case 128231: return run_tile<128, 2, 3, true>(a, mk, mv, mc, ms, stream);
+    case 64331: return run_tile<64, 3, 3, true>(a, mk, mv, mc, ms, stream);
+    case 128440: return run_tile<128, 4, 4, false>(a, mk, mv, mc, ms, stream);
+    case 128330: return run_tile<128, 3, 3, false>(a, mk, mv, mc, ms, stream);
+    case 64330: return run_tile<64, 3, 3, false>(a, mk, mv, mc, ms, stream);
+    default: return TQ_ERR_UNSUPPORTED;
+  }
+}

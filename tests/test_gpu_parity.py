@@ -40,6 +40,13 @@ QUANT_CASES = {
     # large call, fp32 input, MSE-only keys (no sketch)
     "llama_lanes_fp32_mse": (synth.WORKLOADS["llama_decode"].scaled(T=1100, dtype="fp32", qjl_k=False,
                                                                      bits_k=3), [(0, 1100)]),
+    # large bf16 calls take the one-thread-per-row tile kernel; the second call
+    # starts mid-tile and mid value group (row 600)
+    "llama_tile_offset": (synth.WORKLOADS["llama_decode"].scaled(B=2, T=1100), [(0, 600), (600, 500)]),
+    "llama_tile_mse4": (synth.WORKLOADS["llama_decode"].scaled(T=1100, qjl_k=False, bits_k=4), [(0, 1100)]),
+    "esm_tile_mse3_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=100, qjl_k=False, bits_k=3),
+                          [(0, 100)]),
+    "esm_tile_offset_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=300), [(0, 45), (45, 255)]),
 }
 
 
@@ -93,8 +100,9 @@ def test_quantize_parity(case, impl, monkeypatch):
     assert not gpu["vnorm"][:, :, written:].any()
 
 
-@pytest.mark.parametrize("T", [64, 4096])   # 4096: 256 token groups, the tensor-core sketch kernel
-def test_quantize_zero_and_nonfinite_rows(T):
+@pytest.mark.parametrize("T,dtype", [(64, "fp32"), (4096, "fp32"), (4096, "bf16")])
+def test_quantize_zero_and_nonfinite_rows(T, dtype):
+    # 4096 rows: 256 token groups, the large-call kernels (bf16: one thread per row)
     w = synth.WORKLOADS["llama_decode"].scaled(B=1, Hkv=2, Hq=8, T=T)
     ocodec, ncodec = tl.codecs(w)
     K, V, K64, V64 = _inputs(w)
@@ -105,14 +113,23 @@ def test_quantize_zero_and_nonfinite_rows(T):
     Vf[0, 0, 9, 2] = np.inf
     Vf[0, 1, 10] = 0.0
     Kf[0, 1, 40, 0] = 1e6          # key norm overflows fp16
+    if dtype == "bf16":            # every value above is exact in bf16
+        Kf = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.nan_to_num(Kf, nan=0.0, posinf=0.0)))
+        Kf[0, 1, 5, 17] = np.nan
+        Vf = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.nan_to_num(Vf, nan=0.0, posinf=0.0)))
+        Vf[0, 0, 9, 2] = np.inf
     w32 = w.scaled(dtype="fp32")
     rope = synth.rope_for(w32, T)
     ocache = oc.empty_cache(ocodec, 1, 2, T)
     diag = oc.quantize_into(ocache, Kf.astype(np.float64), Vf.astype(np.float64), ocodec, rope=rope)
     ncache = native.alloc_cache(ncodec, 1, 2, T)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    native.quantize_kv(ncodec, tl.to_device(Kf, "fp32"), tl.to_device(Vf, "fp32"), ncache,
-                       rope=tl.rope_device(rope), status=status)
+    if dtype == "bf16":
+        kd = torch.from_numpy(Kf).cuda().to(torch.bfloat16)
+        vd = torch.from_numpy(Vf).cuda().to(torch.bfloat16)
+    else:
+        kd, vd = tl.to_device(Kf, "fp32"), tl.to_device(Vf, "fp32")
+    native.quantize_kv(ncodec, kd, vd, ncache, rope=tl.rope_device(rope), status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == diag["bad_rows"] == 3
     gpu = tl.download_cache(ncache)

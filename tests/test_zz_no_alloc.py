@@ -66,6 +66,31 @@ def test_noalloc_matches_workspace_decode_two_calls():
         assert torch.isfinite(out).all()
 
 
+def test_noalloc_leftovers_of_a_larger_call_do_not_leak():
+    """A call with many splits over many heads fills most of the shared
+    scratch; the next call, with fewer splits and unequal lengths (so some of
+    its chunks are empty), must not pick up any of those partials."""
+    big = synth.WORKLOADS["long_decode"].scaled(B=4, Hq=32, Hkv=8, T=4096)
+    ncodec, cache, q, rope = _setup(big, 2)
+    out = torch.empty((big.B, big.Hq, big.d), dtype=torch.float32, device="cuda")
+    native.attention_decode_noalloc(ncodec, q, cache, big.T, 1 / math.sqrt(big.d), out,
+                                    rope=rope, num_splits=128)
+    small = big.scaled(B=3)
+    lens = torch.tensor([4096, 700, 1], dtype=torch.int32, device="cuda")
+    q3 = q[:3].contiguous()
+    cache3 = native.Cache(cache.kcode[:3], cache.kscale[:3], cache.vcode[:3], cache.vnorm[:3], 3,
+                          cache.Hkv, cache.rows_cap)
+    ref = _reference(ncodec, cache3, q3, small, lens, rope, 16)
+    got = torch.full_like(ref, float("nan"))
+    native.attention_decode_noalloc(ncodec, q3, cache3, small.T, 1 / math.sqrt(small.d), got,
+                                    seq_lens=lens, rope=rope, num_splits=16)
+    torch.cuda.synchronize()
+    vscale = torch.as_tensor(tl.channel_scale_of_values(small), dtype=torch.float32,
+                             device="cuda").repeat_interleave(small.G, dim=0)
+    err = ((got - ref).abs() / vscale[None]).max().item()
+    assert err <= TOL, err
+
+
 def test_noalloc_rejects_shapes_beyond_the_static_scratch():
     w = synth.WORKLOADS["long_decode"]
     _, ncodec = tl.codecs(w)
