@@ -45,7 +45,7 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
-                                      "vector_search", "quality"],
+                                      "decode_llama", "vector_search", "quality"],
                    help="run one extra workload alone and print its JSON (1 GPU)")
     p.add_argument("--search-rows", type=int, default=0,
                    help="vector-search database rows for --only vector_search (default 10^6)")
@@ -178,7 +178,8 @@ def describe(w) -> str:
     kdesc = f"{mse_k}+QJL" if w.qjl_k else f"{mse_k}"
     rope = f" RoPE theta={w.rope_theta:g}" if w.rope_theta else ""
     return (f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} T={w.T} keys {kdesc} bits, "
-            f"values {w.bits_v} bits, {w.dtype} inputs{rope}, {w.num_splits} splits")
+            f"values {w.bits_v} bits, {w.dtype} inputs{rope}, "
+            + (f"{w.num_splits} splits" if w.num_splits else "default split count"))
 
 
 class DecodeBench:
@@ -703,6 +704,19 @@ def search_extra(pk: dict, steps: int = 5):
         st.append(e_s0.elapsed_time(e_s1) / 1e3)
         kt.append(ev[2].elapsed_time(ev[3]) / 1e3)
     b, s_, k = statistics.median(bt), statistics.median(st), statistics.median(kt)
+    # the lookup-table scan (fp32 scores) on the first 64 queries, for comparison
+    nql = 64
+    ql = q[:nql].contiguous()
+    il = torch.empty((nql, w.k), dtype=torch.int32, device="cuda")
+    sl = torch.empty((nql, w.k), dtype=torch.float32, device="cuda")
+    native.scan_topk_lut(codec, kcode, kscale, ql, w.k, il, sl, sws)
+    torch.cuda.synchronize()
+    e_l0, e_l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_l0.record()
+    native.scan_topk_lut(codec, kcode, kscale, ql, w.k, il, sl, sws)
+    e_l1.record()
+    torch.cuda.synchronize()
+    lt = e_l0.elapsed_time(e_l1) / 1e3
     in_bytes = w.n * w.d * 4
     sketch_flops = 2 * w.n * w.d * w.d
     scan_flops = 2 * 2 * w.d * w.n * w.nq
@@ -722,6 +736,9 @@ def search_extra(pk: dict, steps: int = 5):
                                      unit="TFLOP/s", frac=scan_flops / k / 1e12 / pk["bf16"],
                                      algorithmic_flops=scan_flops, kernel="ix_scan2_kernel",
                                      kernel_ms=k * 1e3)),
+        scan_topk_lut=dict(queries=nql, ms_per_call=lt * 1e3, queries_per_s=nql / lt,
+                           note="lookup-table scan, fp32 scores, same database; the comparison "
+                                "path to the tensor-core scan"),
         l2="database codes 772 MB and input 6.1 GB > L2")
 
 
@@ -851,6 +868,8 @@ def run_only(args) -> int:
         r = bidir_extra(pk, steps=1)
     elif args.only == "decode_long_context":
         r = decode_extra("long_decode", pk, steps=5, warmup=3)
+    elif args.only == "decode_llama":
+        r = decode_extra("llama_decode", pk, steps=5, warmup=3)
     elif args.only == "quality":
         r = {name: quality_extra(name) for name in ("tiny", "llama_decode", "esm_prefill", "long_decode")}
         r["llama_decode_without_outliers"] = quality_extra(

@@ -165,10 +165,16 @@ int tq_quantize_kv(const tq_codec *codec, const void *k, const void *v, int dtyp
  * seq_lens device int32 [B], nullable (then every batch has max_seq_len);
  *          entries are clamped to 1..max_seq_len; max_seq_len <= rows_cap.
  * rope_cos/rope_sin  as for tq_quantize_kv (nullable together).
- * num_splits  chunks per (b, KV head), at most 512; 0 picks the default 64.
+ * num_splits  chunks per (b, KV head), at most 512; 0 picks a default of at
+ *          most 64 (about two chunks per SM over all (b, KV head), in
+ *          128-row multiples), which a workspace sized with num_splits = 0 fits.
  * workspace   device, >= tq_attention_workspace(...) bytes, 16-byte aligned;
  *             scratch owned by the caller, contents need no initialisation.
  * out      device fp32 [B][Hq][d].
+ * Every wait inside the kernels is bounded.  If one gives up (a copy or MMA
+ * that never completes), the kernel drains its own outstanding copies and
+ * MMAs, records it in a status word of the workspace, and every element of
+ * out is written as NaN instead of a merge of incomplete partials.
  * ------------------------------------------------------------------------ */
 int tq_attention_workspace(const tq_codec *codec, int B, int Hq, int num_splits, size_t *bytes);
 int tq_attention_decode(const tq_codec *codec, const void *q, int dtype, int B, int Hq,
@@ -249,6 +255,16 @@ int tq_scan_topk(const tq_codec *codec, const uint8_t *kcode, const uint16_t *ks
                  const float *q, int nq, int k, int32_t *idx, float *score, void *workspace,
                  size_t ws_bytes, void *stream);
 
+/* Same scan by lookup tables instead of tensor-core tiles (the comparison
+ * path; same pages and estimator): per query, T[i][m] = (Pi q)_i c[m] and
+ * sqrt(pi/2)/1536 (S Pi q)_i in shared memory, one lookup and one signed add
+ * per coordinate in fp32, so scores carry only fp32 rounding (no fp16
+ * products).  Arguments, workspace (tq_scan_workspace covers both paths) and
+ * output order as tq_scan_topk; kcode and kscale need 4-byte alignment. */
+int tq_scan_topk_lut(const tq_codec *codec, const uint8_t *kcode, const uint16_t *kscale,
+                     int64_t n, const float *q, int nq, int k, int32_t *idx, float *score,
+                     void *workspace, size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------
  * Decode without a workspace, for callers that cannot allocate device memory.
  *
@@ -262,12 +278,14 @@ int tq_scan_topk(const tq_codec *codec, const uint8_t *kcode, const uint16_t *ks
  * workspace.
  *   - The first call on each device looks the array's device address up
  *     (cudaGetSymbolAddress, that device current) and caches it.
- *   - Shapes needing more scratch than the limit, i.e.
- *     B*Hq*(2d + num_splits*(d+2))*4 bytes > 16 MiB, return TQ_ERR_WORKSPACE.
- *   - All calls share the array (each leaves its contents there; every word is
- *     written before it is read, so nothing needs clearing).  Calls whose
- *     kernels overlap on the GPU (other streams, other host threads) race on
- *     it: the caller must serialise them.
+ *   - Shapes whose scratch, the byte count tq_attention_workspace() returns
+ *     for the same codec, B, Hq and num_splits, exceeds the 16 MiB limit
+ *     return TQ_ERR_WORKSPACE.
+ *   - All calls share the array and each leaves its contents there.  Every
+ *     scratch word a call reads it has written itself earlier in the same
+ *     call (the status word included), so nothing needs clearing.  Calls
+ *     whose kernels overlap on the GPU (other streams, other host threads)
+ *     race on it: the caller must serialise them.
  * ------------------------------------------------------------------------ */
 #define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 int tq_attention_decode_noalloc(const tq_codec *codec, const void *q, int dtype, int B, int Hq,

@@ -258,7 +258,20 @@ int decode_common(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "decode: scale not finite");
   if ((rope_cos == nullptr) != (rope_sin == nullptr))
     return tq_fail(TQ_ERR_INVALID_ARG, "decode: rope_cos and rope_sin go together");
-  const int splits = num_splits > 0 ? num_splits : 64;
+  int splits = num_splits > 0 ? num_splits : 64;
+  if (num_splits == 0) {
+    // default: about one chunk per resident CTA (two per SM), 128-row
+    // multiples, never more than the 64 splits tq_attention_workspace(.., 0)
+    // sized the workspace for
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int bh = B * Hkv;
+    int s = (2 * sms + bh - 1) / bh;
+    s = s < 1 ? 1 : (s > 64 ? 64 : s);
+    const int chunk = ((max_seq_len + s - 1) / s + 127) / 128 * 128;
+    splits = (max_seq_len + chunk - 1) / chunk;
+  }
   if (splits > 512) return tq_fail(TQ_ERR_INVALID_ARG, "decode: num_splits must be <= 512");
   if (decode_workspace_bytes(c, B, Hq, splits) > ws_bytes)
     return tq_fail(TQ_ERR_WORKSPACE, "decode: workspace smaller than tq_attention_workspace()");

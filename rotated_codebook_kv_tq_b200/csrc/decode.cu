@@ -52,6 +52,7 @@ struct DecodeArgs {
   float *pml;         // [B][Hq][splits][2]
   float *out;         // [B][Hq][D]
   float *logits;      // optional [B][Hq][max_len] (phase-1 logits)
+  const uint32_t *err;  // optional: nonzero when the chunk kernel gave up a wait
   TqBooks books;
 };
 
@@ -301,6 +302,11 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
   const int c = tid % D, gq = tid / D;
   const int64_t head = blockIdx.x;
   const int S = a.splits;
+  if (a.err && *a.err) {
+    // a bounded wait of the chunk kernel gave up: its partials are incomplete
+    if (tid < D) a.out[head * D + tid] = CUDART_NAN_F;
+    return;
+  }
   float m = -CUDART_INF_F;
   for (int s = tid; s < S; s += NT) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
@@ -398,8 +404,10 @@ size_t ws_bk_bytes(const tq_codec *c, int B, int Hq) {
 }
 }  // namespace
 
+// Layout: q', q'', chunk partials (ws_core_bytes) | tensor-core B operands
+// (ws_bk_bytes) | one status word (128-byte slot).
 size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits) {
-  return ws_core_bytes(c, B, Hq, splits) + ws_bk_bytes(c, B, Hq);
+  return ws_core_bytes(c, B, Hq, splits) + ws_bk_bytes(c, B, Hq) + 128;
 }
 
 int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
@@ -437,6 +445,7 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   a.pml = a.po + heads * static_cast<size_t>(splits) * c->d;
   a.out = out;
   a.logits = logits;
+  a.err = nullptr;
   a.books = c->books;
   // TQ_DECODE_IMPL=simt selects the CUDA-core kernels (a complete second
   // implementation, used to cross-check the tensor-core path)
@@ -444,8 +453,10 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   const bool want_tc = !(impl && impl[0] == 's');
   if (want_tc && tc_supported(c, a.G)) {
     uint8_t *bk = static_cast<uint8_t *>(ws) + ws_core_bytes(c, B, Hq, splits);
+    uint32_t *err = reinterpret_cast<uint32_t *>(bk + ws_bk_bytes(c, B, Hq));
+    a.err = err;
     if (int e = launch_decode_tc(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_len, scale, rc,
-                                 rs, splits, a.po, a.pml, bk, logits, stream))
+                                 rs, splits, a.po, a.pml, bk, logits, err, stream))
       return e;
     combine_kernel<128><<<B * Hq, CMB * 128, 0, stream>>>(a);
     tq_count_launch(1);

@@ -19,14 +19,14 @@
 //   Values: M = 128 coordinates (TMEM lane = coordinate; the cache's 32-token
 //   column groups give each lane its own words), N = 4 limbs x G heads,
 //   K = 32 tokens; one accumulator per Walsh term, combined at the end.
-// * Persistent CTAs, one per SM, stream (chunk, sub-chunk) units through a
-//   double-buffered shared-memory ring filled by cp.async.bulk.  Each CTA has
-//   two 4-warp slices over the same 128 TMEM lanes that split the Walsh terms
-//   of every expansion, and key tiles are double-buffered in tensor memory so
-//   the expansion of tile j+1 overlaps the MMAs of tile j.
+// * dec_kernel (two CTAs per SM) walks (batch, KV head, split) units of at
+//   most 1024 rows phase by phase: key tiles through a ring of tensor-memory
+//   term slots, the unit's softmax and value-side B operand, then value
+//   groups; bulk copies run ahead of use in shared-memory rings, and two
+//   warps issue the MMAs side by side.
 //
 // Kernels: tc_prep (per (batch, KV head): RoPE, rotation and sketch of the G
-// query heads, fixed-point B operand for the keys) and tc_chunk (the split-K
+// query heads, fixed-point B operand for the keys) and dec_kernel (the split-K
 // main loop); the chunk partials are merged by decode.cu's combine kernel.
 #include <math_constants.h>
 
@@ -41,9 +41,6 @@ namespace {
 constexpr int TD = 128;   // head dim of this path
 constexpr int TNW = TD / 32;
 constexpr int TCT = 128;  // threads of tc_prep: one TMEM lane each
-constexpr int CW = 256;   // worker threads of tc_chunk: two slices of 128 TMEM lanes
-constexpr int CT = CW + 32;   // + the MMA-issuing warp
-
 // Odd subsets of {0..nb-1} in increasing bit-mask order (the Walsh terms).
 __host__ __device__ constexpr int odd_mask(int nb, int t) {
   int seen = 0;
@@ -56,33 +53,6 @@ __host__ __device__ constexpr int odd_mask(int nb, int t) {
     }
   }
   return 0;
-}
-
-// Columns used by tc_chunk: key phase (two accumulator pairs in [0, 64), two
-// A buffers of 32 columns per key term from 64) or value phase (two A buffers
-// of 8 columns per Walsh term, then one accumulator of N columns per term).
-__host__ __device__ constexpr int tc_tmem_cols(int G, int MBK, int BV, bool QJL) {
-  return (64 + 64 * ((1 << (MBK - 1)) + (QJL ? 1 : 0))) > (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G))
-             ? (64 + 64 * ((1 << (MBK - 1)) + (QJL ? 1 : 0)))
-             : (2 * (1 << (BV - 1)) * 8 + (1 << (BV - 1)) * tc_n(G));
-}
-__host__ __device__ constexpr int tc_tmem_alloc(int G, int MBK, int BV, bool QJL) {
-  return tc_tmem_cols(G, MBK, BV, QJL) <= 64    ? 64
-         : tc_tmem_cols(G, MBK, BV, QJL) <= 128 ? 128
-         : tc_tmem_cols(G, MBK, BV, QJL) <= 256 ? 256
-                                                 : 512;
-}
-
-// Signed base-256 digits of v (|v| < 2^31): v = L0 + 2^8 L1 + 2^16 L2 + 2^24 L3.
-__device__ __forceinline__ int8_t limb_of(int v, int l) {
-  int8_t d = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    d = static_cast<int8_t>(v & 0xff);
-    if (i == l) break;
-    v = (v - d) >> 8;
-  }
-  return d;
 }
 
 // Byte offset of element (n, k) in a K-major, no-swizzle operand of N rows.
@@ -117,6 +87,7 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
   const int b = bh / a.Hkv, kvh = bh % a.Hkv;
   const int len = a.seq_lens ? min(max(a.seq_lens[b], 1), a.max_len) : a.max_len;
   const int64_t pos = len - 1;
+  if (bh == 0 && tid == 0 && a.err) *a.err = 0u;   // this call's give-up flag
 
   if (warp < G) {
     const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + warp;
@@ -277,23 +248,6 @@ __device__ __forceinline__ float comb_limbs(const uint32_t *d) {
   return fmaf(v, 256.f, static_cast<float>(static_cast<int>(d[0])));
 }
 
-struct TcLayout {
-  int o_ks, o_vc, o_vn, o_bk, ubytes, o_bv, o_lg, total;
-};
-
-__host__ __device__ inline TcLayout tc_layout(int sub, int PK, int BV, int G, int N, int BKC) {
-  TcLayout L;
-  L.o_ks = sub * PK * 16;
-  L.o_vc = L.o_ks + sub * 4;
-  L.o_vn = L.o_vc + (sub / 32) * BV * TD * 4;
-  L.o_bk = L.o_vn + sub * 2;
-  L.ubytes = (L.o_bk + BKC + 127) & ~127;
-  L.o_bv = 2 * L.ubytes;
-  L.o_lg = L.o_bv + (sub / 32) * N * 32;
-  L.total = L.o_lg + sub * G * 4;
-  return L;
-}
-
 __device__ __forceinline__ int tc_len(const TcArgs &a, int b) {
   return a.seq_lens ? min(max(a.seq_lens[b], 1), a.max_len) : a.max_len;
 }
@@ -313,18 +267,79 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
   return false;
 }
 
-// tc_chunk: 288 threads = 8 worker warps (two slices of 4) + 1 MMA warp.
-// Worker warp w serves TMEM lane quarter w % 4 (rows or coordinates
-// 32 (w % 4) .. +31) for slice w / 4; the slices split the Walsh terms of
-// every expansion and the rows of the value B-operand build.  A tcgen05.mma
-// issue blocks for about as long as the MMA runs, so one lane of the last
-// warp does nothing but issue: workers publish each filled tensor-memory
-// buffer on an mbarrier (ak_full / av_full) and the MMA warp waits on those;
-// workers wait on the MMA commits (mb_k / mb_v) before reusing a buffer.
-// Key tiles are double-buffered: tile j+1 is expanded while tile j runs.
+// ---------------------------------------------------------------------------
+// dec_kernel: split-K decode main loop.  Two CTAs per SM, each walking its
+// (batch, KV head, split) units (at most UMAX rows) phase by phase:
+//   K  key tiles of 128 rows: bit planes -> Walsh-term operands in tensor
+//      memory (a ring of NSLOT term slots) -> kind::i8 MMAs against the
+//      fixed-point query (B, shared memory) -> logits of the G heads;
+//   S  softmax statistics of the unit and the value-side B operand (24-bit
+//      weights p * nu_v as four int8 limbs) for all of its 32-token groups;
+//   V  value groups: bit planes -> Walsh-term operands (lane = coordinate) ->
+//      MMAs accumulating the rotated-domain sums over the unit;
+//   E  fold the value accumulators into the running output of the chunk.
+// The two CTAs of an SM overlap each other's S and E phases with streaming.
+// Warp roles: 0-3 expand key tiles and value groups and run E (one TMEM lane
+// each); 4-7 run the key epilogue; 0-7 share S; 8-9 issue MMAs (a tcgen05.mma
+// issue holds its thread for ~45 cycles at these N, so two warps issue side
+// by side: key terms alternate between them, each into its own accumulator,
+// summed exactly in the epilogue); 10 issues every bulk copy ahead of use.
+// Every wait is bounded and warp-uniform; one that gives up makes the whole
+// CTA drain its copies and MMAs and set the call's status word.
+// ---------------------------------------------------------------------------
+constexpr int DT = 352;        // 11 warps
+constexpr int UMAX = 1024;     // rows per unit
+constexpr int KS = 3;          // key tile stages (shared memory)
+constexpr int VS = 6;          // value group stages (shared memory)
+constexpr int NSLOT = 4;       // key term slots in tensor memory (32 columns each)
+constexpr int DCOLS = 256;     // tensor memory per CTA
+
+struct DecLayout {
+  int ktb, vgb, bkc, o_kt, o_vt, o_bk, o_vn, o_lg, o_bv, total;
+};
+
+__host__ __device__ inline DecLayout dec_layout(int PK, int BV, int G, int N, int BKC) {
+  DecLayout L;
+  L.ktb = (128 * PK * 16 + 128 * 4 + 127) & ~127;
+  L.vgb = BV * TD * 4;
+  L.bkc = (BKC + 127) & ~127;
+  L.o_kt = 0;
+  L.o_vt = L.o_kt + KS * L.ktb;
+  L.o_bk = L.o_vt + VS * L.vgb;
+  L.o_vn = L.o_bk + 2 * L.bkc;
+  L.o_lg = L.o_vn + 2 * UMAX * 2;
+  L.o_bv = L.o_lg + UMAX * G * 4;
+  L.total = L.o_bv + (UMAX / 32) * N * 32;
+  return L;
+}
+
+// Warp-uniform bounded wait: every lane polls (so every lane acquires the
+// phase), the loop ends for all lanes together.  Gives up when the budget
+// runs out or another warp has given up.
+__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, uint32_t outer,
+                                      volatile int *abort_flag) {
+  for (uint32_t it = 0; it < outer; ++it) {
+    const bool ok = sm100::mbar_wait(bar, parity, 1u << 8);
+    if (__all_sync(TQ_FULL, ok)) return true;
+    if (__shfl_sync(TQ_FULL, *abort_flag, 0)) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// Single-thread bounded wait for the issuing and copying lanes.
+__device__ __forceinline__ bool dwait1(uint64_t *bar, uint32_t parity, uint32_t outer,
+                                       volatile int *abort_flag) {
+  for (uint32_t it = 0; it < outer; ++it) {
+    if (sm100::mbar_wait(bar, parity, 1u << 8)) return true;
+    if (*abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
 template <int G, int MBK, int BV, bool QJL>
-__global__ void __launch_bounds__(CT, 1) tc_chunk_kernel(TcArgs a) {
-  constexpr int NWW = CW / 32;               // worker warps
+__global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
   constexpr int TK = 1 << (MBK - 1);
   constexpr int TV = 1 << (BV - 1);
   constexpr int N = tc_n(G);
@@ -333,50 +348,47 @@ __global__ void __launch_bounds__(CT, 1) tc_chunk_kernel(TcArgs a) {
   constexpr int KTOT = KM + (QJL ? TD : 0);
   constexpr int BKB = N * KTOT;
   constexpr int BKC = BKB + G * 16;
-  constexpr int NKT = TK + (QJL ? 1 : 0);   // key terms: TK Walsh terms + the sign plane
-  // Tensor memory: the key phase and the value phase of a unit never overlap
-  // in time, so their regions share columns.
-  //   key phase:   DK[b] [32 b, 32 b + 2N)   AK[b] [64 + 32 NKT b, 64 + 32 NKT (b + 1))
-  //   value phase: AV [0, 16 TV) (two buffers)   DV [16 TV, 16 TV + N TV)
-  constexpr int C_DK = 0;
-  constexpr int C_AK = 64;
-  constexpr int C_AV = 0;
-  constexpr int C_DV = 2 * TV * 8;
-  constexpr int USED = tc_tmem_cols(G, MBK, BV, QJL);
-  constexpr int NCOLS = tc_tmem_alloc(G, MBK, BV, QJL);
-  static_assert(USED <= 512, "tensor memory budget");
-  static_assert(2 * N <= 32, "key accumulators must fit in 32 columns");
+  constexpr int NKT = TK + (QJL ? 1 : 0);
+  constexpr int NACC = (TK >= 2 ? 2 : 1) + (QJL ? 1 : 0);   // key accumulators per tile
+  // tensor memory (256 columns): key phase: term slots [0, 128), D_k[2] from 128;
+  // value phase: A_v[2] [0, 16 TV), D_v [128, 128 + N TV)
+  constexpr int C_SLOT = 0, C_DK = 128, C_AV = 0, C_DV = 128;
+  static_assert(C_DK + 2 * NACC * N <= DCOLS && C_DV + TV * N <= DCOLS && 2 * TV * 8 <= 128,
+                "tensor memory budget");
   constexpr uint32_t IDESC = sm100::idesc_i8(128, N);
+  const DecLayout L = dec_layout(PK, BV, G, N, BKC);
 
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t mb_load[2], mb_k[2], mb_v[2], ak_full[2], av_full[2];
+  __shared__ __align__(8) uint64_t kf[KS], ke[KS], vf[VS], ve[VS], hdr[2], hdr_free[2];
+  __shared__ __align__(8) uint64_t as_full[NSLOT], as_empty[NSLOT], dk_full[2], dk_empty[2];
+  __shared__ __align__(8) uint64_t av_full[2], av_empty[2], bv_full, dv_full, tm_free, sbar, done[2];
   __shared__ uint32_t tmem_s;
-  __shared__ float redf[NWW][2 * G + 1];
-  __shared__ long long redi[NWW][G];
-  __shared__ float part[G][TD];
-  __shared__ int abort_s;
+  __shared__ volatile int abort_s;
+  __shared__ float redf[8][2 * G + 1];
+  __shared__ unsigned long long wsum_s[8];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int wq = warp & 3;            // TMEM lane quarter
-  const int slice = warp >> 2;        // 0 or 1
-  const int lt = tid & 127;           // TMEM lane = row (keys) or coordinate (values)
-  const int sub = a.sub;
-  const TcLayout L = tc_layout(sub, PK, BV, G, N, BKC);
-  int8_t *bvs = reinterpret_cast<int8_t *>(smem + L.o_bv);
-  float *lg = reinterpret_cast<float *>(smem + L.o_lg);
+  const int lt = tid & 127;
+  const uint32_t outer = a.wait_limit >> 8;
 
-  if (warp == 0) sm100::tmem_alloc(&tmem_s, NCOLS);
+  if (warp == 0) sm100::tmem_alloc(&tmem_s, DCOLS);
   if (tid == 0) {
-    sm100::mbar_init(&mb_load[0], 1);
-    sm100::mbar_init(&mb_load[1], 1);
-    sm100::mbar_init(&mb_k[0], 1);
-    sm100::mbar_init(&mb_k[1], 1);
-    sm100::mbar_init(&mb_v[0], 1);
-    sm100::mbar_init(&mb_v[1], 1);
-    sm100::mbar_init(&ak_full[0], NWW);
-    sm100::mbar_init(&ak_full[1], NWW);
-    sm100::mbar_init(&av_full[0], NWW);
-    sm100::mbar_init(&av_full[1], NWW);
+    for (int i = 0; i < KS; ++i) { sm100::mbar_init(&kf[i], 1); sm100::mbar_init(&ke[i], 8); }
+    for (int i = 0; i < VS; ++i) { sm100::mbar_init(&vf[i], 1); sm100::mbar_init(&ve[i], 4); }
+    for (int i = 0; i < NSLOT; ++i) { sm100::mbar_init(&as_full[i], 4); sm100::mbar_init(&as_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&hdr[i], 1);
+      sm100::mbar_init(&hdr_free[i], 8);
+      sm100::mbar_init(&dk_full[i], 2);
+      sm100::mbar_init(&dk_empty[i], 4);
+      sm100::mbar_init(&av_full[i], 4);
+      sm100::mbar_init(&av_empty[i], 2);
+      sm100::mbar_init(&done[i], 1);
+    }
+    sm100::mbar_init(&bv_full, 8);
+    sm100::mbar_init(&dv_full, 2);
+    sm100::mbar_init(&tm_free, 4);
+    sm100::mbar_init(&sbar, 8);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -385,452 +397,488 @@ __global__ void __launch_bounds__(CT, 1) tc_chunk_kernel(TcArgs a) {
   sm100::fence_after_sync();
   const uint32_t tm = tmem_s;
 
-  if (warp == NWW) {
-    // ---------------- MMA warp: walks the same units as the workers
+  // empty chunks (beyond a batch's length) merge with weight zero
+  if (warp < 8) {
+    const int items = a.B * a.Hkv * a.splits;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv, sp = it % a.splits;
+      if (sp * a.chunk < tc_len(a, b)) continue;
+      if (tid < TD)
+        for (int h = 0; h < G; ++h) {
+          const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
+          a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
+          if (tid == 0) {
+            a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
+            a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
+          }
+        }
+    }
+  }
+
+  if (warp == 10) {
+    // ------------------------------------------------------------ copies
     if (lane == 0) {
       int cit = blockIdx.x, cr0 = -1, u = 0;
-      uint32_t akph = 0, avph = 0;
+      uint32_t kt = 0, vg = 0;
+      // per stage: 1 + the parity of its last issued copy (0 = never issued)
+      uint8_t lk[KS] = {}, lv[VS] = {}, lh[2] = {};
+      bool have = tc_next(a, cit, cr0);
+      while (have && !abort_s) {
+        const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
+        const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
+        const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
+        const int nvalid = min(a.sub, c1 - cr0);
+        const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
+        // unit header: this unit's B operand and value norms (buffer u & 1),
+        // once unit u - 2 has finished its softmax phase with that buffer
+        {
+          const int hb = u & 1;
+          if (u >= 2 && !dwait1(&hdr_free[hb], ((u >> 1) - 1) & 1, outer, &abort_s)) break;
+          const uint32_t nvn = static_cast<uint32_t>(ngroups) * 64;
+          sm100::mbar_expect_tx(&hdr[hb], static_cast<uint32_t>((BKC + 15) & ~15) + nvn);
+          sm100::bulk_g2s(smem + L.o_bk + hb * L.bkc, a.bk + bh * a.bk_stride, (BKC + 15) & ~15, &hdr[hb]);
+          sm100::bulk_g2s(smem + L.o_vn + hb * UMAX * 2, a.vnorm + bh * a.rows_cap + cr0, nvn, &hdr[hb]);
+          lh[hb] = static_cast<uint8_t>(1 + ((u >> 1) & 1));
+        }
+        for (int j = 0; j < ntile && !abort_s; ++j, ++kt) {
+          const int s = kt % KS;
+          if (kt >= KS && !dwait1(&ke[s], ((kt / KS) - 1) & 1, outer, &abort_s)) break;
+          const int64_t row = cr0 + j * 128;
+          const uint32_t nrow = static_cast<uint32_t>(min(static_cast<int64_t>(128), a.rows_cap - row));
+          uint8_t *st = smem + L.o_kt + s * L.ktb;
+          sm100::mbar_expect_tx(&kf[s], nrow * PK * 16 + nrow * 4);
+          sm100::bulk_g2s(st, a.kcode + (bh * a.rows_cap + row) * PK * 16, nrow * PK * 16, &kf[s]);
+          sm100::bulk_g2s(st + 128 * PK * 16, a.kscale + (bh * a.rows_cap + row) * 2, nrow * 4, &kf[s]);
+          lk[s] = static_cast<uint8_t>(1 + ((kt / KS) & 1));
+        }
+        for (int g = 0; g < ngroups && !abort_s; ++g, ++vg) {
+          const int s = vg % VS;
+          if (vg >= VS && !dwait1(&ve[s], ((vg / VS) - 1) & 1, outer, &abort_s)) break;
+          sm100::mbar_expect_tx(&vf[s], L.vgb);
+          sm100::bulk_g2s(smem + L.o_vt + s * L.vgb,
+                          a.vcode + (bh * (a.rows_cap / 32) + cr0 / 32 + g) * BV * TD, L.vgb, &vf[s]);
+          lv[s] = static_cast<uint8_t>(1 + ((vg / VS) & 1));
+        }
+        cr0 += a.sub;
+        have = tc_next(a, cit, cr0);
+        ++u;
+      }
+      if (abort_s) {
+        // this CTA's own copies land before its shared memory is released:
+        // each stage's last issued phase completes (at once if consumed)
+        for (int i = 0; i < KS; ++i)
+          if (lk[i]) sm100::mbar_wait(&kf[i], lk[i] - 1u, 1u << 20);
+        for (int i = 0; i < VS; ++i)
+          if (lv[i]) sm100::mbar_wait(&vf[i], lv[i] - 1u, 1u << 20);
+        for (int i = 0; i < 2; ++i)
+          if (lh[i]) sm100::mbar_wait(&hdr[i], lh[i] - 1u, 1u << 20);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ MMA issue
+    const int is = warp - 8;
+    if (lane == 0) {
+      int cit = blockIdx.x, cr0 = -1, u = 0;
+      uint32_t kt = 0, ts = 0, vg = 0;
       bool have = tc_next(a, cit, cr0);
       bool ok = true;
       while (have && ok) {
-        int nit = cit, nr0 = cr0 + sub;
-        const bool nhave = tc_next(a, nit, nr0);
-        uint8_t *ub = smem + (u & 1) * L.ubytes;
         const int b = cit / (a.Hkv * a.splits), sp = cit % a.splits;
         const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
-        const int nvalid = min(sub, c1 - cr0);
-        const uint32_t bk_addr = sm100::smem_addr(ub + L.o_bk);
+        const int nvalid = min(a.sub, c1 - cr0);
         const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
-        for (int j = 0; j < ntile && ok; ++j) {
-          const int kb = j & 1;
-          ok = sm100::mbar_wait(&ak_full[kb], (akph >> kb) & 1);
-          akph ^= 1u << kb;
-          if (!ok) break;
-          sm100::fence_after_sync();
-          const uint32_t ak = tm + C_AK + kb * 32 * NKT, dk = tm + C_DK + kb * 32;
+        const uint32_t bk_addr = sm100::smem_addr(smem + L.o_bk + (u & 1) * L.bkc);
+        // the previous unit's value epilogue has read D_v (it overlaps D_k)
+        if (u > 0) ok = dwait1(&tm_free, (u - 1) & 1, outer, &abort_s);
+        if (ok) ok = dwait1(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);
+        for (int j = 0; j < ntile && ok; ++j, ++kt) {
+          const int kb = kt & 1;
+          if (kt >= 2 && !(ok = dwait1(&dk_empty[kb], ((kt >> 1) - 1) & 1, outer, &abort_s))) break;
+          const uint32_t dk = tm + C_DK + kb * NACC * N;
+          bool any = false, first_mse = true;
 #pragma unroll
-          for (int s = 0; s < TK * 4; ++s)
-            sm100::mma_i8_ts(dk, ak + s * 8, sm100::smem_desc(bk_addr + s * 2 * N * 16, N * 16, 128),
-                             IDESC, s > 0);
-          if (QJL) {
+          for (int t = 0; t < NKT; ++t, ++ts) {
+            // owner: MSE terms alternate between the two issuers, the sign
+            // plane goes to issuer 1 (issuer 0 when there is one MSE term)
+            const int owner = t < TK ? (t & 1) : (TK >= 2 ? 1 : 0);
+            if (owner != is) continue;
+            const int slot = ts % NSLOT;
+            if (!(ok = dwait1(&as_full[slot], (ts / NSLOT) & 1, outer, &abort_s))) break;
+            sm100::fence_after_sync();
+            const uint32_t acc = t < TK ? dk + is * N : dk + (NACC - 1) * N;
+            const uint32_t boff = t < TK ? static_cast<uint32_t>(t) * 4 * 2 * N * 16 : N * KM;
+            const bool fresh = t < TK ? first_mse : true;
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-              sm100::mma_i8_ts(dk + N, ak + TK * 32 + s * 8,
-                               sm100::smem_desc(bk_addr + N * KM + s * 2 * N * 16, N * 16, 128),
-                               IDESC, s > 0);
+            for (int s4 = 0; s4 < 4; ++s4)
+              sm100::mma_i8_ts(acc, tm + C_SLOT + slot * 32 + s4 * 8,
+                               sm100::smem_desc(bk_addr + boff + s4 * 2 * N * 16, N * 16, 128), IDESC,
+                               (fresh && s4 == 0) ? 0u : 1u);
+            if (t < TK) first_mse = false;
+            sm100::mma_commit(&as_empty[slot]);
+            any = true;
           }
-          sm100::mma_commit(&mb_k[kb]);
-        }
-        const uint32_t bv_addr = sm100::smem_addr(bvs);
-        for (int g = 0; g < ngroups && ok; ++g) {
-          const int ab = g & 1;
-          ok = sm100::mbar_wait(&av_full[ab], (avph >> ab) & 1);
-          avph ^= 1u << ab;
           if (!ok) break;
+          if (any) sm100::mma_commit(&dk_full[kb]);
+          else sm100::mbar_arrive(&dk_full[kb]);
+        }
+        if (!ok) break;
+        // value groups: the unit's B operand is complete
+        ok = dwait1(&bv_full, u & 1, outer, &abort_s);
+        const uint32_t bv_addr = sm100::smem_addr(smem + L.o_bv);
+        for (int g = 0; g < ngroups && ok; ++g, ++vg) {
+          const int ab = vg & 1;
+          if (!(ok = dwait1(&av_full[ab], (vg >> 1) & 1, outer, &abort_s))) break;
           sm100::fence_after_sync();
           const uint64_t bd = sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128);
+          bool any = false;
 #pragma unroll
-          for (int ti = 0; ti < TV; ++ti)
+          for (int ti = 0; ti < TV; ++ti) {
+            if ((ti & 1) != is) continue;
             sm100::mma_i8_ts(tm + C_DV + ti * N, tm + C_AV + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
-          sm100::mma_commit(&mb_v[ab]);
+            any = true;
+          }
+          if (any) sm100::mma_commit(&av_empty[ab]);
+          else sm100::mbar_arrive(&av_empty[ab]);
         }
-        cit = nit;
-        cr0 = nr0;
-        have = nhave;
+        if (!ok) break;
+        sm100::mma_commit(&dv_full);
+        cr0 += a.sub;
+        have = tc_next(a, cit, cr0);
         ++u;
       }
-      // a wait that gave up leaves the workers to time out on the commits
-      // they expect and take their own abort path
+      // every MMA of this thread has landed before tensor memory is freed
+      sm100::mma_commit(&done[is]);
+      sm100::mbar_wait(&done[is], 0, 1u << 20);
     }
     __syncwarp();
   } else {
-  // ---------------- workers
-  // empty chunks (beyond a batch's length) merge with weight zero
-  const int items = a.B * a.Hkv * a.splits;
-  for (int it = blockIdx.x; it < items; it += gridDim.x) {
-    const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv, sp = it % a.splits;
-    if (sp * a.chunk < tc_len(a, b)) continue;
-    if (tid < TD)
-      for (int h = 0; h < G; ++h) {
-        const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-        a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
-        if (tid == 0) {
-          a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
-          a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
-        }
-      }
-  }
-
-  auto issue = [&](int buf, int it, int r0) {
-    const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv;
-    const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
-    const int nrow = static_cast<int>(min(static_cast<int64_t>(sub), a.rows_cap - r0));
-    uint8_t *u = smem + buf * L.ubytes;
-    const uint32_t b_kc = nrow * PK * 16, b_ks = nrow * 4, b_vc = (nrow / 32) * BV * TD * 4,
-                   b_vn = nrow * 2, b_bk = (BKC + 15) & ~15;
-    sm100::mbar_expect_tx(&mb_load[buf], b_kc + b_ks + b_vc + b_vn + b_bk);
-    sm100::bulk_g2s(u, a.kcode + (bh * a.rows_cap + r0) * PK * 16, b_kc, &mb_load[buf]);
-    sm100::bulk_g2s(u + L.o_ks, a.kscale + (bh * a.rows_cap + r0) * 2, b_ks, &mb_load[buf]);
-    sm100::bulk_g2s(u + L.o_vc, a.vcode + (bh * (a.rows_cap / 32) + r0 / 32) * BV * TD, b_vc,
-                    &mb_load[buf]);
-    sm100::bulk_g2s(u + L.o_vn, a.vnorm + bh * a.rows_cap + r0, b_vn, &mb_load[buf]);
-    sm100::bulk_g2s(u + L.o_bk, a.bk + bh * a.bk_stride, b_bk, &mb_load[buf]);
-  };
-  // worker-only barrier (named barrier 1 over the 256 worker threads)
-  auto wsync = [&]() { sm100::named_sync(1, CW); };
-  auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
-    if (lane == 0 && !sm100::mbar_wait(bar, parity)) abort_s = 1;
-    wsync();
-    return abort_s == 0;
-  };
-  auto sync_tc = [&]() {
-    sm100::fence_before_sync();
-    wsync();
-    sm100::fence_after_sync();
-  };
-  // this warp's tcgen05.st are complete: publish them to the MMA warp
-  auto publish = [&](uint64_t *bar) {
-    sm100::fence_before_sync();
-    __syncwarp();
-    if (lane == 0) sm100::mbar_arrive(bar);
-  };
-
-  int cit = blockIdx.x, cr0 = -1;
-  bool have = tc_next(a, cit, cr0);
-  if (have && tid == 0) issue(0, cit, cr0);
-  int inflight = have ? 0 : -1;   // buffer whose bulk copies were issued, not yet waited
-  // barrier parities: bit b of kph / vph / lph is the parity to wait for next on buffer b
-  uint32_t kph = 0, vph = 0, lph = 0;
-  float o[G], m_run[G], l_run[G];
-  int u = 0;
-  while (have) {
-    int nit = cit, nr0 = cr0 + sub;
-    const bool nhave = tc_next(a, nit, nr0);
-    if (nhave && tid == 0) {
-      sm100::fence_async_smem();
-      issue((u + 1) & 1, nit, nr0);
-    }
-    const int buf = u & 1;
-    if (!wait_all(&mb_load[buf], (lph >> buf) & 1)) break;
-    lph ^= 1u << buf;
-    inflight = nhave ? (u + 1) & 1 : -1;
-    uint8_t *ub = smem + buf * L.ubytes;
-
-    const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
-    const int len = tc_len(a, b);
-    const int c0 = sp * a.chunk, c1 = min(len, c0 + a.chunk);
-    const int nvalid = min(sub, c1 - cr0);
-    if (cr0 == c0) {
+    // ------------------------------------------------------------ rows / coordinates
+    const bool rw = warp < 4;          // expansion + value epilogue; else key epilogue
+    const int wq = warp & 3;
+    float *lg = reinterpret_cast<float *>(smem + L.o_lg);
+    int8_t *bvs = reinterpret_cast<int8_t *>(smem + L.o_bv);
+    int cit = blockIdx.x, cr0 = -1, u = 0;
+    uint32_t kt = 0, ts = 0, vg = 0, sp_par = 0;
+    float o[G], m_run[G], l_run[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        o[h] = 0.f;
-        m_run[h] = -CUDART_INF_F;
-        l_run[h] = 0.f;
-      }
-    }
-    const float *kcst = reinterpret_cast<const float *>(ub + L.o_bk + BKB);
-    const uint32_t bk_addr = sm100::smem_addr(ub + L.o_bk);
-
-    // ---------------- keys: logits of the G heads, 128 rows per tile
-    // expand tile j's bit planes (this slice's terms) into AK[kb]
-    auto expand_keys = [&](int j, int kb) {
-      const int rl = j * 128 + lt;
-      uint32_t pw[PK][TNW];
-      const uint4 *kr = reinterpret_cast<const uint4 *>(ub + rl * PK * 16);
-#pragma unroll
-      for (int p = 0; p < PK; ++p) {
-        const uint4 v = kr[p];
-        pw[p][0] = v.x;
-        pw[p][1] = v.y;
-        pw[p][2] = v.z;
-        pw[p][3] = v.w;
-      }
-      const uint32_t ak = tm + C_AK + kb * 32 * NKT;
-#pragma unroll
-      for (int t = 0; t < NKT; ++t) {
-        if ((t & 1) != slice) continue;
-#pragma unroll
-        for (int w = 0; w < TNW; ++w) {
-          uint32_t x = 0;
-          if (t < TK) {
-            const int mask = odd_mask(MBK, t);
-#pragma unroll
-            for (int p = 0; p < MBK; ++p)
-              if ((mask >> p) & 1) x ^= pw[p][w];
-          } else {
-            x = pw[PK - 1][w];
-          }
-          uint32_t r8[8];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-          sm100::tmem_st8(sm100::tmem_lane(ak + t * 32 + w * 8, wq), r8);
-        }
-      }
-      sm100::wait_st();
-    };
-    float mloc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
-    const int ntile = (nvalid + 127) / 128;
-    bool ok = true;
-    expand_keys(0, 0);
-    publish(&ak_full[0]);
-    for (int j = 0; j < ntile; ++j) {
-      const int kb = j & 1;
-      if (j + 1 < ntile) {
-        // AK[kb ^ 1] and DK[kb ^ 1] were released by tile j - 1 (waited, read)
-        expand_keys(j + 1, kb ^ 1);
-        publish(&ak_full[kb ^ 1]);
-      }
-      ok = wait_all(&mb_k[kb], (kph >> kb) & 1);
-      kph ^= 1u << kb;
-      if (!ok) break;
+    for (int h = 0; h < G; ++h) { o[h] = 0.f; m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; }
+    bool have = tc_next(a, cit, cr0);
+    // all 8 row warps meet (bounded)
+    auto sync8 = [&]() -> bool {
+      sm100::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&sbar);
+      const bool r = dwait(&sbar, sp_par, outer, &abort_s);
+      sp_par ^= 1u;
       sm100::fence_after_sync();
-      if (slice == 0) {
-        const int rl = j * 128 + lt;
-        const bool valid = rl < nvalid;
-        uint32_t dk[2 * N];
-        const uint32_t dka = tm + C_DK + kb * 32;
-        if (N == 16) {
-          uint32_t t0[16], t1[16];
-          sm100::tmem_ld16(sm100::tmem_lane(dka, wq), t0);
-          sm100::tmem_ld16(sm100::tmem_lane(dka + 16, wq), t1);
-          sm100::wait_ld();
+      return r;
+    };
+    while (have) {
+      const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
+      const int len = tc_len(a, b);
+      const int c0 = sp * a.chunk, c1 = min(len, c0 + a.chunk);
+      const int nvalid = min(a.sub, c1 - cr0);
+      const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
+      const float *kcst = reinterpret_cast<const float *>(smem + L.o_bk + (u & 1) * L.bkc + BKB);
+      if (cr0 == c0) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            dk[c] = t0[c];
-            dk[N + c] = t1[c];
+        for (int h = 0; h < G; ++h) { o[h] = 0.f; m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; }
+      }
+      float mloc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
+      bool ok = true;
+      // ---------------- K phase
+      if (rw) {
+        for (int j = 0; j < ntile && ok; ++j, ++kt) {
+          const int s = kt % KS;
+          if (!(ok = dwait(&kf[s], (kt / KS) & 1, outer, &abort_s))) break;
+          const uint4 *kr = reinterpret_cast<const uint4 *>(smem + L.o_kt + s * L.ktb + lt * PK * 16);
+          uint32_t pw[PK][TNW];
+#pragma unroll
+          for (int p = 0; p < PK; ++p) {
+            const uint4 v = kr[p];
+            pw[p][0] = v.x; pw[p][1] = v.y; pw[p][2] = v.z; pw[p][3] = v.w;
           }
-        } else {
-          uint32_t t0[8], t1[8];
-          sm100::tmem_ld8(sm100::tmem_lane(dka, wq), t0);
-          sm100::tmem_ld8(sm100::tmem_lane(dka + N, wq), t1);
-          sm100::wait_ld();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&ke[s]);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            dk[c] = t0[c];
-            dk[N + c] = t1[c];
+          for (int t = 0; t < NKT; ++t, ++ts) {
+            const int slot = ts % NSLOT;
+            if (ts >= NSLOT && !(ok = dwait(&as_empty[slot], ((ts / NSLOT) - 1) & 1, outer, &abort_s))) break;
+            sm100::fence_after_sync();
+#pragma unroll
+            for (int w = 0; w < TNW; ++w) {
+              uint32_t x = 0;
+              if (t < TK) {
+                const int mask = odd_mask(MBK, t);
+#pragma unroll
+                for (int p = 0; p < MBK; ++p)
+                  if ((mask >> p) & 1) x ^= pw[p][w];
+              } else {
+                x = pw[PK - 1][w];
+              }
+              uint32_t r8[8];
+#pragma unroll
+              for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
+              sm100::tmem_st8(sm100::tmem_lane(tm + C_SLOT + slot * 32 + w * 8, wq), r8);
+            }
+            sm100::wait_st();
+            sm100::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&as_full[slot]);
           }
         }
-        const uint32_t sc = reinterpret_cast<const uint32_t *>(ub + L.o_ks)[rl];
-        const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
-        const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+      } else {
+        ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);   // kcst of this unit
+        for (int j = 0; j < ntile && ok; ++j, ++kt) {
+          const int kb = kt & 1, s = kt % KS;
+          if (!(ok = dwait(&dk_full[kb], (kt >> 1) & 1, outer, &abort_s))) break;
+          sm100::fence_after_sync();
+          const uint32_t dka = tm + C_DK + kb * NACC * N;
+          uint32_t dm[N], dq[N];
+#pragma unroll
+          for (int c = 0; c < N; ++c) dm[c] = dq[c] = 0u;
+#pragma unroll
+          for (int ac = 0; ac < NACC; ++ac) {
+            uint32_t tv[N];
+            if (N == 16) {
+              uint32_t t16[16];
+              sm100::tmem_ld16(sm100::tmem_lane(dka + ac * N, wq), t16);
+              sm100::wait_ld();
+#pragma unroll
+              for (int c = 0; c < 16; ++c) tv[c % N] = t16[c];
+            } else {
+              uint32_t t8[8];
+              sm100::tmem_ld8(sm100::tmem_lane(dka + ac * N, wq), t8);
+              sm100::wait_ld();
+#pragma unroll
+              for (int c = 0; c < 8; ++c) tv[c % N] = t8[c];
+            }
+            const bool sign_acc = QJL && ac == NACC - 1;
+#pragma unroll
+            for (int c = 0; c < N; ++c) {
+              if (sign_acc) dq[c] = tv[c];
+              else dm[c] += tv[c];
+            }
+          }
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&dk_empty[kb]);
+          const int rl = j * 128 + lt;
+          const bool valid = rl < nvalid;
+          const uint32_t sc = reinterpret_cast<const uint32_t *>(smem + L.o_kt + s * L.ktb + 128 * PK * 16)[lt];
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&ke[s]);
+          const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+          const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float dmv = comb_limbs(dm + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
+            float est = dmv;
+            if (QJL) {
+              const float dj = comb_limbs(dq + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
+              est = fmaf(a.qjl_coef * rho, dj, dmv);
+            }
+            const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
+            lg[rl * G + h] = l;
+            mloc[h] = fmaxf(mloc[h], l);
+            if (a.logits && valid)
+              a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
+          }
+        }
+      }
+      // ---------------- S phase (8 warps)
+      if (ok) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float dm = comb_limbs(dk + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
-          float est = dm;
-          if (QJL) {
-            const float dj = comb_limbs(dk + N + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
-            est = fmaf(a.qjl_coef * rho, dj, dm);
+          const float m = tq_warp_max(mloc[h]);
+          if (lane == 0) redf[warp][h] = m;
+        }
+        ok = sync8();
+      }
+      float mnew[G], corr[G], lsum[G], FV = 1.f, invFV = 1.f;
+      if (ok) ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);
+      if (ok) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float m = redf[0][h];
+#pragma unroll
+          for (int w = 1; w < 8; ++w) m = fmaxf(m, redf[w][h]);
+          mnew[h] = fmaxf(m_run[h], m);
+          corr[h] = __expf(m_run[h] - mnew[h]);
+          lsum[h] = 0.f;
+        }
+        const uint16_t *vn = reinterpret_cast<const uint16_t *>(smem + L.o_vn + (u & 1) * UMAX * 2);
+        float numax = 0.f;
+        for (int rl = tid; rl < nvalid; rl += 256) {
+          numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float p = __expf(lg[rl * G + h] - mnew[h]);
+            lg[rl * G + h] = p;
+            lsum[h] += p;
           }
-          const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
-          lg[rl * G + h] = l;
-          mloc[h] = fmaxf(mloc[h], l);
-          if (a.logits && valid)
-            a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
+        }
+        ok = sync8();   // redf is free again; the weights are in place
+        if (ok) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float sm = tq_warp_sum(lsum[h]);
+            if (lane == 0) redf[warp][h] = sm;
+          }
+          const float nm = tq_warp_max(numax);
+          if (lane == 0) redf[warp][2 * G] = nm;
+          if (tid < 8) wsum_s[tid] = 0ull;
+          ok = sync8();
+        }
+        if (ok) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float sm = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) sm += redf[w][h];
+            lsum[h] = sm;
+          }
+          float nmax = redf[0][2 * G];
+#pragma unroll
+          for (int w = 1; w < 8; ++w) nmax = fmaxf(nmax, redf[w][2 * G]);
+          FV = pow2_scale(nmax);
+          invFV = 1.0f / (128.0f * FV);
+          // value-side B operand: element (n = 4h + l, k) of group g holds limb
+          // l of W(token) * 2^(7-r) for token 32g + 8nb + r, k = 4r + nb; one
+          // item = (group, r, head) makes the four consecutive k of one limb
+          // row and stores them as one 32-bit word; rows n >= 4G are zero
+          constexpr int NH = N / 4;
+          long long wpart = 0;
+          const int h = tid % NH;
+          for (int it = tid; it < ngroups * 8 * NH; it += 256) {
+            const int r = (it / NH) & 7, g = it / (8 * NH);
+            uint32_t word[4] = {0u, 0u, 0u, 0u};
+            if (h < G) {
+#pragma unroll
+              for (int nb = 0; nb < 4; ++nb) {
+                const int rl = 32 * g + 8 * nb + r;
+                int W = 0;
+                if (rl < nvalid) W = __float2int_rn(lg[rl * G + h] * tq_half_to_f32(vn[rl]) * FV);
+                wpart += W;
+                int v = W * (1 << (7 - r));
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                  const int8_t dgt = static_cast<int8_t>(v & 0xff);
+                  word[l] |= static_cast<uint32_t>(static_cast<uint8_t>(dgt)) << (8 * nb);
+                  v = (v - dgt) >> 8;
+                }
+              }
+            }
+            int8_t *dst = bvs + g * N * 32;
+#pragma unroll
+            for (int l = 0; l < 4; ++l)
+              *reinterpret_cast<uint32_t *>(dst + kmajor_off(4 * h + l, 4 * r, N)) = word[l];
+          }
+          if (h < G) atomicAdd(&wsum_s[h], static_cast<unsigned long long>(wpart));
+          sm100::fence_async_smem();
+          ok = sync8();
+          if (ok && lane == 0) {
+            sm100::mbar_arrive(&bv_full);
+            sm100::mbar_arrive(&hdr_free[u & 1]);   // B operand and value norms no longer read
+          }
         }
       }
-    }
-    if (!ok) break;
-
-    // ---------------- softmax statistics of the unit
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float m = tq_warp_max(mloc[h]);
-      if (lane == 0) redf[warp][h] = m;
-    }
-    sync_tc();   // the key epilogue's TMEM reads are complete before any value-phase store
-    float mnew[G], corr[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float m = redf[0][h];
-#pragma unroll
-      for (int w = 1; w < NWW; ++w) m = fmaxf(m, redf[w][h]);
-      mnew[h] = fmaxf(m_run[h], m);
-      corr[h] = __expf(m_run[h] - mnew[h]);
-    }
-    const uint16_t *vn = reinterpret_cast<const uint16_t *>(ub + L.o_vn);
-    float lsum[G], numax = 0.f;
-#pragma unroll
-    for (int h = 0; h < G; ++h) lsum[h] = 0.f;
-    for (int rl = tid; rl < nvalid; rl += CW) {
-      numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
+      if (!ok) break;
+      float wtot[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float p = __expf(lg[rl * G + h] - mnew[h]);
-        lg[rl * G + h] = p;
-        lsum[h] += p;
+        wtot[h] = static_cast<float>(static_cast<long long>(wsum_s[h])) / FV;
+        o[h] *= corr[h];
+        l_run[h] = l_run[h] * corr[h] + lsum[h];
+        m_run[h] = mnew[h];
       }
-    }
-    wsync();
+      // ---------------- V and E phases (warps 0-3, lane = coordinate)
+      if (rw) {
+        for (int g = 0; g < ngroups && ok; ++g, ++vg) {
+          const int s = vg % VS, ab = vg & 1;
+          if (!(ok = dwait(&vf[s], (vg / VS) & 1, outer, &abort_s))) break;
+          const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
+          uint32_t pw[BV];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float s = tq_warp_sum(lsum[h]);
-      if (lane == 0) redf[warp][h] = s;
-    }
-    {
-      const float m = tq_warp_max(numax);
-      if (lane == 0) redf[warp][2 * G] = m;
-    }
-    wsync();
+          for (int p = 0; p < BV; ++p) pw[p] = vc[p * TD + lt];
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&ve[s]);
+          if (vg >= 2 && !(ok = dwait(&av_empty[ab], ((vg >> 1) - 1) & 1, outer, &abort_s))) break;
+          sm100::fence_after_sync();
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float s = 0.f;
+          for (int ti = 0; ti < TV; ++ti) {
+            const int mask = odd_mask(BV, ti);
+            uint32_t x = 0;
 #pragma unroll
-      for (int w = 0; w < NWW; ++w) s += redf[w][h];
-      lsum[h] = s;
-    }
-    float nmax = redf[0][2 * G];
+            for (int p = 0; p < BV; ++p)
+              if ((mask >> p) & 1) x ^= pw[p];
+            uint32_t r8[8];
 #pragma unroll
-    for (int w = 1; w < NWW; ++w) nmax = fmaxf(nmax, redf[w][2 * G]);
-    const float FV = pow2_scale(nmax);
-    const float invFV = 1.0f / (128.0f * FV);
-
-    // ---------------- value-side B operand: 24-bit weights p * nu_v, limbs
-    const int ngroups = (nvalid + 31) / 32;
-    long long wsum[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) wsum[h] = 0;
-    for (int rl = tid; rl < ngroups * 32; rl += CW) {
-      const int g = rl >> 5, jj = rl & 31, r = jj & 7, nb = jj >> 3;
-      const int k = 4 * r + nb;
-      int8_t *dst = bvs + g * N * 32;
-      const float nv = rl < nvalid ? tq_half_to_f32(vn[rl]) : 0.f;
-#pragma unroll
-      for (int h = 0; h < N / 4; ++h) {
-        int W = 0;
-        if (h < G && rl < nvalid) W = __float2int_rn(lg[rl * G + h] * nv * FV);
-        if (h < G) wsum[h] += W;
-        const int v = W * (1 << (7 - r));
-#pragma unroll
-        for (int l = 0; l < 4; ++l) dst[kmajor_off(4 * h + l, k, N)] = limb_of(v, l);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      long long s = wsum[h];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(TQ_FULL, s, off);
-      if (lane == 0) redi[warp][h] = s;
-    }
-    sm100::fence_async_smem();
-    wsync();
-    float wtot[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      long long s = 0;
-#pragma unroll
-      for (int w = 0; w < NWW; ++w) s += redi[w][h];
-      wtot[h] = static_cast<float>(s) / FV;
-      o[h] *= corr[h];
-      l_run[h] = l_run[h] * corr[h] + lsum[h];
-      m_run[h] = mnew[h];
-    }
-
-    // ---------------- values: rotated-domain sums, 32 tokens per MMA step
-    const uint32_t *vc = reinterpret_cast<const uint32_t *>(ub + L.o_vc);
-    for (int g = 0; g < ngroups && ok; ++g) {
-      const int ab = g & 1;
-      if (g >= 2) {  // buffer ab was last fed to the MMAs of group g - 2
-        ok = wait_all(&mb_v[ab], (vph >> ab) & 1);
-        vph ^= 1u << ab;
-        if (!ok) break;
-      }
-      uint32_t pw[BV];
-#pragma unroll
-      for (int p = 0; p < BV; ++p) pw[p] = vc[(g * BV + p) * TD + lt];
-#pragma unroll
-      for (int ti = 0; ti < TV; ++ti) {
-        if ((ti & 1) != slice) continue;
-        const int mask = odd_mask(BV, ti);
-        uint32_t x = 0;
-#pragma unroll
-        for (int p = 0; p < BV; ++p)
-          if ((mask >> p) & 1) x ^= pw[p];
-        uint32_t r8[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-        sm100::tmem_st8(sm100::tmem_lane(tm + C_AV + ab * TV * 8 + ti * 8, wq), r8);
-      }
-      sm100::wait_st();
-      publish(&av_full[ab]);
-    }
-    // the last one or two groups' MMAs are still outstanding
-    for (int g = ngroups > 2 ? ngroups - 2 : 0; g < ngroups && ok; ++g) {
-      const int ab = g & 1;
-      ok = wait_all(&mb_v[ab], (vph >> ab) & 1);
-      vph ^= 1u << ab;
-    }
-    if (!ok) break;
-    sm100::fence_after_sync();
-    // each slice folds its Walsh terms for coordinate lt; slice 1 hands its
-    // partial sums to slice 0, which keeps the running output
-    {
-      float acc[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll
-      for (int ti = 0; ti < TV; ++ti) {
-        if ((ti & 1) != slice) continue;
-        uint32_t dv[N];
-        if (N == 16) {
-          uint32_t t0[16];
-          sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-          sm100::wait_ld();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) dv[c] = t0[c];
-        } else {
-          uint32_t t0[8];
-          sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-          sm100::wait_ld();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) dv[c] = t0[c];
+            for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
+            sm100::tmem_st8(sm100::tmem_lane(tm + C_AV + ab * TV * 8 + ti * 8, wq), r8);
+          }
+          sm100::wait_st();
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&av_full[ab]);
         }
+        if (ok) ok = dwait(&dv_full, u & 1, outer, &abort_s);
+        if (ok) {
+          sm100::fence_after_sync();
+          float acc[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
-      }
-      if (slice == 1) {
+          for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) part[h][lt] = acc[h];
-      }
-      wsync();
-      if (slice == 0) {
+          for (int ti = 0; ti < TV; ++ti) {
+            uint32_t dv[N];
+            if (N == 16) {
+              uint32_t t0[16];
+              sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
+              sm100::wait_ld();
 #pragma unroll
-        for (int h = 0; h < G; ++h) o[h] += (acc[h] + part[h][lt]) * invFV - a.wv_sum * wtot[h];
-      }
-    }
-    if (cr0 + sub >= c1 && slice == 0) {
+              for (int c = 0; c < 16; ++c) dv[c % N] = t0[c];
+            } else {
+              uint32_t t0[8];
+              sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
+              sm100::wait_ld();
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-        a.po[(hq * a.splits + sp) * TD + lt] = o[h];
-        if (tid == 0) {
-          a.pml[(hq * a.splits + sp) * 2] = m_run[h];
-          a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
+              for (int c = 0; c < 8; ++c) dv[c % N] = t0[c];
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
+          }
+          sm100::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&tm_free);
+#pragma unroll
+          for (int h = 0; h < G; ++h) o[h] += acc[h] * invFV - a.wv_sum * wtot[h];
+          if (cr0 + a.sub >= c1) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
+              a.po[(hq * a.splits + sp) * TD + lt] = o[h];
+              if (tid == 0) {
+                a.pml[(hq * a.splits + sp) * 2] = m_run[h];
+                a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
+              }
+            }
+          }
         }
       }
+      if (!ok) break;
+      cr0 += a.sub;
+      have = tc_next(a, cit, cr0);
+      ++u;
     }
-    sync_tc();
-    cit = nit;
-    cr0 = nr0;
-    have = nhave;
-    ++u;
   }
-  if (abort_s) {
-    // a bounded wait gave up: let this CTA's own outstanding copies and MMAs
-    // land (again bounded) before its shared and tensor memory are released
-    if (inflight >= 0) sm100::mbar_wait(&mb_load[inflight], (lph >> inflight) & 1, 1u << 20);
-    sm100::mbar_wait(&mb_k[0], kph & 1, 1u << 20);
-    sm100::mbar_wait(&mb_k[1], (kph >> 1) & 1, 1u << 20);
-    sm100::mbar_wait(&mb_v[0], vph & 1, 1u << 20);
-    sm100::mbar_wait(&mb_v[1], (vph >> 1) & 1, 1u << 20);
-    if (tid == 0 && a.err) atomicExch(a.err, 1u);
-  }
-  }  // workers
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  if (warp == 0) sm100::tmem_dealloc(tm, NCOLS);
+  if (abort_s && tid == 0 && a.err) atomicExch(a.err, 1u);
+  if (warp == 0) sm100::tmem_dealloc(tm, DCOLS);
 }
 
 // ---------------------------------------------------------------------------
@@ -842,10 +890,11 @@ struct TcCfg {
 
 constexpr TcCfg kTcConfigs[] = {{4, 3, 4, 1}, {4, 1, 2, 1}, {4, 2, 3, 1}, {2, 3, 4, 1},
                                 {2, 1, 2, 1}, {2, 2, 3, 1}, {1, 3, 4, 1}, {1, 1, 2, 1},
-                                {1, 2, 3, 1}};
+                                {1, 2, 3, 1}, {4, 4, 4, 0}, {4, 2, 2, 0}, {4, 3, 3, 0},
+                                {1, 3, 3, 0}};
 
 template <int G, int MBK, int BV, bool QJL>
-int run_tc(TcArgs &a, cudaStream_t stream) {
+int run_dec(TcArgs &a, cudaStream_t stream) {
   constexpr int TK = 1 << (MBK - 1);
   constexpr int N = tc_n(G);
   constexpr int PK = MBK + (QJL ? 1 : 0);
@@ -853,35 +902,19 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // CTAs per SM: one by default (largest sub-chunks); TQ_TC_CTAS_PER_SM asks
-  // for more, capped by tensor-memory slots, after which the sub-chunk shrinks
-  // until that many fit in shared memory (each unit is double-buffered)
-  constexpr int NCOLS = tc_tmem_alloc(G, MBK, BV, QJL);
-  int per_sm = 1;
-  if (const char *e = getenv("TQ_TC_CTAS_PER_SM")) per_sm = atoi(e);
-  if (per_sm > 512 / NCOLS) per_sm = 512 / NCOLS;
-  if (per_sm > 4) per_sm = 4;
-  if (per_sm < 1) per_sm = 1;
-  const int budget = per_sm == 1 ? 200 * 1024 : (227 * 1024) / per_sm - 2048;
-  int sub = a.chunk;
-  while (sub > 128 && tc_layout(sub, PK, BV, G, N, BKC).total > budget) sub -= 128;
-  a.sub = sub;
-  const int smem = tc_layout(sub, PK, BV, G, N, BKC).total;
+  a.sub = a.chunk < UMAX ? a.chunk : UMAX;
+  const int smem = dec_layout(PK, BV, G, N, BKC).total;
   static bool attr_done[64] = {};
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(tc_chunk_kernel<G, MBK, BV, QJL>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, 210 * 1024) != cudaSuccess)
-      return tq_check_launch("cudaFuncSetAttribute(tc_chunk)");
+    if (cudaFuncSetAttribute(dec_kernel<G, MBK, BV, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return tq_check_launch("cudaFuncSetAttribute(dec_kernel)");
     attr_done[dev] = true;
   }
-  int occ = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tc_chunk_kernel<G, MBK, BV, QJL>, CT, smem);
-  if (occ < 1) occ = 1;
-  if (occ < per_sm) per_sm = occ;
   tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, 0, stream>>>(a);
   if (int e = tq_check_launch("tc_prep_kernel")) return e;
   const int items = a.B * a.Hkv * a.splits;
-  const int grid = items < sms * per_sm ? items : sms * per_sm;
+  const int grid = items < 2 * sms ? items : 2 * sms;
   cudaEvent_t ev0, ev1;
   tq_timing_events(&ev0, &ev1);
   unsigned ev_flags = cudaEventRecordDefault;
@@ -891,8 +924,8 @@ int run_tc(TcArgs &a, cudaStream_t stream) {
     if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
     cudaEventRecordWithFlags(ev0, stream, ev_flags);
   }
-  tc_chunk_kernel<G, MBK, BV, QJL><<<grid, CT, smem, stream>>>(a);
-  if (int e = tq_check_launch("tc_chunk_kernel")) return e;
+  dec_kernel<G, MBK, BV, QJL><<<grid, DT, smem, stream>>>(a);
+  if (int e = tq_check_launch("dec_kernel")) return e;
   if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
   tq_count_launch(2);
   return TQ_OK;
@@ -916,7 +949,7 @@ int tc_bk_stride(const tq_codec *c, int G) {
 int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                      const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
                      const float *rc, const float *rs, int splits, float *po, float *pml,
-                     uint8_t *bk, float *logits, cudaStream_t stream) {
+                     uint8_t *bk, float *logits, uint32_t *err, cudaStream_t stream) {
   TcArgs a;
   a.q = q;
   a.dtype = dtype;
@@ -952,19 +985,25 @@ int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq,
   }
   a.wk_absmax = c->walsh_k_absmax;
   a.wv_sum = c->walsh_v_sum;
-  a.err = nullptr;
+  a.err = err;
+  a.wait_limit = 1u << 26;
+  if (const char *e = getenv("TQ_WAIT_LIMIT")) a.wait_limit = static_cast<uint32_t>(strtoul(e, nullptr, 10));
   a.books = c->books;
   const int key = G * 1000 + c->mse_bits_k * 100 + c->bits_v * 10 + c->qjl_k;
   switch (key) {
-    case 4341: return run_tc<4, 3, 4, true>(a, stream);
-    case 4121: return run_tc<4, 1, 2, true>(a, stream);
-    case 4231: return run_tc<4, 2, 3, true>(a, stream);
-    case 2341: return run_tc<2, 3, 4, true>(a, stream);
-    case 2121: return run_tc<2, 1, 2, true>(a, stream);
-    case 2231: return run_tc<2, 2, 3, true>(a, stream);
-    case 1341: return run_tc<1, 3, 4, true>(a, stream);
-    case 1121: return run_tc<1, 1, 2, true>(a, stream);
-    case 1231: return run_tc<1, 2, 3, true>(a, stream);
+    case 4341: return run_dec<4, 3, 4, true>(a, stream);
+    case 4121: return run_dec<4, 1, 2, true>(a, stream);
+    case 4231: return run_dec<4, 2, 3, true>(a, stream);
+    case 2341: return run_dec<2, 3, 4, true>(a, stream);
+    case 2121: return run_dec<2, 1, 2, true>(a, stream);
+    case 2231: return run_dec<2, 2, 3, true>(a, stream);
+    case 1341: return run_dec<1, 3, 4, true>(a, stream);
+    case 1121: return run_dec<1, 1, 2, true>(a, stream);
+    case 1231: return run_dec<1, 2, 3, true>(a, stream);
+    case 4440: return run_dec<4, 4, 4, false>(a, stream);
+    case 4220: return run_dec<4, 2, 2, false>(a, stream);
+    case 4330: return run_dec<4, 3, 3, false>(a, stream);
+    case 1330: return run_dec<1, 3, 3, false>(a, stream);
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "tensor-core decode: configuration not built");
   }
 }

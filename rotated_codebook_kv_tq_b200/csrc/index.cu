@@ -828,6 +828,115 @@ __global__ void ix_merge_kernel(const float *cs, const int32_t *ci, int nq, int 
   }
 }
 
+// ---------------------------------------------------------------------------
+// LUT-path scan (the comparison path to the tensor-core scan): per query a
+// table T[i][m] = q'_i c_m over every coordinate i and code m, and the QJL
+// column coef * q''_i, in shared memory; a warp scores one database row at a
+// time, lane l taking coordinates 32 w + l, with one table lookup and one
+// signed add per coordinate in fp32 (no fp16 rounding of the products).
+// Every warp keeps its own top-k; the block merges its 8 lists into one
+// candidate list per (query, row block), merged across blocks by
+// ix_merge_kernel.
+// ---------------------------------------------------------------------------
+constexpr int LT = 256;        // threads (8 warps) of ix_lut_kernel
+constexpr int LSTR = 9;        // padded table row: 8 codes + 1 (bank spread)
+constexpr uint32_t LUT_SMEM = XD * (LSTR + 1) * 4;
+
+struct LutArgs {
+  const uint8_t *kcode;   // [n][planes][XD / 8]
+  const uint16_t *kscale; // [n][2]
+  int64_t n;
+  const float *q1;        // [nq][XD]  q' = Pi q
+  const float *q2;        // [nq][XD]  q'' = S q'
+  int nq;
+  float coef;             // sqrt(pi/2) / XD
+  int mbk;
+  float ck[8];            // key centroids
+  int64_t rows_per_block;
+  float *cand_s;          // [nq][lists][k]
+  int32_t *cand_i;
+  int k;
+  int lists;
+};
+
+// Insert (v, j) into a descending list of k (ties to the lower index).
+__device__ __forceinline__ void topk_insert(float *bs, int *bi, int k, float v, int j) {
+  const bool better = v > bs[k - 1] || (v == bs[k - 1] && j < bi[k - 1]);
+  if (!better) return;
+  int e = k - 1;
+  while (e > 0 && (v > bs[e - 1] || (v == bs[e - 1] && j < bi[e - 1]))) {
+    bs[e] = bs[e - 1];
+    bi[e] = bi[e - 1];
+    --e;
+  }
+  bs[e] = v;
+  bi[e] = j;
+}
+
+__global__ void __launch_bounds__(LT) ix_lut_kernel(LutArgs a) {
+  extern __shared__ float lut_smem[];
+  float *tq = lut_smem;                  // [XD][LSTR]
+  float *sq = lut_smem + XD * LSTR;      // [XD]
+  __shared__ float ws[LT / 32][SKMAX];
+  __shared__ int wi[LT / 32][SKMAX];
+  const int q = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < XD; i += LT) {
+    const float v = a.q1[static_cast<int64_t>(q) * XD + i];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tq[i * LSTR + m] = v * a.ck[m];
+    sq[i] = a.coef * a.q2[static_cast<int64_t>(q) * XD + i];
+  }
+  __syncthreads();
+  float bs[SKMAX];
+  int bi[SKMAX];
+  for (int e = 0; e < SKMAX; ++e) {
+    bs[e] = -CUDART_INF_F;
+    bi[e] = 0x7fffffff;
+  }
+  const int planes = a.mbk + 1;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.y) * a.rows_per_block;
+  const int64_t r_end = min(a.n, r_begin + a.rows_per_block);
+  for (int64_t row = r_begin + warp; row < r_end; row += LT / 32) {
+    const uint32_t *kr = reinterpret_cast<const uint32_t *>(a.kcode + row * planes * (XD / 8));
+    float acc = 0.f, sacc = 0.f;
+    for (int w = 0; w < XW; ++w) {
+      const uint32_t w0 = kr[w];
+      const uint32_t w1 = a.mbk > 1 ? kr[XW + w] : 0u;
+      const uint32_t w2 = a.mbk > 2 ? kr[2 * XW + w] : 0u;
+      const uint32_t wsg = kr[a.mbk * XW + w];
+      const int idx = static_cast<int>(((w0 >> lane) & 1u) | (((w1 >> lane) & 1u) << 1) |
+                                       (((w2 >> lane) & 1u) << 2));
+      const int i = 32 * w + lane;
+      acc += tq[i * LSTR + idx];
+      const float sv = sq[i];
+      sacc += ((wsg >> lane) & 1u) ? sv : -sv;
+    }
+    acc = tq_warp_sum(acc);
+    sacc = tq_warp_sum(sacc);
+    const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale)[row];
+    const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+    const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+    const float score = nu * fmaf(rho, sacc, acc);
+    if (lane == 0) topk_insert(bs, bi, a.k, score, static_cast<int>(row));
+  }
+  if (lane == 0)
+    for (int e = 0; e < a.k; ++e) {
+      ws[warp][e] = bs[e];
+      wi[warp][e] = bi[e];
+    }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < LT / 32; ++w)
+      for (int e = 0; e < a.k; ++e) topk_insert(bs, bi, a.k, ws[w][e], wi[w][e]);
+    const int64_t base = (static_cast<int64_t>(q) * a.lists + blockIdx.y) * a.k;
+    for (int e = 0; e < a.k; ++e) {
+      a.cand_s[base + e] = bs[e];
+      a.cand_i[base + e] = bi[e];
+    }
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -878,6 +987,38 @@ int scan_grid_y(int64_t n, int nq) {
   int64_t gy = sm_count() / qblocks;   // one wave: grid.x * grid.y <= SMs (one CTA per SM)
   if (gy > tiles) gy = tiles;
   return static_cast<int>(gy < 1 ? 1 : gy);
+}
+
+// Row blocks of the LUT scan: about two CTAs per SM in all, whole queries per CTA.
+int lut_blocks(int64_t n, int nq) {
+  int64_t b = (2LL * sm_count() + nq - 1) / nq;
+  const int64_t max_b = (n + 255) / 256;
+  if (b > max_b) b = max_b;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+// q' = Pi q and q'' = S q' into the scan workspace (both scan paths).
+int scan_query_prologue(const tq_codec *c, const float *q, int nq, float *q1, uint16_t *q1hl,
+                        float *q2, cudaStream_t st) {
+  QrotArgs qa;
+  qa.q = q;
+  qa.nq = nq;
+  qa.q1 = q1;
+  qa.q1hl = q1hl;
+  for (int i = 0; i < XW; ++i) qa.dneg[i] = c->books.dneg[i];
+  ix_qrot_kernel<<<(nq + 7) / 8, 256, 0, st>>>(qa);
+  tq_count_launch(1);
+  if (int e = tq_check_launch("ix_qrot_kernel")) return e;
+  GemmArgs g;
+  g.A = q1hl;
+  g.B = c->S_dev;
+  g.M = nq;
+  g.N = XD;
+  g.KA = 2 * XD;
+  g.KB = XD;
+  g.out = q2;
+  g.status = nullptr;
+  return run_gemm(g, st);
 }
 
 }  // namespace
@@ -983,7 +1124,9 @@ ScanWs scan_ws(int nq, int k, int gy) {
 int tq_scan_workspace(const tq_codec *c, int64_t n, int nq, int k, size_t *bytes) {
   if (!c || !bytes || n < 1 || nq < 1 || k < 1 || k > SKMAX)
     return tq_fail(TQ_ERR_INVALID_ARG, "scan workspace: bad arguments (1 <= k <= 16)");
-  *bytes = scan_ws(nq, k, scan_grid_y(n, nq)).total;
+  const int gy = scan_grid_y(n, nq), lb = lut_blocks(n, nq);
+  // covers both scan paths: 2 gy candidate lists (tensor cores) or lb (LUT)
+  *bytes = scan_ws(nq, k, gy > (lb + 1) / 2 ? gy : (lb + 1) / 2).total;
   return TQ_OK;
 }
 
@@ -1012,27 +1155,8 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   float *qinv = reinterpret_cast<float *>(w + W.qinv);
   float *cand_s = reinterpret_cast<float *>(w + W.cand_s);
   int32_t *cand_i = reinterpret_cast<int32_t *>(w + W.cand_i);
-  // q' = Pi q (fp32 and bf16 hi | lo)
-  QrotArgs qa;
-  qa.q = q;
-  qa.nq = nq;
-  qa.q1 = q1;
-  qa.q1hl = q1hl;
-  for (int i = 0; i < XW; ++i) qa.dneg[i] = c->books.dneg[i];
-  ix_qrot_kernel<<<(nq + 7) / 8, 256, 0, st>>>(qa);
-  tq_count_launch(1);
-  if (int e = tq_check_launch("ix_qrot_kernel")) return e;
-  // q'' = S q' (fp32) on the tensor cores
-  GemmArgs g;
-  g.A = q1hl;
-  g.B = c->S_dev;
-  g.M = nq;
-  g.N = XD;
-  g.KA = 2 * XD;
-  g.KB = XD;
-  g.out = q2;
-  g.status = nullptr;
-  if (int e = run_gemm(g, st)) return e;
+  // q' = Pi q (fp32 and bf16 hi | lo), q'' = S q' (fp32) on the tensor cores
+  if (int e = scan_query_prologue(c, q, nq, q1, q1hl, q2, st)) return e;
   // fp16 B operand with a power-of-two scale per query
   const float coef = sqrtf(static_cast<float>(M_PI) / 2.0f) / XD;
   QpackArgs pa;
@@ -1086,6 +1210,66 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   if (int e = tq_check_launch("ix_scan2_kernel")) return e;
   if (ev1) cudaEventRecord(ev1, st);
   ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(cand_s, cand_i, nq, 2 * gy, k, idx, score);
+  tq_count_launch(2);
+  return tq_check_launch("ix_merge_kernel");
+}
+
+int tq_scan_topk_lut(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale, int64_t n,
+                     const float *q, int nq, int k, int32_t *idx, float *score, void *workspace,
+                     size_t ws_bytes, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "scan (LUT): NULL codec");
+  if (!index_codec_ok(c))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "scan (LUT): needs a d = 1536 codec with QJL keys and 1..3 MSE bits");
+  if (!kcode || !kscale || !q || !idx || !score || !workspace || n < 1 || nq < 1 || k < 1 ||
+      k > SKMAX || k > n)
+    return tq_fail(TQ_ERR_INVALID_ARG, "scan (LUT): NULL buffer or bad n / nq / k (1 <= k <= min(16, n))");
+  if (n > 0x7fffffffLL) return tq_fail(TQ_ERR_INVALID_ARG, "scan (LUT): n must fit in int32 indices");
+  size_t need = 0;
+  tq_scan_workspace(c, n, nq, k, &need);
+  if (ws_bytes < need) return tq_fail(TQ_ERR_WORKSPACE, "scan (LUT): workspace too small");
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(workspace)) % 16 ||
+      reinterpret_cast<uintptr_t>(kcode) % 4 || reinterpret_cast<uintptr_t>(kscale) % 4)
+    return tq_fail(TQ_ERR_ALIGNMENT, "scan (LUT): q/workspace need 16-byte, kcode/kscale 4-byte alignment");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int lb = lut_blocks(n, nq);
+  const int gy = scan_grid_y(n, nq);
+  const ScanWs W = scan_ws(nq, k, gy > (lb + 1) / 2 ? gy : (lb + 1) / 2);
+  uint8_t *w = static_cast<uint8_t *>(workspace);
+  float *q1 = reinterpret_cast<float *>(w + W.q1);
+  uint16_t *q1hl = reinterpret_cast<uint16_t *>(w + W.q1hl);
+  float *q2 = reinterpret_cast<float *>(w + W.q2);
+  if (int e = scan_query_prologue(c, q, nq, q1, q1hl, q2, st)) return e;
+  LutArgs la;
+  la.kcode = kcode;
+  la.kscale = kscale;
+  la.n = n;
+  la.q1 = q1;
+  la.q2 = q2;
+  la.nq = nq;
+  la.coef = sqrtf(static_cast<float>(M_PI) / 2.0f) / XD;
+  la.mbk = c->mse_bits_k;
+  for (int m = 0; m < 8; ++m) la.ck[m] = m < (1 << c->mse_bits_k) ? c->books.ck[m] : 0.f;
+  la.rows_per_block = (n + lb - 1) / lb;
+  la.cand_s = reinterpret_cast<float *>(w + W.cand_s);
+  la.cand_i = reinterpret_cast<int32_t *>(w + W.cand_i);
+  la.k = k;
+  la.lists = lb;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !done[dev]) {
+    if (cudaFuncSetAttribute(ix_lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(LUT_SMEM)) != cudaSuccess)
+      return tq_check_launch("cudaFuncSetAttribute(ix_lut)");
+    done[dev] = true;
+  }
+  cudaEvent_t ev0, ev1;
+  tq_timing_events(&ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, st);
+  ix_lut_kernel<<<dim3(nq, lb), LT, LUT_SMEM, st>>>(la);
+  if (int e = tq_check_launch("ix_lut_kernel")) return e;
+  if (ev1) cudaEventRecord(ev1, st);
+  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(la.cand_s, la.cand_i, nq, lb, k, idx, score);
   tq_count_launch(2);
   return tq_check_launch("ix_merge_kernel");
 }

@@ -14,7 +14,8 @@
 // code its name is only a host-side stand-in, so its device address is looked
 // up once per device with cudaGetSymbolAddress (with that device current) and
 // cached.  Every call shares the array and leaves the previous call's contents
-// in it; the decode kernels write every scratch word before reading it, so no
+// in it; each call writes every scratch word it reads (the partials of each
+// chunk, and the status word, which the query prologue clears), so no
 // clearing is needed.  Calls whose kernels overlap on the GPU (different
 // streams, or several host threads) race on the array and must be serialised
 // by the caller.
@@ -63,7 +64,8 @@ extern "C" int tq_attention_decode_noalloc(const tq_codec *c, const void *q, int
   const size_t need = decode_workspace_bytes(c, B, Hq, splits);
   if (need > static_cast<size_t>(TQ_NOALLOC_SCRATCH_BYTES))
     return tq_fail(TQ_ERR_WORKSPACE,
-                   "no-alloc decode: B*Hq*(2d + splits*(d+2))*4 bytes exceed the 16 MiB static scratch");
+                   "no-alloc decode: the scratch this shape needs (tq_attention_workspace for the same "
+                   "codec, B, Hq and num_splits) exceeds the 16 MiB static array");
   void *ws = nullptr;
   if (int e = scratch_for_current_device(&ws)) return e;
   return tq_attention_decode(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale,

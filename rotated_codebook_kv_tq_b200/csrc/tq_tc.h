@@ -37,7 +37,8 @@ struct TcArgs {
   float wk_absmax;
   float wv[8];          // value Walsh coefficients
   float wv_sum;
-  uint32_t *err;        // optional device flag set when a bounded wait times out
+  uint32_t *err;        // optional device flag set when a bounded wait gives up
+  uint32_t wait_limit;  // polls before a wait gives up (TQ_WAIT_LIMIT overrides, for tests)
   TqBooks books;
 };
 
@@ -48,4 +49,4 @@ int tc_bk_stride(const tq_codec *c, int G);
 int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                      const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
                      const float *rc, const float *rs, int splits, float *po, float *pml,
-                     uint8_t *bk, float *logits, cudaStream_t stream);
+                     uint8_t *bk, float *logits, uint32_t *err, cudaStream_t stream);

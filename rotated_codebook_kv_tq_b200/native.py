@@ -25,7 +25,7 @@ EXPORTS = [
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
     "tq_attention_logits", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
-    "tq_scan_topk", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
+    "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
     "tq_last_error",
 ]
 
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
         L.tq_index_build.argtypes = [vp, vp, i64, vp, vp, vp, vp, sz, vp]
         L.tq_scan_workspace.argtypes = [vp, i64, i32, i32, ctypes.POINTER(sz)]
         L.tq_scan_topk.argtypes = [vp, vp, vp, i64, vp, i32, i32, vp, vp, vp, sz, vp]
+        L.tq_scan_topk_lut.argtypes = [vp, vp, vp, i64, vp, i32, i32, vp, vp, vp, sz, vp]
         L.tq_dequantize.argtypes = [vp, ctypes.POINTER(CacheDesc), i32, i64, i64, vp, vp]
         L.tq_set_timing_events.argtypes = [vp, vp]
         L.tq_launch_count.argtypes = []
@@ -300,6 +301,17 @@ def scan_topk(codec: Codec, kcode, kscale, q, k: int, idx, score, workspace,
                              q.data_ptr(), nq, k, idx.data_ptr(), score.data_ptr(),
                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                              _stream(stream)))
+
+
+def scan_topk_lut(codec: Codec, kcode, kscale, q, k: int, idx, score, workspace,
+                  stream=None) -> None:
+    """tq_scan_topk_lut: the lookup-table scan (fp32 scores), same arguments as scan_topk."""
+    n = kcode.shape[0]
+    nq = q.shape[0]
+    check(lib().tq_scan_topk_lut(codec.handle, kcode.data_ptr(), kscale.data_ptr(), ctypes.c_int64(n),
+                                 q.data_ptr(), nq, k, idx.data_ptr(), score.data_ptr(),
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

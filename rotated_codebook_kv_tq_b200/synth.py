@@ -115,7 +115,7 @@ class Workload:
     sigma_scale: Optional[float]   # lognormal sigma of channel scales (None: unit)
     n_outliers: int
     outlier_gain: float
-    num_splits: int
+    num_splits: int      # split-K chunks per (batch, KV head); 0 = the library's default
     Lq: int = 1          # queries per head (1 = decode, T = bidirectional)
 
     @property
@@ -129,7 +129,7 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", 0, 1, 1, 1, 128, 1024, 3, True, 3, "fp32", None, None, 0, 1.0, 8),
     "llama_decode": Workload("llama_decode", 1, 1, 32, 8, 128, 32768, 4, True, 4, "bf16",
-                             500000.0, 1.0, 4, 20.0, 64),
+                             500000.0, 1.0, 4, 20.0, 0),
     "esm_prefill": Workload("esm_prefill", 2, 16, 20, 20, 64, 1024, 3, True, 3, "bf16",
                             10000.0, 1.0, 4, 20.0, 8, Lq=1024),
     "long_decode": Workload("long_decode", 3, 4, 32, 8, 128, 131072, 2, True, 2, "bf16",

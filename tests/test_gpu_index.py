@@ -4,11 +4,13 @@ bits) through the C ABI, against the oracle.
 Encode parity: codes and signs bit-exact up to the boundary windows of the KV
 tests (coordinates within 1e-5 of a threshold on the unit-variance scale, signs
 with |S r|_i / rho < 1e-5), norms within one fp16 ulp.  Scan parity on an
-oracle-encoded database: every returned score within 1e-3 of the query's
-largest |score| (relative error of the estimated inner product), the returned
-list ordered by (score descending, index ascending), and the returned set equal
-to the oracle's top-k up to rows whose oracle scores lie within twice that
-tolerance of the k-th best.
+oracle-encoded database, for both the tensor-core scan and the lookup-table
+scan: every returned score within a tolerance of the oracle's score of that
+row (relative to the RMS of the query's oracle scores; see LUT_SCORE_TOL and
+MMA_SCORE_TOL), the returned list ordered by (score descending, index
+ascending), the returned set equal to the oracle's top-k up to rows whose
+oracle scores lie within twice that tolerance of the k-th best, and any two
+returned rows further apart than that in the oracle's order.
 """
 import numpy as np
 import pytest
@@ -22,7 +24,14 @@ import tq_testlib as tl
 pytestmark = pytest.mark.gpu
 
 D = 1536
-SCORE_TOL = 1e-3
+# Score tolerances relative to the RMS of a query's oracle scores.  The LUT
+# path scores in fp32 and takes the survey's 1e-3 reading as is.  The
+# tensor-core path rounds both operands of every product to fp16 (rows
+# [c[idx] | rho (2 sigma - 1)], queries scaled by a power of two) and sums
+# 3072 of them: emulating that arithmetic on the oracle gives up to 1.1e-3 of
+# the RMS on 3000 rows, so its bound is the derived 3e-3.
+LUT_SCORE_TOL = 1e-3
+MMA_SCORE_TOL = 3e-3
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -66,14 +75,20 @@ def _check_codes(ocodec, gk: np.ndarray, gs: np.ndarray, enc: dict, stats: dict)
     stats["coords"] += 2 * cm.size
 
 
-def _check_topk(s: np.ndarray, gi: np.ndarray, gv: np.ndarray, k: int):
-    """s: oracle scores [nq, n]; gi/gv: GPU indices/scores [nq, k]."""
-    exact = 0
+def _check_topk(s: np.ndarray, gi: np.ndarray, gv: np.ndarray, k: int, rel: float):
+    """s: oracle scores [nq, n]; gi/gv: GPU indices/scores [nq, k].
+
+    With tol = rel * RMS of the query's oracle scores: every returned score is
+    within tol of the oracle's score of that row; the list is ordered by
+    (-score, index); every row whose oracle score beats the k-th best by more
+    than 2 tol is returned and nothing returned falls below it by more than
+    2 tol; and any two returned rows whose oracle scores differ by more than
+    2 tol appear in the oracle's order."""
     for i in range(s.shape[0]):
-        tol = SCORE_TOL * float(np.max(np.abs(s[i])))
+        tol = rel * float(np.sqrt(np.mean(s[i] ** 2)))
         idx = gi[i].astype(np.int64)
         assert len(set(idx.tolist())) == k and idx.min() >= 0 and idx.max() < s.shape[1]
-        assert np.all(np.abs(gv[i] - s[i, idx]) <= tol), (i, gv[i], s[i, idx])
+        assert np.all(np.abs(gv[i] - s[i, idx]) <= tol), (i, np.max(np.abs(gv[i] - s[i, idx])) / tol)
         for a in range(k - 1):   # ordered by (-score, index)
             assert gv[i, a] > gv[i, a + 1] or (gv[i, a] == gv[i, a + 1] and idx[a] < idx[a + 1])
         ref_idx, ref_val = oscan.topk(s[i:i + 1], k)
@@ -81,8 +96,10 @@ def _check_topk(s: np.ndarray, gi: np.ndarray, gv: np.ndarray, k: int):
         assert np.all(s[i, idx] >= kth - 2 * tol)
         must = ref_idx[0][ref_val[0] > kth + 2 * tol]
         assert set(must.tolist()) <= set(idx.tolist())
-        exact += int(list(idx) == list(ref_idx[0]))
-    return exact
+        os_ = s[i, idx]
+        for a in range(k):
+            for b in range(a + 1, k):
+                assert os_[a] >= os_[b] - 2 * tol, (i, a, b)
 
 
 def _special_rows(x: np.ndarray) -> np.ndarray:
@@ -131,8 +148,13 @@ def test_scan_topk_parity(codecs, n, nq, k):
     ws = torch.empty(native.scan_workspace(ncodec, n, nq, k), dtype=torch.uint8, device="cuda")
     native.scan_topk(ncodec, kcode, kscale, qd, k, idx, score, ws)
     torch.cuda.synchronize()
-    exact = _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k)
-    assert exact >= nq - max(1, nq // 10)
+    _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k, MMA_SCORE_TOL)
+    # the lookup-table path on the same database and queries: fp32 scores
+    idx2 = torch.empty_like(idx)
+    score2 = torch.empty_like(score)
+    native.scan_topk_lut(ncodec, kcode, kscale, qd, k, idx2, score2, ws)
+    torch.cuda.synchronize()
+    _check_topk(s, idx2.cpu().numpy(), score2.cpu().numpy().astype(np.float64), k, LUT_SCORE_TOL)
 
 
 def test_scan_rejects_bad_arguments(codecs):
@@ -195,7 +217,9 @@ def test_vector_search_fullsize_sampled(codecs):
         kc, ks = oc.pack_keys(e, ocodec)
         sp = oscan.scores(Q[qi:qi + 1].astype(np.float64), kc, ks, ocodec)[0]
         where = {int(j): t for t, j in enumerate(pool)}
-        tol = SCORE_TOL * float(np.max(np.abs(sp)))
+        # RMS of the exact inner products over all rows stands in for the
+        # RMS of the query's oracle scores (slightly smaller: conservative)
+        tol = MMA_SCORE_TOL * float(np.sqrt(np.mean(true_ip.astype(np.float64) ** 2)))
         mine = np.array([sp[where[int(j)]] for j in gi[qi]])
         assert np.all(np.abs(gv[qi] - mine) <= tol), (qi, gv[qi], mine)
         kth = gv[qi, -1]
@@ -227,11 +251,13 @@ def test_index_and_scan_other_bit_widths(bits):
     idx = torch.empty((nq, k), dtype=torch.int32, device="cuda")
     score = torch.empty((nq, k), dtype=torch.float32, device="cuda")
     ws = torch.empty(native.scan_workspace(ncodec, n, nq, k), dtype=torch.uint8, device="cuda")
-    native.scan_topk(ncodec, torch.from_numpy(kc).cuda(), torch.from_numpy(ks).cuda(),
-                     torch.from_numpy(q).cuda(), k, idx, score, ws)
+    kcd, ksd, qd = torch.from_numpy(kc).cuda(), torch.from_numpy(ks).cuda(), torch.from_numpy(q).cuda()
+    native.scan_topk(ncodec, kcd, ksd, qd, k, idx, score, ws)
     torch.cuda.synchronize()
-    exact = _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k)
-    assert exact >= nq - max(1, nq // 10)
+    _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k, MMA_SCORE_TOL)
+    native.scan_topk_lut(ncodec, kcd, ksd, qd, k, idx, score, ws)
+    torch.cuda.synchronize()
+    _check_topk(s, idx.cpu().numpy(), score.cpu().numpy().astype(np.float64), k, LUT_SCORE_TOL)
 
 
 def test_index_rejects_four_mse_bits():
