@@ -947,11 +947,15 @@ def main():
                                f"({n_sets * per_set / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)",
                             parallelism=f"{world} independent replicas" if world > 1 else "1 GPU"),
                 roofline=dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
-                              frac=achieved / pk["hbm"], traffic=ncu_traffic("tc_chunk_kernel"),
-                              kernel="tc_chunk_kernel (split-K decode main loop, tcgen05)",
+                              frac=achieved / pk["hbm"], traffic=ncu_traffic("dec_kernel"),
+                              kernel="dec_kernel (split-K decode main loop, tcgen05)",
                               kernel_us=kern * 1e6, algorithmic_bytes=alg,
                               bytes_per_token_head=row_bytes(w),
                               peak_source=f"{pk['source']} hbm_gbs"),
+                roofline_step=dict(bound="hbm", achieved=alg / (total / K) / 1e9, peak=pk["hbm"],
+                                   unit="GB/s", frac=alg / (total / K) / 1e9 / pk["hbm"],
+                                   note="the same algorithmic bytes over the whole step (append, "
+                                        "query prologue, chunk kernel, combine)"),
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d,
                          d2h_bytes_per_step=d2h, us_per_step=dt / K_e2e * 1e6,
                          note="public API, pinned host buffers, host sync every step"),

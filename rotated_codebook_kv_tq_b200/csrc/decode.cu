@@ -19,6 +19,7 @@
 #include <cstdlib>
 
 #include "tq_device.cuh"
+#include "tq_sm100.cuh"
 #include "tq_tc.h"
 
 namespace {
@@ -302,6 +303,7 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
   const int c = tid % D, gq = tid / D;
   const int64_t head = blockIdx.x;
   const int S = a.splits;
+  sm100::pdl_wait();   // the chunk kernel has completed (no-op for a plain launch)
   if (a.err && *a.err) {
     // a bounded wait of the chunk kernel gave up: its partials are incomplete
     if (tid < D) a.out[head * D + tid] = CUDART_NAN_F;
@@ -458,9 +460,10 @@ int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
     if (int e = launch_decode_tc(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_len, scale, rc,
                                  rs, splits, a.po, a.pml, bk, logits, err, stream))
       return e;
-    combine_kernel<128><<<B * Hq, CMB * 128, 0, stream>>>(a);
+    if (tq_launch_pdl(combine_kernel<128>, dim3(B * Hq), dim3(CMB * 128), 0, stream, a) != cudaSuccess)
+      return tq_check_launch("combine_kernel");
     tq_count_launch(1);
-    return tq_check_launch("combine_kernel");
+    return TQ_OK;
   }
   switch (c->d) {
     case 64: return run_decode<64>(a, stream);

@@ -69,7 +69,8 @@ __device__ __forceinline__ float pow2_scale(float maxabs) {
 }
 
 // ---------------------------------------------------------------------------
-// tc_prep: one block (128 threads) per (batch, KV head).
+// tc_prep: one block (128 threads) per query head: its RoPE, rotation and
+// sketch, and its four limb rows of the (batch, KV head) group's B operand.
 // ---------------------------------------------------------------------------
 template <int G, int MBK, bool QJL>
 __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
@@ -77,20 +78,27 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
   constexpr int N = tc_n(G);
   constexpr int KM = TK * TD;                 // MSE K bytes
   constexpr int KTOT = KM + (QJL ? TD : 0);
-  __shared__ float q1s[G][TD], q2s[G][TD];
-  __shared__ float red[TCT / 32][2 * G];
-  __shared__ double dred[TCT / 32][2 * G];
-  __shared__ float Fs[2 * G];
+  __shared__ float q1s[TD], q2s[TD];
+  __shared__ float red[TCT / 32][2];
+  __shared__ double dred[TCT / 32][2];
+  __shared__ float Fs[2];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x / G, h = blockIdx.x % G;   // one block per query head
   const int b = bh / a.Hkv, kvh = bh % a.Hkv;
   const int len = a.seq_lens ? min(max(a.seq_lens[b], 1), a.max_len) : a.max_len;
   const int64_t pos = len - 1;
-  if (bh == 0 && tid == 0 && a.err) *a.err = 0u;   // this call's give-up flag
-
-  if (warp < G) {
-    const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + warp;
+  sm100::pdl_trigger();   // the main loop may launch and set itself up meanwhile
+  if (blockIdx.x == 0 && tid == 0 && a.err) *a.err = 0u;   // this call's give-up flag
+  // row tid of S (bf16) is loaded while warp 0 rotates the query
+  uint4 srow[QJL ? TD / 8 : 1];
+  if (QJL) {
+    const uint4 *sp = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * TD);
+#pragma unroll
+    for (int q = 0; q < TD / 8; ++q) srow[q] = sp[q];
+  }
+  if (warp == 0) {
+    const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
     float x[TNW];
 #pragma unroll
     for (int k = 0; k < TNW; ++k) x[k] = tq_load_elem(a.q, hq * TD + lane + 32 * k, a.dtype);
@@ -109,60 +117,47 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
     tq_warp_wht<TNW>(x, lane);
     const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(TD));
 #pragma unroll
-    for (int k = 0; k < TNW; ++k) q1s[warp][lane + 32 * k] = x[k] * inv_sqrt_d;
+    for (int k = 0; k < TNW; ++k) q1s[lane + 32 * k] = x[k] * inv_sqrt_d;
   }
   __syncthreads();
   if (QJL) {
-    // q''_i = sum_j S[i][j] q'_j: thread i reads row i of S (bf16) as 16-byte loads
-    const uint4 *srow = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * TD);
-    float acc[G];
+    // q''_i = sum_j S[i][j] q'_j for i = tid
+    float acc = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 4
     for (int q = 0; q < TD / 8; ++q) {
-      const uint4 v = srow[q];
-      const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
+      const uint32_t wds[4] = {srow[q].x, srow[q].y, srow[q].z, srow[q].w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float sv = __uint_as_float((e & 1) ? (wds[e >> 1] & 0xffff0000u) : (wds[e >> 1] << 16));
-#pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, q1s[h][8 * q + e], acc[h]);
+        acc = fmaf(sv, q1s[8 * q + e], acc);
       }
     }
-#pragma unroll
-    for (int h = 0; h < G; ++h) q2s[h][tid] = acc[h];
+    q2s[tid] = acc;
   }
   __syncthreads();
-  // fixed-point scales: largest |B value| of each head and part
+  // fixed-point scales: largest |B value| of each part
   {
-    float m1[G], m2[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m1[h] = tq_warp_max(fabsf(q1s[h][tid]));
-      m2[h] = QJL ? tq_warp_max(fabsf(q2s[h][tid])) : 0.f;
+    const float m1 = tq_warp_max(fabsf(q1s[tid]));
+    const float m2 = QJL ? tq_warp_max(fabsf(q2s[tid])) : 0.f;
+    if (lane == 0) {
+      red[warp][0] = m1;
+      red[warp][1] = m2;
     }
-    if (lane == 0)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        red[warp][h] = m1[h];
-        red[warp][G + h] = m2[h];
-      }
     __syncthreads();
-    if (tid < 2 * G) {
+    if (tid < 2) {
       float m = red[0][tid];
       for (int w = 1; w < TCT / 32; ++w) m = fmaxf(m, red[w][tid]);
-      Fs[tid] = pow2_scale(2.f * (tid < G ? a.wk_absmax : 1.f) * m);
+      Fs[tid] = pow2_scale(2.f * (tid == 0 ? a.wk_absmax : 1.f) * m);
     }
     __syncthreads();
   }
-  // B operand (K-major, no swizzle): MSE part then QJL part.  One item =
-  // (head h, K chunk kc): its 16 fixed-point values are computed once and
+  // B operand (K-major, no swizzle): MSE part then QJL part.  One item = K
+  // chunk kc: its 16 fixed-point values of this head are computed once and
   // split into the four limb rows n = 4h + l, each stored as one 16-byte
   // write straight to the group's global B region.
   uint8_t *dst = a.bk + static_cast<int64_t>(bh) * a.bk_stride;
   constexpr int NKC = KTOT / 16, NKM = KM / 16;
-  for (int it = tid; it < G * NKC; it += TCT) {
-    const int h = it % G, kc = it / G;
+  for (int kc = tid; kc < NKC; kc += TCT) {
     const bool mse = kc < NKM;
     const int kb = mse ? kc * 16 : (kc - NKM) * 16;
     uint32_t wv[4][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
@@ -172,7 +167,7 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
       const int col = kk >> 2, nb = kk & 3;
       const int ti = col >> 5, w = (col & 31) >> 3, r = col & 7;
       const int i = 32 * w + 8 * nb + r;
-      const float val = mse ? 2.f * a.wk[ti] * q1s[h][i] * Fs[h] : 2.f * q2s[h][i] * Fs[G + h];
+      const float val = mse ? 2.f * a.wk[ti] * q1s[i] * Fs[0] : 2.f * q2s[i] * Fs[1];
       int v = __float2int_rn(val) * (1 << (7 - r));
       // signed base-256 digits: v = L0 + 2^8 L1 + 2^16 L2 + 2^24 L3
 #pragma unroll
@@ -187,54 +182,48 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
       *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(4 * h + l, kb, N)) =
           make_uint4(wv[l][0], wv[l][1], wv[l][2], wv[l][3]);
   }
-  // rows beyond the G heads' limbs (N > 4 G) are zero
+  // rows beyond the G heads' limbs (N > 4 G) are zero (written by head 0's block)
   if constexpr (N > 4 * G) {
-    for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
-      const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
-      const bool mse = kc < NKM;
-      const int kb = mse ? kc * 16 : (kc - NKM) * 16;
-      *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
-    }
+    if (h == 0)
+      for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
+        const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
+        const bool mse = kc < NKM;
+        const int kb = mse ? kc * 16 : (kc - NKM) * 16;
+        *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
+      }
   }
-  // constants: C = sum of the quantized B values / (2F), per head and part
+  // constants: C = sum of the quantized B values / (2F) of each part
   {
-    double c1[G], c2[G];
+    double s1 = 0.0;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      double s1 = 0.0;
+    for (int ti = 0; ti < TK; ++ti) s1 += __float2int_rn(2.f * a.wk[ti] * q1s[tid] * Fs[0]);
+    double s2 = QJL ? static_cast<double>(__float2int_rn(2.f * q2s[tid] * Fs[1])) : 0.0;
 #pragma unroll
-      for (int ti = 0; ti < TK; ++ti) s1 += __float2int_rn(2.f * a.wk[ti] * q1s[h][tid] * Fs[h]);
-      c1[h] = s1;
-      c2[h] = QJL ? static_cast<double>(__float2int_rn(2.f * q2s[h][tid] * Fs[G + h])) : 0.0;
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(TQ_FULL, s1, o);
+      s2 += __shfl_xor_sync(TQ_FULL, s2, o);
     }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        c1[h] += __shfl_xor_sync(TQ_FULL, c1[h], o);
-        c2[h] += __shfl_xor_sync(TQ_FULL, c2[h], o);
-      }
+    if (lane == 0) {
+      dred[warp][0] = s1;
+      dred[warp][1] = s2;
     }
-    if (lane == 0)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        dred[warp][h] = c1[h];
-        dred[warp][G + h] = c2[h];
-      }
   }
   __syncthreads();
-  if (tid < G) {
+  if (tid == 0) {
     double s1 = 0.0, s2 = 0.0;
     for (int w = 0; w < TCT / 32; ++w) {
-      s1 += dred[w][tid];
-      s2 += dred[w][G + tid];
+      s1 += dred[w][0];
+      s2 += dred[w][1];
     }
     float *kc = reinterpret_cast<float *>(dst + N * KTOT);
-    kc[tid * 4 + 0] = static_cast<float>(s1 / (2.0 * Fs[tid]));
-    kc[tid * 4 + 1] = 1.0f / (128.0f * Fs[tid]);
-    kc[tid * 4 + 2] = static_cast<float>(s2 / (2.0 * Fs[G + tid]));
-    kc[tid * 4 + 3] = 1.0f / (128.0f * Fs[G + tid]);
+    kc[h * 4 + 0] = static_cast<float>(s1 / (2.0 * Fs[0]));
+    kc[h * 4 + 1] = 1.0f / (128.0f * Fs[0]);
+    kc[h * 4 + 2] = static_cast<float>(s2 / (2.0 * Fs[1]));
+    kc[h * 4 + 3] = 1.0f / (128.0f * Fs[1]);
   }
+  // the main loop reads the cache rows the preceding append kernel writes:
+  // this grid completes only after that one (which it may have overlapped)
+  sm100::pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -271,7 +260,7 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
 // dec_kernel: split-K decode main loop.  Two CTAs per SM, each walking its
 // (batch, KV head, split) units (at most UMAX rows) phase by phase:
 //   K  key tiles of 128 rows: bit planes -> Walsh-term operands in tensor
-//      memory (a ring of NSLOT term slots) -> kind::i8 MMAs against the
+//      memory (two term slots per warp group) -> kind::i8 MMAs against the
 //      fixed-point query (B, shared memory) -> logits of the G heads;
 //   S  softmax statistics of the unit and the value-side B operand (24-bit
 //      weights p * nu_v as four int8 limbs) for all of its 32-token groups;
@@ -279,19 +268,20 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
 //      MMAs accumulating the rotated-domain sums over the unit;
 //   E  fold the value accumulators into the running output of the chunk.
 // The two CTAs of an SM overlap each other's S and E phases with streaming.
-// Warp roles: 0-3 expand key tiles and value groups and run E (one TMEM lane
-// each); 4-7 run the key epilogue; 0-7 share S; 8-9 issue MMAs (a tcgen05.mma
-// issue holds its thread for ~45 cycles at these N, so two warps issue side
-// by side: key terms alternate between them, each into its own accumulator,
-// summed exactly in the epilogue); 10 issues every bulk copy ahead of use.
-// Every wait is bounded and warp-uniform; one that gives up makes the whole
-// CTA drain its copies and MMAs and set the call's status word.
+// Warp roles: warp groups 0 (warps 0-3) and 1 (warps 4-7), one TMEM lane per
+// thread, take alternate key tiles (expansion and epilogue) and alternate
+// value groups, share S, and group 0 runs E.  Warp 8 + g issues the key MMAs
+// of group g's tiles (a tcgen05.mma issue holds its thread for ~45 cycles at
+// these N, so the two issue side by side) and the value MMAs of Walsh terms
+// of parity g (each term's accumulator has one issuer).  Warp 10 issues every
+// bulk copy ahead of use.  Every wait is bounded and warp-uniform; one that
+// gives up makes the whole CTA drain its copies and MMAs and set the call's
+// status word.
 // ---------------------------------------------------------------------------
 constexpr int DT = 352;        // 11 warps
 constexpr int UMAX = 1024;     // rows per unit
-constexpr int KS = 3;          // key tile stages (shared memory)
-constexpr int VS = 6;          // value group stages (shared memory)
-constexpr int NSLOT = 4;       // key term slots in tensor memory (32 columns each)
+constexpr int KS = 4;          // key tile stages (shared memory)
+constexpr int VS = 8;          // value group stages (shared memory)
 constexpr int DCOLS = 256;     // tensor memory per CTA
 
 struct DecLayout {
@@ -349,10 +339,10 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
   constexpr int BKB = N * KTOT;
   constexpr int BKC = BKB + G * 16;
   constexpr int NKT = TK + (QJL ? 1 : 0);
-  constexpr int NACC = (TK >= 2 ? 2 : 1) + (QJL ? 1 : 0);   // key accumulators per tile
-  // tensor memory (256 columns): key phase: term slots [0, 128), D_k[2] from 128;
-  // value phase: A_v[2] [0, 16 TV), D_v [128, 128 + N TV)
-  constexpr int C_SLOT = 0, C_DK = 128, C_AV = 0, C_DV = 128;
+  constexpr int NACC = QJL ? 2 : 1;      // key accumulators per tile: MSE terms, sign plane
+  // tensor memory (256 columns): key phase: group g's term slots [64 g, 64 g + 64),
+  // D_k[g] [128 + 2 N g, ...); value phase: A_v[g] [8 TV g, ...), D_v [128, 128 + N TV)
+  constexpr int C_DK = 128, C_DV = 128;
   static_assert(C_DK + 2 * NACC * N <= DCOLS && C_DV + TV * N <= DCOLS && 2 * TV * 8 <= 128,
                 "tensor memory budget");
   constexpr uint32_t IDESC = sm100::idesc_i8(128, N);
@@ -360,7 +350,7 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t kf[KS], ke[KS], vf[VS], ve[VS], hdr[2], hdr_free[2];
-  __shared__ __align__(8) uint64_t as_full[NSLOT], as_empty[NSLOT], dk_full[2], dk_empty[2];
+  __shared__ __align__(8) uint64_t as_full[4], as_empty[4], dk_full[2], dk_empty[2];
   __shared__ __align__(8) uint64_t av_full[2], av_empty[2], bv_full, dv_full, tm_free, sbar, done[2];
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
@@ -373,13 +363,13 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
 
   if (warp == 0) sm100::tmem_alloc(&tmem_s, DCOLS);
   if (tid == 0) {
-    for (int i = 0; i < KS; ++i) { sm100::mbar_init(&kf[i], 1); sm100::mbar_init(&ke[i], 8); }
+    for (int i = 0; i < KS; ++i) { sm100::mbar_init(&kf[i], 1); sm100::mbar_init(&ke[i], 4); }
     for (int i = 0; i < VS; ++i) { sm100::mbar_init(&vf[i], 1); sm100::mbar_init(&ve[i], 4); }
-    for (int i = 0; i < NSLOT; ++i) { sm100::mbar_init(&as_full[i], 4); sm100::mbar_init(&as_empty[i], 1); }
+    for (int i = 0; i < 4; ++i) { sm100::mbar_init(&as_full[i], 4); sm100::mbar_init(&as_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       sm100::mbar_init(&hdr[i], 1);
       sm100::mbar_init(&hdr_free[i], 8);
-      sm100::mbar_init(&dk_full[i], 2);
+      sm100::mbar_init(&dk_full[i], 1);
       sm100::mbar_init(&dk_empty[i], 4);
       sm100::mbar_init(&av_full[i], 4);
       sm100::mbar_init(&av_empty[i], 2);
@@ -396,6 +386,9 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
   __syncthreads();
   sm100::fence_after_sync();
   const uint32_t tm = tmem_s;
+  // the query prologue (and, through it, the append) has completed
+  sm100::pdl_wait();
+  sm100::pdl_trigger();
 
   // empty chunks (beyond a batch's length) merge with weight zero
   if (warp < 8) {
@@ -477,10 +470,10 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
     __syncwarp();
   } else if (warp >= 8) {
     // ------------------------------------------------------------ MMA issue
-    const int is = warp - 8;
+    const int is = warp - 8;           // serves warp group `is`
     if (lane == 0) {
       int cit = blockIdx.x, cr0 = -1, u = 0;
-      uint32_t kt = 0, ts = 0, vg = 0;
+      uint32_t tw = 0, ktw = 0, vu[2] = {0u, 0u};   // terms / tiles of group is; uses of A_v[b]
       bool have = tc_next(a, cit, cr0);
       bool ok = true;
       while (have && ok) {
@@ -492,50 +485,42 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         // the previous unit's value epilogue has read D_v (it overlaps D_k)
         if (u > 0) ok = dwait1(&tm_free, (u - 1) & 1, outer, &abort_s);
         if (ok) ok = dwait1(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);
-        for (int j = 0; j < ntile && ok; ++j, ++kt) {
-          const int kb = kt & 1;
-          if (kt >= 2 && !(ok = dwait1(&dk_empty[kb], ((kt >> 1) - 1) & 1, outer, &abort_s))) break;
-          const uint32_t dk = tm + C_DK + kb * NACC * N;
-          bool any = false, first_mse = true;
+        const uint32_t dk = tm + C_DK + is * NACC * N;
+        for (int j = is; j < ntile && ok; j += 2, ++ktw) {
+          if (ktw >= 1 && !(ok = dwait1(&dk_empty[is], (ktw - 1) & 1, outer, &abort_s))) break;
 #pragma unroll
-          for (int t = 0; t < NKT; ++t, ++ts) {
-            // owner: MSE terms alternate between the two issuers, the sign
-            // plane goes to issuer 1 (issuer 0 when there is one MSE term)
-            const int owner = t < TK ? (t & 1) : (TK >= 2 ? 1 : 0);
-            if (owner != is) continue;
-            const int slot = ts % NSLOT;
-            if (!(ok = dwait1(&as_full[slot], (ts / NSLOT) & 1, outer, &abort_s))) break;
+          for (int t = 0; t < NKT; ++t, ++tw) {
+            const int slot = 2 * is + (tw & 1);
+            if (!(ok = dwait1(&as_full[slot], (tw >> 1) & 1, outer, &abort_s))) break;
             sm100::fence_after_sync();
-            const uint32_t acc = t < TK ? dk + is * N : dk + (NACC - 1) * N;
-            const uint32_t boff = t < TK ? static_cast<uint32_t>(t) * 4 * 2 * N * 16 : N * KM;
-            const bool fresh = t < TK ? first_mse : true;
+            const bool sign = QJL && t == TK;
+            const uint32_t acc = sign ? dk + N : dk;
+            const uint32_t boff = sign ? N * KM : static_cast<uint32_t>(t) * 4 * 2 * N * 16;
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4)
-              sm100::mma_i8_ts(acc, tm + C_SLOT + slot * 32 + s4 * 8,
+              sm100::mma_i8_ts(acc, tm + slot * 32 + s4 * 8,
                                sm100::smem_desc(bk_addr + boff + s4 * 2 * N * 16, N * 16, 128), IDESC,
-                               (fresh && s4 == 0) ? 0u : 1u);
-            if (t < TK) first_mse = false;
+                               ((t == 0 || sign) && s4 == 0) ? 0u : 1u);
             sm100::mma_commit(&as_empty[slot]);
-            any = true;
           }
           if (!ok) break;
-          if (any) sm100::mma_commit(&dk_full[kb]);
-          else sm100::mbar_arrive(&dk_full[kb]);
+          sm100::mma_commit(&dk_full[is]);
         }
         if (!ok) break;
         // value groups: the unit's B operand is complete
         ok = dwait1(&bv_full, u & 1, outer, &abort_s);
         const uint32_t bv_addr = sm100::smem_addr(smem + L.o_bv);
-        for (int g = 0; g < ngroups && ok; ++g, ++vg) {
-          const int ab = vg & 1;
-          if (!(ok = dwait1(&av_full[ab], (vg >> 1) & 1, outer, &abort_s))) break;
+        for (int g = 0; g < ngroups && ok; ++g) {
+          const int ab = g & 1;
+          if (!(ok = dwait1(&av_full[ab], vu[ab] & 1, outer, &abort_s))) break;
+          ++vu[ab];
           sm100::fence_after_sync();
           const uint64_t bd = sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128);
           bool any = false;
 #pragma unroll
           for (int ti = 0; ti < TV; ++ti) {
             if ((ti & 1) != is) continue;
-            sm100::mma_i8_ts(tm + C_DV + ti * N, tm + C_AV + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
+            sm100::mma_i8_ts(tm + C_DV + ti * N, tm + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
             any = true;
           }
           if (any) sm100::mma_commit(&av_empty[ab]);
@@ -553,13 +538,13 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ rows / coordinates
-    const bool rw = warp < 4;          // expansion + value epilogue; else key epilogue
+    // ------------------------------------------------------------ warp groups 0 and 1
+    const int wg = warp >> 2;
     const int wq = warp & 3;
     float *lg = reinterpret_cast<float *>(smem + L.o_lg);
     int8_t *bvs = reinterpret_cast<int8_t *>(smem + L.o_bv);
     int cit = blockIdx.x, cr0 = -1, u = 0;
-    uint32_t kt = 0, ts = 0, vg = 0, sp_par = 0;
+    uint32_t kt = 0, tw = 0, ktw = 0, vg = 0, vu = 0, sp_par = 0;
     float o[G], m_run[G], l_run[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { o[h] = 0.f; m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; }
@@ -588,107 +573,107 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
       float mloc[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
-      bool ok = true;
-      // ---------------- K phase
-      if (rw) {
-        for (int j = 0; j < ntile && ok; ++j, ++kt) {
-          const int s = kt % KS;
-          if (!(ok = dwait(&kf[s], (kt / KS) & 1, outer, &abort_s))) break;
-          const uint4 *kr = reinterpret_cast<const uint4 *>(smem + L.o_kt + s * L.ktb + lt * PK * 16);
-          uint32_t pw[PK][TNW];
+      bool ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);   // kcst of this unit
+      // ---------------- K phase: this group's tiles (expansion, then epilogue)
+      for (int j = wg; j < ntile && ok; j += 2, ++ktw) {
+        const uint32_t ktj = kt + j;
+        const int s = ktj % KS;
+        if (!(ok = dwait(&kf[s], (ktj / KS) & 1, outer, &abort_s))) break;
+        const uint8_t *stg = smem + L.o_kt + s * L.ktb;
+        const uint4 *kr = reinterpret_cast<const uint4 *>(stg + lt * PK * 16);
+        uint32_t pw[PK][TNW];
 #pragma unroll
-          for (int p = 0; p < PK; ++p) {
-            const uint4 v = kr[p];
-            pw[p][0] = v.x; pw[p][1] = v.y; pw[p][2] = v.z; pw[p][3] = v.w;
-          }
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&ke[s]);
-#pragma unroll
-          for (int t = 0; t < NKT; ++t, ++ts) {
-            const int slot = ts % NSLOT;
-            if (ts >= NSLOT && !(ok = dwait(&as_empty[slot], ((ts / NSLOT) - 1) & 1, outer, &abort_s))) break;
-            sm100::fence_after_sync();
-#pragma unroll
-            for (int w = 0; w < TNW; ++w) {
-              uint32_t x = 0;
-              if (t < TK) {
-                const int mask = odd_mask(MBK, t);
-#pragma unroll
-                for (int p = 0; p < MBK; ++p)
-                  if ((mask >> p) & 1) x ^= pw[p][w];
-              } else {
-                x = pw[PK - 1][w];
-              }
-              uint32_t r8[8];
-#pragma unroll
-              for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-              sm100::tmem_st8(sm100::tmem_lane(tm + C_SLOT + slot * 32 + w * 8, wq), r8);
-            }
-            sm100::wait_st();
-            sm100::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&as_full[slot]);
-          }
+        for (int p = 0; p < PK; ++p) {
+          const uint4 v = kr[p];
+          pw[p][0] = v.x; pw[p][1] = v.y; pw[p][2] = v.z; pw[p][3] = v.w;
         }
-      } else {
-        ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);   // kcst of this unit
-        for (int j = 0; j < ntile && ok; ++j, ++kt) {
-          const int kb = kt & 1, s = kt % KS;
-          if (!(ok = dwait(&dk_full[kb], (kt >> 1) & 1, outer, &abort_s))) break;
+        const uint32_t sc = reinterpret_cast<const uint32_t *>(stg + 128 * PK * 16)[lt];
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&ke[s]);
+#pragma unroll
+        for (int t = 0; t < NKT; ++t, ++tw) {
+          const int slot = 2 * wg + (tw & 1);
+          if (tw >= 2 && !(ok = dwait(&as_empty[slot], ((tw >> 1) - 1) & 1, outer, &abort_s))) break;
           sm100::fence_after_sync();
-          const uint32_t dka = tm + C_DK + kb * NACC * N;
-          uint32_t dm[N], dq[N];
+          uint32_t r32[32];
 #pragma unroll
-          for (int c = 0; c < N; ++c) dm[c] = dq[c] = 0u;
+          for (int w = 0; w < TNW; ++w) {
+            uint32_t x = 0;
+            if (t < TK) {
+              const int mask = odd_mask(MBK, t);
 #pragma unroll
-          for (int ac = 0; ac < NACC; ++ac) {
-            uint32_t tv[N];
-            if (N == 16) {
-              uint32_t t16[16];
-              sm100::tmem_ld16(sm100::tmem_lane(dka + ac * N, wq), t16);
-              sm100::wait_ld();
-#pragma unroll
-              for (int c = 0; c < 16; ++c) tv[c % N] = t16[c];
+              for (int p = 0; p < MBK; ++p)
+                if ((mask >> p) & 1) x ^= pw[p][w];
             } else {
-              uint32_t t8[8];
-              sm100::tmem_ld8(sm100::tmem_lane(dka + ac * N, wq), t8);
-              sm100::wait_ld();
-#pragma unroll
-              for (int c = 0; c < 8; ++c) tv[c % N] = t8[c];
+              x = pw[PK - 1][w];
             }
-            const bool sign_acc = QJL && ac == NACC - 1;
 #pragma unroll
-            for (int c = 0; c < N; ++c) {
-              if (sign_acc) dq[c] = tv[c];
-              else dm[c] += tv[c];
-            }
+            for (int r = 0; r < 8; ++r) r32[w * 8 + r] = x & (0x01010101u << r);
           }
+          sm100::tmem_st32(sm100::tmem_lane(tm + slot * 32, wq), r32);
+          sm100::wait_st();
           sm100::fence_before_sync();
           __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&dk_empty[kb]);
-          const int rl = j * 128 + lt;
-          const bool valid = rl < nvalid;
-          const uint32_t sc = reinterpret_cast<const uint32_t *>(smem + L.o_kt + s * L.ktb + 128 * PK * 16)[lt];
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&ke[s]);
-          const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
-          const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+          if (lane == 0) sm100::mbar_arrive(&as_full[slot]);
+        }
+        if (!ok) break;
+        // epilogue of this tile
+        if (!(ok = dwait(&dk_full[wg], ktw & 1, outer, &abort_s))) break;
+        sm100::fence_after_sync();
+        const uint32_t dka = tm + C_DK + wg * NACC * N;
+        uint32_t dm[N], dq[N];
+        if (N == 16) {
+          uint32_t t16[16];
+          sm100::tmem_ld16(sm100::tmem_lane(dka, wq), t16);
+          if (QJL) {
+            uint32_t q16[16];
+            sm100::tmem_ld16(sm100::tmem_lane(dka + N, wq), q16);
+            sm100::wait_ld();
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float dmv = comb_limbs(dm + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
-            float est = dmv;
-            if (QJL) {
-              const float dj = comb_limbs(dq + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
-              est = fmaf(a.qjl_coef * rho, dj, dmv);
-            }
-            const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
-            lg[rl * G + h] = l;
-            mloc[h] = fmaxf(mloc[h], l);
-            if (a.logits && valid)
-              a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
+            for (int c = 0; c < 16; ++c) dq[c % N] = q16[c];
+          } else {
+            sm100::wait_ld();
           }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) dm[c % N] = t16[c];
+        } else {
+          uint32_t t8[8];
+          sm100::tmem_ld8(sm100::tmem_lane(dka, wq), t8);
+          if (QJL) {
+            uint32_t q8[8];
+            sm100::tmem_ld8(sm100::tmem_lane(dka + N, wq), q8);
+            sm100::wait_ld();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) dq[c % N] = q8[c];
+          } else {
+            sm100::wait_ld();
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) dm[c % N] = t8[c];
+        }
+        sm100::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&dk_empty[wg]);
+        const int rl = j * 128 + lt;
+        const bool valid = rl < nvalid;
+        const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+        const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float dmv = comb_limbs(dm + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
+          float est = dmv;
+          if (QJL) {
+            const float dj = comb_limbs(dq + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
+            est = fmaf(a.qjl_coef * rho, dj, dmv);
+          }
+          const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
+          lg[rl * G + h] = l;
+          mloc[h] = fmaxf(mloc[h], l);
+          if (a.logits && valid)
+            a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
         }
       }
+      kt += ntile;
       // ---------------- S phase (8 warps)
       if (ok) {
 #pragma unroll
@@ -699,7 +684,6 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         ok = sync8();
       }
       float mnew[G], corr[G], lsum[G], FV = 1.f, invFV = 1.f;
-      if (ok) ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);
       if (ok) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -795,75 +779,92 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         l_run[h] = l_run[h] * corr[h] + lsum[h];
         m_run[h] = mnew[h];
       }
-      // ---------------- V and E phases (warps 0-3, lane = coordinate)
-      if (rw) {
-        for (int g = 0; g < ngroups && ok; ++g, ++vg) {
-          const int s = vg % VS, ab = vg & 1;
-          if (!(ok = dwait(&vf[s], (vg / VS) & 1, outer, &abort_s))) break;
-          const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
-          uint32_t pw[BV];
+      // ---------------- V phase: this group's value groups (lane = coordinate)
+      for (int g = wg; g < ngroups && ok; g += 2, ++vu) {
+        const uint32_t vgg = vg + g;
+        const int s = vgg % VS;
+        if (!(ok = dwait(&vf[s], (vgg / VS) & 1, outer, &abort_s))) break;
+        const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
+        uint32_t pw[BV];
 #pragma unroll
-          for (int p = 0; p < BV; ++p) pw[p] = vc[p * TD + lt];
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&ve[s]);
-          if (vg >= 2 && !(ok = dwait(&av_empty[ab], ((vg >> 1) - 1) & 1, outer, &abort_s))) break;
-          sm100::fence_after_sync();
+        for (int p = 0; p < BV; ++p) pw[p] = vc[p * TD + lt];
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&ve[s]);
+        if (vu >= 1 && !(ok = dwait(&av_empty[wg], (vu - 1) & 1, outer, &abort_s))) break;
+        sm100::fence_after_sync();
 #pragma unroll
-          for (int ti = 0; ti < TV; ++ti) {
-            const int mask = odd_mask(BV, ti);
+        for (int h4 = 0; h4 < (TV + 3) / 4; ++h4) {
+          uint32_t r32[32];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ti = 4 * h4 + q;
             uint32_t x = 0;
+            if (ti < TV) {
+              const int mask = odd_mask(BV, ti);
 #pragma unroll
-            for (int p = 0; p < BV; ++p)
-              if ((mask >> p) & 1) x ^= pw[p];
-            uint32_t r8[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) r8[r] = x & (0x01010101u << r);
-            sm100::tmem_st8(sm100::tmem_lane(tm + C_AV + ab * TV * 8 + ti * 8, wq), r8);
-          }
-          sm100::wait_st();
-          sm100::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&av_full[ab]);
-        }
-        if (ok) ok = dwait(&dv_full, u & 1, outer, &abort_s);
-        if (ok) {
-          sm100::fence_after_sync();
-          float acc[G];
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll
-          for (int ti = 0; ti < TV; ++ti) {
-            uint32_t dv[N];
-            if (N == 16) {
-              uint32_t t0[16];
-              sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-              sm100::wait_ld();
-#pragma unroll
-              for (int c = 0; c < 16; ++c) dv[c % N] = t0[c];
-            } else {
-              uint32_t t0[8];
-              sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-              sm100::wait_ld();
-#pragma unroll
-              for (int c = 0; c < 8; ++c) dv[c % N] = t0[c];
+              for (int p = 0; p < BV; ++p)
+                if ((mask >> p) & 1) x ^= pw[p];
             }
 #pragma unroll
-            for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
+            for (int r = 0; r < 8; ++r) r32[q * 8 + r] = x & (0x01010101u << r);
           }
-          sm100::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&tm_free);
+          if (TV >= 4) {
+            sm100::tmem_st32(sm100::tmem_lane(tm + wg * TV * 8 + h4 * 32, wq), r32);
+          } else {
+            uint32_t r8[8];
 #pragma unroll
-          for (int h = 0; h < G; ++h) o[h] += acc[h] * invFV - a.wv_sum * wtot[h];
-          if (cr0 + a.sub >= c1) {
+            for (int q = 0; q < TV; ++q) {
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-              a.po[(hq * a.splits + sp) * TD + lt] = o[h];
-              if (tid == 0) {
-                a.pml[(hq * a.splits + sp) * 2] = m_run[h];
-                a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
-              }
+              for (int r = 0; r < 8; ++r) r8[r] = r32[q * 8 + r];
+              sm100::tmem_st8(sm100::tmem_lane(tm + wg * TV * 8 + q * 8, wq), r8);
+            }
+          }
+        }
+        sm100::wait_st();
+        sm100::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&av_full[wg]);
+      }
+      vg += ngroups;
+      // ---------------- E phase: all value MMAs of the unit have landed
+      if (ok) ok = dwait(&dv_full, u & 1, outer, &abort_s);
+      if (ok && wg == 0) {
+        sm100::fence_after_sync();
+        float acc[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll
+        for (int ti = 0; ti < TV; ++ti) {
+          uint32_t dv[N];
+          if (N == 16) {
+            uint32_t t0[16];
+            sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
+            sm100::wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) dv[c % N] = t0[c];
+          } else {
+            uint32_t t0[8];
+            sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
+            sm100::wait_ld();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) dv[c % N] = t0[c];
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
+        }
+        sm100::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&tm_free);
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] += acc[h] * invFV - a.wv_sum * wtot[h];
+        if (cr0 + a.sub >= c1) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
+            a.po[(hq * a.splits + sp) * TD + lt] = o[h];
+            if (tid == 0) {
+              a.pml[(hq * a.splits + sp) * 2] = m_run[h];
+              a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
             }
           }
         }
@@ -911,8 +912,9 @@ int run_dec(TcArgs &a, cudaStream_t stream) {
       return tq_check_launch("cudaFuncSetAttribute(dec_kernel)");
     attr_done[dev] = true;
   }
-  tc_prep_kernel<G, MBK, QJL><<<a.B * a.Hkv, TCT, 0, stream>>>(a);
-  if (int e = tq_check_launch("tc_prep_kernel")) return e;
+  if (tq_launch_pdl(tc_prep_kernel<G, MBK, QJL>, dim3(a.B * a.Hkv * G), dim3(TCT), 0, stream, a) !=
+      cudaSuccess)
+    return tq_check_launch("tc_prep_kernel");
   const int items = a.B * a.Hkv * a.splits;
   const int grid = items < 2 * sms ? items : 2 * sms;
   cudaEvent_t ev0, ev1;
@@ -924,8 +926,8 @@ int run_dec(TcArgs &a, cudaStream_t stream) {
     if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
     cudaEventRecordWithFlags(ev0, stream, ev_flags);
   }
-  dec_kernel<G, MBK, BV, QJL><<<grid, DT, smem, stream>>>(a);
-  if (int e = tq_check_launch("dec_kernel")) return e;
+  if (tq_launch_pdl(dec_kernel<G, MBK, BV, QJL>, dim3(grid), dim3(DT), smem, stream, a) != cudaSuccess)
+    return tq_check_launch("dec_kernel");
   if (ev1) cudaEventRecordWithFlags(ev1, stream, ev_flags);
   tq_count_launch(2);
   return TQ_OK;

@@ -253,6 +253,16 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
   }
   __syncthreads();
   const int planes_k = a.books.mse_bits_k + a.books.qjl;
+  // a following decode's query prologue may start now (it waits for this
+  // grid before it completes)
+  sm100::pdl_trigger();
+  // row tid of S (bf16), loaded up front so its latency overlaps the rows'
+  uint4 srow[D / 8];
+  if (a.books.qjl && tid < D) {
+    const uint4 *sp = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * D);
+#pragma unroll
+    for (int q = 0; q < D / 8; ++q) srow[q] = sp[q];
+  }
   const int64_t it = blockIdx.x;
   const int64_t g = a.g_first + it % a.n_groups;
   const int64_t bh = it / a.n_groups;
@@ -316,9 +326,8 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
     __syncthreads();
     if (a.books.qjl && tid < D) {
       // z_tid = sum_j S[tid][j] r_j; whole warps take part (D is a multiple of 32)
-      const uint4 *srow = reinterpret_cast<const uint4 *>(a.S + static_cast<int64_t>(tid) * D);
       float z = 0.f;
-#pragma unroll 4
+#pragma unroll
       for (int q = 0; q < D / 8; ++q) {
         const uint4 v = srow[q];
         const float4 r0 = reinterpret_cast<const float4 *>(rsm)[2 * q];
@@ -352,7 +361,8 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
     __syncthreads();   // rsm and sgw are reused by the next row
   }
   if (warp == 1) {
-    // the group's value words (read-modify-write for partial groups)
+    // the group's value words (read-modify-write for partial groups; this
+    // block is the only writer of the group within the call)
     const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
     const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
     uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
@@ -360,12 +370,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
         uint32_t *w = vg + p * D + lane + 32 * k;
-        if (mask == TQ_FULL) {
-          *w = vw[p][k];
-        } else {
-          atomicAnd(w, ~mask);
-          atomicOr(w, vw[p][k] & mask);
-        }
+        *w = mask == TQ_FULL ? vw[p][k] : ((*w & ~mask) | (vw[p][k] & mask));
       }
     }
   }

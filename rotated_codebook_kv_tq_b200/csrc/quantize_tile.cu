@@ -504,10 +504,10 @@ int run_tile(const TileArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, co
       return tq_check_launch("cudaFuncSetAttribute(qtile)");
     done[dev] = true;
   }
-  int occ = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, qtile_kernel<D, MBK, BV, QJL>, QT, shm);
-  if (occ < 1) occ = 1;
-  const int64_t cap = static_cast<int64_t>(sms) * occ;
+  // resident CTAs per SM: two at d = 64 (shared memory, registers and 2 x 128
+  // tensor-memory columns all fit), one at d = 128
+  const int per_sm = D == 64 ? 2 : 1;
+  const int64_t cap = static_cast<int64_t>(sms) * per_sm;
   const int grid = static_cast<int>(a.ntiles < cap ? a.ntiles : cap);
   qtile_kernel<D, MBK, BV, QJL><<<grid, QT, shm, stream>>>(mk, mv, mc, ms, a);
   tq_count_launch(1);

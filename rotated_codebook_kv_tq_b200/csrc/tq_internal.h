@@ -44,6 +44,25 @@ struct tq_codec {
   int device;
 };
 
+// Launch `kern` on `stream` allowing programmatic dependent launch: the kernel
+// may be scheduled while the previous kernel of the stream is still running,
+// and must call pdl_wait() (tq_sm100.cuh) before touching that kernel's output.
+template <typename... Params, typename... Args>
+cudaError_t tq_launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+}
+
 // Profiling hooks (api.cu).
 void tq_count_launch(int n);
 void tq_timing_events(cudaEvent_t *start, cudaEvent_t *stop);

@@ -14,6 +14,12 @@
 
 namespace sm100 {
 
+// Programmatic dependent launch: let the next kernel in the stream start its
+// launch now (it still waits in pdl_wait for this grid to complete), and wait
+// for the previous kernel's grid to complete with its memory visible.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
