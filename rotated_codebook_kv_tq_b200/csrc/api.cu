@@ -41,6 +41,24 @@ void walsh_coefficients(const float *c, int bits, float *out, float *absmax, flo
   if (sum) *sum = static_cast<float>(total);
 }
 
+// 21-bit fixed-point centroids as three 7-bit digits: V_i = 2^20 + round(c_i F)
+// with F = (2^20 - 1) / max |c|, V_i = 2^14 d0 + 2^7 d1 + d2.  tab[k] packs
+// digit k of entries 0..15 little-endian, four per word.
+void digit_tables(const float *c, int bits, uint32_t tab[3][4], float *scale) {
+  const int n = 1 << bits;
+  double cmax = 0.0;
+  for (int i = 0; i < n; ++i) cmax = std::fmax(cmax, std::fabs(static_cast<double>(c[i])));
+  const double F = cmax > 0.0 ? 1048575.0 / cmax : 1.0;
+  std::memset(tab, 0, sizeof(uint32_t) * 12);
+  for (int i = 0; i < n; ++i) {
+    long v = 1048576 + std::lrint(static_cast<double>(c[i]) * F);
+    v = v < 0 ? 0 : (v > 2097151 ? 2097151 : v);
+    for (int k = 0; k < 3; ++k)
+      tab[k][i / 4] |= static_cast<uint32_t>((v >> (14 - 7 * k)) & 127) << (8 * (i % 4));
+  }
+  *scale = static_cast<float>(F);
+}
+
 int check_cache(const tq_codec *c, const tq_cache *cache) {
   if (c && c->d > 128)
     return tq_fail(TQ_ERR_UNSUPPORTED, "KV-cache calls support d = 64 and 128 (d = 1536 is index-only)");
@@ -146,6 +164,8 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   c->books.qjl = c->qjl_k;
   walsh_coefficients(c->books.ck, mse_k, c->walsh_k, &c->walsh_k_absmax, nullptr);
   walsh_coefficients(c->books.cv, c->bits_v, c->walsh_v, nullptr, &c->walsh_v_sum);
+  digit_tables(c->books.ck, mse_k, c->digit_k, &c->digit_k_scale);
+  digit_tables(c->books.cv, c->bits_v, c->digit_v, &c->digit_v_scale);
   c->books.bits_v = c->bits_v;
 
   c->ST_dev = nullptr;

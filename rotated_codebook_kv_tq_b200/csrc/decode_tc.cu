@@ -3,31 +3,32 @@
 // Same computation as decode.cu ("TurboESM ..." section 2.E: one pass over the
 // compressed cache; "Google presenta TurboQuant ...", "Eliminacion del sesgo":
 // the prod estimator), restructured so every per-coordinate product runs on
-// the 5th-generation tensor cores as exact integer MMAs:
+// the 5th-generation tensor cores as integer MMAs (kind::i8, int32
+// accumulators, A unsigned from tensor memory, B signed from shared memory):
 //
-// * A symmetric Lloyd-Max codebook is an odd function of its code bits, so
-//   c[idx] = sum_S a_S (2 x_S - 1) over odd subsets S of the bit planes, with
-//   x_S the XOR of the planes in S (exact; a_S solved on the host).  Every
-//   key/value term is therefore a 0/1 plane.
-// * A plane word w (32 coordinates or 32 tokens) becomes 8 registers
-//   w & (0x01010101 << r), r = 0..7: four u8 MMA elements each, worth
-//   x * 2^r.  They are stored straight into tensor memory (tcgen05.st) and fed
-//   to tcgen05.mma kind::i8 as the A operand.  The 2^r weight is undone on the
-//   B side: B holds 24-bit fixed-point values times 2^(7-r), split into four
-//   signed 8-bit limbs, so each int32 accumulator is exact.
-// * Keys: M = 128 key rows (TMEM lane = row), N = 4 limbs x G heads, K = terms x d.
-//   Values: M = 128 coordinates (TMEM lane = coordinate; the cache's 32-token
-//   column groups give each lane its own words), N = 4 limbs x G heads,
-//   K = 32 tokens; one accumulator per Walsh term, combined at the end.
-// * dec_kernel (two CTAs per SM) walks (batch, KV head, split) units of at
-//   most 1024 rows phase by phase: key tiles through a ring of tensor-memory
-//   term slots, the unit's softmax and value-side B operand, then value
-//   groups; bulk copies run ahead of use in shared-memory rings, and two
-//   warps issue the MMAs side by side.
+// * Operands.  Each 32-element slice of a code (32 coordinates of a key row,
+//   or 32 tokens of a value coordinate) becomes 32 A bytes per operand:
+//   - 1- and 2-bit codebooks: one operand per code bit.  A symmetric
+//     codebook is an odd function of its bits, so with one or two bits
+//     c[idx] = sum_p a_p (2 bit_p - 1) exactly (the odd Walsh terms; a_p
+//     solved on the host).  Byte j of A word r holds bit 8j + r as 2^r
+//     (w & (0x01010101 << r)); the 2^r is undone on the B side (x 2^(7-r)).
+//   - 3- and 4-bit codebooks: three operands, the 7-bit digits of the
+//     centroid in 21-bit fixed point, V = 2^20 + round(c F) = 2^14 d0 +
+//     2^7 d1 + d2.  A byte permute (prmt) looks up four codes at once from
+//     the nibble-packed code bits; 16-entry books take both 8-entry halves
+//     and keep one per byte.
+//   The QJL sign plane is a one-bit operand of its own.
+// * B holds the other factor in 24-bit fixed point as four signed 8-bit limbs
+//   (N = 4 limbs x G query heads), so every accumulator is exact; the host
+//   constants undo the fixed-point scales and offsets.
+// * Keys: M = 128 key rows (TMEM lane = row), K = d, one accumulator per
+//   operand.  Values: M = 128 coordinates (lane = coordinate; the cache's
+//   32-token column groups give each lane its own words), K = 32 tokens.
 //
-// Kernels: tc_prep (per (batch, KV head): RoPE, rotation and sketch of the G
-// query heads, fixed-point B operand for the keys) and dec_kernel (the split-K
-// main loop); the chunk partials are merged by decode.cu's combine kernel.
+// Kernels: tc_prep (one block per query head: RoPE, rotation and sketch, the
+// head's rows of the key-side B operand) and dec_kernel (the split-K main
+// loop); the chunk partials are merged by decode.cu's combine kernel.
 #include <math_constants.h>
 
 #include <cstdlib>
@@ -40,19 +41,22 @@ namespace {
 
 constexpr int TD = 128;   // head dim of this path
 constexpr int TNW = TD / 32;
-constexpr int TCT = 128;  // threads of tc_prep: one TMEM lane each
-// Odd subsets of {0..nb-1} in increasing bit-mask order (the Walsh terms).
-__host__ __device__ constexpr int odd_mask(int nb, int t) {
-  int seen = 0;
-  for (int m = 1; m < (1 << nb); ++m) {
-    int pc = 0;
-    for (int x = m; x; x >>= 1) pc += x & 1;
-    if (pc & 1) {
-      if (seen == t) return m;
-      ++seen;
-    }
-  }
-  return 0;
+constexpr int TCT = 128;  // threads of tc_prep
+
+// 3- and 4-bit codebooks use centroid digits, 1- and 2-bit ones bit planes.
+__host__ __device__ constexpr bool use_digits(int bits) { return bits >= 3; }
+// A operands per 32-element slice.
+__host__ __device__ constexpr int n_ops(int bits) { return use_digits(bits) ? 3 : bits; }
+constexpr int NDIG = 3;             // centroid digits
+constexpr float DIG_W0 = 16384.f;   // their weights: 2^14, 2^7, 1
+constexpr float DIG_W1 = 128.f;
+constexpr double DIG_OFF = 1048576.0;   // V = 2^20 + round(c F)
+
+// Element of a 32-element slice at byte k (0..31) of an operand chunk.  Bit
+// planes: byte j of word r holds element 8j + r.  Digits: byte b of word
+// 2j + h holds element 16h + 4b + j.
+__host__ __device__ constexpr int elem_of(bool digits, int k) {
+  return digits ? 16 * ((k >> 2) & 1) + 4 * (k & 3) + (k >> 3) : 8 * (k & 3) + (k >> 2);
 }
 
 // Byte offset of element (n, k) in a K-major, no-swizzle operand of N rows.
@@ -68,15 +72,79 @@ __device__ __forceinline__ float pow2_scale(float maxabs) {
   return ldexpf(1.f, 23 - e);
 }
 
+// prmt.b32: byte i of the result is byte s[4i+2:4i] of {b, a}; bit 4i+3 set
+// replicates that byte's top bit instead.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+  return d;
+}
+
+// The 8 A words of a bit plane: word r = bit 8j + r of x in byte j, as 2^r.
+__device__ __forceinline__ void plane_words(uint32_t x, uint32_t *o) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) o[r] = x & (0x01010101u << r);
+}
+
+// Code of element 4i + j (bit p from plane word pl[p]) in nibble i.
+template <int NB>
+__device__ __forceinline__ uint32_t gather_nibbles(const uint32_t *pl, int j) {
+  uint32_t n = 0;
+#pragma unroll
+  for (int p = 0; p < NB; ++p) {
+    const uint32_t x = p >= j ? pl[p] << (p - j) : pl[p] >> (j - p);
+    n |= x & (0x11111111u << p);
+  }
+  return n;
+}
+
+// Digit words of a 32-element slice: o[k][2j + h], byte b = digit k of the
+// centroid of element 16h + 4b + j (tab[k]: entries 0..15, four per word;
+// every digit is below 128).
+template <int NB>
+__device__ __forceinline__ void digit_words(const uint32_t *pl, const uint32_t (&tab)[NDIG][4],
+                                            uint32_t (&o)[NDIG][8]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t nib = gather_nibbles<NB>(pl, j);
+    if constexpr (NB <= 3) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = h ? nib >> 16 : nib;
+#pragma unroll
+        for (int k = 0; k < NDIG; ++k) o[k][2 * j + h] = prmt(tab[k][0], tab[k][1], sel);
+      }
+    } else {
+      // 16 entries: look both halves up with the low three code bits and
+      // keep, byte by byte, the half that bit 3 picks.  The mask comes from
+      // prmt's sign mode: 0xff where bit 3 is set, else 0x80, whose top bit
+      // is harmless since no digit has it.
+      const uint32_t s7 = nib & 0x77777777u;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = h ? s7 >> 16 : s7;
+        const uint32_t m = prmt(0x80808080u, 0x80808080u, h ? nib >> 16 : nib);
+#pragma unroll
+        for (int k = 0; k < NDIG; ++k) {
+          const uint32_t lo = prmt(tab[k][0], tab[k][1], sel);
+          const uint32_t hi = prmt(tab[k][2], tab[k][3], sel);
+          o[k][2 * j + h] = (hi & m) | (lo & ~m);
+        }
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // tc_prep: one block (128 threads) per query head: its RoPE, rotation and
 // sketch, and its four limb rows of the (batch, KV head) group's B operand.
 // ---------------------------------------------------------------------------
 template <int G, int MBK, bool QJL>
 __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
-  constexpr int TK = 1 << (MBK - 1);
+  constexpr bool DIG = use_digits(MBK);
+  constexpr int NT = n_ops(MBK);
   constexpr int N = tc_n(G);
-  constexpr int KM = TK * TD;                 // MSE K bytes
+  constexpr int KM = NT * TD;                 // MSE K bytes
   constexpr int KTOT = KM + (QJL ? TD : 0);
   __shared__ float q1s[TD], q2s[TD];
   __shared__ float red[TCT / 32][2];
@@ -147,28 +215,34 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
     if (tid < 2) {
       float m = red[0][tid];
       for (int w = 1; w < TCT / 32; ++w) m = fmaxf(m, red[w][tid]);
-      Fs[tid] = pow2_scale(2.f * (tid == 0 ? a.wk_absmax : 1.f) * m);
+      Fs[tid] = pow2_scale(2.f * ((tid == 0 && !DIG) ? a.wk_absmax : 1.f) * m);
     }
     __syncthreads();
   }
-  // B operand (K-major, no swizzle): MSE part then QJL part.  One item = K
-  // chunk kc: its 16 fixed-point values of this head are computed once and
-  // split into the four limb rows n = 4h + l, each stored as one 16-byte
-  // write straight to the group's global B region.
+  // B operand (K-major, no swizzle): the NT MSE operands, then the sign plane,
+  // 128 K bytes each (a digit operand's B is the query itself: the digit
+  // weights are applied to its accumulator).  One item = a 16-byte K slice kb: its 16 fixed-point
+  // values of this head are computed once and split into the four limb rows
+  // n = 4h + l, each stored as one 16-byte write to the group's B region.
   uint8_t *dst = a.bk + static_cast<int64_t>(bh) * a.bk_stride;
-  constexpr int NKC = KTOT / 16, NKM = KM / 16;
+  constexpr int NKC = KTOT / 16;
   for (int kc = tid; kc < NKC; kc += TCT) {
-    const bool mse = kc < NKM;
-    const int kb = mse ? kc * 16 : (kc - NKM) * 16;
+    const int kb = kc * 16;
+    const int op = kb / TD;                  // operand (NT = the sign plane)
+    const int w = (kb % TD) >> 5;            // 32-coordinate chunk
+    const bool dig = DIG && op < NT;
     uint32_t wv[4][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const int kk = kb + e;
-      const int col = kk >> 2, nb = kk & 3;
-      const int ti = col >> 5, w = (col & 31) >> 3, r = col & 7;
-      const int i = 32 * w + 8 * nb + r;
-      const float val = mse ? 2.f * a.wk[ti] * q1s[i] * Fs[0] : 2.f * q2s[i] * Fs[1];
-      int v = __float2int_rn(val) * (1 << (7 - r));
+      const int k = (kb & 31) + e;
+      const int i = 32 * w + elem_of(dig, k);
+      int v;
+      if (dig)
+        v = __float2int_rn(q1s[i] * Fs[0]);
+      else if (op < NT)
+        v = __float2int_rn(2.f * a.wk[op] * q1s[i] * Fs[0]) * (1 << (7 - (k >> 2)));
+      else
+        v = __float2int_rn(2.f * q2s[i] * Fs[1]) * (1 << (7 - (k >> 2)));
       // signed base-256 digits: v = L0 + 2^8 L1 + 2^16 L2 + 2^24 L3
 #pragma unroll
       for (int l = 0; l < 4; ++l) {
@@ -179,7 +253,7 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
     }
 #pragma unroll
     for (int l = 0; l < 4; ++l)
-      *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(4 * h + l, kb, N)) =
+      *reinterpret_cast<uint4 *>(dst + kmajor_off(4 * h + l, kb, N)) =
           make_uint4(wv[l][0], wv[l][1], wv[l][2], wv[l][3]);
   }
   // rows beyond the G heads' limbs (N > 4 G) are zero (written by head 0's block)
@@ -187,16 +261,18 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
     if (h == 0)
       for (int it = tid; it < (N - 4 * G) * NKC; it += TCT) {
         const int n = 4 * G + it % (N - 4 * G), kc = it / (N - 4 * G);
-        const bool mse = kc < NKM;
-        const int kb = mse ? kc * 16 : (kc - NKM) * 16;
-        *reinterpret_cast<uint4 *>(dst + (mse ? 0 : N * KM) + kmajor_off(n, kb, N)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(dst + kmajor_off(n, kc * 16, N)) = make_uint4(0u, 0u, 0u, 0u);
       }
   }
-  // constants: C = sum of the quantized B values / (2F) of each part
+  // constants: the offset of each part in B units, and its scale
   {
     double s1 = 0.0;
+    if (DIG) {
+      s1 = __float2int_rn(q1s[tid] * Fs[0]);
+    } else {
 #pragma unroll
-    for (int ti = 0; ti < TK; ++ti) s1 += __float2int_rn(2.f * a.wk[ti] * q1s[tid] * Fs[0]);
+      for (int t = 0; t < NT; ++t) s1 += __float2int_rn(2.f * a.wk[t] * q1s[tid] * Fs[0]);
+    }
     double s2 = QJL ? static_cast<double>(__float2int_rn(2.f * q2s[tid] * Fs[1])) : 0.0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -216,8 +292,15 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
       s2 += dred[w][1];
     }
     float *kc = reinterpret_cast<float *>(dst + N * KTOT);
-    kc[h * 4 + 0] = static_cast<float>(s1 / (2.0 * Fs[0]));
-    kc[h * 4 + 1] = 1.0f / (128.0f * Fs[0]);
+    if (DIG) {
+      // sum_j (V_j - 2^20) B_j / (F_c F): the rotated query against the centroids
+      kc[h * 4 + 0] = static_cast<float>(DIG_OFF * s1 / (static_cast<double>(Fs[0]) * a.kfc));
+      kc[h * 4 + 1] = static_cast<float>(1.0 / (static_cast<double>(Fs[0]) * a.kfc));
+    } else {
+      // sum_t a_t (2 x_t - 1): the 0/1 planes weigh 2 a_t, minus sum_t a_t
+      kc[h * 4 + 0] = static_cast<float>(s1 / (2.0 * Fs[0]));
+      kc[h * 4 + 1] = 1.0f / (128.0f * Fs[0]);
+    }
     kc[h * 4 + 2] = static_cast<float>(s2 / (2.0 * Fs[1]));
     kc[h * 4 + 3] = 1.0f / (128.0f * Fs[1]);
   }
@@ -227,7 +310,7 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// tc_chunk: persistent, one CTA (128 threads, one TMEM lane each) per SM.
+// dec_kernel helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float comb_limbs(const uint32_t *d) {
   // int32 accumulators of limbs 0..3 -> value (exact digits, fp32 rounding)
@@ -256,32 +339,84 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
   return false;
 }
 
+// Warp-uniform bounded wait: every lane polls (so every lane acquires the
+// phase), the loop ends for all lanes together.  Gives up when the budget
+// runs out or another warp has given up.
+__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, uint32_t outer,
+                                      volatile int *abort_flag) {
+  for (uint32_t it = 0; it < outer; ++it) {
+    const bool ok = sm100::mbar_wait(bar, parity, 1u << 8);
+    if (__all_sync(TQ_FULL, ok)) return true;
+    if (__shfl_sync(TQ_FULL, *abort_flag, 0)) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// Single-thread bounded wait for the copying lanes.
+__device__ __forceinline__ bool dwait1(uint64_t *bar, uint32_t parity, uint32_t outer,
+                                       volatile int *abort_flag) {
+  for (uint32_t it = 0; it < outer; ++it) {
+    if (sm100::mbar_wait(bar, parity, 1u << 8)) return true;
+    if (*abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// Barrier of the warp group (warps 0-3) that also tells every thread whether
+// all of them are still on track; the tensor-memory fences order the group's
+// tcgen05 traffic around it.
+__device__ __forceinline__ bool wg_sync(bool ok) {
+  sm100::fence_before_sync();
+  uint32_t bad;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.eq.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(bad)
+      : "r"(ok ? 1u : 0u)
+      : "memory");
+  sm100::fence_after_sync();
+  return bad == 0u;
+}
+
+// N accumulator columns of this warp's lanes (N = 8 or 16), loads in flight.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[16]) {
+  if constexpr (N == 16) {
+    sm100::tmem_ld16(taddr, r);
+  } else {
+    uint32_t t[8];
+    sm100::tmem_ld8(taddr, t);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) r[c] = t[c];
+  }
+}
+
 // ---------------------------------------------------------------------------
 // dec_kernel: split-K decode main loop.  Two CTAs per SM, each walking its
 // (batch, KV head, split) units (at most UMAX rows) phase by phase:
-//   K  key tiles of 128 rows: bit planes -> Walsh-term operands in tensor
-//      memory (two term slots per warp group) -> kind::i8 MMAs against the
-//      fixed-point query (B, shared memory) -> logits of the G heads;
+//   K  key tiles of 128 rows: code planes -> A operands in tensor memory ->
+//      MMAs against the fixed-point query (accumulators for two tiles) ->
+//      logits, two tiles later;
 //   S  softmax statistics of the unit and the value-side B operand (24-bit
 //      weights p * nu_v as four int8 limbs) for all of its 32-token groups;
-//   V  value groups: bit planes -> Walsh-term operands (lane = coordinate) ->
-//      MMAs accumulating the rotated-domain sums over the unit;
+//   V  value batches of four 32-token groups (two batch buffers) -> MMAs
+//      accumulating the rotated-domain sums over the unit;
 //   E  fold the value accumulators into the running output of the chunk.
-// The two CTAs of an SM overlap each other's S and E phases with streaming.
-// Warp roles: warp groups 0 (warps 0-3) and 1 (warps 4-7), one TMEM lane per
-// thread, take alternate key tiles (expansion and epilogue) and alternate
-// value groups, share S, and group 0 runs E.  Warp 8 + g issues the key MMAs
-// of group g's tiles (a tcgen05.mma issue holds its thread for ~45 cycles at
-// these N, so the two issue side by side) and the value MMAs of Walsh terms
-// of parity g (each term's accumulator has one issuer).  Warp 10 issues every
-// bulk copy ahead of use.  Every wait is bounded and warp-uniform; one that
-// gives up makes the whole CTA drain its copies and MMAs and set the call's
-// status word.
+// Warps 0-3 (one TMEM lane per thread) expand, issue and fold: after a
+// warp-group barrier, lane 0 of warp w issues the MMAs of operand w, so MMAs
+// are issued from several threads at once and no other warp sits between
+// expansion and issue.  Warp 4 copies unit headers and key tiles, warp 5
+// value groups, ahead of use.  Every wait is bounded; a warp that gives up
+// makes the group leave at its next barrier, the CTA drain its copies and
+// MMAs, and the call's status word report it.
 // ---------------------------------------------------------------------------
-constexpr int DT = 352;        // 11 warps
+constexpr int DT = 192;        // 6 warps
 constexpr int UMAX = 1024;     // rows per unit
 constexpr int KS = 4;          // key tile stages (shared memory)
 constexpr int VS = 8;          // value group stages (shared memory)
+constexpr int VB = 4;          // value groups per batch
 constexpr int DCOLS = 256;     // tensor memory per CTA
 
 struct DecLayout {
@@ -303,82 +438,51 @@ __host__ __device__ inline DecLayout dec_layout(int PK, int BV, int G, int N, in
   return L;
 }
 
-// Warp-uniform bounded wait: every lane polls (so every lane acquires the
-// phase), the loop ends for all lanes together.  Gives up when the budget
-// runs out or another warp has given up.
-__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, uint32_t outer,
-                                      volatile int *abort_flag) {
-  for (uint32_t it = 0; it < outer; ++it) {
-    const bool ok = sm100::mbar_wait(bar, parity, 1u << 8);
-    if (__all_sync(TQ_FULL, ok)) return true;
-    if (__shfl_sync(TQ_FULL, *abort_flag, 0)) return false;
-  }
-  *abort_flag = 1;
-  return false;
-}
-
-// Single-thread bounded wait for the issuing and copying lanes.
-__device__ __forceinline__ bool dwait1(uint64_t *bar, uint32_t parity, uint32_t outer,
-                                       volatile int *abort_flag) {
-  for (uint32_t it = 0; it < outer; ++it) {
-    if (sm100::mbar_wait(bar, parity, 1u << 8)) return true;
-    if (*abort_flag) return false;
-  }
-  *abort_flag = 1;
-  return false;
-}
-
 template <int G, int MBK, int BV, bool QJL>
 __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
-  constexpr int TK = 1 << (MBK - 1);
-  constexpr int TV = 1 << (BV - 1);
+  constexpr bool KDIG = use_digits(MBK), VDIG = use_digits(BV);
+  constexpr int NT = n_ops(MBK);             // key MSE operands
+  constexpr int NV = n_ops(BV);              // value operands
+  constexpr int NKO = NT + (QJL ? 1 : 0);    // key operands (one accumulator each)
   constexpr int N = tc_n(G);
+  constexpr int NH = N / 4;
   constexpr int PK = MBK + (QJL ? 1 : 0);
-  constexpr int KM = TK * TD;
-  constexpr int KTOT = KM + (QJL ? TD : 0);
-  constexpr int BKB = N * KTOT;
+  constexpr int BKB = N * TD * NKO;
   constexpr int BKC = BKB + G * 16;
-  constexpr int NKT = TK + (QJL ? 1 : 0);
-  constexpr int NACC = QJL ? 2 : 1;      // key accumulators per tile: MSE terms, sign plane
-  // tensor memory (256 columns): key phase: group g's term slots [64 g, 64 g + 64),
-  // D_k[g] [128 + 2 N g, ...); value phase: A_v[g] [8 TV g, ...), D_v [128, 128 + N TV)
-  constexpr int C_DK = 128, C_DV = 128;
-  static_assert(C_DK + 2 * NACC * N <= DCOLS && C_DV + TV * N <= DCOLS && 2 * TV * 8 <= 128,
-                "tensor memory budget");
+  // tensor memory: key phase: the tile's operands [0, KA) (chunk-major MSE
+  // operands, then the sign plane), accumulators D_k[tile parity][op] at
+  // C_DK + N (NKO parity + op); value phase: batch buffers [VA b, VA (b + 1))
+  // (group g at 8 NV g, operand at 8 op), accumulators D_v[op] at C_DV + N op
+  constexpr int KA = 32 * NKO;
+  constexpr int C_DK = KA;
+  constexpr int VA = VB * NV * 8;
+  constexpr int C_DV = 2 * VA;
+  static_assert(C_DK + 2 * NKO * N <= DCOLS && C_DV + NV * N <= DCOLS, "tensor memory budget");
   constexpr uint32_t IDESC = sm100::idesc_i8(128, N);
   const DecLayout L = dec_layout(PK, BV, G, N, BKC);
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t kf[KS], ke[KS], vf[VS], ve[VS], hdr[2], hdr_free[2];
-  __shared__ __align__(8) uint64_t as_full[4], as_empty[4], dk_full[2], dk_empty[2];
-  __shared__ __align__(8) uint64_t av_full[2], av_empty[2], bv_full, dv_full, tm_free, sbar, done[2];
+  __shared__ __align__(8) uint64_t kdone, vdone[2], fin[4];
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
-  __shared__ float redf[8][2 * G + 1];
-  __shared__ unsigned long long wsum_s[8];
+  __shared__ float redf[4][2 * G + 1];
+  __shared__ unsigned long long wsum_s[G];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int lt = tid & 127;
   const uint32_t outer = a.wait_limit >> 8;
 
   if (warp == 0) sm100::tmem_alloc(&tmem_s, DCOLS);
   if (tid == 0) {
     for (int i = 0; i < KS; ++i) { sm100::mbar_init(&kf[i], 1); sm100::mbar_init(&ke[i], 4); }
     for (int i = 0; i < VS; ++i) { sm100::mbar_init(&vf[i], 1); sm100::mbar_init(&ve[i], 4); }
-    for (int i = 0; i < 4; ++i) { sm100::mbar_init(&as_full[i], 4); sm100::mbar_init(&as_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       sm100::mbar_init(&hdr[i], 1);
-      sm100::mbar_init(&hdr_free[i], 8);
-      sm100::mbar_init(&dk_full[i], 1);
-      sm100::mbar_init(&dk_empty[i], 4);
-      sm100::mbar_init(&av_full[i], 4);
-      sm100::mbar_init(&av_empty[i], 2);
-      sm100::mbar_init(&done[i], 1);
+      sm100::mbar_init(&hdr_free[i], 1);
+      sm100::mbar_init(&vdone[i], NV);
     }
-    sm100::mbar_init(&bv_full, 8);
-    sm100::mbar_init(&dv_full, 2);
-    sm100::mbar_init(&tm_free, 4);
-    sm100::mbar_init(&sbar, 8);
+    sm100::mbar_init(&kdone, NKO);
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&fin[i], 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -390,31 +494,13 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
   sm100::pdl_wait();
   sm100::pdl_trigger();
 
-  // empty chunks (beyond a batch's length) merge with weight zero
-  if (warp < 8) {
-    const int items = a.B * a.Hkv * a.splits;
-    for (int it = blockIdx.x; it < items; it += gridDim.x) {
-      const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv, sp = it % a.splits;
-      if (sp * a.chunk < tc_len(a, b)) continue;
-      if (tid < TD)
-        for (int h = 0; h < G; ++h) {
-          const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-          a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
-          if (tid == 0) {
-            a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
-            a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
-          }
-        }
-    }
-  }
-
-  if (warp == 10) {
-    // ------------------------------------------------------------ copies
+  if (warp == 4) {
+    // ------------------------------------------------ unit headers, key tiles
     if (lane == 0) {
       int cit = blockIdx.x, cr0 = -1, u = 0;
-      uint32_t kt = 0, vg = 0;
+      uint32_t kt = 0;
       // per stage: 1 + the parity of its last issued copy (0 = never issued)
-      uint8_t lk[KS] = {}, lv[VS] = {}, lh[2] = {};
+      uint8_t lk[KS] = {}, lh[2] = {};
       bool have = tc_next(a, cit, cr0);
       while (have && !abort_s) {
         const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
@@ -422,7 +508,7 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
         const int nvalid = min(a.sub, c1 - cr0);
         const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
-        // unit header: this unit's B operand and value norms (buffer u & 1),
+        // unit header: B operand, constants and value norms (buffer u & 1),
         // once unit u - 2 has finished its softmax phase with that buffer
         {
           const int hb = u & 1;
@@ -444,6 +530,33 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
           sm100::bulk_g2s(st + 128 * PK * 16, a.kscale + (bh * a.rows_cap + row) * 2, nrow * 4, &kf[s]);
           lk[s] = static_cast<uint8_t>(1 + ((kt / KS) & 1));
         }
+        cr0 += a.sub;
+        have = tc_next(a, cit, cr0);
+        ++u;
+      }
+      if (abort_s) {
+        // this CTA's own copies land before its shared memory is released:
+        // each stage's last issued phase completes (at once if consumed)
+        for (int i = 0; i < KS; ++i)
+          if (lk[i]) sm100::mbar_wait(&kf[i], lk[i] - 1u, 1u << 20);
+        for (int i = 0; i < 2; ++i)
+          if (lh[i]) sm100::mbar_wait(&hdr[i], lh[i] - 1u, 1u << 20);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ value groups
+    if (lane == 0) {
+      int cit = blockIdx.x, cr0 = -1;
+      uint32_t vg = 0;
+      uint8_t lv[VS] = {};
+      bool have = tc_next(a, cit, cr0);
+      while (have && !abort_s) {
+        const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
+        const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
+        const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
+        const int nvalid = min(a.sub, c1 - cr0);
+        const int ngroups = (nvalid + 31) / 32;
         for (int g = 0; g < ngroups && !abort_s; ++g, ++vg) {
           const int s = vg % VS;
           if (vg >= VS && !dwait1(&ve[s], ((vg / VS) - 1) & 1, outer, &abort_s)) break;
@@ -454,111 +567,48 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         }
         cr0 += a.sub;
         have = tc_next(a, cit, cr0);
-        ++u;
       }
-      if (abort_s) {
-        // this CTA's own copies land before its shared memory is released:
-        // each stage's last issued phase completes (at once if consumed)
-        for (int i = 0; i < KS; ++i)
-          if (lk[i]) sm100::mbar_wait(&kf[i], lk[i] - 1u, 1u << 20);
+      if (abort_s)
         for (int i = 0; i < VS; ++i)
           if (lv[i]) sm100::mbar_wait(&vf[i], lv[i] - 1u, 1u << 20);
-        for (int i = 0; i < 2; ++i)
-          if (lh[i]) sm100::mbar_wait(&hdr[i], lh[i] - 1u, 1u << 20);
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ MMA issue
-    const int is = warp - 8;           // serves warp group `is`
-    if (lane == 0) {
-      int cit = blockIdx.x, cr0 = -1, u = 0;
-      uint32_t tw = 0, ktw = 0, vu[2] = {0u, 0u};   // terms / tiles of group is; uses of A_v[b]
-      bool have = tc_next(a, cit, cr0);
-      bool ok = true;
-      while (have && ok) {
-        const int b = cit / (a.Hkv * a.splits), sp = cit % a.splits;
-        const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
-        const int nvalid = min(a.sub, c1 - cr0);
-        const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
-        const uint32_t bk_addr = sm100::smem_addr(smem + L.o_bk + (u & 1) * L.bkc);
-        // the previous unit's value epilogue has read D_v (it overlaps D_k)
-        if (u > 0) ok = dwait1(&tm_free, (u - 1) & 1, outer, &abort_s);
-        if (ok) ok = dwait1(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);
-        const uint32_t dk = tm + C_DK + is * NACC * N;
-        for (int j = is; j < ntile && ok; j += 2, ++ktw) {
-          if (ktw >= 1 && !(ok = dwait1(&dk_empty[is], (ktw - 1) & 1, outer, &abort_s))) break;
-#pragma unroll
-          for (int t = 0; t < NKT; ++t, ++tw) {
-            const int slot = 2 * is + (tw & 1);
-            if (!(ok = dwait1(&as_full[slot], (tw >> 1) & 1, outer, &abort_s))) break;
-            sm100::fence_after_sync();
-            const bool sign = QJL && t == TK;
-            const uint32_t acc = sign ? dk + N : dk;
-            const uint32_t boff = sign ? N * KM : static_cast<uint32_t>(t) * 4 * 2 * N * 16;
-#pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4)
-              sm100::mma_i8_ts(acc, tm + slot * 32 + s4 * 8,
-                               sm100::smem_desc(bk_addr + boff + s4 * 2 * N * 16, N * 16, 128), IDESC,
-                               ((t == 0 || sign) && s4 == 0) ? 0u : 1u);
-            sm100::mma_commit(&as_empty[slot]);
-          }
-          if (!ok) break;
-          sm100::mma_commit(&dk_full[is]);
-        }
-        if (!ok) break;
-        // value groups: the unit's B operand is complete
-        ok = dwait1(&bv_full, u & 1, outer, &abort_s);
-        const uint32_t bv_addr = sm100::smem_addr(smem + L.o_bv);
-        for (int g = 0; g < ngroups && ok; ++g) {
-          const int ab = g & 1;
-          if (!(ok = dwait1(&av_full[ab], vu[ab] & 1, outer, &abort_s))) break;
-          ++vu[ab];
-          sm100::fence_after_sync();
-          const uint64_t bd = sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128);
-          bool any = false;
-#pragma unroll
-          for (int ti = 0; ti < TV; ++ti) {
-            if ((ti & 1) != is) continue;
-            sm100::mma_i8_ts(tm + C_DV + ti * N, tm + ab * TV * 8 + ti * 8, bd, IDESC, g > 0);
-            any = true;
-          }
-          if (any) sm100::mma_commit(&av_empty[ab]);
-          else sm100::mbar_arrive(&av_empty[ab]);
-        }
-        if (!ok) break;
-        sm100::mma_commit(&dv_full);
-        cr0 += a.sub;
-        have = tc_next(a, cit, cr0);
-        ++u;
-      }
-      // every MMA of this thread has landed before tensor memory is freed
-      sm100::mma_commit(&done[is]);
-      sm100::mbar_wait(&done[is], 0, 1u << 20);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ warp groups 0 and 1
-    const int wg = warp >> 2;
-    const int wq = warp & 3;
+    // --------------------------------------------------------- the warp group
+    // empty chunks (beyond a batch's length) merge with weight zero
+    {
+      const int items = a.B * a.Hkv * a.splits;
+      for (int it = blockIdx.x; it < items; it += gridDim.x) {
+        const int b = it / (a.Hkv * a.splits), kvh = (it / a.splits) % a.Hkv, sp = it % a.splits;
+        if (sp * a.chunk < tc_len(a, b)) continue;
+        for (int h = 0; h < G; ++h) {
+          const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
+          a.po[(hq * a.splits + sp) * TD + tid] = 0.f;
+          if (tid == 0) {
+            a.pml[(hq * a.splits + sp) * 2] = -CUDART_INF_F;
+            a.pml[(hq * a.splits + sp) * 2 + 1] = 0.f;
+          }
+        }
+      }
+    }
+    uint32_t ktab[NDIG][4], vtab[NDIG][4];
+#pragma unroll
+    for (int d = 0; d < NDIG; ++d)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        ktab[d][i] = a.ktab[d][i];
+        vtab[d][i] = a.vtab[d][i];
+      }
     float *lg = reinterpret_cast<float *>(smem + L.o_lg);
     int8_t *bvs = reinterpret_cast<int8_t *>(smem + L.o_bv);
+    const uint32_t bv_addr = sm100::smem_addr(bvs);
     int cit = blockIdx.x, cr0 = -1, u = 0;
-    uint32_t kt = 0, tw = 0, ktw = 0, vg = 0, vu = 0, sp_par = 0;
+    uint32_t kt = 0, vg = 0, vb = 0;
     float o[G], m_run[G], l_run[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { o[h] = 0.f; m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; }
+    bool ok = true;
     bool have = tc_next(a, cit, cr0);
-    // all 8 row warps meet (bounded)
-    auto sync8 = [&]() -> bool {
-      sm100::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&sbar);
-      const bool r = dwait(&sbar, sp_par, outer, &abort_s);
-      sp_par ^= 1u;
-      sm100::fence_after_sync();
-      return r;
-    };
     while (have) {
       const int b = cit / (a.Hkv * a.splits), kvh = (cit / a.splits) % a.Hkv, sp = cit % a.splits;
       const int len = tc_len(a, b);
@@ -566,6 +616,7 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
       const int nvalid = min(a.sub, c1 - cr0);
       const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
       const float *kcst = reinterpret_cast<const float *>(smem + L.o_bk + (u & 1) * L.bkc + BKB);
+      const uint32_t bk_addr = sm100::smem_addr(smem + L.o_bk + (u & 1) * L.bkc);
       if (cr0 == c0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) { o[h] = 0.f; m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; }
@@ -573,204 +624,197 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
       float mloc[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) mloc[h] = -CUDART_INF_F;
-      bool ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);   // kcst of this unit
-      // ---------------- K phase: this group's tiles (expansion, then epilogue)
-      for (int j = wg; j < ntile && ok; j += 2, ++ktw) {
-        const uint32_t ktj = kt + j;
-        const int s = ktj % KS;
-        if (!(ok = dwait(&kf[s], (ktj / KS) & 1, outer, &abort_s))) break;
-        const uint8_t *stg = smem + L.o_kt + s * L.ktb;
-        const uint4 *kr = reinterpret_cast<const uint4 *>(stg + lt * PK * 16);
+      if (ok) ok = dwait(&hdr[u & 1], (u >> 1) & 1, outer, &abort_s);   // B operand, constants
+      if (!wg_sync(ok)) break;
+      // ---------------- K phase: tile j is expanded once the MMAs of tile j - 1
+      // have released the operand buffer; its epilogue runs two tiles later
+      // (accumulators double-buffered), so MMAs overlap expansion both ways
+      uint32_t sc_hist[2] = {0u, 0u};
+      for (int j = 0; j <= ntile + 1; ++j) {
+        const uint32_t ti = kt + j;
+        const bool expand = j < ntile;
         uint32_t pw[PK][TNW];
+        uint32_t sc = 0u;
+        if (expand && ok) ok = dwait(&kf[ti % KS], (ti / KS) & 1, outer, &abort_s);
+        if (expand && ok) {
+          const uint8_t *stg = smem + L.o_kt + (ti % KS) * L.ktb;
+          const uint4 *kr = reinterpret_cast<const uint4 *>(stg + tid * PK * 16);
 #pragma unroll
-        for (int p = 0; p < PK; ++p) {
-          const uint4 v = kr[p];
-          pw[p][0] = v.x; pw[p][1] = v.y; pw[p][2] = v.z; pw[p][3] = v.w;
-        }
-        const uint32_t sc = reinterpret_cast<const uint32_t *>(stg + 128 * PK * 16)[lt];
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&ke[s]);
-#pragma unroll
-        for (int t = 0; t < NKT; ++t, ++tw) {
-          const int slot = 2 * wg + (tw & 1);
-          if (tw >= 2 && !(ok = dwait(&as_empty[slot], ((tw >> 1) - 1) & 1, outer, &abort_s))) break;
-          sm100::fence_after_sync();
-          uint32_t r32[32];
-#pragma unroll
-          for (int w = 0; w < TNW; ++w) {
-            uint32_t x = 0;
-            if (t < TK) {
-              const int mask = odd_mask(MBK, t);
-#pragma unroll
-              for (int p = 0; p < MBK; ++p)
-                if ((mask >> p) & 1) x ^= pw[p][w];
-            } else {
-              x = pw[PK - 1][w];
-            }
-#pragma unroll
-            for (int r = 0; r < 8; ++r) r32[w * 8 + r] = x & (0x01010101u << r);
+          for (int p = 0; p < PK; ++p) {
+            const uint4 v = kr[p];
+            pw[p][0] = v.x; pw[p][1] = v.y; pw[p][2] = v.z; pw[p][3] = v.w;
           }
-          sm100::tmem_st32(sm100::tmem_lane(tm + slot * 32, wq), r32);
-          sm100::wait_st();
-          sm100::fence_before_sync();
+          sc = reinterpret_cast<const uint32_t *>(stg + 128 * PK * 16)[tid];
           __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&as_full[slot]);
+          if (lane == 0) sm100::mbar_arrive(&ke[ti % KS]);
         }
-        if (!ok) break;
-        // epilogue of this tile
-        if (!(ok = dwait(&dk_full[wg], ktw & 1, outer, &abort_s))) break;
-        sm100::fence_after_sync();
-        const uint32_t dka = tm + C_DK + wg * NACC * N;
-        uint32_t dm[N], dq[N];
-        if (N == 16) {
-          uint32_t t16[16];
-          sm100::tmem_ld16(sm100::tmem_lane(dka, wq), t16);
-          if (QJL) {
-            uint32_t q16[16];
-            sm100::tmem_ld16(sm100::tmem_lane(dka + N, wq), q16);
+        // epilogue of tile j - 2
+        if (j >= 2) {
+          if (j - 1 >= ntile && ok) ok = dwait(&kdone, (ti - 2) & 1, outer, &abort_s);
+          if (ok) {
+            sm100::fence_after_sync();
+            uint32_t dacc[NKO][16];
+#pragma unroll
+            for (int op = 0; op < NKO; ++op)
+              tmem_ldn<N>(sm100::tmem_lane(tm + C_DK + (((ti - 2) & 1) * NKO + op) * N, warp), dacc[op]);
             sm100::wait_ld();
+            const uint32_t scj = sc_hist[(ti - 2) & 1];
+            const int rl = (j - 2) * 128 + tid;
+            const bool valid = rl < nvalid;
+            const float nu = tq_half_to_f32(static_cast<uint16_t>(scj & 0xffffu));
+            const float rho = tq_half_to_f32(static_cast<uint16_t>(scj >> 16));
 #pragma unroll
-            for (int c = 0; c < 16; ++c) dq[c % N] = q16[c];
-          } else {
-            sm100::wait_ld();
-          }
-#pragma unroll
-          for (int c = 0; c < 16; ++c) dm[c % N] = t16[c];
-        } else {
-          uint32_t t8[8];
-          sm100::tmem_ld8(sm100::tmem_lane(dka, wq), t8);
-          if (QJL) {
-            uint32_t q8[8];
-            sm100::tmem_ld8(sm100::tmem_lane(dka + N, wq), q8);
-            sm100::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dq[c % N] = q8[c];
-          } else {
-            sm100::wait_ld();
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c) dm[c % N] = t8[c];
-        }
-        sm100::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&dk_empty[wg]);
-        const int rl = j * 128 + lt;
-        const bool valid = rl < nvalid;
-        const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
-        const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float dmv = comb_limbs(dm + 4 * h) * kcst[4 * h + 1] - kcst[4 * h + 0];
-          float est = dmv;
-          if (QJL) {
-            const float dj = comb_limbs(dq + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
-            est = fmaf(a.qjl_coef * rho, dj, dmv);
-          }
-          const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
-          lg[rl * G + h] = l;
-          mloc[h] = fmaxf(mloc[h], l);
-          if (a.logits && valid)
-            a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
-        }
-      }
-      kt += ntile;
-      // ---------------- S phase (8 warps)
-      if (ok) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float m = tq_warp_max(mloc[h]);
-          if (lane == 0) redf[warp][h] = m;
-        }
-        ok = sync8();
-      }
-      float mnew[G], corr[G], lsum[G], FV = 1.f, invFV = 1.f;
-      if (ok) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float m = redf[0][h];
-#pragma unroll
-          for (int w = 1; w < 8; ++w) m = fmaxf(m, redf[w][h]);
-          mnew[h] = fmaxf(m_run[h], m);
-          corr[h] = __expf(m_run[h] - mnew[h]);
-          lsum[h] = 0.f;
-        }
-        const uint16_t *vn = reinterpret_cast<const uint16_t *>(smem + L.o_vn + (u & 1) * UMAX * 2);
-        float numax = 0.f;
-        for (int rl = tid; rl < nvalid; rl += 256) {
-          numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float p = __expf(lg[rl * G + h] - mnew[h]);
-            lg[rl * G + h] = p;
-            lsum[h] += p;
+            for (int h = 0; h < G; ++h) {
+              float raw;
+              if constexpr (KDIG)
+                raw = fmaf(DIG_W0, comb_limbs(dacc[0] + 4 * h),
+                           fmaf(DIG_W1, comb_limbs(dacc[1] + 4 * h), comb_limbs(dacc[2] + 4 * h)));
+              else if constexpr (NT == 2)
+                raw = comb_limbs(dacc[0] + 4 * h) + comb_limbs(dacc[1] + 4 * h);
+              else
+                raw = comb_limbs(dacc[0] + 4 * h);
+              const float dmv = raw * kcst[4 * h + 1] - kcst[4 * h + 0];
+              float est = dmv;
+              if (QJL) {
+                const float dj = comb_limbs(dacc[NKO - 1] + 4 * h) * kcst[4 * h + 3] - kcst[4 * h + 2];
+                est = fmaf(a.qjl_coef * rho, dj, dmv);
+              }
+              const float l = valid ? a.scale * nu * est : -CUDART_INF_F;
+              lg[rl * G + h] = l;
+              mloc[h] = fmaxf(mloc[h], l);
+              if (a.logits && valid)
+                a.logits[(static_cast<int64_t>(b) * a.Hq + kvh * G + h) * a.max_len + cr0 + rl] = l;
+            }
           }
         }
-        ok = sync8();   // redf is free again; the weights are in place
-        if (ok) {
+        if (expand) {
+          // the MMAs of tile j - 1 have released the operand buffer
+          if (j >= 1 && ok) ok = dwait(&kdone, (ti - 1) & 1, outer, &abort_s);
+          if (ok) {
+            sm100::fence_after_sync();
+            const uint32_t abuf = sm100::tmem_lane(tm, warp);
+            // operand op, chunk w at columns 32 op + 8 w
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float sm = tq_warp_sum(lsum[h]);
-            if (lane == 0) redf[warp][h] = sm;
-          }
-          const float nm = tq_warp_max(numax);
-          if (lane == 0) redf[warp][2 * G] = nm;
-          if (tid < 8) wsum_s[tid] = 0ull;
-          ok = sync8();
-        }
-        if (ok) {
+            for (int w = 0; w < TNW; ++w) {
+              if constexpr (KDIG) {
+                uint32_t pl[MBK], dw[NDIG][8];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float sm = 0.f;
+                for (int p = 0; p < MBK; ++p) pl[p] = pw[p][w];
+                digit_words<MBK>(pl, ktab, dw);
 #pragma unroll
-            for (int w = 0; w < 8; ++w) sm += redf[w][h];
-            lsum[h] = sm;
-          }
-          float nmax = redf[0][2 * G];
+                for (int k = 0; k < NDIG; ++k) sm100::tmem_st8(abuf + 32 * k + 8 * w, dw[k]);
+              } else {
 #pragma unroll
-          for (int w = 1; w < 8; ++w) nmax = fmaxf(nmax, redf[w][2 * G]);
-          FV = pow2_scale(nmax);
-          invFV = 1.0f / (128.0f * FV);
-          // value-side B operand: element (n = 4h + l, k) of group g holds limb
-          // l of W(token) * 2^(7-r) for token 32g + 8nb + r, k = 4r + nb; one
-          // item = (group, r, head) makes the four consecutive k of one limb
-          // row and stores them as one 32-bit word; rows n >= 4G are zero
-          constexpr int NH = N / 4;
-          long long wpart = 0;
-          const int h = tid % NH;
-          for (int it = tid; it < ngroups * 8 * NH; it += 256) {
-            const int r = (it / NH) & 7, g = it / (8 * NH);
-            uint32_t word[4] = {0u, 0u, 0u, 0u};
-            if (h < G) {
-#pragma unroll
-              for (int nb = 0; nb < 4; ++nb) {
-                const int rl = 32 * g + 8 * nb + r;
-                int W = 0;
-                if (rl < nvalid) W = __float2int_rn(lg[rl * G + h] * tq_half_to_f32(vn[rl]) * FV);
-                wpart += W;
-                int v = W * (1 << (7 - r));
-#pragma unroll
-                for (int l = 0; l < 4; ++l) {
-                  const int8_t dgt = static_cast<int8_t>(v & 0xff);
-                  word[l] |= static_cast<uint32_t>(static_cast<uint8_t>(dgt)) << (8 * nb);
-                  v = (v - dgt) >> 8;
+                for (int t = 0; t < NT; ++t) {
+                  uint32_t r8[8];
+                  plane_words(pw[t][w], r8);
+                  sm100::tmem_st8(abuf + 32 * t + 8 * w, r8);
                 }
               }
             }
-            int8_t *dst = bvs + g * N * 32;
+            if (QJL) {
+              uint32_t r32[32];
 #pragma unroll
-            for (int l = 0; l < 4; ++l)
-              *reinterpret_cast<uint32_t *>(dst + kmajor_off(4 * h + l, 4 * r, N)) = word[l];
+              for (int w = 0; w < TNW; ++w) plane_words(pw[PK - 1][w], r32 + 8 * w);
+              sm100::tmem_st32(abuf + 32 * NT, r32);
+            }
+            sm100::wait_st();
           }
-          if (h < G) atomicAdd(&wsum_s[h], static_cast<unsigned long long>(wpart));
-          sm100::fence_async_smem();
-          ok = sync8();
-          if (ok && lane == 0) {
-            sm100::mbar_arrive(&bv_full);
-            sm100::mbar_arrive(&hdr_free[u & 1]);   // B operand and value norms no longer read
-          }
+          sc_hist[ti & 1] = sc;
         }
+        // tile j's operands are stored, D_k[j & 1] has been read: issue
+        if (!(ok = wg_sync(ok))) break;
+        if (expand && warp < NKO && lane == 0) {
+          const uint32_t acc = tm + C_DK + ((ti & 1) * NKO + warp) * N;
+#pragma unroll
+          for (int w = 0; w < TNW; ++w)
+            sm100::mma_i8_ts(acc, tm + 32 * warp + 8 * w,
+                             sm100::smem_desc(bk_addr + warp * 128 * N + w * 32 * N, N * 16, 128), IDESC,
+                             w > 0 ? 1u : 0u);
+          sm100::mma_commit(&kdone);
+        }
+        __syncwarp();
       }
       if (!ok) break;
+      kt += ntile;
+      // ---------------- S phase: softmax statistics and the value-side B operand
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float m = tq_warp_max(mloc[h]);
+        if (lane == 0) redf[warp][h] = m;
+      }
+      if (!(ok = wg_sync(ok))) break;
+      float mnew[G], corr[G], lsum[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float m = fmaxf(fmaxf(redf[0][h], redf[1][h]), fmaxf(redf[2][h], redf[3][h]));
+        mnew[h] = fmaxf(m_run[h], m);
+        corr[h] = __expf(m_run[h] - mnew[h]);
+        lsum[h] = 0.f;
+      }
+      const uint16_t *vn = reinterpret_cast<const uint16_t *>(smem + L.o_vn + (u & 1) * UMAX * 2);
+      float numax = 0.f;
+      for (int rl = tid; rl < nvalid; rl += 128) {
+        numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float p = __expf(lg[rl * G + h] - mnew[h]);
+          lg[rl * G + h] = p;
+          lsum[h] += p;
+        }
+      }
+      if (!(ok = wg_sync(ok))) break;   // redf is free again; the weights are in place
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float sm = tq_warp_sum(lsum[h]);
+        if (lane == 0) redf[warp][h] = sm;
+      }
+      {
+        const float nm = tq_warp_max(numax);
+        if (lane == 0) redf[warp][2 * G] = nm;
+      }
+      if (tid < G) wsum_s[tid] = 0ull;
+      if (!(ok = wg_sync(ok))) break;
+#pragma unroll
+      for (int h = 0; h < G; ++h) lsum[h] = redf[0][h] + redf[1][h] + redf[2][h] + redf[3][h];
+      const float FV = pow2_scale(fmaxf(fmaxf(redf[0][2 * G], redf[1][2 * G]),
+                                        fmaxf(redf[2][2 * G], redf[3][2 * G])));
+      {
+        // element (n = 4h + l, k = 4w + b) of group g's B operand holds limb l
+        // of W(token) for the token at byte b of A word w (times 2^(7-w) for
+        // bit planes); one item = (group, word, head) stores the 4 bytes of
+        // each limb row as one 32-bit word; rows n >= 4G are zero
+        long long wpart = 0;
+        const int h = tid % NH;
+        for (int it = tid; it < ngroups * 8 * NH; it += 128) {
+          const int w = (it / NH) & 7, g = it / (8 * NH);
+          uint32_t word[4] = {0u, 0u, 0u, 0u};
+          if (h < G) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int rl = 32 * g + elem_of(VDIG, 4 * w + e);
+              int W = 0;
+              if (rl < nvalid) W = __float2int_rn(lg[rl * G + h] * tq_half_to_f32(vn[rl]) * FV);
+              wpart += W;
+              int v = VDIG ? W : W * (1 << (7 - w));
+#pragma unroll
+              for (int l = 0; l < 4; ++l) {
+                const int8_t dgt = static_cast<int8_t>(v & 0xff);
+                word[l] |= static_cast<uint32_t>(static_cast<uint8_t>(dgt)) << (8 * e);
+                v = (v - dgt) >> 8;
+              }
+            }
+          }
+          int8_t *dst = bvs + g * N * 32;
+#pragma unroll
+          for (int l = 0; l < 4; ++l)
+            *reinterpret_cast<uint32_t *>(dst + kmajor_off(4 * h + l, 4 * w, N)) = word[l];
+        }
+        if (h < G) atomicAdd(&wsum_s[h], static_cast<unsigned long long>(wpart));
+      }
+      sm100::fence_async_smem();
+      if (!(ok = wg_sync(ok))) break;
+      if (tid == 0) sm100::mbar_arrive(&hdr_free[u & 1]);   // header no longer read
       float wtot[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -779,89 +823,85 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         l_run[h] = l_run[h] * corr[h] + lsum[h];
         m_run[h] = mnew[h];
       }
-      // ---------------- V phase: this group's value groups (lane = coordinate)
-      for (int g = wg; g < ngroups && ok; g += 2, ++vu) {
-        const uint32_t vgg = vg + g;
-        const int s = vgg % VS;
-        if (!(ok = dwait(&vf[s], (vgg / VS) & 1, outer, &abort_s))) break;
-        const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
-        uint32_t pw[BV];
+      // ---------------- V phase: batches of VB groups (lane = coordinate)
+      const int nbat = (ngroups + VB - 1) / VB;
+      for (int bi = 0; bi < nbat; ++bi) {
+        const uint32_t vbi = vb + bi;
+        const uint32_t abuf = sm100::tmem_lane(tm + (vbi & 1) * VA, warp);
+        // the buffer's previous batch (vbi - 2) has been multiplied
+        if (vbi >= 2 && ok) ok = dwait(&vdone[vbi & 1], ((vbi >> 1) - 1) & 1, outer, &abort_s);
+        if (ok) sm100::fence_after_sync();
 #pragma unroll
-        for (int p = 0; p < BV; ++p) pw[p] = vc[p * TD + lt];
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&ve[s]);
-        if (vu >= 1 && !(ok = dwait(&av_empty[wg], (vu - 1) & 1, outer, &abort_s))) break;
-        sm100::fence_after_sync();
+        for (int gi = 0; gi < VB; ++gi) {
+          const int g = bi * VB + gi;
+          if (g >= ngroups) break;
+          const uint32_t vgg = vg + g;
+          const int s = vgg % VS;
+          if (ok) ok = dwait(&vf[s], (vgg / VS) & 1, outer, &abort_s);
+          if (ok) {
+            const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
+            uint32_t pv[BV];
 #pragma unroll
-        for (int h4 = 0; h4 < (TV + 3) / 4; ++h4) {
-          uint32_t r32[32];
+            for (int p = 0; p < BV; ++p) pv[p] = vc[p * TD + tid];
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&ve[s]);
+            if constexpr (VDIG) {
+              uint32_t dw[NDIG][8];
+              digit_words<BV>(pv, vtab, dw);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int ti = 4 * h4 + q;
-            uint32_t x = 0;
-            if (ti < TV) {
-              const int mask = odd_mask(BV, ti);
+              for (int k = 0; k < NDIG; ++k) sm100::tmem_st8(abuf + gi * NV * 8 + 8 * k, dw[k]);
+            } else {
 #pragma unroll
-              for (int p = 0; p < BV; ++p)
-                if ((mask >> p) & 1) x ^= pw[p];
-            }
-#pragma unroll
-            for (int r = 0; r < 8; ++r) r32[q * 8 + r] = x & (0x01010101u << r);
-          }
-          if (TV >= 4) {
-            sm100::tmem_st32(sm100::tmem_lane(tm + wg * TV * 8 + h4 * 32, wq), r32);
-          } else {
-            uint32_t r8[8];
-#pragma unroll
-            for (int q = 0; q < TV; ++q) {
-#pragma unroll
-              for (int r = 0; r < 8; ++r) r8[r] = r32[q * 8 + r];
-              sm100::tmem_st8(sm100::tmem_lane(tm + wg * TV * 8 + q * 8, wq), r8);
+              for (int t = 0; t < NV; ++t) {
+                uint32_t r8[8];
+                plane_words(pv[t], r8);
+                sm100::tmem_st8(abuf + gi * NV * 8 + 8 * t, r8);
+              }
             }
           }
         }
         sm100::wait_st();
-        sm100::fence_before_sync();
+        if (!(ok = wg_sync(ok))) break;
+        if (warp < NV && lane == 0) {
+          // warp op issues accumulator D_v[op] (its first group starts it)
+          const uint32_t acc = tm + C_DV + warp * N;
+#pragma unroll
+          for (int gi = 0; gi < VB; ++gi) {
+            const int g = bi * VB + gi;
+            if (g < ngroups)
+              sm100::mma_i8_ts(acc, tm + (vbi & 1) * VA + gi * NV * 8 + warp * 8,
+                               sm100::smem_desc(bv_addr + g * N * 32, N * 16, 128), IDESC, g > 0 ? 1u : 0u);
+          }
+          sm100::mma_commit(&vdone[vbi & 1]);
+        }
         __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&av_full[wg]);
       }
+      if (!ok) break;
+      vb += nbat;
       vg += ngroups;
       // ---------------- E phase: all value MMAs of the unit have landed
-      if (ok) ok = dwait(&dv_full, u & 1, outer, &abort_s);
-      if (ok && wg == 0) {
+      ok = dwait(&vdone[(vb - 1) & 1], ((vb - 1) >> 1) & 1, outer, &abort_s);
+      if (ok) {
         sm100::fence_after_sync();
+        uint32_t dv[NV][16];
+#pragma unroll
+        for (int op = 0; op < NV; ++op) tmem_ldn<N>(sm100::tmem_lane(tm + C_DV + op * N, warp), dv[op]);
+        sm100::wait_ld();
         float acc[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = 0.f;
+        for (int h = 0; h < G; ++h) {
+          acc[h] = 0.f;
 #pragma unroll
-        for (int ti = 0; ti < TV; ++ti) {
-          uint32_t dv[N];
-          if (N == 16) {
-            uint32_t t0[16];
-            sm100::tmem_ld16(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-            sm100::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) dv[c % N] = t0[c];
-          } else {
-            uint32_t t0[8];
-            sm100::tmem_ld8(sm100::tmem_lane(tm + C_DV + ti * N, wq), t0);
-            sm100::wait_ld();
-#pragma unroll
-            for (int c = 0; c < 8; ++c) dv[c % N] = t0[c];
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] = fmaf(2.f * a.wv[ti], comb_limbs(dv + 4 * h), acc[h]);
+          for (int op = 0; op < NV; ++op) acc[h] = fmaf(a.vcoef[op], comb_limbs(dv[op] + 4 * h), acc[h]);
         }
-        sm100::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&tm_free);
+        const float ivs = 1.0f / FV;
 #pragma unroll
-        for (int h = 0; h < G; ++h) o[h] += acc[h] * invFV - a.wv_sum * wtot[h];
+        for (int h = 0; h < G; ++h) o[h] += acc[h] * ivs - a.vbias * wtot[h];
         if (cr0 + a.sub >= c1) {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const int64_t hq = static_cast<int64_t>(b) * a.Hq + kvh * G + h;
-            a.po[(hq * a.splits + sp) * TD + lt] = o[h];
+            a.po[(hq * a.splits + sp) * TD + tid] = o[h];
             if (tid == 0) {
               a.pml[(hq * a.splits + sp) * 2] = m_run[h];
               a.pml[(hq * a.splits + sp) * 2 + 1] = l_run[h];
@@ -869,11 +909,16 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
           }
         }
       }
-      if (!ok) break;
       cr0 += a.sub;
       have = tc_next(a, cit, cr0);
       ++u;
     }
+    // every MMA this thread issued has landed before tensor memory is freed
+    if (lane == 0) {
+      sm100::mma_commit(&fin[warp]);
+      sm100::mbar_wait(&fin[warp], 0, 1u << 20);
+    }
+    __syncwarp();
   }
   sm100::fence_before_sync();
   __syncthreads();
@@ -896,10 +941,9 @@ constexpr TcCfg kTcConfigs[] = {{4, 3, 4, 1}, {4, 1, 2, 1}, {4, 2, 3, 1}, {2, 3,
 
 template <int G, int MBK, int BV, bool QJL>
 int run_dec(TcArgs &a, cudaStream_t stream) {
-  constexpr int TK = 1 << (MBK - 1);
   constexpr int N = tc_n(G);
   constexpr int PK = MBK + (QJL ? 1 : 0);
-  constexpr int BKC = N * (TK * TD + (QJL ? TD : 0)) + G * 16;
+  constexpr int BKC = N * TD * (n_ops(MBK) + (QJL ? 1 : 0)) + G * 16;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -943,8 +987,7 @@ bool tc_supported(const tq_codec *c, int G) {
 }
 
 int tc_bk_stride(const tq_codec *c, int G) {
-  const int TK = 1 << (c->mse_bits_k - 1);
-  const int bytes = tc_n(G) * (TK * TD + (c->qjl_k ? TD : 0)) + G * 16;
+  const int bytes = tc_n(G) * TD * (n_ops(c->mse_bits_k) + (c->qjl_k ? 1 : 0)) + G * 16;
   return (bytes + 127) & ~127;
 }
 
@@ -981,12 +1024,27 @@ int launch_decode_tc(const tq_codec *c, const void *q, int dtype, int B, int Hq,
   a.po = po;
   a.pml = pml;
   a.logits = logits;
-  for (int i = 0; i < 8; ++i) {
-    a.wk[i] = c->walsh_k[i];
-    a.wv[i] = c->walsh_v[i];
-  }
+  for (int i = 0; i < 8; ++i) a.wk[i] = c->walsh_k[i];
   a.wk_absmax = c->walsh_k_absmax;
-  a.wv_sum = c->walsh_v_sum;
+  for (int d = 0; d < 3; ++d)
+    for (int i = 0; i < 4; ++i) {
+      a.ktab[d][i] = c->digit_k[d][i];
+      a.vtab[d][i] = c->digit_v[d][i];
+    }
+  a.kfc = c->digit_k_scale;
+  if (use_digits(c->bits_v)) {
+    // value = sum_tokens W (V - 2^20) / F_c with V = 2^14 d0 + 2^7 d1 + d2
+    a.vcoef[0] = 16384.0f / c->digit_v_scale;
+    a.vcoef[1] = 128.0f / c->digit_v_scale;
+    a.vcoef[2] = 1.0f / c->digit_v_scale;
+    a.vbias = 1048576.0f / c->digit_v_scale;
+  } else {
+    // value = sum_t a_t (2 x_t - 1); the planes' B carries an extra 2^7
+    a.vcoef[0] = c->walsh_v[0] / 64.0f;
+    a.vcoef[1] = c->walsh_v[1] / 64.0f;
+    a.vcoef[2] = 0.f;
+    a.vbias = c->walsh_v_sum;
+  }
   a.err = err;
   a.wait_limit = 1u << 26;
   if (const char *e = getenv("TQ_WAIT_LIMIT")) a.wait_limit = static_cast<uint32_t>(strtoul(e, nullptr, 10));

@@ -41,6 +41,11 @@ struct tq_codec {
   // over the odd subsets of the code bits (tensor-core decode path)
   float walsh_k[8], walsh_v[8];
   float walsh_k_absmax, walsh_v_sum;
+  // 3- and 4-bit codebooks on that path: centroids c_i ~ (V_i - 2^20) / scale
+  // as three 7-bit digits of V_i (weights 2^14, 2^7, 1), entries packed four
+  // per word
+  uint32_t digit_k[3][4], digit_v[3][4];
+  float digit_k_scale, digit_v_scale;
   int device;
 };
 

@@ -33,10 +33,13 @@ struct TcArgs {
   float *po;            // [B][Hq][splits][128]
   float *pml;           // [B][Hq][splits][2]
   float *logits;        // optional [B][Hq][max_len]
-  float wk[8];          // key Walsh coefficients a_S
+  float wk[8];          // key Walsh coefficients a_S (1- and 2-bit key codebooks)
   float wk_absmax;
-  float wv[8];          // value Walsh coefficients
-  float wv_sum;
+  uint32_t ktab[3][4];  // key centroid digits (3- and 4-bit key codebooks)
+  float kfc;            // their fixed-point scale
+  uint32_t vtab[3][4];  // value centroid digits (3- and 4-bit value codebooks)
+  float vcoef[3];       // value: weight of each operand's accumulator
+  float vbias;          // value: constant per unit of softmax weight
   uint32_t *err;        // optional device flag set when a bounded wait gives up
   uint32_t wait_limit;  // polls before a wait gives up (TQ_WAIT_LIMIT overrides, for tests)
   TqBooks books;
