@@ -344,6 +344,7 @@ __device__ __forceinline__ bool tc_next(const TcArgs &a, int &it, int &r0) {
 // runs out or another warp has given up.
 __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, uint32_t outer,
                                       volatile int *abort_flag) {
+#pragma unroll 1
   for (uint32_t it = 0; it < outer; ++it) {
     const bool ok = sm100::mbar_wait(bar, parity, 1u << 8);
     if (__all_sync(TQ_FULL, ok)) return true;
@@ -356,6 +357,7 @@ __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, uint32_t o
 // Single-thread bounded wait for the copying lanes.
 __device__ __forceinline__ bool dwait1(uint64_t *bar, uint32_t parity, uint32_t outer,
                                        volatile int *abort_flag) {
+#pragma unroll 1
   for (uint32_t it = 0; it < outer; ++it) {
     if (sm100::mbar_wait(bar, parity, 1u << 8)) return true;
     if (*abort_flag) return false;
@@ -378,6 +380,16 @@ __device__ __forceinline__ bool wg_sync(bool ok) {
       : "memory");
   sm100::fence_after_sync();
   return bad == 0u;
+}
+
+// x[i] for a runtime i without indexing the register array (x[0] when i is
+// out of range).
+template <int K>
+__device__ __forceinline__ float pick(const float (&x)[K], int i) {
+  float v = x[0];
+#pragma unroll
+  for (int k = 1; k < K; ++k) v = i == k ? x[k] : v;
+  return v;
 }
 
 // N accumulator columns of this warp's lanes (N = 8 or 16), loads in flight.
@@ -466,8 +478,9 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
   __shared__ __align__(8) uint64_t kdone, vdone[2], fin[4];
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
-  __shared__ float redf[4][2 * G + 1];
-  __shared__ unsigned long long wsum_s[G];
+  __shared__ float redf[4][G + 1];
+  __shared__ float redl[4][4];
+  __shared__ long long redw[4][4];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t outer = a.wait_limit >> 8;
@@ -738,54 +751,39 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
       if (!ok) break;
       kt += ntile;
       // ---------------- S phase: softmax statistics and the value-side B operand
+      const uint16_t *vn = reinterpret_cast<const uint16_t *>(smem + L.o_vn + (u & 1) * UMAX * 2);
+      {
+        // the unit's largest logit of each head and largest value norm
+        float numax = 0.f;
+        for (int rl = tid; rl < nvalid; rl += 128) numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float m = tq_warp_max(mloc[h]);
-        if (lane == 0) redf[warp][h] = m;
+        for (int h = 0; h < G; ++h) {
+          const float m = tq_warp_max(mloc[h]);
+          if (lane == 0) redf[warp][h] = m;
+        }
+        const float nm = tq_warp_max(numax);
+        if (lane == 0) redf[warp][G] = nm;
       }
       if (!(ok = wg_sync(ok))) break;
-      float mnew[G], corr[G], lsum[G];
+      float mnew[G], corr[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float m = fmaxf(fmaxf(redf[0][h], redf[1][h]), fmaxf(redf[2][h], redf[3][h]));
         mnew[h] = fmaxf(m_run[h], m);
         corr[h] = __expf(m_run[h] - mnew[h]);
-        lsum[h] = 0.f;
       }
-      const uint16_t *vn = reinterpret_cast<const uint16_t *>(smem + L.o_vn + (u & 1) * UMAX * 2);
-      float numax = 0.f;
-      for (int rl = tid; rl < nvalid; rl += 128) {
-        numax = fmaxf(numax, tq_half_to_f32(vn[rl]));
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float p = __expf(lg[rl * G + h] - mnew[h]);
-          lg[rl * G + h] = p;
-          lsum[h] += p;
-        }
-      }
-      if (!(ok = wg_sync(ok))) break;   // redf is free again; the weights are in place
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float sm = tq_warp_sum(lsum[h]);
-        if (lane == 0) redf[warp][h] = sm;
-      }
-      {
-        const float nm = tq_warp_max(numax);
-        if (lane == 0) redf[warp][2 * G] = nm;
-      }
-      if (tid < G) wsum_s[tid] = 0ull;
-      if (!(ok = wg_sync(ok))) break;
-#pragma unroll
-      for (int h = 0; h < G; ++h) lsum[h] = redf[0][h] + redf[1][h] + redf[2][h] + redf[3][h];
-      const float FV = pow2_scale(fmaxf(fmaxf(redf[0][2 * G], redf[1][2 * G]),
-                                        fmaxf(redf[2][2 * G], redf[3][2 * G])));
+      const float FV = pow2_scale(fmaxf(fmaxf(redf[0][G], redf[1][G]), fmaxf(redf[2][G], redf[3][G])));
       {
         // element (n = 4h + l, k = 4w + b) of group g's B operand holds limb l
-        // of W(token) for the token at byte b of A word w (times 2^(7-w) for
-        // bit planes); one item = (group, word, head) stores the 4 bytes of
-        // each limb row as one 32-bit word; rows n >= 4G are zero
-        long long wpart = 0;
+        // of W = round(p nu_v FV), p = exp(l - m_new), for the token at byte b
+        // of A word w (times 2^(7-w) for bit planes); one item = (group, word,
+        // head) makes the 4 bytes of each limb row, stored as one 32-bit word;
+        // rows n >= 4G are zero.  Every (token, head) weight is made once, so
+        // the softmax sums are taken here too.
         const int h = tid % NH;
+        const float mh = pick(mnew, h);
+        float lpart = 0.f;
+        long long wpart = 0;
         for (int it = tid; it < ngroups * 8 * NH; it += 128) {
           const int w = (it / NH) & 7, g = it / (8 * NH);
           uint32_t word[4] = {0u, 0u, 0u, 0u};
@@ -794,7 +792,11 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
             for (int e = 0; e < 4; ++e) {
               const int rl = 32 * g + elem_of(VDIG, 4 * w + e);
               int W = 0;
-              if (rl < nvalid) W = __float2int_rn(lg[rl * G + h] * tq_half_to_f32(vn[rl]) * FV);
+              if (rl < nvalid) {
+                const float p = __expf(lg[rl * G + h] - mh);
+                lpart += p;
+                W = __float2int_rn(p * tq_half_to_f32(vn[rl]) * FV);
+              }
               wpart += W;
               int v = VDIG ? W : W * (1 << (7 - w));
 #pragma unroll
@@ -810,7 +812,16 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
           for (int l = 0; l < 4; ++l)
             *reinterpret_cast<uint32_t *>(dst + kmajor_off(4 * h + l, 4 * w, N)) = word[l];
         }
-        if (h < G) atomicAdd(&wsum_s[h], static_cast<unsigned long long>(wpart));
+        // sums over the lanes of this warp that share head h
+#pragma unroll
+        for (int o = NH; o < 32; o <<= 1) {
+          lpart += __shfl_xor_sync(TQ_FULL, lpart, o);
+          wpart += __shfl_xor_sync(TQ_FULL, wpart, o);
+        }
+        if (lane < NH) {
+          redl[warp][lane] = lpart;
+          redw[warp][lane] = wpart;
+        }
       }
       sm100::fence_async_smem();
       if (!(ok = wg_sync(ok))) break;
@@ -818,9 +829,10 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
       float wtot[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        wtot[h] = static_cast<float>(static_cast<long long>(wsum_s[h])) / FV;
+        const float lsum = redl[0][h] + redl[1][h] + redl[2][h] + redl[3][h];
+        wtot[h] = static_cast<float>(redw[0][h] + redw[1][h] + redw[2][h] + redw[3][h]) / FV;
         o[h] *= corr[h];
-        l_run[h] = l_run[h] * corr[h] + lsum[h];
+        l_run[h] = l_run[h] * corr[h] + lsum;
         m_run[h] = mnew[h];
       }
       // ---------------- V phase: batches of VB groups (lane = coordinate)

@@ -49,6 +49,7 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 // Bounded wait for the phase with the given parity; false after `limit` polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = 1u << 26) {
   const uint32_t a = smem_addr(bar);
+#pragma unroll 1
   for (uint32_t it = 0; it < limit; ++it) {
     uint32_t ok;
     asm volatile(
