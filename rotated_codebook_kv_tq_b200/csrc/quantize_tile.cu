@@ -98,19 +98,64 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
   return false;
 }
 
+// Packed fp32 pair arithmetic (sm_100): each half rounds exactly like the
+// scalar instruction.
+__device__ __forceinline__ void addsub2(float &a0, float &a1, float &b0, float &b1) {
+  // (a, b) <- (a + b, a - b) for both halves of the pairs (a0, a1), (b0, b1)
+  asm("{\n\t.reg .b64 p, q, s, d;\n\t"
+      "mov.b64 p, {%0, %1};\n\tmov.b64 q, {%2, %3};\n\t"
+      "add.rn.f32x2 s, p, q;\n\tsub.rn.f32x2 d, p, q;\n\t"
+      "mov.b64 {%0, %1}, s;\n\tmov.b64 {%2, %3}, d;\n\t}\n"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+// (a, b) packed into one 64-bit register.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// (d0, d1) = (a0, a1) - c
+__device__ __forceinline__ void sub2c(float a0, float a1, uint64_t c, float &d0, float &d1) {
+  asm("{\n\t.reg .b64 p, d;\n\tmov.b64 p, {%2, %3};\n\tsub.rn.f32x2 d, p, %4;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "l"(c));
+}
+
+// acc += (a0 * a0, a1 * a1)
+__device__ __forceinline__ void sq2acc(float a0, float a1, uint64_t &acc) {
+  asm("{\n\t.reg .b64 p;\n\tmov.b64 p, {%1, %2};\n\tfma.rn.f32x2 %0, p, p, %0;\n\t}\n"
+      : "+l"(acc)
+      : "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ float hsum2(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
+
 // In-register Walsh-Hadamard transform, Sylvester natural order: y = H_D x.
+// Stages of stride s < D/2 pair element i with i + D/2 (the same butterfly
+// in both halves) and run on packed pairs; the stride-D/2 stage is scalar.
+// Same stage order and operations as the plain radix-2 loop.
 template <int D>
 __device__ __forceinline__ void wht_regs(float (&x)[D]) {
+  constexpr int H = D / 2;
 #pragma unroll
-  for (int s = 1; s < D; s <<= 1) {
+  for (int s = 1; s < H; s <<= 1) {
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
-      if (!(i & s)) {
-        const float a = x[i], b = x[i + s];
-        x[i] = a + b;
-        x[i + s] = a - b;
-      }
+    for (int i = 0; i < H; ++i) {
+      if (!(i & s)) addsub2(x[i], x[i + H], x[i + s], x[i + s + H]);
     }
+  }
+#pragma unroll
+  for (int i = 0; i < H; ++i) {
+    const float a = x[i], b = x[i + H];
+    x[i] = a + b;
+    x[i + H] = a - b;
   }
 }
 
@@ -136,6 +181,42 @@ __device__ __forceinline__ void plane_msbs(float y, const float *th, uint32_t (&
     w[2] = s[3] ^ sy;
     w[1] = s[1] ^ s[3] ^ s[5] ^ sy;
     w[0] = s[0] ^ s[1] ^ s[2] ^ s[3] ^ s[4] ^ s[5] ^ s[6] ^ sy;
+  }
+}
+
+// plane_msbs for two coordinates at once, the threshold differences taken as
+// packed pairs (th2[j] = (th[j], th[j])).
+template <int NB>
+__device__ __forceinline__ void plane_msbs2(float y0, float y1, const uint64_t *th2, uint32_t (&w0)[4],
+                                            uint32_t (&w1)[4]) {
+  constexpr int NT = (1 << (NB - 1)) - 1;   // thresholds above 0
+  const float a0 = fabsf(y0), a1 = fabsf(y1);
+  uint32_t s0[NT > 0 ? NT : 1], s1[NT > 0 ? NT : 1];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    float d0, d1;
+    sub2c(a0, a1, th2[j], d0, d1);
+    s0[j] = __float_as_uint(d0);
+    s1[j] = __float_as_uint(d1);
+  }
+  const uint32_t sy0 = __float_as_uint(y0), sy1 = __float_as_uint(y1);
+  w0[NB - 1] = sy0;
+  w1[NB - 1] = sy1;
+  if (NB == 2) {
+    w0[0] = s0[0] ^ sy0;
+    w1[0] = s1[0] ^ sy1;
+  } else if (NB == 3) {
+    w0[1] = s0[1] ^ sy0;
+    w0[0] = s0[0] ^ s0[1] ^ s0[2] ^ sy0;
+    w1[1] = s1[1] ^ sy1;
+    w1[0] = s1[0] ^ s1[1] ^ s1[2] ^ sy1;
+  } else if (NB == 4) {
+    w0[2] = s0[3] ^ sy0;
+    w0[1] = s0[1] ^ s0[3] ^ s0[5] ^ sy0;
+    w0[0] = s0[0] ^ s0[1] ^ s0[2] ^ s0[3] ^ s0[4] ^ s0[5] ^ s0[6] ^ sy0;
+    w1[2] = s1[3] ^ sy1;
+    w1[1] = s1[1] ^ s1[3] ^ s1[5] ^ sy1;
+    w1[0] = s1[0] ^ s1[1] ^ s1[2] ^ s1[3] ^ s1[4] ^ s1[5] ^ s1[6] ^ sy1;
   }
 }
 
@@ -313,9 +394,10 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&empty);
       // ---- norm, sign flip, transform
-      float ss = 0.f;
+      uint64_t ss2 = 0ull;
 #pragma unroll
-      for (int j = 0; j < D; ++j) ss = fmaf(x[j], x[j], ss);
+      for (int j = 0; j < D / 2; ++j) sq2acc(x[j], x[j + D / 2], ss2);
+      const float ss = hsum2(ss2);
       float nu = sqrtf(ss);
       bool bad = !(ss <= 3.402823466e38f) || isinf(__half2float(__float2half_rn(nu)));
       if (bad) nu = 0.f;
@@ -338,26 +420,38 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
         for (int p = 0; p < PK; ++p)
 #pragma unroll
           for (int w = 0; w < NW; ++w) pw[p][w] = 0u;
-        float r2 = 0.f;
+        uint64_t r2p = 0ull;
         float cks[HK];
 #pragma unroll
         for (int m = 0; m < HK; ++m) cks[m] = a.ck[m] * sc;
+        uint64_t th2[HK > 1 ? HK - 1 : 1];
 #pragma unroll
-        for (int j = D - 1; j >= 0; --j) {
-          uint32_t ms[4];
-          plane_msbs<MBK>(x[j], thr, ms);
+        for (int j = 0; j < HK - 1; ++j) th2[j] = pk2(thr[j], thr[j]);
+        // coordinates j and j + D/2 together (their words take the same bit)
 #pragma unroll
-          for (int p = 0; p < MBK; ++p) pw[p][j >> 5] = __funnelshift_l(ms[p], pw[p][j >> 5], 1);
+        for (int j = D / 2 - 1; j >= 0; --j) {
+          constexpr int H2 = D / 2;
+          uint32_t ms0[4], ms1[4];
+          plane_msbs2<MBK>(x[j], x[j + H2], th2, ms0, ms1);
+#pragma unroll
+          for (int p = 0; p < MBK; ++p) {
+            pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
+            pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
+          }
           if (QJL) {
-            const float aa = fabsf(x[j]);
-            float cm = cks[0];
+            const float aa0 = fabsf(x[j]), aa1 = fabsf(x[j + H2]);
+            float cm0 = cks[0], cm1 = cks[0];
 #pragma unroll
-            for (int m = 1; m < HK; ++m) cm = aa >= thr[m - 1] ? cks[m] : cm;
-            const float cval = x[j] >= 0.f ? cm : -cm;
-            x[j] = x[j] - cval;            // residual (scaled by sc)
-            r2 = fmaf(x[j], x[j], r2);
+            for (int m = 1; m < HK; ++m) {
+              cm0 = aa0 >= thr[m - 1] ? cks[m] : cm0;
+              cm1 = aa1 >= thr[m - 1] ? cks[m] : cm1;
+            }
+            const float cv0 = x[j] >= 0.f ? cm0 : -cm0, cv1 = x[j + H2] >= 0.f ? cm1 : -cm1;
+            sub2c(x[j], x[j + H2], pk2(cv0, cv1), x[j], x[j + H2]);   // residual (scaled by sc)
+            sq2acc(x[j], x[j + H2], r2p);
           }
         }
+        const float r2 = hsum2(r2p);
         // funnel shifts accumulated coordinate 32 w + 31 first: bit i = coord 32 w + i
 #pragma unroll
         for (int p = 0; p < MBK; ++p)
@@ -433,12 +527,19 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
         for (int p = 0; p < BV; ++p)
 #pragma unroll
           for (int w = 0; w < NW; ++w) pw[p][w] = 0u;
+        uint64_t th2[HV > 1 ? HV - 1 : 1];
 #pragma unroll
-        for (int j = D - 1; j >= 0; --j) {
-          uint32_t ms[4];
-          plane_msbs<BV>(x[j], thr, ms);
+        for (int j = 0; j < HV - 1; ++j) th2[j] = pk2(thr[j], thr[j]);
 #pragma unroll
-          for (int p = 0; p < BV; ++p) pw[p][j >> 5] = __funnelshift_l(ms[p], pw[p][j >> 5], 1);
+        for (int j = D / 2 - 1; j >= 0; --j) {
+          constexpr int H2 = D / 2;
+          uint32_t ms0[4], ms1[4];
+          plane_msbs2<BV>(x[j], x[j + H2], th2, ms0, ms1);
+#pragma unroll
+          for (int p = 0; p < BV; ++p) {
+            pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
+            pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
+          }
         }
         const int64_t crow = bh * a.rows_cap + R;
         if (active) a.vnorm[crow] = tq_f32_to_half(nu);
