@@ -521,17 +521,9 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         const int c0 = sp * a.chunk, c1 = min(tc_len(a, b), c0 + a.chunk);
         const int nvalid = min(a.sub, c1 - cr0);
         const int ntile = (nvalid + 127) / 128, ngroups = (nvalid + 31) / 32;
-        // unit header: B operand, constants and value norms (buffer u & 1),
-        // once unit u - 2 has finished its softmax phase with that buffer
-        {
-          const int hb = u & 1;
-          if (u >= 2 && !dwait1(&hdr_free[hb], ((u >> 1) - 1) & 1, outer, &abort_s)) break;
-          const uint32_t nvn = static_cast<uint32_t>(ngroups) * 64;
-          sm100::mbar_expect_tx(&hdr[hb], static_cast<uint32_t>((BKC + 15) & ~15) + nvn);
-          sm100::bulk_g2s(smem + L.o_bk + hb * L.bkc, a.bk + bh * a.bk_stride, (BKC + 15) & ~15, &hdr[hb]);
-          sm100::bulk_g2s(smem + L.o_vn + hb * UMAX * 2, a.vnorm + bh * a.rows_cap + cr0, nvn, &hdr[hb]);
-          lh[hb] = static_cast<uint8_t>(1 + ((u >> 1) & 1));
-        }
+        // key tiles; the unit header (B operand, constants and value norms,
+        // buffer u & 1, once unit u - 2 has finished its softmax phase with
+        // it) follows the first tile, whose data has the longer way to come
         for (int j = 0; j < ntile && !abort_s; ++j, ++kt) {
           const int s = kt % KS;
           if (kt >= KS && !dwait1(&ke[s], ((kt / KS) - 1) & 1, outer, &abort_s)) break;
@@ -542,6 +534,15 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
           sm100::bulk_g2s(st, a.kcode + (bh * a.rows_cap + row) * PK * 16, nrow * PK * 16, &kf[s]);
           sm100::bulk_g2s(st + 128 * PK * 16, a.kscale + (bh * a.rows_cap + row) * 2, nrow * 4, &kf[s]);
           lk[s] = static_cast<uint8_t>(1 + ((kt / KS) & 1));
+          if (j == 0) {
+            const int hb = u & 1;
+            if (u >= 2 && !dwait1(&hdr_free[hb], ((u >> 1) - 1) & 1, outer, &abort_s)) break;
+            const uint32_t nvn = static_cast<uint32_t>(ngroups) * 64;
+            sm100::mbar_expect_tx(&hdr[hb], static_cast<uint32_t>((BKC + 15) & ~15) + nvn);
+            sm100::bulk_g2s(smem + L.o_bk + hb * L.bkc, a.bk + bh * a.bk_stride, (BKC + 15) & ~15, &hdr[hb]);
+            sm100::bulk_g2s(smem + L.o_vn + hb * UMAX * 2, a.vnorm + bh * a.rows_cap + cr0, nvn, &hdr[hb]);
+            lh[hb] = static_cast<uint8_t>(1 + ((u >> 1) & 1));
+          }
         }
         cr0 += a.sub;
         have = tc_next(a, cit, cr0);

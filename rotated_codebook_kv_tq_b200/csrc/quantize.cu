@@ -274,6 +274,18 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
   for (int p = 0; p < 4; ++p)
 #pragma unroll
     for (int k = 0; k < NPL; ++k) vw[p][k] = 0u;
+  // a partial group keeps its other rows: their words are read now, so the
+  // load overlaps the rows' pipeline instead of trailing it
+  const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
+  const uint32_t vmask = nrows >= 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
+  uint32_t *vgw = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
+  uint32_t vold[4][NPL];
+  if (warp == 1 && vmask != TQ_FULL) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) vold[p][k] = p < a.books.bits_v ? vgw[p * D + lane + 32 * k] : 0u;
+  }
 
   for (int64_t r = r_begin; r < r_end; ++r) {
     const int64_t t = r - a.row0;
@@ -361,17 +373,14 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
     __syncthreads();   // rsm and sgw are reused by the next row
   }
   if (warp == 1) {
-    // the group's value words (read-modify-write for partial groups; this
-    // block is the only writer of the group within the call)
-    const uint32_t nrows = static_cast<uint32_t>(r_end - r_begin);
-    const uint32_t mask = nrows == 32 ? TQ_FULL : (((1u << nrows) - 1u) << (r_begin & 31));
-    uint32_t *vg = a.vcode + (cache_bh * (a.rows_cap / 32) + g) * a.books.bits_v * D;
-    for (int p = 0; p < a.books.bits_v; ++p) {
+    // the group's value words (partial groups merge the words read above;
+    // this block is the only writer of the group within the call)
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) {
-        uint32_t *w = vg + p * D + lane + 32 * k;
-        *w = mask == TQ_FULL ? vw[p][k] : ((*w & ~mask) | (vw[p][k] & mask));
-      }
+    for (int p = 0; p < 4; ++p) {
+      if (p >= a.books.bits_v) break;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k)
+        vgw[p * D + lane + 32 * k] = vmask == TQ_FULL ? vw[p][k] : ((vold[p][k] & ~vmask) | (vw[p][k] & vmask));
     }
   }
 }
