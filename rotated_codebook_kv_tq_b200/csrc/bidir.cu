@@ -129,55 +129,63 @@ __device__ __forceinline__ void split3_store(uint8_t *base, uint32_t stride, int
   *reinterpret_cast<__nv_bfloat16 *>(base + 2 * stride + off) = c;
 }
 
-// Eight consecutive K elements (k0 a multiple of 8) of one row: the three
-// split planes are each one 16-byte core-matrix row, stored with one write.
-__device__ __forceinline__ void split3_store8(uint8_t *base, uint32_t stride, int off, const float (&v)[8]) {
-  uint32_t w0[4], w1[4], w2[4];
+// v = p0 + p1 in bf16 (|error| < 2^-17 |v|), planes at base and base + stride.
+__device__ __forceinline__ void split2_store8(uint8_t *base, uint32_t stride, int off, const float (&v)[8]) {
+  uint32_t w0[4], w1[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    uint32_t p0[2], p1[2], p2[2];
+    uint32_t p0[2], p1[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const float x = v[2 * e + h];
-      const __nv_bfloat16 a = __float2bfloat16_rn(x);
-      const float r1 = x - __bfloat162float(a);
-      const __nv_bfloat16 b = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 c = __float2bfloat16_rn(r1 - __bfloat162float(b));
-      p0[h] = __bfloat16_as_ushort(a);
-      p1[h] = __bfloat16_as_ushort(b);
-      p2[h] = __bfloat16_as_ushort(c);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      p0[h] = __bfloat16_as_ushort(hi);
+      p1[h] = __bfloat16_as_ushort(lo);
     }
     w0[e] = p0[0] | (p0[1] << 16);
     w1[e] = p1[0] | (p1[1] << 16);
-    w2[e] = p2[0] | (p2[1] << 16);
   }
   *reinterpret_cast<uint4 *>(base + off) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
   *reinterpret_cast<uint4 *>(base + stride + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-  *reinterpret_cast<uint4 *>(base + 2 * stride + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
 }
 
-// The six split products of order <= 2: a0 b0 + a0 b1 + a1 b0 + a0 b2 + a1 b1 + a2 b0
-// (about 2^-26 relative).  The five small ones go first into d_small; the
-// K steps of a0 b0 go round-robin into `nbig` accumulators d_big + i * dstride
-// (nbig = 1 folds everything into d_small, for the P V product).
-__device__ __forceinline__ void mma6(uint32_t d_small, uint32_t d_big, uint32_t dstride, int nbig,
-                                     uint32_t a, uint32_t astr, uint32_t b, uint32_t bstr,
-                                     int ksteps, uint32_t lbo_a, uint32_t lbo_b, uint32_t idesc,
-                                     bool acc_first) {
-  const int pa[6] = {2, 1, 0, 1, 0, 0}, pb[6] = {0, 1, 2, 0, 1, 0};
-  int n = 0;
-#pragma unroll
-  for (int t = 0; t < 5; ++t)
-    for (int s = 0; s < ksteps; ++s, ++n)
-      sm100::mma_bf16_ss(d_small, sm100::smem_desc(a + pa[t] * astr + s * 2 * lbo_a, lbo_a, 128),
-                         sm100::smem_desc(b + pb[t] * bstr + s * 2 * lbo_b, lbo_b, 128), idesc,
-                         (n > 0 || acc_first) ? 1u : 0u);
-  for (int s = 0; s < ksteps; ++s) {
-    const uint32_t d = nbig > 1 ? d_big + (s % nbig) * dstride : d_small;
-    sm100::mma_bf16_ss(d, sm100::smem_desc(a + s * 2 * lbo_a, lbo_a, 128),
-                       sm100::smem_desc(b + s * 2 * lbo_b, lbo_b, 128), idesc,
-                       nbig > 1 ? (s >= nbig ? 1u : 0u) : 1u);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+  return d;
+}
+
+// bf16 entries i0 and i1 (< 2^nbits <= 16) of a table packed two per word,
+// returned as one packed pair (i0 in the low half): byte permutes pick from
+// four entries at a time, bits 2 and 3 of the index select between them.
+__device__ __forceinline__ uint32_t lut2(const uint32_t *t, uint32_t i0, uint32_t i1, int nbits) {
+  const uint32_t sel = (0x22u * (i0 & 3u) + 0x10u) | ((0x22u * (i1 & 3u) + 0x10u) << 8);
+  uint32_t r = prmt(t[0], t[1], sel);
+  if (nbits > 2) {
+    const uint32_t m2 = ((i0 & 4u) ? 0xffffu : 0u) | ((i1 & 4u) ? 0xffff0000u : 0u);
+    r = (prmt(t[2], t[3], sel) & m2) | (r & ~m2);
+    if (nbits > 3) {
+      uint32_t r8 = prmt(t[4], t[5], sel);
+      r8 = (prmt(t[6], t[7], sel) & m2) | (r8 & ~m2);
+      const uint32_t m3 = ((i0 & 8u) ? 0xffffu : 0u) | ((i1 & 8u) ? 0xffff0000u : 0u);
+      r = (r8 & m3) | (r & ~m3);
+    }
   }
+  return r;
+}
+
+// Codes of elements `bit` and `bit + 1` from nb plane words.
+__device__ __forceinline__ void code_pair(const uint32_t (&pw)[4], int nb, int bit, uint32_t &i0, uint32_t &i1) {
+  i0 = 0u;
+  i1 = 0u;
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    if (p < nb) {
+      const uint32_t x = (pw[p] >> bit) & 3u;
+      i0 |= (x & 1u) << p;
+      i1 |= (x >> 1) << p;
+    }
 }
 
 template <int D>
@@ -190,16 +198,22 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   constexpr uint32_t IDESC_S = sm100::idesc_bf16(128, BK);
   constexpr uint32_t IDESC_O = sm100::idesc_bf16(128, D);
   constexpr int NPL = D / 32;
+  constexpr uint32_t STG = 4608;                   // one stage of compressed rows
   extern __shared__ __align__(128) float smem_b[];
-  // each operand is stored as three bf16 planes (split3_store)
+  // each operand is stored as bf16 split planes (three, two for P)
   uint8_t *qs3 = reinterpret_cast<uint8_t *>(smem_b);
   uint8_t *ks3 = qs3 + 3 * Q_BYTES;
   uint8_t *ps3 = ks3 + 3 * K_BYTES;
-  uint8_t *vs3 = ps3 + 3 * P_BYTES;
+  uint8_t *vs3 = ps3 + 2 * P_BYTES;
   float *nuk = reinterpret_cast<float *>(vs3 + 3 * V_BYTES);  // [BK]
-  __shared__ float cks[TQ_MAX_LEVELS], cvs[TQ_MAX_LEVELS];
+  // two stages of one key tile's compressed rows, copied a tile ahead:
+  // key planes, (nu, rho), the two value groups' words, value norms
+  uint8_t *stg0 = reinterpret_cast<uint8_t *>(nuk + BK);
+  // the three bf16 split planes of every key and value centroid, two entries
+  // per word: K_rot's MSE half and V_rot are table lookups
+  __shared__ __align__(16) uint16_t tabk[3][8], tabv[3][16];
   __shared__ float vns[BK];   // value norms of the current key tile
-  __shared__ __align__(8) uint64_t mb;
+  __shared__ __align__(8) uint64_t mbS, mbO, fin[4], kvf[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
@@ -209,13 +223,31 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
   const int q0 = qt * BQ;
   const int mbk = a.books.mse_bits_k, planes_k = mbk + a.books.qjl, nbv = a.books.bits_v;
-  if (tid < TQ_MAX_LEVELS) {
-    cks[tid] = a.books.ck[tid];
-    cvs[tid] = a.books.cv[tid];
+  if (tid < 16) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const float v = w == 0 ? (tid < 8 && tid < (1 << mbk) ? a.books.ck[tid] : 0.f)
+                             : (tid < (1 << nbv) ? a.books.cv[tid] : 0.f);
+      const __nv_bfloat16 p0 = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(p0);
+      const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+      uint16_t *t = w == 0 ? &tabk[0][0] : &tabv[0][0];
+      const int ne = w == 0 ? 8 : 16;
+      if (w == 1 || tid < 8) {
+        t[0 * ne + tid] = __bfloat16_as_ushort(p0);
+        t[1 * ne + tid] = __bfloat16_as_ushort(p1);
+        t[2 * ne + tid] = __bfloat16_as_ushort(p2);
+      }
+    }
   }
   if (warp == 0) sm100::tmem_alloc(&tmem_s, 512);
   if (tid == 0) {
-    sm100::mbar_init(&mb, 1);
+    sm100::mbar_init(&mbS, 4);
+    sm100::mbar_init(&mbO, 2);
+    for (int i = 0; i < 4; ++i) sm100::mbar_init(&fin[i], 1);
+    sm100::mbar_init(&kvf[0], 1);
+    sm100::mbar_init(&kvf[1], 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -229,32 +261,80 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
-  // columns: S small-product accumulator, four hi*hi accumulators, O
-  constexpr int NBIG = 4;
-  const uint32_t tm = tmem_s, tS = tm, tSb = tm + BK, tO = tm + (1 + NBIG) * BK;
+  // columns: three small-product S accumulators, two for the leading hi*hi
+  // product, two O accumulators (warps 0-3 issue S, warps 0-1 issue O, each
+  // lane 0 into its own accumulators, so the MMAs are issued in parallel and
+  // no accumulator takes a chain longer than 16)
+  constexpr int NBIG = 2;
+  const uint32_t tm = tmem_s;
+  const uint32_t tS0 = tm, tSb = tm + BK, tO = tm + 3 * BK, tS1 = tm + 4 * BK, tS2 = tm + 5 * BK,
+                 tO2 = tm + 6 * BK;
   const uint32_t a_q = sm100::smem_addr(qs3), a_k = sm100::smem_addr(ks3);
   const uint32_t a_p = sm100::smem_addr(ps3), a_v = sm100::smem_addr(vs3);
+
+  // stage layout (bytes): key planes [0, 2048), (nu, rho) [2048, 2304),
+  // value words [2304, 4352), value norms [4352, 4480)
+  auto issue_tile = [&](int jt) {
+    const int j0 = jt * BK;
+    uint8_t *st = stg0 + (jt & 1) * STG;
+    const uint32_t n = static_cast<uint32_t>(min(static_cast<int64_t>(BK), a.rows_cap - j0));
+    const uint32_t ng = n / 32;
+    const uint32_t bk_ = n * planes_k * (D / 8), bs = n * 4, bv = ng * nbv * D * 4, bn = n * 2;
+    sm100::mbar_expect_tx(&kvf[jt & 1], bk_ + bs + bv + bn);
+    sm100::bulk_g2s(st, a.kcode + (bh * a.rows_cap + j0) * planes_k * (D / 8), bk_, &kvf[jt & 1]);
+    sm100::bulk_g2s(st + 2048, a.kscale + (bh * a.rows_cap + j0) * 2, bs, &kvf[jt & 1]);
+    sm100::bulk_g2s(st + 2304, a.vcode + (bh * (a.rows_cap / 32) + j0 / 32) * nbv * D, bv, &kvf[jt & 1]);
+    sm100::bulk_g2s(st + 4352, a.vnorm + bh * a.rows_cap + j0, bn, &kvf[jt & 1]);
+  };
+  const int ntiles = (a.T + BK - 1) / BK;
+  if (tid == 0 && ntiles > 0) issue_tile(0);
+  int issued = 0;   // tiles whose copies were issued (thread 0)
 
   float m = -CUDART_INF_F, l = 0.f;
   uint32_t phase = 0;
   for (int j0 = 0; j0 < a.T; j0 += BK) {
+    const int jt = j0 / BK;
+    // the next tile's rows stream in while this one is worked on (its stage
+    // was last read two tiles ago)
+    if (tid == 0 && jt + 1 < ntiles) {
+      issue_tile(jt + 1);
+      issued = jt + 2;
+    } else if (tid == 0 && issued < jt + 1) {
+      issued = jt + 1;
+    }
+    if (!sm100::mbar_wait(&kvf[jt & 1], (jt >> 1) & 1)) abort_s = 1;
+    __syncthreads();
+    if (abort_s) break;
+    const uint8_t *st = stg0 + (jt & 1) * STG;
     // ---- key tile: thread (row tid % BK, half tid / BK) writes the MSE half
     // (c[idx]) or the sign half (+-coef rho) of one key row; value tile:
     // thread (coordinate tid % D, key group tid / D) writes 32 keys of V_rot^T.
     static_assert(BQ == 2 * BK && BQ == 2 * D && BK == 64, "thread mapping");
     if (tid < BK)
-      vns[tid] = j0 + tid < a.T ? tq_half_to_f32(a.vnorm[bh * a.rows_cap + j0 + tid]) : 0.f;
+      vns[tid] = j0 + tid < a.T ? tq_half_to_f32(reinterpret_cast<const uint16_t *>(st + 4352)[tid]) : 0.f;
     __syncthreads();
     {
       const int row = tid % BK, half = tid / BK;
       const int j = j0 + row;
       const bool ok = j < a.T;
-      const uint8_t *krow = a.kcode + (bh * a.rows_cap + (ok ? j : 0)) * planes_k * (D / 8);
-      const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale)[bh * a.rows_cap + (ok ? j : 0)];
+      const uint8_t *krow = st + row * planes_k * (D / 8);
+      const uint32_t sc = ok ? reinterpret_cast<const uint32_t *>(st + 2048)[row] : 0u;
       const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
       const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
       if (half == 0) nuk[row] = ok ? nu : 0.f;
       const float qv = a.qjl_coef * rho;
+      // the sign half is +-qv: its split, negated where the sign bit is 0
+      uint32_t pos[3];
+      {
+        const __nv_bfloat16 p0 = __float2bfloat16_rn(qv);
+        const float r1 = qv - __bfloat162float(p0);
+        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+        const uint32_t u[3] = {__bfloat16_as_ushort(p0), __bfloat16_as_ushort(p1), __bfloat16_as_ushort(p2)};
+#pragma unroll
+        for (int p = 0; p < 3; ++p) pos[p] = (ok && a.books.qjl) ? (u[p] | (u[p] << 16)) : 0u;
+      }
+      const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
 #pragma unroll 1
       for (int w = 0; w < D / 32; ++w) {
         uint32_t pw[4] = {0u, 0u, 0u, 0u};
@@ -267,105 +347,128 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
           if (p == mbk) sgn = pw[p];
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
-          float v[8];
+          uint32_t o[3][4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int bit = 8 * c8 + e;
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int bit = 8 * c8 + 2 * e2;
             if (half == 0) {
-              int idx = 0;
+              uint32_t i0, i1;
+              code_pair(pw, mbk, bit, i0, i1);
 #pragma unroll
-              for (int p = 0; p < 3; ++p)
-                if (p < mbk) idx |= ((pw[p] >> bit) & 1) << p;
-              v[e] = ok ? cks[idx] : 0.f;
+              for (int p = 0; p < 3; ++p) o[p][e2] = ok ? lut2(tk32 + 4 * p, i0, i1, mbk) : 0u;
             } else {
-              v[e] = (ok && a.books.qjl) ? (((sgn >> bit) & 1) ? qv : -qv) : 0.f;
+              const uint32_t sb = ~(sgn >> bit);
+              const uint32_t neg = ((sb & 1u) << 15) | ((sb & 2u) << 30);
+#pragma unroll
+              for (int p = 0; p < 3; ++p) o[p][e2] = pos[p] ^ (pos[p] ? neg : 0u);
             }
           }
-          split3_store8(ks3, K_BYTES, kmaj16(row, half * D + 32 * w + 8 * c8, BK), v);
+          const int off = kmaj16(row, half * D + 32 * w + 8 * c8, BK);
+#pragma unroll
+          for (int p = 0; p < 3; ++p)
+            *reinterpret_cast<uint4 *>(ks3 + p * K_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
         }
       }
     }
     {
+      // V_rot^T: centroids only (the value norms scale P instead); thread
+      // (coordinate tid % D, key group tid / D) writes 32 keys
       const int coord = tid % D, g = tid / D;
-      {
-        const int jg = j0 + 32 * g;
-        uint32_t vw[4] = {0u, 0u, 0u, 0u};
-        if (jg < a.T)
-          for (int p = 0; p < nbv; ++p)
-            vw[p] = a.vcode[(bh * (a.rows_cap / 32) + jg / 32) * nbv * D + p * D + coord];
+      const int jg = j0 + 32 * g;
+      uint32_t vw[4] = {0u, 0u, 0u, 0u};
+      if (jg < a.T)
+        for (int p = 0; p < nbv; ++p)
+          vw[p] = reinterpret_cast<const uint32_t *>(st + 2304)[(g * nbv + p) * D + coord];
+      const uint32_t *tv32 = reinterpret_cast<const uint32_t *>(&tabv[0][0]);
 #pragma unroll
-        for (int t8 = 0; t8 < 4; ++t8) {
-          float v[8];
+      for (int t8 = 0; t8 < 4; ++t8) {
+        uint32_t o[3][4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int t = 8 * t8 + e;
-            int idx = 0;
+        for (int e2 = 0; e2 < 4; ++e2) {
+          uint32_t i0, i1;
+          code_pair(vw, nbv, 8 * t8 + 2 * e2, i0, i1);
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
-              if (p < nbv) idx |= ((vw[p] >> t) & 1) << p;
-            v[e] = jg + t < a.T ? vns[32 * g + t] * cvs[idx] : 0.f;
-          }
-          split3_store8(vs3, V_BYTES, kmaj16(coord, 32 * g + 8 * t8, D), v);
+          for (int p = 0; p < 3; ++p) o[p][e2] = lut2(tv32 + 8 * p, i0, i1, nbv);
         }
+        const int off = kmaj16(coord, 32 * g + 8 * t8, D);
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          *reinterpret_cast<uint4 *>(vs3 + p * V_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
       }
     }
     sm100::fence_async_smem();
     sm100::fence_before_sync();
     __syncthreads();
     sm100::fence_after_sync();
-    // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d)
-    if (tid == 0) {
-      mma6(tS, tSb, BK, NBIG, a_q, Q_BYTES, a_k, K_BYTES, DP / 16, BQ * 16, BK * 16, IDESC_S, false);
-      sm100::mma_commit(&mb);
+    // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d): the six
+    // split products of order <= 2 (about 2^-26 relative); warp 0 issues
+    // a2 b0 + a1 b1, warp 1 a0 b2 + a1 b0, warp 2 a0 b1, warp 3 the K steps
+    // of a0 b0 alternating over two accumulators
+    if ((tid & 31) == 0) {
+      constexpr uint32_t LA = BQ * 16, LB = BK * 16;
+      if (warp < 3) {
+        const int pa[5] = {2, 1, 0, 1, 0}, pb[5] = {0, 1, 2, 0, 1};
+        const int t0 = 2 * warp, nt = warp == 2 ? 1 : 2;
+        const uint32_t d = warp == 0 ? tS0 : warp == 1 ? tS1 : tS2;
+        int n = 0;
+        for (int t = t0; t < t0 + nt; ++t)
+#pragma unroll
+          for (int st = 0; st < DP / 16; ++st, ++n)
+            sm100::mma_bf16_ss(d, sm100::smem_desc(a_q + pa[t] * Q_BYTES + st * 2 * LA, LA, 128),
+                               sm100::smem_desc(a_k + pb[t] * K_BYTES + st * 2 * LB, LB, 128), IDESC_S,
+                               n > 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int st = 0; st < DP / 16; ++st)
+          sm100::mma_bf16_ss(tSb + (st % NBIG) * BK, sm100::smem_desc(a_q + st * 2 * LA, LA, 128),
+                             sm100::smem_desc(a_k + st * 2 * LB, LB, 128), IDESC_S, st >= NBIG ? 1u : 0u);
+      }
+      sm100::mma_commit(&mbS);
     }
-    if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
-    phase ^= 1;
+    if (!sm100::mbar_wait(&mbS, phase)) abort_s = 1;
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
-    // scores of 16 keys (c .. c+15) of this query row from the five accumulators
-    auto scores16 = [&](int c, float (&v)[16]) {
-      uint32_t r[16];
-      sm100::tmem_ld16(sm100::tmem_lane(tS + c, warp), r);
+    // the 64 scores of this query row: the five S accumulators added in fp32
+    float sv[BK];
+#pragma unroll
+    for (int c = 0; c < BK; c += 32) {
+      uint32_t r[32];
+      sm100::tmem_ld32(sm100::tmem_lane(tS0 + c, warp), r);
       sm100::wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 32; ++e) sv[c + e] = __uint_as_float(r[e]);
+      const uint32_t others[4] = {tS1, tS2, tSb, tSb + BK};
 #pragma unroll
-      for (int i = 0; i < NBIG; ++i) {
-        sm100::tmem_ld16(sm100::tmem_lane(tSb + i * BK + c, warp), r);
+      for (int i = 0; i < 4; ++i) {
+        sm100::tmem_ld32(sm100::tmem_lane(others[i] + c, warp), r);
         sm100::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] += __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) sv[c + e] += __uint_as_float(r[e]);
       }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = j0 + c + e < a.T ? a.scale * nuk[c + e] * v[e] : -CUDART_INF_F;
-    };
-    // pass 1: the tile's maximum; pass 2: probabilities into the P planes
+    }
     float tmax = -CUDART_INF_F;
-#pragma unroll 1
-    for (int c = 0; c < BK; c += 16) {
-      float v[16];
-      scores16(c, v);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) tmax = fmaxf(tmax, v[e]);
+    for (int c = 0; c < BK; ++c) {
+      sv[c] = j0 + c < a.T ? a.scale * nuk[c] * sv[c] : -CUDART_INF_F;
+      tmax = fmaxf(tmax, sv[c]);
     }
     const float mn = fmaxf(m, tmax);
     const float corr = __expf(m - mn);
+    // P nu_v (the value norms of the keys, so V_rot holds centroids only),
+    // as a two-term bf16 split: its 2^-17 error reaches the output directly,
+    // not through the softmax
     float ps = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < BK; c += 16) {
-      float v[16];
-      scores16(c, v);
 #pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
-        float w[8];
+    for (int c = 0; c < BK; c += 8) {
+      float w[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          w[e] = __expf(v[8 * h8 + e] - mn);
-          ps += w[e];
-        }
-        split3_store8(ps3, P_BYTES, kmaj16(tid, c + 8 * h8, BQ), w);
+      for (int e = 0; e < 8; ++e) {
+        const float pe = __expf(sv[c + e] - mn);
+        ps += pe;
+        w[e] = pe * vns[c + e];
       }
+      split2_store8(ps3, P_BYTES, kmaj16(tid, c, BQ), w);
     }
     l = l * corr + ps;
     m = mn;
@@ -373,26 +476,40 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     // when some row's maximum moved, before the P V MMAs add this tile
     if (j0 > 0 && __any_sync(TQ_FULL, corr != 1.f)) {
 #pragma unroll
-      for (int c = 0; c < D; c += 8) {
-        uint32_t r[8];
-        sm100::tmem_ld8(sm100::tmem_lane(tO + c, warp), r);
-        sm100::wait_ld();
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
-        sm100::tmem_st8(sm100::tmem_lane(tO + c, warp), r);
-      }
+        for (int c = 0; c < D; c += 32) {
+          const uint32_t t = (i ? tO2 : tO) + c;
+          uint32_t r[32];
+          sm100::tmem_ld32(sm100::tmem_lane(t, warp), r);
+          sm100::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+          sm100::tmem_st32(sm100::tmem_lane(t, warp), r);
+        }
       sm100::wait_st();
     }
     sm100::fence_async_smem();
     sm100::fence_before_sync();
     __syncthreads();
     sm100::fence_after_sync();
-    // ---- O_tile = P V_rot (M = 128 queries, N = d, K = 64 keys)
-    if (tid == 0) {
-      mma6(tO, tO, 0, 1, a_p, P_BYTES, a_v, V_BYTES, BK / 16, BQ * 16, D * 16, IDESC_O, j0 > 0);
-      sm100::mma_commit(&mb);
+    // ---- O_tile = (P nu) V_rot (M = 128 queries, N = d, K = 64 keys): the
+    // five products of a two-term P and a three-term V of order <= 2: warp 0
+    // issues a1 b0 + a1 b1 + a0 b2 into O, warp 1 a0 b1 + a0 b0 into O2
+    if ((tid & 31) == 0 && warp < 2) {
+      constexpr uint32_t LA = BQ * 16, LB = D * 16;
+      const int pa[5] = {1, 1, 0, 0, 0}, pb[5] = {0, 1, 2, 1, 0};
+      const uint32_t d = warp == 0 ? tO : tO2;
+      int n = 0;
+      for (int t = 3 * warp; t < (warp == 0 ? 3 : 5); ++t)
+#pragma unroll
+        for (int st = 0; st < BK / 16; ++st, ++n)
+          sm100::mma_bf16_ss(d, sm100::smem_desc(a_p + pa[t] * P_BYTES + st * 2 * LA, LA, 128),
+                             sm100::smem_desc(a_v + pb[t] * V_BYTES + st * 2 * LB, LB, 128), IDESC_O,
+                             (n > 0 || j0 > 0) ? 1u : 0u);
+      sm100::mma_commit(&mbO);
     }
-    if (!sm100::mbar_wait(&mb, phase)) abort_s = 1;
+    if (!sm100::mbar_wait(&mbO, phase)) abort_s = 1;
     phase ^= 1;
     __syncthreads();
     if (abort_s) break;
@@ -401,11 +518,12 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   float o[D];
 #pragma unroll
   for (int c = 0; c < D; c += 16) {
-    uint32_t r[16];
+    uint32_t r[16], r2[16];
     sm100::tmem_ld16(sm100::tmem_lane(tO + c, warp), r);
+    sm100::tmem_ld16(sm100::tmem_lane(tO2 + c, warp), r2);
     sm100::wait_ld();
 #pragma unroll
-    for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r[e]);
+    for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r[e]) + __uint_as_float(r2[e]);
   }
   // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l)
   if (!abort_s && q0 + tid < a.Lq) {
@@ -426,10 +544,15 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
       dst[i] = o[i] * sgn * f;
     }
   }
-  if (abort_s) {
-    sm100::mbar_wait(&mb, phase, 1u << 20);
-    if (tid == 0 && a.err) atomicExch(a.err, 1u);
+  // this CTA's copies have landed before its shared memory is released: the
+  // last issued tile's phase completes (at once if it was consumed)
+  if (tid == 0 && issued > 0) sm100::mbar_wait(&kvf[(issued - 1) & 1], ((issued - 1) >> 1) & 1, 1u << 20);
+  // every MMA this thread issued has landed before tensor memory is released
+  if ((tid & 31) == 0) {
+    sm100::mma_commit(&fin[warp]);
+    sm100::mbar_wait(&fin[warp], 0, 1u << 20);
   }
+  if (abort_s && tid == 0 && a.err) atomicExch(a.err, 1u);
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
@@ -481,8 +604,8 @@ int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int 
   const int64_t qb = (nq + 7) / 8;
   bidir_qprep_kernel<D><<<static_cast<int>(qb < 8LL * sms ? qb : 8LL * sms), 256, qshm, stream>>>(a);
   if (int e = tq_check_launch("bidir_qprep_kernel")) return e;
-  constexpr size_t shm = 3 * (BQ * 2 * D * 2) + 3 * (BK * 2 * D * 2) + 3 * (BQ * BK * 2) +
-                         3 * (D * BK * 2) + BK * 4;
+  constexpr size_t shm = 3 * (BQ * 2 * D * 2) + 3 * (BK * 2 * D * 2) + 2 * (BQ * BK * 2) +
+                         3 * (D * BK * 2) + BK * 4 + 2 * 4608;
   static bool done[64] = {};
   if (dev < 64 && !done[dev]) {
     if (cudaFuncSetAttribute(bidir_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
