@@ -34,6 +34,7 @@ namespace {
 
 constexpr int BQ = 128;   // queries per CTA
 constexpr int BK = 64;    // keys per tile
+constexpr int BT = 256;   // threads of the tile kernel: two per query row
 
 struct BidirArgs {
   const void *q;
@@ -189,16 +190,16 @@ __device__ __forceinline__ void code_pair(const uint32_t (&pw)[4], int nb, int b
 }
 
 template <int D>
-__global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
+__global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   constexpr int DP = 2 * D;                        // rotated-domain width of Q/K
-  constexpr uint32_t Q_BYTES = BQ * DP * 2;        // one of hi / lo
+  constexpr uint32_t Q_BYTES = BQ * DP * 2;        // one split plane
   constexpr uint32_t K_BYTES = BK * DP * 2;
   constexpr uint32_t P_BYTES = BQ * BK * 2;
   constexpr uint32_t V_BYTES = D * BK * 2;
   constexpr uint32_t IDESC_S = sm100::idesc_bf16(128, BK);
   constexpr uint32_t IDESC_O = sm100::idesc_bf16(128, D);
-  constexpr int NPL = D / 32;
   constexpr uint32_t STG = 4608;                   // one stage of compressed rows
+  static_assert(BT == 2 * BQ && BQ == 2 * BK && D == BK && BK == 64, "thread mapping");
   extern __shared__ __align__(128) float smem_b[];
   // each operand is stored as bf16 split planes (three, two for P)
   uint8_t *qs3 = reinterpret_cast<uint8_t *>(smem_b);
@@ -212,12 +213,15 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   // the three bf16 split planes of every key and value centroid, two entries
   // per word: K_rot's MSE half and V_rot are table lookups
   __shared__ __align__(16) uint16_t tabk[3][8], tabv[3][16];
-  __shared__ float vns[BK];   // value norms of the current key tile
+  __shared__ float vns[BK];        // value norms of the current key tile
+  __shared__ float xmax[2][BQ];    // the two halves' tile maxima of each query row
+  __shared__ float lsum_s[BQ];
   __shared__ __align__(8) uint64_t mbS, mbO, fin[4], kvf[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = tid & (BQ - 1), hf = tid >> 7;   // query row (TMEM lane), half of its keys / columns
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / (a.H / a.Hkv);
   const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
@@ -251,11 +255,12 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // query tile: row tid = query q0 + tid (rows past Lq are zero)
+  // query tile: row r = query q0 + r (rows past Lq are zero), columns of half hf
   {
-    const int qi = q0 + tid;
+    const int qi = q0 + r;
     const float *src = a.qrot + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + qi) * DP;
-    for (int k = 0; k < DP; ++k) split3_store(qs3, Q_BYTES, kmaj16(tid, k, BQ), qi < a.Lq ? src[k] : 0.f);
+    for (int k = hf * D; k < hf * D + D; ++k)
+      split3_store(qs3, Q_BYTES, kmaj16(r, k, BQ), qi < a.Lq ? src[k] : 0.f);
   }
   sm100::fence_async_smem();
   sm100::fence_before_sync();
@@ -271,6 +276,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
                  tO2 = tm + 6 * BK;
   const uint32_t a_q = sm100::smem_addr(qs3), a_k = sm100::smem_addr(ks3);
   const uint32_t a_p = sm100::smem_addr(ps3), a_v = sm100::smem_addr(vs3);
+  const int lq = warp & 3;    // this warp's TMEM lane quarter
 
   // stage layout (bytes): key planes [0, 2048), (nu, rho) [2048, 2304),
   // value words [2304, 4352), value norms [4352, 4480)
@@ -288,44 +294,47 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   };
   const int ntiles = (a.T + BK - 1) / BK;
   if (tid == 0 && ntiles > 0) issue_tile(0);
-  int issued = 0;   // tiles whose copies were issued (thread 0)
+  int issued = ntiles > 0 ? 1 : 0;   // tiles whose copies were issued (thread 0)
 
-  float m = -CUDART_INF_F, l = 0.f;
+  float m = -CUDART_INF_F, l = 0.f;   // l: this half's share of the row sum
   uint32_t phase = 0;
-  for (int j0 = 0; j0 < a.T; j0 += BK) {
-    const int jt = j0 / BK;
+  for (int jt = 0; jt < ntiles; ++jt) {
+    const int j0 = jt * BK;
     // the next tile's rows stream in while this one is worked on (its stage
     // was last read two tiles ago)
     if (tid == 0 && jt + 1 < ntiles) {
       issue_tile(jt + 1);
       issued = jt + 2;
-    } else if (tid == 0 && issued < jt + 1) {
-      issued = jt + 1;
     }
     if (!sm100::mbar_wait(&kvf[jt & 1], (jt >> 1) & 1)) abort_s = 1;
     __syncthreads();
     if (abort_s) break;
     const uint8_t *st = stg0 + (jt & 1) * STG;
-    // ---- key tile: thread (row tid % BK, half tid / BK) writes the MSE half
-    // (c[idx]) or the sign half (+-coef rho) of one key row; value tile:
-    // thread (coordinate tid % D, key group tid / D) writes 32 keys of V_rot^T.
-    static_assert(BQ == 2 * BK && BQ == 2 * D && BK == 64, "thread mapping");
     if (tid < BK)
       vns[tid] = j0 + tid < a.T ? tq_half_to_f32(reinterpret_cast<const uint16_t *>(st + 4352)[tid]) : 0.f;
-    __syncthreads();
+    // ---- key tile: thread (row tid % BK, part tid / BK) writes 32 columns of
+    // one key row: part 0-1 the MSE half (c[idx]), part 2-3 the sign half
+    // (+-coef rho); value tile: thread (coordinate tid % D, group and half of
+    // tid / D) writes 16 keys of V_rot^T
     {
-      const int row = tid % BK, half = tid / BK;
+      const int row = tid % BK, part = tid / BK;
+      const int half = part >> 1, w = part & 1;
       const int j = j0 + row;
       const bool ok = j < a.T;
-      const uint8_t *krow = st + row * planes_k * (D / 8);
+      const uint32_t *krow = reinterpret_cast<const uint32_t *>(st + row * planes_k * (D / 8));
       const uint32_t sc = ok ? reinterpret_cast<const uint32_t *>(st + 2048)[row] : 0u;
       const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
       const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-      if (half == 0) nuk[row] = ok ? nu : 0.f;
-      const float qv = a.qjl_coef * rho;
-      // the sign half is +-qv: its split, negated where the sign bit is 0
-      uint32_t pos[3];
-      {
+      if (part == 0) nuk[row] = ok ? nu : 0.f;
+      uint32_t pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        if (p < planes_k) pw[p] = krow[p * (D / 32) + w];
+      uint32_t pos[3] = {0u, 0u, 0u};
+      uint32_t sgn = 0u;
+      if (half == 1) {
+        // the sign half is +-qv: its split, negated where the sign bit is 0
+        const float qv = a.qjl_coef * rho;
         const __nv_bfloat16 p0 = __float2bfloat16_rn(qv);
         const float r1 = qv - __bfloat162float(p0);
         const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
@@ -333,47 +342,38 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
         const uint32_t u[3] = {__bfloat16_as_ushort(p0), __bfloat16_as_ushort(p1), __bfloat16_as_ushort(p2)};
 #pragma unroll
         for (int p = 0; p < 3; ++p) pos[p] = (ok && a.books.qjl) ? (u[p] | (u[p] << 16)) : 0u;
-      }
-      const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
-#pragma unroll 1
-      for (int w = 0; w < D / 32; ++w) {
-        uint32_t pw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          if (p < planes_k) pw[p] = reinterpret_cast<const uint32_t *>(krow)[p * (D / 32) + w];
-        uint32_t sgn = 0u;
 #pragma unroll
         for (int p = 0; p < 4; ++p)
           if (p == mbk) sgn = pw[p];
+      }
+      const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t o[3][4];
+      for (int c8 = 0; c8 < 4; ++c8) {
+        uint32_t o[3][4];
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const int bit = 8 * c8 + 2 * e2;
-            if (half == 0) {
-              uint32_t i0, i1;
-              code_pair(pw, mbk, bit, i0, i1);
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int bit = 8 * c8 + 2 * e2;
+          if (half == 0) {
+            uint32_t i0, i1;
+            code_pair(pw, mbk, bit, i0, i1);
 #pragma unroll
-              for (int p = 0; p < 3; ++p) o[p][e2] = ok ? lut2(tk32 + 4 * p, i0, i1, mbk) : 0u;
-            } else {
-              const uint32_t sb = ~(sgn >> bit);
-              const uint32_t neg = ((sb & 1u) << 15) | ((sb & 2u) << 30);
+            for (int p = 0; p < 3; ++p) o[p][e2] = ok ? lut2(tk32 + 4 * p, i0, i1, mbk) : 0u;
+          } else {
+            const uint32_t sb = ~(sgn >> bit);
+            const uint32_t neg = ((sb & 1u) << 15) | ((sb & 2u) << 30);
 #pragma unroll
-              for (int p = 0; p < 3; ++p) o[p][e2] = pos[p] ^ (pos[p] ? neg : 0u);
-            }
+            for (int p = 0; p < 3; ++p) o[p][e2] = pos[p] ^ (pos[p] ? neg : 0u);
           }
-          const int off = kmaj16(row, half * D + 32 * w + 8 * c8, BK);
-#pragma unroll
-          for (int p = 0; p < 3; ++p)
-            *reinterpret_cast<uint4 *>(ks3 + p * K_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
         }
+        const int off = kmaj16(row, half * D + 32 * w + 8 * c8, BK);
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+          *reinterpret_cast<uint4 *>(ks3 + p * K_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
       }
     }
     {
-      // V_rot^T: centroids only (the value norms scale P instead); thread
-      // (coordinate tid % D, key group tid / D) writes 32 keys
-      const int coord = tid % D, g = tid / D;
+      // V_rot^T: centroids only (the value norms scale P instead)
+      const int coord = tid % D, g = (tid / D) & 1, th = tid / (2 * D);
       const int jg = j0 + 32 * g;
       uint32_t vw[4] = {0u, 0u, 0u, 0u};
       if (jg < a.T)
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
           vw[p] = reinterpret_cast<const uint32_t *>(st + 2304)[(g * nbv + p) * D + coord];
       const uint32_t *tv32 = reinterpret_cast<const uint32_t *>(&tabv[0][0]);
 #pragma unroll
-      for (int t8 = 0; t8 < 4; ++t8) {
+      for (int t8 = 2 * th; t8 < 2 * th + 2; ++t8) {
         uint32_t o[3][4];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     // split products of order <= 2 (about 2^-26 relative); warp 0 issues
     // a2 b0 + a1 b1, warp 1 a0 b2 + a1 b0, warp 2 a0 b1, warp 3 the K steps
     // of a0 b0 alternating over two accumulators
-    if ((tid & 31) == 0) {
+    if ((tid & 31) == 0 && warp < 4) {
       constexpr uint32_t LA = BQ * 16, LB = BK * 16;
       if (warp < 3) {
         const int pa[5] = {2, 1, 0, 1, 0}, pb[5] = {0, 1, 2, 0, 1};
@@ -413,15 +413,15 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
         int n = 0;
         for (int t = t0; t < t0 + nt; ++t)
 #pragma unroll
-          for (int st = 0; st < DP / 16; ++st, ++n)
-            sm100::mma_bf16_ss(d, sm100::smem_desc(a_q + pa[t] * Q_BYTES + st * 2 * LA, LA, 128),
-                               sm100::smem_desc(a_k + pb[t] * K_BYTES + st * 2 * LB, LB, 128), IDESC_S,
+          for (int k = 0; k < DP / 16; ++k, ++n)
+            sm100::mma_bf16_ss(d, sm100::smem_desc(a_q + pa[t] * Q_BYTES + k * 2 * LA, LA, 128),
+                               sm100::smem_desc(a_k + pb[t] * K_BYTES + k * 2 * LB, LB, 128), IDESC_S,
                                n > 0 ? 1u : 0u);
       } else {
 #pragma unroll
-        for (int st = 0; st < DP / 16; ++st)
-          sm100::mma_bf16_ss(tSb + (st % NBIG) * BK, sm100::smem_desc(a_q + st * 2 * LA, LA, 128),
-                             sm100::smem_desc(a_k + st * 2 * LB, LB, 128), IDESC_S, st >= NBIG ? 1u : 0u);
+        for (int k = 0; k < DP / 16; ++k)
+          sm100::mma_bf16_ss(tSb + (k % NBIG) * BK, sm100::smem_desc(a_q + k * 2 * LA, LA, 128),
+                             sm100::smem_desc(a_k + k * 2 * LB, LB, 128), IDESC_S, k >= NBIG ? 1u : 0u);
       }
       sm100::mma_commit(&mbS);
     }
@@ -429,64 +429,64 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
-    // the 64 scores of this query row: the five S accumulators added in fp32
-    float sv[BK];
-#pragma unroll
-    for (int c = 0; c < BK; c += 32) {
-      uint32_t r[32];
-      sm100::tmem_ld32(sm100::tmem_lane(tS0 + c, warp), r);
+    // this half's 32 scores of row r: the five S accumulators added in fp32
+    const int c0 = 32 * hf;
+    float sv[32];
+    {
+      uint32_t rr[32];
+      sm100::tmem_ld32(sm100::tmem_lane(tS0 + c0, lq), rr);
       sm100::wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) sv[c + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(rr[e]);
       const uint32_t others[4] = {tS1, tS2, tSb, tSb + BK};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        sm100::tmem_ld32(sm100::tmem_lane(others[i] + c, warp), r);
+        sm100::tmem_ld32(sm100::tmem_lane(others[i] + c0, lq), rr);
         sm100::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c + e] += __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) sv[e] += __uint_as_float(rr[e]);
       }
     }
     float tmax = -CUDART_INF_F;
 #pragma unroll
-    for (int c = 0; c < BK; ++c) {
-      sv[c] = j0 + c < a.T ? a.scale * nuk[c] * sv[c] : -CUDART_INF_F;
-      tmax = fmaxf(tmax, sv[c]);
+    for (int e = 0; e < 32; ++e) {
+      sv[e] = j0 + c0 + e < a.T ? a.scale * nuk[c0 + e] * sv[e] : -CUDART_INF_F;
+      tmax = fmaxf(tmax, sv[e]);
     }
-    const float mn = fmaxf(m, tmax);
+    xmax[hf][r] = tmax;
+    __syncthreads();
+    const float mn = fmaxf(m, fmaxf(xmax[0][r], xmax[1][r]));
     const float corr = __expf(m - mn);
     // P nu_v (the value norms of the keys, so V_rot holds centroids only),
     // as a two-term bf16 split: its 2^-17 error reaches the output directly,
     // not through the softmax
     float ps = 0.f;
 #pragma unroll
-    for (int c = 0; c < BK; c += 8) {
+    for (int c = 0; c < 32; c += 8) {
       float w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float pe = __expf(sv[c + e] - mn);
         ps += pe;
-        w[e] = pe * vns[c + e];
+        w[e] = pe * vns[c0 + c + e];
       }
-      split2_store8(ps3, P_BYTES, kmaj16(tid, c, BQ), w);
+      split2_store8(ps3, P_BYTES, kmaj16(r, c0 + c, BQ), w);
     }
     l = l * corr + ps;
     m = mn;
-    // the running output lives in TMEM (columns tO): rescale a warp's rows
-    // when some row's maximum moved, before the P V MMAs add this tile
-    if (j0 > 0 && __any_sync(TQ_FULL, corr != 1.f)) {
+    // the running output lives in TMEM: rescale this half's columns of both
+    // O accumulators when some row of the warp moved its maximum
+    if (jt > 0 && __any_sync(TQ_FULL, corr != 1.f)) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i)
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t t = (i ? tO2 : tO) + 32 * hf;
+        uint32_t rr[32];
+        sm100::tmem_ld32(sm100::tmem_lane(t, lq), rr);
+        sm100::wait_ld();
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          const uint32_t t = (i ? tO2 : tO) + c;
-          uint32_t r[32];
-          sm100::tmem_ld32(sm100::tmem_lane(t, warp), r);
-          sm100::wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
-          sm100::tmem_st32(sm100::tmem_lane(t, warp), r);
-        }
+        for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
+        sm100::tmem_st32(sm100::tmem_lane(t, lq), rr);
+      }
       sm100::wait_st();
     }
     sm100::fence_async_smem();
@@ -503,10 +503,10 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
       int n = 0;
       for (int t = 3 * warp; t < (warp == 0 ? 3 : 5); ++t)
 #pragma unroll
-        for (int st = 0; st < BK / 16; ++st, ++n)
-          sm100::mma_bf16_ss(d, sm100::smem_desc(a_p + pa[t] * P_BYTES + st * 2 * LA, LA, 128),
-                             sm100::smem_desc(a_v + pb[t] * V_BYTES + st * 2 * LB, LB, 128), IDESC_O,
-                             (n > 0 || j0 > 0) ? 1u : 0u);
+        for (int k = 0; k < BK / 16; ++k, ++n)
+          sm100::mma_bf16_ss(d, sm100::smem_desc(a_p + pa[t] * P_BYTES + k * 2 * LA, LA, 128),
+                             sm100::smem_desc(a_v + pb[t] * V_BYTES + k * 2 * LB, LB, 128), IDESC_O,
+                             (n > 0 || jt > 0) ? 1u : 0u);
       sm100::mma_commit(&mbO);
     }
     if (!sm100::mbar_wait(&mbO, phase)) abort_s = 1;
@@ -515,40 +515,44 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
     if (abort_s) break;
     sm100::fence_after_sync();
   }
-  float o[D];
+  // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l), by the half-0 threads
+  if (hf == 1) lsum_s[r] = l;
+  __syncthreads();
+  if (hf == 0) {
+    float o[D];
 #pragma unroll
-  for (int c = 0; c < D; c += 16) {
-    uint32_t r[16], r2[16];
-    sm100::tmem_ld16(sm100::tmem_lane(tO + c, warp), r);
-    sm100::tmem_ld16(sm100::tmem_lane(tO2 + c, warp), r2);
-    sm100::wait_ld();
+    for (int c = 0; c < D; c += 16) {
+      uint32_t r1[16], r2[16];
+      sm100::tmem_ld16(sm100::tmem_lane(tO + c, lq), r1);
+      sm100::tmem_ld16(sm100::tmem_lane(tO2 + c, lq), r2);
+      sm100::wait_ld();
 #pragma unroll
-    for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r[e]) + __uint_as_float(r2[e]);
-  }
-  // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l)
-  if (!abort_s && q0 + tid < a.Lq) {
+      for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r1[e]) + __uint_as_float(r2[e]);
+    }
+    if (!abort_s && q0 + r < a.Lq) {
 #pragma unroll
-    for (int s = 1; s < D; s <<= 1)
+      for (int s2 = 1; s2 < D; s2 <<= 1)
 #pragma unroll
-      for (int i = 0; i < D; ++i)
-        if (!(i & s)) {
-          const float x = o[i], y = o[i + s];
-          o[i] = x + y;
-          o[i + s] = x - y;
-        }
-    const float f = 1.0f / (sqrtf(static_cast<float>(D)) * l);
-    float *dst = a.out + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + q0 + tid) * D;
+        for (int i = 0; i < D; ++i)
+          if (!(i & s2)) {
+            const float x = o[i], y = o[i + s2];
+            o[i] = x + y;
+            o[i + s2] = x - y;
+          }
+      const float f = 1.0f / (sqrtf(static_cast<float>(D)) * (l + lsum_s[r]));
+      float *dst = a.out + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + q0 + r) * D;
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
-      const float sgn = ((a.books.dneg[i >> 5] >> (i & 31)) & 1) ? -1.f : 1.f;
-      dst[i] = o[i] * sgn * f;
+      for (int i = 0; i < D; ++i) {
+        const float sgn = ((a.books.dneg[i >> 5] >> (i & 31)) & 1) ? -1.f : 1.f;
+        dst[i] = o[i] * sgn * f;
+      }
     }
   }
   // this CTA's copies have landed before its shared memory is released: the
   // last issued tile's phase completes (at once if it was consumed)
   if (tid == 0 && issued > 0) sm100::mbar_wait(&kvf[(issued - 1) & 1], ((issued - 1) >> 1) & 1, 1u << 20);
   // every MMA this thread issued has landed before tensor memory is released
-  if ((tid & 31) == 0) {
+  if ((tid & 31) == 0 && warp < 4) {
     sm100::mma_commit(&fin[warp]);
     sm100::mbar_wait(&fin[warp], 0, 1u << 20);
   }
@@ -557,7 +561,6 @@ __global__ void __launch_bounds__(BQ, 1) bidir_tile_kernel(BidirArgs a) {
   __syncthreads();
   sm100::fence_after_sync();
   if (warp == 0) sm100::tmem_dealloc(tm, 512);
-  (void)NPL;
 }
 
 }  // namespace
@@ -617,7 +620,7 @@ int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int 
   cudaEvent_t ev0, ev1;
   tq_timing_events(&ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, stream);
-  bidir_tile_kernel<D><<<grid, BQ, shm, stream>>>(a);
+  bidir_tile_kernel<D><<<grid, BT, shm, stream>>>(a);
   if (int e = tq_check_launch("bidir_tile_kernel")) return e;
   if (ev1) cudaEventRecord(ev1, stream);
   tq_count_launch(2);
