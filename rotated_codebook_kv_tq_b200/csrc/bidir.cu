@@ -34,7 +34,8 @@ namespace {
 
 constexpr int BQ = 128;   // queries per CTA
 constexpr int BK = 64;    // keys per tile
-constexpr int BT = 256;   // threads of the tile kernel: two per query row
+constexpr int PR = 4;     // threads per query row in the tile kernel
+constexpr int BT = PR * BQ;
 
 struct BidirArgs {
   const void *q;
@@ -199,7 +200,10 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   constexpr uint32_t IDESC_S = sm100::idesc_bf16(128, BK);
   constexpr uint32_t IDESC_O = sm100::idesc_bf16(128, D);
   constexpr uint32_t STG = 4608;                   // one stage of compressed rows
-  static_assert(BT == 2 * BQ && BQ == 2 * BK && D == BK && BK == 64, "thread mapping");
+  static_assert(BT == PR * BQ && BQ == 2 * BK && D == BK && BK == 64 && (PR == 2 || PR == 4), "thread mapping");
+  constexpr int CPT = 16 * BK / BT;   // 8-column chunks of K_rot per thread (16 per key row)
+  constexpr int TPT = 8 * D / BT;     // 8-key chunks of V_rot^T per thread (8 per coordinate)
+  constexpr int KPT = BK / PR;        // keys (scores) and output columns per thread
   extern __shared__ __align__(128) float smem_b[];
   // each operand is stored as bf16 split planes (three, two for P)
   uint8_t *qs3 = reinterpret_cast<uint8_t *>(smem_b);
@@ -214,14 +218,14 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   // per word: K_rot's MSE half and V_rot are table lookups
   __shared__ __align__(16) uint16_t tabk[3][8], tabv[3][16];
   __shared__ float vns[BK];        // value norms of the current key tile
-  __shared__ float xmax[2][BQ];    // the two halves' tile maxima of each query row
-  __shared__ float lsum_s[BQ];
+  __shared__ float xmax[PR][BQ];   // the parts' tile maxima of each query row
+  __shared__ float lsum_s[PR][BQ];
   __shared__ __align__(8) uint64_t mbS, mbO, fin[4], kvf[2];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int r = tid & (BQ - 1), hf = tid >> 7;   // query row (TMEM lane), half of its keys / columns
+  const int r = tid & (BQ - 1), hf = tid >> 7;   // query row (TMEM lane), part of its keys / columns
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / (a.H / a.Hkv);
   const int64_t bh = static_cast<int64_t>(b) * a.Hkv + kvh;
@@ -255,11 +259,11 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // query tile: row r = query q0 + r (rows past Lq are zero), columns of half hf
+  // query tile: row r = query q0 + r (rows past Lq are zero), columns of part hf
   {
     const int qi = q0 + r;
     const float *src = a.qrot + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + qi) * DP;
-    for (int k = hf * D; k < hf * D + D; ++k)
+    for (int k = hf * (DP / PR); k < (hf + 1) * (DP / PR); ++k)
       split3_store(qs3, Q_BYTES, kmaj16(r, k, BQ), qi < a.Lq ? src[k] : 0.f);
   }
   sm100::fence_async_smem();
@@ -312,20 +316,21 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     const uint8_t *st = stg0 + (jt & 1) * STG;
     if (tid < BK)
       vns[tid] = j0 + tid < a.T ? tq_half_to_f32(reinterpret_cast<const uint16_t *>(st + 4352)[tid]) : 0.f;
-    // ---- key tile: thread (row tid % BK, part tid / BK) writes 32 columns of
-    // one key row: part 0-1 the MSE half (c[idx]), part 2-3 the sign half
-    // (+-coef rho); value tile: thread (coordinate tid % D, group and half of
-    // tid / D) writes 16 keys of V_rot^T
+    // ---- key tile: thread (row tid % BK, q = tid / BK) writes CPT of the 16
+    // 8-column chunks of one key row (chunk k: half k / 8 (the MSE half
+    // c[idx], or the sign half +-coef rho), word (k / 4) % 2, slice k % 4);
+    // value tile: thread (coordinate, group, slice) writes TPT 8-key chunks of
+    // V_rot^T
     {
-      const int row = tid % BK, part = tid / BK;
-      const int half = part >> 1, w = part & 1;
+      const int row = tid % BK, qk = tid / BK;
+      const int half = (qk * CPT) >> 3, w = ((qk * CPT) >> 2) & 1;   // the same for all CPT chunks
       const int j = j0 + row;
       const bool ok = j < a.T;
       const uint32_t *krow = reinterpret_cast<const uint32_t *>(st + row * planes_k * (D / 8));
       const uint32_t sc = ok ? reinterpret_cast<const uint32_t *>(st + 2048)[row] : 0u;
       const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
       const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-      if (part == 0) nuk[row] = ok ? nu : 0.f;
+      if (qk == 0) nuk[row] = ok ? nu : 0.f;
       uint32_t pw[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int p = 0; p < 4; ++p)
@@ -348,7 +353,8 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
       }
       const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
+      for (int ci = 0; ci < CPT; ++ci) {
+        const int c8 = (qk * CPT + ci) & 3;
         uint32_t o[3][4];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
@@ -373,7 +379,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     }
     {
       // V_rot^T: centroids only (the value norms scale P instead)
-      const int coord = tid % D, g = (tid / D) & 1, th = tid / (2 * D);
+      const int coord = tid % D, g = (tid / D) & 1, th = tid / (2 * D);   // th: which TPT slices
       const int jg = j0 + 32 * g;
       uint32_t vw[4] = {0u, 0u, 0u, 0u};
       if (jg < a.T)
@@ -381,7 +387,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
           vw[p] = reinterpret_cast<const uint32_t *>(st + 2304)[(g * nbv + p) * D + coord];
       const uint32_t *tv32 = reinterpret_cast<const uint32_t *>(&tabv[0][0]);
 #pragma unroll
-      for (int t8 = 2 * th; t8 < 2 * th + 2; ++t8) {
+      for (int t8 = TPT * th; t8 < TPT * th + TPT; ++t8) {
         uint32_t o[3][4];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
@@ -429,40 +435,45 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     __syncthreads();
     if (abort_s) break;
     sm100::fence_after_sync();
-    // this half's 32 scores of row r: the five S accumulators added in fp32
-    const int c0 = 32 * hf;
-    float sv[32];
+    // this part's KPT scores of row r: the five S accumulators added in fp32
+    const int c0 = KPT * hf;
+    float sv[KPT];
     {
-      uint32_t rr[32];
-      sm100::tmem_ld32(sm100::tmem_lane(tS0 + c0, lq), rr);
-      sm100::wait_ld();
+      uint32_t rr[16];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) sv[e] = __uint_as_float(rr[e]);
-      const uint32_t others[4] = {tS1, tS2, tSb, tSb + BK};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sm100::tmem_ld32(sm100::tmem_lane(others[i] + c0, lq), rr);
+      for (int c = 0; c < KPT; c += 16) {
+        sm100::tmem_ld16(sm100::tmem_lane(tS0 + c0 + c, lq), rr);
         sm100::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[e] += __uint_as_float(rr[e]);
+        for (int e = 0; e < 16; ++e) sv[c + e] = __uint_as_float(rr[e]);
+        const uint32_t others[4] = {tS1, tS2, tSb, tSb + BK};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sm100::tmem_ld16(sm100::tmem_lane(others[i] + c0 + c, lq), rr);
+          sm100::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) sv[c + e] += __uint_as_float(rr[e]);
+        }
       }
     }
     float tmax = -CUDART_INF_F;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
+    for (int e = 0; e < KPT; ++e) {
       sv[e] = j0 + c0 + e < a.T ? a.scale * nuk[c0 + e] * sv[e] : -CUDART_INF_F;
       tmax = fmaxf(tmax, sv[e]);
     }
     xmax[hf][r] = tmax;
     __syncthreads();
-    const float mn = fmaxf(m, fmaxf(xmax[0][r], xmax[1][r]));
+    float mn = m;
+#pragma unroll
+    for (int i = 0; i < PR; ++i) mn = fmaxf(mn, xmax[i][r]);
     const float corr = __expf(m - mn);
     // P nu_v (the value norms of the keys, so V_rot holds centroids only),
     // as a two-term bf16 split: its 2^-17 error reaches the output directly,
     // not through the softmax
     float ps = 0.f;
 #pragma unroll
-    for (int c = 0; c < 32; c += 8) {
+    for (int c = 0; c < KPT; c += 8) {
       float w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -478,15 +489,17 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     // O accumulators when some row of the warp moved its maximum
     if (jt > 0 && __any_sync(TQ_FULL, corr != 1.f)) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t t = (i ? tO2 : tO) + 32 * hf;
-        uint32_t rr[32];
-        sm100::tmem_ld32(sm100::tmem_lane(t, lq), rr);
-        sm100::wait_ld();
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
-        sm100::tmem_st32(sm100::tmem_lane(t, lq), rr);
-      }
+        for (int c = 0; c < KPT; c += 8) {
+          const uint32_t t = (i ? tO2 : tO) + KPT * hf + c;
+          uint32_t rr[8];
+          sm100::tmem_ld8(sm100::tmem_lane(t, lq), rr);
+          sm100::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * corr);
+          sm100::tmem_st8(sm100::tmem_lane(t, lq), rr);
+        }
       sm100::wait_st();
     }
     sm100::fence_async_smem();
@@ -515,8 +528,8 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     if (abort_s) break;
     sm100::fence_after_sync();
   }
-  // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l), by the half-0 threads
-  if (hf == 1) lsum_s[r] = l;
+  // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l), by the part-0 threads
+  lsum_s[hf][r] = l;
   __syncthreads();
   if (hf == 0) {
     float o[D];
@@ -539,7 +552,10 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
             o[i] = x + y;
             o[i + s2] = x - y;
           }
-      const float f = 1.0f / (sqrtf(static_cast<float>(D)) * (l + lsum_s[r]));
+      float lt = 0.f;
+#pragma unroll
+      for (int i = 0; i < PR; ++i) lt += lsum_s[i][r];
+      const float f = 1.0f / (sqrtf(static_cast<float>(D)) * lt);
       float *dst = a.out + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + q0 + r) * D;
 #pragma unroll
       for (int i = 0; i < D; ++i) {
