@@ -120,15 +120,30 @@ __device__ __forceinline__ int kmaj16(int row, int k, int R) {
 }
 
 // v = p0 + p1 + p2 in bf16 (each the rounding of what is left): |error| < 2^-26 |v|.
-// Plane j of the split lives at base + j * stride.
-__device__ __forceinline__ void split3_store(uint8_t *base, uint32_t stride, int off, float v) {
-  const __nv_bfloat16 a = __float2bfloat16_rn(v);
-  const float r1 = v - __bfloat162float(a);
-  const __nv_bfloat16 b = __float2bfloat16_rn(r1);
-  const __nv_bfloat16 c = __float2bfloat16_rn(r1 - __bfloat162float(b));
-  *reinterpret_cast<__nv_bfloat16 *>(base + off) = a;
-  *reinterpret_cast<__nv_bfloat16 *>(base + stride + off) = b;
-  *reinterpret_cast<__nv_bfloat16 *>(base + 2 * stride + off) = c;
+// Eight consecutive K elements (k0 a multiple of 8) of one row as the three
+// split planes, each one 16-byte core-matrix row written with one store.
+__device__ __forceinline__ void split3_store8(uint8_t *base, uint32_t stride, int off, const float (&v)[8]) {
+  uint32_t w[3][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    uint32_t pp[3][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x = v[2 * e + h];
+      const __nv_bfloat16 p0 = __float2bfloat16_rn(x);
+      const float r1 = x - __bfloat162float(p0);
+      const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+      pp[0][h] = __bfloat16_as_ushort(p0);
+      pp[1][h] = __bfloat16_as_ushort(p1);
+      pp[2][h] = __bfloat16_as_ushort(p2);
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) w[j][e] = pp[j][0] | (pp[j][1] << 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 3; ++j)
+    *reinterpret_cast<uint4 *>(base + j * stride + off) = make_uint4(w[j][0], w[j][1], w[j][2], w[j][3]);
 }
 
 // v = p0 + p1 in bf16 (|error| < 2^-17 |v|), planes at base and base + stride.
@@ -259,12 +274,31 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // query tile: row r = query q0 + r (rows past Lq are zero), columns of part hf
+  // query tile: row r = query q0 + r (rows past Lq are zero), the DP / PR
+  // columns of part hf, read as 16-byte loads all in flight at once
   {
+    constexpr int QC = DP / PR;
     const int qi = q0 + r;
-    const float *src = a.qrot + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + qi) * DP;
-    for (int k = hf * (DP / PR); k < (hf + 1) * (DP / PR); ++k)
-      split3_store(qs3, Q_BYTES, kmaj16(r, k, BQ), qi < a.Lq ? src[k] : 0.f);
+    float qv[QC];
+    if (qi < a.Lq) {
+      const float4 *src = reinterpret_cast<const float4 *>(
+          a.qrot + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + qi) * DP + hf * QC);
+#pragma unroll
+      for (int c = 0; c < QC / 4; ++c) {
+        const float4 v = src[c];
+        qv[4 * c] = v.x; qv[4 * c + 1] = v.y; qv[4 * c + 2] = v.z; qv[4 * c + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < QC; ++c) qv[c] = 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < QC; c += 8) {
+      float v8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] = qv[c + e];
+      split3_store8(qs3, Q_BYTES, kmaj16(r, hf * QC + c, BQ), v8);
+    }
   }
   sm100::fence_async_smem();
   sm100::fence_before_sync();
