@@ -304,6 +304,77 @@ int tq_dequantize(const tq_codec *codec, const tq_cache *cache, int which, int64
                   int64_t rows, float *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Outlier-channel mixed precision ("Google presenta TurboQuant ...",
+ * "Desempeno teorico y empirico": for non-integer rates, specific outlier
+ * channels get more bits than the rest, e.g. 3 and 2 bits for 2.5 bits per
+ * channel, 4 and 3 for 3.5).
+ *
+ * A head vector of d = 2 * hi->d channels is split, per KV head and separately
+ * for keys and values, into two channel sets of d/2 each.  Each set is an
+ * independent TurboQuant vector coded by its own codec (own norm, rotation,
+ * codebooks and QJL sketch) into its own cache: `hi` (more bits) codes the
+ * outlier channels, `lo` the rest.  The rate per channel is the mean of the two
+ * codecs' bit widths.  Keys are RoPE-rotated over all d channels before the
+ * split ("TurboESM ...", section 2.A).  Decode sums the two codecs' logit
+ * estimates; each value half is summed in its own rotated domain and rotated
+ * back onto its channels.
+ *
+ * hi, lo     codecs with the same d (64 or 128); any bit widths and QJL flags.
+ * channels   device int16 [Hkv][2][d], 2-byte aligned, owned by the caller:
+ *            per KV head, list 0 (keys) and list 1 (values), each a
+ *            permutation of 0..d-1 whose first d/2 entries are the channels
+ *            coded by `hi` and whose last d/2 are coded by `lo`.  Entries are
+ *            taken modulo d; lists that are not permutations give unspecified
+ *            (but in-bounds) results.
+ * cache_hi, cache_lo  caches of the hi and lo codecs with equal B, Hkv and
+ *            rows_cap (tq_cache_bytes with each codec).
+ * Bytes per (token, head): the sum of both caches' (keys: d/16 * (planes_hi +
+ * planes_lo) + 8; values: d/16 * (bits_v_hi + bits_v_lo) + 4).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const tq_codec *hi;
+  const tq_codec *lo;
+  const int16_t *channels;
+} tq_split;
+
+/* Host helper: for each of n rows of score (host fp32 [n][d]), the d/2
+ * highest-scoring channels (ties to the lower index) in ascending order, then
+ * the other channels ascending -> channels (host int16 [n][d]).  With n = 2 Hkv
+ * rows ordered (head, keys|values) the result is the layout above.
+ * Errors: TQ_ERR_INVALID_ARG for NULL pointers, n < 1, odd d or a NaN score. */
+int tq_split_channels(const float *score, int n, int d, int16_t *channels);
+
+/* Quantize-append into both caches.  Arguments as tq_quantize_kv with d-wide
+ * rows of k and v (d = 2 * hi->d); status counts bad half rows (each half is
+ * checked on its own). */
+int tq_quantize_kv_split(const tq_split *split, const void *k, const void *v, int dtype, int B,
+                         int Hkv, int T, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                         const float *rope_cos, const float *rope_sin, int64_t pos0,
+                         const tq_cache *cache_hi, const tq_cache *cache_lo, int64_t row0,
+                         uint32_t *status, void *stream);
+
+/* Decode over the split caches (CUDA cores, split-K):
+ *   l_j = scale * sum over the halves of nu_j (<q'_h, c_h[idx]> +
+ *         sqrt(pi/2)/(d/2) rho_j <q''_h, 2 sigma - 1>),
+ *   q'_h = Pi_h (RoPE(q, T_b - 1) restricted to half h's key channels),
+ * out = each half's sum_j softmax(l)_j nu^v_j Pi_h^T c_v,h[idx] on its value
+ * channels.  Arguments as tq_attention_decode (q and out are d wide); the
+ * workspace size comes from tq_attention_split_workspace. */
+int tq_attention_split_workspace(const tq_split *split, int B, int Hq, int num_splits,
+                                 size_t *bytes);
+int tq_attention_decode_split(const tq_split *split, const void *q, int dtype, int B, int Hq,
+                              int Hkv, const tq_cache *cache_hi, const tq_cache *cache_lo,
+                              const int32_t *seq_lens, int max_seq_len, float scale,
+                              const float *rope_cos, const float *rope_sin, int num_splits,
+                              void *workspace, size_t ws_bytes, float *out, void *stream);
+
+/* Dequantize rows [row0, row0 + rows) of both caches back onto their channels:
+ * out device fp32 [B][Hkv][rows][d]. */
+int tq_dequantize_split(const tq_split *split, const tq_cache *cache_hi,
+                        const tq_cache *cache_lo, int which, int64_t row0, int64_t rows,
+                        float *out, void *stream);
+
+/* ------------------------------------------------------------------------
  * Profiling hooks (no counterpart on the pages; used by the benchmark).
  * tq_set_timing_events: when both are non-NULL, every later
  *   tq_attention_decode / tq_attention_logits on this thread records `start`

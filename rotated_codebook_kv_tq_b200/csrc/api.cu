@@ -1,4 +1,5 @@
 // C ABI entry points: argument validation, codec lifetime, kernel dispatch.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <string>
@@ -263,6 +264,21 @@ int tq_attention_workspace(const tq_codec *c, int B, int Hq, int num_splits, siz
 }
 
 namespace {
+// Split-K chunks per (b, KV head).  Default (num_splits = 0): about one chunk
+// per resident CTA (two per SM), 128-row multiples, never more than the 64
+// splits a workspace sized with num_splits = 0 holds.
+int pick_splits(int num_splits, int max_seq_len, int B, int Hkv) {
+  if (num_splits > 0) return num_splits;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int bh = B * Hkv;
+  int s = (2 * sms + bh - 1) / bh;
+  s = s < 1 ? 1 : (s > 64 ? 64 : s);
+  const int chunk = ((max_seq_len + s - 1) / s + 127) / 128 * 128;
+  return (max_seq_len + chunk - 1) / chunk;
+}
+
 int decode_common(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                   const tq_cache *cache, const int32_t *seq_lens, int max_seq_len, float scale,
                   const float *rope_cos, const float *rope_sin, int num_splits, void *workspace,
@@ -278,20 +294,7 @@ int decode_common(const tq_codec *c, const void *q, int dtype, int B, int Hq, in
   if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "decode: scale not finite");
   if ((rope_cos == nullptr) != (rope_sin == nullptr))
     return tq_fail(TQ_ERR_INVALID_ARG, "decode: rope_cos and rope_sin go together");
-  int splits = num_splits > 0 ? num_splits : 64;
-  if (num_splits == 0) {
-    // default: about one chunk per resident CTA (two per SM), 128-row
-    // multiples, never more than the 64 splits tq_attention_workspace(.., 0)
-    // sized the workspace for
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int bh = B * Hkv;
-    int s = (2 * sms + bh - 1) / bh;
-    s = s < 1 ? 1 : (s > 64 ? 64 : s);
-    const int chunk = ((max_seq_len + s - 1) / s + 127) / 128 * 128;
-    splits = (max_seq_len + chunk - 1) / chunk;
-  }
+  const int splits = pick_splits(num_splits, max_seq_len, B, Hkv);
   if (splits > 512) return tq_fail(TQ_ERR_INVALID_ARG, "decode: num_splits must be <= 512");
   if (decode_workspace_bytes(c, B, Hq, splits) > ws_bytes)
     return tq_fail(TQ_ERR_WORKSPACE, "decode: workspace smaller than tq_attention_workspace()");
@@ -361,6 +364,136 @@ int tq_dequantize(const tq_codec *c, const tq_cache *cache, int which, int64_t r
     return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: rows outside the cache");
   if (rows > 0 && !out) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize: NULL out");
   return launch_dequant(c, cache, which, row0, rows, out, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Outlier-channel split
+// ---------------------------------------------------------------------------
+
+namespace {
+int check_split(const tq_split *s, const tq_cache *chi, const tq_cache *clo) {
+  if (!s || !s->hi || !s->lo || !s->channels)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split: NULL codec or channel map");
+  if (s->hi->d != s->lo->d || (s->hi->d != 64 && s->hi->d != 128))
+    return tq_fail(TQ_ERR_UNSUPPORTED, "split: both codecs need the same d, 64 or 128");
+  if (int e = check_cache(s->hi, chi)) return e;
+  if (int e = check_cache(s->lo, clo)) return e;
+  if (chi->B != clo->B || chi->Hkv != clo->Hkv || chi->rows_cap != clo->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split: the two caches differ in B, Hkv or rows_cap");
+  if (!aligned(s->channels, 2)) return tq_fail(TQ_ERR_ALIGNMENT, "split: channel map alignment");
+  return TQ_OK;
+}
+
+// Row maps of the two halves: hi reads entries [0, d/2) of each list, lo
+// entries [d/2, d); keys use list 0 and values list 1 of every KV head.
+TqRowMap split_map(const tq_split *s, int half) {
+  const int d = 2 * s->hi->d;
+  TqRowMap m;
+  m.k = s->channels + half * (d / 2);
+  m.v = s->channels + d + half * (d / 2);
+  m.hstride = 2 * d;
+  m.dfull = d;
+  return m;
+}
+}  // namespace
+
+int tq_split_channels(const float *score, int n, int d, int16_t *channels) {
+  if (!score || !channels || n <= 0 || d < 2 || d % 2 || d > 32767)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split_channels: bad arguments");
+  std::vector<int> order(d);
+  for (int r = 0; r < n; ++r) {
+    const float *sr = score + static_cast<size_t>(r) * d;
+    for (int i = 0; i < d; ++i) {
+      if (std::isnan(sr[i])) return tq_fail(TQ_ERR_INVALID_ARG, "split_channels: NaN score");
+      order[i] = i;
+    }
+    // highest score first, ties to the lower channel
+    std::stable_sort(order.begin(), order.end(), [sr](int x, int y) { return sr[x] > sr[y]; });
+    std::sort(order.begin(), order.begin() + d / 2);
+    std::sort(order.begin() + d / 2, order.end());
+    for (int i = 0; i < d; ++i) channels[static_cast<size_t>(r) * d + i] = static_cast<int16_t>(order[i]);
+  }
+  return TQ_OK;
+}
+
+int tq_quantize_kv_split(const tq_split *s, const void *k, const void *v, int dtype, int B,
+                         int Hkv, int T, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                         const float *rope_cos, const float *rope_sin, int64_t pos0,
+                         const tq_cache *cache_hi, const tq_cache *cache_lo, int64_t row0,
+                         uint32_t *status, void *stream) {
+  if (int e = check_split(s, cache_hi, cache_lo)) return e;
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: dtype");
+  if (B != cache_hi->B || Hkv != cache_hi->Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: B/Hkv differ from the caches'");
+  if (T < 0 || row0 < 0 || row0 + T > cache_hi->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: rows [row0, row0+T) outside the caches");
+  if (T == 0) return TQ_OK;
+  if (!k || !v) return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: NULL k or v");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: rope_cos and rope_sin go together");
+  if (rope_cos && pos0 < 0) return tq_fail(TQ_ERR_INVALID_ARG, "quantize split: pos0 < 0");
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(k, es) || !aligned(v, es))
+    return tq_fail(TQ_ERR_ALIGNMENT, "quantize split: k/v not aligned to their element size");
+  const tq_codec *cd[2] = {s->hi, s->lo};
+  const tq_cache *cc[2] = {cache_hi, cache_lo};
+  for (int half = 0; half < 2; ++half)
+    if (int e = launch_quantize(cd[half], k, v, dtype, B, Hkv, T, stride_b, stride_h, stride_t,
+                                rope_cos, rope_sin, pos0, cc[half], row0, status,
+                                static_cast<cudaStream_t>(stream), split_map(s, half)))
+      return e;
+  return TQ_OK;
+}
+
+int tq_attention_split_workspace(const tq_split *s, int B, int Hq, int num_splits, size_t *bytes) {
+  if (!s || !s->hi || !bytes || B <= 0 || Hq <= 0 || num_splits < 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split workspace: bad arguments");
+  *bytes = split_workspace_bytes(s->hi, B, Hq, num_splits > 0 ? num_splits : 64);
+  return TQ_OK;
+}
+
+int tq_attention_decode_split(const tq_split *s, const void *q, int dtype, int B, int Hq,
+                              int Hkv, const tq_cache *cache_hi, const tq_cache *cache_lo,
+                              const int32_t *seq_lens, int max_seq_len, float scale,
+                              const float *rope_cos, const float *rope_sin, int num_splits,
+                              void *workspace, size_t ws_bytes, float *out, void *stream) {
+  if (int e = check_split(s, cache_hi, cache_lo)) return e;
+  if (!q || !out || !workspace)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split decode: NULL q/out/workspace");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "split decode: dtype");
+  if (B != cache_hi->B || Hkv != cache_hi->Hkv || Hq <= 0 || Hq % Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split decode: B/Hkv differ from the caches' or Hq % Hkv != 0");
+  if (max_seq_len < 1 || max_seq_len > cache_hi->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "split decode: max_seq_len outside 1..rows_cap");
+  if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "split decode: scale not finite");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "split decode: rope_cos and rope_sin go together");
+  const int splits = pick_splits(num_splits, max_seq_len, B, Hkv);
+  if (splits > 512) return tq_fail(TQ_ERR_INVALID_ARG, "split decode: num_splits must be <= 512");
+  if (split_workspace_bytes(s->hi, B, Hq, splits) > ws_bytes)
+    return tq_fail(TQ_ERR_WORKSPACE, "split decode: workspace smaller than tq_attention_split_workspace()");
+  if (!aligned(workspace, 16)) return tq_fail(TQ_ERR_ALIGNMENT, "split decode: workspace alignment");
+  if (!aligned(out, 4) || !aligned(q, dtype == TQ_BF16 ? 2 : 4))
+    return tq_fail(TQ_ERR_ALIGNMENT, "split decode: q/out alignment");
+  return launch_decode_split(s->hi, s->lo, s->channels, q, dtype, B, Hq, Hkv, cache_hi, cache_lo,
+                             seq_lens, max_seq_len, scale, rope_cos, rope_sin, splits, workspace,
+                             out, static_cast<cudaStream_t>(stream));
+}
+
+int tq_dequantize_split(const tq_split *s, const tq_cache *cache_hi, const tq_cache *cache_lo,
+                        int which, int64_t row0, int64_t rows, float *out, void *stream) {
+  if (int e = check_split(s, cache_hi, cache_lo)) return e;
+  if (which != 0 && which != 1) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize split: which is 0 or 1");
+  if (row0 < 0 || rows < 0 || row0 + rows > cache_hi->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "dequantize split: rows outside the caches");
+  if (rows > 0 && !out) return tq_fail(TQ_ERR_INVALID_ARG, "dequantize split: NULL out");
+  const tq_codec *cd[2] = {s->hi, s->lo};
+  const tq_cache *cc[2] = {cache_hi, cache_lo};
+  for (int half = 0; half < 2; ++half)
+    if (int e = launch_dequant(cd[half], cc[half], which, row0, rows, out,
+                               static_cast<cudaStream_t>(stream), split_map(s, half)))
+      return e;
+  return TQ_OK;
 }
 
 }  // extern "C"

@@ -22,6 +22,8 @@ struct DequantArgs {
   float qjl_coef;
   const uint16_t *S;
   float *out;
+  int Hkv;
+  TqRowMap map;
   TqBooks books;
 };
 
@@ -87,6 +89,14 @@ __global__ void __launch_bounds__(DW * 32) dequant_kernel(DequantArgs a) {
     tq_warp_wht<NPL>(y, lane);
     tq_apply_signs<NPL>(y, a.books.dneg, lane);
     const float f = nu / sqrtf(static_cast<float>(D));
+    if (a.map.k != nullptr) {
+      // outlier-channel split: coordinate i goes to channel map[h][i]
+      const int16_t *m = (a.which == 0 ? a.map.k : a.map.v) + (bh % a.Hkv) * a.map.hstride;
+      float *o = a.out + it * a.map.dfull;
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) o[m[lane + 32 * k] & (a.map.dfull - 1)] = y[k] * f;
+      continue;
+    }
     float *o = a.out + it * D;
 #pragma unroll
     for (int k = 0; k < NPL; ++k) o[lane + 32 * k] = y[k] * f;
@@ -109,7 +119,7 @@ int run_dequant(const DequantArgs &a, cudaStream_t stream) {
 }  // namespace
 
 int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
-                   int64_t rows, float *out, cudaStream_t stream) {
+                   int64_t rows, float *out, cudaStream_t stream, const TqRowMap &map) {
   DequantArgs a;
   a.kcode = cache->kcode;
   a.kscale = cache->kscale;
@@ -123,6 +133,8 @@ int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t 
   a.qjl_coef = c->qjl_k ? sqrtf(static_cast<float>(M_PI) / 2.0f) / c->d : 0.f;
   a.S = c->S_dev;
   a.out = out;
+  a.Hkv = cache->Hkv;
+  a.map = map;
   a.books = c->books;
   if (rows == 0) return TQ_OK;
   switch (c->d) {

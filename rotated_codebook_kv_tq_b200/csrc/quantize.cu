@@ -44,14 +44,41 @@ struct QuantArgs {
   const uint16_t *ST;  // S transposed (bf16)
   int64_t g_first;   // first 32-token group touched
   int64_t n_groups;  // groups touched per (b, h)
+  TqRowMap map;      // channel map of an outlier-channel split (k == nullptr: none)
   TqBooks books;
 };
 
+// Channel map of KV head h (nullptr without a map).
+__device__ __forceinline__ const int16_t *head_map(const int16_t *m, int64_t hs, int h) {
+  return m != nullptr ? m + h * hs : nullptr;
+}
+
 // Load one row (coordinates lane + 32 k), optional RoPE at position pos.
+// With a channel map (outlier-channel split), coordinate i is channel cmap[i]
+// of a dfull-wide input row, and RoPE pairs channels (c, c + dfull/2) of that
+// whole row, as in the unsplit case.
 template <int NPL>
 __device__ __forceinline__ void load_row(float (&x)[NPL], const void *base, int64_t off,
                                          int dtype, int lane, const float *rc, const float *rs,
-                                         int64_t pos) {
+                                         int64_t pos, const int16_t *cmap = nullptr,
+                                         int dfull = 0) {
+  if (cmap != nullptr) {
+    const int half = dfull >> 1;
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      const int c = cmap[lane + 32 * k] & (dfull - 1);   // in bounds for any map
+      float v = tq_load_elem(base, off + c, dtype);
+      if (rc != nullptr) {
+        const bool first = c < half;
+        const int f = first ? c : c - half;
+        const float w = tq_load_elem(base, off + (first ? c + half : c - half), dtype);
+        const float cs = rc[pos * half + f], sn = rs[pos * half + f];
+        v = first ? v * cs - w * sn : v * cs + w * sn;
+      }
+      x[k] = v;
+    }
+    return;
+  }
 #pragma unroll
   for (int k = 0; k < NPL; ++k) x[k] = tq_load_elem(base, off + lane + 32 * k, dtype);
   if (rc != nullptr) {
@@ -144,7 +171,8 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
       const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
       // ------------------------------------------------------------ keys
       float x[NPL];
-      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
+                    head_map(a.map.k, a.map.hstride, h), a.map.dfull);
       bool bad;
       const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
@@ -197,7 +225,8 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
         if (bad && a.status) atomicAdd(a.status, 1u);
       }
       // ------------------------------------------------------------ values
-      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
+                    head_map(a.map.v, a.map.hstride, h), a.map.dfull);
       const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
@@ -295,7 +324,8 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
     bool bad = false;
     if (warp == 0) {
       float x[NPL];
-      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
+      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
+                    head_map(a.map.k, a.map.hstride, h), a.map.dfull);
       nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
       int idx[NPL];
 #pragma unroll
@@ -319,7 +349,8 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       }
     } else if (warp == 1) {
       float x[NPL];
-      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
+                    head_map(a.map.v, a.map.hstride, h), a.map.dfull);
       bool vbad;
       const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, vbad);
       const uint32_t bit = 1u << (r & 31);
@@ -477,8 +508,10 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       if (r0 + i < re) {
         const int64_t t = r0 + i - a.row0;
         const int64_t in_off = b * a.sb + h * a.sh + t * a.st;
-        load_row<NPL>(xk[i], a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t);
-        load_row<NPL>(xv[i], a.v, in_off, a.dtype, lane, nullptr, nullptr, 0);
+        load_row<NPL>(xk[i], a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
+                      head_map(a.map.k, a.map.hstride, h), a.map.dfull);
+        load_row<NPL>(xv[i], a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
+                      head_map(a.map.v, a.map.hstride, h), a.map.dfull);
       }
     }
 #pragma unroll
@@ -706,7 +739,7 @@ int run_quantize(const QuantArgs &a, cudaStream_t stream) {
 int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
                     int T, int64_t sb, int64_t sh, int64_t st, const float *rc, const float *rs,
                     int64_t pos0, const tq_cache *cache, int64_t row0, uint32_t *status,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, const TqRowMap &map) {
   QuantArgs a;
   a.k = k;
   a.v = v;
@@ -731,6 +764,7 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   a.ST = c->ST_dev;
   a.g_first = row0 / 32;
   a.n_groups = (row0 + T - 1) / 32 - row0 / 32 + 1;
+  a.map = map;
   a.books = c->books;
   if (T == 0) return TQ_OK;
   const int64_t items = static_cast<int64_t>(B) * H * a.n_groups;
@@ -738,8 +772,9 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   // implementation, used to cross-check the tensor-core one)
   const char *impl = getenv("TQ_QUANT_IMPL");
   const bool simt = impl && impl[0] == 's';
-  if (items >= 256 && !simt) {
-    // large bf16 calls: one thread per row, TMA tiles (quantize_tile.cu)
+  if (items >= 256 && !simt && map.k == nullptr) {
+    // large bf16 calls: one thread per row, TMA tiles (quantize_tile.cu); a
+    // channel map (gathered loads) takes the warp-per-row kernels below
     const int e = launch_quantize_tile(c, k, v, dtype, B, H, T, sb, sh, st, rc, rs, pos0, cache,
                                        row0, status, stream);
     if (e != TQ_ERR_UNSUPPORTED) return e;

@@ -30,6 +30,16 @@ struct TqBooks {
   int bits_v;
 };
 
+// Channel map of an outlier-channel split: coordinate i of KV head h's half
+// row is channel k[h * hstride + i] (keys) or v[h * hstride + i] (values) of
+// the dfull-wide head vector.  k == nullptr: no map.
+struct TqRowMap {
+  const int16_t *k = nullptr;
+  const int16_t *v = nullptr;
+  int64_t hstride = 0;
+  int dfull = 0;
+};
+
 struct tq_codec {
   int d;
   int bits_k, qjl_k, bits_v, mse_bits_k;
@@ -80,7 +90,7 @@ int tq_check_launch(const char *what);
 int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
                     int T, int64_t sb, int64_t sh, int64_t st, const float *rc, const float *rs,
                     int64_t pos0, const tq_cache *cache, int64_t row0, uint32_t *status,
-                    cudaStream_t stream);
+                    cudaStream_t stream, const TqRowMap &map = TqRowMap());
 // Prefill quantize with one thread per row (quantize_tile.cu); returns
 // TQ_ERR_UNSUPPORTED without launching when the call does not fit its rules.
 int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
@@ -96,5 +106,15 @@ size_t bidir_workspace_bytes(const tq_codec *c, int B, int H, int Lq);
 int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int Hkv, int Lq,
                  const tq_cache *cache, int T, float scale, const float *rc, const float *rs,
                  void *ws, float *out, cudaStream_t stream);
+// With a map, out is [B][Hkv][rows][map.dfull] and half-row coordinate i lands
+// on channel map.k (keys) or map.v (values) of its head.
 int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
-                   int64_t rows, float *out, cudaStream_t stream);
+                   int64_t rows, float *out, cudaStream_t stream,
+                   const TqRowMap &map = TqRowMap());
+// Decode over an outlier-channel split cache (split.cu).
+size_t split_workspace_bytes(const tq_codec *hi, int B, int Hq, int splits);
+int launch_decode_split(const tq_codec *hi, const tq_codec *lo, const int16_t *channels,
+                        const void *q, int dtype, int B, int Hq, int Hkv, const tq_cache *chi,
+                        const tq_cache *clo, const int32_t *seq_lens, int max_len, float scale,
+                        const float *rc, const float *rs, int splits, void *ws, float *out,
+                        cudaStream_t stream);

@@ -25,8 +25,9 @@ EXPORTS = [
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
     "tq_attention_logits", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
-    "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_set_timing_events", "tq_launch_count",
-    "tq_last_error",
+    "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_split_channels",
+    "tq_quantize_kv_split", "tq_attention_split_workspace", "tq_attention_decode_split",
+    "tq_dequantize_split", "tq_set_timing_events", "tq_launch_count", "tq_last_error",
 ]
 
 
@@ -46,6 +47,10 @@ class CacheDesc(ctypes.Structure):
     _fields_ = [("kcode", ctypes.c_void_p), ("kscale", ctypes.c_void_p),
                 ("vcode", ctypes.c_void_p), ("vnorm", ctypes.c_void_p),
                 ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("rows_cap", ctypes.c_int64)]
+
+
+class SplitDesc(ctypes.Structure):
+    _fields_ = [("hi", ctypes.c_void_p), ("lo", ctypes.c_void_p), ("channels", ctypes.c_void_p)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -85,6 +90,14 @@ def lib() -> ctypes.CDLL:
         L.tq_scan_topk.argtypes = [vp, vp, vp, i64, vp, i32, i32, vp, vp, vp, sz, vp]
         L.tq_scan_topk_lut.argtypes = [vp, vp, vp, i64, vp, i32, i32, vp, vp, vp, sz, vp]
         L.tq_dequantize.argtypes = [vp, ctypes.POINTER(CacheDesc), i32, i64, i64, vp, vp]
+        sp, cp = ctypes.POINTER(SplitDesc), ctypes.POINTER(CacheDesc)
+        L.tq_split_channels.argtypes = [vp, i32, i32, vp]
+        L.tq_quantize_kv_split.argtypes = [sp, vp, vp, i32, i32, i32, i32, i64, i64, i64, vp, vp,
+                                           i64, cp, cp, i64, vp, vp]
+        L.tq_attention_split_workspace.argtypes = [sp, i32, i32, i32, ctypes.POINTER(sz)]
+        L.tq_attention_decode_split.argtypes = [sp, vp, i32, i32, i32, i32, cp, cp, vp, i32,
+                                                ctypes.c_float, vp, vp, i32, vp, sz, vp, vp]
+        L.tq_dequantize_split.argtypes = [sp, cp, cp, i32, i64, i64, vp, vp]
         L.tq_set_timing_events.argtypes = [vp, vp]
         L.tq_launch_count.argtypes = []
         L.tq_launch_count.restype = ctypes.c_uint64
@@ -336,6 +349,73 @@ def dequantize(codec: Codec, cache: Cache, which: int, row0: int, rows: int, out
     desc = cache.desc()
     check(lib().tq_dequantize(codec.handle, ctypes.byref(desc), which, row0, rows,
                               _ptr(out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- outlier-channel split
+
+def split_channels(score: np.ndarray) -> np.ndarray:
+    """tq_split_channels: score [..., d] (host) -> int16 channel lists [..., d]."""
+    sc = np.ascontiguousarray(score, dtype=np.float32)
+    d = sc.shape[-1]
+    out = np.zeros(sc.shape, dtype=np.int16)
+    check(lib().tq_split_channels(sc.ctypes.data, sc.size // d, d, out.ctypes.data))
+    return out
+
+
+@dataclass
+class Split:
+    """A ``tq_split``: two codecs and the device channel lists [Hkv, 2, d]
+    (int16) that assign each KV head's key and value channels to them."""
+    hi: Codec
+    lo: Codec
+    channels: "object"
+
+    def desc(self) -> SplitDesc:
+        return SplitDesc(self.hi.handle, self.lo.handle, self.channels.data_ptr())
+
+
+def quantize_kv_split(split: Split, k, v, cache_hi: Cache, cache_lo: Cache, row0: int = 0,
+                      rope=None, pos0: int = 0, status=None, stream=None) -> None:
+    """tq_quantize_kv_split on k, v [B, Hkv, T, d]."""
+    B, H, T, d = k.shape
+    if tuple(v.shape) != tuple(k.shape) or v.stride() != k.stride() or k.stride(3) != 1:
+        raise ValueError("k and v need the same shape and strides, last dim contiguous")
+    rc, rs = (None, None) if rope is None else rope
+    sd, dh, dl = split.desc(), cache_hi.desc(), cache_lo.desc()
+    check(lib().tq_quantize_kv_split(ctypes.byref(sd), k.data_ptr(), v.data_ptr(), _dtype_code(k),
+                                     B, H, T, k.stride(0), k.stride(1), k.stride(2), _ptr(rc),
+                                     _ptr(rs), pos0, ctypes.byref(dh), ctypes.byref(dl), row0,
+                                     _ptr(status), _stream(stream)))
+
+
+def attention_split_workspace(split: Split, B: int, Hq: int, num_splits: int) -> int:
+    n = ctypes.c_size_t(0)
+    sd = split.desc()
+    check(lib().tq_attention_split_workspace(ctypes.byref(sd), B, Hq, num_splits, ctypes.byref(n)))
+    return n.value
+
+
+def attention_decode_split(split: Split, q, cache_hi: Cache, cache_lo: Cache, max_seq_len: int,
+                           scale: float, out, workspace, seq_lens=None, rope=None,
+                           num_splits: int = 0, stream=None) -> None:
+    """tq_attention_decode_split: q [B, Hq, d] -> out [B, Hq, d] fp32."""
+    B, Hq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    sd, dh, dl = split.desc(), cache_hi.desc(), cache_lo.desc()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib().tq_attention_decode_split(ctypes.byref(sd), q.data_ptr(), _dtype_code(q), B, Hq,
+                                          cache_hi.Hkv, ctypes.byref(dh), ctypes.byref(dl),
+                                          _ptr(seq_lens), max_seq_len, float(scale), _ptr(rc),
+                                          _ptr(rs), num_splits, workspace.data_ptr(), ws_bytes,
+                                          out.data_ptr(), _stream(stream)))
+
+
+def dequantize_split(split: Split, cache_hi: Cache, cache_lo: Cache, which: int, row0: int,
+                     rows: int, out, stream=None) -> None:
+    """tq_dequantize_split -> out [B, Hkv, rows, d] fp32."""
+    sd, dh, dl = split.desc(), cache_hi.desc(), cache_lo.desc()
+    check(lib().tq_dequantize_split(ctypes.byref(sd), ctypes.byref(dh), ctypes.byref(dl), which,
+                                    row0, rows, _ptr(out), _stream(stream)))
 
 
 def set_timing_events(start=None, stop=None) -> None:

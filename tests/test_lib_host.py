@@ -95,3 +95,34 @@ def test_cache_bytes_formula(L):
     c = oc.make_codec(128, 4, True, 4, synth.rotation_signs(128, 0), synth.qjl_matrix_bf16(128, 0))
     kb, vb = oc.bytes_per_row(c)
     assert kb + vb == 134
+
+
+def test_split_channels_matches_oracle(L):
+    """tq_split_channels (host C) against the oracle's choice of outlier
+    channels, ties included."""
+    from oracle import split as osp
+    rng = np.random.default_rng(4)
+    score = rng.lognormal(0.0, 1.0, size=(8, 2, 128)).astype(np.float32)
+    score[0, 0, :10] = 7.0          # ties straddling the cut
+    score[1, 1] = 1.0               # all equal
+    got = native.split_channels(score)
+    np.testing.assert_array_equal(got.astype(np.int64), osp.outlier_channels(score))
+    assert got.dtype == np.int16 and got.shape == score.shape
+    bad = score.copy()
+    bad[2, 0, 5] = np.nan
+    with pytest.raises(native.TqError):
+        native.split_channels(bad)
+    assert L.tq_split_channels(score.ctypes.data, 1, 7, got.ctypes.data) == native.TQ_ERR_INVALID_ARG
+
+
+def test_split_calls_validate_before_device_work(L):
+    sz = ctypes.c_size_t(0)
+    assert L.tq_attention_split_workspace(None, 1, 8, 0, ctypes.byref(sz)) == native.TQ_ERR_INVALID_ARG
+    empty = native.SplitDesc(None, None, None)
+    cd = native.CacheDesc(None, None, None, None, 1, 1, 32)
+    assert L.tq_quantize_kv_split(ctypes.byref(empty), None, None, 0, 1, 1, 1, 0, 0, 0, None, None,
+                                  0, ctypes.byref(cd), ctypes.byref(cd), 0, None,
+                                  None) == native.TQ_ERR_INVALID_ARG
+    assert L.tq_dequantize_split(ctypes.byref(empty), ctypes.byref(cd), ctypes.byref(cd), 0, 0, 1,
+                                 None, None) == native.TQ_ERR_INVALID_ARG
+    assert b"split" in L.tq_last_error()
