@@ -45,7 +45,7 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
-                                      "decode_llama", "vector_search", "quality"],
+                                      "decode_llama", "vector_search", "quality", "decode_split"],
                    help="run one extra workload alone and print its JSON (1 GPU)")
     p.add_argument("--search-rows", type=int, default=0,
                    help="vector-search database rows for --only vector_search (default 10^6)")
@@ -448,6 +448,36 @@ def cpu_baselines(seconds: float = 1.0) -> dict:
         out[name] = entry("tokens/s", t1, tn, th, lambda t: w.B / (t * scale),
                           f"one decode step over the first {rows} of {w.T} tokens, all "
                           f"{w.B * w.Hq} query heads, time x {w.T}/{rows}")
+    # the 2.5-bit outlier split on the Llama shape, same sampling as above
+    from oracle import split as osp
+    from oracle.rotation import apply_rope
+    w = synth.WORKLOADS["llama_decode"]
+    rows = 1024
+    ww = w.scaled(T=rows)
+    K, V = synth.kv_inputs(ww)
+    K64, V64 = synth.as_float64(K, w.dtype), synth.as_float64(V, w.dtype)
+    q = synth.as_float64(synth.query_inputs(ww, Lq=1)[:, :, 0], w.dtype)
+    rope = synth.rope_for(w, rows)
+    halves = []
+    for i, (bk, bv) in enumerate(SPLIT_RATES["2.5"]):
+        ds, sd = w.d // 2, w.seed + 100 * (i + 1)
+        halves.append(oc.make_codec(ds, bk, True, bv, synth.rotation_signs(ds, sd),
+                                    synth.qjl_matrix_bf16(ds, sd)))
+    Kr = np.stack([[apply_rope(K64[b, h], rope[0], rope[1], np.arange(rows)) for h in range(w.Hkv)]
+                   for b in range(w.B)])
+    score = np.stack([np.mean(Kr ** 2, axis=(0, 2)), np.mean(V64 ** 2, axis=(0, 2))], axis=1)
+    sc = osp.make_split_codec(halves[0], halves[1], osp.outlier_channels(score))
+    caches = osp.empty_caches(sc, w.B, w.Hkv, rows)
+    osp.quantize_into(caches, K64[:, :, :rows - 1], V64[:, :, :rows - 1], sc, rope=rope)
+
+    def split_step():
+        osp.quantize_into(caches, K64[:, :, rows - 1:], V64[:, :, rows - 1:], sc, rope=rope,
+                          pos0=rows - 1, row0=rows - 1)
+        osp.decode(q, caches, sc, [rows] * w.B, 1.0 / math.sqrt(w.d), rope=rope)
+    t1, tn, th = _one_and_all(split_step, seconds)
+    out["decode_split_2.5bit"] = entry("tokens/s", t1, tn, th, lambda t: w.B / (t * w.T / rows),
+                                       f"one split decode step over the first {rows} of {w.T} "
+                                       f"tokens, all {w.B * w.Hq} query heads, time x {w.T}/{rows}")
     # ESM-2-shaped prefill quantize: two (batch, head) pairs of the 320
     w = synth.WORKLOADS["esm_prefill"]
     ww = w.scaled(B=1, Hq=2, Hkv=2)
@@ -768,6 +798,199 @@ def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
     return res
 
 
+# ---------------------------------------------------------------------------
+# Outlier-channel split ("Google presenta TurboQuant ...", "Desempeno teorico y
+# empirico": outlier channels at more bits than the rest)
+# ---------------------------------------------------------------------------
+
+SPLIT_RATES = {"2.5": ((3, 3), (2, 2)), "3.5": ((4, 4), (3, 3))}
+
+
+def split_codecs(w, rate: str):
+    """(hi, lo) library codecs of d/2 channels each, QJL keys: ``rate`` bits per
+    channel as the mean of the two codecs' widths."""
+    from rotated_codebook_kv_tq_b200 import native, synth
+    out = []
+    for i, (bk, bv) in enumerate(SPLIT_RATES[rate]):
+        ds, seed = w.d // 2, w.seed + 100 * (i + 1)
+        out.append(native.Codec(ds, bk, True, bv, synth.rotation_signs(ds, seed),
+                                synth.qjl_matrix_bf16(ds, seed)))
+    return out
+
+
+def split_row_bytes(hi, lo) -> int:
+    return sum(c.planes_k * c.d // 8 + 4 + c.bits_v * c.d // 8 + 2 for c in (hi, lo))
+
+
+def split_channel_lists(Kr, V):
+    """Per KV head: keys' and values' d/2 highest mean-square channels (keys
+    after RoPE, as the codec sees them) -> device int16 [Hkv, 2, d]."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native
+    score = torch.stack([(Kr.float() ** 2).mean(dim=(0, 2)), (V.float() ** 2).mean(dim=(0, 2))], dim=1)
+    return torch.from_numpy(native.split_channels(score.cpu().numpy())).cuda()
+
+
+class SplitBench:
+    """Decode step over the split cache: quantize-append of the new token into
+    both caches, then tq_attention_decode_split (same interface as DecodeBench
+    for time_decode)."""
+
+    def __init__(self, w, rate: str, n_sets: int):
+        import torch
+        from rotated_codebook_kv_tq_b200 import native, synth
+        self.w, self.native, self.n_sets = w, native, n_sets
+        hi, lo = split_codecs(w, rate)
+        T = w.T
+        self.rows_cap = (T + 31) // 32 * 32
+        K, V = synth.kv_inputs_torch(w, T=T)
+        r = synth.rope_for(w, self.rows_cap)
+        self.rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+        Kr = K.float() if self.rope is None else _rope_rows(K.float(), self.rope[0][:T], self.rope[1][:T])
+        self.split = native.Split(hi, lo, split_channel_lists(Kr, V))
+        del Kr
+        self.caches = []
+        for _ in range(n_sets):
+            ch = native.alloc_cache(hi, w.B, w.Hkv, self.rows_cap)
+            cl = native.alloc_cache(lo, w.B, w.Hkv, self.rows_cap)
+            native.quantize_kv_split(self.split, K[:, :, :T - 1], V[:, :, :T - 1], ch, cl,
+                                     rope=self.rope)
+            self.caches.append((ch, cl))
+        self.knew = K[:, :, T - 1:T].contiguous()
+        self.vnew = V[:, :, T - 1:T].contiguous()
+        self.q = synth.query_inputs_torch(w)[:, :, 0].contiguous()
+        self.scale = 1.0 / math.sqrt(w.d)
+        self.splits = w.num_splits
+        self.ws = torch.empty(native.attention_split_workspace(self.split, w.B, w.Hq, self.splits),
+                              dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        self.row_bytes = split_row_bytes(hi, lo)
+        torch.cuda.synchronize()
+
+    def step(self, s: int) -> None:
+        w, n = self.w, self.native
+        ch, cl = self.caches[s % self.n_sets]
+        n.quantize_kv_split(self.split, self.knew, self.vnew, ch, cl, row0=w.T - 1, rope=self.rope,
+                            pos0=w.T - 1)
+        n.attention_decode_split(self.split, self.q, ch, cl, w.T, self.scale, self.out, self.ws,
+                                 rope=self.rope, num_splits=self.splits)
+
+    def cache_bytes_per_step(self) -> int:
+        return self.w.B * self.w.Hkv * self.w.T * self.row_bytes
+
+
+def split_decode_extra(pk: dict, rate: str = "2.5", steps: int = 40, warmup: int = 5):
+    """Llama-shaped decode over the outlier-channel split cache (CUDA-core
+    split-K kernels): tokens/s and the chunk kernel's HBM roofline fraction."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import synth
+    w = synth.WORKLOADS["llama_decode"]
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    hi, lo = split_codecs(w, rate)
+    per_set = w.B * w.Hkv * ((w.T + 31) // 32 * 32) * split_row_bytes(hi, lo)
+    hi.close()
+    lo.close()
+    bench = SplitBench(w, rate, max(1, math.ceil(3 * l2 / per_set)))
+
+    class _Null:
+        def start(self):
+            pass
+
+        def stop(self):
+            return {}
+
+    total, kern, per_step, _ = time_decode(bench, steps, warmup, 1, _Null())
+    alg = bench.cache_bytes_per_step()
+    res = dict(workload=f"llama_decode split {rate} bits per channel: B={w.B} Hq={w.Hq} "
+                        f"Hkv={w.Hkv} d={w.d} T={w.T}, outlier halves {SPLIT_RATES[rate]} "
+                        "(keys incl. QJL, values), per-head channel lists from the prefill",
+               us_per_step=total / steps * 1e6, tokens_per_s=w.B * steps / total,
+               launches_per_step=per_step,
+               roofline=dict(bound="hbm", achieved=alg / kern / 1e9, peak=pk["hbm"], unit="GB/s",
+                             frac=alg / kern / 1e9 / pk["hbm"], algorithmic_bytes=alg,
+                             bytes_per_token_head=bench.row_bytes, kernel="split_chunk_kernel",
+                             kernel_us=kern * 1e6),
+               l2=f"rotating {bench.n_sets} split caches ({bench.n_sets * alg / 1e6:.0f} MB)")
+    del bench
+    torch.cuda.empty_cache()
+    return res
+
+
+def split_quality_extra(wname: str = "llama_decode"):
+    """relMSE_K, relMSE_V and attention-output cosine (definitions as in
+    quality_extra) of the 2.5- and 3.5-bit outlier splits, beside uniform
+    codecs of 2, 3 and 4 bits (keys with QJL) on the same inputs."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.WORKLOADS[wname]
+    rows_cap = (w.T + 31) // 32 * 32
+    K, V = synth.kv_inputs_torch(w)
+    q = synth.query_inputs_torch(w, Lq=1)[:, :, 0].contiguous()
+    r = synth.rope_for(w, rows_cap)
+    rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+    Kf, Vf, qf = K.float(), V.float(), q.float()
+    if rope is not None:
+        Kf = _rope_rows(Kf, rope[0][:w.T], rope[1][:w.T])
+        qf = _rope_rows(qf, rope[0][w.T - 1], rope[1][w.T - 1])
+    scale = 1.0 / math.sqrt(w.d)
+    Ke = Kf.repeat_interleave(w.G, dim=1)
+    Ve = Vf.repeat_interleave(w.G, dim=1)
+    p = torch.softmax(torch.einsum("bhd,bhtd->bht", qf, Ke) * scale, dim=-1)
+    o_ref = torch.einsum("bht,bhtd->bhd", p, Ve)
+    del Ke, Ve, p
+    chan = split_channel_lists(Kf, Vf)
+
+    def scores(deq, decode):
+        rel = {}
+        for which, x in ((0, Kf), (1, Vf)):
+            xh = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.float32, device="cuda")
+            deq(which, xh)
+            rel["K" if which == 0 else "V"] = float(((xh - x) ** 2).sum() / (x ** 2).sum())
+            del xh
+        o = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        decode(o)
+        cos = torch.nn.functional.cosine_similarity(o, o_ref, dim=-1)
+        return dict(relMSE_K=rel["K"], relMSE_V=rel["V"], output_cosine_mean=float(cos.mean()),
+                    output_cosine_min=float(cos.min()))
+
+    out = {}
+    for rate in SPLIT_RATES:
+        hi, lo = split_codecs(w, rate)
+        sp = native.Split(hi, lo, chan)
+        ch = native.alloc_cache(hi, w.B, w.Hkv, rows_cap)
+        cl = native.alloc_cache(lo, w.B, w.Hkv, rows_cap)
+        native.quantize_kv_split(sp, K, V, ch, cl, rope=rope)
+        ws = torch.empty(native.attention_split_workspace(sp, w.B, w.Hq, w.num_splits),
+                         dtype=torch.uint8, device="cuda")
+        out[f"split_{rate}"] = dict(
+            bits_per_channel=float(rate), halves=SPLIT_RATES[rate],
+            **scores(lambda which, xh: native.dequantize_split(sp, ch, cl, which, 0, w.T, xh),
+                     lambda o: native.attention_decode_split(sp, q, ch, cl, w.T, scale, o, ws,
+                                                             rope=rope, num_splits=w.num_splits)))
+        del ch, cl
+        hi.close()
+        lo.close()
+    for bits in (2, 3, 4):
+        D = synth.rotation_signs(w.d, w.seed)
+        S = synth.qjl_matrix_bf16(w.d, w.seed)
+        codec = native.Codec(w.d, bits, True, bits, D, S)
+        cache = native.alloc_cache(codec, w.B, w.Hkv, rows_cap)
+        native.quantize_kv(codec, K, V, cache, rope=rope)
+        ws = torch.empty(native.attention_workspace(codec, w.B, w.Hq, w.num_splits),
+                         dtype=torch.uint8, device="cuda")
+        out[f"uniform_{bits}"] = dict(
+            bits_per_channel=float(bits),
+            **scores(lambda which, xh: native.dequantize(codec, cache, which, 0, w.T, xh),
+                     lambda o: native.attention_decode(codec, q, cache, w.T, scale, o, ws,
+                                                       rope=rope, num_splits=w.num_splits)))
+        del cache
+        codec.close()
+    torch.cuda.synchronize()
+    return dict(workload=describe(w), rows=out,
+                channels="per KV head, the d/2 highest mean-square channels of the keys (after "
+                         "RoPE) and of the values over the whole prefill")
+
+
 def ncu_traffic(kernel: str):
     """Per-launch DRAM bytes of ``kernel`` from the committed ncu summary, or
     None when the kernel's source changed after the capture."""
@@ -874,6 +1097,9 @@ def run_only(args) -> int:
         r = {name: quality_extra(name) for name in ("tiny", "llama_decode", "esm_prefill", "long_decode")}
         r["llama_decode_without_outliers"] = quality_extra(
             "llama_decode", overrides=dict(n_outliers=0, sigma_scale=None))
+        r["llama_decode_outlier_split"] = split_quality_extra("llama_decode")
+    elif args.only == "decode_split":
+        r = {rate: split_decode_extra(pk, rate) for rate in SPLIT_RATES}
     else:
         from rotated_codebook_kv_tq_b200 import synth
         if args.search_rows:
@@ -995,6 +1221,10 @@ def main():
             extras["vector_search"] = search_extra(pk)
         except Exception as e:
             extras["vector_search"] = dict(error=repr(e))
+        try:
+            extras["decode_split_2.5bit"] = split_decode_extra(pk, "2.5")
+        except Exception as e:
+            extras["decode_split_2.5bit"] = dict(error=repr(e))
         line["extras"] = extras
     if rank == 0:
         print(json.dumps(line))
