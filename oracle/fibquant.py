@@ -29,8 +29,10 @@ Readings (the page names the parts without formulas):
   a fixed number of steps (nearest codeword, ties to the lower index; each
   codeword moves to the mean of its points, an empty cell keeps its codeword).
   Restarts: delta in {1/4, 1/2, 3/4} (rotating a start changes nothing, f is
-  radially symmetric); the restart with the smallest quadrature MSE wins, ties
-  to the earlier one.  Codewords stored as fp32.
+  radially symmetric); the restart with the smallest quadrature MSE wins, an
+  earlier one unless a later one is lower by more than a relative 1e-9 (so
+  restarts that reach the same code keep the earlier labels).  Codewords
+  stored as fp32.
 * N = 2^m with m bits per block (fixed-address planes); blocks are the
   coordinate pairs (2j, 2j + 1) of the rotated unit vector (the randomized
   Walsh-Hadamard rotation of the TurboQuant codec stands in for Haar).
@@ -59,6 +61,7 @@ RESTART_DELTAS = (0.25, 0.5, 0.75)
 GRID_NU = 256
 GRID_NA = 256
 LLOYD_STEPS = 100
+RESTART_MARGIN = 1e-9
 
 
 def pair_density(x: np.ndarray, d: int) -> np.ndarray:
@@ -157,7 +160,9 @@ def pair_codebook(d: int, bits: int) -> PairCodebook:
         for j, delta in enumerate(RESTART_DELTAS):
             cb = lloyd(start_codebook(d, 1 << bits, delta), pts)
             m = quad_mse(cb, pts)
-            if best is None or m < best[1]:
+            # a later restart wins only by a clear margin, so restarts that
+            # reach the same code (up to rounding) keep the earlier labels
+            if best is None or m < best[1] * (1.0 - RESTART_MARGIN):
                 best = (cb, m, j)
         _CACHE[key] = PairCodebook(d, bits, best[0], best[1], best[2])
     return _CACHE[key]
