@@ -375,6 +375,71 @@ int tq_dequantize_split(const tq_split *split, const tq_cache *cache_hi,
                         float *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * FibQuant k = 2: a shared vector code for pairs of rotated coordinates
+ * ("FibQuant: Quantizzazione Vettoriale Universale ...", sections 2.1-2.3).
+ *
+ * Same normalise-rotate interface as the scalar codec (nu = |x|, u = Pi x / nu
+ * with the randomized Walsh-Hadamard Pi, RoPE on keys first), but each block
+ * (u_2j, u_2j+1) is coded by its nearest codeword of a 2^m-point code of the
+ * unit disk, m bits per block: rate m/2 bits per coordinate (0.5 .. 3).  Keys
+ * and values both use it (no QJL stage); the logit is
+ *   l_j = scale * nu_j * sum_b <q'_(2b, 2b+1), c_k[idx_jb]>,  q' = Pi RoPE(q),
+ * and out = Pi^T (sum_j softmax(l)_j nu^v_j concat_b c_v[idx^v_jb]).
+ *
+ * tq_fq_build_codebook (host, no device work): the code for the law of two
+ * coordinates of a uniform point on S^{d-1}, f(x) = (d-2)/(2 pi) (1-|x|^2)^((d-4)/2):
+ * codeword n starts at radius sqrt(1 - (1 - (n + delta)/N)^(4/d)) (the
+ * Bennett-Gersho density f^(1/2)) and angle n pi (3 - sqrt 5) (golden-angle
+ * spiral), then 100 Lloyd steps on a fixed 256 x 256 quadrature of f, from
+ * delta = 1/4, 1/2, 3/4, keeping the lowest quadrature MSE.
+ *   centroids  host, 2 * 2^bits floats (x0, y0, x1, y1, ...).
+ *   mse_per_pair host, nullable: quadrature MSE per block.
+ *   Errors: TQ_ERR_INVALID_ARG for d < 4, bits outside 1..8 or NULL output.
+ *   Solved once per (d, bits) per process (about a second at 6 bits).
+ *
+ * Codec: d in {64, 128}, bits_k and bits_v (bits per block) 1..6.  The codec
+ * holds no device memory (codebooks travel as kernel parameters), so it can be
+ * created without a GPU.
+ *
+ * Cache planes (struct tq_cache, every plane 16-byte aligned):
+ *   kcode  u8 [B][Hkv][rows_cap][bits_k][d/16]: bit p of block j's code at byte
+ *          j/8, bit j%8 of plane p.   kscale fp16 [...][rows_cap][2] = (nu, 0).
+ *   vcode  u32 [B][Hkv][rows_cap/32][bits_v][d/2]: bit t%32 of word [t/32][p][j]
+ *          = bit p of block j's code of token t.   vnorm fp16 [...][rows_cap].
+ * The quantize, decode and dequantize calls take the arguments, layouts and
+ * error codes of tq_quantize_kv, tq_attention_decode and tq_dequantize.
+ * ------------------------------------------------------------------------ */
+typedef struct tq_fq_codec tq_fq_codec;
+
+typedef struct {
+  int d;
+  int bits_k;
+  int bits_v;
+  const int8_t *rotation_signs;   /* host, d entries of +1 / -1 */
+} tq_fq_codec_desc;
+
+int tq_fq_build_codebook(int d, int bits, float *centroids, double *mse_per_pair);
+int tq_fq_codec_create(const tq_fq_codec_desc *desc, tq_fq_codec **out);
+void tq_fq_codec_destroy(tq_fq_codec *codec);
+/* Host copies of the codec's codewords (x, y pairs); either pointer may be NULL. */
+int tq_fq_codec_codebooks(const tq_fq_codec *codec, float *ck, float *cv);
+int tq_fq_cache_bytes(const tq_fq_codec *codec, int B, int Hkv, int64_t rows_cap,
+                      size_t bytes[4]);
+int tq_fq_quantize_kv(const tq_fq_codec *codec, const void *k, const void *v, int dtype, int B,
+                      int Hkv, int T, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                      const float *rope_cos, const float *rope_sin, int64_t pos0,
+                      const tq_cache *cache, int64_t row0, uint32_t *status, void *stream);
+int tq_fq_attention_workspace(const tq_fq_codec *codec, int B, int Hq, int num_splits,
+                              size_t *bytes);
+int tq_fq_attention_decode(const tq_fq_codec *codec, const void *q, int dtype, int B, int Hq,
+                           int Hkv, const tq_cache *cache, const int32_t *seq_lens,
+                           int max_seq_len, float scale, const float *rope_cos,
+                           const float *rope_sin, int num_splits, void *workspace,
+                           size_t ws_bytes, float *out, void *stream);
+int tq_fq_dequantize(const tq_fq_codec *codec, const tq_cache *cache, int which, int64_t row0,
+                     int64_t rows, float *out, void *stream);
+
+/* ------------------------------------------------------------------------
  * Profiling hooks (no counterpart on the pages; used by the benchmark).
  * tq_set_timing_events: when both are non-NULL, every later
  *   tq_attention_decode / tq_attention_logits on this thread records `start`

@@ -496,4 +496,141 @@ int tq_dequantize_split(const tq_split *s, const tq_cache *cache_hi, const tq_ca
   return TQ_OK;
 }
 
+// ---------------------------------------------------------------------------
+// FibQuant k = 2 codec
+// ---------------------------------------------------------------------------
+
+int tq_fq_build_codebook(int d, int bits, float *centroids, double *mse_per_pair) {
+  if (!centroids) return tq_fail(TQ_ERR_INVALID_ARG, "fq codebook: NULL output");
+  std::vector<double> c;
+  double mse = 0.0;
+  if (!tqhost::fq_pair_codebook(d, bits, c, mse))
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq codebook: need d >= 4 and 1 <= bits <= 8");
+  for (size_t i = 0; i < c.size(); ++i) centroids[i] = static_cast<float>(c[i]);
+  if (mse_per_pair) *mse_per_pair = mse;
+  return TQ_OK;
+}
+
+int tq_fq_codec_create(const tq_fq_codec_desc *desc, tq_fq_codec **out) {
+  if (!desc || !out || !desc->rotation_signs)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq codec: NULL descriptor, output or signs");
+  *out = nullptr;
+  const int d = desc->d;
+  if (d != 64 && d != 128) return tq_fail(TQ_ERR_UNSUPPORTED, "fq codec: d must be 64 or 128");
+  if (desc->bits_k < 1 || desc->bits_k > FQ_MAX_BITS || desc->bits_v < 1 || desc->bits_v > FQ_MAX_BITS)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "fq codec: bits per block must be 1..6");
+  tq_fq_codec *c = new tq_fq_codec();
+  c->d = d;
+  c->bits_k = desc->bits_k;
+  c->bits_v = desc->bits_v;
+  std::memset(&c->books, 0, sizeof(c->books));
+  for (int i = 0; i < d; ++i) {
+    const int s = desc->rotation_signs[i];
+    if (s != 1 && s != -1) {
+      delete c;
+      return tq_fail(TQ_ERR_INVALID_ARG, "fq codec: rotation signs must be +1 or -1");
+    }
+    if (s < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
+  }
+  std::vector<double> ck, cv;
+  tqhost::fq_pair_codebook(d, c->bits_k, ck, c->mse_k);
+  tqhost::fq_pair_codebook(d, c->bits_v, cv, c->mse_v);
+  for (int n = 0; n < (1 << c->bits_k); ++n)
+    c->books.ck[n] = make_float2(static_cast<float>(ck[2 * n]), static_cast<float>(ck[2 * n + 1]));
+  for (int n = 0; n < (1 << c->bits_v); ++n)
+    c->books.cv[n] = make_float2(static_cast<float>(cv[2 * n]), static_cast<float>(cv[2 * n + 1]));
+  c->books.bits_k = c->bits_k;
+  c->books.bits_v = c->bits_v;
+  *out = c;
+  return TQ_OK;
+}
+
+void tq_fq_codec_destroy(tq_fq_codec *codec) { delete codec; }
+
+int tq_fq_codec_codebooks(const tq_fq_codec *c, float *ck, float *cv) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "fq codebooks: NULL codec");
+  if (ck) std::memcpy(ck, c->books.ck, sizeof(float) * 2 * (1 << c->bits_k));
+  if (cv) std::memcpy(cv, c->books.cv, sizeof(float) * 2 * (1 << c->bits_v));
+  return TQ_OK;
+}
+
+int tq_fq_cache_bytes(const tq_fq_codec *c, int B, int Hkv, int64_t rows_cap, size_t bytes[4]) {
+  if (!c || !bytes || B <= 0 || Hkv <= 0 || rows_cap <= 0 || rows_cap % 32)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq cache_bytes: bad shape (rows_cap multiple of 32)");
+  const size_t rows = static_cast<size_t>(B) * Hkv * rows_cap;
+  bytes[0] = rows * c->bits_k * (c->d / 16);
+  bytes[1] = rows * 2 * sizeof(uint16_t);
+  bytes[2] = rows / 32 * c->bits_v * (c->d / 2) * sizeof(uint32_t);
+  bytes[3] = rows * sizeof(uint16_t);
+  return TQ_OK;
+}
+
+int tq_fq_quantize_kv(const tq_fq_codec *c, const void *k, const void *v, int dtype, int B,
+                      int Hkv, int T, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                      const float *rope_cos, const float *rope_sin, int64_t pos0,
+                      const tq_cache *cache, int64_t row0, uint32_t *status, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: NULL codec");
+  if (int e = check_cache(nullptr, cache)) return e;
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: dtype");
+  if (B != cache->B || Hkv != cache->Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: B/Hkv differ from the cache's");
+  if (T < 0 || row0 < 0 || row0 + T > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: rows [row0, row0+T) outside the cache");
+  if (T == 0) return TQ_OK;
+  if (!k || !v) return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: NULL k or v");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: rope_cos and rope_sin go together");
+  if (rope_cos && pos0 < 0) return tq_fail(TQ_ERR_INVALID_ARG, "fq quantize: pos0 < 0");
+  const size_t es = dtype == TQ_BF16 ? 2 : 4;
+  if (!aligned(k, es) || !aligned(v, es))
+    return tq_fail(TQ_ERR_ALIGNMENT, "fq quantize: k/v not aligned to their element size");
+  return launch_fq_quantize(c, k, v, dtype, B, Hkv, T, stride_b, stride_h, stride_t, rope_cos,
+                            rope_sin, pos0, cache, row0, status, static_cast<cudaStream_t>(stream));
+}
+
+int tq_fq_attention_workspace(const tq_fq_codec *c, int B, int Hq, int num_splits, size_t *bytes) {
+  if (!c || !bytes || B <= 0 || Hq <= 0 || num_splits < 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq workspace: bad arguments");
+  *bytes = fq_workspace_bytes(c, B, Hq, num_splits > 0 ? num_splits : 64);
+  return TQ_OK;
+}
+
+int tq_fq_attention_decode(const tq_fq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                           const tq_cache *cache, const int32_t *seq_lens, int max_seq_len,
+                           float scale, const float *rope_cos, const float *rope_sin,
+                           int num_splits, void *workspace, size_t ws_bytes, float *out,
+                           void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: NULL codec");
+  if (int e = check_cache(nullptr, cache)) return e;
+  if (!q || !out || !workspace) return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: NULL q/out/workspace");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: dtype");
+  if (B != cache->B || Hkv != cache->Hkv || Hq <= 0 || Hq % Hkv)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: B/Hkv differ from the cache's or Hq % Hkv != 0");
+  if (max_seq_len < 1 || max_seq_len > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: max_seq_len outside 1..rows_cap");
+  if (!std::isfinite(scale)) return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: scale not finite");
+  if ((rope_cos == nullptr) != (rope_sin == nullptr))
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: rope_cos and rope_sin go together");
+  const int splits = pick_splits(num_splits, max_seq_len, B, Hkv);
+  if (splits > 512) return tq_fail(TQ_ERR_INVALID_ARG, "fq decode: num_splits must be <= 512");
+  if (fq_workspace_bytes(c, B, Hq, splits) > ws_bytes)
+    return tq_fail(TQ_ERR_WORKSPACE, "fq decode: workspace smaller than tq_fq_attention_workspace()");
+  if (!aligned(workspace, 16)) return tq_fail(TQ_ERR_ALIGNMENT, "fq decode: workspace alignment");
+  if (!aligned(out, 4) || !aligned(q, dtype == TQ_BF16 ? 2 : 4))
+    return tq_fail(TQ_ERR_ALIGNMENT, "fq decode: q/out alignment");
+  return launch_fq_decode(c, q, dtype, B, Hq, Hkv, cache, seq_lens, max_seq_len, scale, rope_cos,
+                          rope_sin, splits, workspace, out, static_cast<cudaStream_t>(stream));
+}
+
+int tq_fq_dequantize(const tq_fq_codec *c, const tq_cache *cache, int which, int64_t row0,
+                     int64_t rows, float *out, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "fq dequantize: NULL codec");
+  if (int e = check_cache(nullptr, cache)) return e;
+  if (which != 0 && which != 1) return tq_fail(TQ_ERR_INVALID_ARG, "fq dequantize: which is 0 or 1");
+  if (row0 < 0 || rows < 0 || row0 + rows > cache->rows_cap)
+    return tq_fail(TQ_ERR_INVALID_ARG, "fq dequantize: rows outside the cache");
+  if (rows > 0 && !out) return tq_fail(TQ_ERR_INVALID_ARG, "fq dequantize: NULL out");
+  return launch_fq_dequant(c, cache, which, row0, rows, out, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -11,6 +11,8 @@
 
 namespace tqhost {
 bool lloyd_max(int d, int bits, std::vector<double> &c, std::vector<double> &t, double &mse);
+// FibQuant k = 2 pair codebook (fq_codebook.cpp): c = x0, y0, x1, y1, ...
+bool fq_pair_codebook(int d, int bits, std::vector<double> &c, double &mse);
 }
 
 // Largest head dim the kernels are instantiated for.
@@ -57,6 +59,23 @@ struct tq_codec {
   uint32_t digit_k[3][4], digit_v[3][4];
   float digit_k_scale, digit_v_scale;
   int device;
+};
+
+// FibQuant k = 2 codec: 2^bits codewords of the plane per block of two rotated
+// coordinates, passed by value to its kernels.
+constexpr int FQ_MAX_BITS = 6;
+struct FqBooks {
+  float2 ck[1 << FQ_MAX_BITS];   // key codewords
+  float2 cv[1 << FQ_MAX_BITS];   // value codewords
+  uint32_t dneg[4];              // bit i set <=> D_i = -1 (d <= 128)
+  int bits_k, bits_v;
+};
+
+struct tq_fq_codec {
+  int d;
+  int bits_k, bits_v;
+  double mse_k, mse_v;   // quadrature MSE per block of the two codebooks
+  FqBooks books;
 };
 
 // Launch `kern` on `stream` allowing programmatic dependent launch: the kernel
@@ -111,6 +130,18 @@ int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int 
 int launch_dequant(const tq_codec *c, const tq_cache *cache, int which, int64_t row0,
                    int64_t rows, float *out, cudaStream_t stream,
                    const TqRowMap &map = TqRowMap());
+// FibQuant k = 2 kernels (fq.cu).
+int launch_fq_quantize(const tq_fq_codec *c, const void *k, const void *v, int dtype, int B, int H,
+                       int T, int64_t sb, int64_t sh, int64_t st, const float *rc,
+                       const float *rs, int64_t pos0, const tq_cache *cache, int64_t row0,
+                       uint32_t *status, cudaStream_t stream);
+size_t fq_workspace_bytes(const tq_fq_codec *c, int B, int Hq, int splits);
+int launch_fq_decode(const tq_fq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
+                     const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,
+                     const float *rc, const float *rs, int splits, void *ws, float *out,
+                     cudaStream_t stream);
+int launch_fq_dequant(const tq_fq_codec *c, const tq_cache *cache, int which, int64_t row0,
+                      int64_t rows, float *out, cudaStream_t stream);
 // Decode over an outlier-channel split cache (split.cu).
 size_t split_workspace_bytes(const tq_codec *hi, int B, int Hq, int splits);
 int launch_decode_split(const tq_codec *hi, const tq_codec *lo, const int16_t *channels,

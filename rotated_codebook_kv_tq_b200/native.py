@@ -27,7 +27,10 @@ EXPORTS = [
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
     "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_split_channels",
     "tq_quantize_kv_split", "tq_attention_split_workspace", "tq_attention_decode_split",
-    "tq_dequantize_split", "tq_set_timing_events", "tq_launch_count", "tq_last_error",
+    "tq_dequantize_split", "tq_fq_build_codebook", "tq_fq_codec_create", "tq_fq_codec_destroy",
+    "tq_fq_codec_codebooks", "tq_fq_cache_bytes", "tq_fq_quantize_kv", "tq_fq_attention_workspace",
+    "tq_fq_attention_decode", "tq_fq_dequantize", "tq_set_timing_events", "tq_launch_count",
+    "tq_last_error",
 ]
 
 
@@ -47,6 +50,11 @@ class CacheDesc(ctypes.Structure):
     _fields_ = [("kcode", ctypes.c_void_p), ("kscale", ctypes.c_void_p),
                 ("vcode", ctypes.c_void_p), ("vnorm", ctypes.c_void_p),
                 ("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("rows_cap", ctypes.c_int64)]
+
+
+class FqCodecDesc(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("bits_k", ctypes.c_int), ("bits_v", ctypes.c_int),
+                ("rotation_signs", ctypes.c_void_p)]
 
 
 class SplitDesc(ctypes.Structure):
@@ -98,6 +106,16 @@ def lib() -> ctypes.CDLL:
         L.tq_attention_decode_split.argtypes = [sp, vp, i32, i32, i32, i32, cp, cp, vp, i32,
                                                 ctypes.c_float, vp, vp, i32, vp, sz, vp, vp]
         L.tq_dequantize_split.argtypes = [sp, cp, cp, i32, i64, i64, vp, vp]
+        L.tq_fq_build_codebook.argtypes = [i32, i32, vp, vp]
+        L.tq_fq_codec_create.argtypes = [ctypes.POINTER(FqCodecDesc), ctypes.POINTER(vp)]
+        L.tq_fq_codec_destroy.argtypes = [vp]
+        L.tq_fq_codec_destroy.restype = None
+        L.tq_fq_codec_codebooks.argtypes = [vp, vp, vp]
+        L.tq_fq_cache_bytes.argtypes = [vp, i32, i32, i64, ctypes.POINTER(sz)]
+        L.tq_fq_quantize_kv.argtypes = L.tq_quantize_kv.argtypes
+        L.tq_fq_attention_workspace.argtypes = [vp, i32, i32, i32, ctypes.POINTER(sz)]
+        L.tq_fq_attention_decode.argtypes = L.tq_attention_decode.argtypes
+        L.tq_fq_dequantize.argtypes = L.tq_dequantize.argtypes
         L.tq_set_timing_events.argtypes = [vp, vp]
         L.tq_launch_count.argtypes = []
         L.tq_launch_count.restype = ctypes.c_uint64
@@ -416,6 +434,102 @@ def dequantize_split(split: Split, cache_hi: Cache, cache_lo: Cache, which: int,
     sd, dh, dl = split.desc(), cache_hi.desc(), cache_lo.desc()
     check(lib().tq_dequantize_split(ctypes.byref(sd), ctypes.byref(dh), ctypes.byref(dl), which,
                                     row0, rows, _ptr(out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- FibQuant k = 2
+
+def fq_build_codebook(d: int, bits: int):
+    """tq_fq_build_codebook -> (codewords fp32 [2^bits, 2], quadrature MSE per block)."""
+    c = np.zeros((1 << bits, 2), np.float32)
+    mse = ctypes.c_double(0.0)
+    check(lib().tq_fq_build_codebook(d, bits, c.ctypes.data, ctypes.addressof(mse)))
+    return c, mse.value
+
+
+class FqCodec:
+    """Owns a ``tq_fq_codec`` (host only: its codebooks travel as kernel
+    parameters)."""
+
+    def __init__(self, d: int, bits_k: int, bits_v: int, rotation_signs: np.ndarray):
+        self.d, self.bits_k, self.bits_v = d, bits_k, bits_v
+        signs = np.ascontiguousarray(rotation_signs, dtype=np.int8)
+        desc = FqCodecDesc(d, bits_k, bits_v, signs.ctypes.data)
+        h = ctypes.c_void_p()
+        check(lib().tq_fq_codec_create(ctypes.byref(desc), ctypes.byref(h)))
+        self.handle = h
+
+    def codebooks(self):
+        ck = np.zeros((1 << self.bits_k, 2), np.float32)
+        cv = np.zeros((1 << self.bits_v, 2), np.float32)
+        check(lib().tq_fq_codec_codebooks(self.handle, ck.ctypes.data, cv.ctypes.data))
+        return ck, cv
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            lib().tq_fq_codec_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def fq_alloc_cache(codec: FqCodec, B: int, Hkv: int, rows_cap: int, device="cuda") -> Cache:
+    import torch
+    d = codec.d
+    return Cache(
+        kcode=torch.zeros((B, Hkv, rows_cap, codec.bits_k, d // 16), dtype=torch.uint8, device=device),
+        kscale=torch.zeros((B, Hkv, rows_cap, 2), dtype=torch.float16, device=device),
+        vcode=torch.zeros((B, Hkv, rows_cap // 32, codec.bits_v, d // 2), dtype=torch.int32, device=device),
+        vnorm=torch.zeros((B, Hkv, rows_cap), dtype=torch.float16, device=device),
+        B=B, Hkv=Hkv, rows_cap=rows_cap)
+
+
+def fq_cache_bytes(codec: FqCodec, B: int, Hkv: int, rows_cap: int):
+    out = (ctypes.c_size_t * 4)()
+    check(lib().tq_fq_cache_bytes(codec.handle, B, Hkv, rows_cap, out))
+    return list(out)
+
+
+def fq_quantize_kv(codec: FqCodec, k, v, cache: Cache, row0: int = 0, rope=None, pos0: int = 0,
+                   status=None, stream=None) -> None:
+    B, H, T, d = k.shape
+    if tuple(v.shape) != tuple(k.shape) or v.stride() != k.stride() or k.stride(3) != 1:
+        raise ValueError("k and v need the same shape and strides, last dim contiguous")
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    check(lib().tq_fq_quantize_kv(codec.handle, k.data_ptr(), v.data_ptr(), _dtype_code(k), B, H,
+                                  T, k.stride(0), k.stride(1), k.stride(2), _ptr(rc), _ptr(rs),
+                                  pos0, ctypes.byref(desc), row0, _ptr(status), _stream(stream)))
+
+
+def fq_attention_workspace(codec: FqCodec, B: int, Hq: int, num_splits: int) -> int:
+    n = ctypes.c_size_t(0)
+    check(lib().tq_fq_attention_workspace(codec.handle, B, Hq, num_splits, ctypes.byref(n)))
+    return n.value
+
+
+def fq_attention_decode(codec: FqCodec, q, cache: Cache, max_seq_len: int, scale: float, out,
+                        workspace, seq_lens=None, rope=None, num_splits: int = 0,
+                        stream=None) -> None:
+    B, Hq, d = q.shape
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(lib().tq_fq_attention_decode(codec.handle, q.data_ptr(), _dtype_code(q), B, Hq,
+                                       cache.Hkv, ctypes.byref(desc), _ptr(seq_lens), max_seq_len,
+                                       float(scale), _ptr(rc), _ptr(rs), num_splits,
+                                       workspace.data_ptr(), ws_bytes, out.data_ptr(),
+                                       _stream(stream)))
+
+
+def fq_dequantize(codec: FqCodec, cache: Cache, which: int, row0: int, rows: int, out,
+                  stream=None) -> None:
+    desc = cache.desc()
+    check(lib().tq_fq_dequantize(codec.handle, ctypes.byref(desc), which, row0, rows, _ptr(out),
+                                 _stream(stream)))
 
 
 def set_timing_events(start=None, stop=None) -> None:

@@ -126,3 +126,33 @@ def test_split_calls_validate_before_device_work(L):
     assert L.tq_dequantize_split(ctypes.byref(empty), ctypes.byref(cd), ctypes.byref(cd), 0, 0, 1,
                                  None, None) == native.TQ_ERR_INVALID_ARG
     assert b"split" in L.tq_last_error()
+
+
+@pytest.mark.parametrize("d,bits", [(64, 1), (64, 3), (128, 2), (128, 4), (128, 6)])
+def test_fq_host_codebook_matches_oracle(L, d, bits):
+    """tq_fq_build_codebook (host C++) against the oracle's FibQuant k = 2 code:
+    same start, quadrature, Lloyd steps and restart rule, written separately."""
+    from oracle import fibquant as ofq
+    c, mse = native.fq_build_codebook(d, bits)
+    ref = ofq.pair_codebook(d, bits)
+    np.testing.assert_allclose(c.astype(np.float64), ref.centroids, rtol=0, atol=1e-7)
+    assert abs(mse / ref.mse_per_pair - 1) < 1e-9
+
+
+def test_fq_codec_is_host_only_and_validates(L):
+    signs = synth.rotation_signs(128, 0)
+    c = native.FqCodec(128, 4, 3, signs)
+    ck, cv = c.codebooks()
+    ref_k, _ = native.fq_build_codebook(128, 4)
+    assert np.array_equal(ck, ref_k) and cv.shape == (8, 2)
+    assert native.fq_cache_bytes(c, 1, 2, 64) == [2 * 64 * 4 * 8, 2 * 64 * 4, 2 * 2 * 3 * 64 * 4, 2 * 64 * 2]
+    c.close()
+    for d, bk, bv, code in [(96, 2, 2, native.TQ_ERR_UNSUPPORTED), (128, 0, 2, native.TQ_ERR_UNSUPPORTED),
+                            (128, 2, 7, native.TQ_ERR_UNSUPPORTED)]:
+        with pytest.raises(native.TqError) as e:
+            native.FqCodec(d, bk, bv, synth.rotation_signs(d, 0))
+        assert e.value.code == code
+    bad = signs.copy()
+    bad[5] = 0
+    with pytest.raises(native.TqError):
+        native.FqCodec(128, 2, 2, bad)
