@@ -45,7 +45,8 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
-                                      "decode_llama", "vector_search", "quality", "decode_split"],
+                                      "decode_llama", "vector_search", "quality", "decode_split",
+                                      "decode_fibquant", "quality_fibquant"],
                    help="run one extra workload alone and print its JSON (1 GPU)")
     p.add_argument("--search-rows", type=int, default=0,
                    help="vector-search database rows for --only vector_search (default 10^6)")
@@ -478,6 +479,20 @@ def cpu_baselines(seconds: float = 1.0) -> dict:
     out["decode_split_2.5bit"] = entry("tokens/s", t1, tn, th, lambda t: w.B / (t * w.T / rows),
                                        f"one split decode step over the first {rows} of {w.T} "
                                        f"tokens, all {w.B * w.Hq} query heads, time x {w.T}/{rows}")
+    # FibQuant k = 2 at 2 bits per coordinate on the Llama shape, same sampling
+    from oracle import fibquant as ofq
+    fqc = ofq.make_codec(w.d, 4, 4, synth.rotation_signs(w.d, w.seed))
+    fcache = ofq.empty_cache(fqc, w.B, w.Hkv, rows)
+    ofq.quantize_into(fcache, K64[:, :, :rows - 1], V64[:, :, :rows - 1], fqc, rope=rope)
+
+    def fq_step():
+        ofq.quantize_into(fcache, K64[:, :, rows - 1:], V64[:, :, rows - 1:], fqc, rope=rope,
+                          pos0=rows - 1, row0=rows - 1)
+        ofq.decode(q, fcache, fqc, [rows] * w.B, 1.0 / math.sqrt(w.d), rope=rope)
+    t1, tn, th = _one_and_all(fq_step, seconds)
+    out["decode_fibquant_2bit"] = entry("tokens/s", t1, tn, th, lambda t: w.B / (t * w.T / rows),
+                                        f"one FibQuant decode step over the first {rows} of {w.T} "
+                                        f"tokens, all {w.B * w.Hq} query heads, time x {w.T}/{rows}")
     # ESM-2-shaped prefill quantize: two (batch, head) pairs of the 320
     w = synth.WORKLOADS["esm_prefill"]
     ww = w.scaled(B=1, Hq=2, Hkv=2)
@@ -991,6 +1006,163 @@ def split_quality_extra(wname: str = "llama_decode"):
                          "RoPE) and of the values over the whole prefill")
 
 
+# ---------------------------------------------------------------------------
+# FibQuant k = 2 ("FibQuant ...", sections 2.1-2.3: a shared code for pairs of
+# rotated coordinates, rate log2(N)/2 bits per coordinate)
+# ---------------------------------------------------------------------------
+
+def fq_row_bytes(codec) -> int:
+    return codec.bits_k * codec.d // 16 + 4 + codec.bits_v * codec.d // 16 + 2
+
+
+class FqBench:
+    """Decode step with the FibQuant codec: quantize-append of the new token,
+    then tq_fq_attention_decode (same interface as DecodeBench for time_decode)."""
+
+    def __init__(self, w, bits: int, n_sets: int):
+        import torch
+        from rotated_codebook_kv_tq_b200 import native, synth
+        self.w, self.native, self.n_sets = w, native, n_sets
+        self.codec = native.FqCodec(w.d, bits, bits, synth.rotation_signs(w.d, w.seed))
+        T = w.T
+        self.rows_cap = (T + 31) // 32 * 32
+        K, V = synth.kv_inputs_torch(w, T=T)
+        r = synth.rope_for(w, self.rows_cap)
+        self.rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+        self.caches = []
+        for _ in range(n_sets):
+            c = native.fq_alloc_cache(self.codec, w.B, w.Hkv, self.rows_cap)
+            native.fq_quantize_kv(self.codec, K[:, :, :T - 1], V[:, :, :T - 1], c, rope=self.rope)
+            self.caches.append(c)
+        self.knew = K[:, :, T - 1:T].contiguous()
+        self.vnew = V[:, :, T - 1:T].contiguous()
+        self.q = synth.query_inputs_torch(w)[:, :, 0].contiguous()
+        self.scale = 1.0 / math.sqrt(w.d)
+        self.splits = w.num_splits
+        self.ws = torch.empty(native.fq_attention_workspace(self.codec, w.B, w.Hq, self.splits),
+                              dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        self.row_bytes = fq_row_bytes(self.codec)
+        torch.cuda.synchronize()
+
+    def step(self, s: int) -> None:
+        w, n = self.w, self.native
+        c = self.caches[s % self.n_sets]
+        n.fq_quantize_kv(self.codec, self.knew, self.vnew, c, row0=w.T - 1, rope=self.rope,
+                         pos0=w.T - 1)
+        n.fq_attention_decode(self.codec, self.q, c, w.T, self.scale, self.out, self.ws,
+                              rope=self.rope, num_splits=self.splits)
+
+    def cache_bytes_per_step(self) -> int:
+        return self.w.B * self.w.Hkv * self.w.T * self.row_bytes
+
+
+def fq_decode_extra(pk: dict, bits: int = 4, steps: int = 40, warmup: int = 5):
+    """Llama-shaped decode over a FibQuant cache (bits per pair for keys and
+    values; bits/2 per coordinate): tokens/s and the chunk kernel's roofline."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import synth
+    w = synth.WORKLOADS["llama_decode"]
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    per_set = w.B * w.Hkv * ((w.T + 31) // 32 * 32) * (2 * bits * w.d // 16 + 6)
+    bench = FqBench(w, bits, max(1, math.ceil(3 * l2 / per_set)))
+
+    class _Null:
+        def start(self):
+            pass
+
+        def stop(self):
+            return {}
+
+    total, kern, per_step, _ = time_decode(bench, steps, warmup, 1, _Null())
+    alg = bench.cache_bytes_per_step()
+    res = dict(workload=f"llama_decode with FibQuant k=2, {bits} bits per pair ({bits / 2:g} per "
+                        f"coordinate) for keys and values: B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} "
+                        f"T={w.T}",
+               us_per_step=total / steps * 1e6, tokens_per_s=w.B * steps / total,
+               launches_per_step=per_step,
+               roofline=dict(bound="hbm", achieved=alg / kern / 1e9, peak=pk["hbm"], unit="GB/s",
+                             frac=alg / kern / 1e9 / pk["hbm"], algorithmic_bytes=alg,
+                             bytes_per_token_head=bench.row_bytes, kernel="fq_chunk_kernel",
+                             kernel_us=kern * 1e6),
+               l2=f"rotating {bench.n_sets} caches ({bench.n_sets * alg / 1e6:.0f} MB)")
+    del bench
+    torch.cuda.empty_cache()
+    return res
+
+
+def fq_quality_extra(wname: str = "llama_decode", overrides=None):
+    """relMSE_K, relMSE_V and output cosine (as in quality_extra) of FibQuant
+    k = 2 at 0.5 .. 3 bits per coordinate beside the scalar MSE-only codec
+    (TQ-KV) at 1, 2 and 3 bits, on the same inputs."""
+    import torch
+    from rotated_codebook_kv_tq_b200 import native, synth
+    w = synth.WORKLOADS[wname]
+    if overrides:
+        w = w.scaled(**overrides)
+    rows_cap = (w.T + 31) // 32 * 32
+    K, V = synth.kv_inputs_torch(w)
+    q = synth.query_inputs_torch(w, Lq=1)[:, :, 0].contiguous()
+    r = synth.rope_for(w, rows_cap)
+    rope = None if r is None else (torch.from_numpy(r[0]).cuda(), torch.from_numpy(r[1]).cuda())
+    Kf, Vf, qf = K.float(), V.float(), q.float()
+    if rope is not None:
+        Kf = _rope_rows(Kf, rope[0][:w.T], rope[1][:w.T])
+        qf = _rope_rows(qf, rope[0][w.T - 1], rope[1][w.T - 1])
+    scale = 1.0 / math.sqrt(w.d)
+    Ke = Kf.repeat_interleave(w.G, dim=1)
+    Ve = Vf.repeat_interleave(w.G, dim=1)
+    p = torch.softmax(torch.einsum("bhd,bhtd->bht", qf, Ke) * scale, dim=-1)
+    o_ref = torch.einsum("bht,bhtd->bhd", p, Ve)
+    del Ke, Ve, p
+    D = synth.rotation_signs(w.d, w.seed)
+
+    def scores(deq, decode):
+        rel = {}
+        for which, x in ((0, Kf), (1, Vf)):
+            xh = torch.empty((w.B, w.Hkv, w.T, w.d), dtype=torch.float32, device="cuda")
+            deq(which, xh)
+            rel["K" if which == 0 else "V"] = float(((xh - x) ** 2).sum() / (x ** 2).sum())
+            del xh
+        o = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        decode(o)
+        cos = torch.nn.functional.cosine_similarity(o, o_ref, dim=-1)
+        return dict(relMSE_K=rel["K"], relMSE_V=rel["V"], output_cosine_mean=float(cos.mean()),
+                    output_cosine_min=float(cos.min()))
+
+    out = {}
+    for bits in (1, 2, 3, 4, 5, 6):
+        c = native.FqCodec(w.d, bits, bits, D)
+        cache = native.fq_alloc_cache(c, w.B, w.Hkv, rows_cap)
+        native.fq_quantize_kv(c, K, V, cache, rope=rope)
+        ws = torch.empty(native.fq_attention_workspace(c, w.B, w.Hq, w.num_splits), dtype=torch.uint8,
+                         device="cuda")
+        out[f"fibquant_{bits / 2:g}"] = dict(
+            bits_per_coordinate=bits / 2,
+            **scores(lambda which, xh: native.fq_dequantize(c, cache, which, 0, w.T, xh),
+                     lambda o: native.fq_attention_decode(c, q, cache, w.T, scale, o, ws, rope=rope,
+                                                          num_splits=w.num_splits)))
+        del cache
+        c.close()
+    for bits in (1, 2, 3):
+        c = native.Codec(w.d, bits, False, bits, D, None)
+        cache = native.alloc_cache(c, w.B, w.Hkv, rows_cap)
+        native.quantize_kv(c, K, V, cache, rope=rope)
+        ws = torch.empty(native.attention_workspace(c, w.B, w.Hq, w.num_splits), dtype=torch.uint8,
+                         device="cuda")
+        out[f"scalar_{bits}"] = dict(
+            bits_per_coordinate=float(bits),
+            **scores(lambda which, xh: native.dequantize(c, cache, which, 0, w.T, xh),
+                     lambda o: native.attention_decode(c, q, cache, w.T, scale, o, ws, rope=rope,
+                                                       num_splits=w.num_splits)))
+        del cache
+        c.close()
+    torch.cuda.synchronize()
+    return dict(workload=describe(w), rows=out,
+                note="FibQuant keys and values both use the pair code (no QJL); scalar rows are "
+                     "the MSE-only key codec (TQ-KV) at the same bits for keys and values")
+
+
 def ncu_traffic(kernel: str):
     """Per-launch DRAM bytes of ``kernel`` from the committed ncu summary, or
     None when the kernel's source changed after the capture."""
@@ -1100,6 +1272,12 @@ def run_only(args) -> int:
         r["llama_decode_outlier_split"] = split_quality_extra("llama_decode")
     elif args.only == "decode_split":
         r = {rate: split_decode_extra(pk, rate) for rate in SPLIT_RATES}
+    elif args.only == "decode_fibquant":
+        r = {f"{b / 2:g}": fq_decode_extra(pk, b) for b in (2, 4, 6)}
+    elif args.only == "quality_fibquant":
+        r = dict(llama_decode=fq_quality_extra("llama_decode"),
+                 llama_decode_without_outliers=fq_quality_extra(
+                     "llama_decode", overrides=dict(n_outliers=0, sigma_scale=None)))
     else:
         from rotated_codebook_kv_tq_b200 import synth
         if args.search_rows:
@@ -1225,6 +1403,10 @@ def main():
             extras["decode_split_2.5bit"] = split_decode_extra(pk, "2.5")
         except Exception as e:
             extras["decode_split_2.5bit"] = dict(error=repr(e))
+        try:
+            extras["decode_fibquant_2bit"] = fq_decode_extra(pk, 4)
+        except Exception as e:
+            extras["decode_fibquant_2bit"] = dict(error=repr(e))
         line["extras"] = extras
     if rank == 0:
         print(json.dumps(line))
