@@ -75,13 +75,16 @@ class Codec:
 
 
 def make_codec(d: int, bits_k: int, qjl_k: bool, bits_v: int, D: np.ndarray,
-               S_bf16: Optional[np.ndarray]) -> Codec:
+               S_bf16: Optional[np.ndarray], Pi: Optional[np.ndarray] = None) -> Codec:
+    """Pi (optional): a dense orthogonal rotation used instead of the
+    randomized Walsh-Hadamard H diag(D) / sqrt(d) (e.g. rotation.haar_rotation)."""
     mse_k = bits_k - 1 if qjl_k else bits_k
     if mse_k < 1 or bits_v < 1:
         raise ValueError("each codebook needs at least one bit")
     S = synth.bf16_bits_to_f32(S_bf16).astype(np.float64) if qjl_k else None
+    P = rotation_matrix(D) if Pi is None else np.asarray(Pi, np.float64)
     return Codec(d, bits_k, qjl_k, bits_v, np.asarray(D, np.int8), S,
-                 rotation_matrix(D), cbmod.codebook(d, mse_k), cbmod.codebook(d, bits_v))
+                 P, cbmod.codebook(d, mse_k), cbmod.codebook(d, bits_v))
 
 
 # ---------------------------------------------------------------------------

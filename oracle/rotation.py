@@ -63,6 +63,21 @@ def rotation_matrix(D: np.ndarray) -> np.ndarray:
     return hadamard(d) * D[None, :] / np.sqrt(d)
 
 
+def haar_rotation(G: np.ndarray) -> np.ndarray:
+    """A Haar-distributed orthogonal matrix from a square matrix G of i.i.d.
+    N(0,1) entries: the Q factor of G = QR with every diagonal entry of R made
+    positive (Q's columns scaled by sign(R_kk)); without that step the law of Q
+    depends on the QR routine's sign convention and is not Haar.  Source: the
+    shared random rotation of the theory ("Google presenta TurboQuant ...",
+    "La mecanica geometrica de TurboQuant"; "FibQuant ...", section 2.1, Haar
+    rotation)."""
+    G = np.asarray(G, dtype=np.float64)
+    q, r = np.linalg.qr(G)
+    s = np.sign(np.diag(r))
+    s[s == 0] = 1.0
+    return q * s[None, :]
+
+
 def apply_rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray, pos) -> np.ndarray:
     """Rotate-half RoPE: for i < d/2,
     x'_i = x_i cos - x_{i+d/2} sin,  x'_{i+d/2} = x_{i+d/2} cos + x_i sin,

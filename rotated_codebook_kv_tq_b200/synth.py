@@ -9,7 +9,8 @@ oracle and the library see the same bits.
 Generator: numpy PCG64 seeded with ``SeedSequence([seed, stream])``; the
 ablation page (gist.science 2607.09683, "Validazione") runs its oracle on
 PCG64 as well.  Streams: 0 = keys, 1 = values, 2 = queries,
-3 = channel scales / outlier channels, 4 = rotation signs D, 5 = QJL matrix S.
+3 = channel scales / outlier channels, 4 = rotation signs D, 5 = QJL matrix S,
+6 = the Gaussian matrix behind a dense Haar rotation.
 Draw order is row-major over [B, H, T, d].
 
 Workload recipes (shapes follow the pages' workloads; values are synthetic
@@ -37,7 +38,7 @@ from typing import Optional
 
 import numpy as np
 
-STREAM_K, STREAM_V, STREAM_Q, STREAM_SCALES, STREAM_D, STREAM_S = range(6)
+STREAM_K, STREAM_V, STREAM_Q, STREAM_SCALES, STREAM_D, STREAM_S, STREAM_HAAR = range(7)
 
 
 def generator(seed: int, stream: int) -> np.random.Generator:
@@ -85,6 +86,12 @@ def qjl_matrix_bf16(d: int, seed: int, m: Optional[int] = None) -> np.ndarray:
 # RoPE angle table (positional-encoding input of the model, computed in fp64
 # and handed to both sides as fp32)
 # ----------------------------------------------------------------------------
+
+def haar_gaussian(d: int, seed: int) -> np.ndarray:
+    """d x d i.i.d. N(0,1) fp32 (row-major): the random input of a dense Haar
+    rotation (its QR factorisation is the method's arithmetic, not done here)."""
+    return generator(seed, STREAM_HAAR).standard_normal((d, d), dtype=np.float32)
+
 
 def rope_table(t_max: int, d: int, theta: float) -> tuple[np.ndarray, np.ndarray]:
     """cos/sin tables [t_max, d/2] fp32 for rotate-half RoPE with base theta."""
