@@ -83,9 +83,19 @@ int tq_build_codebook(int d, int bits, float *centroids, float *thresholds,
  *                 qjl_k != 0.
  * bits_k          total key bits; with qjl_k the MSE stage uses bits_k - 1.
  * bits_v          value bits (TURBOQUANT_mse).
+ * rotation        host, d*d fp32 row-major Pi[i][j], nullable: a dense
+ *                 orthogonal rotation used instead of H_d diag(D) / sqrt(d)
+ *                 (the theory's shared Haar rotation: "Google presenta
+ *                 TurboQuant ...", "La mecanica geometrica de TurboQuant";
+ *                 "FibQuant ...", section 2.1; see tq_haar_rotation).  Only for
+ *                 d = 64 and 128; rotation_signs may then be NULL.  Quantize,
+ *                 decode and dequantize apply it as fp32 matrix-vector
+ *                 products; the bidirectional pass and the outlier-channel split
+ *                 return TQ_ERR_UNSUPPORTED for such a codec.  Rows of Pi must
+ *                 be orthonormal to 1e-5 (TQ_ERR_INVALID_ARG otherwise).
  * tq_codec_create solves both codebooks with tq_build_codebook and copies D,
- * S and the codebooks to the current device (the only allocation the library
- * makes); tq_codec_destroy frees them.
+ * S, the dense rotation and the codebooks to the current device (the only
+ * allocations the library makes); tq_codec_destroy frees them.
  * ------------------------------------------------------------------------ */
 typedef struct tq_codec tq_codec;
 
@@ -96,7 +106,16 @@ typedef struct {
   int bits_v;
   const int8_t *rotation_signs;
   const uint16_t *qjl_bf16;
+  const float *rotation;
 } tq_codec_desc;
+
+/* Host helper: a Haar-distributed rotation from a d x d matrix of i.i.d.
+ * N(0,1) entries (host fp32, row-major): the orthogonal factor Q of G = QR
+ * with every diagonal entry of R made positive (Householder reflections in
+ * fp64), written to rotation (host fp32 d x d, row-major).
+ * Errors: TQ_ERR_INVALID_ARG for NULL buffers, d outside 1..4096 or a
+ * non-finite entry. */
+int tq_haar_rotation(int d, const float *gaussian, float *rotation);
 
 int tq_codec_create(const tq_codec_desc *desc, tq_codec **out);
 void tq_codec_destroy(tq_codec *codec);

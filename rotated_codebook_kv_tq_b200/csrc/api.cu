@@ -130,12 +130,30 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   if (mse_k < 1 || mse_k > 4 || desc->bits_v < 1 || desc->bits_v > 4)
     return tq_fail(TQ_ERR_UNSUPPORTED,
                    "codec: key MSE bits and value bits must be 1..4 (bits_k >= 2 with QJL)");
-  if (!desc->rotation_signs) return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs required");
+  const bool dense = desc->rotation != nullptr;
+  if (dense && desc->d > 128)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "codec: a dense rotation needs d = 64 or 128");
+  if (!dense && !desc->rotation_signs)
+    return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs required without a dense rotation");
   if (desc->qjl_k && !desc->qjl_bf16)
     return tq_fail(TQ_ERR_INVALID_ARG, "codec: qjl_bf16 required when qjl_k != 0");
-  for (int i = 0; i < desc->d; ++i)
-    if (desc->rotation_signs[i] != 1 && desc->rotation_signs[i] != -1)
-      return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs entries must be +1 or -1");
+  if (desc->rotation_signs)
+    for (int i = 0; i < desc->d; ++i)
+      if (desc->rotation_signs[i] != 1 && desc->rotation_signs[i] != -1)
+        return tq_fail(TQ_ERR_INVALID_ARG, "codec: rotation_signs entries must be +1 or -1");
+  if (dense) {
+    // orthogonality to fp32 accuracy: |Pi Pi^T - I| <= 1e-5 entrywise
+    const int d = desc->d;
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k)
+          acc += static_cast<double>(desc->rotation[static_cast<size_t>(i) * d + k]) *
+                 desc->rotation[static_cast<size_t>(j) * d + k];
+        if (std::fabs(acc - (i == j ? 1.0 : 0.0)) > 1e-5)
+          return tq_fail(TQ_ERR_INVALID_ARG, "codec: the dense rotation is not orthogonal");
+      }
+  }
 
   tq_codec *c = new tq_codec();
   std::memset(&c->books, 0, sizeof(c->books));
@@ -145,6 +163,7 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   c->bits_v = desc->bits_v;
   c->mse_bits_k = mse_k;
   c->S_dev = nullptr;
+  c->rot_dev = nullptr;
   cudaGetDevice(&c->device);
 
   std::vector<double> cc, tt;
@@ -159,8 +178,31 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
   // runs over all TQ_MAX_LEVELS - 1 slots)
   for (int i = (1 << mse_k) - 1; i < TQ_MAX_LEVELS; ++i) c->books.tk[i] = INFINITY;
   for (int i = (1 << c->bits_v) - 1; i < TQ_MAX_LEVELS; ++i) c->books.tv[i] = INFINITY;
-  for (int i = 0; i < c->d; ++i)
-    if (desc->rotation_signs[i] < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
+  if (desc->rotation_signs)
+    for (int i = 0; i < c->d; ++i)
+      if (desc->rotation_signs[i] < 0) c->books.dneg[i / 32] |= 1u << (i % 32);
+  if (dense) {
+    const size_t n = static_cast<size_t>(c->d) * c->d;
+    std::vector<float> both(2 * n);
+    for (int i = 0; i < c->d; ++i)
+      for (int j = 0; j < c->d; ++j) {
+        const float v = desc->rotation[static_cast<size_t>(i) * c->d + j];
+        both[static_cast<size_t>(i) * c->d + j] = v;       // Pi, row-major
+        both[n + static_cast<size_t>(j) * c->d + i] = v;   // Pi^T, row-major
+      }
+    if (cudaMalloc(&c->rot_dev, both.size() * sizeof(float)) != cudaSuccess) {
+      delete c;
+      return tq_check_launch("codec: cudaMalloc (rotation)");
+    }
+    if (cudaMemcpy(c->rot_dev, both.data(), both.size() * sizeof(float), cudaMemcpyHostToDevice) !=
+        cudaSuccess) {
+      cudaFree(c->rot_dev);
+      delete c;
+      return tq_check_launch("codec: cudaMemcpy (rotation)");
+    }
+    c->books.pi = c->rot_dev;
+    c->books.pi_t = c->rot_dev + n;
+  }
   c->books.mse_bits_k = mse_k;
   c->books.qjl = c->qjl_k;
   walsh_coefficients(c->books.ck, mse_k, c->walsh_k, &c->walsh_k_absmax, nullptr);
@@ -190,6 +232,7 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
         }
       }
     if (cudaMalloc(&c->S_dev, both.size() * sizeof(uint16_t)) != cudaSuccess) {
+      if (c->rot_dev) cudaFree(c->rot_dev);
       delete c;
       return tq_check_launch("codec: cudaMalloc");
     }
@@ -198,6 +241,7 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
     if (cudaMemcpy(c->S_dev, both.data(), both.size() * sizeof(uint16_t), cudaMemcpyHostToDevice) !=
         cudaSuccess) {
       cudaFree(c->S_dev);
+      if (c->rot_dev) cudaFree(c->rot_dev);
       delete c;
       return tq_check_launch("codec: cudaMemcpy");
     }
@@ -209,6 +253,7 @@ int tq_codec_create(const tq_codec_desc *desc, tq_codec **out) {
 void tq_codec_destroy(tq_codec *codec) {
   if (!codec) return;
   if (codec->S_dev) cudaFree(codec->S_dev);
+  if (codec->rot_dev) cudaFree(codec->rot_dev);
   delete codec;
 }
 
@@ -338,6 +383,7 @@ int tq_attention_bidir(const tq_codec *c, const void *q, int dtype, int B, int H
                        const float *rope_sin, void *workspace, size_t ws_bytes, float *out,
                        void *stream) {
   if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: NULL codec");
+  if (c->books.pi) return tq_fail(TQ_ERR_UNSUPPORTED, "bidir: built for the Walsh-Hadamard rotation only");
   if (int e = check_cache(c, cache)) return e;
   if (!q || !out || !workspace) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: NULL q/out/workspace");
   if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_ERR_INVALID_ARG, "bidir: dtype");
@@ -376,6 +422,8 @@ int check_split(const tq_split *s, const tq_cache *chi, const tq_cache *clo) {
     return tq_fail(TQ_ERR_INVALID_ARG, "split: NULL codec or channel map");
   if (s->hi->d != s->lo->d || (s->hi->d != 64 && s->hi->d != 128))
     return tq_fail(TQ_ERR_UNSUPPORTED, "split: both codecs need the same d, 64 or 128");
+  if (s->hi->books.pi || s->lo->books.pi)
+    return tq_fail(TQ_ERR_UNSUPPORTED, "split: built for the Walsh-Hadamard rotation only");
   if (int e = check_cache(s->hi, chi)) return e;
   if (int e = check_cache(s->lo, clo)) return e;
   if (chi->B != clo->B || chi->Hkv != clo->Hkv || chi->rows_cap != clo->rows_cap)
@@ -499,6 +547,17 @@ int tq_dequantize_split(const tq_split *s, const tq_cache *cache_hi, const tq_ca
 // ---------------------------------------------------------------------------
 // FibQuant k = 2 codec
 // ---------------------------------------------------------------------------
+
+int tq_haar_rotation(int d, const float *gaussian, float *rotation) {
+  if (!gaussian || !rotation || d < 1 || d > 4096)
+    return tq_fail(TQ_ERR_INVALID_ARG, "haar: need 1 <= d <= 4096 and non-NULL buffers");
+  for (size_t i = 0; i < static_cast<size_t>(d) * d; ++i)
+    if (!std::isfinite(gaussian[i])) return tq_fail(TQ_ERR_INVALID_ARG, "haar: non-finite input");
+  std::vector<double> pi;
+  tqhost::haar_rotation(d, gaussian, pi);
+  for (size_t i = 0; i < pi.size(); ++i) rotation[i] = static_cast<float>(pi[i]);
+  return TQ_OK;
+}
 
 int tq_fq_build_codebook(int d, int bits, float *centroids, double *mse_per_pair) {
   if (!centroids) return tq_fail(TQ_ERR_INVALID_ARG, "fq codebook: NULL output");

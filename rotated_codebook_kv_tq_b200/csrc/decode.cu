@@ -88,12 +88,17 @@ __global__ void __launch_bounds__(D) qprep_kernel(DecodeArgs a) {
         x[k + HALF] = v * c + u * s;
       }
     }
-    tq_apply_signs<NPL>(x, a.books.dneg, lane);
-    tq_warp_wht<NPL>(x, lane);
-    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+    float scl = 1.0f;
+    if (a.books.pi_t != nullptr) {
+      tq_warp_dense<NPL>(x, a.books.pi_t, qs, lane);   // q' = Pi q (dense rotation)
+    } else {
+      tq_apply_signs<NPL>(x, a.books.dneg, lane);
+      tq_warp_wht<NPL>(x, lane);
+      scl = 1.0f / sqrtf(static_cast<float>(D));
+    }
 #pragma unroll
     for (int k = 0; k < NPL; ++k) {
-      x[k] *= inv_sqrt_d;
+      x[k] *= scl;
       a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
       qs[lane + 32 * k] = x[k];
     }
@@ -350,9 +355,14 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
       for (int g = 0; g < CMB; ++g) v += os[g][lane + 32 * k];
       x[k] = v;
     }
-    tq_warp_wht<NPL>(x, lane);
-    tq_apply_signs<NPL>(x, a.books.dneg, lane);
-    const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * L);
+    float norm = 1.0f / L;
+    if (a.books.pi != nullptr) {
+      tq_warp_dense<NPL>(x, a.books.pi, os[0], lane);   // Pi^T o (dense rotation)
+    } else {
+      tq_warp_wht<NPL>(x, lane);
+      tq_apply_signs<NPL>(x, a.books.dneg, lane);
+      norm /= sqrtf(static_cast<float>(D));
+    }
 #pragma unroll
     for (int k = 0; k < NPL; ++k) a.out[head * D + lane + 32 * k] = x[k] * norm;
   }

@@ -181,11 +181,16 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
         x[k + HALF] = v * c + u * s;
       }
     }
-    tq_apply_signs<TNW>(x, a.books.dneg, lane);
-    tq_warp_wht<TNW>(x, lane);
-    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(TD));
+    float scl = 1.0f;
+    if (a.books.pi_t != nullptr) {
+      tq_warp_dense<TNW>(x, a.books.pi_t, q1s, lane);   // q' = Pi q (dense rotation)
+    } else {
+      tq_apply_signs<TNW>(x, a.books.dneg, lane);
+      tq_warp_wht<TNW>(x, lane);
+      scl = 1.0f / sqrtf(static_cast<float>(TD));
+    }
 #pragma unroll
-    for (int k = 0; k < TNW; ++k) q1s[lane + 32 * k] = x[k] * inv_sqrt_d;
+    for (int k = 0; k < TNW; ++k) q1s[lane + 32 * k] = x[k] * scl;
   }
   __syncthreads();
   if (QJL) {

@@ -31,6 +31,7 @@ template <int D>
 __global__ void __launch_bounds__(DW * 32) dequant_kernel(DequantArgs a) {
   constexpr int NPL = D / 32;
   __shared__ float cs[TQ_MAX_LEVELS];
+  __shared__ float dsc[DW][D];   // dense-rotation scratch, one row per warp
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x < TQ_MAX_LEVELS)
     cs[threadIdx.x] = a.which == 0 ? a.books.ck[threadIdx.x] : a.books.cv[threadIdx.x];
@@ -85,10 +86,15 @@ __global__ void __launch_bounds__(DW * 32) dequant_kernel(DequantArgs a) {
       }
       nu = tq_half_to_f32(a.vnorm[bh * a.rows_cap + r]);
     }
-    // Pi^T y = D (H y) / sqrt(d)
-    tq_warp_wht<NPL>(y, lane);
-    tq_apply_signs<NPL>(y, a.books.dneg, lane);
-    const float f = nu / sqrtf(static_cast<float>(D));
+    // Pi^T y = D (H y) / sqrt(d), or the dense Pi^T
+    float f = nu;
+    if (a.books.pi != nullptr) {
+      tq_warp_dense<NPL>(y, a.books.pi, dsc[warp], lane);
+    } else {
+      tq_warp_wht<NPL>(y, lane);
+      tq_apply_signs<NPL>(y, a.books.dneg, lane);
+      f /= sqrtf(static_cast<float>(D));
+    }
     if (a.map.k != nullptr) {
       // outlier-channel split: coordinate i goes to channel map[h][i]
       const int16_t *m = (a.which == 0 ? a.map.k : a.map.v) + (bh % a.Hkv) * a.map.hstride;

@@ -95,10 +95,12 @@ __device__ __forceinline__ void load_row(float (&x)[NPL], const void *base, int6
   }
 }
 
-// Normalise and rotate: returns nu (0 for bad rows), u = H D x / (sqrt(d) nu).
+// Normalise and rotate: returns nu (0 for bad rows), u = H D x / (sqrt(d) nu),
+// or u = Pi x / nu with a dense rotation (scratch: this warp's d floats of
+// shared memory, used only then).
 template <int NPL>
-__device__ __forceinline__ float normalize_rotate(float (&x)[NPL], const uint32_t *dneg,
-                                                  int lane, bool &bad) {
+__device__ __forceinline__ float normalize_rotate(float (&x)[NPL], const TqBooks &bk,
+                                                  float *scratch, int lane, bool &bad) {
   bool finite = true;
   float ss = 0.f;
 #pragma unroll
@@ -111,10 +113,17 @@ __device__ __forceinline__ float normalize_rotate(float (&x)[NPL], const uint32_
   float nu = sqrtf(ss);
   if (!bad && isinf(__half2float(__float2half_rn(nu)))) bad = true;
   if (bad) nu = 0.f;
-  const float inv = nu > 0.f ? 1.0f / (sqrtf(static_cast<float>(NPL * 32)) * nu) : 0.f;
 #pragma unroll
   for (int k = 0; k < NPL; ++k) x[k] = bad ? 0.f : x[k];
-  tq_apply_signs<NPL>(x, dneg, lane);
+  if (bk.pi_t != nullptr) {
+    const float inv = nu > 0.f ? 1.0f / nu : 0.f;
+    tq_warp_dense<NPL>(x, bk.pi_t, scratch, lane);
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) x[k] *= inv;
+    return nu;
+  }
+  const float inv = nu > 0.f ? 1.0f / (sqrtf(static_cast<float>(NPL * 32)) * nu) : 0.f;
+  tq_apply_signs<NPL>(x, bk.dneg, lane);
   tq_warp_wht<NPL>(x, lane);
 #pragma unroll
   for (int k = 0; k < NPL; ++k) x[k] *= inv;
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
       load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
                     head_map(a.map.k, a.map.hstride, h), a.map.dfull);
       bool bad;
-      const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      const float nu = normalize_rotate<NPL>(x, a.books, rbuf[warp], lane, bad);
       int idx[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
       // ------------------------------------------------------------ values
       load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
                     head_map(a.map.v, a.map.hstride, h), a.map.dfull);
-      const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      const float nv = normalize_rotate<NPL>(x, a.books, rbuf[warp], lane, bad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
@@ -274,6 +283,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
   __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
   __shared__ __align__(16) float rsm[D];
   __shared__ uint32_t sgw[NPL];
+  __shared__ float dsc[2][D];          // dense-rotation scratch of warps 0 and 1
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < TQ_MAX_LEVELS) {
     cks[tid] = a.books.ck[tid];
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       float x[NPL];
       load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
                     head_map(a.map.k, a.map.hstride, h), a.map.dfull);
-      nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      nu = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
       int idx[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
@@ -352,7 +362,7 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
                     head_map(a.map.v, a.map.hstride, h), a.map.dfull);
       bool vbad;
-      const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, vbad);
+      const float nv = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, vbad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
@@ -442,6 +452,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   uint8_t *Bs = As + A_BYTES;
   __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
   __shared__ uint32_t vbuf[4][4][D];   // value column words of the tile's 4 groups
+  __shared__ float dsc[QTC_T / 32][D];  // dense-rotation scratch, one row per warp
   __shared__ __align__(8) uint64_t mb;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
@@ -522,7 +533,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
 #pragma unroll
       for (int k = 0; k < NPL; ++k) x[k] = xk[i][k];
       bool bad;
-      const float nu = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      const float nu = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
       int idx[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) idx[k] = tq_code<MBK>(x[k], tks);
@@ -562,7 +573,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       }
 #pragma unroll
       for (int k = 0; k < NPL; ++k) x[k] = xv[i][k];
-      const float nv = normalize_rotate<NPL>(x, a.books.dneg, lane, bad);
+      const float nv = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
@@ -772,9 +783,10 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
   // implementation, used to cross-check the tensor-core one)
   const char *impl = getenv("TQ_QUANT_IMPL");
   const bool simt = impl && impl[0] == 's';
-  if (items >= 256 && !simt && map.k == nullptr) {
+  if (items >= 256 && !simt && map.k == nullptr && c->books.pi == nullptr) {
     // large bf16 calls: one thread per row, TMA tiles (quantize_tile.cu); a
-    // channel map (gathered loads) takes the warp-per-row kernels below
+    // channel map (gathered loads) or a dense rotation takes the warp-per-row
+    // kernels below
     const int e = launch_quantize_tile(c, k, v, dtype, B, H, T, sb, sh, st, rc, rs, pos0, cache,
                                        row0, status, stream);
     if (e != TQ_ERR_UNSUPPORTED) return e;

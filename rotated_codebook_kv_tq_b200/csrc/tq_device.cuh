@@ -97,3 +97,29 @@ __device__ __forceinline__ int tq_code(float u, const float *t) {
   for (int s = STEPS - 1; s >= 0; --s) idx += (u >= t[idx + (1 << s) - 1]) ? (1 << s) : 0;
   return idx;
 }
+
+// Dense rotation of a warp-held d-vector (coordinate lane + 32 k in x[k]):
+// x <- M x with M given through MT[j*d + i] = M[i][j] (so a row j of MT is
+// read by the warp as one coalesced line).  scratch: d floats of shared memory
+// that belong to this warp.  fp32 products and sums in order j = 0 .. d-1.
+template <int NPL>
+__device__ __forceinline__ void tq_warp_dense(float (&x)[NPL], const float *__restrict__ MT,
+                                              float *scratch, int lane) {
+  constexpr int D = NPL * 32;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) scratch[lane + 32 * k] = x[k];
+  __syncwarp();
+  float acc[NPL];
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) acc[k] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < D; ++j) {
+    const float xj = scratch[j];
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) acc[k] = fmaf(__ldg(MT + j * D + lane + 32 * k), xj, acc[k]);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) x[k] = acc[k];
+}
+

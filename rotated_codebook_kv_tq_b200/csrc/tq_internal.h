@@ -13,6 +13,8 @@ namespace tqhost {
 bool lloyd_max(int d, int bits, std::vector<double> &c, std::vector<double> &t, double &mse);
 // FibQuant k = 2 pair codebook (fq_codebook.cpp): c = x0, y0, x1, y1, ...
 bool fq_pair_codebook(int d, int bits, std::vector<double> &c, double &mse);
+// Dense Haar rotation from a d x d Gaussian matrix (haar.cpp), row-major.
+bool haar_rotation(int d, const float *g, std::vector<double> &pi);
 }
 
 // Largest head dim the kernels are instantiated for.
@@ -27,6 +29,11 @@ struct TqBooks {
   float cv[TQ_MAX_LEVELS];   // value centroids
   float tv[TQ_MAX_LEVELS];   // value thresholds
   uint32_t dneg[TQ_MAX_D / 32];  // bit i set <=> D_i = -1
+  // dense rotation (device, fp32, row-major), both null for the randomized
+  // Walsh-Hadamard Pi = H diag(D) / sqrt(d): pi[i*d + j] = Pi[i][j] and
+  // pi_t[j*d + i] = Pi[i][j]
+  const float *pi;
+  const float *pi_t;
   int mse_bits_k;
   int qjl;
   int bits_v;
@@ -46,6 +53,7 @@ struct tq_codec {
   int d;
   int bits_k, qjl_k, bits_v, mse_bits_k;
   TqBooks books;
+  float *rot_dev;      // dense rotation: Pi then Pi^T (2 d^2 floats), or null
   uint16_t *S_dev;     // bf16 [d][d] row-major S[i][j]
   uint16_t *ST_dev;    // bf16 [d][d] transpose, ST[j][i] = S[i][j] (same allocation)
   uint16_t *S_tile;    // d = 1536 only: S as 256 x 64 K-major core-matrix tiles (same allocation)

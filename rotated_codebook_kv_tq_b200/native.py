@@ -27,7 +27,7 @@ EXPORTS = [
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
     "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_split_channels",
     "tq_quantize_kv_split", "tq_attention_split_workspace", "tq_attention_decode_split",
-    "tq_dequantize_split", "tq_fq_build_codebook", "tq_fq_codec_create", "tq_fq_codec_destroy",
+    "tq_dequantize_split", "tq_haar_rotation", "tq_fq_build_codebook", "tq_fq_codec_create", "tq_fq_codec_destroy",
     "tq_fq_codec_codebooks", "tq_fq_cache_bytes", "tq_fq_quantize_kv", "tq_fq_attention_workspace",
     "tq_fq_attention_decode", "tq_fq_dequantize", "tq_set_timing_events", "tq_launch_count",
     "tq_last_error",
@@ -43,7 +43,7 @@ class TqError(RuntimeError):
 class CodecDesc(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("bits_k", ctypes.c_int), ("qjl_k", ctypes.c_int),
                 ("bits_v", ctypes.c_int), ("rotation_signs", ctypes.c_void_p),
-                ("qjl_bf16", ctypes.c_void_p)]
+                ("qjl_bf16", ctypes.c_void_p), ("rotation", ctypes.c_void_p)]
 
 
 class CacheDesc(ctypes.Structure):
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         L.tq_attention_decode_split.argtypes = [sp, vp, i32, i32, i32, i32, cp, cp, vp, i32,
                                                 ctypes.c_float, vp, vp, i32, vp, sz, vp, vp]
         L.tq_dequantize_split.argtypes = [sp, cp, cp, i32, i64, i64, vp, vp]
+        L.tq_haar_rotation.argtypes = [i32, vp, vp]
         L.tq_fq_build_codebook.argtypes = [i32, i32, vp, vp]
         L.tq_fq_codec_create.argtypes = [ctypes.POINTER(FqCodecDesc), ctypes.POINTER(vp)]
         L.tq_fq_codec_destroy.argtypes = [vp]
@@ -159,14 +160,18 @@ class Codec:
     """Owns a ``tq_codec`` (device copies of D, S and the codebooks)."""
 
     def __init__(self, d: int, bits_k: int, qjl_k: bool, bits_v: int,
-                 rotation_signs: np.ndarray, qjl_bf16: Optional[np.ndarray]):
+                 rotation_signs: Optional[np.ndarray], qjl_bf16: Optional[np.ndarray],
+                 rotation: Optional[np.ndarray] = None):
         self.d, self.bits_k, self.qjl_k, self.bits_v = d, bits_k, bool(qjl_k), bits_v
         self.mse_bits_k = bits_k - 1 if qjl_k else bits_k
         self.planes_k = self.mse_bits_k + (1 if qjl_k else 0)
-        signs = np.ascontiguousarray(rotation_signs, dtype=np.int8)
+        signs = None if rotation_signs is None else np.ascontiguousarray(rotation_signs, dtype=np.int8)
         s = None if qjl_bf16 is None else np.ascontiguousarray(qjl_bf16, dtype=np.uint16)
-        desc = CodecDesc(d, bits_k, 1 if qjl_k else 0, bits_v, signs.ctypes.data,
-                         None if s is None else s.ctypes.data)
+        rot = None if rotation is None else np.ascontiguousarray(rotation, dtype=np.float32)
+        desc = CodecDesc(d, bits_k, 1 if qjl_k else 0, bits_v,
+                         None if signs is None else signs.ctypes.data,
+                         None if s is None else s.ctypes.data,
+                         None if rot is None else rot.ctypes.data)
         h = ctypes.c_void_p()
         check(lib().tq_codec_create(ctypes.byref(desc), ctypes.byref(h)))
         self.handle = h
@@ -434,6 +439,14 @@ def dequantize_split(split: Split, cache_hi: Cache, cache_lo: Cache, which: int,
     sd, dh, dl = split.desc(), cache_hi.desc(), cache_lo.desc()
     check(lib().tq_dequantize_split(ctypes.byref(sd), ctypes.byref(dh), ctypes.byref(dl), which,
                                     row0, rows, _ptr(out), _stream(stream)))
+
+
+def haar_rotation(gaussian: np.ndarray) -> np.ndarray:
+    """tq_haar_rotation: d x d Gaussian (host) -> Haar rotation fp32 [d, d]."""
+    g = np.ascontiguousarray(gaussian, dtype=np.float32)
+    out = np.zeros(g.shape, np.float32)
+    check(lib().tq_haar_rotation(g.shape[0], g.ctypes.data, out.ctypes.data))
+    return out
 
 
 # ---------------------------------------------------------------- FibQuant k = 2

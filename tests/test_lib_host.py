@@ -156,3 +156,32 @@ def test_fq_codec_is_host_only_and_validates(L):
     bad[5] = 0
     with pytest.raises(native.TqError):
         native.FqCodec(128, 2, 2, bad)
+
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_haar_rotation_matches_oracle(L, d):
+    """tq_haar_rotation (host Householder QR) against the oracle's sign-fixed
+    numpy QR of the same Gaussian matrix."""
+    from oracle.rotation import haar_rotation
+    G = synth.haar_gaussian(d, 4)
+    got = native.haar_rotation(G).astype(np.float64)
+    ref = haar_rotation(G)
+    assert np.max(np.abs(got - ref)) < 1e-6
+    assert np.max(np.abs(got @ got.T - np.eye(d))) < 1e-5
+
+
+def test_dense_rotation_validation(L):
+    bad = np.eye(64, dtype=np.float32)
+    bad[3, 3] = 0.5
+    S = synth.qjl_matrix_bf16(64, 0)
+    desc = native.CodecDesc(64, 3, 1, 3, None, S.ctypes.data, bad.ctypes.data)
+    h = ctypes.c_void_p()
+    assert L.tq_codec_create(ctypes.byref(desc), ctypes.byref(h)) == native.TQ_ERR_INVALID_ARG
+    assert b"orthogonal" in L.tq_last_error()
+    big = np.eye(1536, dtype=np.float32)
+    desc = native.CodecDesc(1536, 3, 1, 3, None, None, big.ctypes.data)
+    assert L.tq_codec_create(ctypes.byref(desc), ctypes.byref(h)) == native.TQ_ERR_UNSUPPORTED
+    g = synth.haar_gaussian(16, 0)
+    g[2, 2] = np.nan
+    with pytest.raises(native.TqError):
+        native.haar_rotation(g)

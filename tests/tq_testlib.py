@@ -33,9 +33,18 @@ def require_cuda():
     build()
 
 
-def codecs(w: synth.Workload, seed_offset: int = 0):
+def codecs(w: synth.Workload, seed_offset: int = 0, haar: bool = False):
+    """Matching oracle and library codecs.  haar: a dense Haar rotation from
+    the workload's Gaussian matrix, factorised by each side on its own."""
     D = synth.rotation_signs(w.d, w.seed + seed_offset)
     S = synth.qjl_matrix_bf16(w.d, w.seed + seed_offset) if w.qjl_k else None
+    if haar:
+        from oracle.rotation import haar_rotation
+        G = synth.haar_gaussian(w.d, w.seed + seed_offset)
+        ocodec = oc.make_codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S, Pi=haar_rotation(G))
+        ncodec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, None, S,
+                              rotation=native.haar_rotation(G))
+        return ocodec, ncodec
     ocodec = oc.make_codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
     ncodec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
     return ocodec, ncodec
