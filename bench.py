@@ -46,7 +46,7 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--only", choices=["quantize_esm_prefill", "bidir_esm_prefill", "decode_long_context",
                                       "decode_llama", "vector_search", "quality", "decode_split",
-                                      "decode_fibquant", "quality_fibquant"],
+                                      "decode_fibquant", "quality_fibquant", "haar"],
                    help="run one extra workload alone and print its JSON (1 GPU)")
     p.add_argument("--search-rows", type=int, default=0,
                    help="vector-search database rows for --only vector_search (default 10^6)")
@@ -183,8 +183,14 @@ def describe(w) -> str:
             + (f"{w.num_splits} splits" if w.num_splits else "default split count"))
 
 
+def haar_for(w):
+    """Dense Haar rotation of a workload (library factorisation)."""
+    from rotated_codebook_kv_tq_b200 import native, synth
+    return native.haar_rotation(synth.haar_gaussian(w.d, w.seed))
+
+
 class DecodeBench:
-    def __init__(self, w, n_sets: int):
+    def __init__(self, w, n_sets: int, haar: bool = False):
         import torch
         from rotated_codebook_kv_tq_b200 import native, synth
         self.w, self.n_sets = w, n_sets
@@ -192,7 +198,8 @@ class DecodeBench:
         D = synth.rotation_signs(w.d, w.seed)
         S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
         self.D, self.S = D, S
-        self.codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
+        self.codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S,
+                                  rotation=haar_for(w) if haar else None)
         T = w.T
         self.rows_cap = (T + 31) // 32 * 32
         K, V = synth.kv_inputs_torch(w, T=T)
@@ -533,15 +540,17 @@ def cpu_baselines(seconds: float = 1.0) -> dict:
 # Extra workloads
 # ---------------------------------------------------------------------------
 
-def quantize_extra(wname: str, pk: dict, steps: int = 40):
+def quantize_extra(wname: str, pk: dict, steps: int = 40, haar: bool = False):
     """Prefill quantize of a whole [B, H, T, d] K/V batch: input GB/s and the
-    kernel's HBM roofline fraction.  Rotates over input sets larger than L2."""
+    kernel's HBM roofline fraction.  Rotates over input sets larger than L2.
+    haar: the codec on a dense Haar rotation instead of the randomized WHT."""
     import torch
     from rotated_codebook_kv_tq_b200 import native, synth
     w = synth.WORKLOADS[wname]
     D = synth.rotation_signs(w.d, w.seed)
     S = synth.qjl_matrix_bf16(w.d, w.seed) if w.qjl_k else None
-    codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S)
+    codec = native.Codec(w.d, w.bits_k, w.qjl_k, w.bits_v, D, S,
+                         rotation=haar_for(w) if haar else None)
     rows_cap = (w.T + 31) // 32 * 32
     in_bytes = 2 * w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4)
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
@@ -566,7 +575,8 @@ def quantize_extra(wname: str, pk: dict, steps: int = 40):
     t = statistics.median(a.elapsed_time(b) for a, b in evs) / 1e3
     out_bytes = w.B * w.Hkv * w.T * row_bytes(w)
     alg = in_bytes + out_bytes
-    return dict(workload=describe(w), input_GBps=in_bytes / t / 1e9, us_per_call=t * 1e6,
+    return dict(workload=describe(w), rotation="dense Haar" if haar else "randomized WHT",
+                input_GBps=in_bytes / t / 1e9, us_per_call=t * 1e6,
                 roofline=dict(bound="hbm", achieved=alg / t / 1e9, peak=pk["hbm"], unit="GB/s",
                               frac=alg / t / 1e9 / pk["hbm"], algorithmic_bytes=alg),
                 l2="rotating %d input sets (%.0f MB)" % (n_sets, n_sets * in_bytes / 1e6))
@@ -787,11 +797,12 @@ def search_extra(pk: dict, steps: int = 5):
         l2="database codes 772 MB and input 6.1 GB > L2")
 
 
-def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
+def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5, haar: bool = False,
+                 n_sets: int = 1):
     import torch
     from rotated_codebook_kv_tq_b200 import synth
     w = synth.WORKLOADS[wname]
-    bench = DecodeBench(w, n_sets=1)
+    bench = DecodeBench(w, n_sets=n_sets, haar=haar)
 
     class _Null:
         def start(self):
@@ -802,12 +813,12 @@ def decode_extra(wname: str, pk: dict, steps: int = 60, warmup: int = 5):
 
     total, kern, _, _ = time_decode(bench, steps, warmup, 1, _Null())
     alg = bench.cache_bytes_per_step()
-    res = dict(workload=describe(w), us_per_step=total / steps * 1e6,
-               tokens_per_s=w.B * steps / total,
+    res = dict(workload=describe(w), rotation="dense Haar" if haar else "randomized WHT",
+               us_per_step=total / steps * 1e6, tokens_per_s=w.B * steps / total,
                roofline=dict(bound="hbm", achieved=alg / kern / 1e9, peak=pk["hbm"], unit="GB/s",
                              frac=alg / kern / 1e9 / pk["hbm"], algorithmic_bytes=alg,
                              kernel_us=kern * 1e6),
-               l2="cache %.0f MB per step > L2" % (alg / 1e6))
+               l2="rotating %d cache(s) of %.0f MB" % (n_sets, alg / 1e6))
     del bench
     torch.cuda.empty_cache()
     return res
@@ -1272,6 +1283,10 @@ def run_only(args) -> int:
         r["llama_decode_outlier_split"] = split_quality_extra("llama_decode")
     elif args.only == "decode_split":
         r = {rate: split_decode_extra(pk, rate) for rate in SPLIT_RATES}
+    elif args.only == "haar":
+        r = dict(decode_llama=decode_extra("llama_decode", pk, steps=40, haar=True, n_sets=12),
+                 decode_llama_wht=decode_extra("llama_decode", pk, steps=40, n_sets=12),
+                 quantize_esm_prefill=quantize_extra("esm_prefill", pk, steps=10, haar=True))
     elif args.only == "decode_fibquant":
         r = {f"{b / 2:g}": fq_decode_extra(pk, b) for b in (2, 4, 6)}
     elif args.only == "quality_fibquant":

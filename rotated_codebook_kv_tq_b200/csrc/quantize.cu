@@ -130,6 +130,28 @@ __device__ __forceinline__ float normalize_rotate(float (&x)[NPL], const TqBooks
   return nu;
 }
 
+// nu of a warp-held row and x <- x / nu (zero for a bad row), as in
+// normalize_rotate but without the rotation (applied later to several rows).
+template <int NPL>
+__device__ __forceinline__ float normalize_only(float (&x)[NPL], int lane, bool &bad) {
+  bool finite = true;
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) {
+    finite &= isfinite(x[k]);
+    ss += x[k] * x[k];
+  }
+  bad = __any_sync(TQ_FULL, !finite);
+  ss = tq_warp_sum(ss);
+  float nu = sqrtf(ss);
+  if (!bad && isinf(__half2float(__float2half_rn(nu)))) bad = true;
+  if (bad) nu = 0.f;
+  const float inv = nu > 0.f ? 1.0f / nu : 0.f;
+#pragma unroll
+  for (int k = 0; k < NPL; ++k) x[k] = bad ? 0.f : x[k] * inv;
+  return nu;
+}
+
 template <int D>
 __global__ void __launch_bounds__(QWARPS * 32) quantize_kernel(QuantArgs a) {
   constexpr int NPL = D / 32;
@@ -452,7 +474,8 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   uint8_t *Bs = As + A_BYTES;
   __shared__ float cks[TQ_MAX_LEVELS], tks[TQ_MAX_LEVELS], tvs[TQ_MAX_LEVELS];
   __shared__ uint32_t vbuf[4][4][D];   // value column words of the tile's 4 groups
-  __shared__ float dsc[QTC_T / 32][D];  // dense-rotation scratch, one row per warp
+  // dense-rotation scratch: the PF rows of each warp
+  __shared__ __align__(16) float dsc[QTC_T / 32][(D == 64 ? 8 : 4) * D];
   __shared__ __align__(8) uint64_t mb;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
@@ -523,7 +546,24 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
                       head_map(a.map.k, a.map.hstride, h), a.map.dfull);
         load_row<NPL>(xv[i], a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
                       head_map(a.map.v, a.map.hstride, h), a.map.dfull);
+      } else {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) xk[i][k] = xv[i][k] = 0.f;
       }
+    }
+    // dense rotation: norms first, then the PF rows of K and of V rotated
+    // together (each line of Pi^T read once per PF rows)
+    const bool dense = a.books.pi_t != nullptr;
+    float nuk[PF], nuv[PF];
+    bool badk[PF], badv[PF];
+    if (dense) {
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        nuk[i] = normalize_only<NPL>(xk[i], lane, badk[i]);
+        nuv[i] = normalize_only<NPL>(xv[i], lane, badv[i]);
+      }
+      tq_warp_dense_rows<NPL, PF>(xk, a.books.pi_t, dsc[warp], lane);
+      tq_warp_dense_rows<NPL, PF>(xv, a.books.pi_t, dsc[warp], lane);
     }
 #pragma unroll
     for (int i = 0; i < PF; ++i) {
@@ -532,8 +572,8 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       float x[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) x[k] = xk[i][k];
-      bool bad;
-      const float nu = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
+      bool bad = dense ? badk[i] : false;
+      const float nu = dense ? nuk[i] : normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
       int idx[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) idx[k] = tq_code<MBK>(x[k], tks);
@@ -573,7 +613,8 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
       }
 #pragma unroll
       for (int k = 0; k < NPL; ++k) x[k] = xv[i][k];
-      const float nv = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
+      if (dense) bad = badv[i];
+      const float nv = dense ? nuv[i] : normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {

@@ -123,3 +123,48 @@ __device__ __forceinline__ void tq_warp_dense(float (&x)[NPL], const float *__re
   for (int k = 0; k < NPL; ++k) x[k] = acc[k];
 }
 
+// Same rotation for R rows held by one warp at once (x[r][k]: coordinate
+// lane + 32 k of row r): each line of MT is read once for all R rows and the
+// inputs are broadcast four at a time from shared memory.  scratch: R * d
+// floats of this warp's shared memory, 16-byte aligned.  Per row the sums run
+// in the same order as tq_warp_dense, so the results are identical.
+template <int NPL, int R>
+__device__ __forceinline__ void tq_warp_dense_rows(float (&x)[R][NPL], const float *__restrict__ MT,
+                                                   float *scratch, int lane) {
+  constexpr int D = NPL * 32;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) scratch[r * D + lane + 32 * k] = x[r][k];
+  __syncwarp();
+  float acc[R][NPL];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) acc[r][k] = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < D; j += 4) {
+    float m[4][NPL];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) m[jj][k] = __ldg(MT + (j + jj) * D + lane + 32 * k);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 xv = *reinterpret_cast<const float4 *>(scratch + r * D + j);
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        acc[r][k] = fmaf(m[0][k], xv.x, acc[r][k]);
+        acc[r][k] = fmaf(m[1][k], xv.y, acc[r][k]);
+        acc[r][k] = fmaf(m[2][k], xv.z, acc[r][k]);
+        acc[r][k] = fmaf(m[3][k], xv.w, acc[r][k]);
+      }
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) x[r][k] = acc[r][k];
+}
+
