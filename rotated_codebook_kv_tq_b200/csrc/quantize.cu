@@ -832,6 +832,12 @@ int launch_quantize(const tq_codec *c, const void *k, const void *v, int dtype, 
                                        row0, status, stream);
     if (e != TQ_ERR_UNSUPPORTED) return e;
   }
+  if (items >= 256 && !simt && map.k == nullptr && c->books.pi != nullptr) {
+    // dense rotation: the tile's rotation as a tensor-core product (quantize_rot.cu)
+    const int e = launch_quantize_rot(c, k, v, dtype, B, H, T, sb, sh, st, rc, rs, pos0, cache,
+                                      row0, status, stream);
+    if (e != TQ_ERR_UNSUPPORTED) return e;
+  }
   const bool tc = c->qjl_k && items >= 256 && !simt;
   const bool append = items < 256 && !simt;
   switch (c->d) {

@@ -124,6 +124,13 @@ int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dt
                          int T, int64_t sb, int64_t sh, int64_t st, const float *rc,
                          const float *rs, int64_t pos0, const tq_cache *cache, int64_t row0,
                          uint32_t *status, cudaStream_t stream);
+// Prefill quantize for a codec with a dense rotation, the rotation on the
+// tensor cores (quantize_rot.cu); TQ_ERR_UNSUPPORTED without launching when
+// the codec has no dense rotation.
+int launch_quantize_rot(const tq_codec *c, const void *k, const void *v, int dtype, int B, int H,
+                        int T, int64_t sb, int64_t sh, int64_t st, const float *rc,
+                        const float *rs, int64_t pos0, const tq_cache *cache, int64_t row0,
+                        uint32_t *status, cudaStream_t stream);
 size_t decode_workspace_bytes(const tq_codec *c, int B, int Hq, int splits);
 int launch_decode(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                   const tq_cache *cache, const int32_t *seq_lens, int max_len, float scale,

@@ -31,11 +31,13 @@ ESM = synth.WORKLOADS["esm_prefill"]
 
 QUANT_CASES = {
     "llama_appends": (LLAMA.scaled(T=138), [(0, 100), (100, 1), (101, 37)]),
-    # >= 256 token groups: the tensor-core sketch kernel (QJL) ...
+    # >= 256 token groups: the tile kernel with the rotation on the tensor
+    # cores (with and without the sketch; "simt" takes the CUDA-core kernels)
     "llama_tc_sketch": (LLAMA.scaled(T=1100), [(0, 1037), (1037, 63)]),
-    # ... and the warp-per-group kernel (MSE-only keys), fp32 input
     "llama_large_mse_fp32": (LLAMA.scaled(T=1100, qjl_k=False, bits_k=3, dtype="fp32"), [(0, 1100)]),
     "esm_d64": (ESM.scaled(B=2, Hq=3, Hkv=3, T=100), [(0, 100)]),
+    # >= 256 token groups with d = 64, starting mid-group (row 45)
+    "esm_large_d64": (ESM.scaled(B=4, Hq=20, Hkv=20, T=300), [(0, 45), (45, 255)]),
 }
 
 
