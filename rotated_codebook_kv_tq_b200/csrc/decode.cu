@@ -88,22 +88,39 @@ __global__ void __launch_bounds__(D) qprep_kernel(DecodeArgs a) {
         x[k + HALF] = v * c + u * s;
       }
     }
-    float scl = 1.0f;
-    if (a.books.pi_t != nullptr) {
-      tq_warp_dense<NPL>(x, a.books.pi_t, qs, lane);   // q' = Pi q (dense rotation)
+    if (a.books.pi != nullptr) {
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) qs[lane + 32 * k] = x[k];   // RoPE'd q for the product below
     } else {
       tq_apply_signs<NPL>(x, a.books.dneg, lane);
       tq_warp_wht<NPL>(x, lane);
-      scl = 1.0f / sqrtf(static_cast<float>(D));
-    }
+      const float scl = 1.0f / sqrtf(static_cast<float>(D));
 #pragma unroll
-    for (int k = 0; k < NPL; ++k) {
-      x[k] *= scl;
-      a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
-      qs[lane + 32 * k] = x[k];
+      for (int k = 0; k < NPL; ++k) {
+        x[k] *= scl;
+        a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k];
+        qs[lane + 32 * k] = x[k];
+      }
     }
   }
   __syncthreads();
+  if (a.books.pi != nullptr) {
+    // dense rotation q' = Pi q: thread i takes row i of Pi, sums j = 0 .. d-1
+    const float4 *row = reinterpret_cast<const float4 *>(a.books.pi + tid * D);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 p = row[c];
+      acc = fmaf(p.x, qs[4 * c], acc);
+      acc = fmaf(p.y, qs[4 * c + 1], acc);
+      acc = fmaf(p.z, qs[4 * c + 2], acc);
+      acc = fmaf(p.w, qs[4 * c + 3], acc);
+    }
+    __syncthreads();
+    qs[tid] = acc;
+    a.q1[static_cast<int64_t>(head) * D + tid] = acc;
+    __syncthreads();
+  }
   if (!a.books.qjl) return;
   float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 8
@@ -346,6 +363,31 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
   if (s < S) o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
   os[gq][c] = o0 + o1;
   __syncthreads();
+  if (a.books.pi != nullptr) {
+    // dense rotation: out = Pi^T o / l, thread i takes row i of Pi^T
+    float v = 0.f;
+    if (tid < D) {
+#pragma unroll
+      for (int g = 0; g < CMB; ++g) v += os[g][tid];
+    }
+    __syncthreads();
+    if (tid < D) os[0][tid] = v;
+    __syncthreads();
+    if (tid < D) {
+      const float4 *row = reinterpret_cast<const float4 *>(a.books.pi_t + tid * D);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 p = row[c4];
+        acc = fmaf(p.x, os[0][4 * c4], acc);
+        acc = fmaf(p.y, os[0][4 * c4 + 1], acc);
+        acc = fmaf(p.z, os[0][4 * c4 + 2], acc);
+        acc = fmaf(p.w, os[0][4 * c4 + 3], acc);
+      }
+      a.out[head * D + tid] = acc / L;
+    }
+    return;
+  }
   if (warp == 0) {
     float x[NPL];
 #pragma unroll
@@ -355,14 +397,9 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
       for (int g = 0; g < CMB; ++g) v += os[g][lane + 32 * k];
       x[k] = v;
     }
-    float norm = 1.0f / L;
-    if (a.books.pi != nullptr) {
-      tq_warp_dense<NPL>(x, a.books.pi, os[0], lane);   // Pi^T o (dense rotation)
-    } else {
-      tq_warp_wht<NPL>(x, lane);
-      tq_apply_signs<NPL>(x, a.books.dneg, lane);
-      norm /= sqrtf(static_cast<float>(D));
-    }
+    tq_warp_wht<NPL>(x, lane);
+    tq_apply_signs<NPL>(x, a.books.dneg, lane);
+    const float norm = 1.0f / (sqrtf(static_cast<float>(D)) * L);
 #pragma unroll
     for (int k = 0; k < NPL; ++k) a.out[head * D + lane + 32 * k] = x[k] * norm;
   }

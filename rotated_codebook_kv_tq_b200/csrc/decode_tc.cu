@@ -181,18 +181,34 @@ __global__ void __launch_bounds__(TCT) tc_prep_kernel(TcArgs a) {
         x[k + HALF] = v * c + u * s;
       }
     }
-    float scl = 1.0f;
-    if (a.books.pi_t != nullptr) {
-      tq_warp_dense<TNW>(x, a.books.pi_t, q1s, lane);   // q' = Pi q (dense rotation)
+    if (a.books.pi != nullptr) {
+#pragma unroll
+      for (int k = 0; k < TNW; ++k) q2s[lane + 32 * k] = x[k];   // RoPE'd q for the product below
     } else {
       tq_apply_signs<TNW>(x, a.books.dneg, lane);
       tq_warp_wht<TNW>(x, lane);
-      scl = 1.0f / sqrtf(static_cast<float>(TD));
-    }
+      const float scl = 1.0f / sqrtf(static_cast<float>(TD));
 #pragma unroll
-    for (int k = 0; k < TNW; ++k) q1s[lane + 32 * k] = x[k] * scl;
+      for (int k = 0; k < TNW; ++k) q1s[lane + 32 * k] = x[k] * scl;
+    }
   }
   __syncthreads();
+  if (a.books.pi != nullptr) {
+    // dense rotation q' = Pi q: thread i takes row i of Pi (16-byte loads, all
+    // in flight at once), sums in order j = 0 .. d-1
+    const float4 *row = reinterpret_cast<const float4 *>(a.books.pi + tid * TD);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < TD / 4; ++c) {
+      const float4 p = row[c];
+      acc = fmaf(p.x, q2s[4 * c], acc);
+      acc = fmaf(p.y, q2s[4 * c + 1], acc);
+      acc = fmaf(p.z, q2s[4 * c + 2], acc);
+      acc = fmaf(p.w, q2s[4 * c + 3], acc);
+    }
+    q1s[tid] = acc;
+    __syncthreads();
+  }
   if (QJL) {
     // q''_i = sum_j S[i][j] q'_j for i = tid
     float acc = 0.f;

@@ -354,11 +354,57 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
     uint32_t myword = 0u;
     float nu = 0.f, rho = 0.f;
     bool bad = false;
+    // dense rotation: warps 0 and 1 normalise their rows, then the whole block
+    // forms u = Pi x for both (thread i: row i of Pi, 16-byte loads in flight)
+    const bool dense = a.books.pi != nullptr;
+    float dnu = 0.f;
+    bool dbad = false;
+    if (dense) {
+      if (warp < 2) {
+        float x[NPL];
+        load_row<NPL>(x, warp == 0 ? a.k : a.v, in_off, a.dtype, lane, warp == 0 ? a.rc : nullptr,
+                      warp == 0 ? a.rs : nullptr, a.pos0 + t,
+                      head_map(warp == 0 ? a.map.k : a.map.v, a.map.hstride, h), a.map.dfull);
+        dnu = normalize_only<NPL>(x, lane, dbad);
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) dsc[warp][lane + 32 * k] = x[k];
+      }
+      __syncthreads();
+      float u0 = 0.f, u1 = 0.f;
+      if (tid < D) {
+        const float4 *row = reinterpret_cast<const float4 *>(a.books.pi + tid * D);
+#pragma unroll 8
+        for (int c = 0; c < D / 4; ++c) {
+          const float4 pv = row[c];
+          u0 = fmaf(pv.x, dsc[0][4 * c], u0);
+          u0 = fmaf(pv.y, dsc[0][4 * c + 1], u0);
+          u0 = fmaf(pv.z, dsc[0][4 * c + 2], u0);
+          u0 = fmaf(pv.w, dsc[0][4 * c + 3], u0);
+          u1 = fmaf(pv.x, dsc[1][4 * c], u1);
+          u1 = fmaf(pv.y, dsc[1][4 * c + 1], u1);
+          u1 = fmaf(pv.z, dsc[1][4 * c + 2], u1);
+          u1 = fmaf(pv.w, dsc[1][4 * c + 3], u1);
+        }
+      }
+      __syncthreads();
+      if (tid < D) {
+        dsc[0][tid] = u0;
+        dsc[1][tid] = u1;
+      }
+      __syncthreads();
+    }
     if (warp == 0) {
       float x[NPL];
-      load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
-                    head_map(a.map.k, a.map.hstride, h), a.map.dfull);
-      nu = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
+      if (dense) {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) x[k] = dsc[0][lane + 32 * k];
+        nu = dnu;
+        bad = dbad;
+      } else {
+        load_row<NPL>(x, a.k, in_off, a.dtype, lane, a.rc, a.rs, a.pos0 + t,
+                      head_map(a.map.k, a.map.hstride, h), a.map.dfull);
+        nu = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, bad);
+      }
       int idx[NPL];
 #pragma unroll
       for (int k = 0; k < NPL; ++k) idx[k] = tq_code(x[k], tks);
@@ -381,10 +427,18 @@ __global__ void __launch_bounds__(128) quantize_append_kernel(QuantArgs a) {
       }
     } else if (warp == 1) {
       float x[NPL];
-      load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
-                    head_map(a.map.v, a.map.hstride, h), a.map.dfull);
       bool vbad;
-      const float nv = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, vbad);
+      float nv;
+      if (dense) {
+#pragma unroll
+        for (int k = 0; k < NPL; ++k) x[k] = dsc[1][lane + 32 * k];
+        nv = dnu;
+        vbad = dbad;
+      } else {
+        load_row<NPL>(x, a.v, in_off, a.dtype, lane, nullptr, nullptr, 0,
+                      head_map(a.map.v, a.map.hstride, h), a.map.dfull);
+        nv = normalize_rotate<NPL>(x, a.books, dsc[warp], lane, vbad);
+      }
       const uint32_t bit = 1u << (r & 31);
 #pragma unroll
       for (int k = 0; k < NPL; ++k) {
