@@ -70,7 +70,7 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 }
 
 template <int D, bool QJL>
-__global__ void __launch_bounds__(RT, 1) qrot_kernel(RotArgs a) {
+__global__ void __launch_bounds__(RT, D == 64 ? 2 : 1) qrot_kernel(RotArgs a) {
   constexpr int KE = 2 * D;                       // K elements of the rotation product
   constexpr uint32_t A_BYTES = 128u * KE * 2u;
   constexpr uint32_t B_BYTES = static_cast<uint32_t>(D) * D * 2u;
@@ -435,7 +435,8 @@ int run_qrot(const RotArgs &a, cudaStream_t stream) {
   }
   const int64_t items = static_cast<int64_t>(a.B) * a.H * a.n_groups;
   const int64_t tiles = (items + 3) / 4;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int64_t cap = static_cast<int64_t>(sms) * (D == 64 ? 2 : 1);   // resident CTAs
+  const int grid = static_cast<int>(tiles < cap ? tiles : cap);
   qrot_kernel<D, QJL><<<grid, RT, shm, stream>>>(a);
   tq_count_launch(1);
   return tq_check_launch("qrot_kernel");
