@@ -116,13 +116,22 @@ __global__ void __launch_bounds__(2 * DS) split_qprep_kernel(SplitArgs a) {
   a.q2[static_cast<int64_t>(head) * D + tid] = acc;
 }
 
-template <int DS, int G>
+// LIN (key codebooks of at most 2 bits): a symmetric codebook of 1 or 2 bits
+// is linear in its bit planes, c[idx] = sum_p alpha_p (2 bit_p - 1), and so is
+// the sign term; then sum_i q_i (2 b_i - 1) = 2 sum_{b_i = 1} q_i - sum_i q_i,
+// and the first sum is read from nibble tables T[n][v] = sum over the set bits
+// t of v of q_{4n + t}: one lookup per 4 coordinates, plane and head instead
+// of per-coordinate index assembly and multiply-adds.
+template <int DS, int G, bool LIN>
 __global__ void __launch_bounds__(SCT) split_chunk_kernel(SplitArgs a) {
   constexpr int D = 2 * DS, NPS = DS / 32;
   constexpr int SLICES = SCT / D;         // thread groups sharing one coordinate
   constexpr int SUB = G >= 8 ? 256 : 512;  // rows per pass inside a chunk
+  constexpr int NN = LIN ? DS / 4 : 1;     // nibbles of a half
   __shared__ float q1s[D][G], q2s[D][G];
   __shared__ float cks[2][TQ_MAX_LEVELS], cvs[2][TQ_MAX_LEVELS];
+  __shared__ float lut[LIN ? 2 * G * 2 : 1][NN][16];   // [(half, head, q'|q'')][nibble][value]
+  __shared__ float qsum[2][2][G];                      // [half][q'|q''][head]
   __shared__ float w[2][SUB][G];          // logits, then p * nu_v of each half
   __shared__ float red[SCT / 32][G];
   __shared__ float stat[2][G];            // running max, running sum
@@ -152,6 +161,24 @@ __global__ void __launch_bounds__(SCT) split_chunk_kernel(SplitArgs a) {
     stat[1][tid] = 0.f;
   }
   __syncthreads();
+  if (LIN) {
+    for (int e = tid; e < 2 * G * 2 * NN * 16; e += SCT) {
+      const int v = e & 15, n = (e >> 4) % NN, tab = (e >> 4) / NN;
+      const int vec = tab & 1, h = (tab >> 1) % G, hf = (tab >> 1) / G;
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if ((v >> t) & 1) acc += vec ? q2s[hf * DS + 4 * n + t][h] : q1s[hf * DS + 4 * n + t][h];
+      lut[tab][n][v] = acc;
+    }
+    if (tid < 4 * G) {
+      const int h = tid % G, vec = (tid / G) & 1, hf = tid / (2 * G);
+      float acc = 0.f;
+      for (int i = 0; i < DS; ++i) acc += vec ? q2s[hf * DS + i][h] : q1s[hf * DS + i][h];
+      qsum[hf][vec][h] = acc;
+    }
+    __syncthreads();
+  }
 
   const int coord = tid % D, slice = tid / D;
   const int vhalf = coord / DS, vcol = coord % DS;
@@ -167,6 +194,51 @@ __global__ void __launch_bounds__(SCT) split_chunk_kernel(SplitArgs a) {
       float tot[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) tot[h] = 0.f;
+      if (LIN) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int mbk = a.books[hf].mse_bits_k;
+          const int qjl = a.books[hf].qjl;
+          const uint32_t *krow = reinterpret_cast<const uint32_t *>(
+              a.kcode[hf] + (bh * a.rows_cap + r) * (mbk + qjl) * (DS / 8));
+          const uint32_t sc = reinterpret_cast<const uint32_t *>(a.kscale[hf])[bh * a.rows_cap + r];
+          const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+          const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+          // plane p < mbk: alpha_p; the sign plane: coef rho
+          const float c0 = cks[hf][0], c1 = cks[hf][1], c2 = cks[hf][2];
+          float est[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) est[h] = 0.f;
+#pragma unroll
+          for (int p = 0; p < 3; ++p) {
+            if (p >= mbk + qjl) break;
+            const bool sgn = p == mbk;
+            const float coefp = sgn ? a.qjl_coef[hf] * rho
+                                    : (mbk == 1 ? 0.5f * (c1 - c0) : (p == 0 ? 0.5f * (c1 - c0) : 0.5f * (c2 - c0)));
+            const int tab0 = sgn ? 1 : 0;
+            float acc[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll
+            for (int k = 0; k < NPS; ++k) {
+              const uint32_t wd = krow[p * NPS + k];
+#pragma unroll
+              for (int n8 = 0; n8 < 8; ++n8) {
+                const int v = (wd >> (4 * n8)) & 15, n = 8 * k + n8;
+#pragma unroll
+                for (int h = 0; h < G; ++h) acc[h] += lut[(hf * G + h) * 2 + tab0][n][v];
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) est[h] = fmaf(coefp, 2.f * acc[h] - qsum[hf][tab0][h], est[h]);
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) tot[h] = fmaf(nu, est[h], tot[h]);
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) w[0][r - s0][h] = a.scale * tot[h];
+        continue;
+      }
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const int mbk = a.books[hf].mse_bits_k;
@@ -365,6 +437,17 @@ __global__ void __launch_bounds__(SCMB * 2 * DS) split_combine_kernel(SplitArgs 
   }
 }
 
+template <int DS, int G>
+void launch_chunk(SplitArgs &a, dim3 grid, cudaStream_t stream) {
+  // the table path for key codebooks of at most 2 bits (d/2 = 64, G <= 4:
+  // its tables fit the static shared memory)
+  const bool lin = DS == 64 && G <= 4 && a.books[0].mse_bits_k <= 2 && a.books[1].mse_bits_k <= 2;
+  if (lin)
+    split_chunk_kernel<DS, G, DS == 64 && G <= 4><<<grid, SCT, 0, stream>>>(a);
+  else
+    split_chunk_kernel<DS, G, false><<<grid, SCT, 0, stream>>>(a);
+}
+
 template <int DS>
 int run_split(SplitArgs &a, cudaStream_t stream) {
   const int heads = a.B * a.Hq;
@@ -381,10 +464,10 @@ int run_split(SplitArgs &a, cudaStream_t stream) {
     cudaEventRecordWithFlags(ev0, stream, ev_flags);
   }
   switch (a.G) {
-    case 1: split_chunk_kernel<DS, 1><<<grid, SCT, 0, stream>>>(a); break;
-    case 2: split_chunk_kernel<DS, 2><<<grid, SCT, 0, stream>>>(a); break;
-    case 4: split_chunk_kernel<DS, 4><<<grid, SCT, 0, stream>>>(a); break;
-    case 8: split_chunk_kernel<DS, 8><<<grid, SCT, 0, stream>>>(a); break;
+    case 1: launch_chunk<DS, 1>(a, grid, stream); break;
+    case 2: launch_chunk<DS, 2>(a, grid, stream); break;
+    case 4: launch_chunk<DS, 4>(a, grid, stream); break;
+    case 8: launch_chunk<DS, 8>(a, grid, stream); break;
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "split decode: GQA group size must be 1, 2, 4 or 8");
   }
   if (int e = tq_check_launch("split_chunk_kernel")) return e;

@@ -30,6 +30,7 @@ RATES = {
     "r2.5": ((3, True, 3), (2, True, 2)),
     "r3.5": ((4, True, 4), (3, True, 3)),
     "r2.5_mse": ((3, False, 3), (2, False, 2)),
+    "r1.5_mse": ((2, False, 2), (1, False, 1)),
 }
 
 LLAMA = synth.WORKLOADS["llama_decode"]
@@ -39,6 +40,8 @@ CASES = {
     "llama_appends": (LLAMA.scaled(B=1, Hq=8, Hkv=2, T=300), "r3.5", [(0, 250), (250, 1), (251, 49)],
                       [300], 0),
     "llama_mse_g2": (LLAMA.scaled(B=1, Hq=4, Hkv=2, T=400), "r2.5_mse", [(0, 400)], [400], 5),
+    # key codebooks of at most 2 bits without QJL, GQA group 1 (table path)
+    "llama_mse_lin_g1": (LLAMA.scaled(B=2, Hq=2, Hkv=2, T=500), "r1.5_mse", [(0, 500)], [500, 129], 3),
     # >= 256 token groups per call: the tensor-core sketch kernel with the map
     "llama_tc_sketch": (LLAMA.scaled(B=2, Hq=16, Hkv=8, T=600), "r2.5", [(0, 600)], [600, 411], 0),
     # halves of 128 channels, GQA group 8, fp32 inputs
