@@ -136,10 +136,22 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+_RAW_STREAM = None
+
+
 def _stream(stream) -> Optional[int]:
+    """The cudaStream_t of ``stream`` (None: torch's current stream)."""
+    global _RAW_STREAM
     if stream is None:
-        import torch
-        return torch.cuda.current_stream().cuda_stream
+        if _RAW_STREAM is None:
+            import torch
+            # torch's direct query of the current raw stream (no Stream
+            # object per call); the public route when it is missing
+            raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+            dev = getattr(torch._C, "_cuda_getDevice", None)
+            _RAW_STREAM = ((lambda: raw(dev())) if raw is not None and dev is not None
+                           else (lambda: torch.cuda.current_stream().cuda_stream))
+        return _RAW_STREAM()
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
@@ -208,8 +220,13 @@ class Cache:
     rows_cap: int
 
     def desc(self) -> CacheDesc:
-        return CacheDesc(self.kcode.data_ptr(), self.kscale.data_ptr(), self.vcode.data_ptr(),
-                         self.vnorm.data_ptr(), self.B, self.Hkv, self.rows_cap)
+        key = (self.kcode.data_ptr(), self.kscale.data_ptr(), self.vcode.data_ptr(),
+               self.vnorm.data_ptr(), self.B, self.Hkv, self.rows_cap)
+        cached = self.__dict__.get("_desc")
+        if cached is None or cached[0] != key:
+            cached = (key, CacheDesc(*key))
+            self.__dict__["_desc"] = cached
+        return cached[1]
 
 
 def cache_bytes(codec: Codec, B: int, Hkv: int, rows_cap: int):
@@ -229,13 +246,19 @@ def alloc_cache(codec: Codec, B: int, Hkv: int, rows_cap: int, device="cuda") ->
         B=B, Hkv=Hkv, rows_cap=rows_cap)
 
 
+_DTYPES = None
+
+
 def _dtype_code(t) -> int:
-    import torch
-    if t.dtype == torch.float32:
-        return TQ_F32
-    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
-        return TQ_BF16
-    raise TypeError(f"unsupported dtype {t.dtype}")
+    global _DTYPES
+    if _DTYPES is None:
+        import torch
+        _DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.int16: TQ_BF16,
+                   torch.uint16: TQ_BF16}
+    code = _DTYPES.get(t.dtype)
+    if code is None:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return code
 
 
 # ---------------------------------------------------------------- calls
