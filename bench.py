@@ -224,13 +224,13 @@ class DecodeBench:
         torch.cuda.synchronize()
 
     def step(self, s: int, knew=None, vnew=None, q=None) -> None:
+        """One decode step through tq_decode_step: append of the new token's
+        K/V at row T - 1, then the decode of every query head over T rows."""
         w, n = self.w, self.native
         c = self.caches[s % self.n_sets]
-        n.quantize_kv(self.codec, self.knew if knew is None else knew,
-                      self.vnew if vnew is None else vnew, c, row0=w.T - 1, rope=self.rope,
-                      pos0=w.T - 1)
-        n.attention_decode(self.codec, self.q if q is None else q, c, w.T, self.scale, self.out,
-                           self.ws, rope=self.rope, num_splits=self.splits)
+        n.decode_step(self.codec, self.knew if knew is None else knew,
+                      self.vnew if vnew is None else vnew, self.q if q is None else q, c, w.T,
+                      self.scale, self.out, self.ws, rope=self.rope, num_splits=self.splits)
 
     def cache_bytes_per_step(self) -> int:
         return self.w.B * self.w.Hkv * self.w.T * row_bytes(self.w)

@@ -202,6 +202,18 @@ int tq_attention_decode(const tq_codec *codec, const void *q, int dtype, int B, 
                         const float *rope_sin, int num_splits, void *workspace,
                         size_t ws_bytes, float *out, void *stream);
 
+/* One decode step in one call: append the new token's key and value at row
+ * T - 1 of every (b, KV head) (the key RoPE-rotated at position T - 1), then
+ * decode the queries over rows 0 .. T - 1.  Equal to tq_quantize_kv (T = 1,
+ * row0 = pos0 = T - 1) followed by tq_attention_decode (max_seq_len = T, no
+ * seq_lens), with their validation and error codes.
+ * k_new, v_new  device [B][Hkv][d], kv_dtype TQ_F32 or TQ_BF16 (contiguous).
+ * q             device [B][Hq][d], q_dtype.   out  device fp32 [B][Hq][d]. */
+int tq_decode_step(const tq_codec *codec, const void *k_new, const void *v_new, int kv_dtype,
+                   const void *q, int q_dtype, int B, int Hq, int Hkv, const tq_cache *cache, int T,
+                   float scale, const float *rope_cos, const float *rope_sin, int num_splits,
+                   void *workspace, size_t ws_bytes, float *out, void *stream);
+
 /* Same as tq_attention_decode, and also writes the estimated logits
  * l_j (the formula above, scale included) of every query head:
  * logits  device fp32 [B][Hq][max_seq_len]; entries j >= T_b are left

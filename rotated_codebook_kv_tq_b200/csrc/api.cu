@@ -361,6 +361,21 @@ int tq_attention_decode(const tq_codec *c, const void *q, int dtype, int B, int 
                        rope_sin, num_splits, workspace, ws_bytes, out, nullptr, stream);
 }
 
+int tq_decode_step(const tq_codec *c, const void *k_new, const void *v_new, int kv_dtype,
+                   const void *q, int q_dtype, int B, int Hq, int Hkv, const tq_cache *cache, int T,
+                   float scale, const float *rope_cos, const float *rope_sin, int num_splits,
+                   void *workspace, size_t ws_bytes, float *out, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "decode step: NULL codec");
+  if (T < 1 || (cache && T > cache->rows_cap))
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode step: T outside 1..rows_cap");
+  const int64_t d = c->d;
+  if (int e = tq_quantize_kv(c, k_new, v_new, kv_dtype, B, Hkv, 1, Hkv * d, d, d, rope_cos,
+                             rope_sin, T - 1, cache, T - 1, nullptr, stream))
+    return e;
+  return decode_common(c, q, q_dtype, B, Hq, Hkv, cache, nullptr, T, scale, rope_cos, rope_sin,
+                       num_splits, workspace, ws_bytes, out, nullptr, stream);
+}
+
 int tq_attention_logits(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                         const tq_cache *cache, const int32_t *seq_lens, int max_seq_len,
                         float scale, const float *rope_cos, const float *rope_sin,

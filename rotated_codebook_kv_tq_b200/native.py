@@ -23,7 +23,7 @@ TQ_F32, TQ_BF16 = 0, 1
 EXPORTS = [
     "tq_build_codebook", "tq_codec_create", "tq_codec_destroy", "tq_codec_codebooks",
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
-    "tq_attention_logits", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
+    "tq_attention_logits", "tq_decode_step", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
     "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_split_channels",
     "tq_quantize_kv_split", "tq_attention_split_workspace", "tq_attention_decode_split",
@@ -86,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.tq_attention_decode.argtypes = [vp, vp, i32, i32, i32, i32, ctypes.POINTER(CacheDesc),
                                           vp, i32, f32, vp, vp, i32, vp, sz, vp, vp]
         L.tq_attention_logits.argtypes = L.tq_attention_decode.argtypes[:-1] + [vp, vp]
+        L.tq_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32,
+                                     ctypes.POINTER(CacheDesc), i32, ctypes.c_float, vp, vp, i32,
+                                     vp, sz, vp, vp]
         L.tq_attention_decode_noalloc.argtypes = [vp, vp, i32, i32, i32, i32,
                                                   ctypes.POINTER(CacheDesc), vp, i32, f32, vp,
                                                   vp, i32, vp, vp]
@@ -295,6 +298,22 @@ def attention_decode(codec: Codec, q, cache: Cache, max_seq_len: int, scale: flo
                                     float(scale), _ptr(rc), _ptr(rs), num_splits,
                                     workspace.data_ptr(), ws_bytes, out.data_ptr(),
                                     _stream(stream)))
+
+
+def decode_step(codec: Codec, k_new, v_new, q, cache: Cache, T: int, scale: float, out, workspace,
+                rope=None, num_splits: int = 0, stream=None) -> None:
+    """tq_decode_step: append k_new, v_new [B, Hkv, d] (or [B, Hkv, 1, d]) at
+    row T - 1, then decode q [B, Hq, d] over rows 0 .. T - 1 into out."""
+    B, Hq = q.shape[0], q.shape[1]
+    if not (k_new.is_contiguous() and v_new.is_contiguous() and k_new.dtype == v_new.dtype):
+        raise ValueError("k_new and v_new must be contiguous and of one dtype")
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    check(lib().tq_decode_step(codec.handle, k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new),
+                               q.data_ptr(), _dtype_code(q), B, Hq, cache.Hkv, ctypes.byref(desc), T,
+                               float(scale), _ptr(rc), _ptr(rs), num_splits, workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), out.data_ptr(),
+                               _stream(stream)))
 
 
 def attention_logits(codec: Codec, q, cache: Cache, max_seq_len: int, scale: float, out,

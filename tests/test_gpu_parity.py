@@ -261,3 +261,33 @@ def test_decode_rejects_bad_arguments():
     with pytest.raises(native.TqError):
         native.quantize_kv(ncodec, torch.zeros((1, 1, 70, 128), device="cuda"),
                            torch.zeros((1, 1, 70, 128), device="cuda"), cache)
+
+
+def test_decode_step_equals_append_then_decode():
+    """tq_decode_step is tq_quantize_kv at row T - 1 followed by
+    tq_attention_decode over T rows: same cache bytes, same output bits."""
+    w = synth.WORKLOADS["llama_decode"].scaled(B=2, Hq=8, Hkv=2, T=333)
+    _, ncodec = tl.codecs(w)
+    K, V = synth.kv_inputs(w)
+    kd, vd = tl.to_device(K, w.dtype), tl.to_device(V, w.dtype)
+    q = tl.to_device(np.ascontiguousarray(synth.query_inputs(w, Lq=1)[:, :, 0]), w.dtype)
+    rope = tl.rope_device(synth.rope_for(w, 352))
+    caches, outs = [], []
+    for fused in (False, True):
+        c = native.alloc_cache(ncodec, w.B, w.Hkv, 352)
+        native.quantize_kv(ncodec, kd[:, :, :w.T - 1], vd[:, :, :w.T - 1], c, rope=rope)
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+        ws = torch.empty(native.attention_workspace(ncodec, w.B, w.Hq, 5), dtype=torch.uint8,
+                         device="cuda")
+        kn, vn = kd[:, :, w.T - 1:].contiguous(), vd[:, :, w.T - 1:].contiguous()
+        if fused:
+            native.decode_step(ncodec, kn, vn, q, c, w.T, 0.088, out, ws, rope=rope, num_splits=5)
+        else:
+            native.quantize_kv(ncodec, kn, vn, c, row0=w.T - 1, rope=rope, pos0=w.T - 1)
+            native.attention_decode(ncodec, q, c, w.T, 0.088, out, ws, rope=rope, num_splits=5)
+        torch.cuda.synchronize()
+        caches.append(tl.download_cache(c))
+        outs.append(out.cpu().numpy())
+    for key in ("kcode", "kscale", "vcode", "vnorm"):
+        assert np.array_equal(caches[0][key], caches[1][key]), key
+    assert np.array_equal(outs[0], outs[1])
