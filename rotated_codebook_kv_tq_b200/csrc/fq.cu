@@ -236,6 +236,51 @@ __global__ void __launch_bounds__(32) fq_qprep_kernel(FqDecArgs a) {
   for (int k = 0; k < NPL; ++k) a.q1[static_cast<int64_t>(head) * D + lane + 32 * k] = x[k] * inv;
 }
 
+// Key row: acc[h] += sum over blocks j of <q'_(2j, 2j+1), c[idx_j]>, with the
+// block codes gathered from KB planes of NPW words (only the nb planes the row
+// has are read; the generic KB = FQ_MAX_BITS case takes any nb).
+template <int KB, int NPW, int G>
+__device__ __forceinline__ void fq_key_sums(const uint32_t *krow, int nb, const float2 *cks,
+                                            const float (*q1s)[G], float (&acc)[G]) {
+#pragma unroll
+  for (int k = 0; k < NPW; ++k) {
+    uint32_t pw[KB];
+#pragma unroll
+    for (int p = 0; p < KB; ++p) pw[p] = p < nb ? krow[p * NPW + k] : 0u;
+#pragma unroll 4
+    for (int t = 0; t < 32; ++t) {
+      int idx = 0;
+#pragma unroll
+      for (int p = 0; p < KB; ++p) idx |= ((pw[p] >> t) & 1) << p;
+      const float2 c = cks[idx];
+      const int j = 32 * k + t;
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(q1s[2 * j][h], c.x, fmaf(q1s[2 * j + 1][h], c.y, acc[h]));
+    }
+  }
+}
+
+// Values of one 32-token column group for one rotated coordinate (component
+// comp of block vg's codes): o[h] += w[r][h] c[idx_r].comp for rows rlo..rhi.
+template <int VB, int G>
+__device__ __forceinline__ void fq_value_rows(const uint32_t *vg, int nb, int pstride,
+                                              const float2 *cvs, int comp, const float (*w)[G],
+                                              int s0, int rlo, int rhi, float (&o)[G]) {
+  uint32_t vw[VB];
+#pragma unroll
+  for (int p = 0; p < VB; ++p) vw[p] = p < nb ? vg[p * pstride] : 0u;
+  for (int r = rlo; r < rhi; ++r) {
+    const int bit = r & 31;
+    int idx = 0;
+#pragma unroll
+    for (int p = 0; p < VB; ++p) idx |= ((vw[p] >> bit) & 1) << p;
+    const float2 c = cvs[idx];
+    const float val = comp ? c.y : c.x;
+#pragma unroll
+    for (int h = 0; h < G; ++h) o[h] = fmaf(w[r - s0][h], val, o[h]);
+  }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
   constexpr int NPW = D / 64;
@@ -284,21 +329,13 @@ __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
       float acc[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll
-      for (int k = 0; k < NPW; ++k) {
-        uint32_t pw[FQ_MAX_BITS];
-#pragma unroll
-        for (int p = 0; p < FQ_MAX_BITS; ++p) pw[p] = p < bk ? krow[p * NPW + k] : 0u;
-#pragma unroll 4
-        for (int t = 0; t < 32; ++t) {
-          int idx = 0;
-#pragma unroll
-          for (int p = 0; p < FQ_MAX_BITS; ++p) idx |= ((pw[p] >> t) & 1) << p;
-          const float2 c = cks[idx];
-          const int j = 32 * k + t;
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] = fmaf(q1s[2 * j][h], c.x, fmaf(q1s[2 * j + 1][h], c.y, acc[h]));
-        }
+      // the code width selects an instantiation with exactly that many planes
+      switch (bk) {
+        case 1: fq_key_sums<1, NPW, G>(krow, bk, cks, q1s, acc); break;
+        case 2: fq_key_sums<2, NPW, G>(krow, bk, cks, q1s, acc); break;
+        case 3: fq_key_sums<3, NPW, G>(krow, bk, cks, q1s, acc); break;
+        case 4: fq_key_sums<4, NPW, G>(krow, bk, cks, q1s, acc); break;
+        default: fq_key_sums<FQ_MAX_BITS, NPW, G>(krow, bk, cks, q1s, acc); break;   // planes >= bk read as 0
       }
       const float nu = tq_half_to_f32(a.kscale[2 * (bh * a.rows_cap + r)]);
 #pragma unroll
@@ -356,19 +393,13 @@ __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
     // ---------------- values: thread per rotated coordinate
     for (int g = s0 / 32 + slice; g * 32 < s1; g += SLICES) {
       const uint32_t *vg = a.vcode + (bh * (a.rows_cap / 32) + g) * bv * (D / 2) + blk;
-      uint32_t vw[FQ_MAX_BITS];
-#pragma unroll
-      for (int p = 0; p < FQ_MAX_BITS; ++p) vw[p] = p < bv ? vg[p * (D / 2)] : 0u;
       const int rlo = max(s0, g * 32), rhi = min(s1, g * 32 + 32);
-      for (int r = rlo; r < rhi; ++r) {
-        const int bit = r & 31;
-        int idx = 0;
-#pragma unroll
-        for (int p = 0; p < FQ_MAX_BITS; ++p) idx |= ((vw[p] >> bit) & 1) << p;
-        const float2 c = cvs[idx];
-        const float val = comp ? c.y : c.x;
-#pragma unroll
-        for (int h = 0; h < G; ++h) o[h] = fmaf(w[r - s0][h], val, o[h]);
+      switch (bv) {
+        case 1: fq_value_rows<1, G>(vg, bv, D / 2, cvs, comp, w, s0, rlo, rhi, o); break;
+        case 2: fq_value_rows<2, G>(vg, bv, D / 2, cvs, comp, w, s0, rlo, rhi, o); break;
+        case 3: fq_value_rows<3, G>(vg, bv, D / 2, cvs, comp, w, s0, rlo, rhi, o); break;
+        case 4: fq_value_rows<4, G>(vg, bv, D / 2, cvs, comp, w, s0, rlo, rhi, o); break;
+        default: fq_value_rows<FQ_MAX_BITS, G>(vg, bv, D / 2, cvs, comp, w, s0, rlo, rhi, o); break;
       }
     }
     __syncthreads();
