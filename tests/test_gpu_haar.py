@@ -156,3 +156,30 @@ def test_haar_codec_rejected_where_not_built():
     with pytest.raises(native.TqError) as e:
         native.attention_bidir(ncodec, q, cache, 64, 0.125, out, ws)
     assert e.value.code == native.TQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T", [40, 1100])
+def test_haar_quantize_nonfinite_rows(T):
+    """Rows with a NaN or Inf are stored as zero rows and counted once per row,
+    in the warp-per-group kernels (T = 40) and the tensor-core rotation kernel
+    (T = 1100, >= 256 token groups)."""
+    w = LLAMA.scaled(B=1, Hq=8, Hkv=8, T=T, dtype="fp32")
+    ocodec, ncodec = tl.codecs(w, haar=True)
+    K = torch.randn((1, 8, T, 128), device="cuda")
+    V = torch.randn((1, 8, T, 128), device="cuda")
+    K[0, 3, 17, 5] = float("nan")
+    V[0, 6, T - 1, 100] = float("inf")
+    rows_cap = (T + 31) // 32 * 32
+    cache = native.alloc_cache(ncodec, 1, 8, rows_cap)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    native.quantize_kv(ncodec, K, V, cache, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 2
+    assert float(cache.kscale[0, 3, 17, 0]) == 0.0 and float(cache.vnorm[0, 6, T - 1]) == 0.0
+    # the zero rows decode to zero vectors; a finite row next to them is intact
+    out = torch.empty((1, 8, T, 128), device="cuda")
+    native.dequantize(ncodec, cache, 0, 0, T, out)
+    assert torch.all(out[0, 3, 17] == 0)
+    ref = K[0, 3, 18].double().cpu().numpy()
+    got = out[0, 3, 18].double().cpu().numpy()
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 0.5

@@ -178,3 +178,22 @@ def test_split_rejects_bad_arguments():
     with pytest.raises(native.TqError) as e:
         native.attention_decode_split(bad, q, chi, clo, 64, 0.1, out, ws, num_splits=2)
     assert e.value.code == native.TQ_ERR_UNSUPPORTED
+
+
+def test_split_quantize_nonfinite_rows():
+    """A NaN in an outlier channel spoils only the half that holds it: that
+    half row is stored as a zero row and counted, the other half is coded."""
+    w, sc, ns, *_ = _setup("llama_mse_g2")
+    T = 64
+    K = torch.randn((1, 2, T, 128), device="cuda")
+    V = torch.randn((1, 2, T, 128), device="cuda")
+    ch = sc.channels[0, 0]
+    K[0, 0, 10, int(ch[3])] = float("nan")          # an outlier (hi) key channel of head 0
+    chi = native.alloc_cache(ns.hi, 1, 2, T)
+    clo = native.alloc_cache(ns.lo, 1, 2, T)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    native.quantize_kv_split(ns, K, V, chi, clo, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    assert float(chi.kscale[0, 0, 10, 0]) == 0.0
+    assert float(clo.kscale[0, 0, 10, 0]) > 0.0
