@@ -21,11 +21,18 @@
 // * Keys: the residual of the tile, split into bf16 hi + lo, is stored into
 //   tensor memory and sketched against S (exactly bf16) by tcgen05 kind::f16
 //   MMAs with fp32 accumulation; each thread reads its row of S r back.
-// * Warps 0-3 take key rows, warps 4-7 value rows, warp 8 issues the copies of
-//   the next tile (as soon as every row of the current one is in registers)
-//   and the sketch MMAs.  CTAs are persistent over tile ranges ordered by
-//   position first, so the RoPE table tile is reloaded only when the position
-//   range changes.
+// * One CTA per SM with NTL row-warp groups (four at d = 64, two at d = 128),
+//   group g taking the rows of tile g of a unit.  A unit is NTL tiles at the
+//   same positions (consecutive heads of the flattened batch x head index)
+//   and one kind, keys or values; units are ordered (position tile, head
+//   group, kind), and each CTA takes a contiguous range of them, first all of
+//   its key units, then its value units, so the SM's instruction cache holds
+//   one row path at a time and the load stays balanced to half a unit.
+//   Thread 0 issues the copies of the next unit (once a barrier shows every
+//   row of the current one in registers) and, for keys, the sketch MMAs of
+//   the unit (once a barrier shows every operand stored).  Without a separate
+//   copy warp a thread keeps 128 (d = 64) or 255 (d = 128) registers.  The
+//   RoPE table tile is reloaded only when the position range changes.
 //
 // Codes are decided on the scaled transform y = H D x against t_k * sqrt(d) nu
 // (the same decision as u = y / (sqrt(d) nu) against t_k, up to fp32
@@ -41,7 +48,9 @@
 namespace {
 
 constexpr int QR = 128;         // rows per tile
-constexpr int QT = 288;         // 4 key warps, 4 value warps, 1 copy / MMA warp
+// tiles per unit: at d = 64 four tiles' sketch accumulators (4 x 128 tensor
+// memory columns) and 16 row warps of 128 registers fill an SM; at d = 128 two
+__host__ __device__ constexpr int tiles_per_unit(int d) { return d == 64 ? 4 : 2; }
 constexpr uint32_t BOX = QR * 128;   // bytes of one swizzled 128-row box
 
 struct TileArgs {
@@ -49,7 +58,8 @@ struct TileArgs {
   int64_t row0, pos0, rows_cap;
   int64_t R_first;   // cache row of the first row tile (multiple of 128)
   int64_t nrt;       // row tiles per (batch, head)
-  int64_t ntiles;    // nrt * B * H, ordered (row tile, batch, head)
+  int64_t groups;    // head groups per row tile: ceil(B * H / tiles per unit)
+  int64_t nunits;    // 2 * nrt * groups, ordered (row tile, head group, kind)
   uint8_t *kcode;
   uint16_t *kscale;
   uint32_t *vcode;
@@ -60,7 +70,7 @@ struct TileArgs {
   float ck[8];       // key centroid magnitudes c[half + m], m = 0 .. half-1
   float tk[8];       // key thresholds above 0: t[half - 1 + j], j = 1 .. half-1 (tk[j - 1])
   float tv[8];       // value thresholds above 0
-  uint32_t dneg[4];  // bit i set <=> D_i = -1
+  float dsg[128];    // D as +-1 pairs: dsg[2 j] = D_j, dsg[2 j + 1] = D_{j + d/2}, j < d/2
 };
 
 // ---------------------------------------------------------------- TMA
@@ -98,6 +108,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
   return false;
 }
 
+// Barrier of the CTA that also tells every thread whether all of them are
+// still on track (bar.red.or over the give-up flags); the tensor-memory
+// fences order tcgen05 traffic around it.
+template <int NT>
+__device__ __forceinline__ bool cta_all_ok(bool ok) {
+  sm100::fence_before_sync();
+  uint32_t bad;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.eq.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(bad)
+      : "r"(ok ? 1u : 0u), "n"(NT)
+      : "memory");
+  sm100::fence_after_sync();
+  return bad == 0u;
+}
+
 // Packed fp32 pair arithmetic (sm_100): each half rounds exactly like the
 // scalar instruction.
 __device__ __forceinline__ void addsub2(float &a0, float &a1, float &b0, float &b1) {
@@ -122,6 +149,14 @@ __device__ __forceinline__ void sub2c(float a0, float a1, uint64_t c, float &d0,
       "mov.b64 {%0, %1}, d;\n\t}\n"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "l"(c));
+}
+
+// (a0, a1) *= c (exact for c = (+-1, +-1))
+__device__ __forceinline__ void mul2c(float &a0, float &a1, uint64_t c) {
+  asm("{\n\t.reg .b64 p, d;\n\tmov.b64 p, {%0, %1};\n\tmul.rn.f32x2 d, p, %2;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}\n"
+      : "+f"(a0), "+f"(a1)
+      : "l"(c));
 }
 
 // acc += (a0 * a0, a1 * a1)
@@ -220,6 +255,47 @@ __device__ __forceinline__ void plane_msbs2(float y0, float y1, const uint64_t *
   }
 }
 
+// Raw decision bits of coordinates i and i + D/2, accumulated one funnel shift
+// per bit (coordinate 32 w + 31 first, so bit e of word w is coordinate
+// 32 w + e): acc[t] gathers the sign bits of |y| - th[t] (t < NT, th2[t] =
+// (th[t], th[t])), acc[NT] those of y.  planes_of() then forms each code
+// plane word from them by the thermometer identities of plane_msbs.
+template <int NB, int NW>
+__device__ __forceinline__ void raw_bits2(float y0, float y1, const uint64_t *th2,
+                                          uint32_t (&acc)[1 << (NB - 1)][NW], int i, int i1) {
+  constexpr int NT = (1 << (NB - 1)) - 1;   // thresholds above 0
+  const float a0 = fabsf(y0), a1 = fabsf(y1);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    float d0, d1;
+    sub2c(a0, a1, th2[t], d0, d1);
+    acc[t][i >> 5] = __funnelshift_l(__float_as_uint(d0), acc[t][i >> 5], 1);
+    acc[t][i1 >> 5] = __funnelshift_l(__float_as_uint(d1), acc[t][i1 >> 5], 1);
+  }
+  acc[NT][i >> 5] = __funnelshift_l(__float_as_uint(y0), acc[NT][i >> 5], 1);
+  acc[NT][i1 >> 5] = __funnelshift_l(__float_as_uint(y1), acc[NT][i1 >> 5], 1);
+}
+
+template <int NB, int NW>
+__device__ __forceinline__ void planes_of(const uint32_t (&r)[1 << (NB - 1)][NW], uint32_t (&pw)[NB][NW]) {
+  constexpr int NT = (1 << (NB - 1)) - 1;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t sy = r[NT][w];
+    pw[NB - 1][w] = sy;
+    if constexpr (NB == 2) {
+      pw[0][w] = r[0][w] ^ sy;
+    } else if constexpr (NB == 3) {
+      pw[1][w] = r[1][w] ^ sy;
+      pw[0][w] = r[0][w] ^ r[1][w] ^ r[2][w] ^ sy;
+    } else if constexpr (NB == 4) {
+      pw[2][w] = r[3][w] ^ sy;
+      pw[1][w] = r[1][w] ^ r[3][w] ^ r[5][w] ^ sy;
+      pw[0][w] = r[0][w] ^ r[1][w] ^ r[2][w] ^ r[3][w] ^ r[4][w] ^ r[5][w] ^ r[6][w] ^ sy;
+    }
+  }
+}
+
 // 32 x 32 bit transpose across a warp: on return bit L of lane i's word is
 // bit i of lane L's input word.
 __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
@@ -237,7 +313,7 @@ __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
 }
 
 template <int D, int MBK, int BV, bool QJL>
-__global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
     qtile_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                  const __grid_constant__ CUtensorMap tmc, const __grid_constant__ CUtensorMap tms,
                  TileArgs a) {
@@ -246,22 +322,28 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
   constexpr int NW = D / 32;              // words per plane row
   constexpr int HK = 1 << (MBK - 1), HV = 1 << (BV - 1);
   constexpr uint32_t IDESC = sm100::idesc_bf16(128, D);
-  constexpr int TCOLS = 2 * D;            // A (hi | lo, D/2 columns each) + z (D columns)
+  constexpr int NTL = tiles_per_unit(D);
+  constexpr int QT = 128 * NTL;
+  constexpr int TCOLS = 2 * D;            // per tile: A (hi | lo, D/2 columns each) + z (D columns)
   extern __shared__ uint8_t qsm_raw[];
   uint8_t *qsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *Kt = qsm;
-  uint8_t *Vt = Kt + NBX * BOX;
-  uint8_t *Ct = Vt + NBX * BOX;
+  uint8_t *Xt0 = qsm;                     // the unit's tiles, NBX boxes each
+  uint8_t *Ct = Xt0 + NTL * NBX * BOX;
   uint8_t *Snt = Ct + NBX * BOX;
   uint8_t *Bs = Snt + NBX * BOX;
-  __shared__ __align__(8) uint64_t full, empty, a_ready, z_ready;
+  __shared__ __align__(8) uint64_t full, z_ready;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t BH = static_cast<int64_t>(a.B) * a.H;
-  const int64_t t_begin = a.ntiles * blockIdx.x / gridDim.x;
-  const int64_t t_end = a.ntiles * (blockIdx.x + 1) / gridDim.x;
+  // this CTA's units [u0, u1): its key units (even u) first, then its value units
+  const int64_t u0 = a.nunits * blockIdx.x / gridDim.x;
+  const int64_t u1 = a.nunits * (blockIdx.x + 1) / gridDim.x;
+  const int64_t k_first = u0 + (u0 & 1), v_first = u0 + 1 - (u0 & 1);
+  const int64_t nk = u1 > k_first ? (u1 - k_first + 1) / 2 : 0;
+  const int64_t nloc = u1 - u0;
+  auto unit_of = [&](int64_t s) { return s < nk ? k_first + 2 * s : v_first + 2 * (s - nk); };
 
   if (QJL) {
     for (int e = tid; e < D * D; e += QT) {
@@ -269,12 +351,10 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
       *reinterpret_cast<uint16_t *>(Bs + (kb >> 4) * (D * 16) + (i >> 3) * 128 + (i & 7) * 16 +
                                     (kb & 15)) = a.S[e];
     }
-    if (warp == 0) sm100::tmem_alloc(&tmem_s, TCOLS);
+    if (warp == 0) sm100::tmem_alloc(&tmem_s, NTL * TCOLS);
   }
   if (tid == 0) {
     sm100::mbar_init(&full, 1);
-    sm100::mbar_init(&empty, 8);
-    sm100::mbar_init(&a_ready, 4);
     sm100::mbar_init(&z_ready, 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -285,81 +365,60 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
   sm100::fence_after_sync();
   const uint32_t tm = QJL ? tmem_s : 0u;
 
-  if (warp == 8) {
-    // ------------------------------------------------ copies and sketch MMAs
-    if (lane == 0) {
-      int64_t cur_pt = -1;
-      int issued = -1, committed = -1;
-      auto issue = [&](int64_t tau) {
-        const int64_t pt = tau / BH, bh = tau % BH;
-        const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
-        const int t0 = static_cast<int>(a.R_first + pt * QR - a.row0);
-        const bool table = a.rope && pt != cur_pt;
-        sm100::mbar_expect_tx(&full, (2 + (table ? 2 : 0)) * NBX * BOX);
+  // thread 0: the position tile of the RoPE table in shared memory, the
+  // last step whose copies were issued and the last sketch commit
+  int64_t cur_pt = -1;
+  int issued = -1, committed = -1;
+  auto issue = [&](int64_t s, int idx) {
+    const int64_t u = unit_of(s), q = u >> 1;
+    const bool keys = !(u & 1);
+    const int64_t pt = q / a.groups, bh0 = (q % a.groups) * NTL;
+    const int nt = static_cast<int>(BH - bh0 < NTL ? BH - bh0 : NTL);   // the last group may be short
+    const int t0 = static_cast<int>(a.R_first + pt * QR - a.row0);
+    const bool table = keys && a.rope && pt != cur_pt;
+    sm100::mbar_expect_tx(&full, (nt + (table ? 2 : 0)) * NBX * BOX);
+    const CUtensorMap *src = keys ? &tmk : &tmv;
+    for (int g = 0; g < nt; ++g) {
+      const int64_t bh = bh0 + g;
 #pragma unroll
-        for (int x = 0; x < NBX; ++x) {
-          tma_4d(Kt + x * BOX, &tmk, 64 * x, t0, h, b, &full);
-          tma_4d(Vt + x * BOX, &tmv, 64 * x, t0, h, b, &full);
-        }
-        if (table) {
-          const int p0 = static_cast<int>(a.pos0) + t0;
-#pragma unroll
-          for (int x = 0; x < NBX; ++x) {
-            tma_2d(Ct + x * BOX, &tmc, 32 * x, p0, &full);
-            tma_2d(Snt + x * BOX, &tms, 32 * x, p0, &full);
-          }
-          cur_pt = pt;
-        }
-        ++issued;
-      };
-      if (t_begin < t_end) issue(t_begin);
-      int i = 0;
-      for (int64_t tau = t_begin; tau < t_end && !abort_s; ++tau, ++i) {
-        if (tau + 1 < t_end) {
-          // every row of tile i is in registers: the buffers are free
-          if (!wait_or_abort(&empty, i & 1, &abort_s)) { abort_s = 1; break; }
-          issue(tau + 1);
-        }
-        if (QJL) {
-          if (!wait_or_abort(&a_ready, i & 1, &abort_s)) { abort_s = 1; break; }
-          sm100::fence_after_sync();
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s)
-            sm100::mma_f16_ts(tm + D, tm + 8 * s,
-                              sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
-                              IDESC, s > 0);
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s)
-            sm100::mma_f16_ts(tm + D, tm + D / 2 + 8 * s,
-                              sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
-                              IDESC, 1);
-          sm100::mma_commit(&z_ready);
-          committed = i;
-        }
-      }
-      if (abort_s) {
-        // let this CTA's own copies and MMAs land before its memory is released
-        if (issued >= 0) sm100::mbar_wait(&full, issued & 1, 1u << 20);
-        if (committed >= 0) sm100::mbar_wait(&z_ready, committed & 1, 1u << 20);
-      }
+      for (int x = 0; x < NBX; ++x)
+        tma_4d(Xt0 + (g * NBX + x) * BOX, src, 64 * x, t0, static_cast<int>(bh % a.H),
+               static_cast<int>(bh / a.H), &full);
     }
-    __syncwarp();
-  } else {
+    if (table) {
+      const int p0 = static_cast<int>(a.pos0) + t0;
+#pragma unroll
+      for (int x = 0; x < NBX; ++x) {
+        tma_2d(Ct + x * BOX, &tmc, 32 * x, p0, &full);
+        tma_2d(Snt + x * BOX, &tms, 32 * x, p0, &full);
+      }
+      cur_pt = pt;
+    }
+    issued = idx;
+  };
+  if (tid == 0 && nloc > 0) issue(0, 0);
+  {
     // ------------------------------------------------ row threads
-    const bool is_key = warp < 4;
     const int rl = tid & 127;                 // row of the tile = TMEM lane
     const int wq = warp & 3;
-    const uint8_t *Xt = is_key ? Kt : Vt;
+    const int wg = warp >> 2;                 // which tile of the unit
+    const uint8_t *Xt = Xt0 + wg * NBX * BOX;
+    const uint32_t tmg = tm + wg * TCOLS;
     float thr[8];
-    int i = 0;
-    for (int64_t tau = t_begin; tau < t_end; ++tau, ++i) {
-      if (abort_s) break;
-      const int64_t pt = tau / BH, bh = tau % BH;
+    // every thread passes every barrier of a step; a wait that gives up
+    // clears ok, and the next barrier makes the whole CTA leave together
+    bool ok = true;
+    int kz = 0;                               // sketch commits so far
+    for (int i = 0; i < nloc; ++i) {
+      const int64_t u = unit_of(i), q = u >> 1;
+      const bool is_key = !(u & 1);
+      const int64_t pt = q / a.groups, bh = (q % a.groups) * NTL + wg;
       const int64_t R = a.R_first + pt * QR + rl;     // cache row
       const int64_t t = R - a.row0;                    // token of the call
-      const bool active = t >= 0 && t < a.T;
-      if (!wait_or_abort(&full, i & 1, &abort_s)) { abort_s = 1; break; }
-      // ---- row into registers (+ RoPE for keys)
+      const bool active = t >= 0 && t < a.T && bh < BH;
+      if (ok && !wait_or_abort(&full, i & 1, &abort_s)) { abort_s = 1; ok = false; }
+      // ---- row into registers (+ RoPE for keys); after a give-up the
+      // values read are never used
       float x[D];
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
@@ -390,9 +449,9 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
           }
         }
       }
-      // the tile's buffers may be refilled now
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&empty);
+      // every row of the step is in registers: the buffers may be refilled
+      if (!(ok = cta_all_ok<QT>(ok))) break;
+      if (tid == 0 && i + 1 < nloc) issue(i + 1, i + 1);
       // ---- norm, sign flip, transform
       uint64_t ss2 = 0ull;
 #pragma unroll
@@ -402,8 +461,7 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
       bool bad = !(ss <= 3.402823466e38f) || isinf(__half2float(__float2half_rn(nu)));
       if (bad) nu = 0.f;
 #pragma unroll
-      for (int j = 0; j < D; ++j)
-        x[j] = __uint_as_float(__float_as_uint(x[j]) ^ (((a.dneg[j >> 5] >> (j & 31)) & 1u) << 31));
+      for (int j = 0; j < D / 2; ++j) mul2c(x[j], x[j + D / 2], pk2(a.dsg[2 * j], a.dsg[2 * j + 1]));
       wht_regs<D>(x);
       if (bad || !(nu > 0.f)) {
 #pragma unroll
@@ -415,11 +473,11 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
         // ---------------------------------------------- key row
 #pragma unroll
         for (int j = 0; j < HK - 1; ++j) thr[j] = a.tk[j] * sc;
-        uint32_t pw[PK][NW];
+        uint32_t raw[HK][NW];
 #pragma unroll
-        for (int p = 0; p < PK; ++p)
+        for (int p = 0; p < HK; ++p)
 #pragma unroll
-          for (int w = 0; w < NW; ++w) pw[p][w] = 0u;
+          for (int w = 0; w < NW; ++w) raw[p][w] = 0u;
         uint64_t r2p = 0ull;
         float cks[HK];
 #pragma unroll
@@ -431,13 +489,7 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
 #pragma unroll
         for (int j = D / 2 - 1; j >= 0; --j) {
           constexpr int H2 = D / 2;
-          uint32_t ms0[4], ms1[4];
-          plane_msbs2<MBK>(x[j], x[j + H2], th2, ms0, ms1);
-#pragma unroll
-          for (int p = 0; p < MBK; ++p) {
-            pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
-            pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
-          }
+          raw_bits2<MBK, NW>(x[j], x[j + H2], th2, raw, j, j + H2);
           if (QJL) {
             const float aa0 = fabsf(x[j]), aa1 = fabsf(x[j + H2]);
             float cm0 = cks[0], cm1 = cks[0];
@@ -452,7 +504,8 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
           }
         }
         const float r2 = hsum2(r2p);
-        // funnel shifts accumulated coordinate 32 w + 31 first: bit i = coord 32 w + i
+        uint32_t pw[MBK][NW];
+        planes_of<MBK, NW>(raw, pw);
 #pragma unroll
         for (int p = 0; p < MBK; ++p)
 #pragma unroll
@@ -463,24 +516,21 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
           // tensor memory A: columns [0, D/2) hi, [D/2, D) lo (two bf16 per
           // column, lower K index in the low half); lane = row
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint32_t h32[32], l32[32];
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t h8[8], l8[8];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int j = 32 * c + e;
+            for (int e = 0; e < 8; ++e) {
+              const int j = 8 * c + e;
               const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
               const float2 hf = __bfloat1622float2(hi);
               const __nv_bfloat162 lo = __floats2bfloat162_rn(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
-              h32[e] = *reinterpret_cast<const uint32_t *>(&hi);
-              l32[e] = *reinterpret_cast<const uint32_t *>(&lo);
+              h8[e] = *reinterpret_cast<const uint32_t *>(&hi);
+              l8[e] = *reinterpret_cast<const uint32_t *>(&lo);
             }
-            sm100::tmem_st32(sm100::tmem_lane(tm + 32 * c, wq), h32);
-            sm100::tmem_st32(sm100::tmem_lane(tm + D / 2 + 32 * c, wq), l32);
+            sm100::tmem_st8(sm100::tmem_lane(tmg + 8 * c, wq), h8);
+            sm100::tmem_st8(sm100::tmem_lane(tmg + D / 2 + 8 * c, wq), l8);
           }
           sm100::wait_st();
-          sm100::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&a_ready);
         }
         const int64_t crow = bh * a.rows_cap + R;
         if (active) {
@@ -497,13 +547,37 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
               static_cast<uint32_t>(tq_f32_to_half(nu)) | (static_cast<uint32_t>(tq_f32_to_half(rho)) << 16);
         }
         if (QJL) {
-          if (!wait_or_abort(&z_ready, i & 1, &abort_s)) { abort_s = 1; break; }
+          // every tile's operand is stored: thread 0 issues their sketches
+          if (!(ok = cta_all_ok<QT>(ok))) break;
+          if (tid == 0) {
+#pragma unroll
+            for (int g = 0; g < NTL; ++g) {
+              const uint32_t tg = tm + g * TCOLS;
+#pragma unroll
+              for (int s = 0; s < D / 16; ++s)
+                sm100::mma_f16_ts(tg + D, tg + 8 * s,
+                                  sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
+                                  IDESC, s > 0);
+#pragma unroll
+              for (int s = 0; s < D / 16; ++s)
+                sm100::mma_f16_ts(tg + D, tg + D / 2 + 8 * s,
+                                  sm100::smem_desc(sm100::smem_addr(Bs) + s * 2 * D * 16, D * 16, 128),
+                                  IDESC, 1);
+            }
+            sm100::mma_commit(&z_ready);
+            committed = kz;
+          }
+          if (!wait_or_abort(&z_ready, (kz++) & 1, &abort_s)) {
+            abort_s = 1;
+            ok = false;
+            continue;   // the next step's first barrier takes the CTA out
+          }
           sm100::fence_after_sync();
           uint32_t sg[NW];
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
             uint32_t z[32];
-            sm100::tmem_ld32(sm100::tmem_lane(tm + D + 32 * w, wq), z);
+            sm100::tmem_ld32(sm100::tmem_lane(tmg + D + 32 * w, wq), z);
             sm100::wait_ld();
             uint32_t acc = 0u;
 #pragma unroll
@@ -563,11 +637,16 @@ __global__ void __launch_bounds__(QT, D == 64 ? 2 : 1)
       }
     }
   }
+  if (tid == 0 && abort_s) {
+    // this CTA's own copies and MMAs land before its memory is released
+    if (issued >= 0) sm100::mbar_wait(&full, issued & 1, 1u << 20);
+    if (committed >= 0) sm100::mbar_wait(&z_ready, committed & 1, 1u << 20);
+  }
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
   if (abort_s && tid == 0 && a.status) atomicOr(a.status, 1u << 31);
-  if (QJL && warp == 0) sm100::tmem_dealloc(tm, TCOLS);
+  if (QJL && warp == 0) sm100::tmem_dealloc(tm, NTL * TCOLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -594,7 +673,9 @@ EncodeFn encode_fn() {
 template <int D, int MBK, int BV, bool QJL>
 int run_tile(const TileArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mc,
              const CUtensorMap &ms, cudaStream_t stream) {
-  constexpr size_t shm = 1024 + 4 * (D / 64) * BOX + (QJL ? static_cast<size_t>(D) * D * 2 : 0);
+  constexpr int NTL = tiles_per_unit(D);
+  // the unit's X tiles, the RoPE table tiles and S
+  constexpr size_t shm = 1024 + (NTL + 2) * (D / 64) * BOX + (QJL ? static_cast<size_t>(D) * D * 2 : 0);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -605,12 +686,9 @@ int run_tile(const TileArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, co
       return tq_check_launch("cudaFuncSetAttribute(qtile)");
     done[dev] = true;
   }
-  // resident CTAs per SM: two at d = 64 (shared memory, registers and 2 x 128
-  // tensor-memory columns all fit), one at d = 128
-  const int per_sm = D == 64 ? 2 : 1;
-  const int64_t cap = static_cast<int64_t>(sms) * per_sm;
-  const int grid = static_cast<int>(a.ntiles < cap ? a.ntiles : cap);
-  qtile_kernel<D, MBK, BV, QJL><<<grid, QT, shm, stream>>>(mk, mv, mc, ms, a);
+  // one CTA per SM (its tensor memory takes all 512 columns)
+  const int grid = static_cast<int>(a.nunits < sms ? a.nunits : sms);
+  qtile_kernel<D, MBK, BV, QJL><<<grid, 128 * NTL, shm, stream>>>(mk, mv, mc, ms, a);
   tq_count_launch(1);
   return tq_check_launch("qtile_kernel");
 }
@@ -654,7 +732,9 @@ int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dt
   a.rows_cap = cache->rows_cap;
   a.R_first = row0 / QR * QR;
   a.nrt = (row0 + T - 1) / QR - row0 / QR + 1;
-  a.ntiles = a.nrt * B * H;
+  const int ntl = tiles_per_unit(d);
+  a.groups = (static_cast<int64_t>(B) * H + ntl - 1) / ntl;
+  a.nunits = 2 * a.nrt * a.groups;
   a.kcode = cache->kcode;
   a.kscale = cache->kscale;
   a.vcode = cache->vcode;
@@ -668,7 +748,11 @@ int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dt
     a.tk[m] = m < hk - 1 ? c->books.tk[hk + m] : 0.f;
     a.tv[m] = m < hv - 1 ? c->books.tv[hv + m] : 0.f;
   }
-  for (int w = 0; w < 4; ++w) a.dneg[w] = w < d / 32 ? c->books.dneg[w] : 0u;
+  for (int j = 0; j < 64; ++j) {
+    const auto sgn = [&](int i) { return i < d && ((c->books.dneg[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f; };
+    a.dsg[2 * j] = sgn(j);
+    a.dsg[2 * j + 1] = sgn(j + d / 2);
+  }
   // tensor maps: K and V [B][H][T][d] bf16 (4-D, innermost d); RoPE tables [pos0 + T][d/2] fp32
   CUtensorMap mk, mv, mc, ms;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),

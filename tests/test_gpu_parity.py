@@ -47,6 +47,11 @@ QUANT_CASES = {
     "esm_tile_mse3_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=100, qjl_k=False, bits_k=3),
                           [(0, 100)]),
     "esm_tile_offset_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=4, T=300), [(0, 45), (45, 255)]),
+    # an odd number of (batch, head) rows: the tile kernel's last step holds one tile
+    "esm_tile_odd_heads_d64": (synth.WORKLOADS["esm_prefill"].scaled(B=1, Hq=3, Hkv=3, T=2800),
+                               [(0, 2800)]),
+    "llama_tile_odd_heads": (synth.WORKLOADS["llama_decode"].scaled(B=1, Hq=20, Hkv=5, T=3600),
+                             [(0, 1700), (1700, 1900)]),
 }
 
 
