@@ -255,6 +255,40 @@ __device__ __forceinline__ void plane_msbs2(float y0, float y1, const uint64_t *
   }
 }
 
+// The code planes below the top one for two coordinates, without their sign
+// term (plane_msbs's thermometer XORs with sy left out): word p's top bit is
+// plane p's bit for |y| alone.  a0, a1: |y|; th2: packed thresholds above 0
+// times the row scale.
+template <int NB>
+__device__ __forceinline__ void therm_msbs2(float a0, float a1, const uint64_t *th2, uint32_t (&w0)[4],
+                                            uint32_t (&w1)[4]) {
+  constexpr int NT = (1 << (NB - 1)) - 1;   // thresholds above 0
+  uint32_t s0[NT > 0 ? NT : 1], s1[NT > 0 ? NT : 1];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    float d0, d1;
+    sub2c(a0, a1, th2[j], d0, d1);
+    s0[j] = __float_as_uint(d0);
+    s1[j] = __float_as_uint(d1);
+  }
+  if constexpr (NB == 2) {
+    w0[0] = s0[0];
+    w1[0] = s1[0];
+  } else if constexpr (NB == 3) {
+    w0[1] = s0[1];
+    w0[0] = s0[0] ^ s0[1] ^ s0[2];
+    w1[1] = s1[1];
+    w1[0] = s1[0] ^ s1[1] ^ s1[2];
+  } else if constexpr (NB == 4) {
+    w0[2] = s0[3];
+    w0[1] = s0[1] ^ s0[3] ^ s0[5];
+    w0[0] = s0[0] ^ s0[1] ^ s0[2] ^ s0[3] ^ s0[4] ^ s0[5] ^ s0[6];
+    w1[2] = s1[3];
+    w1[1] = s1[1] ^ s1[3] ^ s1[5];
+    w1[0] = s1[0] ^ s1[1] ^ s1[2] ^ s1[3] ^ s1[4] ^ s1[5] ^ s1[6];
+  }
+}
+
 // Raw decision bits of coordinates i and i + D/2, accumulated one funnel shift
 // per bit (coordinate 32 w + 31 first, so bit e of word w is coordinate
 // 32 w + e): acc[t] gathers the sign bits of |y| - th[t] (t < NT, th2[t] =
@@ -296,21 +330,33 @@ __device__ __forceinline__ void planes_of(const uint32_t (&r)[1 << (NB - 1)][NW]
   }
 }
 
-// 32 x 32 bit transpose across a warp: on return bit L of lane i's word is
-// bit i of lane L's input word.
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
-  const uint32_t masks[5] = {0xffff0000u, 0xff00ff00u, 0xf0f0f0f0u, 0xccccccccu, 0xaaaaaaaau};
+// 32 x 32 bit transposes across a warp: on return bit L of lane i's word is
+// bit i of lane L's input word.  Stage j (16, 8, 4, 2, 1) swaps j-bit blocks
+// between lanes i and i ^ j: the partner's word rotated left by j (lanes
+// without bit j) or right by j (lanes with it) brings the wanted block into
+// place, and one bitwise select keeps the rest of the lane's own word.
+struct WarpTranspose {
+  uint32_t keep[5], rot[5];
+  __device__ __forceinline__ explicit WarpTranspose(int lane) {
+    const uint32_t masks[5] = {0xffff0000u, 0xff00ff00u, 0xf0f0f0f0u, 0xccccccccu, 0xaaaaaaaau};
 #pragma unroll
-  for (int st = 0; st < 5; ++st) {
-    const int j = 16 >> st;
-    const uint32_t y = __shfl_xor_sync(TQ_FULL, x, j);
-    const bool hi = lane & j;
-    // lanes without bit j take the partner's low bits into their high
-    // positions; lanes with bit j take the partner's high bits into their low
-    x = hi ? ((x & masks[st]) | ((y >> j) & ~masks[st])) : ((x & ~masks[st]) | ((y << j) & masks[st]));
+    for (int st = 0; st < 5; ++st) {
+      const int j = 16 >> st;
+      const bool hi = lane & j;
+      keep[st] = hi ? masks[st] : ~masks[st];
+      rot[st] = hi ? 32u - j : static_cast<uint32_t>(j);
+    }
   }
-  return x;
-}
+  __device__ __forceinline__ uint32_t operator()(uint32_t x) const {
+#pragma unroll
+    for (int st = 0; st < 5; ++st) {
+      const uint32_t y = __shfl_xor_sync(TQ_FULL, x, 16 >> st);
+      const uint32_t r = __funnelshift_l(y, y, rot[st]);
+      x = (x & keep[st]) | (r & ~keep[st]);
+    }
+    return x;
+  }
+};
 
 template <int D, int MBK, int BV, bool QJL>
 __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
@@ -604,15 +650,43 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
         uint64_t th2[HV > 1 ? HV - 1 : 1];
 #pragma unroll
         for (int j = 0; j < HV - 1; ++j) th2[j] = pk2(thr[j], thr[j]);
+        if constexpr (BV < 3) {
 #pragma unroll
-        for (int j = D / 2 - 1; j >= 0; --j) {
-          constexpr int H2 = D / 2;
-          uint32_t ms0[4], ms1[4];
-          plane_msbs2<BV>(x[j], x[j + H2], th2, ms0, ms1);
+          for (int j = D / 2 - 1; j >= 0; --j) {
+            constexpr int H2 = D / 2;
+            uint32_t ms0[4], ms1[4];
+            plane_msbs2<BV>(x[j], x[j + H2], th2, ms0, ms1);
 #pragma unroll
-          for (int p = 0; p < BV; ++p) {
-            pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
-            pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
+            for (int p = 0; p < BV; ++p) {
+              pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
+              pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
+            }
+          }
+        } else {
+          // the planes below the top one without their sign term (the
+          // thermometer XORs of plane_msbs with sy left out) and the sign
+          // word beside them; the sign goes into the lower planes once per word
+          uint32_t syw[NW];
+#pragma unroll
+          for (int w = 0; w < NW; ++w) syw[w] = 0u;
+#pragma unroll
+          for (int j = D / 2 - 1; j >= 0; --j) {
+            constexpr int H2 = D / 2;
+            uint32_t ms0[4], ms1[4];
+            therm_msbs2<BV>(fabsf(x[j]), fabsf(x[j + H2]), th2, ms0, ms1);
+#pragma unroll
+            for (int p = 0; p < BV - 1; ++p) {
+              pw[p][j >> 5] = __funnelshift_l(ms0[p], pw[p][j >> 5], 1);
+              pw[p][(j + H2) >> 5] = __funnelshift_l(ms1[p], pw[p][(j + H2) >> 5], 1);
+            }
+            syw[j >> 5] = __funnelshift_l(__float_as_uint(x[j]), syw[j >> 5], 1);
+            syw[(j + H2) >> 5] = __funnelshift_l(__float_as_uint(x[j + H2]), syw[(j + H2) >> 5], 1);
+          }
+#pragma unroll
+          for (int w = 0; w < NW; ++w) {
+#pragma unroll
+            for (int p = 0; p < BV - 1; ++p) pw[p][w] ^= syw[w];
+            pw[BV - 1][w] = syw[w];
           }
         }
         const int64_t crow = bh * a.rows_cap + R;
@@ -620,11 +694,12 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
         // column words: lane i gets coordinate 32 w + i of the warp's 32 rows
         const uint32_t act = __ballot_sync(TQ_FULL, active);
         uint32_t *vg = a.vcode + (bh * (a.rows_cap / 32) + (R >> 5)) * (BV * D);
+        const WarpTranspose tp(lane);
 #pragma unroll
         for (int p = 0; p < BV; ++p) {
 #pragma unroll
           for (int w = 0; w < NW; ++w) {
-            const uint32_t col = warp_transpose32(~pw[p][w], lane);
+            const uint32_t col = tp(~pw[p][w]);
             uint32_t *dst = vg + p * D + 32 * w + lane;
             if (act == TQ_FULL) {
               *dst = col;
