@@ -151,6 +151,14 @@ __device__ __forceinline__ void sub2c(float a0, float a1, uint64_t c, float &d0,
       : "f"(a0), "f"(a1), "l"(c));
 }
 
+// (d0, d1) = (a0, a1) - (b0, b1)
+__device__ __forceinline__ void sub2(float a0, float a1, float b0, float b1, float &d0, float &d1) {
+  asm("{\n\t.reg .b64 p, q, d;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, p, q;\n\tmov.b64 {%0, %1}, d;\n\t}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // (a0, a1) *= c (exact for c = (+-1, +-1))
 __device__ __forceinline__ void mul2c(float &a0, float &a1, uint64_t c) {
   asm("{\n\t.reg .b64 p, d;\n\tmov.b64 p, {%0, %1};\n\tmul.rn.f32x2 d, p, %2;\n\t"
@@ -537,6 +545,7 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
           constexpr int H2 = D / 2;
           raw_bits2<MBK, NW>(x[j], x[j + H2], th2, raw, j, j + H2);
           if (QJL) {
+            // residual (scaled by sc): y - sign(y) c_m = sign(y) (|y| - c_m)
             const float aa0 = fabsf(x[j]), aa1 = fabsf(x[j + H2]);
             float cm0 = cks[0], cm1 = cks[0];
 #pragma unroll
@@ -544,9 +553,11 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
               cm0 = aa0 >= thr[m - 1] ? cks[m] : cm0;
               cm1 = aa1 >= thr[m - 1] ? cks[m] : cm1;
             }
-            const float cv0 = x[j] >= 0.f ? cm0 : -cm0, cv1 = x[j + H2] >= 0.f ? cm1 : -cm1;
-            sub2c(x[j], x[j + H2], pk2(cv0, cv1), x[j], x[j + H2]);   // residual (scaled by sc)
-            sq2acc(x[j], x[j + H2], r2p);
+            float r0, r1;
+            sub2c(aa0, aa1, pk2(cm0, cm1), r0, r1);
+            sq2acc(r0, r1, r2p);
+            x[j] = __uint_as_float(__float_as_uint(r0) ^ (__float_as_uint(x[j]) & 0x80000000u));
+            x[j + H2] = __uint_as_float(__float_as_uint(r1) ^ (__float_as_uint(x[j + H2]) & 0x80000000u));
           }
         }
         const float r2 = hsum2(r2p);
@@ -569,7 +580,9 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
               const int j = 8 * c + e;
               const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
               const float2 hf = __bfloat1622float2(hi);
-              const __nv_bfloat162 lo = __floats2bfloat162_rn(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
+              float l0, l1;
+              sub2(x[2 * j], x[2 * j + 1], hf.x, hf.y, l0, l1);
+              const __nv_bfloat162 lo = __floats2bfloat162_rn(l0, l1);
               h8[e] = *reinterpret_cast<const uint32_t *>(&hi);
               l8[e] = *reinterpret_cast<const uint32_t *>(&lo);
             }
