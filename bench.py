@@ -311,30 +311,25 @@ def time_decode(bench: DecodeBench, K: int, W: int, world: int, sampler):
 
 
 def time_e2e(bench: DecodeBench, K: int, W: int):
-    """Same step through the public API with host buffers: pinned H2D of the new
-    token's K/V and the query, the calls, D2H of the output, host sync each step."""
+    """Same step through the public API with host buffers: one tq_decode_step_host
+    call per step copies the new token's K/V and the query from pinned host
+    memory, runs the step and returns with the output in pinned host memory."""
     import torch
+    native = bench.native
     # the step's inputs (new token's K and V, the query) packed in one pinned
     # host buffer, so each step is one host-to-device copy
     parts = (bench.knew, bench.vnew, bench.q)
     assert len({t.dtype for t in parts}) == 1
-    sizes = [t.numel() for t in parts]
-    hbuf = torch.empty(sum(sizes), dtype=parts[0].dtype).pin_memory()
+    hbuf = torch.cat([t.reshape(-1).cpu() for t in parts]).pin_memory()
     dbuf = torch.empty_like(hbuf, device=bench.q.device)
-    views, off = [], 0
-    for t, n in zip(parts, sizes):
-        hbuf[off:off + n].copy_(t.reshape(-1).cpu())
-        views.append(dbuf[off:off + n].view(t.shape))
-        off += n
-    kd, vd, qd = views
     oh = torch.empty(bench.out.shape, dtype=torch.float32).pin_memory()
-    stream = torch.cuda.current_stream()
+    w = bench.w
+    kvt, qt = bench.knew.dtype, bench.q.dtype
 
     def one(i):
-        dbuf.copy_(hbuf, non_blocking=True)
-        bench.step(i, kd, vd, qd)
-        oh.copy_(bench.out, non_blocking=True)
-        stream.synchronize()
+        native.decode_step_host(bench.codec, hbuf, dbuf, kvt, qt, w.B, w.Hq, w.Hkv,
+                                bench.caches[i % bench.n_sets], w.T, bench.scale, bench.out, oh,
+                                bench.ws, rope=bench.rope, num_splits=bench.splits)
 
     for i in range(W):
         one(i)

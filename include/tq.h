@@ -214,6 +214,24 @@ int tq_decode_step(const tq_codec *codec, const void *k_new, const void *v_new, 
                    float scale, const float *rope_cos, const float *rope_sin, int num_splits,
                    void *workspace, size_t ws_bytes, float *out, void *stream);
 
+/* tq_decode_step fed from and read back to host memory, for a caller whose
+ * new token and query live on the host.  The step's input is one host buffer
+ * holding k_new [B][Hkv][d], v_new [B][Hkv][d] (both kv_dtype) and q
+ * [B][Hq][d] (q_dtype), in that order, each part starting where the previous
+ * one ends; in_bytes is its total size.  The call copies it to the device
+ * buffer in_dev (in_bytes, 16-byte aligned; owned by the caller), runs
+ * tq_decode_step over the three parts, copies out_dev (device fp32
+ * [B][Hq][d]) to out_host, and returns once out_host holds the result (the
+ * stream is synchronised).  in_host and out_host should be page-locked for
+ * the copies to run asynchronously; pageable memory works, more slowly.
+ * Errors: those of tq_decode_step, TQ_ERR_INVALID_ARG for NULL buffers or
+ * an in_bytes that is not the parts' total, TQ_ERR_CUDA for a failed copy. */
+int tq_decode_step_host(const tq_codec *codec, const void *in_host, void *in_dev, size_t in_bytes,
+                        int kv_dtype, int q_dtype, int B, int Hq, int Hkv, const tq_cache *cache,
+                        int T, float scale, const float *rope_cos, const float *rope_sin,
+                        int num_splits, void *workspace, size_t ws_bytes, float *out_dev,
+                        float *out_host, void *stream);
+
 /* Same as tq_attention_decode, and also writes the estimated logits
  * l_j (the formula above, scale included) of every query head:
  * logits  device fp32 [B][Hq][max_seq_len]; entries j >= T_b are left

@@ -376,6 +376,42 @@ int tq_decode_step(const tq_codec *c, const void *k_new, const void *v_new, int 
                        num_splits, workspace, ws_bytes, out, nullptr, stream);
 }
 
+int tq_decode_step_host(const tq_codec *c, const void *in_host, void *in_dev, size_t in_bytes,
+                        int kv_dtype, int q_dtype, int B, int Hq, int Hkv, const tq_cache *cache,
+                        int T, float scale, const float *rope_cos, const float *rope_sin,
+                        int num_splits, void *workspace, size_t ws_bytes, float *out_dev,
+                        float *out_host, void *stream) {
+  if (!c) return tq_fail(TQ_ERR_INVALID_ARG, "decode step (host): NULL codec");
+  if (!in_host || !in_dev || !out_dev || !out_host)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode step (host): NULL buffer");
+  const size_t kvs = kv_dtype == TQ_BF16 ? 2 : 4, qs = q_dtype == TQ_BF16 ? 2 : 4;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode step (host): bad shape");
+  const size_t kv_part = static_cast<size_t>(B) * Hkv * c->d * kvs;
+  const size_t q_part = static_cast<size_t>(B) * Hq * c->d * qs;
+  if (in_bytes != 2 * kv_part + q_part)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode step (host): in_bytes is not the size of k_new, v_new and q");
+  if (reinterpret_cast<uintptr_t>(in_dev) % 16)
+    return tq_fail(TQ_ERR_INVALID_ARG, "decode step (host): in_dev not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto cuda_fail = [](cudaError_t e, const char *what) {
+    cudaGetLastError();   // the error is reported here, not left for a later call
+    return tq_fail(TQ_ERR_CUDA, std::string("decode step (host): ") + what + ": " + cudaGetErrorString(e));
+  };
+  if (cudaError_t e = cudaMemcpyAsync(in_dev, in_host, in_bytes, cudaMemcpyHostToDevice, st))
+    return cuda_fail(e, "input copy");
+  const uint8_t *base = static_cast<const uint8_t *>(in_dev);
+  if (int e = tq_decode_step(c, base, base + kv_part, kv_dtype, base + 2 * kv_part, q_dtype, B, Hq, Hkv,
+                             cache, T, scale, rope_cos, rope_sin, num_splits, workspace, ws_bytes,
+                             out_dev, stream))
+    return e;
+  const size_t out_bytes = static_cast<size_t>(B) * Hq * c->d * sizeof(float);
+  if (cudaError_t e = cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, st))
+    return cuda_fail(e, "output copy");
+  if (cudaError_t e = cudaStreamSynchronize(st)) return cuda_fail(e, "synchronise");
+  return TQ_OK;
+}
+
 int tq_attention_logits(const tq_codec *c, const void *q, int dtype, int B, int Hq, int Hkv,
                         const tq_cache *cache, const int32_t *seq_lens, int max_seq_len,
                         float scale, const float *rope_cos, const float *rope_sin,

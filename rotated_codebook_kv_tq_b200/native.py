@@ -23,7 +23,7 @@ TQ_F32, TQ_BF16 = 0, 1
 EXPORTS = [
     "tq_build_codebook", "tq_codec_create", "tq_codec_destroy", "tq_codec_codebooks",
     "tq_cache_bytes", "tq_quantize_kv", "tq_attention_workspace", "tq_attention_decode",
-    "tq_attention_logits", "tq_decode_step", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
+    "tq_attention_logits", "tq_decode_step", "tq_decode_step_host", "tq_attention_decode_noalloc", "tq_attention_bidir_workspace",
     "tq_attention_bidir", "tq_index_workspace", "tq_index_build", "tq_scan_workspace",
     "tq_scan_topk", "tq_scan_topk_lut", "tq_dequantize", "tq_split_channels",
     "tq_quantize_kv_split", "tq_attention_split_workspace", "tq_attention_decode_split",
@@ -89,6 +89,9 @@ def lib() -> ctypes.CDLL:
         L.tq_decode_step.argtypes = [vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                      ctypes.POINTER(CacheDesc), i32, ctypes.c_float, vp, vp, i32,
                                      vp, sz, vp, vp]
+        L.tq_decode_step_host.argtypes = [vp, vp, vp, sz, i32, i32, i32, i32, i32,
+                                          ctypes.POINTER(CacheDesc), i32, ctypes.c_float, vp, vp, i32,
+                                          vp, sz, vp, vp, vp]
         L.tq_attention_decode_noalloc.argtypes = [vp, vp, i32, i32, i32, i32,
                                                   ctypes.POINTER(CacheDesc), vp, i32, f32, vp,
                                                   vp, i32, vp, vp]
@@ -253,14 +256,18 @@ _DTYPES = None
 
 
 def _dtype_code(t) -> int:
+    return _code_of(t.dtype)
+
+
+def _code_of(dtype) -> int:
     global _DTYPES
     if _DTYPES is None:
         import torch
         _DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.int16: TQ_BF16,
                    torch.uint16: TQ_BF16}
-    code = _DTYPES.get(t.dtype)
+    code = _DTYPES.get(dtype)
     if code is None:
-        raise TypeError(f"unsupported dtype {t.dtype}")
+        raise TypeError(f"unsupported dtype {dtype}")
     return code
 
 
@@ -314,6 +321,22 @@ def decode_step(codec: Codec, k_new, v_new, q, cache: Cache, T: int, scale: floa
                                float(scale), _ptr(rc), _ptr(rs), num_splits, workspace.data_ptr(),
                                workspace.numel() * workspace.element_size(), out.data_ptr(),
                                _stream(stream)))
+
+
+def decode_step_host(codec: Codec, in_host, in_dev, kv_dtype, q_dtype, B: int, Hq: int, Hkv: int,
+                     cache: Cache, T: int, scale: float, out_dev, out_host, workspace, rope=None,
+                     num_splits: int = 0, stream=None) -> None:
+    """tq_decode_step_host: in_host (pinned) holds k_new, v_new [B, Hkv, d] and
+    q [B, Hq, d] back to back; it is copied to in_dev, the step runs, out_dev
+    is copied to out_host and the call returns with the result on the host."""
+    rc, rs = (None, None) if rope is None else rope
+    desc = cache.desc()
+    check(lib().tq_decode_step_host(codec.handle, in_host.data_ptr(), in_dev.data_ptr(),
+                                    in_host.numel() * in_host.element_size(), _code_of(kv_dtype),
+                                    _code_of(q_dtype), B, Hq, Hkv, ctypes.byref(desc), T, float(scale),
+                                    _ptr(rc), _ptr(rs), num_splits, workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(), out_dev.data_ptr(),
+                                    out_host.data_ptr(), _stream(stream)))
 
 
 def attention_logits(codec: Codec, q, cache: Cache, max_seq_len: int, scale: float, out,

@@ -270,7 +270,8 @@ def test_decode_rejects_bad_arguments():
 
 def test_decode_step_equals_append_then_decode():
     """tq_decode_step is tq_quantize_kv at row T - 1 followed by
-    tq_attention_decode over T rows: same cache bytes, same output bits."""
+    tq_attention_decode over T rows: same cache bytes, same output bits; so is
+    tq_decode_step_host, fed from and read back to host memory."""
     w = synth.WORKLOADS["llama_decode"].scaled(B=2, Hq=8, Hkv=2, T=333)
     _, ncodec = tl.codecs(w)
     K, V = synth.kv_inputs(w)
@@ -278,21 +279,36 @@ def test_decode_step_equals_append_then_decode():
     q = tl.to_device(np.ascontiguousarray(synth.query_inputs(w, Lq=1)[:, :, 0]), w.dtype)
     rope = tl.rope_device(synth.rope_for(w, 352))
     caches, outs = [], []
-    for fused in (False, True):
+    for mode in ("separate", "fused", "host"):
         c = native.alloc_cache(ncodec, w.B, w.Hkv, 352)
         native.quantize_kv(ncodec, kd[:, :, :w.T - 1], vd[:, :, :w.T - 1], c, rope=rope)
         out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
         ws = torch.empty(native.attention_workspace(ncodec, w.B, w.Hq, 5), dtype=torch.uint8,
                          device="cuda")
         kn, vn = kd[:, :, w.T - 1:].contiguous(), vd[:, :, w.T - 1:].contiguous()
-        if fused:
+        if mode == "fused":
             native.decode_step(ncodec, kn, vn, q, c, w.T, 0.088, out, ws, rope=rope, num_splits=5)
+        elif mode == "host":
+            # the three parts back to back in one pinned host buffer, the
+            # output read back into pinned host memory by the call itself
+            hin = torch.cat([kn.reshape(-1), vn.reshape(-1), q.reshape(-1)]).cpu().pin_memory()
+            din = torch.empty_like(hin, device="cuda")
+            hout = torch.full((w.B, w.Hq, w.d), float("nan")).pin_memory()
+            native.decode_step_host(ncodec, hin, din, kn.dtype, q.dtype, w.B, w.Hq, w.Hkv, c, w.T, 0.088,
+                                    out, hout, ws, rope=rope, num_splits=5)
+            assert torch.equal(hout, out.cpu())
         else:
             native.quantize_kv(ncodec, kn, vn, c, row0=w.T - 1, rope=rope, pos0=w.T - 1)
             native.attention_decode(ncodec, q, c, w.T, 0.088, out, ws, rope=rope, num_splits=5)
         torch.cuda.synchronize()
         caches.append(tl.download_cache(c))
         outs.append(out.cpu().numpy())
-    for key in ("kcode", "kscale", "vcode", "vnorm"):
-        assert np.array_equal(caches[0][key], caches[1][key]), key
-    assert np.array_equal(outs[0], outs[1])
+    for i in (1, 2):
+        for key in ("kcode", "kscale", "vcode", "vnorm"):
+            assert np.array_equal(caches[0][key], caches[i][key]), (i, key)
+        assert np.array_equal(outs[0], outs[i]), i
+    # the input size must be the parts' total
+    with pytest.raises(native.TqError) as e:
+        native.decode_step_host(ncodec, hin[:-8], din, kn.dtype, q.dtype, w.B, w.Hq, w.Hkv, c, w.T,
+                                0.088, out, hout, ws, rope=rope, num_splits=5)
+    assert e.value.code == native.TQ_ERR_INVALID_ARG

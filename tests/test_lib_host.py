@@ -40,6 +40,13 @@ def test_exports_every_declared_symbol(L):
     assert set(names) == set(native.EXPORTS)
 
 
+def test_every_call_has_a_ctypes_signature(L):
+    # without argtypes, ctypes cannot pass a Python float as a C float
+    for n in native.EXPORTS:
+        if n != "tq_last_error":
+            assert getattr(L, n).argtypes is not None, n
+
+
 @pytest.mark.parametrize("d,bits", [(64, 2), (64, 3), (128, 1), (128, 2), (128, 3), (128, 4)])
 def test_host_codebook_matches_oracle(L, d, bits):
     c, t, mse = native.build_codebook(d, bits)
