@@ -450,6 +450,7 @@ constexpr int UMAX = 1024;     // rows per unit
 constexpr int KS = 4;          // key tile stages (shared memory)
 constexpr int VS = 8;          // value group stages (shared memory)
 constexpr int VB = 4;          // value groups per batch
+static_assert(VB % 2 == 0, "value groups are expanded in pairs");
 constexpr int DCOLS = 256;     // tensor memory per CTA
 
 struct DecLayout {
@@ -865,32 +866,47 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
         // the buffer's previous batch (vbi - 2) has been multiplied
         if (vbi >= 2 && ok) ok = dwait(&vdone[vbi & 1], ((vbi >> 1) - 1) & 1, outer, &abort_s);
         if (ok) sm100::fence_after_sync();
+        // the batch's groups: every wait first, then the column words of all
+        // of them, then the expansion as straight-line code (two groups at
+        // a time, so their independent chains interleave).  A group past the
+        // unit's end is expanded from whatever its stage holds and never
+        // multiplied; only real groups release their stages.
+        const int gcount = min(VB, ngroups - bi * VB);
 #pragma unroll
         for (int gi = 0; gi < VB; ++gi) {
-          const int g = bi * VB + gi;
-          if (g >= ngroups) break;
-          const uint32_t vgg = vg + g;
-          const int s = vgg % VS;
-          if (ok) ok = dwait(&vf[s], (vgg / VS) & 1, outer, &abort_s);
-          if (ok) {
-            const uint32_t *vc = reinterpret_cast<const uint32_t *>(smem + L.o_vt + s * L.vgb);
-            uint32_t pv[BV];
+          const uint32_t vgg = vg + bi * VB + gi;
+          if (gi < gcount && ok) ok = dwait(&vf[vgg % VS], (vgg / VS) & 1, outer, &abort_s);
+        }
+        if (ok) {
+          uint32_t pv[VB][BV];
 #pragma unroll
-            for (int p = 0; p < BV; ++p) pv[p] = vc[p * TD + tid];
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&ve[s]);
+          for (int gi = 0; gi < VB; ++gi) {
+            const uint32_t *vc =
+                reinterpret_cast<const uint32_t *>(smem + L.o_vt + ((vg + bi * VB + gi) % VS) * L.vgb);
+#pragma unroll
+            for (int p = 0; p < BV; ++p) pv[gi][p] = vc[p * TD + tid];
+          }
+          __syncwarp();
+          if (lane < gcount) sm100::mbar_arrive(&ve[(vg + bi * VB + lane) % VS]);
+#pragma unroll
+          for (int g2 = 0; g2 < VB; g2 += 2) {
             if constexpr (VDIG) {
-              uint32_t dw[NDIG][8];
-              digit_words<BV>(pv, vtab, dw);
+              uint32_t dw[2][NDIG][8];
+              digit_words<BV>(pv[g2], vtab, dw[0]);
+              digit_words<BV>(pv[g2 + 1], vtab, dw[1]);
 #pragma unroll
-              for (int k = 0; k < NDIG; ++k) sm100::tmem_st8(abuf + gi * NV * 8 + 8 * k, dw[k]);
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int k = 0; k < NDIG; ++k) sm100::tmem_st8(abuf + (g2 + e) * NV * 8 + 8 * k, dw[e][k]);
             } else {
 #pragma unroll
-              for (int t = 0; t < NV; ++t) {
-                uint32_t r8[8];
-                plane_words(pv[t], r8);
-                sm100::tmem_st8(abuf + gi * NV * 8 + 8 * t, r8);
-              }
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int t = 0; t < NV; ++t) {
+                  uint32_t r8[8];
+                  plane_words(pv[g2 + e][t], r8);
+                  sm100::tmem_st8(abuf + (g2 + e) * NV * 8 + 8 * t, r8);
+                }
             }
           }
         }
