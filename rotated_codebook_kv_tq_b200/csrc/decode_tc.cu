@@ -811,6 +811,10 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
           const int w = (it / NH) & 7, g = it / (8 * NH);
           uint32_t word[4] = {0u, 0u, 0u, 0u};
           if (h < G) {
+            // v + 0x808080 = sum_l 256^l b_l: limbs l < 3 are b_l - 128 (the
+            // byte XOR 0x80), limb 3 is b_3; a 4 x 4 byte transpose gathers
+            // limb l of the four tokens into word l
+            uint32_t bv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int rl = 32 * g + elem_of(VDIG, 4 * w + e);
@@ -821,14 +825,15 @@ __global__ void __launch_bounds__(DT, 2) dec_kernel(TcArgs a) {
                 W = __float2int_rn(p * tq_half_to_f32(vn[rl]) * FV);
               }
               wpart += W;
-              int v = VDIG ? W : W * (1 << (7 - w));
-#pragma unroll
-              for (int l = 0; l < 4; ++l) {
-                const int8_t dgt = static_cast<int8_t>(v & 0xff);
-                word[l] |= static_cast<uint32_t>(static_cast<uint8_t>(dgt)) << (8 * e);
-                v = (v - dgt) >> 8;
-              }
+              const int v = VDIG ? W : W * (1 << (7 - w));
+              bv[e] = static_cast<uint32_t>(v) + 0x808080u;
             }
+            const uint32_t lo01 = prmt(bv[0], bv[1], 0x5140u), hi01 = prmt(bv[0], bv[1], 0x7362u);
+            const uint32_t lo23 = prmt(bv[2], bv[3], 0x5140u), hi23 = prmt(bv[2], bv[3], 0x7362u);
+            word[0] = prmt(lo01, lo23, 0x5410u) ^ 0x80808080u;
+            word[1] = prmt(lo01, lo23, 0x7632u) ^ 0x80808080u;
+            word[2] = prmt(hi01, hi23, 0x5410u) ^ 0x80808080u;
+            word[3] = prmt(hi01, hi23, 0x7632u);
           }
           int8_t *dst = bvs + g * N * 32;
 #pragma unroll
