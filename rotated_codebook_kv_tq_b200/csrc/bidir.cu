@@ -473,21 +473,22 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     const int c0 = KPT * hf;
     float sv[KPT];
     {
-      uint32_t rr[16];
+      // the five accumulators in two rounds of loads in flight together
 #pragma unroll
       for (int c = 0; c < KPT; c += 16) {
-        sm100::tmem_ld16(sm100::tmem_lane(tS0 + c0 + c, lq), rr);
+        uint32_t r0[16], r1[16], r2[16];
+        sm100::tmem_ld16(sm100::tmem_lane(tS0 + c0 + c, lq), r0);
+        sm100::tmem_ld16(sm100::tmem_lane(tS1 + c0 + c, lq), r1);
+        sm100::tmem_ld16(sm100::tmem_lane(tS2 + c0 + c, lq), r2);
         sm100::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c + e] = __uint_as_float(rr[e]);
-        const uint32_t others[4] = {tS1, tS2, tSb, tSb + BK};
+        for (int e = 0; e < 16; ++e)
+          sv[c + e] = (__uint_as_float(r0[e]) + __uint_as_float(r1[e])) + __uint_as_float(r2[e]);
+        sm100::tmem_ld16(sm100::tmem_lane(tSb + c0 + c, lq), r0);
+        sm100::tmem_ld16(sm100::tmem_lane(tSb + BK + c0 + c, lq), r1);
+        sm100::wait_ld();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sm100::tmem_ld16(sm100::tmem_lane(others[i] + c0 + c, lq), rr);
-          sm100::wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) sv[c + e] += __uint_as_float(rr[e]);
-        }
+        for (int e = 0; e < 16; ++e) sv[c + e] += __uint_as_float(r0[e]) + __uint_as_float(r1[e]);
       }
     }
     float tmax = -CUDART_INF_F;
@@ -498,9 +499,13 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     }
     xmax[hf][r] = tmax;
     __syncthreads();
-    float mn = m;
+    float tmx = -CUDART_INF_F;
 #pragma unroll
-    for (int i = 0; i < PR; ++i) mn = fmaxf(mn, xmax[i][r]);
+    for (int i = 0; i < PR; ++i) tmx = fmaxf(tmx, xmax[i][r]);
+    // the reference maximum of the row moves only when a tile exceeds it by
+    // more than 8 (so exp(s - m) stays below e^8): the running output is
+    // rescaled in tensor memory rarely, not on most tiles
+    const float mn = tmx > m + 8.f ? tmx : m;
     const float corr = __expf(m - mn);
     // P nu_v (the value norms of the keys, so V_rot holds centroids only),
     // as a two-term bf16 split: its 2^-17 error reaches the output directly,
