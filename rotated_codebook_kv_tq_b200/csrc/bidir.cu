@@ -331,143 +331,172 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     sm100::bulk_g2s(st + 4352, a.vnorm + bh * a.rows_cap + j0, bn, &kvf[jt & 1]);
   };
   const int ntiles = (a.T + BK - 1) / BK;
-  if (tid == 0 && ntiles > 0) issue_tile(0);
-  int issued = ntiles > 0 ? 1 : 0;   // tiles whose copies were issued (thread 0)
+  // thread 0: the parity of the last copy issued into each stage (-1: none)
+  int last_par[2] = {-1, -1};
+  auto issue_next = [&](int jt) {
+    issue_tile(jt);
+    last_par[jt & 1] = (jt >> 1) & 1;
+  };
+  if (tid == 0) {
+    if (ntiles > 0) issue_next(0);
+    if (ntiles > 1) issue_next(1);
+  }
+  // The tile loop is software-pipelined so that each MMA set overlaps the
+  // CUDA-core work of the next step:
+  //   softmax(j) -> P(j) | issue O(j) | expand K(j+1) while O(j) runs |
+  //   issue S(j+1) | wait O(j) | expand V(j+1) while S(j+1) runs | wait S(j+1)
+  // Buffers: K_rot (ks3) is rewritten once S(j) has completed, V_rot (vs3)
+  // and P (ps3) once O(j) has; the nu_k / nu_v arrays of tile j+1 are
+  // written after softmax(j) has read tile j's.  A two-stage ring holds the
+  // compressed rows; tile j+2 is copied into the stage of tile j once both of
+  // its expansions are done.
+  auto expand_k = [&](int jt) {
+    const int j0 = jt * BK;
+    const uint8_t *st = stg0 + (jt & 1) * STG;
+      // ---- key tile: thread (row tid % BK, q = tid / BK) writes CPT of the 16
+      // 8-column chunks of one key row (chunk k: half k / 8 (the MSE half
+      // c[idx], or the sign half +-coef rho), word (k / 4) % 2, slice k % 4);
+      // value tile: thread (coordinate, group, slice) writes TPT 8-key chunks of
+      // V_rot^T
+      {
+        const int row = tid % BK, qk = tid / BK;
+        const int half = (qk * CPT) >> 3, w = ((qk * CPT) >> 2) & 1;   // the same for all CPT chunks
+        const int j = j0 + row;
+        const bool ok = j < a.T;
+        const uint32_t *krow = reinterpret_cast<const uint32_t *>(st + row * planes_k * (D / 8));
+        const uint32_t sc = ok ? reinterpret_cast<const uint32_t *>(st + 2048)[row] : 0u;
+        const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
+        const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
+        if (qk == 0) nuk[row] = ok ? nu : 0.f;
+        uint32_t pw[4] = {0u, 0u, 0u, 0u};
+  #pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (p < planes_k) pw[p] = krow[p * (D / 32) + w];
+        uint32_t pos[3] = {0u, 0u, 0u};
+        uint32_t sgn = 0u;
+        if (half == 1) {
+          // the sign half is +-qv: its split, negated where the sign bit is 0
+          const float qv = a.qjl_coef * rho;
+          const __nv_bfloat16 p0 = __float2bfloat16_rn(qv);
+          const float r1 = qv - __bfloat162float(p0);
+          const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+          const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+          const uint32_t u[3] = {__bfloat16_as_ushort(p0), __bfloat16_as_ushort(p1), __bfloat16_as_ushort(p2)};
+  #pragma unroll
+          for (int p = 0; p < 3; ++p) pos[p] = (ok && a.books.qjl) ? (u[p] | (u[p] << 16)) : 0u;
+  #pragma unroll
+          for (int p = 0; p < 4; ++p)
+            if (p == mbk) sgn = pw[p];
+        }
+        const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
+  #pragma unroll
+        for (int ci = 0; ci < CPT; ++ci) {
+          const int c8 = (qk * CPT + ci) & 3;
+          uint32_t o[3][4];
+  #pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const int bit = 8 * c8 + 2 * e2;
+            if (half == 0) {
+              uint32_t i0, i1;
+              code_pair(pw, mbk, bit, i0, i1);
+  #pragma unroll
+              for (int p = 0; p < 3; ++p) o[p][e2] = ok ? lut2(tk32 + 4 * p, i0, i1, mbk) : 0u;
+            } else {
+              const uint32_t sb = ~(sgn >> bit);
+              const uint32_t neg = ((sb & 1u) << 15) | ((sb & 2u) << 30);
+  #pragma unroll
+              for (int p = 0; p < 3; ++p) o[p][e2] = pos[p] ^ (pos[p] ? neg : 0u);
+            }
+          }
+          const int off = kmaj16(row, half * D + 32 * w + 8 * c8, BK);
+  #pragma unroll
+          for (int p = 0; p < 3; ++p)
+            *reinterpret_cast<uint4 *>(ks3 + p * K_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
+        }
+      }
+  };
+  auto expand_v = [&](int jt) {
+    const int j0 = jt * BK;
+    const uint8_t *st = stg0 + (jt & 1) * STG;
+      if (tid < BK)
+        vns[tid] = j0 + tid < a.T ? tq_half_to_f32(reinterpret_cast<const uint16_t *>(st + 4352)[tid]) : 0.f;
+      {
+        // V_rot^T: centroids only (the value norms scale P instead)
+        const int coord = tid % D, g = (tid / D) & 1, th = tid / (2 * D);   // th: which TPT slices
+        const int jg = j0 + 32 * g;
+        uint32_t vw[4] = {0u, 0u, 0u, 0u};
+        if (jg < a.T)
+          for (int p = 0; p < nbv; ++p)
+            vw[p] = reinterpret_cast<const uint32_t *>(st + 2304)[(g * nbv + p) * D + coord];
+        const uint32_t *tv32 = reinterpret_cast<const uint32_t *>(&tabv[0][0]);
+  #pragma unroll
+        for (int t8 = TPT * th; t8 < TPT * th + TPT; ++t8) {
+          uint32_t o[3][4];
+  #pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            uint32_t i0, i1;
+            code_pair(vw, nbv, 8 * t8 + 2 * e2, i0, i1);
+  #pragma unroll
+            for (int p = 0; p < 3; ++p) o[p][e2] = lut2(tv32 + 8 * p, i0, i1, nbv);
+          }
+          const int off = kmaj16(coord, 32 * g + 8 * t8, D);
+  #pragma unroll
+          for (int p = 0; p < 3; ++p)
+            *reinterpret_cast<uint4 *>(vs3 + p * V_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
+        }
+      }
+  };
+  auto issue_s = [&]() {
+      // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d): the six
+      // split products of order <= 2 (about 2^-26 relative); warp 0 issues
+      // a2 b0 + a1 b1, warp 1 a0 b2 + a1 b0, warp 2 a0 b1, warp 3 the K steps
+      // of a0 b0 alternating over two accumulators
+      if ((tid & 31) == 0 && warp < 4) {
+        constexpr uint32_t LA = BQ * 16, LB = BK * 16;
+        if (warp < 3) {
+          const int pa[5] = {2, 1, 0, 1, 0}, pb[5] = {0, 1, 2, 0, 1};
+          const int t0 = 2 * warp, nt = warp == 2 ? 1 : 2;
+          const uint32_t d = warp == 0 ? tS0 : warp == 1 ? tS1 : tS2;
+          int n = 0;
+          for (int t = t0; t < t0 + nt; ++t)
+  #pragma unroll
+            for (int k = 0; k < DP / 16; ++k, ++n)
+              sm100::mma_bf16_ss(d, sm100::smem_desc(a_q + pa[t] * Q_BYTES + k * 2 * LA, LA, 128),
+                                 sm100::smem_desc(a_k + pb[t] * K_BYTES + k * 2 * LB, LB, 128), IDESC_S,
+                                 n > 0 ? 1u : 0u);
+        } else {
+  #pragma unroll
+          for (int k = 0; k < DP / 16; ++k)
+            sm100::mma_bf16_ss(tSb + (k % NBIG) * BK, sm100::smem_desc(a_q + k * 2 * LA, LA, 128),
+                               sm100::smem_desc(a_k + k * 2 * LB, LB, 128), IDESC_S, k >= NBIG ? 1u : 0u);
+        }
+        sm100::mma_commit(&mbS);
+      }
+  };
 
   float m = -CUDART_INF_F, l = 0.f;   // l: this half's share of the row sum
-  uint32_t phase = 0;
-  for (int jt = 0; jt < ntiles; ++jt) {
-    const int j0 = jt * BK;
-    // the next tile's rows stream in while this one is worked on (its stage
-    // was last read two tiles ago)
-    if (tid == 0 && jt + 1 < ntiles) {
-      issue_tile(jt + 1);
-      issued = jt + 2;
-    }
-    if (!sm100::mbar_wait(&kvf[jt & 1], (jt >> 1) & 1)) abort_s = 1;
-    __syncthreads();
-    if (abort_s) break;
-    const uint8_t *st = stg0 + (jt & 1) * STG;
-    if (tid < BK)
-      vns[tid] = j0 + tid < a.T ? tq_half_to_f32(reinterpret_cast<const uint16_t *>(st + 4352)[tid]) : 0.f;
-    // ---- key tile: thread (row tid % BK, q = tid / BK) writes CPT of the 16
-    // 8-column chunks of one key row (chunk k: half k / 8 (the MSE half
-    // c[idx], or the sign half +-coef rho), word (k / 4) % 2, slice k % 4);
-    // value tile: thread (coordinate, group, slice) writes TPT 8-key chunks of
-    // V_rot^T
-    {
-      const int row = tid % BK, qk = tid / BK;
-      const int half = (qk * CPT) >> 3, w = ((qk * CPT) >> 2) & 1;   // the same for all CPT chunks
-      const int j = j0 + row;
-      const bool ok = j < a.T;
-      const uint32_t *krow = reinterpret_cast<const uint32_t *>(st + row * planes_k * (D / 8));
-      const uint32_t sc = ok ? reinterpret_cast<const uint32_t *>(st + 2048)[row] : 0u;
-      const float nu = tq_half_to_f32(static_cast<uint16_t>(sc & 0xffffu));
-      const float rho = tq_half_to_f32(static_cast<uint16_t>(sc >> 16));
-      if (qk == 0) nuk[row] = ok ? nu : 0.f;
-      uint32_t pw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-        if (p < planes_k) pw[p] = krow[p * (D / 32) + w];
-      uint32_t pos[3] = {0u, 0u, 0u};
-      uint32_t sgn = 0u;
-      if (half == 1) {
-        // the sign half is +-qv: its split, negated where the sign bit is 0
-        const float qv = a.qjl_coef * rho;
-        const __nv_bfloat16 p0 = __float2bfloat16_rn(qv);
-        const float r1 = qv - __bfloat162float(p0);
-        const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
-        const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
-        const uint32_t u[3] = {__bfloat16_as_ushort(p0), __bfloat16_as_ushort(p1), __bfloat16_as_ushort(p2)};
-#pragma unroll
-        for (int p = 0; p < 3; ++p) pos[p] = (ok && a.books.qjl) ? (u[p] | (u[p] << 16)) : 0u;
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          if (p == mbk) sgn = pw[p];
-      }
-      const uint32_t *tk32 = reinterpret_cast<const uint32_t *>(&tabk[0][0]);
-#pragma unroll
-      for (int ci = 0; ci < CPT; ++ci) {
-        const int c8 = (qk * CPT + ci) & 3;
-        uint32_t o[3][4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int bit = 8 * c8 + 2 * e2;
-          if (half == 0) {
-            uint32_t i0, i1;
-            code_pair(pw, mbk, bit, i0, i1);
-#pragma unroll
-            for (int p = 0; p < 3; ++p) o[p][e2] = ok ? lut2(tk32 + 4 * p, i0, i1, mbk) : 0u;
-          } else {
-            const uint32_t sb = ~(sgn >> bit);
-            const uint32_t neg = ((sb & 1u) << 15) | ((sb & 2u) << 30);
-#pragma unroll
-            for (int p = 0; p < 3; ++p) o[p][e2] = pos[p] ^ (pos[p] ? neg : 0u);
-          }
-        }
-        const int off = kmaj16(row, half * D + 32 * w + 8 * c8, BK);
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-          *reinterpret_cast<uint4 *>(ks3 + p * K_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
-      }
-    }
-    {
-      // V_rot^T: centroids only (the value norms scale P instead)
-      const int coord = tid % D, g = (tid / D) & 1, th = tid / (2 * D);   // th: which TPT slices
-      const int jg = j0 + 32 * g;
-      uint32_t vw[4] = {0u, 0u, 0u, 0u};
-      if (jg < a.T)
-        for (int p = 0; p < nbv; ++p)
-          vw[p] = reinterpret_cast<const uint32_t *>(st + 2304)[(g * nbv + p) * D + coord];
-      const uint32_t *tv32 = reinterpret_cast<const uint32_t *>(&tabv[0][0]);
-#pragma unroll
-      for (int t8 = TPT * th; t8 < TPT * th + TPT; ++t8) {
-        uint32_t o[3][4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          uint32_t i0, i1;
-          code_pair(vw, nbv, 8 * t8 + 2 * e2, i0, i1);
-#pragma unroll
-          for (int p = 0; p < 3; ++p) o[p][e2] = lut2(tv32 + 8 * p, i0, i1, nbv);
-        }
-        const int off = kmaj16(coord, 32 * g + 8 * t8, D);
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-          *reinterpret_cast<uint4 *>(vs3 + p * V_BYTES + off) = make_uint4(o[p][0], o[p][1], o[p][2], o[p][3]);
-      }
-    }
+  uint32_t sph = 0, oph = 0;           // phases of the S and O commit barriers
+  if (ntiles > 0) {
+    if (!sm100::mbar_wait(&kvf[0], 0)) abort_s = 1;
+    expand_k(0);
+    expand_v(0);
     sm100::fence_async_smem();
     sm100::fence_before_sync();
     __syncthreads();
     sm100::fence_after_sync();
-    // ---- S = Q_rot K_rot^T (M = 128 queries, N = 64 keys, K = 2d): the six
-    // split products of order <= 2 (about 2^-26 relative); warp 0 issues
-    // a2 b0 + a1 b1, warp 1 a0 b2 + a1 b0, warp 2 a0 b1, warp 3 the K steps
-    // of a0 b0 alternating over two accumulators
-    if ((tid & 31) == 0 && warp < 4) {
-      constexpr uint32_t LA = BQ * 16, LB = BK * 16;
-      if (warp < 3) {
-        const int pa[5] = {2, 1, 0, 1, 0}, pb[5] = {0, 1, 2, 0, 1};
-        const int t0 = 2 * warp, nt = warp == 2 ? 1 : 2;
-        const uint32_t d = warp == 0 ? tS0 : warp == 1 ? tS1 : tS2;
-        int n = 0;
-        for (int t = t0; t < t0 + nt; ++t)
-#pragma unroll
-          for (int k = 0; k < DP / 16; ++k, ++n)
-            sm100::mma_bf16_ss(d, sm100::smem_desc(a_q + pa[t] * Q_BYTES + k * 2 * LA, LA, 128),
-                               sm100::smem_desc(a_k + pb[t] * K_BYTES + k * 2 * LB, LB, 128), IDESC_S,
-                               n > 0 ? 1u : 0u);
-      } else {
-#pragma unroll
-        for (int k = 0; k < DP / 16; ++k)
-          sm100::mma_bf16_ss(tSb + (k % NBIG) * BK, sm100::smem_desc(a_q + k * 2 * LA, LA, 128),
-                             sm100::smem_desc(a_k + k * 2 * LB, LB, 128), IDESC_S, k >= NBIG ? 1u : 0u);
-      }
-      sm100::mma_commit(&mbS);
-    }
-    if (!sm100::mbar_wait(&mbS, phase)) abort_s = 1;
+    if (!abort_s) issue_s();
+  }
+  // every thread passes every barrier of an iteration and leaves only right
+  // after one, so a give-up (abort_s) takes the whole CTA out together
+  for (int jt = 0; jt < ntiles; ++jt) {
+    const int j0 = jt * BK;
+    // S(jt) has completed
+    if (!abort_s && !sm100::mbar_wait(&mbS, sph)) abort_s = 1;
+    sph ^= 1;
     __syncthreads();
     if (abort_s) break;
+    // the stage of tile jt is free (both its expansions are done): tile jt + 2
+    if (tid == 0 && jt + 2 < ntiles) issue_next(jt + 2);
     sm100::fence_after_sync();
     // this part's KPT scores of row r: the five S accumulators added in fp32
     const int c0 = KPT * hf;
@@ -561,10 +590,27 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
                              (n > 0 || jt > 0) ? 1u : 0u);
       sm100::mma_commit(&mbO);
     }
-    if (!sm100::mbar_wait(&mbO, phase)) abort_s = 1;
-    phase ^= 1;
-    __syncthreads();
-    if (abort_s) break;
+    if (jt + 1 < ntiles) {
+      // K(jt + 1) while O(jt) runs: S(jt) has read K_rot, softmax(jt) nu_k
+      if (!abort_s && !sm100::mbar_wait(&kvf[(jt + 1) & 1], ((jt + 1) >> 1) & 1)) abort_s = 1;
+      expand_k(jt + 1);
+      sm100::fence_async_smem();
+      sm100::fence_before_sync();
+      __syncthreads();
+      sm100::fence_after_sync();
+      if (abort_s) break;
+      issue_s();
+    }
+    // O(jt) has completed: V_rot, P and nu_v are free
+    if (!abort_s && !sm100::mbar_wait(&mbO, oph)) abort_s = 1;
+    oph ^= 1;
+    if (jt + 1 < ntiles) {
+      sm100::fence_after_sync();
+      expand_v(jt + 1);
+      sm100::fence_async_smem();
+    } else {
+      __syncthreads();
+    }
     sm100::fence_after_sync();
   }
   // ---- out = Pi^T O_rot / l = D (H O_rot) / (sqrt(d) l), by the part-0 threads
@@ -605,7 +651,9 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   }
   // this CTA's copies have landed before its shared memory is released: the
   // last issued tile's phase completes (at once if it was consumed)
-  if (tid == 0 && issued > 0) sm100::mbar_wait(&kvf[(issued - 1) & 1], ((issued - 1) >> 1) & 1, 1u << 20);
+  if (tid == 0)
+    for (int i = 0; i < 2; ++i)
+      if (last_par[i] >= 0) sm100::mbar_wait(&kvf[i], static_cast<uint32_t>(last_par[i]), 1u << 20);
   // every MMA this thread issued has landed before tensor memory is released
   if ((tid & 31) == 0 && warp < 4) {
     sm100::mma_commit(&fin[warp]);
