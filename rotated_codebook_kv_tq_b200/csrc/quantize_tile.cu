@@ -379,6 +379,9 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
   constexpr int NTL = tiles_per_unit(D);
   constexpr int QT = 128 * NTL;
   constexpr int TCOLS = 2 * D;            // per tile: A (hi | lo, D/2 columns each) + z (D columns)
+  // tensor memory is allocated in powers of two columns
+  constexpr int TALLOC = NTL * TCOLS <= 256 ? 256 : 512;
+  static_assert(NTL * TCOLS <= 512, "tensor memory budget");
   extern __shared__ uint8_t qsm_raw[];
   uint8_t *qsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *Xt0 = qsm;                     // the unit's tiles, NBX boxes each
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
       *reinterpret_cast<uint16_t *>(Bs + (kb >> 4) * (D * 16) + (i >> 3) * 128 + (i & 7) * 16 +
                                     (kb & 15)) = a.S[e];
     }
-    if (warp == 0) sm100::tmem_alloc(&tmem_s, NTL * TCOLS);
+    if (warp == 0) sm100::tmem_alloc(&tmem_s, TALLOC);
   }
   if (tid == 0) {
     sm100::mbar_init(&full, 1);
@@ -734,7 +737,7 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
   __syncthreads();
   sm100::fence_after_sync();
   if (abort_s && tid == 0 && a.status) atomicOr(a.status, 1u << 31);
-  if (QJL && warp == 0) sm100::tmem_dealloc(tm, NTL * TCOLS);
+  if (QJL && warp == 0) sm100::tmem_dealloc(tm, TALLOC);
 }
 
 // ---------------------------------------------------------------- host side
