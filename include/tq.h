@@ -255,6 +255,9 @@ int tq_attention_logits(const tq_codec *codec, const void *q, int dtype, int B, 
  * T      cached tokens per (b, KV head), 1..rows_cap.
  * Supported: d = 64 with the codec's key MSE bits 1..3 (+QJL) and value bits 1..4.
  * workspace: >= tq_attention_bidir_workspace(...) bytes, 16-byte aligned.
+ * Every wait inside the kernel is bounded; a CTA whose wait gives up lets its
+ * own copies and MMAs land and writes NaN to every element of its 128
+ * queries' output rows (the other queries are exact).
  * ------------------------------------------------------------------------ */
 int tq_attention_bidir_workspace(const tq_codec *codec, int B, int H, int Lq, size_t *bytes);
 int tq_attention_bidir(const tq_codec *codec, const void *q, int dtype, int B, int H, int Hkv,
@@ -293,7 +296,11 @@ int tq_attention_bidir(const tq_codec *codec, const void *q, int dtype, int B, i
  * Scores come from one fp16 product per element on the tensor cores (rows
  * [c[idx] | rho (2 sigma - 1)] against the query scaled by a power of two),
  * accumulated in fp32: about 1e-5 |q| absolute error for unit rows, so rows
- * whose scores differ by less than that may swap places.
+ * whose scores differ by less than that may swap places.  Every wait inside
+ * the scan kernel is bounded; if one gives up, the kernel lets its own copies
+ * and MMAs land, records it in a status word of the workspace (cleared by
+ * every call), and every result of the call is written as index -1, score
+ * NaN.  An index build that gives up sets bit 31 of its status word.
  * ------------------------------------------------------------------------ */
 int tq_index_workspace(const tq_codec *codec, int64_t n, size_t *bytes);
 int tq_index_build(const tq_codec *codec, const float *x, int64_t n, uint8_t *kcode,

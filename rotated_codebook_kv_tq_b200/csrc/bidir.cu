@@ -27,6 +27,8 @@
 // K steps over four, each a chain of two; they are added in fp32 registers.
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "tq_device.cuh"
 #include "tq_sm100.cuh"
 
@@ -53,6 +55,7 @@ struct BidirArgs {
   float *qrot;      // [B][H][Lq][2d] fp32
   float *out;       // [B][H][Lq][d]
   uint32_t *err;
+  uint32_t wait_limit;   // polls per wait before giving up
   TqBooks books;
 };
 
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   float m = -CUDART_INF_F, l = 0.f;   // l: this half's share of the row sum
   uint32_t sph = 0, oph = 0;           // phases of the S and O commit barriers
   if (ntiles > 0) {
-    if (!sm100::mbar_wait(&kvf[0], 0)) abort_s = 1;
+    if (!sm100::mbar_wait(&kvf[0], 0, a.wait_limit)) abort_s = 1;
     expand_k(0);
     expand_v(0);
     sm100::fence_async_smem();
@@ -491,7 +494,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
   for (int jt = 0; jt < ntiles; ++jt) {
     const int j0 = jt * BK;
     // S(jt) has completed
-    if (!abort_s && !sm100::mbar_wait(&mbS, sph)) abort_s = 1;
+    if (!abort_s && !sm100::mbar_wait(&mbS, sph, a.wait_limit)) abort_s = 1;
     sph ^= 1;
     __syncthreads();
     if (abort_s) break;
@@ -592,7 +595,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
     }
     if (jt + 1 < ntiles) {
       // K(jt + 1) while O(jt) runs: S(jt) has read K_rot, softmax(jt) nu_k
-      if (!abort_s && !sm100::mbar_wait(&kvf[(jt + 1) & 1], ((jt + 1) >> 1) & 1)) abort_s = 1;
+      if (!abort_s && !sm100::mbar_wait(&kvf[(jt + 1) & 1], ((jt + 1) >> 1) & 1, a.wait_limit)) abort_s = 1;
       expand_k(jt + 1);
       sm100::fence_async_smem();
       sm100::fence_before_sync();
@@ -602,7 +605,7 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
       issue_s();
     }
     // O(jt) has completed: V_rot, P and nu_v are free
-    if (!abort_s && !sm100::mbar_wait(&mbO, oph)) abort_s = 1;
+    if (!abort_s && !sm100::mbar_wait(&mbO, oph, a.wait_limit)) abort_s = 1;
     oph ^= 1;
     if (jt + 1 < ntiles) {
       sm100::fence_after_sync();
@@ -627,7 +630,12 @@ __global__ void __launch_bounds__(BT, 1) bidir_tile_kernel(BidirArgs a) {
 #pragma unroll
       for (int e = 0; e < 16; ++e) o[c + e] = __uint_as_float(r1[e]) + __uint_as_float(r2[e]);
     }
-    if (!abort_s && q0 + r < a.Lq) {
+    if (abort_s && q0 + r < a.Lq) {
+      // a bounded wait gave up: this CTA's queries are reported as NaN
+      float *dst = a.out + ((static_cast<int64_t>(b) * a.H + h) * a.Lq + q0 + r) * D;
+#pragma unroll
+      for (int i = 0; i < D; ++i) dst[i] = CUDART_NAN_F;
+    } else if (q0 + r < a.Lq) {
 #pragma unroll
       for (int s2 = 1; s2 < D; s2 <<= 1)
 #pragma unroll
@@ -700,6 +708,8 @@ int launch_bidir(const tq_codec *c, const void *q, int dtype, int B, int H, int 
   a.qrot = static_cast<float *>(ws);
   a.out = out;
   a.err = nullptr;
+  a.wait_limit = 1u << 26;
+  if (const char *e = getenv("TQ_WAIT_LIMIT")) a.wait_limit = static_cast<uint32_t>(strtoul(e, nullptr, 10));
   a.books = c->books;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -31,6 +31,7 @@
 //   ix_merge_kernel    merge of the per-CTA lists into the final top-k
 #include <math_constants.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
@@ -199,7 +200,7 @@ struct SketchArgs {
 
 __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
   extern __shared__ __align__(1024) uint8_t skm[];
-  __shared__ __align__(8) uint64_t full[SKS], empty[SKS], acc_full[2], acc_free[2];
+  __shared__ __align__(8) uint64_t full[SKS], empty[SKS], acc_full[2], acc_free[2], fin;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
       sm100::mbar_init(&acc_full[b], 1);
       sm100::mbar_init(&acc_free[b], 4);
     }
+    sm100::mbar_init(&fin, 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -225,8 +227,14 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
   const int total = ntl * SKA_CH;
   if (warp == 4) {
     if (lane == 0 && total > 0) {
+      // per stage: the parity of its last issued copy (-1: none); whether any
+      // MMA was issued (both drained before the CTA releases its memory)
+      int lastc[SKS];
+      for (int s = 0; s < SKS; ++s) lastc[s] = -1;
+      bool mma_issued = false;
       auto copy = [&](int gc) {
         const int tl = gc / SKA_CH, c = gc % SKA_CH, s = gc % SKS;
+        lastc[s] = (gc / SKS) & 1;
         const int64_t t = blockIdx.x + static_cast<int64_t>(tl) * gridDim.x;
         const int64_t mt = t / SKN_T;
         const int nt = static_cast<int>(t % SKN_T);
@@ -253,6 +261,7 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
           sm100::fence_after_sync();
           const uint32_t a_addr = sm100::smem_addr(skm + s * (SKA_BYTES + SKB_BYTES));
           const uint32_t b_addr = a_addr + SKA_BYTES;
+          mma_issued = true;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             sm100::mma_bf16_ss(tm + ab * 256, sm100::smem_desc(a_addr + kk * 2 * 2048, 2048, 128),
@@ -271,7 +280,17 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
           }
         }
       }
-      if (!ok) abort_s = 1;
+      if (!ok) {
+        abort_s = 1;
+        // this CTA's copies and MMAs land before its shared and tensor
+        // memory are released
+        for (int s = 0; s < SKS; ++s)
+          if (lastc[s] >= 0) sm100::mbar_wait(&full[s], static_cast<uint32_t>(lastc[s]), 1u << 20);
+        if (mma_issued) {
+          sm100::mma_commit(&fin);
+          sm100::mbar_wait(&fin, 0, 1u << 20);
+        }
+      }
     }
     __syncwarp();
   } else {
@@ -526,12 +545,14 @@ struct QpackArgs {
   float coef;           // sqrt(pi/2) / d
   uint16_t *qop;        // [ceil(nq / QN)][XCH][QN * 64] fp16
   float *qinv;          // [nq] 2^-e
+  uint32_t *status;     // the scan's give-up flag, cleared here for this call
 };
 
 // One warp per (padded) query: power-of-two scale putting max |B| in
 // [2^14, 2^15), then the fp16 operand in chunk order.
 __global__ void __launch_bounds__(256) ix_qpack_kernel(QpackArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.status) *a.status = 0u;
   const int q = blockIdx.x * 8 + warp;
   const int nqp = (a.nq + QN - 1) / QN * QN;
   if (q >= nqp) return;
@@ -570,7 +591,8 @@ struct Scan2Args {
   float *cand_s;          // [nq][lists][k]
   int32_t *cand_i;
   int k;
-  uint32_t *err;
+  uint32_t *err;          // set when a bounded wait gave up (read by the merge)
+  uint32_t wait_limit;    // polls per wait before giving up
 };
 
 __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
@@ -578,10 +600,11 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
   uint8_t *bst = ssm + SC_B_OFF;
   float *sb = reinterpret_cast<float *>(ssm + SC_SB_OFF);
   uint32_t *lut = reinterpret_cast<uint32_t *>(ssm + SC_LUT_OFF);
-  __shared__ __align__(8) uint64_t a_full[NAS], b_full[NAS], done[NAS], acc_full, acc_free;
+  __shared__ __align__(8) uint64_t a_full[NAS], b_full[NAS], done[NAS], acc_full, acc_free, fin;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t wl = a.wait_limit;
   for (int e = tid; e < 64 * 32; e += SCT) lut[e] = a.lut[e >> 5];
   if (warp == 0) sm100::tmem_alloc(&tmem_s, 512);
   if (tid == 0) {
@@ -592,6 +615,7 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
     }
     sm100::mbar_init(&acc_full, 1);
     sm100::mbar_init(&acc_free, SCW);
+    sm100::mbar_init(&fin, 1);
     abort_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -609,26 +633,33 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
     // ---------------- MMA warp: query-chunk copies and the MMAs
     if (lane == 0 && total > 0) {
       const uint16_t *qsrc = a.qop + static_cast<int64_t>(blockIdx.x) * XCH * (QN * 64);
+      // per stage: the parity of its last issued copy (-1: none); whether any
+      // MMA was issued (both drained before the CTA releases its memory)
+      int lastb[NAS];
+      for (int s = 0; s < NAS; ++s) lastb[s] = -1;
+      bool mma_issued = false;
       auto copy = [&](int g) {
         const int s = g % NAS, c = g % XCH;
         sm100::mbar_expect_tx(&b_full[s], QCH_BYTES);
         sm100::bulk_g2s(bst + s * QCH_BYTES, qsrc + c * (QN * 64), QCH_BYTES, &b_full[s]);
+        lastb[s] = (g / NAS) & 1;
       };
       for (int g = 0; g < NAS - 1 && g < total; ++g) copy(g);
       constexpr uint32_t IDESC = sm100::idesc_f16(RM, QN);
       bool ok = true;
       for (int tl = 0; tl < nt && ok; ++tl) {
         if (tl >= 1) {
-          ok = sm100::mbar_wait(&acc_free, (tl - 1) & 1);
+          ok = sm100::mbar_wait(&acc_free, (tl - 1) & 1, wl);
           if (!ok) break;
           sm100::fence_after_sync();
         }
         for (int c = 0; c < XCH && ok; ++c) {
           const int g = tl * XCH + c, s = g % NAS, u = g / NAS;
-          ok = sm100::mbar_wait(&a_full[s], u & 1) && sm100::mbar_wait(&b_full[s], u & 1);
+          ok = sm100::mbar_wait(&a_full[s], u & 1, wl) && sm100::mbar_wait(&b_full[s], u & 1, wl);
           if (!ok) break;
           sm100::fence_after_sync();
           const uint32_t bb = sm100::smem_addr(bst + s * QCH_BYTES);
+          mma_issued = true;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             sm100::mma_f16_ts(tm, tm + 256 + s * 32 + kk * 8,
@@ -640,14 +671,24 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
           const int gn = g + NAS - 1;
           if (gn < total) {
             if (gn >= NAS) {
-              ok = sm100::mbar_wait(&done[gn % NAS], ((gn / NAS) - 1) & 1);
+              ok = sm100::mbar_wait(&done[gn % NAS], ((gn / NAS) - 1) & 1, wl);
               if (!ok) break;
             }
             copy(gn);
           }
         }
       }
-      if (!ok) abort_s = 1;
+      if (!ok) {
+        abort_s = 1;
+        // this CTA's copies and MMAs land before its shared and tensor
+        // memory are released
+        for (int s = 0; s < NAS; ++s)
+          if (lastb[s] >= 0) sm100::mbar_wait(&b_full[s], static_cast<uint32_t>(lastb[s]), 1u << 20);
+        if (mma_issued) {
+          sm100::mma_commit(&fin);
+          sm100::mbar_wait(&fin, 0, 1u << 20);
+        }
+      }
     }
     __syncwarp();
   } else {
@@ -670,7 +711,7 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
     // skipped but the loops keep their fixed trip counts, so all worker warps
     // still meet at every named barrier.
     auto wwait = [&](uint64_t *bar, uint32_t par) {
-      if (lane == 0 && !abort_s && !sm100::mbar_wait(bar, par)) abort_s = 1;
+      if (lane == 0 && !abort_s && !sm100::mbar_wait(bar, par, wl)) abort_s = 1;
       __syncwarp();
     };
     auto insert = [&](float (&ts)[SKMAX], int (&ti)[SKMAX], float v, int idx) {
@@ -794,9 +835,17 @@ __global__ void __launch_bounds__(SCT, 1) ix_scan2_kernel(Scan2Args a) {
 
 // Merge the per-CTA candidate lists of each query: order (-score, index).
 __global__ void ix_merge_kernel(const float *cs, const int32_t *ci, int nq, int lists, int k,
-                                int32_t *idx, float *score) {
+                                int32_t *idx, float *score, const uint32_t *err) {
   const int q = blockIdx.x * blockDim.x + threadIdx.x;
   if (q >= nq) return;
+  if (err && *err) {
+    // a bounded wait of the scan gave up: its candidate lists are incomplete
+    for (int e = 0; e < k; ++e) {
+      idx[static_cast<int64_t>(q) * k + e] = -1;
+      score[static_cast<int64_t>(q) * k + e] = CUDART_NAN_F;
+    }
+    return;
+  }
   float bs[SKMAX];
   int bi[SKMAX];
   for (int e = 0; e < SKMAX; ++e) {
@@ -1094,7 +1143,7 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
 // Scan workspace, 256-byte aligned pieces: q' fp32, q' bf16 hi | lo (GEMM A),
 // q'' fp32, the packed fp16 query operand, 2^-e per query, candidate lists.
 struct ScanWs {
-  size_t q1, q1hl, q2, qop, qinv, cand_s, cand_i, total;
+  size_t q1, q1hl, q2, qop, qinv, cand_s, cand_i, status, total;
 };
 
 ScanWs scan_ws(int nq, int k, int gy) {
@@ -1117,6 +1166,8 @@ ScanWs scan_ws(int nq, int k, int gy) {
   o += up(nc * 4);
   w.cand_i = o;
   o += up(nc * 4);
+  w.status = o;
+  o += up(4);
   w.total = o;
   return w;
 }
@@ -1155,6 +1206,7 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   float *qinv = reinterpret_cast<float *>(w + W.qinv);
   float *cand_s = reinterpret_cast<float *>(w + W.cand_s);
   int32_t *cand_i = reinterpret_cast<int32_t *>(w + W.cand_i);
+  uint32_t *status = reinterpret_cast<uint32_t *>(w + W.status);
   // q' = Pi q (fp32 and bf16 hi | lo), q'' = S q' (fp32) on the tensor cores
   if (int e = scan_query_prologue(c, q, nq, q1, q1hl, q2, st)) return e;
   // fp16 B operand with a power-of-two scale per query
@@ -1166,6 +1218,7 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   pa.coef = coef;
   pa.qop = qop;
   pa.qinv = qinv;
+  pa.status = status;
   const int nqp = (nq + QN - 1) / QN * QN;
   ix_qpack_kernel<<<(nqp + 7) / 8, 256, 0, st>>>(pa);
   tq_count_launch(1);
@@ -1192,7 +1245,9 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   sa.cand_s = cand_s;
   sa.cand_i = cand_i;
   sa.k = k;
-  sa.err = nullptr;
+  sa.err = status;
+  sa.wait_limit = 1u << 26;
+  if (const char *e = getenv("TQ_WAIT_LIMIT")) sa.wait_limit = static_cast<uint32_t>(strtoul(e, nullptr, 10));
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1209,7 +1264,7 @@ int tq_scan_topk(const tq_codec *c, const uint8_t *kcode, const uint16_t *kscale
   ix_scan2_kernel<<<grid, SCT, SC_SMEM, st>>>(sa);
   if (int e = tq_check_launch("ix_scan2_kernel")) return e;
   if (ev1) cudaEventRecord(ev1, st);
-  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(cand_s, cand_i, nq, 2 * gy, k, idx, score);
+  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(cand_s, cand_i, nq, 2 * gy, k, idx, score, status);
   tq_count_launch(2);
   return tq_check_launch("ix_merge_kernel");
 }
@@ -1269,7 +1324,7 @@ int tq_scan_topk_lut(const tq_codec *c, const uint8_t *kcode, const uint16_t *ks
   ix_lut_kernel<<<dim3(nq, lb), LT, LUT_SMEM, st>>>(la);
   if (int e = tq_check_launch("ix_lut_kernel")) return e;
   if (ev1) cudaEventRecord(ev1, st);
-  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(la.cand_s, la.cand_i, nq, lb, k, idx, score);
+  ix_merge_kernel<<<(nq + 127) / 128, 128, 0, st>>>(la.cand_s, la.cand_i, nq, lb, k, idx, score, nullptr);
   tq_count_launch(2);
   return tq_check_launch("ix_merge_kernel");
 }
