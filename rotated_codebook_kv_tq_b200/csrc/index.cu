@@ -196,6 +196,7 @@ struct SketchArgs {
   uint8_t *plane;         // sign plane of row 0 of the batch; row stride plane_stride bytes
   int64_t plane_stride;
   uint32_t *status;
+  uint32_t wait_limit;    // polls per wait before giving up
 };
 
 __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
@@ -250,13 +251,13 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
       for (int tl = 0; tl < ntl && ok; ++tl) {
         const int ab = tl & 1;
         if (tl >= 2) {
-          ok = sm100::mbar_wait(&acc_free[ab], ((tl >> 1) - 1) & 1);
+          ok = sm100::mbar_wait(&acc_free[ab], ((tl >> 1) - 1) & 1, g.wait_limit);
           if (!ok) break;
           sm100::fence_after_sync();
         }
         for (int c = 0; c < SKA_CH && ok; ++c) {
           const int gc = tl * SKA_CH + c, s = gc % SKS;
-          ok = sm100::mbar_wait(&full[s], (gc / SKS) & 1);
+          ok = sm100::mbar_wait(&full[s], (gc / SKS) & 1, g.wait_limit);
           if (!ok) break;
           sm100::fence_after_sync();
           const uint32_t a_addr = sm100::smem_addr(skm + s * (SKA_BYTES + SKB_BYTES));
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
           const int gn = gc + SKS - 1;
           if (gn < total) {
             if (gn >= SKS) {
-              ok = sm100::mbar_wait(&empty[gn % SKS], ((gn / SKS) - 1) & 1);
+              ok = sm100::mbar_wait(&empty[gn % SKS], ((gn / SKS) - 1) & 1, g.wait_limit);
               if (!ok) break;
             }
             copy(gn);
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
     // epilogue warp = TMEM lane quarter: row 32 warp + lane of the m tile
     for (int tl = 0; tl < ntl; ++tl) {
       const int ab = tl & 1;
-      if (lane == 0 && !abort_s && !sm100::mbar_wait(&acc_full[ab], (tl >> 1) & 1)) abort_s = 1;
+      if (lane == 0 && !abort_s && !sm100::mbar_wait(&acc_full[ab], (tl >> 1) & 1, g.wait_limit)) abort_s = 1;
       __syncwarp();
       sm100::fence_after_sync();
       const int64_t t = blockIdx.x + static_cast<int64_t>(tl) * gridDim.x;
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(SK_T, 1) ix_sketch_kernel(SketchArgs g) {
       if (lane == 0) sm100::mbar_arrive(&acc_free[ab]);
     }
   }
-  if (abort_s && tid == 0 && g.status) atomicAdd(g.status, 1u << 31);
+  if (abort_s && tid == 0 && g.status) atomicOr(g.status, 1u << 31);
   sm100::fence_before_sync();
   __syncthreads();
   sm100::fence_after_sync();
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(128, 1) ix_gemm_kernel(GemmArgs g) {
       }
     }
   } else if (tid == 0 && g.status) {
-    atomicAdd(g.status, 1u << 31);
+    atomicOr(g.status, 1u << 31);
   }
   sm100::fence_before_sync();
   __syncthreads();
@@ -1122,6 +1123,8 @@ int tq_index_build(const tq_codec *c, const float *x, int64_t n, uint8_t *kcode,
     g.plane = a.kcode + c->mse_bits_k * (XD / 8);
     g.plane_stride = planes * (XD / 8);
     g.status = status;
+    g.wait_limit = 1u << 26;
+    if (const char *e = getenv("TQ_WAIT_LIMIT")) g.wait_limit = static_cast<uint32_t>(strtoul(e, nullptr, 10));
     static bool sk_attr[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);

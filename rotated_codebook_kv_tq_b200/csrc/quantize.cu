@@ -771,7 +771,7 @@ __global__ void __launch_bounds__(QTC_T, 1) quantize_tc_kernel(QuantArgs a) {
   }
   if (abort_s) {
     sm100::mbar_wait(&mb, phase, 1u << 20);
-    if (tid == 0 && a.status) atomicAdd(a.status, 1u << 31);
+    if (tid == 0 && a.status) atomicOr(a.status, 1u << 31);
   }
   sm100::fence_before_sync();
   __syncthreads();

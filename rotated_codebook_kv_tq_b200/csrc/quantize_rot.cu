@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(RT, D == 64 ? 2 : 1) qrot_kernel(RotArgs a) {
       if (n_rot) sm100::mbar_wait(&mb_rot, (n_rot - 1) & 1, 1u << 20);
       if (n_sk) sm100::mbar_wait(&mb_sk, (n_sk - 1) & 1, 1u << 20);
     }
-    if (tid == 0 && a.status) atomicAdd(a.status, 1u << 31);
+    if (tid == 0 && a.status) atomicOr(a.status, 1u << 31);
   }
   sm100::fence_before_sync();
   __syncthreads();

@@ -66,6 +66,7 @@ struct TileArgs {
   uint16_t *vnorm;
   uint32_t *status;
   const uint16_t *S;
+  uint32_t wait_outer;   // rounds of 2^14 polls per wait before giving up
   int rope;
   float ck[8];       // key centroid magnitudes c[half + m], m = 0 .. half-1
   float tk[8];       // key thresholds above 0: t[half - 1 + j], j = 1 .. half-1 (tk[j - 1])
@@ -100,8 +101,9 @@ __device__ __forceinline__ uint4 swz_ld(const uint8_t *box, int r, int c) {
 }
 
 // Bounded wait that also gives up as soon as another thread has.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-  for (int it = 0; it < 4096; ++it) {
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, uint32_t outer,
+                                              volatile int *abort_flag) {
+  for (uint32_t it = 0; it < outer; ++it) {
     if (sm100::mbar_wait(bar, parity, 1u << 14)) return true;
     if (*abort_flag) return false;
   }
@@ -473,7 +475,7 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
       const int64_t R = a.R_first + pt * QR + rl;     // cache row
       const int64_t t = R - a.row0;                    // token of the call
       const bool active = t >= 0 && t < a.T && bh < BH;
-      if (ok && !wait_or_abort(&full, i & 1, &abort_s)) { abort_s = 1; ok = false; }
+      if (ok && !wait_or_abort(&full, i & 1, a.wait_outer, &abort_s)) { abort_s = 1; ok = false; }
       // ---- row into registers (+ RoPE for keys); after a give-up the
       // values read are never used
       float x[D];
@@ -629,7 +631,7 @@ __global__ void __launch_bounds__(128 * tiles_per_unit(D), 1)
             sm100::mma_commit(&z_ready);
             committed = kz;
           }
-          if (!wait_or_abort(&z_ready, (kz++) & 1, &abort_s)) {
+          if (!wait_or_abort(&z_ready, (kz++) & 1, a.wait_outer, &abort_s)) {
             abort_s = 1;
             ok = false;
             continue;   // the next step's first barrier takes the CTA out
@@ -832,6 +834,8 @@ int launch_quantize_tile(const tq_codec *c, const void *k, const void *v, int dt
   a.vnorm = cache->vnorm;
   a.status = status;
   a.S = c->S_dev;
+  a.wait_outer = 4096;
+  if (const char *e = getenv("TQ_WAIT_LIMIT")) a.wait_outer = static_cast<uint32_t>(strtoul(e, nullptr, 10) >> 14);
   a.rope = rc != nullptr;
   const int hk = 1 << (mbk - 1), hv = 1 << (bv - 1);
   for (int m = 0; m < 8; ++m) {

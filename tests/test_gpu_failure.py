@@ -7,7 +7,8 @@ make the failure happen without faulting or hanging anything: the kernel
 drains its own copies and MMAs and reports the give-up (decode: the split-K
 combine writes NaN for every output instead of merging incomplete partials;
 bidirectional pass: the queries of a CTA that gave up are written as NaN;
-scan: every result becomes index -1, score NaN).  The next call without the
+scan: every result becomes index -1, score NaN; tile quantize and index
+build: bit 31 of the call's status word).  The next call without the
 override must be exact again."""
 import math
 
@@ -114,3 +115,55 @@ def test_scan_wait_give_up_is_reported(monkeypatch):
     monkeypatch.delenv("TQ_WAIT_LIMIT")
     ai, as_ = scan()
     assert torch.equal(ai, gi) and torch.equal(as_, gs)
+
+
+def test_tile_quantize_wait_give_up_sets_status_bit(monkeypatch):
+    # a bf16 call of >= 256 token groups takes the tile kernel
+    w = synth.WORKLOADS["esm_prefill"].scaled(B=2, Hq=4, Hkv=4, T=1024)
+    _, ncodec = tl.codecs(w)
+    K, V = synth.kv_inputs_torch(w)
+    r = synth.rope_for(w, w.T)
+    rope = tl.rope_device(r)
+
+    def quantize():
+        cache = native.alloc_cache(ncodec, w.B, w.Hkv, w.T)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        native.quantize_kv(ncodec, K, V, cache, rope=rope, status=status)
+        torch.cuda.synchronize()
+        return tl.download_cache(cache), int(status.item()) & 0xffffffff
+
+    good, st = quantize()
+    assert st == 0
+    monkeypatch.setenv("TQ_WAIT_LIMIT", "0")
+    _, st = quantize()
+    assert st & (1 << 31)
+    monkeypatch.delenv("TQ_WAIT_LIMIT")
+    again, st = quantize()
+    assert st == 0
+    for key in ("kcode", "kscale", "vcode", "vnorm"):
+        assert np.array_equal(again[key], good[key]), key
+
+
+def test_index_build_wait_give_up_sets_status_bit(monkeypatch):
+    D, n = 1536, 3000
+    w = synth.VECTOR_SEARCH
+    ncodec = native.Codec(D, w.bits, True, 4, synth.rotation_signs(D, w.seed), synth.qjl_matrix_bf16(D, w.seed))
+    x = torch.from_numpy(synth.unit_rows(n, D, 78, 0)).cuda()
+
+    def build():
+        kcode = torch.empty((n, ncodec.planes_k, D // 8), dtype=torch.uint8, device="cuda")
+        kscale = torch.empty((n, 2), dtype=torch.float16, device="cuda")
+        ws = torch.empty(native.index_workspace(ncodec, n), dtype=torch.uint8, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        native.index_build(ncodec, x, kcode, kscale, ws, status=status)
+        torch.cuda.synchronize()
+        return kcode.cpu(), kscale.cpu(), int(status.item()) & 0xffffffff
+
+    gk, gs, st = build()
+    assert st == 0
+    monkeypatch.setenv("TQ_WAIT_LIMIT", "0")
+    _, _, st = build()
+    assert st & (1 << 31)
+    monkeypatch.delenv("TQ_WAIT_LIMIT")
+    ak, as_, st = build()
+    assert st == 0 and torch.equal(ak, gk) and torch.equal(as_, gs)
