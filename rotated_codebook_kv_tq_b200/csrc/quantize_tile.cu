@@ -12,12 +12,15 @@
 //   K, V and RoPE-table tiles arrive by TMA tensor copies with the 128-byte
 //   swizzle, so thread r reads its own row from shared memory without bank
 //   conflicts.  Rows outside the call are zero-filled by the copy and skipped
-//   on store.
-// * Every thread runs its row alone: RoPE, norm, the d-point Walsh-Hadamard
-//   transform in registers (no shuffles), codes by compares against the upper
-//   half of the symmetric codebook (the middle threshold is 0), and bit planes
-//   accumulated one funnel shift per coordinate.  Value planes are moved into
-//   the 32-token column layout with warp-wide 32 x 32 bit transposes.
+//   on store; the tiles of a unit's missing heads (the last head group of an
+//   odd B x H) are not copied and their rows are inactive.
+// * Every thread runs its row alone: RoPE, norm, the sign flip D (a packed
+//   multiply by +-1), the d-point Walsh-Hadamard transform in registers (no
+//   shuffles), codes by compares against the upper half of the symmetric
+//   codebook (the middle threshold is 0), and bit planes accumulated one
+//   funnel shift per coordinate (the sign of y enters the lower planes once
+//   per 32-coordinate word).  Value planes are moved into the 32-token column
+//   layout with warp-wide 32 x 32 bit transposes.
 // * Keys: the residual of the tile, split into bf16 hi + lo, is stored into
 //   tensor memory and sketched against S (exactly bf16) by tcgen05 kind::f16
 //   MMAs with fp32 accumulation; each thread reads its row of S r back.
