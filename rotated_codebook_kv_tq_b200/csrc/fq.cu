@@ -260,6 +260,36 @@ __device__ __forceinline__ void fq_key_sums(const uint32_t *krow, int nb, const 
   }
 }
 
+// Key row from the per-query codeword table: acc[h] += sum over blocks j of
+// T[j][idx_j][h], T[j][c][h] = <q'_(2j, 2j+1), c> (16 codewords per block
+// at most, G heads per entry).
+template <int KB, int NPW, int G>
+__device__ __forceinline__ void fq_key_sums_lut(const uint32_t *krow, const float *ktab, float (&acc)[G]) {
+#pragma unroll
+  for (int k = 0; k < NPW; ++k) {
+    uint32_t pw[KB];
+#pragma unroll
+    for (int p = 0; p < KB; ++p) pw[p] = krow[p * NPW + k];
+#pragma unroll 8
+    for (int t = 0; t < 32; ++t) {
+      int idx = 0;
+#pragma unroll
+      for (int p = 0; p < KB; ++p) idx |= ((pw[p] >> t) & 1) << p;
+      const float *te = ktab + ((32 * k + t) * 16 + idx) * G;
+      if constexpr (G == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(te);
+        acc[0] += v.x;
+        acc[1] += v.y;
+        acc[2] += v.z;
+        acc[3] += v.w;
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] += te[h];
+      }
+    }
+  }
+}
+
 // Values of one 32-token column group for one rotated coordinate (component
 // comp of block vg's codes): o[h] += w[r][h] c[idx_r].comp for rows rlo..rhi.
 template <int VB, int G>
@@ -281,11 +311,14 @@ __device__ __forceinline__ void fq_value_rows(const uint32_t *vg, int nb, int ps
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool LUT>
 __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
   constexpr int NPW = D / 64;
   constexpr int SLICES = FCT / D;
   constexpr int SUB = G >= 8 ? 512 : 1024;
+  // LUT: key codes of at most 4 bits per block read the logit terms
+  // <q', c> from a per-query table of (D/2) x 16 x G entries
+  __shared__ __align__(16) float ktab[LUT ? (D / 2) * 16 * G : 4];
   __shared__ float q1s[D][G];
   __shared__ float2 cks[1 << FQ_MAX_BITS], cvs[1 << FQ_MAX_BITS];
   __shared__ float w[SUB][G];
@@ -314,6 +347,13 @@ __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
   }
   __syncthreads();
   const int bk = a.books.bits_k, bv = a.books.bits_v;
+  if (LUT) {
+    for (int e = tid; e < (D / 2) * (1 << bk) * G; e += FCT) {
+      const int h = e % G, c = (e / G) % (1 << bk), j = e / (G << bk);
+      ktab[(j * 16 + c) * G + h] = fmaf(q1s[2 * j][h], cks[c].x, q1s[2 * j + 1][h] * cks[c].y);
+    }
+    __syncthreads();
+  }
   const int coord = tid % D, slice = tid / D;
   const int blk = coord >> 1, comp = coord & 1;
   float o[G];
@@ -330,7 +370,14 @@ __global__ void __launch_bounds__(FCT) fq_chunk_kernel(FqDecArgs a) {
 #pragma unroll
       for (int h = 0; h < G; ++h) acc[h] = 0.f;
       // the code width selects an instantiation with exactly that many planes
-      switch (bk) {
+      if constexpr (LUT) {
+        switch (bk) {
+          case 1: fq_key_sums_lut<1, NPW, G>(krow, ktab, acc); break;
+          case 2: fq_key_sums_lut<2, NPW, G>(krow, ktab, acc); break;
+          case 3: fq_key_sums_lut<3, NPW, G>(krow, ktab, acc); break;
+          default: fq_key_sums_lut<4, NPW, G>(krow, ktab, acc); break;
+        }
+      } else switch (bk) {
         case 1: fq_key_sums<1, NPW, G>(krow, bk, cks, q1s, acc); break;
         case 2: fq_key_sums<2, NPW, G>(krow, bk, cks, q1s, acc); break;
         case 3: fq_key_sums<3, NPW, G>(krow, bk, cks, q1s, acc); break;
@@ -560,11 +607,22 @@ int run_fq_decode(FqDecArgs &a, cudaStream_t stream) {
     if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
     cudaEventRecordWithFlags(ev0, stream, ev_flags);
   }
+  // key codes of at most 4 bits per block: logit terms from a per-query table
+  const bool lut = a.books.bits_k <= 4;
   switch (a.G) {
-    case 1: fq_chunk_kernel<D, 1><<<grid, FCT, 0, stream>>>(a); break;
-    case 2: fq_chunk_kernel<D, 2><<<grid, FCT, 0, stream>>>(a); break;
-    case 4: fq_chunk_kernel<D, 4><<<grid, FCT, 0, stream>>>(a); break;
-    case 8: fq_chunk_kernel<D, 8><<<grid, FCT, 0, stream>>>(a); break;
+    case 1:
+      if (lut) fq_chunk_kernel<D, 1, true><<<grid, FCT, 0, stream>>>(a);
+      else fq_chunk_kernel<D, 1, false><<<grid, FCT, 0, stream>>>(a);
+      break;
+    case 2:
+      if (lut) fq_chunk_kernel<D, 2, true><<<grid, FCT, 0, stream>>>(a);
+      else fq_chunk_kernel<D, 2, false><<<grid, FCT, 0, stream>>>(a);
+      break;
+    case 4:
+      if (lut) fq_chunk_kernel<D, 4, true><<<grid, FCT, 0, stream>>>(a);
+      else fq_chunk_kernel<D, 4, false><<<grid, FCT, 0, stream>>>(a);
+      break;
+    case 8: fq_chunk_kernel<D, 8, false><<<grid, FCT, 0, stream>>>(a); break;
     default: return tq_fail(TQ_ERR_UNSUPPORTED, "fq decode: GQA group size must be 1, 2, 4 or 8");
   }
   if (int e = tq_check_launch("fq_chunk_kernel")) return e;
