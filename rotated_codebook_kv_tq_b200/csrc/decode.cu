@@ -331,6 +331,16 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
     if (tid < D) a.out[head * D + tid] = CUDART_NAN_F;
     return;
   }
+  // this thread's partial outputs (splits gq, gq + CMB, ...) are loaded
+  // first, so their latency overlaps the reductions of the chunk statistics
+  constexpr int PMAX = 16;
+  const float *po = a.po + head * S * D + c;
+  float pv[PMAX];
+#pragma unroll
+  for (int i = 0; i < PMAX; ++i) {
+    const int sp = gq + CMB * i;
+    pv[i] = sp < S ? po[static_cast<int64_t>(sp) * D] : 0.f;
+  }
   float m = -CUDART_INF_F;
   for (int s = tid; s < S; s += NT) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
@@ -354,8 +364,13 @@ __global__ void __launch_bounds__(CMB * D) combine_kernel(DecodeArgs a) {
 #pragma unroll
   for (int w = 0; w < NT / 32; ++w) L += red[w][1];
   float o0 = 0.f, o1 = 0.f;
-  const float *po = a.po + head * S * D + c;
-  int s = gq;
+#pragma unroll
+  for (int i = 0; i < PMAX; i += 2) {
+    const int s0 = gq + CMB * i, s1 = s0 + CMB;
+    if (s0 < S) o0 = fmaf(pv[i], fs[s0], o0);
+    if (s1 < S) o1 = fmaf(pv[i + 1], fs[s1], o1);
+  }
+  int s = gq + CMB * PMAX;   // splits beyond the registers (more than CMB * PMAX)
   for (; s + CMB < S; s += 2 * CMB) {
     o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
     o1 = fmaf(po[static_cast<int64_t>(s + CMB) * D], fs[s + CMB], o1);
