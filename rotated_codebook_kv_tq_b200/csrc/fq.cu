@@ -481,6 +481,15 @@ __global__ void __launch_bounds__(FCMB * D) fq_combine_kernel(FqDecArgs a) {
   const int c = tid % D, gq = tid / D;
   const int64_t head = blockIdx.x;
   const int S = a.splits;
+  // this thread's partial outputs are loaded first, so their latency
+  // overlaps the reductions of the chunk statistics
+  constexpr int PMAX = 16;
+  float pv[PMAX];
+#pragma unroll
+  for (int i = 0; i < PMAX; ++i) {
+    const int sp = gq + FCMB * i;
+    pv[i] = sp < S ? a.po[(head * S + sp) * D + c] : 0.f;
+  }
   float m = -CUDART_INF_F;
   for (int s = tid; s < S; s += NT) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
@@ -504,7 +513,12 @@ __global__ void __launch_bounds__(FCMB * D) fq_combine_kernel(FqDecArgs a) {
 #pragma unroll
   for (int i = 0; i < NT / 32; ++i) L += red[i][1];
   float acc = 0.f;
-  for (int s = gq; s < S; s += FCMB) acc = fmaf(a.po[(head * S + s) * D + c], fs[s], acc);
+#pragma unroll
+  for (int i = 0; i < PMAX; ++i) {
+    const int sp = gq + FCMB * i;
+    if (sp < S) acc = fmaf(pv[i], fs[sp], acc);
+  }
+  for (int s = gq + FCMB * PMAX; s < S; s += FCMB) acc = fmaf(a.po[(head * S + s) * D + c], fs[s], acc);
   os[gq][c] = acc;
   __syncthreads();
   if (warp == 0) {

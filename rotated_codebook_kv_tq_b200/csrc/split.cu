@@ -387,6 +387,16 @@ __global__ void __launch_bounds__(SCMB * 2 * DS) split_combine_kernel(SplitArgs 
   const int64_t head = blockIdx.x;
   const int kvh = static_cast<int>(head % a.Hq) / a.G;
   const int S = a.splits;
+  // this thread's partial outputs are loaded first, so their latency
+  // overlaps the reductions of the chunk statistics
+  constexpr int PMAX = 16;
+  const float *po = a.po + head * S * D + c;
+  float pv[PMAX];
+#pragma unroll
+  for (int i = 0; i < PMAX; ++i) {
+    const int sp = gq + SCMB * i;
+    pv[i] = sp < S ? po[static_cast<int64_t>(sp) * D] : 0.f;
+  }
   float m = -CUDART_INF_F;
   for (int s = tid; s < S; s += NT) m = fmaxf(m, a.pml[(head * S + s) * 2]);
   m = tq_warp_max(m);
@@ -410,8 +420,13 @@ __global__ void __launch_bounds__(SCMB * 2 * DS) split_combine_kernel(SplitArgs 
 #pragma unroll
   for (int i = 0; i < NT / 32; ++i) L += red[i][1];
   float o0 = 0.f, o1 = 0.f;
-  const float *po = a.po + head * S * D + c;
-  int s = gq;
+#pragma unroll
+  for (int i = 0; i < PMAX; i += 2) {
+    const int s0 = gq + SCMB * i, s1 = s0 + SCMB;
+    if (s0 < S) o0 = fmaf(pv[i], fs[s0], o0);
+    if (s1 < S) o1 = fmaf(pv[i + 1], fs[s1], o1);
+  }
+  int s = gq + SCMB * PMAX;   // splits beyond the registers
   for (; s + SCMB < S; s += 2 * SCMB) {
     o0 = fmaf(po[static_cast<int64_t>(s) * D], fs[s], o0);
     o1 = fmaf(po[static_cast<int64_t>(s + SCMB) * D], fs[s + SCMB], o1);
