@@ -146,6 +146,22 @@ def test_fq_host_codebook_matches_oracle(L, d, bits):
     assert abs(mse / ref.mse_per_pair - 1) < 1e-9
 
 
+def test_decode_step_host_validates_before_device_work(L):
+    cd = native.CacheDesc(None, None, None, None, 1, 1, 32)
+    f = L.tq_decode_step_host
+    # no codec
+    assert f(None, 1, 2, 16, native.TQ_BF16, native.TQ_BF16, 1, 1, 1, ctypes.byref(cd), 4, 0.1, None,
+             None, 0, 3, 64, 5, 6, None) == native.TQ_ERR_INVALID_ARG
+    assert b"codec" in L.tq_last_error()
+    # a NULL host or device buffer is rejected before the codec is read
+    fake = ctypes.create_string_buffer(256)
+    for bufs in [(None, 2, 5, 6), (1, None, 5, 6), (1, 2, None, 6), (1, 2, 5, None)]:
+        ih, idv, od, oh = bufs
+        assert f(ctypes.addressof(fake), ih, idv, 16, native.TQ_BF16, native.TQ_BF16, 1, 1, 1,
+                 ctypes.byref(cd), 4, 0.1, None, None, 0, 3, 64, od, oh, None) == native.TQ_ERR_INVALID_ARG
+        assert b"NULL buffer" in L.tq_last_error()
+
+
 def test_fq_codec_is_host_only_and_validates(L):
     signs = synth.rotation_signs(128, 0)
     c = native.FqCodec(128, 4, 3, signs)
